@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Throughput of the fused TileQ MoE-layer forward on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--batch T]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed on the host
+
+A step is one full forward (routing, permutation, column projection, gate/up,
+down-side projection, row accumulation, down/combine) over one batch of T
+synthetic tokens with every input already resident in HBM.  Default workload:
+the Mixtral-8x7B-shaped decode layer (8 experts on a 2x4 grid, d_model 4096,
+d_ff 14336, rank 128, 2-bit residual in groups of 128, top-2) at T=64.
+With N > 1 (torchrun), every rank runs its own batch on its own GPU: weak
+scaling, no data-path collective (the forward has no exchange step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 2**20
+STAGES = ["route", "permute", "zproj", "gateup", "zdown", "rowacc", "residual", "shared", "combine"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="tileq", choices=["tileq", "reference"])
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-compare", action="store_true", help="skip the unfused / rank-0 comparisons")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report no clocks
+            self.err = str(e)
+
+    def _handle(self, idx):
+        import torch
+        nv = self.nv
+        try:
+            props = torch.cuda.get_device_properties(idx)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.0005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def report(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = [n for b, n in REASON_BITS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host (CPU baseline and reference arm)
+# ---------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_step(layer, x, logits, tok):
+    import oracle
+    return oracle.forward(layer, x, logits, tokens=[tok])
+
+
+def cpu_baseline(layer, x, logits, n_tokens=1):
+    """The oracle as it stands on a bounded sample: the first n_tokens tokens."""
+    t0 = time.perf_counter()
+    for t in range(n_tokens):
+        oracle_step(layer, x, logits, t)
+    dt = time.perf_counter() - t0
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n_tokens} token(s) of the batch through the fp64 oracle "
+                      f"(dense reconstruction of each routed expert's 3 projections), {dt:.1f} s"}
+
+
+def run_reference(args, cfg, T):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return  # only rank 0 runs the host oracle
+    layer = synth.make_layer(cfg, seed=args.seed)
+    logits, x = synth.make_inputs(cfg, T, seed=args.seed)
+    for i in range(args.warmup):
+        oracle_step(layer, x, logits, i % T)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_step(layer, x, logits, (args.warmup + i) % T)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    line = {
+        "impl": "reference", "metric": metric_name(cfg, T), "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg, T, args, "host"),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": "each step: one token of the batch through the fp64 oracle"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def metric_name(cfg, T):
+    return "TileQ MoE-layer tokens/s"
+
+
+def workload_config(cfg, T, args, l2):
+    return {"workload": f"{cfg.name} T={T}", "experts": cfg.K, "grid": f"{cfg.M}x{cfg.N}",
+            "d_model": cfg.d_model, "d_ff": cfg.d_ff, "rank": cfg.rank, "group": cfg.group,
+            "top_k": cfg.top_k, "tokens_per_gpu": T, "shared_d_ff": cfg.shared_d_ff,
+            "residual_bits": 2, "parallelism": f"replicas x{args.gpus}", "l2": l2}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    cfg = synth.CONFIGS[args.config]
+    T = args.batch or (64 if args.config == 1 else cfg.batches[-1])
+    if args.impl == "reference":
+        run_reference(args, cfg, T)
+        return
+    if args.warmup < 3:
+        raise SystemExit("at least 3 warm-up steps")
+
+    import torch
+    import torch.distributed as dist
+    import tiled_rank_b200 as tq
+    from tiled_rank_b200 import roofline
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    layer = synth.make_layer(cfg, seed=args.seed)
+    logits_np, x_np = synth.make_inputs(cfg, T, seed=args.seed + 1000 * rank)
+    dl = tq.DeviceLayer(layer, dev)
+    lg = torch.from_numpy(logits_np).to(dev)
+    xt = torch.from_numpy(x_np.view(np.int16)).to(dev).view(torch.bfloat16)
+    out = torch.empty((T, dl.d_y), dtype=torch.bfloat16, device=dev)
+    ws = dl.workspace(T)
+    route = dl.route_buffers(T)
+    stream = torch.cuda.current_stream(dev)
+
+    # realised routing -> algorithmic work
+    dl.forward(xt, lg, out=out, ws=ws, route=route)
+    torch.cuda.synchronize(dev)
+    topk = route["topk_idx"].cpu().numpy()
+    wk = roofline.work(layer, topk)
+    footprint = wk["bytes"]
+    flush = footprint < 3 * L2_BYTES
+    flush_buf = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev) if flush else None
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        dl.forward(xt, lg, out=out, ws=ws)
+    torch.cuda.synchronize(dev)
+
+    # ---------------- timed region: K forwards, inputs resident
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    n0 = tq.tileq_launch_count()
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        if flush:
+            for i in range(args.steps):
+                flush_buf.zero_()
+                ev[2 * i].record(stream)
+                dl.forward(xt, lg, out=out, ws=ws)
+                ev[2 * i + 1].record(stream)
+        else:
+            ev[0].record(stream)
+            for i in range(args.steps):
+                dl.forward(xt, lg, out=out, ws=ws)
+            ev[1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    launches = tq.tileq_launch_count() - n0
+    if flush:
+        ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps))
+    else:
+        ms = ev[0].elapsed_time(ev[1])
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms = float(ms_t.item())
+    ms_per_step = ms / args.steps
+    value = world * T * args.steps / (ms / 1000.0)
+
+    # ---------------- per-stage device times (separate pass, same stream)
+    sev = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+    stage_ms = np.zeros(len(STAGES))
+    tq.tileq_set_stage_events(sev)
+    nprof = max(3, min(args.steps, 50))
+    for _ in range(nprof):
+        if flush:
+            flush_buf.zero_()
+        dl.forward(xt, lg, out=out, ws=ws)
+        torch.cuda.synchronize(dev)
+        stage_ms += np.array([sev[i].elapsed_time(sev[i + 1]) for i in range(len(STAGES))])
+    tq.tileq_set_stage_events(None)
+    stage_ms /= nprof
+    stage_times = {n: round(float(t), 5) for n, t in zip(STAGES, stage_ms)}
+
+    peaks = measured_peaks()
+    dom = max(("gateup", "residual", "zproj", "zdown", "shared"),
+              key=lambda n: stage_times.get(n, 0.0) if n in wk["stages"] else -1)
+    dw = wk["stages"][dom]
+    t_dom = stage_times[dom] / 1000.0
+    hbm_s = dw["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    tc_s = dw["flops"] / (peaks["bf16_tflops"] * 1e12)
+    if hbm_s >= tc_s:
+        roof = {"bound": "hbm", "achieved": dw["bytes"] / t_dom / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": dw["flops"] / t_dom / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["kernel_ms"] = stage_times[dom]
+    roof["alg_bytes"] = dw["bytes"]
+    roof["alg_flops"] = dw["flops"]
+    roof["peak_source"] = peaks["source"]
+    roof["traffic"] = traffic_for(dom, T, cfg)
+    whole = {"alg_bytes": wk["bytes"], "alg_flops": wk["flops"],
+             "t_roof_ms": 1000 * max(wk["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                                     wk["flops"] / (peaks["bf16_tflops"] * 1e12))}
+    whole["frac_of_roofline"] = whole["t_roof_ms"] / ms_per_step
+
+    # ---------------- end to end through the public API with host buffers
+    x_h = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    lg_h = torch.from_numpy(logits_np).pin_memory()
+    out_h = torch.empty((T, dl.d_y), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(xt)
+    lgd = torch.empty_like(lg)
+    for _ in range(3):
+        xd.copy_(x_h, non_blocking=True)
+        lgd.copy_(lg_h, non_blocking=True)
+        dl.forward(xd, lgd, out=out, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        xd.copy_(x_h, non_blocking=True)
+        lgd.copy_(lg_h, non_blocking=True)
+        dl.forward(xd, lgd, out=out, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+    e2e = {"value": world * T * args.steps / (e2e_ms / 1000.0), "unit": "tokens/s",
+           "h2d_bytes_per_step": x_h.numel() * 2 + lg_h.numel() * 4,
+           "d2h_bytes_per_step": out_h.numel() * 2}
+
+    # ---------------- in-run comparisons (rank 0, N = 1)
+    extra = {}
+    if rank == 0 and world == 1 and not args.no_compare:
+        extra = compare_paths(cfg, layer, dl, xt, lg, out, T, args, flush_buf, ms_per_step)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(layer, x_np, logits_np, n_tokens=1)
+
+    if rank == 0:
+        line = {
+            "metric": metric_name(cfg, T), "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic (seeded numpy draws in the stored TileQ format)",
+            "config": workload_config(cfg, T, args,
+                                      "L2 flushed (256 MB write) between steps" if flush else
+                                      f"working set {footprint / 2**20:.0f} MB > 3x L2, no flush"),
+            "roofline": roof, "whole_step": whole, "stage_ms": stage_times,
+            "e2e": e2e, "gpu_launches": launches, "cpu_baseline": cpu,
+            "clocks": clocks.report(),
+        }
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def traffic_for(kernel, T, cfg):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    key = f"{kernel}:{cfg.name}:T={T}"
+    ent = d.get(key)
+    if not ent or ent.get("source_sha") != source_sha():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tiled_rank_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def compare_paths(cfg, layer, dl, xt, lg, out, T, args, flush_buf, fused_ms):
+    """Unfused per-expert low-rank path and the rank-0 (residual only) layer, same batch."""
+    import torch
+    import tiled_rank_b200 as tq
+    dev = xt.device
+    res = {}
+
+    def time_fn(fn, n):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        tot = 0.0
+        for _ in range(n):
+            if flush_buf is not None:
+                flush_buf.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize(dev)
+            tot += a.elapsed_time(b)
+        return tot / n
+
+    n = max(3, min(args.steps, 20))
+    pe = [synth.per_expert_lowrank(layer, p) for p in layer.projs]
+    dl.set_per_expert(pe)
+    t_unf = time_fn(lambda: dl.forward(xt, lg, out=out, unfused=True), n)
+    res["unfused"] = {"ms_per_step": t_unf, "value": T / (t_unf / 1000.0),
+                      "fusion_gain": t_unf / fused_ms}
+    dl.packed_pe = None
+    r0 = tq.DeviceLayer(synth.make_layer(cfg, seed=args.seed, rank=0), dev)
+    t_r0 = time_fn(lambda: r0.forward(xt, lg, out=out), n)
+    res["rank0"] = {"ms_per_step": t_r0, "lowrank_overhead": fused_ms / t_r0 - 1.0}
+    del r0
+    return res
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,200 @@
+/*
+ * tileq.h — C ABI of the TileQ fused MoE-layer forward for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (TileQ paper, "TileQ: Efficient Low-Rank Quantization of
+ * Mixture-of-Experts with 2D Tiling"):
+ *
+ *   The K experts of a projection sit on an M x N tile grid.  Expert k at cell
+ *   (m, n) applies  W_k = U_m diag(Sigma) V_n^T + deq(Q_k)  where U_m is the
+ *   row-m block of the shared left (output-space) factor of the tiled block
+ *   matrix W_big, V_n the column-n block of its shared right (input-space)
+ *   factor, Sigma the shared diagonal, and deq(Q_k) the expert's 2-bit
+ *   group-quantised residual (section 2.1, step 5 and the key technical
+ *   insight).  The forward runs the fused low-rank inference of section 2.2
+ *   ("Efficient Fused Sparse Low-Rank Inference", LoTileMoE): z = Sigma*(V_n^T x)
+ *   is computed once per (token, grid column), U_m is applied per grid row
+ *   through an in-place accumulation buffer, and the residual runs as one
+ *   grouped GEMM instead of K small ones.
+ *
+ *   Routing (implicit on the pages: only a few experts are active per token):
+ *   top-k of the fp32 router logits in descending order, equal logits -> the
+ *   lower expert index first; weights = softmax over the k chosen logits.
+ *   LINEAR layer:  out_t = sum_j w_j W_{e_j} x_t
+ *   SWIGLU layer:  out_t = sum_j w_j W^down_{e_j} (silu(W^gate_{e_j} x_t) * (W^up_{e_j} x_t))
+ *                  (+ an optional always-on dense bf16 SwiGLU shared expert, weight 1)
+ *
+ * Conventions for every call:
+ *   - Tensors are caller-owned.  "device" pointers are CUDA global memory of
+ *     the current device; "host" pointers are ordinary host memory.  Every
+ *     device pointer must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream)
+ *     unless stated otherwise.  Host-side validation errors are returned
+ *     before anything is enqueued.  Launch failures return TILEQ_ERR_CUDA.
+ *   - The library never allocates device memory: the packed weights and the
+ *     workspace are sized by query and passed in.
+ *   - Outputs are overwritten, never accumulated into.
+ *   - Bounded device waits that give up write TILEQ_ERR_TIMEOUT into the
+ *     workspace status word (read it with tileq_device_status).
+ */
+#ifndef TILEQ_H_
+#define TILEQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *tileq_stream_t;
+
+typedef enum {
+  TILEQ_OK = 0,
+  TILEQ_ERR_INVALID_ARG = -1,  /* null pointer, bad size, non-injective grid, bad top_k   */
+  TILEQ_ERR_UNSUPPORTED = -2,  /* shape outside the supported tiling (see tileq_proj)     */
+  TILEQ_ERR_WORKSPACE = -3,    /* workspace or packed buffer smaller than the query says  */
+  TILEQ_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed             */
+  TILEQ_ERR_TIMEOUT = -5       /* a bounded device wait gave up (device status word)      */
+} tileq_status;
+
+enum { TILEQ_LINEAR = 0, TILEQ_SWIGLU = 1 };
+
+/* One TileQ-compressed projection (d_out x d_in) of all K experts, in the
+ * stored format (section 2.1, steps 4-5):
+ *   grid_assign  HOST int32 [K]: cell m*N + n of expert k; must be injective.
+ *   U            device bf16 [M*d_out, rank], row-major; block m = rows m*d_out..
+ *   Sigma        device fp32 [rank]
+ *   V            device bf16 [N*d_in, rank], row-major; block n = rows n*d_in..
+ *   codes        device uint32 [K, d_out, d_in/16]; element j of a word at bits 2*(j%16)
+ *   scales       device fp16 [K, d_out, d_in/group]
+ *   zeros        device uint8 [K, d_out, ceil(d_in/group/4)]; group j at bits 2*(j%4)
+ *                of byte j/4
+ *   Residual: w[o,i] = scales[o,i/group] * (q[o,i] - z[o,i/group]).
+ * Supported: d_out % 16 == 0, d_in % 128 == 0, group % 32 == 0, d_in % group == 0,
+ * 0 <= rank <= 256 and rank % 16 == 0 (rank 0 = residual only); otherwise
+ * TILEQ_ERR_UNSUPPORTED. */
+typedef struct {
+  int d_in, d_out, rank, group;
+  const int32_t *grid_assign;
+  const void *U;
+  const float *Sigma;
+  const void *V;
+  const uint32_t *codes;
+  const void *scales;
+  const uint8_t *zeros;
+} tileq_proj;
+
+/* A TileQ MoE layer.
+ *   kind = TILEQ_LINEAR: proj[0] only; x is [T, proj[0].d_in], out is [T, proj[0].d_out].
+ *   kind = TILEQ_SWIGLU: proj[0] = gate (d_ff x d_model), proj[1] = up (d_ff x d_model),
+ *                        proj[2] = down (d_model x d_ff); x and out are [T, d_model].
+ *   shared_d_ff > 0 adds a dense SwiGLU shared expert (SWIGLU only):
+ *   shared_w[0] gate, shared_w[1] up: device bf16 [shared_d_ff, d_model];
+ *   shared_w[2] down: device bf16 [d_model, shared_d_ff]; shared_d_ff % 128 == 0. */
+typedef struct {
+  int kind;
+  int K, M, N;            /* experts and grid; K <= M*N; K, M, N <= 64 */
+  int d_model, d_ff;      /* SWIGLU widths (ignored for LINEAR) */
+  tileq_proj proj[3];
+  int shared_d_ff;
+  const void *shared_w[3];
+} tileq_layer;
+
+/* Optional copies of the routing results (device pointers, each may be NULL). */
+typedef struct {
+  int32_t *topk_idx;        /* [T, top_k] expert ids, descending logit               */
+  float *topk_w;            /* [T, top_k] softmax weights over the chosen logits      */
+  int32_t *expert_offsets;  /* [K+1] range of each expert in sorted_pairs             */
+  int32_t *sorted_pairs;    /* [T*top_k] pair ids t*top_k+j, stably sorted by expert  */
+} tileq_route_out;
+
+/* Independent per-expert low-rank factors of one projection (the disjoint
+ * per-expert layout the paper compares against, section 1 "Inference
+ * Latency"): U_pe device bf16 [K, d_out, rank], V_pe device bf16 [K, d_in, rank]. */
+typedef struct {
+  const void *U_pe[3];
+  const void *V_pe[3];
+} tileq_per_expert_lr;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *tileq_status_string(tileq_status s);
+
+/* Bytes of the packed (kernel-layout) copy of `layer`.  Host only, synchronous. */
+tileq_status tileq_packed_size(const tileq_layer *layer, size_t *bytes);
+
+/* Repack `layer` into `packed` (device, packed_bytes >= tileq_packed_size).
+ * Reads the layer's device arrays and host grid_assign; validates the grid is
+ * injective.  Asynchronous on `stream`; the layer's arrays must stay valid
+ * until the stream reaches this call.  Call once per set of weights. */
+tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_bytes,
+                        tileq_stream_t stream);
+
+/* Workspace bytes needed by tileq_moe_forward / tileq_route for T tokens. */
+tileq_status tileq_workspace_size(const tileq_layer *layer, int T, int top_k, size_t *bytes);
+
+/* The fused TileQ MoE-layer forward (section 2.2).
+ *   layer, packed   the descriptor and its packed copy (from tileq_pack)
+ *   x               device bf16 [T, d_x]       router_logits  device fp32 [T, K]
+ *   out             device bf16 [T, d_y]       (overwritten)
+ *   ws, ws_bytes    device workspace, ws_bytes >= tileq_workspace_size(layer, T, top_k)
+ *   route           optional copies of the routing results (NULL = none)
+ * 1 <= top_k <= K; T >= 0 (T == 0 enqueues nothing).  Asynchronous. */
+tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, const void *x,
+                               int T, const float *router_logits, int top_k, void *out,
+                               void *ws, size_t ws_bytes, tileq_route_out *route,
+                               tileq_stream_t stream);
+
+/* Bytes of the packed copy of a per-expert low-rank layout. */
+tileq_status tileq_packed_per_expert_size(const tileq_layer *layer, size_t *bytes);
+
+/* Repack the per-expert factors `pe` (same shapes as layer->proj) into `packed_pe`. */
+tileq_status tileq_pack_per_expert(const tileq_layer *layer, const tileq_per_expert_lr *pe,
+                                   void *packed_pe, size_t packed_pe_bytes,
+                                   tileq_stream_t stream);
+
+/* The unfused comparison path: the same residual GEMMs, but the low-rank term
+ * of every expert runs as its own launches from the per-expert layout (K small
+ * GEMMs per projection and stage, no sharing across grid rows or columns).
+ * Same arguments and result as tileq_moe_forward plus `packed_pe`. */
+tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *packed,
+                                       const void *packed_pe, const void *x, int T,
+                                       const float *router_logits, int top_k, void *out,
+                                       void *ws, size_t ws_bytes, tileq_route_out *route,
+                                       tileq_stream_t stream);
+
+/* Routing and permutation alone: top-k, softmax weights and the stable
+ * counting sort of the T*top_k pairs by expert.  Outputs as in tileq_route_out
+ * (all four required).  ws as for tileq_moe_forward (tileq_workspace_size). */
+tileq_status tileq_route(const float *router_logits, int T, int K, int top_k,
+                         tileq_route_out *route, void *ws, size_t ws_bytes,
+                         tileq_stream_t stream);
+
+/* Synchronously read (and clear) the device status word in `ws`.
+ * *status receives TILEQ_OK or the first device error recorded. */
+tileq_status tileq_device_status(void *ws, int *status, tileq_stream_t stream);
+
+/* Self-test of the bounded device wait: launches one block that waits on an
+ * mbarrier nothing arrives on, for at most `max_polls` polls, then records
+ * TILEQ_ERR_TIMEOUT in the status word of `ws` and returns.  Never hangs. */
+tileq_status tileq_selftest_bounded_wait(void *ws, size_t ws_bytes, int max_polls,
+                                         tileq_stream_t stream);
+
+/* Per-stage timing hook.  `events` holds n_events CUDA events (cudaEvent_t,
+ * caller-created and owned) or is NULL to switch the hook off.  While set,
+ * every tileq_moe_forward / tileq_moe_forward_unfused records event i on its
+ * stream at stage boundary i: 0 before routing, 1 after routing, 2 after the
+ * permutation, 3 after the column projection z = Sigma*(V_n^T x), 4 after the
+ * gate/up (or linear residual input) GEMM, 5 after the down-side projection,
+ * 6 after the row accumulation, 7 after the combined residual GEMM, 8 after
+ * the shared expert, 9 after the combine.  Events past n_events are skipped.
+ * Process-wide, not thread-safe; host only. */
+tileq_status tileq_set_stage_events(void **events, int n_events);
+
+/* Number of kernels the library has launched in this process so far. */
+tileq_status tileq_launch_count(unsigned long long *count);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TILEQ_H_ */

@@ -32,8 +32,7 @@ PINS (what each function is checked against, in tests/test_oracle.py):
       block of the global product U diag(Sigma) V^T (W_big), singular values of
       W_big == Sigma with orthonormal factors, 2D-sharing perturbation locality
   forward ... rank-0 == dense integer GEMM, zero residual == W_big block
-      product, SwiGLU / combine / shared-expert closed forms
-      (tests/golden/swiglu_closed_form.txt)
+      product, SwiGLU / combine / shared-expert closed forms written in the tests
 """
 from __future__ import annotations
 
@@ -130,12 +129,13 @@ def unpack_zeros(zeros, n_groups: int) -> np.ndarray:
 def dequant(proj, e: int) -> np.ndarray:
     """deq(Q_e) float64 [d_out, d_in]: w[o, i] = s[o, i//g] * (q[o, i] - z[o, i//g])."""
     g = proj.group
-    q = unpack_codes(proj.codes[e], proj.d_in).astype(np.float64)
-    z = unpack_zeros(proj.zeros[e], proj.d_in // g).astype(np.float64)
+    G = proj.d_in // g
+    q = unpack_codes(proj.codes[e], proj.d_in).reshape(proj.d_out, G, g)
+    z = unpack_zeros(proj.zeros[e], G).astype(np.float64)
     s = widen_fp16(proj.scales[e])
-    z_full = np.repeat(z, g, axis=1)
-    s_full = np.repeat(s, g, axis=1)
-    return s_full * (q - z_full)
+    # group j of row o covers inputs j*g .. j*g+g-1
+    w = (q - z[:, :, None]) * s[:, :, None]
+    return w.reshape(proj.d_out, proj.d_in)
 
 
 # ---------------------------------------------------------------------------

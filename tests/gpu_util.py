@@ -1,0 +1,57 @@
+"""Helpers of the GPU parity tests (CUDA path vs the fp64 oracle)."""
+from __future__ import annotations
+
+import numpy as np
+
+import synth
+
+# parity bar: max|gpu - ref| <= 1e-2 * max|ref| and sum|gpu - ref| / sum|ref| <= 2e-3
+MAX_REL = 1e-2
+MEAN_REL = 2e-3
+
+
+def parity_stats(gpu, ref):
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    diff = np.abs(g - r)
+    return {
+        "max_abs": float(diff.max()) if diff.size else 0.0,
+        "max_ref": float(np.abs(r).max()) if r.size else 0.0,
+        "mean_rel": float(diff.sum() / max(np.abs(r).sum(), 1e-300)),
+    }
+
+
+def assert_parity(gpu, ref, what=""):
+    s = parity_stats(gpu, ref)
+    assert np.all(np.isfinite(np.asarray(gpu, dtype=np.float64))), f"{what}: non-finite output"
+    assert s["max_abs"] <= MAX_REL * s["max_ref"], f"{what}: {s}"
+    assert s["mean_rel"] <= MEAN_REL, f"{what}: {s}"
+    return s
+
+
+def to_numpy(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        t = t.float()
+    return t.detach().cpu().numpy()
+
+
+def device_inputs(logits, x, device):
+    import torch
+    lg = torch.from_numpy(np.ascontiguousarray(logits)).to(device)
+    xt = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(device).view(torch.bfloat16)
+    return lg, xt
+
+
+def zero_residual(layer: synth.Layer) -> synth.Layer:
+    """Same layer with every residual code equal to its group's zero point (deq == 0)."""
+    projs = []
+    for p in layer.projs:
+        G = p.d_in // p.group
+        zb = p.zeros
+        z = np.stack([(zb[..., j // 4] >> (2 * (j % 4))) & 3 for j in range(G)], axis=-1)
+        words_per_group = p.group // 16
+        zw = np.repeat(z.astype(np.uint32), words_per_group, axis=-1) * np.uint32(0x55555555)
+        projs.append(synth.Proj(**{**p.__dict__, "codes": np.ascontiguousarray(zw)}))
+    return synth.Layer(layer.kind, layer.K, layer.M, layer.N, layer.d_model, layer.d_ff,
+                       layer.top_k, projs, layer.shared)

@@ -1,0 +1,143 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+the ctypes structs match the C layout, and host-side validation rejects bad
+arguments before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tileq.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from tiled_rank_b200 import _lib
+    if not os.path.exists(_lib.LIB_PATH):
+        from tiled_rank_b200 import build
+        build.build()
+    return _lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|tileq_status)\s*(tileq_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    fns = declared_functions()
+    assert "tileq_moe_forward" in fns and "tileq_route" in fns and "tileq_pack" in fns
+    assert len(fns) >= 11
+
+
+def test_library_exports_every_declared_symbol(L):
+    lib = ctypes.CDLL(L.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(L.EXPORTS) == set(declared_functions())
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (tileq_\w+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_struct_layout_matches_c(L, tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "tileq.h"\n'
+                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\\n",'
+                   'sizeof(tileq_proj), offsetof(tileq_proj, grid_assign), offsetof(tileq_proj, zeros),'
+                   'sizeof(tileq_layer), offsetof(tileq_layer, proj), offsetof(tileq_layer, shared_d_ff),'
+                   'offsetof(tileq_layer, shared_w), sizeof(tileq_route_out), sizeof(tileq_per_expert_lr));'
+                   'return 0;}\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
+    want = [ctypes.sizeof(L.tileq_proj), L.tileq_proj.grid_assign.offset, L.tileq_proj.zeros.offset,
+            ctypes.sizeof(L.tileq_layer), L.tileq_layer.proj.offset, L.tileq_layer.shared_d_ff.offset,
+            L.tileq_layer.shared_w.offset, ctypes.sizeof(L.tileq_route_out),
+            ctypes.sizeof(L.tileq_per_expert_lr)]
+    assert got == want
+
+
+def _host_layer(L, cfg, rank=None, grids=None):
+    """A tileq_layer with shapes and host grids only (device pointers left NULL)."""
+    layer = synth.make_layer(cfg, seed=0, rank=rank) if not isinstance(cfg, synth.Layer) else cfg
+    c = L.tileq_layer()
+    c.kind, c.K, c.M, c.N = layer.kind, layer.K, layer.M, layer.N
+    c.d_model, c.d_ff = layer.d_model, layer.d_ff
+    keep = []
+    for i, p in enumerate(layer.projs):
+        g = np.ascontiguousarray(p.grid_assign if grids is None else grids[i], dtype=np.int32)
+        keep.append(g)
+        c.proj[i].d_in, c.proj[i].d_out, c.proj[i].rank, c.proj[i].group = p.d_in, p.d_out, p.rank, p.group
+        c.proj[i].grid_assign = g.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    c.shared_d_ff = layer.shared_d_ff
+    c._keep = keep
+    return c, layer
+
+
+def test_packed_size_closed_form(L):
+    c, layer = _host_layer(L, 0)
+    p = layer.projs[0]
+    expect = 0
+    for nbytes in (4 * p.d_out * p.d_in // 4, 4 * p.d_out * (p.d_in // p.group) * 4,
+                   2 * p.d_out * p.rank * 2, 2 * p.d_in * p.rank * 2):
+        expect += (nbytes + 255) // 256 * 256
+    assert L.tileq_packed_size(c) == expect
+
+
+def test_workspace_size_grows_with_T(L):
+    c, _ = _host_layer(L, 0)
+    a = L.tileq_workspace_size(c, 1, 2)
+    b = L.tileq_workspace_size(c, 64, 2)
+    assert 0 < a < b
+
+
+def test_validation_rejects_bad_layers(L):
+    c, layer = _host_layer(L, 0)
+    bad_grid = np.array([0, 1, 1, 3], dtype=np.int32)            # not injective
+    c2, _ = _host_layer(L, 0, grids=[bad_grid])
+    with pytest.raises(L.TileQError) as e:
+        L.tileq_packed_size(c2)
+    assert e.value.status == L.TILEQ_ERR_INVALID_ARG
+    c3, _ = _host_layer(L, 0, grids=[np.array([0, 1, 2, 4], dtype=np.int32)])  # cell out of grid
+    with pytest.raises(L.TileQError):
+        L.tileq_workspace_size(c3, 4, 2)
+    c.proj[0].d_in = 96                                           # not a multiple of 128
+    with pytest.raises(L.TileQError) as e:
+        L.tileq_packed_size(c)
+    assert e.value.status == L.TILEQ_ERR_UNSUPPORTED
+    c.proj[0].d_in = 256
+    with pytest.raises(L.TileQError) as e:
+        L.tileq_workspace_size(c, 4, 5)                           # top_k > K
+    assert e.value.status == L.TILEQ_ERR_INVALID_ARG
+
+
+def test_forward_validation_before_launch(L):
+    """Errors are returned before any CUDA call: no device is needed."""
+    c, _ = _host_layer(L, 0)
+    lib = L.lib()
+    fake = ctypes.c_void_p(0x10000)
+    # NULL packed/x/logits/out/ws -> INVALID_ARG (device pointers of the layer unset too)
+    st = lib.tileq_moe_forward(ctypes.byref(c), None, None, 4, None, 2, None, None, 0, None, None)
+    assert st == L.TILEQ_ERR_INVALID_ARG
+    # T == 0 enqueues nothing and succeeds even with NULL pointers... once the layer is complete
+    for i in range(1):
+        c.proj[i].codes = c.proj[i].scales = c.proj[i].zeros = fake
+        c.proj[i].U = c.proj[i].V = c.proj[i].Sigma = fake
+    st = lib.tileq_moe_forward(ctypes.byref(c), None, None, 0, None, 2, None, None, 0, None, None)
+    assert st == L.TILEQ_OK
+    # too small a workspace
+    st = lib.tileq_moe_forward(ctypes.byref(c), fake, fake, 4, fake, 2, fake, fake, 16, None, None)
+    assert st == L.TILEQ_ERR_WORKSPACE
+    # bad top_k
+    st = lib.tileq_moe_forward(ctypes.byref(c), fake, fake, 4, fake, 0, fake, fake, 1 << 30, None, None)
+    assert st == L.TILEQ_ERR_INVALID_ARG
+    r = L.tileq_route_out()
+    st = lib.tileq_route(fake, 4, 4, 2, ctypes.byref(r), fake, 1 << 20, None)
+    assert st == L.TILEQ_ERR_INVALID_ARG                          # route outputs missing
+    assert L.status_string(L.TILEQ_ERR_TIMEOUT) == "TILEQ_ERR_TIMEOUT"

@@ -1,0 +1,236 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Indices are compared bit-exactly; floating-point outputs must satisfy
+max|gpu-ref| <= 1e-2*max|ref| and sum|gpu-ref|/sum|ref| <= 2e-3.  Small cases
+compare every output; full-size configurations compare seeded samples of
+tokens, which the oracle recomputes one by one.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import assert_parity, device_inputs, to_numpy, zero_residual
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import os
+    from tiled_rank_b200 import _lib
+    if not os.path.exists(_lib.LIB_PATH):
+        from tiled_rank_b200 import build
+        build.build()
+    return torch
+
+
+def run_gpu(torch, layer, logits, x, unfused=False, per_expert=None, dl=None):
+    from tiled_rank_b200 import DeviceLayer
+    dev = torch.device("cuda:0")
+    if dl is None:
+        dl = DeviceLayer(layer, dev, per_expert=per_expert)
+    lg, xt = device_inputs(logits, x, dev)
+    T = x.shape[0]
+    route = dl.route_buffers(T)
+    out = dl.forward(xt, lg, route=route, unfused=unfused)
+    torch.cuda.synchronize()
+    from tiled_rank_b200 import tileq_device_status
+    assert tileq_device_status(dl.workspace(T)) == 0
+    return to_numpy(out), {k: to_numpy(v) for k, v in route.items()}, dl
+
+
+def check_route(route, logits, top_k, K):
+    idx, w = oracle.route(logits, top_k)
+    assert np.array_equal(route["topk_idx"], idx)
+    np.testing.assert_allclose(route["topk_w"], w, rtol=2e-6, atol=1e-7)
+    off, sp = oracle.permute(idx, K)
+    assert np.array_equal(route["expert_offsets"], off)
+    assert np.array_equal(route["sorted_pairs"], sp)
+
+
+# ---------------------------------------------------------------------------
+# routing
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("T,K,k", [(1, 8, 2), (37, 4, 4), (1000, 60, 4), (4096, 8, 2), (2048, 64, 8)])
+def test_route_bitexact(torch_cuda, T, K, k):
+    torch = torch_cuda
+    from tiled_rank_b200 import tileq_route
+    rng = np.random.default_rng(T * 131 + K)
+    # quantised logits: many exact ties between experts
+    logits = (np.round(rng.standard_normal((T, K)) * 4) / 4).astype(np.float32)
+    dev = torch.device("cuda:0")
+    lg = torch.from_numpy(logits).to(dev)
+    route = {
+        "topk_idx": torch.empty((T, k), dtype=torch.int32, device=dev),
+        "topk_w": torch.empty((T, k), dtype=torch.float32, device=dev),
+        "expert_offsets": torch.empty((K + 1,), dtype=torch.int32, device=dev),
+        "sorted_pairs": torch.empty((T * k,), dtype=torch.int32, device=dev),
+    }
+    ws = torch.zeros(64 << 20, dtype=torch.uint8, device=dev)
+    tileq_route(lg, T, K, k, route, ws)
+    torch.cuda.synchronize()
+    check_route({n: to_numpy(v) for n, v in route.items()}, logits, k, K)
+
+
+# ---------------------------------------------------------------------------
+# small layers: every output
+# ---------------------------------------------------------------------------
+def test_config0_full(torch_cuda):
+    cfg = synth.CONFIGS[0]
+    layer = synth.make_layer(cfg)
+    logits, x = synth.make_inputs(cfg, 64)
+    out, route, _ = run_gpu(torch_cuda, layer, logits, x)
+    check_route(route, logits, cfg.top_k, cfg.K)
+    assert_parity(out, oracle.forward(layer, x, logits), "config 0")
+
+
+@pytest.mark.parametrize("variant", ["zero_residual", "rank0"])
+def test_config0_single_terms(torch_cuda, variant):
+    """Each term alone (the low-rank term is too small to be seen in the sum)."""
+    cfg = synth.CONFIGS[0]
+    layer = zero_residual(synth.make_layer(cfg)) if variant == "zero_residual" else \
+        synth.make_layer(cfg, rank=0)
+    logits, x = synth.make_inputs(cfg, 64)
+    out, _, _ = run_gpu(torch_cuda, layer, logits, x)
+    assert_parity(out, oracle.forward(layer, x, logits), f"config 0 {variant}")
+
+
+TINY = [
+    # (kind, K, M, N, d_model, d_ff, rank, group, top_k, shared, T)
+    (synth.SWIGLU, 6, 2, 3, 128, 384, 16, 32, 2, 0, 37),
+    (synth.SWIGLU, 4, 2, 2, 256, 256, 32, 64, 4, 0, 5),       # top_k == K
+    (synth.SWIGLU, 8, 2, 4, 128, 256, 48, 128, 2, 256, 100),  # shared expert, odd rank/16
+    (synth.LINEAR, 5, 2, 3, 384, 144, 16, 128, 3, 0, 1),
+    (synth.LINEAR, 9, 3, 3, 128, 64, 0, 32, 2, 0, 300),
+    (synth.SWIGLU, 12, 3, 4, 128, 128, 16, 128, 1, 0, 513),
+]
+
+
+@pytest.mark.parametrize("case", TINY, ids=[f"tiny{i}" for i in range(len(TINY))])
+def test_tiny_layers(torch_cuda, case):
+    kind, K, M, N, dm, dff, r, g, k, sh, T = case
+    cfg = synth.tiny_config(kind=kind, K=K, M=M, N=N, d_model=dm, d_ff=dff, rank=r, group=g,
+                            top_k=k, shared_d_ff=sh)
+    layer = synth.make_layer(cfg, seed=T)
+    logits, x = synth.make_inputs(cfg, T, seed=T)
+    out, route, _ = run_gpu(torch_cuda, layer, logits, x)
+    check_route(route, logits, k, K)
+    assert_parity(out, oracle.forward(layer, x, logits), str(case))
+    if r > 0:
+        zr = zero_residual(layer)
+        out, _, _ = run_gpu(torch_cuda, zr, logits, x)
+        assert_parity(out, oracle.forward(zr, x, logits), f"{case} zero residual")
+
+
+@pytest.mark.parametrize("case", [TINY[0], TINY[3], TINY[2]], ids=["swiglu", "linear", "shared"])
+def test_unfused_path(torch_cuda, case):
+    kind, K, M, N, dm, dff, r, g, k, sh, T = case
+    cfg = synth.tiny_config(kind=kind, K=K, M=M, N=N, d_model=dm, d_ff=dff, rank=r, group=g,
+                            top_k=k, shared_d_ff=sh)
+    layer = synth.make_layer(cfg, seed=3)
+    logits, x = synth.make_inputs(cfg, T, seed=3)
+    pe = [synth.per_expert_lowrank(layer, p) for p in layer.projs]
+    ref = oracle.forward(layer, x, logits)
+    out_u, route, dl = run_gpu(torch_cuda, layer, logits, x, unfused=True, per_expert=pe)
+    check_route(route, logits, k, K)
+    assert_parity(out_u, ref, f"unfused {case}")
+    zr = zero_residual(layer)
+    out_z, _, _ = run_gpu(torch_cuda, zr, logits, x, unfused=True, per_expert=pe)
+    assert_parity(out_z, oracle.forward(zr, x, logits), f"unfused zero residual {case}")
+
+
+def test_empty_batch_and_status(torch_cuda):
+    torch = torch_cuda
+    from tiled_rank_b200 import DeviceLayer, tileq_device_status, tileq_selftest_bounded_wait
+    cfg = synth.CONFIGS[0]
+    dl = DeviceLayer(synth.make_layer(cfg), torch.device("cuda:0"))
+    dev = torch.device("cuda:0")
+    x = torch.empty((0, cfg.d_model), dtype=torch.bfloat16, device=dev)
+    lg = torch.empty((0, cfg.K), dtype=torch.float32, device=dev)
+    out = dl.forward(x, lg)
+    assert out.shape == (0, cfg.d_ff)
+    ws = dl.workspace(4)
+    tileq_selftest_bounded_wait(ws, 1000)
+    assert tileq_device_status(ws) == -5          # TILEQ_ERR_TIMEOUT recorded by the bounded wait
+    assert tileq_device_status(ws) == 0           # and cleared by the read
+
+
+def test_deterministic(torch_cuda):
+    cfg = synth.tiny_config(K=8, M=2, N=4, d_model=256, d_ff=512, rank=32, group=128, top_k=2)
+    layer = synth.make_layer(cfg, seed=9)
+    logits, x = synth.make_inputs(cfg, 200, seed=9)
+    a, _, dl = run_gpu(torch_cuda, layer, logits, x)
+    b, _, _ = run_gpu(torch_cuda, layer, logits, x, dl=dl)
+    assert np.array_equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# full-size configurations (sampled tokens)
+# ---------------------------------------------------------------------------
+def _sample(T, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(T, size=min(n, T), replace=False))
+
+
+def _full_config_check(torch, cfg_ids, samples, variants=("normal", "zero_residual", "rank0")):
+    """One oracle pass per layer variant over the sampled tokens of every batch."""
+    from tiled_rank_b200 import DeviceLayer
+    cfg0 = synth.CONFIGS[cfg_ids[0]]
+    base = synth.make_layer(cfg0)
+    for variant in variants:
+        if variant == "normal":
+            layer = base
+        elif variant == "zero_residual":
+            layer = zero_residual(base)
+        else:
+            layer = synth.make_layer(cfg0, rank=0)
+        dl = DeviceLayer(layer, torch.device("cuda:0"))
+        xs, ls, gpu_rows = [], [], []
+        for cid in cfg_ids:
+            cfg = synth.CONFIGS[cid]
+            for T in cfg.batches:
+                logits, x = synth.make_inputs(cfg, T)
+                out, route, _ = run_gpu(torch, layer, logits, x, dl=dl)
+                if variant == "normal":
+                    check_route(route, logits, cfg.top_k, cfg.K)
+                toks = _sample(T, samples, seed=T)
+                xs.append(x[toks])
+                ls.append(logits[toks])
+                gpu_rows.append(out[toks])
+                del dl._ws[(T, cfg.top_k)]
+        ref = oracle.forward(layer, np.concatenate(xs), np.concatenate(ls))
+        assert_parity(np.concatenate(gpu_rows), ref, f"configs {cfg_ids} {variant}")
+        del dl
+
+
+@pytest.mark.slow
+def test_mixtral_shaped_decode_and_prefill(torch_cuda):
+    _full_config_check(torch_cuda, (1, 2), samples=3)
+
+
+@pytest.mark.slow
+def test_qwen15moe_shaped(torch_cuda):
+    _full_config_check(torch_cuda, (3,), samples=6)
+
+
+@pytest.mark.slow
+def test_finegrained_64e(torch_cuda):
+    _full_config_check(torch_cuda, (4,), samples=4)
+
+
+@pytest.mark.slow
+def test_finegrained_64e_unfused(torch_cuda):
+    torch = torch_cuda
+    cfg = synth.CONFIGS[4]
+    layer = synth.make_layer(cfg)
+    pe = [synth.per_expert_lowrank(layer, p) for p in layer.projs]
+    T = cfg.batches[0]
+    logits, x = synth.make_inputs(cfg, T)
+    out, route, dl = run_gpu(torch, layer, logits, x, unfused=True, per_expert=pe)
+    check_route(route, logits, cfg.top_k, cfg.K)
+    toks = _sample(T, 3, seed=1)
+    assert_parity(out[toks], oracle.forward(layer, x, logits, tokens=toks), "config 4 unfused")

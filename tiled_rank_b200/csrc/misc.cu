@@ -1,0 +1,95 @@
+// Small element-wise kernels of the TileQ forward: the in-place accumulation
+// of the low-rank projections per (token, grid row), the weighted top-k
+// combine / unpermute, and the helpers of the unfused comparison path.
+#include "kernels.cuh"
+
+namespace tileq {
+
+// a[(t,m)][i] = sum over the token's slots j whose expert sits in grid row m of
+//   zslot[slot(t,j)][i]                (SwiGLU down: routing weight already in h)
+// or w_j * zcol[zidx(slot(t,j))][i]    (linear layer: z per (token, column))
+// TileQ paper, section 2.2: routing weights select the active tiles of the
+// projected [T, N, r] tensor and an in-place buffer accumulates them per grid
+// row, so the shared left factor U_m is applied once per (token, row).
+__global__ void lr_accumulate_kernel(LrAccArgs a) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int c = (int)(gid / a.r), i = (int)(gid % a.r);
+  if (c >= a.row_offsets[a.M]) return;
+  const int t = a.rowpair_tok[c], m = a.rowpair_row[c];
+  float acc = 0.f;
+  for (int j = 0; j < a.k; ++j) {
+    const int p = t * a.k + j;
+    if (a.m_of[a.topk_idx[p]] != m) continue;
+    const int slot = a.slot_of_pair[p];
+    if (a.zslot)
+      acc += a.zslot[(size_t)slot * a.r + i];
+    else
+      acc += a.topk_w[p] * __half2float(a.zcol[(size_t)a.zidx[slot] * a.r + i]);
+  }
+  a.a[(size_t)c * a.r + i] = __float2half_rn(acc);
+}
+
+// out[t][:] = yshared[t][:] + sum_j sum_split ybuf[split][slot(t,j)][:], in bf16.
+// Fixed summation order, so the result is deterministic.
+__global__ void combine_kernel(CombineArgs a) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int d4 = a.d / 4;
+  const int t = (int)(gid / d4), c = (int)(gid % d4);
+  if (t >= a.T) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (a.yshared) acc = reinterpret_cast<const float4 *>(a.yshared + (size_t)t * a.d)[c];
+  for (int j = 0; j < a.k; ++j) {
+    const int slot = a.slot_of_pair[t * a.k + j];
+    for (int s = 0; s < a.ksplit; ++s) {
+      const float4 v =
+          reinterpret_cast<const float4 *>(a.ybuf + s * a.split_stride + (size_t)slot * a.d)[c];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+  }
+  __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(a.out + (size_t)t * a.d + c * 4);
+  o[0] = __floats2bfloat162_rn(acc.x, acc.y);
+  o[1] = __floats2bfloat162_rn(acc.z, acc.w);
+}
+
+// xs[slot][:] = w_slot * x16[token(slot)][:]  (fp16), for the linear layer.
+__global__ void scale_gather_kernel(ScaleGatherArgs a) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int d2 = a.d / 2;
+  const int s = (int)(gid / d2), c = (int)(gid % d2);
+  if (s >= a.P) return;
+  const float w = a.slot_w[s];
+  const __half2 v = reinterpret_cast<const __half2 *>(a.x16 + (size_t)a.slot_tok[s] * a.d)[c];
+  const float2 f = __half22float2(v);
+  reinterpret_cast<__half2 *>(a.xs + (size_t)s * a.d)[c] = __floats2half2_rn(w * f.x, w * f.y);
+}
+
+// h[slot][f] = w_slot * silu(g) * u  (unfused path: activation after the per-expert adds)
+__global__ void swiglu_kernel(SwigluArgs a) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= a.n) return;
+  const int slot = (int)(i / a.F);
+  a.h[i] = __float2half_rn(a.slot_w[slot] * silu_f(a.g[i]) * a.u[i]);
+}
+
+// Bounded wait on an mbarrier that nothing arrives on: gives up after
+// max_polls polls and records TILEQ_ERR_TIMEOUT.  Exercises the same bounded
+// wait the pipelined kernels use, without any chance of a hang.
+__global__ void bounded_wait_kernel(int *status, int max_polls) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t addr = smem_addr(&bar);
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(addr) : "memory");
+  uint32_t done = 0;
+  for (int i = 0; i < max_polls && !done; ++i) {
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr)
+        : "memory");
+  }
+  if (!done) set_status(status, TILEQ_ERR_TIMEOUT);
+  asm volatile("mbarrier.inval.shared::cta.b64 [%0];\n" ::"r"(addr) : "memory");
+}
+
+}  // namespace tileq

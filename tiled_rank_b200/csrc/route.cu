@@ -1,0 +1,252 @@
+// Routing and permutation kernels of the TileQ MoE forward.
+//
+// route_kernel    : one warp per token: exact top-k of the fp32 logits (descending,
+//                   equal logits -> lower expert id), softmax over the chosen
+//                   logits, and the bf16 -> fp16 conversion of the token's x row.
+// permute_kernel  : one CTA: deterministic stable counting sorts of the
+//                   (token, slot) pairs by expert, of the distinct (token, grid
+//                   column) pairs by column (one z = Sigma*(V_n^T x) per pair,
+//                   TileQ paper section 2.2 "project the input once"), and of the
+//                   distinct (token, grid row) pairs by row (the in-place
+//                   accumulation buffer of section 2.2), plus the GEMM tile tables.
+#include "kernels.cuh"
+
+namespace tileq {
+
+__global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= a.T) return;
+  const int t = warp;
+  const float NEG = -INFINITY;
+  const float *lg = a.logits + (size_t)t * a.K;
+  float v0 = lane < a.K ? lg[lane] : NEG;
+  float v1 = lane + 32 < a.K ? lg[lane + 32] : NEG;
+  bool used0 = lane >= a.K, used1 = lane + 32 >= a.K;
+  float sel_v[kMaxTopK];
+  int sel_i[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    if (j < a.k) {
+      float bv = NEG;
+      int bi = 0x7fffffff;
+      if (!used0) { bv = v0; bi = lane; }
+      if (!used1 && (used0 || v1 > v0)) { bv = v1; bi = lane + 32; }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if (bi == lane) used0 = true;
+      if (bi == lane + 32) used1 = true;
+      sel_v[j] = bv;
+      sel_i[j] = bi;
+    }
+  }
+  float sum = 0.f;
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < a.k) sum += expf(sel_v[j] - sel_v[0]);
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j < a.k) {
+        a.topk_idx[t * a.k + j] = sel_i[j];
+        a.topk_w[t * a.k + j] = expf(sel_v[j] - sel_v[0]) / sum;
+      }
+    }
+  }
+  if (a.x != nullptr) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d_x);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.x16 + (size_t)t * a.d_x);
+    for (int c = lane; c < a.d_x / 8; c += 32) {
+      uint4 v = src[c];
+      const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v);
+      uint4 o;
+      __half2 *h = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) h[i] = __float22half2_rn(__bfloat1622float2(b[i]));
+      dst[c] = o;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// single-CTA stable counting sort
+// ---------------------------------------------------------------------------
+constexpr int kPermThreads = 1024;
+constexpr int kPermWarps = kPermThreads / 32;
+
+struct SortSmem {
+  int hist[kPermWarps][kMaxExperts];
+  int total[kMaxExperts + 1];
+};
+
+// Sort the items 0..n-1 whose key(i) >= 0 by key, stably.  dest[i] receives the
+// sorted position of a valid item; offsets[0..nkeys] the bucket starts.
+template <typename KeyFn>
+__device__ void cta_stable_sort(int n, int nkeys, KeyFn key, int *dest, int *offsets,
+                                SortSmem &s) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kPermWarps * kMaxExperts; i += blockDim.x)
+    (&s.hist[0][0])[i] = 0;
+  __syncthreads();
+  const int chunk = (n + kPermWarps - 1) / kPermWarps;
+  const int c0 = min(n, warp * chunk), c1 = min(n, c0 + chunk);
+  for (int i = c0 + lane; i < c1; i += 32) {
+    const int kk = key(i);
+    if (kk >= 0) atomicAdd(&s.hist[warp][kk], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x < nkeys) {
+    int tot = 0;
+    for (int w = 0; w < kPermWarps; ++w) tot += s.hist[w][threadIdx.x];
+    s.total[threadIdx.x] = tot;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int kk = 0; kk < nkeys; ++kk) {
+      const int tt = s.total[kk];
+      s.total[kk] = run;
+      offsets[kk] = run;
+      run += tt;
+    }
+    offsets[nkeys] = run;
+    s.total[nkeys] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x < nkeys) {
+    int run = s.total[threadIdx.x];
+    for (int w = 0; w < kPermWarps; ++w) {
+      const int c = s.hist[w][threadIdx.x];
+      s.hist[w][threadIdx.x] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int base = c0; base < c1; base += 32) {
+    const int i = base + lane;
+    const int kk = i < c1 ? key(i) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, kk);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int pos = 0;
+    if (kk >= 0) pos = s.hist[warp][kk] + rank;
+    __syncwarp();
+    if (kk >= 0) {
+      dest[i] = pos;
+      if (rank == 0) s.hist[warp][kk] += __popc(peers);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+}
+
+// Fill a tile table: group g owns items [off[g], off[g+1]) split into tiles of bn.
+__device__ void build_tiles(const int *off, int ngroups, int bn, int4 *tiles, int *count,
+                            int *first /* [ngroups+1] or null */,
+                            int *scratch /* smem [kMaxExperts+1] */) {
+  if (threadIdx.x < ngroups) {
+    const int cnt = off[threadIdx.x + 1] - off[threadIdx.x];
+    scratch[threadIdx.x] = (cnt + bn - 1) / bn;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int g = 0; g < ngroups; ++g) {
+      const int c = scratch[g];
+      scratch[g] = run;
+      run += c;
+    }
+    scratch[ngroups] = run;
+    *count = run;
+  }
+  __syncthreads();
+  if (first != nullptr && threadIdx.x <= ngroups) first[threadIdx.x] = scratch[threadIdx.x];
+  if (threadIdx.x < ngroups) {
+    const int g = threadIdx.x;
+    const int i0 = off[g], i1 = off[g + 1];
+    int ti = scratch[g];
+    for (int i = i0; i < i1; i += bn) tiles[ti++] = make_int4(g, i, min(bn, i1 - i), 0);
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
+  __shared__ SortSmem s;
+  __shared__ int scratch[kMaxExperts + 1];
+  const int P = a.T * a.k;
+  const int k = a.k;
+  const int32_t *idx = a.topk_idx;
+
+  // 1. pairs by expert
+  cta_stable_sort(P, a.K, [&](int p) { return idx[p]; }, a.dest, a.expert_offsets, s);
+  for (int p = threadIdx.x; p < P; p += blockDim.x) {
+    const int slot = a.dest[p];
+    a.sorted_pairs[slot] = p;
+    a.slot_of_pair[p] = slot;
+    a.slot_tok[slot] = p / k;
+    a.slot_w[slot] = a.topk_w[p];
+  }
+  __syncthreads();
+  build_tiles(a.expert_offsets, a.K, a.bn, a.tiles_main, a.tile_counts + 0, a.tile_first_main,
+              scratch);
+
+  // 2. distinct (token, grid column) pairs by column, per z projection
+  for (int zp = 0; zp < a.n_zproj; ++zp) {
+    const int8_t *ncol = a.n_of[zp];
+    auto key = [&](int p) {
+      const int t = p / k, j = p - t * k;
+      const int c = ncol[idx[p]];
+      for (int jj = 0; jj < j; ++jj)
+        if (ncol[idx[t * k + jj]] == c) return -1;
+      return c;
+    };
+    cta_stable_sort(P, a.N, key, a.dest, a.col_offsets[zp], s);
+    for (int p = threadIdx.x; p < P; p += blockDim.x) {
+      const int t = p / k, j = p - t * k;
+      const int c = ncol[idx[p]];
+      int jd = j;
+      for (int jj = 0; jj < j; ++jj)
+        if (ncol[idx[t * k + jj]] == c) { jd = jj; break; }
+      const int cp = a.dest[t * k + jd];
+      if (jd == j) a.colpair_tok[zp][cp] = t;
+      a.zidx[zp][a.slot_of_pair[p]] = cp;
+    }
+    __syncthreads();
+    build_tiles(a.col_offsets[zp], a.N, a.bn, a.tiles_z[zp], a.tile_counts + 1 + zp, nullptr,
+                scratch);
+  }
+
+  // 3. distinct (token, grid row) pairs by row of the combined projection
+  if (a.row_proj >= 0) {
+    const int8_t *mrow = a.m_of_row;
+    auto key = [&](int p) {
+      const int t = p / k, j = p - t * k;
+      const int r = mrow[idx[p]];
+      for (int jj = 0; jj < j; ++jj)
+        if (mrow[idx[t * k + jj]] == r) return -1;
+      return r;
+    };
+    cta_stable_sort(P, a.M, key, a.dest, a.row_offsets, s);
+    for (int p = threadIdx.x; p < P; p += blockDim.x) {
+      const int t = p / k, j = p - t * k;
+      const int r = mrow[idx[p]];
+      bool designated = true;
+      for (int jj = 0; jj < j; ++jj)
+        if (mrow[idx[t * k + jj]] == r) { designated = false; break; }
+      const int slot = a.slot_of_pair[p];
+      if (designated) {
+        const int rp = a.dest[p];
+        a.rowpair_tok[rp] = t;
+        a.rowpair_row[rp] = r;
+        a.aidx[slot] = rp;
+      } else {
+        a.aidx[slot] = -1;
+      }
+    }
+  }
+}
+
+}  // namespace tileq
