@@ -71,7 +71,8 @@ enum { TILEQ_LINEAR = 0, TILEQ_SWIGLU = 1 };
  *   zeros        device uint8 [K, d_out, ceil(d_in/group/4)]; group j at bits 2*(j%4)
  *                of byte j/4
  *   Residual: w[o,i] = scales[o,i/group] * (q[o,i] - z[o,i/group]).
- * Supported: d_out % 16 == 0, d_in % 128 == 0, group % 32 == 0, d_in % group == 0,
+ * Supported: d_out % 16 == 0, d_in % 128 == 0, group == 64 or a multiple of 128,
+ * d_in % group == 0,
  * 0 <= rank <= 256 and rank % 16 == 0 (rank 0 = residual only); otherwise
  * TILEQ_ERR_UNSUPPORTED. */
 typedef struct {

@@ -43,8 +43,13 @@ def device_inputs(logits, x, device):
     return lg, xt
 
 
-def zero_residual(layer: synth.Layer) -> synth.Layer:
-    """Same layer with every residual code equal to its group's zero point (deq == 0)."""
+def zero_residual(layer: synth.Layer, lr_gain: float = 1.0) -> synth.Layer:
+    """Same layer with every residual code equal to its group's zero point (deq == 0).
+
+    ``lr_gain`` (a power of two, exact in bf16) scales every U block, so that at
+    full model widths the low-rank-only activations keep realistic magnitudes
+    (unit-norm factors alone give outputs near 1e-6, below fp16's normal range).
+    """
     projs = []
     for p in layer.projs:
         G = p.d_in // p.group
@@ -52,6 +57,9 @@ def zero_residual(layer: synth.Layer) -> synth.Layer:
         z = np.stack([(zb[..., j // 4] >> (2 * (j % 4))) & 3 for j in range(G)], axis=-1)
         words_per_group = p.group // 16
         zw = np.repeat(z.astype(np.uint32), words_per_group, axis=-1) * np.uint32(0x55555555)
-        projs.append(synth.Proj(**{**p.__dict__, "codes": np.ascontiguousarray(zw)}))
+        U = p.U
+        if lr_gain != 1.0 and p.rank > 0:
+            U = synth.to_bf16_bits(synth.bf16_bits_to_f32(p.U) * np.float32(lr_gain))
+        projs.append(synth.Proj(**{**p.__dict__, "codes": np.ascontiguousarray(zw), "U": U}))
     return synth.Layer(layer.kind, layer.K, layer.M, layer.N, layer.d_model, layer.d_ff,
                        layer.top_k, projs, layer.shared)

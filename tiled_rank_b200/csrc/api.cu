@@ -1,9 +1,12 @@
 // C ABI of the TileQ MoE forward (include/tileq.h): host-side validation,
-// packed-weight and workspace layouts, and the launch sequence.
+// packed-weight and workspace layouts, the per-GEMM launch plan, and the
+// launch sequence of the fused and of the unfused (per-expert) forward.
 #include <algorithm>
 #include <atomic>
 #include <cstring>
 #include <vector>
+
+#include <cudaTypedefs.h>
 
 #include "kernels.cuh"
 
@@ -17,6 +20,9 @@ namespace {
 
 size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+unsigned nblocks(long long n, int per) { return (unsigned)((n + per - 1) / per); }
+
+constexpr int kNumSMs = 148;
 
 struct ProjInfo {
   int d_in, d_out, rank, group, G;
@@ -39,7 +45,8 @@ tileq_status validate_layer(const tileq_layer *L, LayerInfo *li, bool need_devic
     const tileq_proj &p = L->proj[pi];
     ProjInfo &q = li->p[pi];
     if (p.d_in <= 0 || p.d_out <= 0 || p.rank < 0 || p.group <= 0) return TILEQ_ERR_INVALID_ARG;
-    if (p.d_out % 16 || p.d_in % 128 || p.group % 32 || p.d_in % p.group || p.rank % 16 ||
+    if (p.d_out % 16 || p.d_in % 128 || (p.group != 64 && p.group % 128) || p.d_in % p.group ||
+        p.rank % 16 ||
         p.rank > 256)
       return TILEQ_ERR_UNSUPPORTED;
     if (!p.grid_assign) return TILEQ_ERR_INVALID_ARG;
@@ -81,7 +88,11 @@ tileq_status validate_layer(const tileq_layer *L, LayerInfo *li, bool need_devic
   return TILEQ_OK;
 }
 
-// ------------------------------------------------------------------ packed layout
+// ------------------------------------------------------------------ packed layouts
+size_t frag_bytes(int nblk, int R, int C, int kb) {
+  return (size_t)nblk * pad128(R) * (size_t)cdiv(C, 16 * kb) * 16 * kb * 2;
+}
+
 struct PackedLayout {
   size_t qw[3], sz[3], uf[3], vf[3], sh[3], total;
 };
@@ -92,17 +103,20 @@ PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
   for (int p = 0; p < li.nproj; ++p) {
     const ProjInfo &q = li.p[p];
     pl.qw[p] = off;
-    off += align_up((size_t)L->K * q.d_out * q.d_in / 4);
+    off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 4);
     pl.sz[p] = off;
-    off += align_up((size_t)L->K * q.d_out * q.G * 4);
+    off += align_up((size_t)L->K * pad128(q.d_out) * q.G * 4);
     pl.uf[p] = off;
-    off += align_up((size_t)L->M * q.d_out * q.rank * 2);
+    if (q.rank > 0) off += align_up((size_t)L->M * pad128(q.d_out) * q.rank * 2);
     pl.vf[p] = off;
-    off += align_up((size_t)L->N * q.d_in * q.rank * 2);
+    if (q.rank > 0) off += align_up(frag_bytes(L->N, q.rank, q.d_in, 8));
   }
   for (int i = 0; i < 3; ++i) {
     pl.sh[i] = off;
-    off += align_up((size_t)L->shared_d_ff * L->d_model * 2);
+    if (L->shared_d_ff > 0) {
+      const int R = i < 2 ? L->shared_d_ff : L->d_model, C = i < 2 ? L->d_model : L->shared_d_ff;
+      off += align_up(frag_bytes(1, R, C, 8));
+    }
   }
   pl.total = off;
   return pl;
@@ -118,49 +132,142 @@ PePackedLayout pe_layout(const tileq_layer *L, const LayerInfo &li) {
   for (int p = 0; p < li.nproj; ++p) {
     const ProjInfo &q = li.p[p];
     pl.uf[p] = off;
-    off += align_up((size_t)L->K * q.d_out * q.rank * 2);
+    if (q.rank > 0) off += align_up(frag_bytes(L->K, q.d_out, q.rank, 8));
     pl.vf[p] = off;
-    off += align_up((size_t)L->K * q.d_in * q.rank * 2);
+    if (q.rank > 0) off += align_up(frag_bytes(L->K, q.rank, q.d_in, 8));
   }
   pl.total = off;
   return pl;
 }
 
-// ------------------------------------------------------------------ workspace layout
-struct WsLayout {
-  int P, bn, ksplit, slots_main, slots_z;
-  size_t status, topk_idx, topk_w, expert_offsets, sorted_pairs, slot_of_pair, slot_tok, slot_w,
-      dest, tiles_main, tile_first, tile_counts;
-  size_t col_offsets[2], colpair_tok[2], zidx[2], tiles_z[2];
-  size_t row_offsets, rowpair_tok, rowpair_row, aidx;
-  size_t x16, xs, zc[2], zs, abuf, h, ybuf, hs, ys, g32, u32, zpe[2];
-  size_t total;
+// ------------------------------------------------------------------ launch plan
+struct GemmPlan {
+  int bn = 8, slots = 0, ksplit = 1, m_tiles = 1, np = 1, items = 0;
+  size_t part_floats() const {
+    return ksplit > 1 ? (size_t)ksplit * np * std::max(items, 1) * m_tiles * kRowsPerCta : 0;
+  }
+  int counters(int nprob) const { return ksplit > 1 ? nprob * slots * m_tiles : 0; }
 };
 
-int choose_bn(int P, int K) {
-  const int avg = P / std::max(1, K);
+int choose_bn(long long avg) {
   if (avg <= 8) return 8;
   if (avg <= 16) return 16;
   if (avg <= 32) return 32;
   return 64;
 }
 
+// Items per tile of the tensor-core GEMM (N of one tcgen05.mma: 16..128).
+int choose_bn_tc(long long avg) {
+  if (avg <= 16) return 16;
+  if (avg <= 32) return 32;
+  if (avg <= 64) return 64;
+  return 128;
+}
+
+// Split K until the grid covers about `per_sm` CTAs (or work items) per SM,
+// keeping >= 2 k-blocks per split.
+int choose_ksplit(long long ctas, int d_in, int per_sm = 4) {
+  const int nkb = cdiv(d_in, 128);
+  int ks = (int)std::max(1LL, ((long long)per_sm * kNumSMs + ctas - 1) / std::max(1LL, ctas));
+  ks = std::min(ks, std::max(1, nkb / 2));
+  return std::max(1, std::min(ks, 8));
+}
+
+struct Plan {
+  int T, k, P;
+  int bn_main, slots_main;
+  GemmPlan zproj, gateup, zdown, down, linear, sh_gu, sh_down, pe;
+};
+
+Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
+  Plan pl;
+  pl.T = T;
+  pl.k = k;
+  pl.P = T * k;
+  const int P = pl.P;
+  pl.bn_main = choose_bn_tc(P / std::max(1, L->K));
+  pl.slots_main = cdiv(P, pl.bn_main) + L->K;
+  const long long est_main = std::min(L->K, P) + P / pl.bn_main;
+  const int bn_z = choose_bn(P / std::max(1, L->N));
+  const int slots_z = cdiv(P, bn_z) + L->N;
+  const long long est_z = std::min(L->N, P) + P / bn_z;
+  // residual GEMMs on the tensor cores: persistent CTAs walk (tile, row block, split) items
+  auto tc_plan = [&](int d_out, int d_in, int np) {
+    GemmPlan g;
+    g.bn = pl.bn_main;
+    g.slots = pl.slots_main;
+    g.m_tiles = cdiv(d_out, 128);
+    g.np = np;
+    g.items = P;
+    g.ksplit = choose_ksplit(est_main * g.m_tiles, d_in, 2);
+    return g;
+  };
+  const ProjInfo &q0 = li.p[0];
+  if (L->kind == TILEQ_LINEAR) {
+    pl.linear = tc_plan(q0.d_out, q0.d_in, 1);
+  } else {
+    pl.gateup = tc_plan(L->d_ff, L->d_model, 2);
+    pl.down = tc_plan(L->d_model, L->d_ff, 1);
+    if (li.p[2].rank > 0) {
+      GemmPlan z;
+      z.bn = pl.bn_main;
+      z.slots = pl.slots_main;
+      z.m_tiles = cdiv(li.p[2].rank, 128);
+      z.items = P;
+      z.ksplit = choose_ksplit(est_main * z.m_tiles, L->d_ff);
+      pl.zdown = z;
+    }
+  }
+  if (q0.rank > 0) {
+    GemmPlan z;
+    z.bn = bn_z;
+    z.slots = slots_z;
+    z.m_tiles = cdiv(q0.rank, 128);
+    z.items = P;
+    z.ksplit = choose_ksplit(est_z * z.m_tiles * (L->kind == TILEQ_SWIGLU ? 2 : 1), q0.d_in);
+    pl.zproj = z;
+  }
+  if (L->shared_d_ff > 0) {
+    const int bn = choose_bn(T);
+    GemmPlan g;
+    g.bn = bn;
+    g.slots = cdiv(T, bn);
+    g.items = T;
+    g.np = 2;
+    g.m_tiles = cdiv(L->shared_d_ff, 128);
+    g.ksplit = choose_ksplit((long long)g.slots * g.m_tiles, L->d_model);
+    pl.sh_gu = g;
+    g.np = 1;
+    g.m_tiles = cdiv(L->d_model, 128);
+    g.ksplit = choose_ksplit((long long)g.slots * g.m_tiles, L->shared_d_ff);
+    pl.sh_down = g;
+  }
+  // unfused per-expert launches: one expert per launch, grid sized for T slots, no split
+  pl.pe.bn = pl.bn_main;
+  pl.pe.slots = cdiv(T, pl.bn_main);
+  pl.pe.items = P;
+  return pl;
+}
+
+// ------------------------------------------------------------------ workspace layout
+struct WsLayout {
+  Plan plan;
+  size_t status, topk_idx, topk_w, expert_offsets, sorted_pairs, slot_of_pair, slot_tok, slot_w,
+      dest, tiles_main, tile_first, tile_counts, counters, part;
+  int n_counters;
+  size_t part_zstride;
+  size_t col_offsets[2], colpair_tok[2], zidx[2], tiles_z[2];
+  size_t row_offsets, rowpair_tok, rowpair_row, aidx;
+  size_t x16, xext, hext, zc[2], zs, ybuf, hs, ys, g32, u32, zpe[2];
+  int ld_x, ld_h;
+  size_t total;
+};
+
 WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   WsLayout w{};
-  const int P = T * k;
-  w.P = P;
-  w.bn = choose_bn(P, L->K);
-  w.slots_main = cdiv(P, w.bn) + L->K;
-  w.slots_z = cdiv(P, w.bn) + L->N;
-  {
-    // split K of the last (combined) GEMM until the grid covers ~2 waves of 148 SMs
-    const ProjInfo &q = li.p[li.nproj - 1];
-    const long long ctas = (long long)(std::min(L->K, P) + P / w.bn) * cdiv(q.d_out, 64);
-    const int nkb = q.d_in / 128;
-    int ks = (int)std::max(1LL, (2LL * 148 + ctas - 1) / std::max(1LL, ctas));
-    ks = std::min(ks, std::max(1, nkb / 4));
-    w.ksplit = std::max(1, std::min(ks, 8));
-  }
+  w.plan = make_plan(L, li, T, k);
+  const Plan &pl = w.plan;
+  const int P = pl.P;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -177,14 +284,29 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   w.slot_tok = take(Pz * 4);
   w.slot_w = take(Pz * 4);
   w.dest = take(Pz * 4);
-  w.tiles_main = take((size_t)w.slots_main * 16);
+  w.tiles_main = take((size_t)(pl.slots_main + 1) * 16);
   w.tile_first = take((L->K + 1) * 4);
   w.tile_counts = take(16);
+  int nc = 0;
+  nc = std::max(nc, pl.zproj.counters(2));
+  nc = std::max(nc, pl.gateup.counters(1));
+  nc = std::max(nc, pl.zdown.counters(1));
+  nc = std::max(nc, pl.down.counters(1));
+  nc = std::max(nc, pl.linear.counters(1));
+  nc = std::max(nc, pl.sh_gu.counters(1));
+  nc = std::max(nc, pl.sh_down.counters(1));
+  w.n_counters = nc;
+  w.counters = take((size_t)nc * 4);
+  size_t pf = 2 * pl.zproj.part_floats();
+  w.part_zstride = pl.zproj.part_floats();
+  for (const GemmPlan *g : {&pl.gateup, &pl.zdown, &pl.down, &pl.linear, &pl.sh_gu, &pl.sh_down})
+    pf = std::max(pf, g->part_floats());
+  w.part = take(pf * 4);
   for (int z = 0; z < 2; ++z) {
     w.col_offsets[z] = take((L->N + 1) * 4);
     w.colpair_tok[z] = take(Pz * 4);
     w.zidx[z] = take(Pz * 4);
-    w.tiles_z[z] = take((size_t)w.slots_z * 16);
+    w.tiles_z[z] = take((size_t)(pl.zproj.slots + 1) * 16);
   }
   w.row_offsets = take((L->M + 1) * 4);
   w.rowpair_tok = take(Pz * 4);
@@ -194,21 +316,23 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   const int rmax = std::max(std::max(li.p[0].rank, li.nproj > 1 ? li.p[1].rank : 0),
                             li.p[li.nproj - 1].rank);
   if (L->kind == TILEQ_LINEAR) {
-    w.xs = take(Pz * li.d_x * 2);
+    w.ld_x = li.d_x + li.p[0].rank;
+    w.xext = take(Pz * w.ld_x * 2);
     w.zc[0] = take(Pz * li.p[0].rank * 2);
-    w.abuf = take(Pz * li.p[0].rank * 2);
   } else {
+    w.ld_x = L->d_model + 2 * li.p[0].rank;
+    w.ld_h = L->d_ff + li.p[2].rank;
+    w.xext = take(Pz * w.ld_x * 2);
+    w.hext = take(Pz * w.ld_h * 2);
     w.zc[0] = take(Pz * li.p[0].rank * 2);
     w.zc[1] = take(Pz * li.p[1].rank * 2);
     w.zs = take(Pz * li.p[2].rank * 4);
-    w.abuf = take(Pz * li.p[2].rank * 2);
-    w.h = take(Pz * L->d_ff * 2);
     w.g32 = take(Pz * L->d_ff * 4);
     w.u32 = take(Pz * L->d_ff * 4);
   }
-  w.zpe[0] = take(Pz * rmax * 2);
-  w.zpe[1] = take(Pz * rmax * 2);
-  w.ybuf = take((size_t)w.ksplit * Pz * li.d_y * 4);
+  w.zpe[0] = take(Pz * std::max(rmax, 16) * 2);
+  w.zpe[1] = take(Pz * std::max(rmax, 16) * 2);
+  w.ybuf = take(Pz * li.d_y * 4);
   if (L->shared_d_ff > 0) {
     w.hs = take((size_t)std::max(T, 1) * L->shared_d_ff * 2);
     w.ys = take((size_t)std::max(T, 1) * L->d_model * 4);
@@ -226,22 +350,14 @@ const Tp *at(const void *base, size_t off) {
   return reinterpret_cast<const Tp *>(static_cast<const char *>(base) + off);
 }
 
-GemmProblem problem() {
-  GemmProblem g;
-  std::memset(&g, 0, sizeof(g));
-  g.only_group = -1;
-  g.ksplit = 1;
-  return g;
-}
-
-#define TQ_CUDA(call)                                       \
-  do {                                                      \
-    if ((call) != cudaSuccess) return TILEQ_ERR_CUDA;       \
+#define TQ_CUDA(call)                                 \
+  do {                                                \
+    if ((call) != cudaSuccess) return TILEQ_ERR_CUDA; \
   } while (0)
 
-#define TQ_LAUNCHED()                                       \
-  do {                                                      \
-    count_launches();                                       \
+#define TQ_LAUNCHED()                                             \
+  do {                                                            \
+    count_launches();                                             \
     if (cudaGetLastError() != cudaSuccess) return TILEQ_ERR_CUDA; \
   } while (0)
 
@@ -257,23 +373,82 @@ void mark(int stage, cudaStream_t stream) {
   if (stage < g_n_stage_events) cudaEventRecord(g_stage_events[stage], stream);
 }
 
-unsigned nblocks(long long n, int per) { return (unsigned)((n + per - 1) / per); }
+// A GEMM problem with the plan's tiling and the workspace's split-K scratch.
+GemmProblem problem(const GemmPlan &g, void *ws, const WsLayout &w) {
+  GemmProblem p;
+  std::memset(&p, 0, sizeof(p));
+  p.only_group = -1;
+  p.ksplit = g.ksplit;
+  p.m_tiles = g.m_tiles;
+  p.part = at<float>(ws, w.part);
+  p.part_items = std::max(g.items, 1);
+  p.counters = at<int>(ws, w.counters);
+  p.status = at<int>(ws, w.status);
+  return p;
+}
 
-// Residual projection problem for the Q2 GEMM: A = packed codes of projection p.
-GemmProblem residual_problem(const tileq_layer *L, const LayerInfo &li, const PackedLayout &pl,
-                             const void *packed, int p) {
+tileq_status gemm(const GemmBatch &b, int nprob, int am, int np, const GemmPlan &g, cudaStream_t s) {
+  if (launch_gemm(b, nprob, GemmShape{am, np, g.bn}, g.slots, s) != cudaSuccess)
+    return TILEQ_ERR_CUDA;
+  return TILEQ_OK;
+}
+
+// 2-D tensor map over an fp16 matrix [rows][ld] (ld >= cols), box 64 x box_rows,
+// 128-byte swizzle, zero fill outside the matrix.
+bool make_map(CUtensorMap *m, const void *base, int rows, int cols, int ld, int box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)std::max(rows, 1)};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor-core residual GEMM of projection p over the main tile table.
+tileq_status tc_args(TcArgs *a, const GemmPlan &g, const LayerInfo &li, const PackedLayout &pl,
+                     const void *packed, int p, void *ws, const WsLayout &w, const void *bmat, int bld,
+                     int bcols) {
   const ProjInfo &q = li.p[p];
-  GemmProblem g = problem();
-  g.d_out = q.d_out;
-  g.d_in = q.d_in;
-  g.group_size = q.group;
-  g.a[0] = at<uint4>(packed, pl.qw[p]);
-  g.sz[0] = at<uint32_t>(packed, pl.sz[p]);
-  g.a_stride = (long long)(q.d_out / 16) * (q.d_in / 128) * 32;
-  g.sz_stride = (long long)(q.d_out / 16) * q.G * 16;
-  g.m_tiles = cdiv(q.d_out, 64);
-  (void)L;
-  return g;
+  std::memset(a, 0, sizeof(*a));
+  if (!make_map(&a->bmap, bmat, w.plan.P, bcols, bld, g.bn)) return TILEQ_ERR_CUDA;
+  a->tiles = at<int4>(ws, w.tiles_main);
+  a->tile_count = at<int>(ws, w.tile_counts);
+  a->m_tiles = g.m_tiles;
+  a->ksplit = g.ksplit;
+  a->d_out = q.d_out;
+  a->d_in = q.d_in;
+  a->group = q.group;
+  a->codes[0] = at<uint4>(packed, pl.qw[p]);
+  a->sz[0] = at<uint32_t>(packed, pl.sz[p]);
+  a->part = at<float>(ws, w.part);
+  a->part_items = std::max(g.items, 1);
+  a->counters = at<int>(ws, w.counters);
+  a->status = at<int>(ws, w.status);
+  return TILEQ_OK;
+}
+
+// Low-rank K extension of projection slot `slot` (0/1) of a tensor-core GEMM.
+void tc_ext(TcArgs *a, int slot, const LayerInfo &li, const PackedLayout &pl, const void *packed, int p,
+            int col) {
+  const ProjInfo &q = li.p[p];
+  a->rank = q.rank;
+  a->ext_col[slot] = col;
+  a->u[slot] = at<__half>(packed, pl.uf[p]);
+  std::memcpy(a->u_blk[slot], q.m_of, kMaxExperts);
+}
+
+tileq_status tc_launch(const TcArgs &a, int np, const GemmPlan &g, cudaStream_t stream) {
+  return launch_gemm_tc(a, np, g.bn, kNumSMs, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
 }
 
 tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const WsLayout &w,
@@ -290,6 +465,8 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   ra.k = top_k;
   ra.topk_idx = at<int32_t>(ws, w.topk_idx);
   ra.topk_w = at<float>(ws, w.topk_w);
+  ra.zero = at<int>(ws, w.counters);
+  ra.nzero = w.n_counters;
   mark(ST_BEGIN, stream);
   route_kernel<<<nblocks(T, 8), 256, 0, stream>>>(ra);
   TQ_LAUNCHED();
@@ -302,7 +479,8 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   pa.K = L->K;
   pa.M = L->M;
   pa.N = L->N;
-  pa.bn = w.bn;
+  pa.bn = w.plan.bn_main;
+  pa.bn_z = w.plan.zproj.bn;
   pa.topk_idx = ra.topk_idx;
   pa.topk_w = ra.topk_w;
   pa.dest = at<int>(ws, w.dest);
@@ -359,9 +537,8 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
   const float *yshared = nullptr;
   if (L->shared_d_ff > 0) {
     const int Fs = L->shared_d_ff, D = L->d_model;
-    const int bn = T <= 8 ? 8 : T <= 16 ? 16 : T <= 32 ? 32 : 64;
     GemmBatch b;
-    b.p[0] = problem();
+    b.p[0] = problem(w.plan.sh_gu, ws, w);
     GemmProblem &g = b.p[0];
     g.static_items = T;
     g.d_out = Fs;
@@ -373,11 +550,9 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
     g.epi = EPI_SWIGLU_H;
     g.out[0] = at<__half>(ws, w.hs);
     g.ldo = Fs;
-    g.m_tiles = cdiv(Fs, 64);
-    if (launch_gemm(b, 1, GemmShape{AM_F16, 2, bn, 4}, cdiv(T, bn), stream) != cudaSuccess)
-      return TILEQ_ERR_CUDA;
+    if (gemm(b, 1, AM_F16, 2, w.plan.sh_gu, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
+    b.p[0] = problem(w.plan.sh_down, ws, w);
     GemmProblem &d = b.p[0];
-    d = problem();
     d.static_items = T;
     d.d_out = D;
     d.d_in = Fs;
@@ -387,9 +562,7 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
     d.epi = EPI_STORE_F32;
     d.out[0] = at<float>(ws, w.ys);
     d.ldo = D;
-    d.m_tiles = cdiv(D, 64);
-    if (launch_gemm(b, 1, GemmShape{AM_F16, 1, bn, 4}, cdiv(T, bn), stream) != cudaSuccess)
-      return TILEQ_ERR_CUDA;
+    if (gemm(b, 1, AM_F16, 1, w.plan.sh_down, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
     yshared = at<float>(ws, w.ys);
   }
   mark(ST_SHARED, stream);
@@ -397,8 +570,8 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
   ca.T = T;
   ca.k = top_k;
   ca.d = li.d_y;
-  ca.ksplit = w.ksplit;
-  ca.split_stride = (long long)w.P * li.d_y;
+  ca.ksplit = 1;
+  ca.split_stride = 0;
   ca.slot_of_pair = at<int>(ws, w.slot_of_pair);
   ca.ybuf = at<float>(ws, w.ybuf);
   ca.yshared = yshared;
@@ -417,10 +590,56 @@ tileq_status check_forward_args(const tileq_layer *layer, LayerInfo *li, const v
   if (T < 0 || top_k < 1 || top_k > layer->K || top_k > kMaxTopK) return TILEQ_ERR_INVALID_ARG;
   if (T == 0) return TILEQ_OK;
   if (!packed || !x || !logits || !out || !ws) return TILEQ_ERR_INVALID_ARG;
-  if ((long long)T * top_k > (1LL << 28)) return TILEQ_ERR_UNSUPPORTED;
+  if ((long long)T * top_k > (1LL << 24)) return TILEQ_ERR_UNSUPPORTED;
   const WsLayout w = ws_layout(layer, *li, T, top_k);
   if (ws_bytes < w.total) return TILEQ_ERR_WORKSPACE;
   return TILEQ_OK;
+}
+
+LrAccArgs lracc_args(const ProjInfo &q, const WsLayout &w, void *ws, int top_k, __half *out, int ld,
+                     int col) {
+  LrAccArgs la;
+  std::memset(&la, 0, sizeof(la));
+  la.P = w.plan.P;
+  la.k = top_k;
+  la.r = q.rank;
+  la.sorted_pairs = at<int32_t>(ws, w.sorted_pairs);
+  la.aidx = at<int>(ws, w.aidx);
+  la.topk_idx = at<int32_t>(ws, w.topk_idx);
+  la.topk_w = at<float>(ws, w.topk_w);
+  std::memcpy(la.m_of, q.m_of, kMaxExperts);
+  la.slot_of_pair = at<int>(ws, w.slot_of_pair);
+  la.out = out;
+  la.ld = ld;
+  la.col = col;
+  return la;
+}
+
+// z_{t,n} = Sigma * (V_n^T x_t) once per distinct (token, grid column): one
+// grouped GEMM per projection (gate and up share a launch).
+tileq_status run_zproj(const tileq_layer *layer, const LayerInfo &li, const PackedLayout &pl,
+                       const void *packed, const WsLayout &w, void *ws, int nz,
+                       cudaStream_t stream) {
+  GemmBatch b;
+  for (int p = 0; p < nz; ++p) {
+    const ProjInfo &q = li.p[p];
+    b.p[p] = problem(w.plan.zproj, ws, w);
+    GemmProblem &z = b.p[p];
+    z.tiles = at<int4>(ws, w.tiles_z[p]);
+    z.tile_count = at<int>(ws, w.tile_counts) + 1 + p;
+    z.d_out = q.rank;
+    z.d_in = q.d_in;
+    z.a[0] = at<uint4>(packed, pl.vf[p]);
+    z.b = at<__half>(ws, w.x16);
+    z.ldb = q.d_in;
+    z.b_row = at<int>(ws, w.colpair_tok[p]);
+    z.epi = EPI_STORE_F16;
+    z.col_scale = layer->proj[p].Sigma;
+    z.out[0] = at<__half>(ws, w.zc[p]);
+    z.ldo = q.rank;
+    z.part = at<float>(ws, w.part) + (size_t)p * w.part_zstride;
+  }
+  return gemm(b, nz, AM_F16, 1, w.plan.zproj, stream);
 }
 
 }  // namespace
@@ -462,13 +681,13 @@ tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_by
     const tileq_proj &src = layer->proj[p];
     const ProjInfo &q = li.p[p];
     {
-      const long long n = (long long)K * (q.d_out / 16) * (q.d_in / 128) * 32;
-      pack_codes_kernel<<<nblocks(n, 256), 256, 0, stream>>>(src.codes, at<uint4>(packed, pl.qw[p]),
-                                                              K, q.d_out, q.d_in);
+      const long long n = (long long)K * (pad128(q.d_out) / 128) * (q.d_in / 128) * 128 * 8;
+      pack_codes_tc_kernel<<<nblocks(n, 256), 256, 0, stream>>>(src.codes, at<uint32_t>(packed, pl.qw[p]),
+                                                                 K, q.d_out, q.d_in);
       TQ_LAUNCHED();
     }
     {
-      const long long n = (long long)K * q.d_out * q.G;
+      const long long n = (long long)K * pad128(q.d_out) * q.G;
       pack_sz_kernel<<<nblocks(n, 256), 256, 0, stream>>>(static_cast<const __half *>(src.scales),
                                                            src.zeros, at<uint32_t>(packed, pl.sz[p]),
                                                            K, q.d_out, q.G);
@@ -477,16 +696,15 @@ tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_by
     if (q.rank > 0) {
       const __nv_bfloat16 *U = static_cast<const __nv_bfloat16 *>(src.U);
       const __nv_bfloat16 *V = static_cast<const __nv_bfloat16 *>(src.V);
-      // U block m: rows o (d_out), cols i (rank): element at U[(m*d_out + o)*rank + i]
-      long long n = (long long)layer->M * (q.d_out / 16) * (q.rank / 16) * 32;
-      pack_frag_kernel<<<nblocks(n, 256), 256, 0, stream>>>(U, (long long)q.d_out * q.rank, q.rank, 1,
-                                                             layer->M, q.d_out, q.rank,
-                                                             at<uint4>(packed, pl.uf[p]));
+      // U block m: fp16 rows (padded to 128), the K extension of the residual GEMM
+      long long n = (long long)layer->M * pad128(q.d_out) * q.rank;
+      pack_rows_f16_kernel<<<nblocks(n, 256), 256, 0, stream>>>(U, layer->M, q.d_out, q.rank,
+                                                                 at<__half>(packed, pl.uf[p]));
       TQ_LAUNCHED();
       // V_n^T: rows i (rank), cols k (d_in): element at V[(n*d_in + k)*rank + i]
-      n = (long long)layer->N * (q.rank / 16) * (q.d_in / 16) * 32;
+      n = (long long)frag_bytes(layer->N, q.rank, q.d_in, 8) / 16;
       pack_frag_kernel<<<nblocks(n, 256), 256, 0, stream>>>(V, (long long)q.d_in * q.rank, 1, q.rank,
-                                                             layer->N, q.rank, q.d_in,
+                                                             layer->N, q.rank, q.d_in, 8,
                                                              at<uint4>(packed, pl.vf[p]));
       TQ_LAUNCHED();
     }
@@ -495,9 +713,9 @@ tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_by
     const int Fs = layer->shared_d_ff, D = layer->d_model;
     for (int i = 0; i < 3; ++i) {
       const int R = i < 2 ? Fs : D, Cc = i < 2 ? D : Fs;
-      const long long n = (long long)(R / 16) * (Cc / 16) * 32;
+      const long long n = (long long)frag_bytes(1, R, Cc, 8) / 16;
       pack_frag_kernel<<<nblocks(n, 256), 256, 0, stream>>>(
-          static_cast<const __nv_bfloat16 *>(layer->shared_w[i]), 0, Cc, 1, 1, R, Cc,
+          static_cast<const __nv_bfloat16 *>(layer->shared_w[i]), 0, Cc, 1, 1, R, Cc, 8,
           at<uint4>(packed, pl.sh[i]));
       TQ_LAUNCHED();
     }
@@ -524,7 +742,8 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
   if (st != TILEQ_OK || T == 0) return st;
   const PackedLayout pl = packed_layout(layer, li);
   const WsLayout w = ws_layout(layer, li, T, top_k);
-  const int K = layer->K;
+  const Plan &plan = w.plan;
+  __half *xext = at<__half>(ws, w.xext);
 
   if (layer->kind == TILEQ_LINEAR) {
     const ProjInfo &q = li.p[0];
@@ -532,49 +751,21 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     st = run_route_permute(layer, li, w, x, T, router_logits, top_k, ws, q.rank > 0 ? 1 : 0, zids,
                            q.rank > 0 ? 0 : -1, stream);
     if (st != TILEQ_OK) return st;
-    ScaleGatherArgs sg{w.P, q.d_in, at<int>(ws, w.slot_tok), at<float>(ws, w.slot_w),
-                       at<__half>(ws, w.x16), at<__half>(ws, w.xs)};
-    scale_gather_kernel<<<nblocks((long long)w.P * (q.d_in / 2), 256), 256, 0, stream>>>(sg);
+    // x' = w * x per slot in the first d_in columns of the activation matrix
+    ScaleGatherArgs sg{plan.P, q.d_in, w.ld_x, at<int>(ws, w.slot_tok), at<float>(ws, w.slot_w),
+                       at<__half>(ws, w.x16), xext};
+    scale_gather_kernel<<<nblocks((long long)plan.P * (q.d_in / 2), 256), 256, 0, stream>>>(sg);
     TQ_LAUNCHED();
     if (q.rank > 0) {
-      GemmBatch b;
-      b.p[0] = problem();
-      GemmProblem &z = b.p[0];
-      z.tiles = at<int4>(ws, w.tiles_z[0]);
-      z.tile_count = at<int>(ws, w.tile_counts) + 1;
-      z.d_out = q.rank;
-      z.d_in = q.d_in;
-      z.a[0] = at<uint4>(packed, pl.vf[0]);
-      z.a_stride = (long long)(q.rank / 16) * (q.d_in / 16) * 32;
-      z.b = at<__half>(ws, w.x16);
-      z.ldb = q.d_in;
-      z.b_row = at<int>(ws, w.colpair_tok[0]);
-      z.epi = EPI_STORE_F16;
-      z.col_scale = layer->proj[0].Sigma;
-      z.out[0] = at<__half>(ws, w.zc[0]);
-      z.ldo = q.rank;
-      z.m_tiles = cdiv(q.rank, 64);
-      if (launch_gemm(b, 1, GemmShape{AM_F16, 1, w.bn, 4}, w.slots_z, stream) != cudaSuccess)
-        return TILEQ_ERR_CUDA;
+      if ((st = run_zproj(layer, li, pl, packed, w, ws, 1, stream)) != TILEQ_OK) return st;
       mark(ST_ZPROJ, stream);
       mark(ST_GATEUP, stream);
       mark(ST_ZDOWN, stream);
-      LrAccArgs la;
-      std::memset(&la, 0, sizeof(la));
-      la.k = top_k;
-      la.r = q.rank;
-      la.row_offsets = at<int>(ws, w.row_offsets);
-      la.M = layer->M;
-      la.rowpair_tok = at<int>(ws, w.rowpair_tok);
-      la.rowpair_row = at<int>(ws, w.rowpair_row);
-      la.topk_idx = at<int32_t>(ws, w.topk_idx);
-      la.topk_w = at<float>(ws, w.topk_w);
-      std::memcpy(la.m_of, q.m_of, kMaxExperts);
-      la.slot_of_pair = at<int>(ws, w.slot_of_pair);
+      // a_{t,m} = sum_j w_j z_{t,n_j} over the token's experts in grid row m -> columns d_in..
+      LrAccArgs la = lracc_args(q, w, ws, top_k, xext, w.ld_x, q.d_in);
       la.zcol = at<__half>(ws, w.zc[0]);
       la.zidx = at<int>(ws, w.zidx[0]);
-      la.a = at<__half>(ws, w.abuf);
-      lr_accumulate_kernel<<<nblocks((long long)w.P * q.rank, 256), 256, 0, stream>>>(la);
+      lr_accumulate_kernel<<<nblocks((long long)plan.P * q.rank, 256), 256, 0, stream>>>(la);
       TQ_LAUNCHED();
     } else {
       mark(ST_ZPROJ, stream);
@@ -582,29 +773,14 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       mark(ST_ZDOWN, stream);
     }
     mark(ST_ROWACC, stream);
-    GemmBatch b;
-    b.p[0] = residual_problem(layer, li, pl, packed, 0);
-    GemmProblem &g = b.p[0];
-    g.tiles = at<int4>(ws, w.tiles_main);
-    g.tile_count = at<int>(ws, w.tile_counts);
-    g.b = at<__half>(ws, w.xs);
-    g.ldb = q.d_in;
-    g.rank = q.rank;
-    if (q.rank > 0) {
-      g.u[0] = at<uint4>(packed, pl.uf[0]);
-      g.u_stride = (long long)(q.d_out / 16) * (q.rank / 16) * 32;
-      std::memcpy(g.u_blk[0], q.m_of, kMaxExperts);
-      g.zb[0] = at<__half>(ws, w.abuf);
-      g.ldz = q.rank;
-      g.z_row[0] = at<int>(ws, w.aidx);
-    }
-    g.epi = EPI_STORE_F32;
-    g.out[0] = at<float>(ws, w.ybuf);
-    g.ldo = q.d_out;
-    g.out_split_stride = (long long)w.P * q.d_out;
-    g.ksplit = w.ksplit;
-    if (launch_gemm(b, 1, GemmShape{AM_Q2, 1, w.bn, 4}, w.slots_main, stream) != cudaSuccess)
-      return TILEQ_ERR_CUDA;
+    TcArgs a;
+    if ((st = tc_args(&a, plan.linear, li, pl, packed, 0, ws, w, xext, w.ld_x, w.ld_x)) != TILEQ_OK)
+      return st;
+    if (q.rank > 0) tc_ext(&a, 0, li, pl, packed, 0, q.d_in);
+    a.epi = EPI_STORE_F32;
+    a.out[0] = at<float>(ws, w.ybuf);
+    a.ldo = q.d_out;
+    if ((st = tc_launch(a, 1, plan.linear, stream)) != TILEQ_OK) return st;
     mark(ST_RESIDUAL, stream);
   } else {
     const ProjInfo &qg = li.p[0], &qd = li.p[2];
@@ -614,135 +790,86 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
                            lr_d ? 2 : -1, stream);
     if (st != TILEQ_OK) return st;
     const int D = layer->d_model, F = layer->d_ff;
-    if (lr_gu) {
-      // z_{t,n} = Sigma * (V_n^T x_t) once per distinct (token, grid column), gate and up
-      GemmBatch b;
-      for (int p = 0; p < 2; ++p) {
-        const ProjInfo &q = li.p[p];
-        b.p[p] = problem();
-        GemmProblem &z = b.p[p];
-        z.tiles = at<int4>(ws, w.tiles_z[p]);
-        z.tile_count = at<int>(ws, w.tile_counts) + 1 + p;
-        z.d_out = q.rank;
-        z.d_in = D;
-        z.a[0] = at<uint4>(packed, pl.vf[p]);
-        z.a_stride = (long long)(q.rank / 16) * (D / 16) * 32;
-        z.b = at<__half>(ws, w.x16);
-        z.ldb = D;
-        z.b_row = at<int>(ws, w.colpair_tok[p]);
-        z.epi = EPI_STORE_F16;
-        z.col_scale = layer->proj[p].Sigma;
-        z.out[0] = at<__half>(ws, w.zc[p]);
-        z.ldo = q.rank;
-        z.m_tiles = cdiv(q.rank, 64);
-      }
-      if (launch_gemm(b, 2, GemmShape{AM_F16, 1, w.bn, 4}, w.slots_z, stream) != cudaSuccess)
-        return TILEQ_ERR_CUDA;
+    __half *hext = at<__half>(ws, w.hext);
+    if (lr_gu && (st = run_zproj(layer, li, pl, packed, w, ws, 2, stream)) != TILEQ_OK) return st;
+    {
+      // activation matrix of gate/up: [x_t | z^gate_{t,n} | z^up_{t,n}] per slot
+      GatherExtArgs ga;
+      ga.P = plan.P;
+      ga.d = D;
+      ga.r = qg.rank;
+      ga.ld = w.ld_x;
+      ga.slot_tok = at<int>(ws, w.slot_tok);
+      ga.x16 = at<__half>(ws, w.x16);
+      ga.z[0] = lr_gu ? at<__half>(ws, w.zc[0]) : nullptr;
+      ga.z[1] = lr_gu ? at<__half>(ws, w.zc[1]) : nullptr;
+      ga.zidx[0] = at<int>(ws, w.zidx[0]);
+      ga.zidx[1] = at<int>(ws, w.zidx[1]);
+      ga.out = xext;
+      const long long chunks = (long long)plan.P * (D / 8 + (lr_gu ? 2 * qg.rank / 8 : 0));
+      gather_ext_kernel<<<nblocks(chunks, 256), 256, 0, stream>>>(ga);
+      TQ_LAUNCHED();
     }
     mark(ST_ZPROJ, stream);
     {
-      // gate/up residual + U_m z (K extension) + SwiGLU, h = w * silu(g) * u per slot
-      GemmBatch b;
-      b.p[0] = residual_problem(layer, li, pl, packed, 0);
-      GemmProblem &g = b.p[0];
-      g.a[1] = at<uint4>(packed, pl.qw[1]);
-      g.sz[1] = at<uint32_t>(packed, pl.sz[1]);
-      g.tiles = at<int4>(ws, w.tiles_main);
-      g.tile_count = at<int>(ws, w.tile_counts);
-      g.b = at<__half>(ws, w.x16);
-      g.ldb = D;
-      g.b_row = at<int>(ws, w.slot_tok);
-      g.rank = qg.rank;
+      // gate/up residual + U_m z (K extension) + SwiGLU; h = w * silu(g) * u per slot
+      TcArgs a;
+      if ((st = tc_args(&a, plan.gateup, li, pl, packed, 0, ws, w, xext, w.ld_x, w.ld_x)) != TILEQ_OK)
+        return st;
+      a.codes[1] = at<uint4>(packed, pl.qw[1]);
+      a.sz[1] = at<uint32_t>(packed, pl.sz[1]);
       if (lr_gu) {
-        for (int p = 0; p < 2; ++p) {
-          g.u[p] = at<uint4>(packed, pl.uf[p]);
-          std::memcpy(g.u_blk[p], li.p[p].m_of, kMaxExperts);
-          g.zb[p] = at<__half>(ws, w.zc[p]);
-          g.z_row[p] = at<int>(ws, w.zidx[p]);
-        }
-        g.u_stride = (long long)(F / 16) * (qg.rank / 16) * 32;
-        g.ldz = qg.rank;
+        tc_ext(&a, 0, li, pl, packed, 0, D);
+        tc_ext(&a, 1, li, pl, packed, 1, D + qg.rank);
       }
-      g.epi = EPI_SWIGLU_H;
-      g.out[0] = at<__half>(ws, w.h);
-      g.ldo = F;
-      g.row_scale = at<float>(ws, w.slot_w);
-      if (launch_gemm(b, 1, GemmShape{AM_Q2, 2, w.bn, 4}, w.slots_main, stream) != cudaSuccess)
-        return TILEQ_ERR_CUDA;
+      a.epi = EPI_SWIGLU_H;
+      a.out[0] = hext;
+      a.ldo = w.ld_h;
+      a.row_scale = at<float>(ws, w.slot_w);
+      if ((st = tc_launch(a, 2, plan.gateup, stream)) != TILEQ_OK) return st;
     }
     mark(ST_GATEUP, stream);
     if (lr_d) {
-      // z'_slot = Sigma * (V_n^T h_slot) for the down projection, then the in-place
-      // accumulation a_{t,m} = sum of the token's z' over its experts in grid row m
+      // z'_slot = Sigma * (V_n^T h_slot), then the in-place accumulation
+      // a_{t,m} = sum of the token's z' over its experts in grid row m -> columns F..
       GemmBatch b;
-      b.p[0] = problem();
+      b.p[0] = problem(plan.zdown, ws, w);
       GemmProblem &z = b.p[0];
       z.tiles = at<int4>(ws, w.tiles_main);
       z.tile_count = at<int>(ws, w.tile_counts);
       z.d_out = qd.rank;
       z.d_in = F;
       z.a[0] = at<uint4>(packed, pl.vf[2]);
-      z.a_stride = (long long)(qd.rank / 16) * (F / 16) * 32;
       z.use_a_blk = 1;
       std::memcpy(z.a_blk, qd.n_of, kMaxExperts);
-      z.b = at<__half>(ws, w.h);
-      z.ldb = F;
+      z.b = hext;
+      z.ldb = w.ld_h;
       z.epi = EPI_STORE_F32;
       z.col_scale = layer->proj[2].Sigma;
       z.out[0] = at<float>(ws, w.zs);
       z.ldo = qd.rank;
-      z.m_tiles = cdiv(qd.rank, 64);
-      if (launch_gemm(b, 1, GemmShape{AM_F16, 1, w.bn, 4}, w.slots_main, stream) != cudaSuccess)
-        return TILEQ_ERR_CUDA;
+      if ((st = gemm(b, 1, AM_F16, 1, plan.zdown, stream)) != TILEQ_OK) return st;
       mark(ST_ZDOWN, stream);
-      LrAccArgs la;
-      std::memset(&la, 0, sizeof(la));
-      la.k = top_k;
-      la.r = qd.rank;
-      la.row_offsets = at<int>(ws, w.row_offsets);
-      la.M = layer->M;
-      la.rowpair_tok = at<int>(ws, w.rowpair_tok);
-      la.rowpair_row = at<int>(ws, w.rowpair_row);
-      la.topk_idx = at<int32_t>(ws, w.topk_idx);
-      la.topk_w = at<float>(ws, w.topk_w);
-      std::memcpy(la.m_of, qd.m_of, kMaxExperts);
-      la.slot_of_pair = at<int>(ws, w.slot_of_pair);
+      LrAccArgs la = lracc_args(qd, w, ws, top_k, hext, w.ld_h, F);
       la.zslot = at<float>(ws, w.zs);
-      la.a = at<__half>(ws, w.abuf);
-      lr_accumulate_kernel<<<nblocks((long long)w.P * qd.rank, 256), 256, 0, stream>>>(la);
+      lr_accumulate_kernel<<<nblocks((long long)plan.P * qd.rank, 256), 256, 0, stream>>>(la);
       TQ_LAUNCHED();
     } else {
       mark(ST_ZDOWN, stream);
     }
     mark(ST_ROWACC, stream);
     {
-      GemmBatch b;
-      b.p[0] = residual_problem(layer, li, pl, packed, 2);
-      GemmProblem &g = b.p[0];
-      g.tiles = at<int4>(ws, w.tiles_main);
-      g.tile_count = at<int>(ws, w.tile_counts);
-      g.b = at<__half>(ws, w.h);
-      g.ldb = F;
-      g.rank = qd.rank;
-      if (lr_d) {
-        g.u[0] = at<uint4>(packed, pl.uf[2]);
-        g.u_stride = (long long)(D / 16) * (qd.rank / 16) * 32;
-        std::memcpy(g.u_blk[0], qd.m_of, kMaxExperts);
-        g.zb[0] = at<__half>(ws, w.abuf);
-        g.ldz = qd.rank;
-        g.z_row[0] = at<int>(ws, w.aidx);
-      }
-      g.epi = EPI_STORE_F32;
-      g.out[0] = at<float>(ws, w.ybuf);
-      g.ldo = D;
-      g.out_split_stride = (long long)w.P * D;
-      g.ksplit = w.ksplit;
-      if (launch_gemm(b, 1, GemmShape{AM_Q2, 1, w.bn, 4}, w.slots_main, stream) != cudaSuccess)
-        return TILEQ_ERR_CUDA;
+      TcArgs a;
+      if ((st = tc_args(&a, plan.down, li, pl, packed, 2, ws, w, hext, w.ld_h, w.ld_h)) != TILEQ_OK)
+        return st;
+      if (lr_d) tc_ext(&a, 0, li, pl, packed, 2, F);
+      a.epi = EPI_STORE_F32;
+      a.out[0] = at<float>(ws, w.ybuf);
+      a.ldo = D;
+      if ((st = tc_launch(a, 1, plan.down, stream)) != TILEQ_OK) return st;
     }
     mark(ST_RESIDUAL, stream);
   }
-  (void)K;
   st = run_shared_and_combine(layer, li, pl, w, packed, ws, T, top_k, out, stream);
   if (st != TILEQ_OK) return st;
   return copy_route_out(layer, w, ws, T, top_k, route, stream);
@@ -771,15 +898,15 @@ tileq_status tileq_pack_per_expert(const tileq_layer *layer, const tileq_per_exp
     const ProjInfo &q = li.p[p];
     if (q.rank == 0) continue;
     if (!pe->U_pe[p] || !pe->V_pe[p]) return TILEQ_ERR_INVALID_ARG;
-    long long n = (long long)K * (q.d_out / 16) * (q.rank / 16) * 32;
+    long long n = (long long)frag_bytes(K, q.d_out, q.rank, 8) / 16;
     pack_frag_kernel<<<nblocks(n, 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(pe->U_pe[p]), (long long)q.d_out * q.rank, q.rank, 1, K,
-        q.d_out, q.rank, at<uint4>(packed_pe, pl.uf[p]));
+        q.d_out, q.rank, 8, at<uint4>(packed_pe, pl.uf[p]));
     TQ_LAUNCHED();
-    n = (long long)K * (q.rank / 16) * (q.d_in / 16) * 32;
+    n = (long long)frag_bytes(K, q.rank, q.d_in, 8) / 16;
     pack_frag_kernel<<<nblocks(n, 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(pe->V_pe[p]), (long long)q.d_in * q.rank, 1, q.rank, K,
-        q.rank, q.d_in, at<uint4>(packed_pe, pl.vf[p]));
+        q.rank, q.d_in, 8, at<uint4>(packed_pe, pl.vf[p]));
     TQ_LAUNCHED();
   }
   return TILEQ_OK;
@@ -798,21 +925,29 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
   const PackedLayout pl = packed_layout(layer, li);
   const PePackedLayout ppl = pe_layout(layer, li);
   const WsLayout w = ws_layout(layer, li, T, top_k);
+  const Plan &plan = w.plan;
   const int K = layer->K;
   const int zids[2] = {0, 0};
+  __half *xext = at<__half>(ws, w.xext);
   st = run_route_permute(layer, li, w, x, T, router_logits, top_k, ws, 0, zids, -1, stream);
   if (st != TILEQ_OK) return st;
 
-  // Per-expert low-rank pass of projection p over the expert's slots:
-  //   zpe = Sigma * (V_pe[e]^T B[slot])  then  out[slot] += U_pe[e] zpe
+  // Per-expert low-rank pass of projection(s) over the expert's slots:
+  //   zpe = Sigma * (V_pe[e]^T B[slot])   then   out[slot] += U_pe[e] zpe
+  // The tiles of one expert are contiguous in the main table from
+  // tile_first[e]; their number is known only on the device, so each
+  // per-expert launch covers the largest possible expert (T slots) and its
+  // surplus CTAs return at once.
   auto per_expert_lr = [&](int np, const int *projs, const __half *bsrc, int ldb, const int *b_row,
                            float *const *outs, int ldo) -> tileq_status {
+    const GemmPlan &gp = plan.pe;
     for (int e = 0; e < K; ++e) {
       GemmBatch zb, ub;
       for (int i = 0; i < np; ++i) {
         const ProjInfo &q = li.p[projs[i]];
-        zb.p[i] = problem();
+        zb.p[i] = problem(gp, ws, w);
         GemmProblem &z = zb.p[i];
+        z.m_tiles = cdiv(q.rank, 128);
         z.tiles = at<int4>(ws, w.tiles_main);
         z.tile_count = at<int>(ws, w.tile_counts);
         z.only_group = e;
@@ -820,7 +955,6 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
         z.d_out = q.rank;
         z.d_in = q.d_in;
         z.a[0] = at<uint4>(packed_pe, ppl.vf[projs[i]]);
-        z.a_stride = (long long)(q.rank / 16) * (q.d_in / 16) * 32;
         z.b = bsrc;
         z.ldb = ldb;
         z.b_row = b_row;
@@ -828,9 +962,9 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
         z.col_scale = layer->proj[projs[i]].Sigma;
         z.out[0] = at<__half>(ws, w.zpe[i]);
         z.ldo = q.rank;
-        z.m_tiles = cdiv(q.rank, 64);
-        ub.p[i] = problem();
+        ub.p[i] = problem(gp, ws, w);
         GemmProblem &u = ub.p[i];
+        u.m_tiles = cdiv(q.d_out, 128);
         u.tiles = z.tiles;
         u.tile_count = z.tile_count;
         u.only_group = e;
@@ -838,72 +972,63 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
         u.d_out = q.d_out;
         u.d_in = q.rank;
         u.a[0] = at<uint4>(packed_pe, ppl.uf[projs[i]]);
-        u.a_stride = (long long)(q.d_out / 16) * (q.rank / 16) * 32;
         u.b = at<__half>(ws, w.zpe[i]);
         u.ldb = q.rank;
         u.epi = EPI_ACCUM_F32;
         u.out[0] = outs[i];
         u.ldo = ldo;
-        u.m_tiles = cdiv(q.d_out, 64);
       }
-      if (launch_gemm(zb, np, GemmShape{AM_F16, 1, w.bn, 4}, cdiv(T, w.bn), stream) != cudaSuccess)
-        return TILEQ_ERR_CUDA;
-      if (launch_gemm(ub, np, GemmShape{AM_F16, 1, w.bn, 4}, cdiv(T, w.bn), stream) != cudaSuccess)
-        return TILEQ_ERR_CUDA;
+      if ((st = gemm(zb, np, AM_F16, 1, gp, stream)) != TILEQ_OK) return st;
+      if ((st = gemm(ub, np, AM_F16, 1, gp, stream)) != TILEQ_OK) return st;
     }
     return TILEQ_OK;
   };
-  // The tiles of one expert are contiguous in the main table, from
-  // tile_first[e]; the number is known only on the device, so each
-  // per-expert launch covers the largest possible expert (T slots, one per
-  // token) and its surplus CTAs return at once.
 
   if (layer->kind == TILEQ_LINEAR) {
     const ProjInfo &q = li.p[0];
-    ScaleGatherArgs sg{w.P, q.d_in, at<int>(ws, w.slot_tok), at<float>(ws, w.slot_w),
-                       at<__half>(ws, w.x16), at<__half>(ws, w.xs)};
-    scale_gather_kernel<<<nblocks((long long)w.P * (q.d_in / 2), 256), 256, 0, stream>>>(sg);
+    ScaleGatherArgs sg{plan.P, q.d_in, w.ld_x, at<int>(ws, w.slot_tok), at<float>(ws, w.slot_w),
+                       at<__half>(ws, w.x16), xext};
+    scale_gather_kernel<<<nblocks((long long)plan.P * (q.d_in / 2), 256), 256, 0, stream>>>(sg);
     TQ_LAUNCHED();
-    GemmBatch b;
-    b.p[0] = residual_problem(layer, li, pl, packed, 0);
-    GemmProblem &g = b.p[0];
-    g.tiles = at<int4>(ws, w.tiles_main);
-    g.tile_count = at<int>(ws, w.tile_counts);
-    g.b = at<__half>(ws, w.xs);
-    g.ldb = q.d_in;
-    g.epi = EPI_STORE_F32;
-    g.out[0] = at<float>(ws, w.ybuf);
-    g.ldo = q.d_out;
-    g.out_split_stride = (long long)w.P * q.d_out;
-    g.ksplit = w.ksplit;
-    if (launch_gemm(b, 1, GemmShape{AM_Q2, 1, w.bn, 4}, w.slots_main, stream) != cudaSuccess)
-      return TILEQ_ERR_CUDA;
+    TcArgs a;
+    if ((st = tc_args(&a, plan.linear, li, pl, packed, 0, ws, w, xext, w.ld_x, w.ld_x)) != TILEQ_OK)
+      return st;
+    a.epi = EPI_STORE_F32;
+    a.out[0] = at<float>(ws, w.ybuf);
+    a.ldo = q.d_out;
+    if ((st = tc_launch(a, 1, plan.linear, stream)) != TILEQ_OK) return st;
     if (q.rank > 0) {
       const int projs[1] = {0};
       float *outs[1] = {at<float>(ws, w.ybuf)};
-      st = per_expert_lr(1, projs, at<__half>(ws, w.xs), q.d_in, nullptr, outs, q.d_out);
+      st = per_expert_lr(1, projs, xext, w.ld_x, nullptr, outs, q.d_out);
       if (st != TILEQ_OK) return st;
     }
     for (int sidx = ST_ZPROJ; sidx <= ST_RESIDUAL; ++sidx) mark(sidx, stream);
   } else {
     const ProjInfo &qg = li.p[0], &qd = li.p[2];
     const int D = layer->d_model, F = layer->d_ff;
-    GemmBatch b;
-    b.p[0] = residual_problem(layer, li, pl, packed, 0);
-    GemmProblem &g = b.p[0];
-    g.a[1] = at<uint4>(packed, pl.qw[1]);
-    g.sz[1] = at<uint32_t>(packed, pl.sz[1]);
-    g.tiles = at<int4>(ws, w.tiles_main);
-    g.tile_count = at<int>(ws, w.tile_counts);
-    g.b = at<__half>(ws, w.x16);
-    g.ldb = D;
-    g.b_row = at<int>(ws, w.slot_tok);
-    g.epi = EPI_STORE2_F32;
-    g.out[0] = at<float>(ws, w.g32);
-    g.out[1] = at<float>(ws, w.u32);
-    g.ldo = F;
-    if (launch_gemm(b, 1, GemmShape{AM_Q2, 2, w.bn, 4}, w.slots_main, stream) != cudaSuccess)
-      return TILEQ_ERR_CUDA;
+    __half *hext = at<__half>(ws, w.hext);
+    GatherExtArgs ga;
+    std::memset(&ga, 0, sizeof(ga));
+    ga.P = plan.P;
+    ga.d = D;
+    ga.r = qg.rank;
+    ga.ld = w.ld_x;
+    ga.slot_tok = at<int>(ws, w.slot_tok);
+    ga.x16 = at<__half>(ws, w.x16);
+    ga.out = xext;
+    gather_ext_kernel<<<nblocks((long long)plan.P * (D / 8), 256), 256, 0, stream>>>(ga);
+    TQ_LAUNCHED();
+    TcArgs a;
+    if ((st = tc_args(&a, plan.gateup, li, pl, packed, 0, ws, w, xext, w.ld_x, w.ld_x)) != TILEQ_OK)
+      return st;
+    a.codes[1] = at<uint4>(packed, pl.qw[1]);
+    a.sz[1] = at<uint32_t>(packed, pl.sz[1]);
+    a.epi = EPI_STORE2_F32;
+    a.out[0] = at<float>(ws, w.g32);
+    a.out[1] = at<float>(ws, w.u32);
+    a.ldo = F;
+    if ((st = tc_launch(a, 2, plan.gateup, stream)) != TILEQ_OK) return st;
     if (qg.rank > 0) {
       const int projs[2] = {0, 1};
       float *outs[2] = {at<float>(ws, w.g32), at<float>(ws, w.u32)};
@@ -911,28 +1036,21 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
       if (st != TILEQ_OK) return st;
     }
     mark(ST_ZPROJ, stream);
-    SwigluArgs sa{(long long)w.P * F, F, at<float>(ws, w.g32), at<float>(ws, w.u32),
-                  at<float>(ws, w.slot_w), at<__half>(ws, w.h)};
+    SwigluArgs sa{(long long)plan.P * F, F, w.ld_h, at<float>(ws, w.g32), at<float>(ws, w.u32),
+                  at<float>(ws, w.slot_w), hext};
     swiglu_kernel<<<nblocks(sa.n, 256), 256, 0, stream>>>(sa);
     TQ_LAUNCHED();
     mark(ST_GATEUP, stream);
-    b.p[0] = residual_problem(layer, li, pl, packed, 2);
-    GemmProblem &d = b.p[0];
-    d.tiles = at<int4>(ws, w.tiles_main);
-    d.tile_count = at<int>(ws, w.tile_counts);
-    d.b = at<__half>(ws, w.h);
-    d.ldb = F;
-    d.epi = EPI_STORE_F32;
-    d.out[0] = at<float>(ws, w.ybuf);
-    d.ldo = D;
-    d.out_split_stride = (long long)w.P * D;
-    d.ksplit = w.ksplit;
-    if (launch_gemm(b, 1, GemmShape{AM_Q2, 1, w.bn, 4}, w.slots_main, stream) != cudaSuccess)
-      return TILEQ_ERR_CUDA;
+    if ((st = tc_args(&a, plan.down, li, pl, packed, 2, ws, w, hext, w.ld_h, w.ld_h)) != TILEQ_OK)
+      return st;
+    a.epi = EPI_STORE_F32;
+    a.out[0] = at<float>(ws, w.ybuf);
+    a.ldo = D;
+    if ((st = tc_launch(a, 1, plan.down, stream)) != TILEQ_OK) return st;
     if (qd.rank > 0) {
       const int projs[1] = {2};
       float *outs[1] = {at<float>(ws, w.ybuf)};
-      st = per_expert_lr(1, projs, at<__half>(ws, w.h), F, nullptr, outs, D);
+      st = per_expert_lr(1, projs, hext, w.ld_h, nullptr, outs, D);
       if (st != TILEQ_OK) return st;
     }
     mark(ST_ZDOWN, stream);

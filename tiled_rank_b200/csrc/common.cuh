@@ -100,10 +100,94 @@ __device__ __forceinline__ void dequant_k16(uint32_t w, const DqConst &c, uint32
   a[3] = h2_as_u32(__hmul2(__hfma2(v3, m64, c.nz[3]), c.sc[1]));
 }
 
-__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+// Exact q - z of one k16 step of an m16 A fragment (the group scale is applied
+// to the fp32 partial sums instead).  nz[i] = -(1024 * 4^-i + z_row(i)).
+__device__ __forceinline__ void dequant_qz_k16(uint32_t w, const __half2 (&nz)[4], uint32_t (&a)[4]) {
+  const uint32_t kMagic = 0x64006400u;
+  const __half2 v0 = u32_as_h2(and_or(w, 0x00030003u, kMagic));
+  const __half2 v1 = u32_as_h2(and_or(w, 0x000C000Cu, kMagic));
+  const __half2 v2 = u32_as_h2(and_or(w, 0x00300030u, kMagic));
+  const __half2 v3 = u32_as_h2(and_or(w, 0x00C000C0u, kMagic));
+  a[0] = h2_as_u32(__hfma2(v0, u32_as_h2(0x3C003C00u), nz[0]));
+  a[1] = h2_as_u32(__hfma2(v1, u32_as_h2(0x34003400u), nz[1]));
+  a[2] = h2_as_u32(__hfma2(v2, u32_as_h2(0x2C002C00u), nz[2]));
+  a[3] = h2_as_u32(__hfma2(v3, u32_as_h2(0x24002400u), nz[3]));
+}
+
+// D = A * B (C = 0), fp16 inputs, fp32 result.
+__device__ __forceinline__ void mma_f16_16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
 
 __device__ __forceinline__ void set_status(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+
+// ------------------------------------------------------------------ mbarrier / bulk copy
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
+  return t;
+}
+// Bounded wait: gives up after about one second (device global timer) and
+// records TILEQ_ERR_TIMEOUT in *status; a pipeline wait that long means the
+// producer or consumer on the other side has stopped.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
+  for (int i = 0; i < 64; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kWaitLimitNs) {
+      set_status(status, TILEQ_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+// 1-D bulk copy global -> shared, completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+// Named barrier over `count` threads (count a multiple of 32).
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
+
 
 }  // namespace tileq

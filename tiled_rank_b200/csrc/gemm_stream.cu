@@ -1,0 +1,329 @@
+// Streaming grouped GEMM on warp-level tensor-core MMA for the fp16 products of
+// the TileQ forward: the column projection z = Sigma*(V_n^T x), the down-side
+// projection z' = Sigma*(V_n^T h), the shared expert and the per-expert
+// low-rank launches of the unfused comparison path.  A is a packed fp16
+// fragment matrix; one producer warp feeds eight consumer warps through a ring
+// of shared-memory stages filled by bulk copies (cp.async.bulk) and handed
+// over with mbarriers, so consumer warps never wait on each other inside the
+// K loop.
+//
+//   out[item][o] = sum_k A_g[o][k] * B[row(item)][k]
+//
+// Each consumer warp owns 16 output rows (one m16 tile) of the CTA's 128-row
+// block for every projection of the launch (NP = 2 computes gate and up of
+// the same rows, so a SwiGLU epilogue stays in registers).  Split-K CTAs
+// write fp32 partials; the last CTA of a tile (arrival counter) sums them in
+// split order, so the result does not depend on scheduling.
+#include "kernels.cuh"
+
+namespace tileq {
+
+namespace {
+
+constexpr int W = 8;                     // consumer warps
+constexpr int THREADS = (W + 1) * 32;    // + one producer warp
+constexpr int BK = 128;                  // K per stage
+constexpr int BROW = BK + 8;             // padded smem row of B (halves)
+
+template <int NP, int BN>
+struct SCfg {
+  static constexpr int NT = BN / 8;
+  static constexpr int A_WARP = 8 * 32;  // uint4 per warp per projection per stage
+  static constexpr int A_BYTES = NP * W * A_WARP * 16;
+  static constexpr int B_BYTES = BN * BROW * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = (200 * 1024) / STAGE;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : (STAGES_RAW < 2 ? 2 : STAGES_RAW);
+  static constexpr int BAR_OFF = STAGES * STAGE;
+  static constexpr int SMEM = BAR_OFF + 2 * STAGES * 8 + 16;
+};
+
+__device__ __forceinline__ float epi_value(const GemmProblem &P, int item, int o, float v0, float v1) {
+  if (P.epi == EPI_SWIGLU_H) {
+    float h = silu_f(v0) * v1;
+    if (P.row_scale) h *= P.row_scale[item];
+    return h;
+  }
+  if (P.col_scale) v0 *= P.col_scale[o];
+  return v0;
+}
+
+__device__ __forceinline__ void epi_store(const GemmProblem &P, int item, int o, float v0, float v1) {
+  const size_t idx = (size_t)item * P.ldo + o;
+  switch (P.epi) {
+    case EPI_SWIGLU_H:
+    case EPI_STORE_F16:
+      reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(epi_value(P, item, o, v0, v1));
+      break;
+    case EPI_STORE_F32:
+      reinterpret_cast<float *>(P.out[0])[idx] = epi_value(P, item, o, v0, v1);
+      break;
+    case EPI_ACCUM_F32:
+      reinterpret_cast<float *>(P.out[0])[idx] += v0;
+      break;
+    default:  // EPI_STORE2_F32
+      reinterpret_cast<float *>(P.out[0])[idx] = v0;
+      reinterpret_cast<float *>(P.out[1])[idx] = v1;
+      break;
+  }
+}
+
+template <int NP, int BN>
+__global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_constant__ GemmBatch batch) {
+  using C = SCfg<NP, BN>;
+  const GemmProblem &P = batch.p[blockIdx.y];
+  extern __shared__ __align__(128) uint8_t smem[];
+
+  int bid = blockIdx.x;
+  const int split = bid % P.ksplit;
+  bid /= P.ksplit;
+  const int ob = bid % P.m_tiles;
+  const int jt = bid / P.m_tiles;
+  int grp, item0, nitems;
+  if (P.tiles != nullptr) {
+    int tj = jt;
+    if (P.only_group >= 0) {
+      tj += P.group_first_tile[P.only_group];
+      if (tj >= P.group_first_tile[P.only_group + 1]) return;
+    }
+    if (tj >= *P.tile_count) return;
+    const int4 t = P.tiles[tj];
+    grp = t.x;
+    item0 = t.y;
+    nitems = t.z;
+  } else {
+    grp = 0;
+    item0 = jt * BN;
+    if (item0 >= P.static_items) return;
+    nitems = min(BN, P.static_items - item0);
+  }
+  if (P.only_group >= 0 && grp != P.only_group) return;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ablk = P.use_a_blk ? P.a_blk[grp] : grp;
+  const int nkb = (P.d_in + BK - 1) / BK;
+  const int per = (nkb + P.ksplit - 1) / P.ksplit;
+  const int kb0 = min(nkb, split * per), kb1 = min(nkb, kb0 + per);
+  const int nst = kb1 - kb0;
+  const int n128 = P.m_tiles;
+
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+  uint64_t *empty = full + C::STAGES;
+  int *sflag = reinterpret_cast<int *>(empty + C::STAGES);
+  auto stage_a = [&](int st, int p) {
+    return reinterpret_cast<uint4 *>(smem + st * C::STAGE) + p * W * C::A_WARP;
+  };
+  auto stage_b = [&](int st) { return reinterpret_cast<__half *>(smem + st * C::STAGE + C::A_BYTES); };
+
+  // B rows past the end of K (ragged last stage) must read as zeros: clear once
+  for (int i = threadIdx.x; i < C::STAGES * C::B_BYTES / 16; i += THREADS) {
+    const int st = i / (C::B_BYTES / 16), j = i % (C::B_BYTES / 16);
+    reinterpret_cast<uint4 *>(stage_b(st))[j] = make_uint4(0, 0, 0, 0);
+  }
+  // order the generic zero stores before the bulk copies (async proxy) into the same buffers
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], W);
+    }
+    *sflag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  float acc[NP][C::NT][4];
+#pragma unroll
+  for (int p = 0; p < NP; ++p)
+#pragma unroll
+    for (int j = 0; j < C::NT; ++j)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[p][j][v] = 0.f;
+
+  if (warp == W) {
+    // ------------------------------------------------------------ producer warp
+    int issued = 0;
+    for (int it = 0; it < nst; ++it) {
+      const int s = it % C::STAGES;
+      if (it >= C::STAGES) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1, P.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+      }
+      const int kb = kb0 + it;
+      const int kvalid = min(BK, P.d_in - kb * BK);
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)C::A_BYTES + (uint32_t)nitems * kvalid * 2);
+      __syncwarp();
+      if (lane < NP) {
+        const size_t blk_off = ((size_t)ablk * n128 + ob) * nkb + kb;
+        bulk_g2s(stage_a(s, lane), P.a[lane] + blk_off * W * C::A_WARP, W * C::A_WARP * 16, &full[s]);
+      }
+      for (int n = lane; n < nitems; n += 32) {
+        const int item = item0 + n;
+        const int row = P.b_row ? P.b_row[item] : item;
+        bulk_g2s(stage_b(s) + n * BROW, P.b + (size_t)row * P.ldb + (size_t)kb * BK, kvalid * 2, &full[s]);
+      }
+      issued = it + 1;
+    }
+    // no copy may still be landing in shared memory when the CTA exits
+    if (lane == 0)
+      for (int it = max(0, issued - C::STAGES); it < issued; ++it)
+        mbar_wait(&full[it % C::STAGES], (it / C::STAGES) & 1, P.status);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ consumer warps
+    const int r0 = lane >> 2;
+    for (int it = 0; it < nst; ++it) {
+      const int s = it % C::STAGES;
+      if (!mbar_wait(&full[s], (it / C::STAGES) & 1, P.status)) break;
+      const __half *bs = stage_b(s);
+      const int kvalid = min(BK, P.d_in - (kb0 + it) * BK);
+#pragma unroll
+      for (int ks = 0; ks < BK / 16; ++ks) {
+        if (ks * 16 >= kvalid) break;
+        uint32_t bf[C::NT][2];
+        if constexpr (C::NT == 1) {
+          uint32_t r[2];
+          ldmatrix_x2(r, bs + (lane & 7) * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
+          bf[0][0] = r[0];
+          bf[0][1] = r[1];
+        } else {
+#pragma unroll
+          for (int j = 0; j < C::NT; j += 2) {
+            uint32_t r[4];
+            const int row = (j + (lane >> 4)) * 8 + (lane & 7);
+            ldmatrix_x4(r, bs + row * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
+            bf[j][0] = r[0];
+            bf[j][1] = r[1];
+            bf[j + 1][0] = r[2];
+            bf[j + 1][1] = r[3];
+          }
+        }
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const uint4 v = stage_a(s, p)[(warp * 8 + ks) * 32 + lane];
+          const uint32_t af[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[j][0], bf[j][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+
+    // ---------------------------------------------------------- epilogue / partials
+    const int cq = (lane & 3) * 2;
+    if (P.ksplit == 1) {
+#pragma unroll
+      for (int j = 0; j < C::NT; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int o = ob * kRowsPerCta + warp * 16 + r0 + 8 * h;
+          if (o >= P.d_out) continue;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int n = j * 8 + cq + cc;
+            if (n >= nitems) continue;
+            epi_store(P, item0 + n, o, acc[0][j][2 * h + cc], acc[NP - 1][j][2 * h + cc]);
+          }
+        }
+    } else {
+      const int ldp = n128 * kRowsPerCta;
+#pragma unroll
+      for (int p = 0; p < NP; ++p)
+#pragma unroll
+        for (int j = 0; j < C::NT; ++j)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int o = ob * kRowsPerCta + warp * 16 + r0 + 8 * h;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              const int n = j * 8 + cq + cc;
+              if (n >= nitems) continue;
+              P.part[(((size_t)split * NP + p) * P.part_items + item0 + n) * ldp + o] = acc[p][j][2 * h + cc];
+            }
+          }
+      __threadfence();
+    }
+  }
+
+  if (P.ksplit == 1) return;
+  // ------------------------------------------------------------ split-K: last CTA reduces
+  __syncthreads();
+  const int tile_id = blockIdx.y * (int)(gridDim.x / (P.ksplit)) + jt * P.m_tiles + ob;
+  if (threadIdx.x == 0) {
+    const int old = atomicAdd(&P.counters[tile_id], 1);
+    *sflag = (old == P.ksplit - 1);
+  }
+  __syncthreads();
+  if (!*sflag) return;
+  __threadfence();
+  const int ldp = n128 * kRowsPerCta;
+  for (int idx = threadIdx.x; idx < BN * kRowsPerCta; idx += THREADS) {
+    const int n = idx / kRowsPerCta;
+    const int o = ob * kRowsPerCta + idx % kRowsPerCta;
+    if (n >= nitems || o >= P.d_out) continue;
+    const int item = item0 + n;
+    float v[2] = {0.f, 0.f};
+    for (int sp = 0; sp < P.ksplit; ++sp)
+#pragma unroll
+      for (int p = 0; p < NP; ++p)
+        v[p] += __ldcg(&P.part[(((size_t)sp * NP + p) * P.part_items + item) * ldp + o]);
+    epi_store(P, item, o, v[0], v[NP - 1]);
+  }
+  if (threadIdx.x == 0) P.counters[tile_id] = 0;
+}
+
+template <int NP, int BN>
+cudaError_t launch_one(const GemmBatch &batch, int nprob, int n_tile_slots, cudaStream_t stream) {
+  using C = SCfg<NP, BN>;
+  auto kern = gemm_stream_kernel<NP, BN>;
+  static bool configured = false;  // one attribute call per instantiation and process
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  int mt = 0, ks = 1;
+  for (int i = 0; i < nprob; ++i) {
+    mt = max(mt, batch.p[i].m_tiles);
+    ks = max(ks, batch.p[i].ksplit);
+  }
+  for (int i = 0; i < nprob; ++i)  // the split-K tile ids assume one shape per launch
+    if (batch.p[i].ksplit > 1 && (batch.p[i].m_tiles != mt || batch.p[i].ksplit != ks))
+      return cudaErrorInvalidValue;
+  const dim3 grid((unsigned)n_tile_slots * mt * ks, nprob);
+  kern<<<grid, THREADS, C::SMEM, stream>>>(batch);
+  count_launches();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmBatch &batch, int nprob, GemmShape shape, int n_tile_slots,
+                        cudaStream_t stream) {
+  if (n_tile_slots <= 0 || nprob <= 0) return cudaSuccess;
+  if (shape.am != AM_F16) return cudaErrorInvalidValue;
+  for (int i = 0; i < nprob; ++i)
+    if (batch.p[i].m_tiles <= 0 || batch.p[i].ksplit <= 0) return cudaErrorInvalidValue;
+  if (shape.np == 1) {
+    switch (shape.bn) {
+      case 8: return launch_one<1, 8>(batch, nprob, n_tile_slots, stream);
+      case 16: return launch_one<1, 16>(batch, nprob, n_tile_slots, stream);
+      case 32: return launch_one<1, 32>(batch, nprob, n_tile_slots, stream);
+      case 64: return launch_one<1, 64>(batch, nprob, n_tile_slots, stream);
+      case 128: return launch_one<1, 128>(batch, nprob, n_tile_slots, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (shape.bn) {
+    case 8: return launch_one<2, 8>(batch, nprob, n_tile_slots, stream);
+    case 16: return launch_one<2, 16>(batch, nprob, n_tile_slots, stream);
+    case 32: return launch_one<2, 32>(batch, nprob, n_tile_slots, stream);
+    case 64: return launch_one<2, 64>(batch, nprob, n_tile_slots, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tileq

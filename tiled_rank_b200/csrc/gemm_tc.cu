@@ -1,0 +1,430 @@
+// Grouped mixed-input GEMM on the 5th-generation tensor cores (tcgen05, TMEM).
+//
+//   out[item][o] = sum_k deq(Q_e)[o][k] * B[item][k]  (+ sum_i U_m[o][i] * B[item][ext + i])
+//
+// for the residual projections of the TileQ forward (gate/up with a SwiGLU
+// epilogue, down, the linear layer).  Roles of one persistent CTA per SM:
+//   warp 0        producer: bulk copies of the packed 2-bit codes and group
+//                 scales, 2-D TMA tiles of the activation matrix B
+//                 (128-byte swizzle), into a ring of shared-memory stages;
+//   warp 1        allocates tensor memory and issues tcgen05.mma (M = 128 weight
+//                 rows, N = BN items, K = 16) with A in TMEM and B in smem;
+//   warps 2..     dequantisation: each thread owns one of the 128 weight rows,
+//                 decodes its codes into fp16 (w = s * (q - z)) and writes them
+//                 straight into the TMEM A stage with tcgen05.st; after the K
+//                 loop the same warps read the fp32 accumulators (tcgen05.ld)
+//                 and run the epilogue.
+// The low-rank term is a K extension: after the residual K loop, the A stage
+// holds rows of the shared factor U_m and B the matching columns of the item's
+// z (or a) vector, accumulated into the same TMEM accumulator.
+// Split-K work items write fp32 partials; the last one of a tile reduces them
+// in split order.  Every mbarrier wait is bounded and reports TILEQ_ERR_TIMEOUT.
+#include "kernels.cuh"
+#include "tc.cuh"
+
+namespace tileq {
+
+namespace {
+
+constexpr int BK = 128;  // K per stage
+
+template <int NP, int BN, int DQW>
+struct TcCfg {
+  static constexpr int THREADS = (2 + DQW) * 32;
+  static constexpr int KPW = BK / (DQW / 4);          // K elements per dequant warp per stage
+  static constexpr int CODES = NP * 128 * 32;         // packed codes of one stage (bytes)
+  static constexpr int SZ = NP * 2 * 128 * 4;         // scale/zero words, up to 2 groups per stage
+  static constexpr int BATOM = BN * 128;              // one 64-wide K atom of B (bytes)
+  static constexpr int B = NP * 2 * BATOM;            // main stage uses the first 2 atoms
+  static constexpr int QSTAGE = ((CODES + SZ + B) + 1023) / 1024 * 1024;
+  static constexpr int SQ_RAW = (200 * 1024) / QSTAGE;
+  static constexpr int SQ = SQ_RAW > 8 ? 8 : (SQ_RAW < 2 ? 2 : SQ_RAW);
+  static constexpr int ACC_COLS = NP * BN;
+  static constexpr int A_COLS = NP * (BK / 2);          // TMEM columns of one A stage
+  static constexpr int SA_RAW = (512 - ACC_COLS) / A_COLS;
+  static constexpr int SA = SA_RAW > 4 ? 4 : SA_RAW;
+  static constexpr int BAR_OFF = SQ * QSTAGE;
+  static constexpr int SMEM_USED = BAR_OFF + (2 * SQ + 2 * SA + 4) * 8 + 64 + 1024;  // + align slack
+  // at least half of the SM's shared memory: one CTA per SM, so the 512-column
+  // TMEM allocation never waits for another CTA of this kernel
+  static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static_assert(SA >= 2, "TMEM too small for two A stages");
+};
+
+__device__ __forceinline__ float tc_epi_value(const TcArgs &P, int item, int o, float v0, float v1) {
+  if (P.epi == EPI_SWIGLU_H) {
+    float h = silu_f(v0) * v1;
+    if (P.row_scale) h *= P.row_scale[item];
+    return h;
+  }
+  return v0;
+}
+
+__device__ __forceinline__ void tc_epi_store(const TcArgs &P, int item, int o, float v0, float v1) {
+  const size_t idx = (size_t)item * P.ldo + o;
+  if (P.epi == EPI_SWIGLU_H) {
+    reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(tc_epi_value(P, item, o, v0, v1));
+  } else if (P.epi == EPI_STORE2_F32) {
+    reinterpret_cast<float *>(P.out[0])[idx] = v0;
+    reinterpret_cast<float *>(P.out[1])[idx] = v1;
+  } else {
+    reinterpret_cast<float *>(P.out[0])[idx] = v0;
+  }
+}
+
+// Decode 16 codes (one packed word) into 8 fp16x2 of s * (q - z).
+__device__ __forceinline__ void dq_word(uint32_t w, const __half2 (&nz)[4], __half2 s2, uint32_t *out) {
+  const uint32_t kMagic = 0x64006400u;
+  const __half2 m[4] = {u32_as_h2(0x3C003C00u), u32_as_h2(0x34003400u), u32_as_h2(0x2C002C00u),
+                        u32_as_h2(0x24002400u)};
+#pragma unroll
+  for (int hb = 0; hb < 2; ++hb) {
+    const uint32_t v = hb ? (w >> 8) : w;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 x = u32_as_h2(and_or(v, 0x00030003u << (2 * i), kMagic));
+      out[4 * hb + i] = h2_as_u32(__hmul2(__hfma2(x, m[i], nz[i]), s2));
+    }
+  }
+}
+
+template <int NP, int BN, int DQW>
+__global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid_constant__ TcArgs P) {
+  using C = TcCfg<NP, BN, DQW>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *q_full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+  uint64_t *q_empty = q_full + C::SQ;
+  uint64_t *a_full = q_empty + C::SQ;
+  uint64_t *a_empty = a_full + C::SA;
+  uint64_t *acc_full = a_empty + C::SA;
+  uint64_t *acc_empty = acc_full + 1;
+  uint64_t *drain = acc_full + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 4);
+  int *flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto q_codes = [&](int s, int p) { return smem + s * C::QSTAGE + p * 128 * 32; };
+  auto q_sz = [&](int s, int p) {
+    return reinterpret_cast<uint32_t *>(smem + s * C::QSTAGE + C::CODES) + p * 2 * 128;
+  };
+  auto q_b = [&](int s) { return smem + s * C::QSTAGE + C::CODES + C::SZ; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::SQ; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], DQW + 1);
+    }
+    for (int s = 0; s < C::SA; ++s) {
+      mbar_init(&a_full[s], DQW);
+      mbar_init(&a_empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, DQW);
+    mbar_init(drain, 1);
+    *flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::alloc(tmem_slot, 512);
+    tc::relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int n_tiles = *P.tile_count;
+  const int total = n_tiles * P.m_tiles * P.ksplit;
+  const int nkb = P.d_in / BK;
+  const int per = (nkb + P.ksplit - 1) / P.ksplit;
+  const int g = P.group;
+  const int G = P.d_in / g;
+  const int gps = g == 64 ? 2 : 1;
+  const int n_ext = P.rank > 0 ? (P.rank + BK - 1) / BK : 0;
+  bool ok = true;
+
+  auto decode = [&](int w, int &jt, int &ob, int &split) {
+    split = w % P.ksplit;
+    w /= P.ksplit;
+    ob = w % P.m_tiles;
+    jt = w / P.m_tiles;
+  };
+  auto stages_of = [&](int split, int &kb0, int &nmain, int &next) {
+    kb0 = min(nkb, split * per);
+    nmain = min(nkb, kb0 + per) - kb0;
+    next = split == 0 ? n_ext : 0;
+  };
+
+  if (warp == 0) {
+    // ============================================================ producer
+    if (lane == 0) {
+      uint32_t qi = 0;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        int jt, ob, split, kb0, nmain, next;
+        decode(w, jt, ob, split);
+        stages_of(split, kb0, nmain, next);
+        const int4 t = P.tiles[jt];
+        const int grp = t.x, item0 = t.y;
+        for (int st = 0; st < nmain + next; ++st, ++qi) {
+          const int s = qi % C::SQ;
+          if (qi >= (uint32_t)C::SQ && !(ok = mbar_wait(&q_empty[s], ((qi / C::SQ) - 1) & 1, P.status))) break;
+          if (st < nmain) {
+            const int kb = kb0 + st;
+            mbar_arrive_expect_tx(&q_full[s], NP * (128 * 32 + gps * 512) + 2 * C::BATOM);
+            for (int p = 0; p < NP; ++p) {
+              const size_t cblk = (((size_t)grp * P.m_tiles + ob) * nkb + kb) * (128 * 32);
+              bulk_g2s(q_codes(s, p), reinterpret_cast<const uint8_t *>(P.codes[p]) + cblk, 128 * 32, &q_full[s]);
+              const size_t zoff = (((size_t)grp * P.m_tiles + ob) * G + (kb * BK) / g) * 128;
+              bulk_g2s(q_sz(s, p), P.sz[p] + zoff, gps * 512, &q_full[s]);
+            }
+            for (int a = 0; a < 2; ++a)
+              tc::tma_load_2d(q_b(s) + a * C::BATOM, &P.bmap, kb * BK + a * 64, item0, &q_full[s]);
+          } else {
+            const int e = st - nmain;
+            const int rlen = min(BK, P.rank - e * BK);
+            const int natoms = (rlen + 63) / 64;
+            mbar_arrive_expect_tx(&q_full[s], NP * natoms * C::BATOM);
+            for (int p = 0; p < NP; ++p)
+              for (int a = 0; a < natoms; ++a)
+                tc::tma_load_2d(q_b(s) + (p * 2 + a) * C::BATOM, &P.bmap, P.ext_col[p] + e * BK + a * 64,
+                                item0, &q_full[s]);
+          }
+        }
+      }
+      // no copy may still be landing in shared memory when the CTA exits
+      for (uint32_t i = qi > (uint32_t)C::SQ ? qi - C::SQ : 0; i < qi; ++i)
+        mbar_wait(&q_full[i % C::SQ], (i / C::SQ) & 1, P.status);
+    }
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_f16(BN);
+      uint32_t qi = 0, ai = 0, wi = 0;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++wi) {
+        int jt, ob, split, kb0, nmain, next;
+        decode(w, jt, ob, split);
+        stages_of(split, kb0, nmain, next);
+        if (wi > 0 && !(ok = mbar_wait(acc_empty, (wi - 1) & 1, P.status))) break;
+        tc::fence_after();
+        bool first = true;
+        for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
+          const int s = qi % C::SQ, sa = ai % C::SA;
+          if (!(ok = mbar_wait(&a_full[sa], (ai / C::SA) & 1, P.status))) break;
+          if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
+          tc::fence_after();
+          const bool ext = st >= nmain;
+          const int nk = ext ? (min(BK, P.rank - (st - nmain) * BK) + 15) / 16 : BK / 16;
+          const uint32_t b_base = smem_addr(q_b(s));
+          for (int p = 0; p < NP; ++p) {
+            const uint32_t d = tmem + p * BN;
+            const uint32_t a = tmem + C::ACC_COLS + sa * C::A_COLS + p * (BK / 2);
+            for (int kk = 0; kk < nk; ++kk) {
+              const int atom = (ext ? p * 2 : 0) + kk / 4;
+              const uint64_t bd = tc::sdesc_sw128(b_base + atom * C::BATOM + (kk % 4) * 32);
+              tc::mma_ts(d, a + kk * 8, bd, idesc, (first && kk == 0) ? 0u : 1u);
+            }
+          }
+          first = false;
+          tc::commit(&a_empty[sa]);
+          tc::commit(&q_empty[s]);
+        }
+        if (!ok) break;
+        tc::commit(acc_full);
+      }
+      // all issued MMAs have retired before TMEM is released
+      tc::commit(drain);
+      mbar_wait(drain, 0, P.status);
+    }
+  } else {
+    // ============================================================ dequant + epilogue
+    const int dw = warp - 2;
+    const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+    const int part = dw >> 2;                  // K slice (dequant) / column slice (epilogue)
+    const int row = quad * 32 + lane;          // weight row within the 128-row block
+    const uint32_t lane_addr = tc::lane_base(warp);
+    uint32_t qi = 0, ai = 0, wi = 0;
+    for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++wi) {
+      int jt, ob, split, kb0, nmain, next;
+      decode(w, jt, ob, split);
+      stages_of(split, kb0, nmain, next);
+      const int4 t = P.tiles[jt];
+      const int grp = t.x, item0 = t.y, nitems = t.z;
+      for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
+        const int s = qi % C::SQ, sa = ai % C::SA;
+        if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
+        if (ai >= (uint32_t)C::SA && !(ok = mbar_wait(&a_empty[sa], ((ai / C::SA) - 1) & 1, P.status))) break;
+        tc::fence_after();
+        const bool ext = st >= nmain;
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const uint32_t acol = tmem + lane_addr + C::ACC_COLS + sa * C::A_COLS + p * (BK / 2) + part * (C::KPW / 2);
+#pragma unroll
+          for (int c = 0; c < C::KPW / 32; ++c) {   // chunks of 32 K elements = 16 columns
+            uint32_t v[16];
+            const int k0 = part * C::KPW + c * 32;  // K offset within the stage
+            if (!ext) {
+              const uint32_t *cw = reinterpret_cast<const uint32_t *>(q_codes(s, p) + row * 32) + k0 / 16;
+              const int gl = g == 64 ? (k0 >> 6) : 0;
+              const __half2 sz = u32_as_h2(q_sz(s, p)[gl * 128 + row]);
+              const __half2 z2 = __high2half2(sz), s2 = __low2half2(sz);
+              const __half2 nz[4] = {__hsub2(__float2half2_rn(-1024.f), z2), __hsub2(__float2half2_rn(-256.f), z2),
+                                     __hsub2(__float2half2_rn(-64.f), z2), __hsub2(__float2half2_rn(-16.f), z2)};
+              dq_word(cw[0], nz, s2, v);
+              dq_word(cw[1], nz, s2, v + 8);
+            } else {
+              const int e = st - nmain;
+              const int kg = e * BK + k0;          // column of U
+              const int ub = P.u_blk[p][grp];
+              const __half *ur = P.u[p] + (((size_t)ub * P.m_tiles + ob) * 128 + row) * P.rank;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                uint4 q4 = make_uint4(0, 0, 0, 0);
+                if (kg + j * 8 < P.rank) q4 = *reinterpret_cast<const uint4 *>(ur + kg + j * 8);
+                v[4 * j + 0] = q4.x;
+                v[4 * j + 1] = q4.y;
+                v[4 * j + 2] = q4.z;
+                v[4 * j + 3] = q4.w;
+              }
+            }
+            tc::st16(acol + c * 16, v);
+          }
+        }
+        tc::wait_st();
+        tc::fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&a_full[sa]);
+          mbar_arrive(&q_empty[s]);
+        }
+      }
+      if (!ok) break;
+
+      // -------------------------------------------------------- epilogue
+      if (!(ok = mbar_wait(acc_full, wi & 1, P.status))) break;
+      tc::fence_after();
+      constexpr int COLS = BN / (DQW / 4);     // accumulator columns of this warp
+      constexpr int CH = COLS >= 8 ? 8 : 4;    // columns per TMEM load
+      const int o = ob * 128 + row;
+      const int ldp = P.m_tiles * 128;
+      const bool no_k = nmain + next == 0;     // a split past the end of K contributes zeros
+#pragma unroll 1
+      for (int c = 0; c < COLS; c += CH) {
+        float v[NP][CH];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const uint32_t addr = tmem + lane_addr + p * BN + part * COLS + c;
+          if constexpr (CH == 8) {
+            tc::ld8(addr, v[p]);
+          } else {
+            tc::ld4(addr, v[p]);
+          }
+        }
+        tc::wait_ld();
+        if (no_k)
+#pragma unroll
+          for (int p = 0; p < NP; ++p)
+#pragma unroll
+            for (int i = 0; i < CH; ++i) v[p][i] = 0.f;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+          const int n = part * COLS + c + i;
+          if (n >= nitems) continue;
+          if (P.ksplit == 1) {
+            if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i]);
+          } else {
+#pragma unroll
+            for (int p = 0; p < NP; ++p)
+              P.part[(((size_t)split * NP + p) * P.part_items + item0 + n) * ldp + o] = v[p][i];
+          }
+        }
+      }
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+
+      if (P.ksplit > 1) {
+        __threadfence();
+        named_sync(1, DQW * 32);
+        const int tile_id = jt * P.m_tiles + ob;
+        if (dw == 0 && lane == 0) *flag = (atomicAdd(&P.counters[tile_id], 1) == P.ksplit - 1);
+        named_sync(1, DQW * 32);
+        if (*flag) {
+          __threadfence();
+          for (int idx = dw * 32 + lane; idx < BN * 128; idx += DQW * 32) {
+            const int n = idx / 128, oo = ob * 128 + idx % 128;
+            if (n >= nitems || oo >= P.d_out) continue;
+            float r[2] = {0.f, 0.f};
+            for (int sp = 0; sp < P.ksplit; ++sp)
+#pragma unroll
+              for (int p = 0; p < NP; ++p)
+                r[p] += __ldcg(&P.part[(((size_t)sp * NP + p) * P.part_items + item0 + n) * ldp + oo]);
+            tc_epi_store(P, item0 + n, oo, r[0], r[NP - 1]);
+          }
+          if (dw == 0 && lane == 0) P.counters[tile_id] = 0;
+        }
+        named_sync(1, DQW * 32);
+      }
+    }
+  }
+
+  __syncwarp();
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after();
+    tc::dealloc(tmem, 512);
+  }
+}
+
+template <int NP, int BN, int DQW>
+cudaError_t launch_tc_one(const TcArgs &a, int grid, cudaStream_t stream) {
+  using C = TcCfg<NP, BN, DQW>;
+  auto kern = gemm_tc_kernel<NP, BN, DQW>;
+  static bool configured = false;  // one attribute call per instantiation and process
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  kern<<<grid, C::THREADS, C::SMEM, stream>>>(a);
+  count_launches();
+  return cudaGetLastError();
+}
+
+template <int NP>
+cudaError_t launch_tc_bn(const TcArgs &a, int bn, int grid, cudaStream_t s) {
+  switch (bn) {
+    case 16: return launch_tc_one<NP, 16, 16>(a, grid, s);
+    case 32: return launch_tc_one<NP, 32, 16>(a, grid, s);
+    case 64: return launch_tc_one<NP, 64, 16>(a, grid, s);
+    case 128: return launch_tc_one<NP, 128, 8>(a, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+int tc_smem_bytes(int np, int bn) {
+  if (np == 1) {
+    switch (bn) {
+      case 16: return TcCfg<1, 16, 16>::SMEM;
+      case 32: return TcCfg<1, 32, 16>::SMEM;
+      case 64: return TcCfg<1, 64, 16>::SMEM;
+      default: return TcCfg<1, 128, 8>::SMEM;
+    }
+  }
+  switch (bn) {
+    case 16: return TcCfg<2, 16, 16>::SMEM;
+    case 32: return TcCfg<2, 32, 16>::SMEM;
+    case 64: return TcCfg<2, 64, 16>::SMEM;
+    default: return TcCfg<2, 128, 8>::SMEM;
+  }
+}
+
+cudaError_t launch_gemm_tc(const TcArgs &a, int np, int bn, int grid, cudaStream_t stream) {
+  if (grid <= 0) return cudaSuccess;
+  return np == 1 ? launch_tc_bn<1>(a, bn, grid, stream) : launch_tc_bn<2>(a, bn, grid, stream);
+}
+
+}  // namespace tileq

@@ -1,5 +1,7 @@
 // Kernel argument structs and launch entry points shared by the .cu files.
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace tileq {
@@ -12,10 +14,12 @@ struct RouteArgs {
   int d_x, T, K, k;
   int32_t *topk_idx;
   float *topk_w;
+  int *zero;               // split-K arrival counters, cleared for this forward
+  int nzero;
 };
 
 struct PermuteArgs {
-  int T, k, K, M, N, bn;
+  int T, k, K, M, N, bn, bn_z;
   const int32_t *topk_idx;
   const float *topk_w;
   int *dest;               // scratch [P]
@@ -81,6 +85,13 @@ struct GemmProblem {
   const float *col_scale;
   int ksplit;
   int m_tiles;
+  // split-K (ksplit > 1): fp32 partials [ksplit][NP][items][m_tiles*128] and one
+  // arrival counter per (item tile, row block); the last CTA of a tile reduces
+  // the partials in split order and runs the epilogue.
+  float *part;
+  int part_items;
+  int *counters;
+  int *status;
 };
 
 struct GemmBatch {
@@ -88,22 +99,62 @@ struct GemmBatch {
 };
 
 struct GemmShape {
-  int am, np, bn, warps;
+  int am, np, bn;
 };
 
 // Process-wide count of kernel launches issued by the library.
 void count_launches(int n = 1);
 
+// Rows of A per CTA of the streaming GEMM (eight m16 consumer warps).
+constexpr int kRowsPerCta = 128;
+
 cudaError_t launch_gemm(const GemmBatch &batch, int nprob, GemmShape shape, int n_tile_slots,
                         cudaStream_t stream);
-int gemm_rows_per_cta(GemmShape shape);
+
+// ---------------------------------------------------------------- tcgen05 GEMM
+// Residual GEMM on the tensor cores: A = 2-bit residual of the group's expert
+// (+ the grid row's U block as a K extension), B = rows of an activation matrix
+// [items][ldb] read through a 2-D tensor map (box 64 x BN, 128-byte swizzle).
+struct TcArgs {
+  CUtensorMap bmap;
+  const int4 *tiles;
+  const int *tile_count;
+  int m_tiles, ksplit, d_out, d_in, group, rank;
+  int ext_col[2];            // first B column of the K extension of projection p
+  const uint4 *codes[2];     // [K][d_out/128][d_in/128][128 rows][32 B]
+  const uint32_t *sz[2];     // [K][d_out/128][G][128 rows] {fp16 scale, fp16 zero}
+  const __half *u[2];        // [M][pad128(d_out)][rank] fp16
+  int8_t u_blk[2][kMaxExperts];
+  int epi;
+  void *out[2];
+  int ldo;
+  const float *row_scale;
+  float *part;
+  int part_items;
+  int *counters;
+  int *status;
+};
+
+cudaError_t launch_gemm_tc(const TcArgs &a, int np, int bn, int grid, cudaStream_t stream);
+int tc_smem_bytes(int np, int bn);
 
 // ---------------------------------------------------------------- misc
+struct GatherExtArgs {
+  int P, d, r, ld;            // x_ext[s] = [x16[tok(s)] (d) | z0[zidx0[s]] (r) | z1[zidx1[s]] (r)]
+  const int *slot_tok;
+  const __half *x16;
+  const __half *z[2];
+  const int *zidx[2];
+  __half *out;
+};
+
+// Row accumulation, written per slot into the K-extension columns of the
+// activation matrix: the designated slot of each (token, grid row) gets a_{t,m},
+// every other slot zeros.
 struct LrAccArgs {
-  int k, r;
-  const int *row_offsets;  // [M+1] (only [M] used for the count)
-  int M;
-  const int *rowpair_tok, *rowpair_row;
+  int P, k, r;
+  const int32_t *sorted_pairs;
+  const int *aidx;         // slot -> rowpair (designated) or -1
   const int32_t *topk_idx;
   const float *topk_w;
   int8_t m_of[kMaxExperts];
@@ -112,7 +163,8 @@ struct LrAccArgs {
   const float *zslot;
   const __half *zcol;
   const int *zidx;
-  __half *a;               // [rowpairs][r]
+  __half *out;             // [P][ld], columns col .. col+r-1
+  int ld, col;
 };
 
 struct CombineArgs {
@@ -125,19 +177,19 @@ struct CombineArgs {
 };
 
 struct ScaleGatherArgs {
-  int P, d;
+  int P, d, ld;
   const int *slot_tok;
   const float *slot_w;
   const __half *x16;
-  __half *xs;              // [P][d]
+  __half *xs;              // [P][ld], columns 0 .. d-1
 };
 
 struct SwigluArgs {
   long long n;             // P * F
-  int F;
+  int F, ldh;
   const float *g, *u;
   const float *slot_w;
-  __half *h;
+  __half *h;               // [P][ldh]
 };
 
 __global__ void route_kernel(RouteArgs a);
@@ -145,16 +197,28 @@ __global__ void permute_kernel(PermuteArgs a);
 __global__ void lr_accumulate_kernel(LrAccArgs a);
 __global__ void combine_kernel(CombineArgs a);
 __global__ void scale_gather_kernel(ScaleGatherArgs a);
+__global__ void gather_ext_kernel(GatherExtArgs a);
 __global__ void swiglu_kernel(SwigluArgs a);
 __global__ void bounded_wait_kernel(int *status, int max_polls);
 
 // ---------------------------------------------------------------- packing
+// Packed layouts (rows padded to a multiple of 128, K to a multiple of 16*kb):
+//   codes  [blk][R/128][d_in/128][8 warps][32 lanes] uint4
+//   sz     [blk][R/128][G][8 warps][16 rows] uint32 {fp16 scale, fp16 zero}
+//   frag   [blk][R/128][C/(16*kb)][8 warps][kb k16 steps][32 lanes] uint4 (fp16 A fragments)
 __global__ void pack_codes_kernel(const uint32_t *codes, uint4 *out, int K, int d_out, int d_in);
 __global__ void pack_sz_kernel(const __half *scales, const uint8_t *zeros, uint32_t *out, int K,
                                int d_out, int G);
-// Fragment layout of a bf16 matrix S[R][C] (element (i, j) at src[i*rs + j*cs] of
-// block b at src + b*bs) -> fp16 [B][R/16][C/16][32 lanes] uint4.
+// Element (i, j) of block b of a bf16 matrix S[R][C] is src[b*bs + i*rs + j*cs].
 __global__ void pack_frag_kernel(const __nv_bfloat16 *src, long long bs, long long rs,
-                                 long long cs, int nblk, int R, int C, uint4 *out);
+                                 long long cs, int nblk, int R, int C, int kb, uint4 *out);
+// 2-bit codes -> [K][R/128][d_in/128][128 rows][8 words]: word w of a row holds
+// elements 16w..16w+15 of the 128-wide block, pair p = (2p, 2p+1) at bits
+// (2(p%4) + 8(p/4), 16 + 2(p%4) + 8(p/4)).
+__global__ void pack_codes_tc_kernel(const uint32_t *codes, uint32_t *out, int K, int d_out, int d_in);
+// bf16 [nblk][R][C] -> fp16 [nblk][pad128(R)][C] (zero rows appended).
+__global__ void pack_rows_f16_kernel(const __nv_bfloat16 *src, int nblk, int R, int C, __half *out);
+
+__host__ __device__ inline int pad128(int x) { return (x + 127) / 128 * 128; }
 
 }  // namespace tileq

@@ -5,28 +5,52 @@
 
 namespace tileq {
 
-// a[(t,m)][i] = sum over the token's slots j whose expert sits in grid row m of
-//   zslot[slot(t,j)][i]                (SwiGLU down: routing weight already in h)
-// or w_j * zcol[zidx(slot(t,j))][i]    (linear layer: z per (token, column))
-// TileQ paper, section 2.2: routing weights select the active tiles of the
-// projected [T, N, r] tensor and an in-place buffer accumulates them per grid
-// row, so the shared left factor U_m is applied once per (token, row).
+// For the designated slot s of each (token t, grid row m):
+//   out[s][col + i] = sum over the token's slots j whose expert sits in row m of
+//       zslot[slot(t,j)][i]                (SwiGLU down: routing weight already in h)
+//   or  w_j * zcol[zidx(slot(t,j))][i]     (linear layer: z per (token, column)),
+// and zeros for every other slot.  TileQ paper, section 2.2: routing weights
+// select the active tiles of the projected [T, N, r] tensor and an in-place
+// buffer accumulates them per grid row, so that the shared left factor U_m is
+// applied once per (token, row); here the buffer lives in the K-extension
+// columns of the next GEMM's activation matrix.
 __global__ void lr_accumulate_kernel(LrAccArgs a) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const int c = (int)(gid / a.r), i = (int)(gid % a.r);
-  if (c >= a.row_offsets[a.M]) return;
-  const int t = a.rowpair_tok[c], m = a.rowpair_row[c];
+  const int s = (int)(gid / a.r), i = (int)(gid % a.r);
+  if (s >= a.P) return;
   float acc = 0.f;
-  for (int j = 0; j < a.k; ++j) {
-    const int p = t * a.k + j;
-    if (a.m_of[a.topk_idx[p]] != m) continue;
-    const int slot = a.slot_of_pair[p];
-    if (a.zslot)
-      acc += a.zslot[(size_t)slot * a.r + i];
-    else
-      acc += a.topk_w[p] * __half2float(a.zcol[(size_t)a.zidx[slot] * a.r + i]);
+  if (a.aidx[s] >= 0) {
+    const int p0 = a.sorted_pairs[s];
+    const int t = p0 / a.k;
+    const int m = a.m_of[a.topk_idx[p0]];
+    for (int j = 0; j < a.k; ++j) {
+      const int p = t * a.k + j;
+      if (a.m_of[a.topk_idx[p]] != m) continue;
+      const int slot = a.slot_of_pair[p];
+      if (a.zslot)
+        acc += a.zslot[(size_t)slot * a.r + i];
+      else
+        acc += a.topk_w[p] * __half2float(a.zcol[(size_t)a.zidx[slot] * a.r + i]);
+    }
   }
-  a.a[(size_t)c * a.r + i] = __float2half_rn(acc);
+  a.out[(size_t)s * a.ld + a.col + i] = __float2half_rn(acc);
+}
+
+// x_ext[s] = [x16[tok(s)] | z0[zidx0[s]] | z1[zidx1[s]]]  (fp16, 8-element chunks)
+__global__ void gather_ext_kernel(GatherExtArgs a) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nz = a.z[0] ? (a.z[1] ? 2 : 1) : 0;
+  const int chunks = a.d / 8 + nz * (a.r / 8);
+  const int s = (int)(gid / chunks), c = (int)(gid % chunks);
+  if (s >= a.P) return;
+  uint4 v;
+  if (c < a.d / 8) {
+    v = reinterpret_cast<const uint4 *>(a.x16 + (size_t)a.slot_tok[s] * a.d)[c];
+  } else {
+    const int zc = c - a.d / 8, p = zc / (a.r / 8), cc = zc % (a.r / 8);
+    v = reinterpret_cast<const uint4 *>(a.z[p] + (size_t)a.zidx[p][s] * a.r)[cc];
+  }
+  reinterpret_cast<uint4 *>(a.out + (size_t)s * a.ld)[c] = v;
 }
 
 // out[t][:] = yshared[t][:] + sum_j sum_split ybuf[split][slot(t,j)][:], in bf16.
@@ -60,15 +84,15 @@ __global__ void scale_gather_kernel(ScaleGatherArgs a) {
   const float w = a.slot_w[s];
   const __half2 v = reinterpret_cast<const __half2 *>(a.x16 + (size_t)a.slot_tok[s] * a.d)[c];
   const float2 f = __half22float2(v);
-  reinterpret_cast<__half2 *>(a.xs + (size_t)s * a.d)[c] = __floats2half2_rn(w * f.x, w * f.y);
+  reinterpret_cast<__half2 *>(a.xs + (size_t)s * a.ld)[c] = __floats2half2_rn(w * f.x, w * f.y);
 }
 
 // h[slot][f] = w_slot * silu(g) * u  (unfused path: activation after the per-expert adds)
 __global__ void swiglu_kernel(SwigluArgs a) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.n) return;
-  const int slot = (int)(i / a.F);
-  a.h[i] = __float2half_rn(a.slot_w[slot] * silu_f(a.g[i]) * a.u[i]);
+  const int slot = (int)(i / a.F), f = (int)(i % a.F);
+  a.h[(size_t)slot * a.ldh + f] = __float2half_rn(a.slot_w[slot] * silu_f(a.g[i]) * a.u[i]);
 }
 
 // Bounded wait on an mbarrier that nothing arrives on: gives up after

@@ -1,26 +1,32 @@
 // Repacking of the stored TileQ format into the layouts the GEMM reads.
+// Rows are grouped in blocks of 128 (eight m16 tiles, one per consumer warp),
+// so that one pipeline stage of a CTA is one contiguous bulk copy.
 #include "kernels.cuh"
 
 namespace tileq {
 
 // 2-bit codes [K][d_out][d_in/16] (element j at bits 2*(j%16)) ->
-// [K][d_out/16][d_in/128][32 lanes] uint4.  Word w of lane l covers k32 block w
-// of the k128 block; within it, k16 step s and fragment register i keep the
-// (lo, hi) codes at bits (8s + 2i, 16 + 8s + 2i).  Register i is the m16n8k16
-// A-fragment register: rows r0 = l/4 (+8 for odd i), columns 2*(l%4) (+8 for i >= 2).
+// [K][R/128][d_in/128][8 warps][32 lanes] uint4.  Word w of a lane covers k32
+// block w of the k128 block; within it, k16 step s and fragment register i keep
+// the (lo, hi) codes at bits (8s + 2i, 16 + 8s + 2i).  Register i is the
+// m16n8k16 A-fragment register: rows r0 = l/4 (+8 for odd i), columns
+// 2*(l%4) (+8 for i >= 2).  Rows past d_out hold code 0.
 __global__ void pack_codes_kernel(const uint32_t *codes, uint4 *out, int K, int d_out, int d_in) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const int nkb = d_in / 128, n16 = d_out / 16, wpr = d_in / 16;
-  const long long total = (long long)K * n16 * nkb * 32;
+  const int nkb = d_in / 128, n128 = pad128(d_out) / 128, wpr = d_in / 16;
+  const long long total = (long long)K * n128 * nkb * 8 * 32;
   if (gid >= total) return;
   const int lane = (int)(gid % 32);
   long long rest = gid / 32;
+  const int w8 = (int)(rest % 8);
+  rest /= 8;
   const int kb = (int)(rest % nkb);
   rest /= nkb;
-  const int o16 = (int)(rest % n16);
-  const int e = (int)(rest / n16);
+  const int ob = (int)(rest % n128);
+  const int e = (int)(rest / n128);
   const int r0 = lane >> 2, c = (lane & 3) * 2;
   auto code = [&](int row, int col) -> uint32_t {
+    if (row >= d_out) return 0u;
     const uint32_t word = codes[((size_t)e * d_out + row) * wpr + col / 16];
     return (word >> (2 * (col % 16))) & 3u;
   };
@@ -30,7 +36,7 @@ __global__ void pack_codes_kernel(const uint32_t *codes, uint4 *out, int K, int 
     for (int s = 0; s < 2; ++s) {
       const int ks = kb * 128 + w * 32 + s * 16;
       for (int i = 0; i < 4; ++i) {
-        const int row = o16 * 16 + r0 + 8 * (i & 1);
+        const int row = ob * 128 + w8 * 16 + r0 + 8 * (i & 1);
         const int col = ks + c + 8 * (i >> 1);
         acc |= code(row, col) << (8 * s + 2 * i);
         acc |= code(row, col + 1) << (16 + 8 * s + 2 * i);
@@ -42,19 +48,27 @@ __global__ void pack_codes_kernel(const uint32_t *codes, uint4 *out, int K, int 
 }
 
 // scales fp16 [K][d_out][G], zeros [K][d_out][ceil(G/4)] ->
-// [K][d_out/16][G][16 rows] u32 = {low half: scale bits, high half: fp16(z)}.
+// [K][R/128][G][8 warps][16 rows] u32 = {low half: scale bits, high half: fp16(z)};
+// rows past d_out hold scale 0.
 __global__ void pack_sz_kernel(const __half *scales, const uint8_t *zeros, uint32_t *out, int K,
                                int d_out, int G) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long total = (long long)K * d_out * G;
+  const int n128 = pad128(d_out) / 128;
+  const long long total = (long long)K * n128 * G * 128;
   if (gid >= total) return;
   const int r = (int)(gid % 16);
   long long rest = gid / 16;
+  const int w8 = (int)(rest % 8);
+  rest /= 8;
   const int grp = (int)(rest % G);
   rest /= G;
-  const int o16 = (int)(rest % (d_out / 16));
-  const int e = (int)(rest / (d_out / 16));
-  const int row = o16 * 16 + r;
+  const int ob = (int)(rest % n128);
+  const int e = (int)(rest / n128);
+  const int row = ob * 128 + w8 * 16 + r;
+  if (row >= d_out) {
+    out[gid] = 0u;
+    return;
+  }
   const int zb = (G + 3) / 4;
   const __half s = scales[((size_t)e * d_out + row) * G + grp];
   const uint32_t z = (zeros[((size_t)e * d_out + row) * zb + grp / 4] >> (2 * (grp % 4))) & 3u;
@@ -64,30 +78,78 @@ __global__ void pack_sz_kernel(const __half *scales, const uint8_t *zeros, uint3
   out[gid] = lo | (hi << 16);
 }
 
+// bf16 matrix blocks S_b[R][C] -> fp16 A fragments
+// [nblk][R/128][C/(16*kb)][8 warps][kb k16 steps][32 lanes] uint4 (zero padded).
 __global__ void pack_frag_kernel(const __nv_bfloat16 *src, long long bs, long long rs, long long cs,
-                                 int nblk, int R, int C, uint4 *out) {
+                                 int nblk, int R, int C, int kb, uint4 *out) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const int r16 = R / 16, c16 = C / 16;
-  const long long total = (long long)nblk * r16 * c16 * 32;
+  const int n128 = pad128(R) / 128;
+  const int nkb = (C + 16 * kb - 1) / (16 * kb);
+  const long long total = (long long)nblk * n128 * nkb * 8 * kb * 32;
   if (gid >= total) return;
   const int lane = (int)(gid % 32);
   long long rest = gid / 32;
-  const int tj = (int)(rest % c16);
-  rest /= c16;
-  const int ti = (int)(rest % r16);
-  const int b = (int)(rest / r16);
+  const int ks = (int)(rest % kb);
+  rest /= kb;
+  const int w8 = (int)(rest % 8);
+  rest /= 8;
+  const int kbi = (int)(rest % nkb);
+  rest /= nkb;
+  const int ob = (int)(rest % n128);
+  const int b = (int)(rest / n128);
   const int r0 = lane >> 2, c = (lane & 3) * 2;
   const __nv_bfloat16 *base = src + b * bs;
+  auto at = [&](int row, int col) -> float {
+    if (row >= R || col >= C) return 0.f;
+    return __bfloat162float(base[row * rs + col * cs]);
+  };
   uint32_t regs[4];
   for (int i = 0; i < 4; ++i) {
-    const int row = ti * 16 + r0 + 8 * (i & 1);
-    const int col = tj * 16 + c + 8 * (i >> 1);
-    const float lo = __bfloat162float(base[row * rs + col * cs]);
-    const float hi = __bfloat162float(base[row * rs + (col + 1) * cs]);
-    const __half2 h = __floats2half2_rn(lo, hi);
+    const int row = ob * 128 + w8 * 16 + r0 + 8 * (i & 1);
+    const int col = (kbi * kb + ks) * 16 + c + 8 * (i >> 1);
+    const __half2 h = __floats2half2_rn(at(row, col), at(row, col + 1));
     regs[i] = *reinterpret_cast<const uint32_t *>(&h);
   }
   out[gid] = make_uint4(regs[0], regs[1], regs[2], regs[3]);
+}
+
+__global__ void pack_codes_tc_kernel(const uint32_t *codes, uint32_t *out, int K, int d_out, int d_in) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nkb = d_in / 128, n128 = pad128(d_out) / 128, wpr = d_in / 16;
+  const long long total = (long long)K * n128 * nkb * 128 * 8;
+  if (gid >= total) return;
+  const int w = (int)(gid % 8);
+  long long rest = gid / 8;
+  const int r = (int)(rest % 128);
+  rest /= 128;
+  const int kb = (int)(rest % nkb);
+  rest /= nkb;
+  const int ob = (int)(rest % n128);
+  const int e = (int)(rest / n128);
+  const int row = ob * 128 + r;
+  uint32_t acc = 0;
+  if (row < d_out) {
+    for (int p = 0; p < 8; ++p)
+      for (int h = 0; h < 2; ++h) {
+        const int col = kb * 128 + w * 16 + 2 * p + h;
+        const uint32_t word = codes[((size_t)e * d_out + row) * wpr + col / 16];
+        const uint32_t q = (word >> (2 * (col % 16))) & 3u;
+        acc |= q << ((h ? 16 : 0) + 2 * (p % 4) + 8 * (p / 4));
+      }
+  }
+  out[gid] = acc;
+}
+
+__global__ void pack_rows_f16_kernel(const __nv_bfloat16 *src, int nblk, int R, int C, __half *out) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int Rp = pad128(R);
+  const long long total = (long long)nblk * Rp * C;
+  if (gid >= total) return;
+  const int c = (int)(gid % C);
+  long long rest = gid / C;
+  const int r = (int)(rest % Rp);
+  const int b = (int)(rest / Rp);
+  out[gid] = r < R ? __float2half_rn(__bfloat162float(src[((size_t)b * R + r) * C + c])) : __float2half_rn(0.f);
 }
 
 }  // namespace tileq

@@ -16,6 +16,8 @@ namespace tileq {
 __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.nzero; i += gridDim.x * blockDim.x)
+    a.zero[i] = 0;
   if (warp >= a.T) return;
   const int t = warp;
   const float NEG = -INFINITY;
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
       a.zidx[zp][a.slot_of_pair[p]] = cp;
     }
     __syncthreads();
-    build_tiles(a.col_offsets[zp], a.N, a.bn, a.tiles_z[zp], a.tile_counts + 1 + zp, nullptr,
+    build_tiles(a.col_offsets[zp], a.N, a.bn_z, a.tiles_z[zp], a.tile_counts + 1 + zp, nullptr,
                 scratch);
   }
 
