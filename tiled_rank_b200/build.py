@@ -36,8 +36,8 @@ def sources():
     return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
 
 
-def _compile(src: str, extra) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, extra, build_dir: str = BUILD) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
     deps = [src] + [os.path.join(CSRC, h) for h in os.listdir(CSRC) if h.endswith(".cuh")]
     deps.append(os.path.join(INCLUDE, "tileq.h"))
     if os.path.exists(obj) and all(os.path.getmtime(obj) >= os.path.getmtime(d) for d in deps) \
@@ -52,16 +52,17 @@ def _compile(src: str, extra) -> str:
     return obj
 
 
-def build(extra=(), jobs: int = 8) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(extra=(), jobs: int = 8, out: str = LIB, build_dir: str = BUILD) -> str:
+    """Compile every .cu under csrc/ and link `out` (extra nvcc flags, e.g. -D...)."""
+    os.makedirs(build_dir, exist_ok=True)
     extra = list(extra)
     with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra), sources()))
-    cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, "-lcudart"]
+        objs = list(ex.map(lambda s: _compile(s, extra, build_dir), sources()))
+    cmd = [nvcc(), *ARCH, "-shared", "-o", out, *objs, "-lcudart"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return out
 
 
 if __name__ == "__main__":

@@ -143,6 +143,7 @@ PePackedLayout pe_layout(const tileq_layer *L, const LayerInfo &li) {
 // ------------------------------------------------------------------ launch plan
 struct GemmPlan {
   int bn = 8, slots = 0, ksplit = 1, m_tiles = 1, np = 1, items = 0;
+  bool tc = false;  // residual GEMM on tcgen05 (wide tiles) rather than warp-level MMA
   size_t part_floats() const {
     return ksplit > 1 ? (size_t)ksplit * np * std::max(items, 1) * m_tiles * kRowsPerCta : 0;
   }
@@ -185,21 +186,27 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   pl.k = k;
   pl.P = T * k;
   const int P = pl.P;
-  pl.bn_main = choose_bn_tc(P / std::max(1, L->K));
+  // One tcgen05.mma costs about the same tensor time for any N <= 256, so the
+  // residual GEMMs use it only when an expert sees many tokens; narrow tiles
+  // run on warp-level MMA.
+  const long long avg = P / std::max(1, L->K);
+  const bool use_tc = avg > 32;
+  pl.bn_main = use_tc ? choose_bn_tc(avg) : choose_bn(avg);
   pl.slots_main = cdiv(P, pl.bn_main) + L->K;
   const long long est_main = std::min(L->K, P) + P / pl.bn_main;
   const int bn_z = choose_bn(P / std::max(1, L->N));
   const int slots_z = cdiv(P, bn_z) + L->N;
   const long long est_z = std::min(L->N, P) + P / bn_z;
-  // residual GEMMs on the tensor cores: persistent CTAs walk (tile, row block, split) items
   auto tc_plan = [&](int d_out, int d_in, int np) {
     GemmPlan g;
+    g.tc = use_tc;
     g.bn = pl.bn_main;
     g.slots = pl.slots_main;
     g.m_tiles = cdiv(d_out, 128);
     g.np = np;
     g.items = P;
-    g.ksplit = choose_ksplit(est_main * g.m_tiles, d_in, 2);
+    // tcgen05: persistent CTAs walk (tile, row block, split) items; warp MMA: one CTA each
+    g.ksplit = choose_ksplit(est_main * g.m_tiles, d_in, use_tc ? 2 : 4);
     return g;
   };
   const ProjInfo &q0 = li.p[0];
@@ -449,6 +456,69 @@ void tc_ext(TcArgs *a, int slot, const LayerInfo &li, const PackedLayout &pl, co
 
 tileq_status tc_launch(const TcArgs &a, int np, const GemmPlan &g, cudaStream_t stream) {
   return launch_gemm_tc(a, np, g.bn, kNumSMs, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
+}
+
+// One residual projection (or the gate/up pair) over the main tile table:
+//   out = epi( s*(q-z) B[:, 0:d_in]  +  U_m B[:, ext .. ext + rank] )
+struct Residual {
+  int np = 1;
+  int proj[2] = {0, 0};
+  bool ext = false;
+  int ext_col[2] = {0, 0};
+  const __half *b = nullptr;
+  int ldb = 0;
+  int epi = EPI_STORE_F32;
+  void *out[2] = {nullptr, nullptr};
+  int ldo = 0;
+  const float *row_scale = nullptr;
+};
+
+tileq_status run_residual(const Residual &r, const GemmPlan &g, const LayerInfo &li, const PackedLayout &pl,
+                          const void *packed, void *ws, const WsLayout &w, cudaStream_t stream) {
+  const ProjInfo &q = li.p[r.proj[0]];
+  if (g.tc) {
+    TcArgs a;
+    tileq_status st = tc_args(&a, g, li, pl, packed, r.proj[0], ws, w, r.b, r.ldb, r.ldb);
+    if (st != TILEQ_OK) return st;
+    for (int i = 0; i < r.np; ++i) {
+      a.codes[i] = at<uint4>(packed, pl.qw[r.proj[i]]);
+      a.sz[i] = at<uint32_t>(packed, pl.sz[r.proj[i]]);
+      if (r.ext) tc_ext(&a, i, li, pl, packed, r.proj[i], r.ext_col[i]);
+    }
+    a.epi = r.epi;
+    a.out[0] = r.out[0];
+    a.out[1] = r.out[1];
+    a.ldo = r.ldo;
+    a.row_scale = r.row_scale;
+    return tc_launch(a, r.np, g, stream);
+  }
+  GemmBatch b;
+  b.p[0] = problem(g, ws, w);
+  GemmProblem &p = b.p[0];
+  p.tiles = at<int4>(ws, w.tiles_main);
+  p.tile_count = at<int>(ws, w.tile_counts);
+  p.d_out = q.d_out;
+  p.d_in = q.d_in;
+  p.group_size = q.group;
+  for (int i = 0; i < r.np; ++i) {
+    p.a[i] = at<uint4>(packed, pl.qw[r.proj[i]]);
+    p.sz[i] = at<uint32_t>(packed, pl.sz[r.proj[i]]);
+    if (r.ext) {
+      const ProjInfo &qi = li.p[r.proj[i]];
+      p.rank = qi.rank;
+      p.ext_col[i] = r.ext_col[i];
+      p.u[i] = at<__half>(packed, pl.uf[r.proj[i]]);
+      std::memcpy(p.u_blk[i], qi.m_of, kMaxExperts);
+    }
+  }
+  p.b = r.b;
+  p.ldb = r.ldb;
+  p.epi = r.epi;
+  p.out[0] = r.out[0];
+  p.out[1] = r.out[1];
+  p.ldo = r.ldo;
+  p.row_scale = r.row_scale;
+  return gemm(b, 1, AM_Q2, r.np, g, stream);
 }
 
 tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const WsLayout &w,
@@ -773,14 +843,14 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       mark(ST_ZDOWN, stream);
     }
     mark(ST_ROWACC, stream);
-    TcArgs a;
-    if ((st = tc_args(&a, plan.linear, li, pl, packed, 0, ws, w, xext, w.ld_x, w.ld_x)) != TILEQ_OK)
-      return st;
-    if (q.rank > 0) tc_ext(&a, 0, li, pl, packed, 0, q.d_in);
-    a.epi = EPI_STORE_F32;
-    a.out[0] = at<float>(ws, w.ybuf);
-    a.ldo = q.d_out;
-    if ((st = tc_launch(a, 1, plan.linear, stream)) != TILEQ_OK) return st;
+    Residual r;
+    r.ext = q.rank > 0;
+    r.ext_col[0] = q.d_in;
+    r.b = xext;
+    r.ldb = w.ld_x;
+    r.out[0] = at<float>(ws, w.ybuf);
+    r.ldo = q.d_out;
+    if ((st = run_residual(r, plan.linear, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     mark(ST_RESIDUAL, stream);
   } else {
     const ProjInfo &qg = li.p[0], &qd = li.p[2];
@@ -813,20 +883,19 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     mark(ST_ZPROJ, stream);
     {
       // gate/up residual + U_m z (K extension) + SwiGLU; h = w * silu(g) * u per slot
-      TcArgs a;
-      if ((st = tc_args(&a, plan.gateup, li, pl, packed, 0, ws, w, xext, w.ld_x, w.ld_x)) != TILEQ_OK)
-        return st;
-      a.codes[1] = at<uint4>(packed, pl.qw[1]);
-      a.sz[1] = at<uint32_t>(packed, pl.sz[1]);
-      if (lr_gu) {
-        tc_ext(&a, 0, li, pl, packed, 0, D);
-        tc_ext(&a, 1, li, pl, packed, 1, D + qg.rank);
-      }
-      a.epi = EPI_SWIGLU_H;
-      a.out[0] = hext;
-      a.ldo = w.ld_h;
-      a.row_scale = at<float>(ws, w.slot_w);
-      if ((st = tc_launch(a, 2, plan.gateup, stream)) != TILEQ_OK) return st;
+      Residual r;
+      r.np = 2;
+      r.proj[1] = 1;
+      r.ext = lr_gu;
+      r.ext_col[0] = D;
+      r.ext_col[1] = D + qg.rank;
+      r.b = xext;
+      r.ldb = w.ld_x;
+      r.epi = EPI_SWIGLU_H;
+      r.out[0] = hext;
+      r.ldo = w.ld_h;
+      r.row_scale = at<float>(ws, w.slot_w);
+      if ((st = run_residual(r, plan.gateup, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     }
     mark(ST_GATEUP, stream);
     if (lr_d) {
@@ -859,14 +928,15 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     }
     mark(ST_ROWACC, stream);
     {
-      TcArgs a;
-      if ((st = tc_args(&a, plan.down, li, pl, packed, 2, ws, w, hext, w.ld_h, w.ld_h)) != TILEQ_OK)
-        return st;
-      if (lr_d) tc_ext(&a, 0, li, pl, packed, 2, F);
-      a.epi = EPI_STORE_F32;
-      a.out[0] = at<float>(ws, w.ybuf);
-      a.ldo = D;
-      if ((st = tc_launch(a, 1, plan.down, stream)) != TILEQ_OK) return st;
+      Residual r;
+      r.proj[0] = 2;
+      r.ext = lr_d;
+      r.ext_col[0] = F;
+      r.b = hext;
+      r.ldb = w.ld_h;
+      r.out[0] = at<float>(ws, w.ybuf);
+      r.ldo = D;
+      if ((st = run_residual(r, plan.down, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     }
     mark(ST_RESIDUAL, stream);
   }
@@ -990,13 +1060,12 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
                        at<__half>(ws, w.x16), xext};
     scale_gather_kernel<<<nblocks((long long)plan.P * (q.d_in / 2), 256), 256, 0, stream>>>(sg);
     TQ_LAUNCHED();
-    TcArgs a;
-    if ((st = tc_args(&a, plan.linear, li, pl, packed, 0, ws, w, xext, w.ld_x, w.ld_x)) != TILEQ_OK)
-      return st;
-    a.epi = EPI_STORE_F32;
-    a.out[0] = at<float>(ws, w.ybuf);
-    a.ldo = q.d_out;
-    if ((st = tc_launch(a, 1, plan.linear, stream)) != TILEQ_OK) return st;
+    Residual r;
+    r.b = xext;
+    r.ldb = w.ld_x;
+    r.out[0] = at<float>(ws, w.ybuf);
+    r.ldo = q.d_out;
+    if ((st = run_residual(r, plan.linear, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     if (q.rank > 0) {
       const int projs[1] = {0};
       float *outs[1] = {at<float>(ws, w.ybuf)};
@@ -1019,16 +1088,16 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     ga.out = xext;
     gather_ext_kernel<<<nblocks((long long)plan.P * (D / 8), 256), 256, 0, stream>>>(ga);
     TQ_LAUNCHED();
-    TcArgs a;
-    if ((st = tc_args(&a, plan.gateup, li, pl, packed, 0, ws, w, xext, w.ld_x, w.ld_x)) != TILEQ_OK)
-      return st;
-    a.codes[1] = at<uint4>(packed, pl.qw[1]);
-    a.sz[1] = at<uint32_t>(packed, pl.sz[1]);
-    a.epi = EPI_STORE2_F32;
-    a.out[0] = at<float>(ws, w.g32);
-    a.out[1] = at<float>(ws, w.u32);
-    a.ldo = F;
-    if ((st = tc_launch(a, 2, plan.gateup, stream)) != TILEQ_OK) return st;
+    Residual r;
+    r.np = 2;
+    r.proj[1] = 1;
+    r.b = xext;
+    r.ldb = w.ld_x;
+    r.epi = EPI_STORE2_F32;
+    r.out[0] = at<float>(ws, w.g32);
+    r.out[1] = at<float>(ws, w.u32);
+    r.ldo = F;
+    if ((st = run_residual(r, plan.gateup, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     if (qg.rank > 0) {
       const int projs[2] = {0, 1};
       float *outs[2] = {at<float>(ws, w.g32), at<float>(ws, w.u32)};
@@ -1041,12 +1110,13 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     swiglu_kernel<<<nblocks(sa.n, 256), 256, 0, stream>>>(sa);
     TQ_LAUNCHED();
     mark(ST_GATEUP, stream);
-    if ((st = tc_args(&a, plan.down, li, pl, packed, 2, ws, w, hext, w.ld_h, w.ld_h)) != TILEQ_OK)
-      return st;
-    a.epi = EPI_STORE_F32;
-    a.out[0] = at<float>(ws, w.ybuf);
-    a.ldo = D;
-    if ((st = tc_launch(a, 1, plan.down, stream)) != TILEQ_OK) return st;
+    Residual rd;
+    rd.proj[0] = 2;
+    rd.b = hext;
+    rd.ldb = w.ld_h;
+    rd.out[0] = at<float>(ws, w.ybuf);
+    rd.ldo = D;
+    if ((st = run_residual(rd, plan.down, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     if (qd.rank > 0) {
       const int projs[1] = {2};
       float *outs[1] = {at<float>(ws, w.ybuf)};

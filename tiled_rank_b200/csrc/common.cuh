@@ -155,21 +155,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
-  return t;
-}
-// Bounded wait: gives up after about one second (device global timer) and
-// records TILEQ_ERR_TIMEOUT in *status; a pipeline wait that long means the
-// producer or consumer on the other side has stopped.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// Bounded wait: gives up after about 2^31 SM clock cycles (around a second)
+// and records TILEQ_ERR_TIMEOUT in *status; a pipeline wait that long means
+// the producer or consumer on the other side has stopped.
+constexpr long long kWaitLimitCycles = 1ll << 31;
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
-  for (int i = 0; i < 64; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (clock64() - t0 > kWaitLimitCycles) {
       set_status(status, TILEQ_ERR_TIMEOUT);
       return false;
     }

@@ -1,22 +1,45 @@
-// Streaming grouped GEMM on warp-level tensor-core MMA for the fp16 products of
-// the TileQ forward: the column projection z = Sigma*(V_n^T x), the down-side
-// projection z' = Sigma*(V_n^T h), the shared expert and the per-expert
-// low-rank launches of the unfused comparison path.  A is a packed fp16
-// fragment matrix; one producer warp feeds eight consumer warps through a ring
-// of shared-memory stages filled by bulk copies (cp.async.bulk) and handed
-// over with mbarriers, so consumer warps never wait on each other inside the
-// K loop.
+// Streaming grouped GEMM on warp-level tensor-core MMA (m16n8k16, fp16 in, fp32
+// accumulate) for the narrow products of the TileQ forward: the residual GEMMs
+// when an expert sees few tokens (decode), the column projection
+// z = Sigma*(V_n^T x), the down-side projection z' = Sigma*(V_n^T h), the
+// shared expert and the per-expert launches of the unfused path.  (A tcgen05
+// instruction costs the same tensor-core time for any N up to 256, so with a
+// handful of tokens per expert the warp-level MMA has the higher throughput.)
 //
-//   out[item][o] = sum_k A_g[o][k] * B[row(item)][k]
+//   AM_Q2   out[item][o] = sum_k s*(q - z)[o][k] * B[row(item)][k]
+//                          + sum_i U_m[o][i] * B[row(item)][ext + i]
+//           The exact (q - z) is decoded from the 2-bit codes straight into
+//           A-fragment registers (one AND-OR with the fp16 exponent of 1024 and
+//           one FMA per pair); each 64/128-wide scale group accumulates into a
+//           fresh fp32 fragment that is folded in with its scale.
+//   AM_F16  A is a packed fp16 fragment matrix (V_n^T, shared expert, ...).
 //
-// Each consumer warp owns 16 output rows (one m16 tile) of the CTA's 128-row
-// block for every projection of the launch (NP = 2 computes gate and up of
-// the same rows, so a SwiGLU epilogue stays in registers).  Split-K CTAs
-// write fp32 partials; the last CTA of a tile (arrival counter) sums them in
-// split order, so the result does not depend on scheduling.
+// One producer warp feeds eight consumer warps through a ring of shared-memory
+// stages filled by bulk copies (cp.async.bulk) and handed over with mbarriers,
+// so consumer warps never wait on each other inside the K loop.  Each consumer
+// warp owns 16 output rows of the CTA's 128-row block for every projection of
+// the launch (NP = 2: gate and up of the same rows, SwiGLU in registers).
+// Split-K CTAs write fp32 partials; the last CTA of a tile sums them in split
+// order, so the result does not depend on scheduling.
 #include "kernels.cuh"
 
 namespace tileq {
+
+#ifdef TILEQ_TRACE
+// Debug builds only: clock64 time stamps of pipeline events of CTA 0.
+__device__ unsigned long long g_st_trace[6][1024];
+#define ST_TRACE(kind, idx) \
+  do {                      \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && (idx) < 1024) g_st_trace[kind][idx] = clock64(); \
+  } while (0)
+extern "C" int tileq_debug_st_trace(unsigned long long *host) {
+  return (int)cudaMemcpyFromSymbol(host, g_st_trace, sizeof(g_st_trace));
+}
+#else
+#define ST_TRACE(kind, idx) \
+  do {                      \
+  } while (0)
+#endif
 
 namespace {
 
@@ -25,14 +48,17 @@ constexpr int THREADS = (W + 1) * 32;    // + one producer warp
 constexpr int BK = 128;                  // K per stage
 constexpr int BROW = BK + 8;             // padded smem row of B (halves)
 
-template <int NP, int BN>
+template <int AM, int NP, int BN>
 struct SCfg {
   static constexpr int NT = BN / 8;
-  static constexpr int A_WARP = 8 * 32;  // uint4 per warp per projection per stage
-  static constexpr int A_BYTES = NP * W * A_WARP * 16;
-  static constexpr int B_BYTES = BN * BROW * 2;
-  static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES_RAW = (200 * 1024) / STAGE;
+  static constexpr int A_WARP = (AM == AM_Q2) ? 0 : 8 * 32;  // uint4 per warp per projection (F16)
+  static constexpr int A_BYTES = (AM == AM_Q2) ? NP * 4096 : NP * W * A_WARP * 16;
+  static constexpr int SZ_BYTES = (AM == AM_Q2) ? NP * 2 * 512 : 0;
+  static constexpr int B_ONE = BN * BROW * 2;
+  static constexpr int B_BYTES = (AM == AM_Q2 ? NP : 1) * B_ONE;  // Q2: one B tile per projection for the extension
+  static constexpr int STAGE = A_BYTES + SZ_BYTES + B_BYTES;
+  static constexpr int BUDGET = (AM == AM_Q2 && BN <= 32) ? 74 * 1024 : 200 * 1024;
+  static constexpr int STAGES_RAW = BUDGET / STAGE;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : (STAGES_RAW < 2 ? 2 : STAGES_RAW);
   static constexpr int BAR_OFF = STAGES * STAGE;
   static constexpr int SMEM = BAR_OFF + 2 * STAGES * 8 + 16;
@@ -68,9 +94,9 @@ __device__ __forceinline__ void epi_store(const GemmProblem &P, int item, int o,
   }
 }
 
-template <int NP, int BN>
+template <int AM, int NP, int BN>
 __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_constant__ GemmBatch batch) {
-  using C = SCfg<NP, BN>;
+  using C = SCfg<AM, NP, BN>;
   const GemmProblem &P = batch.p[blockIdx.y];
   extern __shared__ __align__(128) uint8_t smem[];
 
@@ -104,21 +130,29 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
   const int nkb = (P.d_in + BK - 1) / BK;
   const int per = (nkb + P.ksplit - 1) / P.ksplit;
   const int kb0 = min(nkb, split * per), kb1 = min(nkb, kb0 + per);
-  const int nst = kb1 - kb0;
+  const int nmain = kb1 - kb0;
+  const int next = (AM == AM_Q2 && split == 0 && P.rank > 0) ? (P.rank + BK - 1) / BK : 0;
+  const int nst = nmain + next;
   const int n128 = P.m_tiles;
+  const int g = P.group_size;
+  const int G = (AM == AM_Q2) ? P.d_in / g : 1;
+  const int gps = (AM == AM_Q2 && g == 64) ? 2 : 1;
 
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   uint64_t *empty = full + C::STAGES;
   int *sflag = reinterpret_cast<int *>(empty + C::STAGES);
-  auto stage_a = [&](int st, int p) {
-    return reinterpret_cast<uint4 *>(smem + st * C::STAGE) + p * W * C::A_WARP;
+  auto stage_a = [&](int st) { return smem + st * C::STAGE; };
+  auto stage_sz = [&](int st, int p) {
+    return reinterpret_cast<uint32_t *>(smem + st * C::STAGE + C::A_BYTES) + p * 2 * 128;
   };
-  auto stage_b = [&](int st) { return reinterpret_cast<__half *>(smem + st * C::STAGE + C::A_BYTES); };
+  auto stage_b = [&](int st, int p) {
+    return reinterpret_cast<__half *>(smem + st * C::STAGE + C::A_BYTES + C::SZ_BYTES + p * C::B_ONE);
+  };
 
   // B rows past the end of K (ragged last stage) must read as zeros: clear once
-  for (int i = threadIdx.x; i < C::STAGES * C::B_BYTES / 16; i += THREADS) {
+  for (int i = threadIdx.x; i < C::STAGES * (C::B_BYTES / 16); i += THREADS) {
     const int st = i / (C::B_BYTES / 16), j = i % (C::B_BYTES / 16);
-    reinterpret_cast<uint4 *>(stage_b(st))[j] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4 *>(stage_b(st, 0))[j] = make_uint4(0, 0, 0, 0);
   }
   // order the generic zero stores before the bulk copies (async proxy) into the same buffers
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
@@ -151,18 +185,46 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
       }
-      const int kb = kb0 + it;
-      const int kvalid = min(BK, P.d_in - kb * BK);
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)C::A_BYTES + (uint32_t)nitems * kvalid * 2);
-      __syncwarp();
-      if (lane < NP) {
-        const size_t blk_off = ((size_t)ablk * n128 + ob) * nkb + kb;
-        bulk_g2s(stage_a(s, lane), P.a[lane] + blk_off * W * C::A_WARP, W * C::A_WARP * 16, &full[s]);
-      }
-      for (int n = lane; n < nitems; n += 32) {
-        const int item = item0 + n;
-        const int row = P.b_row ? P.b_row[item] : item;
-        bulk_g2s(stage_b(s) + n * BROW, P.b + (size_t)row * P.ldb + (size_t)kb * BK, kvalid * 2, &full[s]);
+      if (lane == 0) ST_TRACE(0, it);
+      if (it < nmain) {
+        const int kb = kb0 + it;
+        const int kvalid = min(BK, P.d_in - kb * BK);
+        uint32_t bytes = (uint32_t)C::A_BYTES + (uint32_t)nitems * kvalid * 2;
+        if (AM == AM_Q2) bytes += NP * gps * 512;
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
+        __syncwarp();
+        if (lane < NP) {
+          const int p = lane;
+          const size_t blk = ((size_t)ablk * n128 + ob) * nkb + kb;
+          if (AM == AM_Q2) {
+            bulk_g2s(stage_a(s) + p * 4096, reinterpret_cast<const uint8_t *>(P.a[p]) + blk * 4096, 4096, &full[s]);
+          } else {
+            bulk_g2s(stage_a(s) + p * W * C::A_WARP * 16, P.a[p] + blk * W * C::A_WARP, W * C::A_WARP * 16,
+                     &full[s]);
+          }
+        } else if (AM == AM_Q2 && lane < 2 * NP) {
+          const int p = lane - NP;
+          const size_t zoff = (((size_t)ablk * n128 + ob) * G + (kb * BK) / g) * 128;
+          bulk_g2s(stage_sz(s, p), P.sz[p] + zoff, gps * 512, &full[s]);
+        }
+        for (int n = lane; n < nitems; n += 32) {
+          const int item = item0 + n;
+          const int row = P.b_row ? P.b_row[item] : item;
+          bulk_g2s(stage_b(s, 0) + n * BROW, P.b + (size_t)row * P.ldb + (size_t)kb * BK, kvalid * 2, &full[s]);
+        }
+      } else {
+        // low-rank extension: B columns ext_col[p] + e*128 .. for each projection
+        const int e = it - nmain;
+        const int rlen = min(BK, P.rank - e * BK);
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)NP * nitems * rlen * 2);
+        __syncwarp();
+        for (int p = 0; p < NP; ++p)
+          for (int n = lane; n < nitems; n += 32) {
+            const int item = item0 + n;
+            const int row = P.b_row ? P.b_row[item] : item;
+            bulk_g2s(stage_b(s, p) + n * BROW, P.b + (size_t)row * P.ldb + P.ext_col[p] + e * BK, rlen * 2,
+                     &full[s]);
+          }
       }
       issued = it + 1;
     }
@@ -174,41 +236,135 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
   } else {
     // ------------------------------------------------------------ consumer warps
     const int r0 = lane >> 2;
+    const int rw = warp * 16 + r0;  // fragment rows rw and rw + 8 of the 128-row block
+    // per-lane decode constants: this lane's fragment columns 2*(lane%4) (+1) sit at
+    // bit 2*(lane%4) of each 16-bit half, so the AND-OR gives 1024 + 4^(lane%4) * q
+    const uint32_t lmask = 0x00030003u << (2 * (lane & 3));
+    const float lbase = 1024.f / (float)(1 << (2 * (lane & 3)));
+    const __half2 lmul = __float2half2_rn(1.f / (float)(1 << (2 * (lane & 3))));
     for (int it = 0; it < nst; ++it) {
       const int s = it % C::STAGES;
+      if (lane == 0 && (warp == 0 || warp == 7)) ST_TRACE(warp == 0 ? 1 : 3, it);
       if (!mbar_wait(&full[s], (it / C::STAGES) & 1, P.status)) break;
-      const __half *bs = stage_b(s);
-      const int kvalid = min(BK, P.d_in - (kb0 + it) * BK);
+      if (lane == 0 && warp == 0) ST_TRACE(2, it);
+      const bool ext = it >= nmain;
+      const int kvalid = ext ? min(BK, P.rank - (it - nmain) * BK) : min(BK, P.d_in - (kb0 + it) * BK);
+      // partial sums of the current scale group (R chains, folded with the scale)
+      constexpr int R = 1;
+      float part[R][NP][C::NT][4];
+      __half2 nz0[NP], nz8[NP];
+      float sc0[NP], sc8[NP];
+      uint2 wr0[NP], wr8[NP];
+      // acc += s_row * (sum of the chains) for one projection's finished scale group
+      auto fold = [&](int p) {
+#pragma unroll
+        for (int j = 0; j < C::NT; ++j)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            float t = part[0][p][j][v];
+#pragma unroll
+            for (int r = 1; r < R; ++r) t += part[r][p][j][v];
+            acc[p][j][v] = fmaf(v < 2 ? sc0[p] : sc8[p], t, acc[p][j][v]);
+          }
+      };
 #pragma unroll
       for (int ks = 0; ks < BK / 16; ++ks) {
         if (ks * 16 >= kvalid) break;
-        uint32_t bf[C::NT][2];
-        if constexpr (C::NT == 1) {
-          uint32_t r[2];
-          ldmatrix_x2(r, bs + (lane & 7) * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
-          bf[0][0] = r[0];
-          bf[0][1] = r[1];
-        } else {
+        // B fragments of this k16 step (the extension reads each projection's own tile)
+        uint32_t bf[NP][C::NT][2];
 #pragma unroll
-          for (int j = 0; j < C::NT; j += 2) {
-            uint32_t r[4];
-            const int row = (j + (lane >> 4)) * 8 + (lane & 7);
-            ldmatrix_x4(r, bs + row * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
-            bf[j][0] = r[0];
-            bf[j][1] = r[1];
-            bf[j + 1][0] = r[2];
-            bf[j + 1][1] = r[3];
+        for (int p = 0; p < NP; ++p) {
+          if (p > 0 && !(AM == AM_Q2 && ext)) {
+#pragma unroll
+            for (int j = 0; j < C::NT; ++j) {
+              bf[p][j][0] = bf[0][j][0];
+              bf[p][j][1] = bf[0][j][1];
+            }
+            continue;
+          }
+          const __half *bs = stage_b(s, p);
+          if constexpr (C::NT == 1) {
+            uint32_t r[2];
+            ldmatrix_x2(r, bs + (lane & 7) * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
+            bf[p][0][0] = r[0];
+            bf[p][0][1] = r[1];
+          } else {
+#pragma unroll
+            for (int j = 0; j < C::NT; j += 2) {
+              uint32_t r[4];
+              const int row = (j + (lane >> 4)) * 8 + (lane & 7);
+              ldmatrix_x4(r, bs + row * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
+              bf[p][j][0] = r[0];
+              bf[p][j][1] = r[1];
+              bf[p][j + 1][0] = r[2];
+              bf[p][j + 1][1] = r[3];
+            }
           }
         }
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-          const uint4 v = stage_a(s, p)[(warp * 8 + ks) * 32 + lane];
-          const uint32_t af[4] = {v.x, v.y, v.z, v.w};
+          uint32_t af[4];
+          if (AM == AM_F16) {
+            const uint4 v = reinterpret_cast<const uint4 *>(stage_a(s) + p * W * C::A_WARP * 16)[(warp * 8 + ks) * 32 + lane];
+            af[0] = v.x;
+            af[1] = v.y;
+            af[2] = v.z;
+            af[3] = v.w;
 #pragma unroll
-          for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[j][0], bf[j][1]);
+            for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[p][j][0], bf[p][j][1]);
+          } else if (ext) {
+            // A = rows of U_m (fp16), columns e*128 + ks*16 ..
+            const int e = it - nmain;
+            const __half *ur = P.u[p] + (((size_t)P.u_blk[p][grp] * n128 + ob) * 128 + rw) * P.rank +
+                               e * BK + ks * 16 + (lane & 3) * 2;
+            af[0] = *reinterpret_cast<const uint32_t *>(ur);
+            af[1] = *reinterpret_cast<const uint32_t *>(ur + 8 * P.rank);
+            af[2] = *reinterpret_cast<const uint32_t *>(ur + 8);
+            af[3] = *reinterpret_cast<const uint32_t *>(ur + 8 * P.rank + 8);
+#pragma unroll
+            for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[p][j][0], bf[p][j][1]);
+          } else {
+            // new scale group at ks 0 (and at ks 4 for groups of 64)
+            const bool gstart = ks == 0 || (g == 64 && ks == 4);
+            const int gbase = (g == 64 && ks >= 4) ? 4 : 0;
+            if (gstart) {
+              if (ks == 4) fold(p);
+              const uint32_t *szs = stage_sz(s, p) + (ks == 4 ? 128 : 0);
+              const __half2 w0 = u32_as_h2(szs[rw]), w8 = u32_as_h2(szs[rw + 8]);
+              nz0[p] = __float2half2_rn(-(lbase + __high2float(w0)));
+              nz8[p] = __float2half2_rn(-(lbase + __high2float(w8)));
+              sc0[p] = __low2float(w0);
+              sc8[p] = __low2float(w8);
+            }
+            if ((ks & 1) == 0) {  // the two 16-wide halves of a 32-wide K slice share one load
+              const uint8_t *cb = stage_a(s) + p * 4096;
+              wr0[p] = *reinterpret_cast<const uint2 *>(cb + ((ks >> 1) * 128 + rw) * 8);
+              wr8[p] = *reinterpret_cast<const uint2 *>(cb + ((ks >> 1) * 128 + rw + 8) * 8);
+            }
+            const uint32_t w0 = (ks & 1) ? wr0[p].y : wr0[p].x;
+            const uint32_t w8 = (ks & 1) ? wr8[p].y : wr8[p].x;
+            const uint32_t kMagic = 0x64006400u;
+            af[0] = h2_as_u32(__hfma2(u32_as_h2(and_or(w0, lmask, kMagic)), lmul, nz0[p]));
+            af[1] = h2_as_u32(__hfma2(u32_as_h2(and_or(w8, lmask, kMagic)), lmul, nz8[p]));
+            af[2] = h2_as_u32(__hfma2(u32_as_h2(and_or(w0 >> 8, lmask, kMagic)), lmul, nz0[p]));
+            af[3] = h2_as_u32(__hfma2(u32_as_h2(and_or(w8 >> 8, lmask, kMagic)), lmul, nz8[p]));
+            if (ks - gbase < R) {  // first step of chain ks % R in this group
+#pragma unroll
+              for (int j = 0; j < C::NT; ++j) mma_f16_16816_z(part[ks % R][p][j], af, bf[p][j][0], bf[p][j][1]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::NT; ++j) mma_f16_16816(part[ks % R][p][j], af, bf[p][j][0], bf[p][j][1]);
+            }
+          }
         }
       }
+      if (AM == AM_Q2 && !ext) {
+        // fold the last group of the stage: acc += s_row * sum_k (q - z) x
+#pragma unroll
+        for (int p = 0; p < NP; ++p) fold(p);
+      }
       __syncwarp();
+      if (lane == 0 && warp == 0) ST_TRACE(4, it);
       if (lane == 0) mbar_arrive(&empty[s]);
     }
 
@@ -275,10 +431,10 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
   if (threadIdx.x == 0) P.counters[tile_id] = 0;
 }
 
-template <int NP, int BN>
+template <int AM, int NP, int BN>
 cudaError_t launch_one(const GemmBatch &batch, int nprob, int n_tile_slots, cudaStream_t stream) {
-  using C = SCfg<NP, BN>;
-  auto kern = gemm_stream_kernel<NP, BN>;
+  using C = SCfg<AM, NP, BN>;
+  auto kern = gemm_stream_kernel<AM, NP, BN>;
   static bool configured = false;  // one attribute call per instantiation and process
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -299,31 +455,49 @@ cudaError_t launch_one(const GemmBatch &batch, int nprob, int n_tile_slots, cuda
   return cudaGetLastError();
 }
 
+template <int AM>
+cudaError_t launch_am(const GemmBatch &batch, int nprob, GemmShape shape, int slots, cudaStream_t stream) {
+  if constexpr (AM == AM_Q2) {
+    // the 2-bit path serves narrow tiles only (wider ones run on tcgen05)
+    switch (shape.bn * 4 + shape.np) {
+      case 8 * 4 + 1: return launch_one<AM, 1, 8>(batch, nprob, slots, stream);
+      case 16 * 4 + 1: return launch_one<AM, 1, 16>(batch, nprob, slots, stream);
+      case 32 * 4 + 1: return launch_one<AM, 1, 32>(batch, nprob, slots, stream);
+      case 8 * 4 + 2: return launch_one<AM, 2, 8>(batch, nprob, slots, stream);
+      case 16 * 4 + 2: return launch_one<AM, 2, 16>(batch, nprob, slots, stream);
+      case 32 * 4 + 2: return launch_one<AM, 2, 32>(batch, nprob, slots, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+  if (shape.np == 1) {
+    switch (shape.bn) {
+      case 8: return launch_one<AM, 1, 8>(batch, nprob, slots, stream);
+      case 16: return launch_one<AM, 1, 16>(batch, nprob, slots, stream);
+      case 32: return launch_one<AM, 1, 32>(batch, nprob, slots, stream);
+      case 64: return launch_one<AM, 1, 64>(batch, nprob, slots, stream);
+      case 128: return launch_one<AM, 1, 128>(batch, nprob, slots, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (shape.bn) {
+    case 8: return launch_one<AM, 2, 8>(batch, nprob, slots, stream);
+    case 16: return launch_one<AM, 2, 16>(batch, nprob, slots, stream);
+    case 32: return launch_one<AM, 2, 32>(batch, nprob, slots, stream);
+    case 64: return launch_one<AM, 2, 64>(batch, nprob, slots, stream);
+    default: return cudaErrorInvalidValue;
+  }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmBatch &batch, int nprob, GemmShape shape, int n_tile_slots,
                         cudaStream_t stream) {
   if (n_tile_slots <= 0 || nprob <= 0) return cudaSuccess;
-  if (shape.am != AM_F16) return cudaErrorInvalidValue;
   for (int i = 0; i < nprob; ++i)
     if (batch.p[i].m_tiles <= 0 || batch.p[i].ksplit <= 0) return cudaErrorInvalidValue;
-  if (shape.np == 1) {
-    switch (shape.bn) {
-      case 8: return launch_one<1, 8>(batch, nprob, n_tile_slots, stream);
-      case 16: return launch_one<1, 16>(batch, nprob, n_tile_slots, stream);
-      case 32: return launch_one<1, 32>(batch, nprob, n_tile_slots, stream);
-      case 64: return launch_one<1, 64>(batch, nprob, n_tile_slots, stream);
-      case 128: return launch_one<1, 128>(batch, nprob, n_tile_slots, stream);
-      default: return cudaErrorInvalidValue;
-    }
-  }
-  switch (shape.bn) {
-    case 8: return launch_one<2, 8>(batch, nprob, n_tile_slots, stream);
-    case 16: return launch_one<2, 16>(batch, nprob, n_tile_slots, stream);
-    case 32: return launch_one<2, 32>(batch, nprob, n_tile_slots, stream);
-    case 64: return launch_one<2, 64>(batch, nprob, n_tile_slots, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  if (shape.am == AM_Q2) return launch_am<AM_Q2>(batch, nprob, shape, n_tile_slots, stream);
+  return launch_am<AM_F16>(batch, nprob, shape, n_tile_slots, stream);
 }
 
 }  // namespace tileq

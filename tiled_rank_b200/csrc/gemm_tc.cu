@@ -24,6 +24,19 @@
 
 namespace tileq {
 
+#ifdef TILEQ_TRACE
+// Debug builds only: clock64 time stamps of pipeline events of CTA 0.
+__device__ unsigned long long g_tc_trace[8][2048];
+#define TC_TRACE(kind, idx) \
+  do {                      \
+    if (blockIdx.x == 0 && (idx) < 2048) g_tc_trace[kind][idx] = clock64(); \
+  } while (0)
+#else
+#define TC_TRACE(kind, idx) \
+  do {                      \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int BK = 128;  // K per stage
@@ -169,6 +182,7 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
         for (int st = 0; st < nmain + next; ++st, ++qi) {
           const int s = qi % C::SQ;
           if (qi >= (uint32_t)C::SQ && !(ok = mbar_wait(&q_empty[s], ((qi / C::SQ) - 1) & 1, P.status))) break;
+          TC_TRACE(0, qi);
           if (st < nmain) {
             const int kb = kb0 + st;
             mbar_arrive_expect_tx(&q_full[s], NP * (128 * 32 + gps * 512) + 2 * C::BATOM);
@@ -211,6 +225,7 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
         for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
           const int s = qi % C::SQ, sa = ai % C::SA;
           if (!(ok = mbar_wait(&a_full[sa], (ai / C::SA) & 1, P.status))) break;
+          TC_TRACE(4, qi);
           if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
           tc::fence_after();
           const bool ext = st >= nmain;
@@ -226,6 +241,7 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
             }
           }
           first = false;
+          TC_TRACE(5, qi);
           tc::commit(&a_empty[sa]);
           tc::commit(&q_empty[s]);
         }
@@ -253,7 +269,9 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
       for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
         const int s = qi % C::SQ, sa = ai % C::SA;
         if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
+        if (dw == 0 && lane == 0) TC_TRACE(1, qi);
         if (ai >= (uint32_t)C::SA && !(ok = mbar_wait(&a_empty[sa], ((ai / C::SA) - 1) & 1, P.status))) break;
+        if (dw == 0 && lane == 0) TC_TRACE(2, qi);
         tc::fence_after();
         const bool ext = st >= nmain;
 #pragma unroll
@@ -264,7 +282,7 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
             uint32_t v[16];
             const int k0 = part * C::KPW + c * 32;  // K offset within the stage
             if (!ext) {
-              const uint32_t *cw = reinterpret_cast<const uint32_t *>(q_codes(s, p) + row * 32) + k0 / 16;
+              const uint32_t *cw = reinterpret_cast<const uint32_t *>(q_codes(s, p)) + ((k0 / 32) * 128 + row) * 2;
               const int gl = g == 64 ? (k0 >> 6) : 0;
               const __half2 sz = u32_as_h2(q_sz(s, p)[gl * 128 + row]);
               const __half2 z2 = __high2half2(sz), s2 = __low2half2(sz);
@@ -290,7 +308,9 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
             tc::st16(acol + c * 16, v);
           }
         }
+        if (dw == 0 && lane == 0) TC_TRACE(3, qi);
         tc::wait_st();
+        if (dw == 0 && lane == 0) TC_TRACE(6, qi);
         tc::fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -301,7 +321,9 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
       if (!ok) break;
 
       // -------------------------------------------------------- epilogue
+      if (dw == 0 && lane == 0) TC_TRACE(7, 2 * wi);
       if (!(ok = mbar_wait(acc_full, wi & 1, P.status))) break;
+      if (dw == 0 && lane == 0) TC_TRACE(7, 2 * wi + 1);
       tc::fence_after();
       constexpr int COLS = BN / (DQW / 4);     // accumulator columns of this warp
       constexpr int CH = COLS >= 8 ? 8 : 4;    // columns per TMEM load
@@ -404,6 +426,12 @@ cudaError_t launch_tc_bn(const TcArgs &a, int bn, int grid, cudaStream_t s) {
 }
 
 }  // namespace
+
+#ifdef TILEQ_TRACE
+extern "C" int tileq_debug_tc_trace(unsigned long long *host) {
+  return (int)cudaMemcpyFromSymbol(host, g_tc_trace, sizeof(g_tc_trace));
+}
+#endif
 
 int tc_smem_bytes(int np, int bn) {
   if (np == 1) {

@@ -50,9 +50,14 @@ enum AMode { AM_Q2 = 0, AM_F16 = 1 };
 enum Epi { EPI_SWIGLU_H = 0, EPI_STORE_F32 = 1, EPI_STORE_F16 = 2, EPI_ACCUM_F32 = 3,
            EPI_STORE2_F32 = 4 };
 
-// One grouped GEMM  out[item][o] = sum_k A_g[o][k] * B[row(item)][k]  (+ low-rank
-// extension), items grouped by tiles (group, item0, nitems).  A rows are
-// output features; items are tokens / slots / (token, column) pairs.
+// One grouped GEMM  out[item][o] = sum_k A_g[o][k] * B[row(item)][k]  (+ a
+// low-rank K extension), items grouped by tiles (group, item0, nitems).  A rows
+// are output features; items are tokens / slots / (token, column) pairs.
+//   AM_F16: A = packed fp16 fragments [blk][R/128][K/128][8 warps][8 k16][32 lanes].
+//   AM_Q2:  A = 2-bit residual of expert `group` in the row layout of the
+//           tensor-core kernel ([4 K slices][128 rows][2 words] per 128x128
+//           block) with scale/zero words; the extension adds U_m (fp16 rows)
+//           times B columns ext_col[p] .. ext_col[p] + rank.
 struct GemmProblem {
   const int4 *tiles;
   const int *tile_count;
@@ -63,24 +68,18 @@ struct GemmProblem {
   const uint4 *a[2];
   const uint32_t *sz[2];
   int group_size;
-  long long a_stride;     // uint4 per A block
-  long long sz_stride;    // u32 per A block
   int use_a_blk;
   int8_t a_blk[kMaxExperts];
   const __half *b;
   int ldb;
   const int *b_row;
   int rank;
-  const uint4 *u[2];
-  long long u_stride;     // uint4 per U block
+  int ext_col[2];
+  const __half *u[2];     // [M][pad128(d_out)][rank] fp16
   int8_t u_blk[2][kMaxExperts];
-  const __half *zb[2];
-  int ldz;
-  const int *z_row[2];
   int epi;
   void *out[2];
   int ldo;
-  long long out_split_stride;
   const float *row_scale;
   const float *col_scale;
   int ksplit;
@@ -121,7 +120,7 @@ struct TcArgs {
   const int *tile_count;
   int m_tiles, ksplit, d_out, d_in, group, rank;
   int ext_col[2];            // first B column of the K extension of projection p
-  const uint4 *codes[2];     // [K][d_out/128][d_in/128][128 rows][32 B]
+  const uint4 *codes[2];     // [K][d_out/128][d_in/128][4 slices][128 rows][8 B]
   const uint32_t *sz[2];     // [K][d_out/128][G][128 rows] {fp16 scale, fp16 zero}
   const __half *u[2];        // [M][pad128(d_out)][rank] fp16
   int8_t u_blk[2][kMaxExperts];
@@ -212,9 +211,10 @@ __global__ void pack_sz_kernel(const __half *scales, const uint8_t *zeros, uint3
 // Element (i, j) of block b of a bf16 matrix S[R][C] is src[b*bs + i*rs + j*cs].
 __global__ void pack_frag_kernel(const __nv_bfloat16 *src, long long bs, long long rs,
                                  long long cs, int nblk, int R, int C, int kb, uint4 *out);
-// 2-bit codes -> [K][R/128][d_in/128][128 rows][8 words]: word w of a row holds
-// elements 16w..16w+15 of the 128-wide block, pair p = (2p, 2p+1) at bits
-// (2(p%4) + 8(p/4), 16 + 2(p%4) + 8(p/4)).
+// 2-bit codes -> [K][R/128][d_in/128][4 K slices][128 rows][2 words]: word wi of
+// slice part of a row holds elements 32*part + 16*wi .. +15 of the 128-wide block,
+// pair p = (2p, 2p+1) at bits (2(p%4) + 8(p/4), 16 + 2(p%4) + 8(p/4)).  One warp
+// reading one slice of 32 consecutive rows touches 256 contiguous bytes.
 __global__ void pack_codes_tc_kernel(const uint32_t *codes, uint32_t *out, int K, int d_out, int d_in);
 // bf16 [nblk][R][C] -> fp16 [nblk][pad128(R)][C] (zero rows appended).
 __global__ void pack_rows_f16_kernel(const __nv_bfloat16 *src, int nblk, int R, int C, __half *out);

@@ -118,10 +118,13 @@ __global__ void pack_codes_tc_kernel(const uint32_t *codes, uint32_t *out, int K
   const int nkb = d_in / 128, n128 = pad128(d_out) / 128, wpr = d_in / 16;
   const long long total = (long long)K * n128 * nkb * 128 * 8;
   if (gid >= total) return;
-  const int w = (int)(gid % 8);
-  long long rest = gid / 8;
-  const int r = (int)(rest % 128);
-  rest /= 128;
+  // word index within the 4 KB block of (expert, row block, k block):
+  // (part * 128 + row) * 2 + wi, part = 32-element K slice, wi = 16-element half
+  const int wi = (int)(gid % 2);
+  const int r = (int)((gid / 2) % 128);
+  const int part = (int)((gid / 256) % 4);
+  const int w = part * 2 + wi;
+  long long rest = gid / 1024;
   const int kb = (int)(rest % nkb);
   rest /= nkb;
   const int ob = (int)(rest % n128);
