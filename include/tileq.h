@@ -171,6 +171,34 @@ tileq_status tileq_route(const float *router_logits, int T, int K, int top_k,
                          tileq_route_out *route, void *ws, size_t ws_bytes,
                          tileq_stream_t stream);
 
+/* Largest T * top_k that tileq_route_static accepts. */
+#define TILEQ_ROUTE_STATIC_MAX_PAIRS 8192
+
+/* Routing and permutation with no workspace argument and no device allocation.
+ * The pages have no counterpart for this call: it is a library convenience.
+ *
+ * Same computation and outputs as tileq_route (all four route outputs
+ * required), but the scratch is a fixed 6 MiB array inside the library, one
+ * per device, instead of a caller-supplied workspace.  It serves callers that
+ * cannot allocate device memory at the point where they route: a C host
+ * program that has no device allocator of its own, or a framework hook that
+ * runs where its memory pool must not grow.  The call itself never calls
+ * cudaMalloc, cudaFree or any other allocating routine.
+ *
+ *   router_logits  device fp32 [T, K]; 1 <= K <= 64, 1 <= top_k <= min(K, 8)
+ *   route          device outputs as in tileq_route_out (all four non-NULL)
+ * T * top_k > TILEQ_ROUTE_STATIC_MAX_PAIRS returns TILEQ_ERR_UNSUPPORTED before
+ * anything is enqueued; T == 0 enqueues nothing.
+ *
+ * Set-up: the first call on a device (with that device current) looks up the
+ * scratch address and zeroes it, synchronously; make that first call before
+ * any stream capture begins.  Later calls are asynchronous on `stream`.
+ * All calls on one device share the one scratch array: two calls whose work
+ * overlaps on the device (different streams, or different host threads) race
+ * and may return wrong results; order them on one stream or with events. */
+tileq_status tileq_route_static(const float *router_logits, int T, int K, int top_k,
+                                tileq_route_out *route, tileq_stream_t stream);
+
 /* Synchronously read (and clear) the device status word in `ws`.
  * *status receives TILEQ_OK or the first device error recorded. */
 tileq_status tileq_device_status(void *ws, int *status, tileq_stream_t stream);

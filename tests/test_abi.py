@@ -145,3 +145,28 @@ def test_forward_validation_before_launch(L):
     st = lib.tileq_route(fake, 4, 4, 2, ctypes.byref(r), fake, 1 << 20, None)
     assert st == L.TILEQ_ERR_INVALID_ARG                          # route outputs missing
     assert L.status_string(L.TILEQ_ERR_TIMEOUT) == "TILEQ_ERR_TIMEOUT"
+
+
+def test_route_static_validation_before_launch(L):
+    """Too many pairs is rejected on the host, before any device work."""
+    fake = L.tileq_route_out(1, 1, 1, 1)  # never dereferenced: validation fails first
+    for T, K, k, want in [(4097, 8, 2, L.TILEQ_ERR_UNSUPPORTED), (16, 8, 9, L.TILEQ_ERR_INVALID_ARG),
+                          (16, 65, 2, L.TILEQ_ERR_INVALID_ARG)]:
+        st = L.lib().tileq_route_static(1, T, K, k, ctypes.byref(fake), None)
+        assert st == want, (T, K, k, st)
+
+
+def test_route_static_scratch_covers_max_pairs(L):
+    """The routing-only workspace at TILEQ_ROUTE_STATIC_MAX_PAIRS fits the 6 MiB static scratch."""
+    max_pairs = 8192
+    hdr = open(os.path.join(ROOT, "include", "tileq.h")).read()
+    assert f"#define TILEQ_ROUTE_STATIC_MAX_PAIRS {max_pairs}" in hdr
+    for K in (2, 8, 60, 64):
+        grid = (ctypes.c_int32 * K)(*range(K))
+        c = L.tileq_layer()
+        c.kind, c.K, c.M, c.N = L.TILEQ_LINEAR, K, K, 1
+        c.proj[0].d_in, c.proj[0].d_out, c.proj[0].group = 128, 16, 128
+        c.proj[0].grid_assign = ctypes.cast(grid, ctypes.POINTER(ctypes.c_int32))
+        for k in (1, 2, 4, 8):
+            if k <= K:
+                assert L.tileq_workspace_size(c, max_pairs // k, k) <= 6 << 20, (K, k)

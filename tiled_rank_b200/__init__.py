@@ -6,7 +6,8 @@ its thin ctypes binding plus a helper that keeps a layer's device tensors.
 from ._lib import (  # noqa: F401
     TILEQ_LINEAR, TILEQ_SWIGLU, TileQError, status_string, tileq_device_status,
     tileq_moe_forward, tileq_moe_forward_unfused, tileq_pack, tileq_pack_per_expert,
-    tileq_packed_per_expert_size, tileq_packed_size, tileq_route, tileq_selftest_bounded_wait,
+    tileq_packed_per_expert_size, tileq_packed_size, tileq_route, tileq_route_static,
+    tileq_selftest_bounded_wait,
     tileq_workspace_size, tileq_set_stage_events, tileq_launch_count,
 )
 from .layer import DeviceLayer  # noqa: F401

@@ -27,7 +27,7 @@ TILEQ_SWIGLU = 1
 EXPORTS = (
     "tileq_status_string", "tileq_packed_size", "tileq_pack", "tileq_workspace_size",
     "tileq_moe_forward", "tileq_packed_per_expert_size", "tileq_pack_per_expert",
-    "tileq_moe_forward_unfused", "tileq_route", "tileq_device_status",
+    "tileq_moe_forward_unfused", "tileq_route", "tileq_route_static", "tileq_device_status",
     "tileq_selftest_bounded_wait", "tileq_set_stage_events", "tileq_launch_count",
 )
 
@@ -85,6 +85,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tileq_moe_forward_unfused": ([P(tileq_layer), vp, vp, vp, c_int, vp, c_int, vp, vp,
                                        c_size, P(tileq_route_out), vp], c_int),
         "tileq_route": ([vp, c_int, c_int, c_int, P(tileq_route_out), vp, c_size, vp], c_int),
+        "tileq_route_static": ([vp, c_int, c_int, c_int, P(tileq_route_out), vp], c_int),
         "tileq_device_status": ([vp, P(c_int), vp], c_int),
         "tileq_selftest_bounded_wait": ([vp, c_size, c_int, vp], c_int),
         "tileq_set_stage_events": ([P(vp), c_int], c_int),
@@ -194,6 +195,11 @@ def tileq_moe_forward_unfused(layer: tileq_layer, packed, packed_pe, x, T: int, 
 def tileq_route(router_logits, T: int, K: int, top_k: int, route: dict, ws, stream=None):
     _check(lib().tileq_route(_ptr(router_logits), T, K, top_k, _route_struct(route), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "tileq_route")
+
+
+def tileq_route_static(router_logits, T: int, K: int, top_k: int, route: dict, stream=None):
+    _check(lib().tileq_route_static(_ptr(router_logits), T, K, top_k, _route_struct(route),
+                                    _stream(stream)), "tileq_route_static")
 
 
 def tileq_device_status(ws, stream=None) -> int:

@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include <cudaTypedefs.h>
@@ -1206,6 +1207,78 @@ tileq_status tileq_selftest_bounded_wait(void *ws, size_t ws_bytes, int max_poll
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free routing
+// tileq_route_static runs the same route and permute kernels as tileq_route,
+// but its scratch is this file's static device array instead of a
+// caller-supplied workspace, so a caller needs no device allocation at all.
+namespace {
+
+constexpr size_t kRouteStaticBytes = (size_t)6 << 20;  // 6 MiB per device
+constexpr int kRouteStaticDevices = 64;
+
+static __device__ __align__(256) unsigned char g_route_scratch[kRouteStaticBytes];
+
+std::mutex g_route_static_mu;
+void *g_route_static_ptr[kRouteStaticDevices] = {};
+
+// Set-up, once per device with that device current: look up the address of
+// the static scratch and zero it (the status word and the split-K counters of
+// the workspace layout must start at zero).  Runs synchronously, so the first
+// call on a device must not be made while a stream is being captured.
+tileq_status route_static_scratch(void **ptr) {
+  int dev = -1;
+  TQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kRouteStaticDevices) return TILEQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_route_static_mu);
+  if (g_route_static_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return TILEQ_ERR_CUDA;
+    TQ_CUDA(cudaMemset(p, 0, kRouteStaticBytes));
+    TQ_CUDA(cudaDeviceSynchronize());
+    g_route_static_ptr[dev] = p;
+  }
+  *ptr = g_route_static_ptr[dev];
+  return TILEQ_OK;
+}
+
+}  // namespace
+
+extern "C" tileq_status tileq_route_static(const float *router_logits, int T, int K, int top_k,
+                                           tileq_route_out *route, tileq_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (T < 0 || K < 1 || K > kMaxExperts || top_k < 1 || top_k > K || top_k > kMaxTopK)
+    return TILEQ_ERR_INVALID_ARG;
+  if (!route || !route->topk_idx || !route->topk_w || !route->expert_offsets || !route->sorted_pairs)
+    return TILEQ_ERR_INVALID_ARG;
+  if ((long long)T * top_k > TILEQ_ROUTE_STATIC_MAX_PAIRS) return TILEQ_ERR_UNSUPPORTED;
+  if (T == 0) return TILEQ_OK;
+  if (!router_logits) return TILEQ_ERR_INVALID_ARG;
+  // the same routing-only layout as tileq_route: K experts on a K x 1 grid
+  tileq_layer L;
+  std::memset(&L, 0, sizeof(L));
+  L.kind = TILEQ_LINEAR;
+  L.K = K;
+  L.M = K;
+  L.N = 1;
+  int32_t grid[kMaxExperts];
+  for (int e = 0; e < K; ++e) grid[e] = e;
+  L.proj[0].d_in = 128;
+  L.proj[0].d_out = 16;
+  L.proj[0].group = 128;
+  L.proj[0].grid_assign = grid;
+  LayerInfo li;
+  tileq_status st = validate_layer(&L, &li, false);
+  if (st != TILEQ_OK) return st;
+  const WsLayout w = ws_layout(&L, li, T, top_k);
+  if (w.total > kRouteStaticBytes) return TILEQ_ERR_UNSUPPORTED;
+  void *ws = nullptr;
+  if ((st = route_static_scratch(&ws)) != TILEQ_OK) return st;
+  const int zids[2] = {0, 0};
+  st = run_route_permute(&L, li, w, nullptr, T, router_logits, top_k, ws, 0, zids, -1, stream);
+  if (st != TILEQ_OK) return st;
+  return copy_route_out(&L, w, ws, T, top_k, route, stream);
+}
 
 namespace tileq {
 void count_launches(int n) { g_launches.fetch_add((unsigned long long)n); }
