@@ -94,8 +94,10 @@ size_t frag_bytes(int nblk, int R, int C, int kb) {
   return (size_t)nblk * pad128(R) * (size_t)cdiv(C, 16 * kb) * 16 * kb * 2;
 }
 
+// qw: codes in the row layout of the tcgen05 kernel; qf: the same codes in the
+// per-lane A-fragment order of the warp-MMA streaming kernel.
 struct PackedLayout {
-  size_t qw[3], sz[3], uf[3], vf[3], sh[3], total;
+  size_t qw[3], qf[3], sz[3], uf[3], vf[3], sh[3], total;
 };
 
 PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
@@ -104,6 +106,8 @@ PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
   for (int p = 0; p < li.nproj; ++p) {
     const ProjInfo &q = li.p[p];
     pl.qw[p] = off;
+    off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 4);
+    pl.qf[p] = off;
     off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 4);
     pl.sz[p] = off;
     off += align_up((size_t)L->K * pad128(q.d_out) * q.G * 4);
@@ -502,7 +506,7 @@ tileq_status run_residual(const Residual &r, const GemmPlan &g, const LayerInfo 
   p.d_in = q.d_in;
   p.group_size = q.group;
   for (int i = 0; i < r.np; ++i) {
-    p.a[i] = at<uint4>(packed, pl.qw[r.proj[i]]);
+    p.a[i] = at<uint4>(packed, pl.qf[r.proj[i]]);
     p.sz[i] = at<uint32_t>(packed, pl.sz[r.proj[i]]);
     if (r.ext) {
       const ProjInfo &qi = li.p[r.proj[i]];
@@ -754,6 +758,9 @@ tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_by
     {
       const long long n = (long long)K * (pad128(q.d_out) / 128) * (q.d_in / 128) * 128 * 8;
       pack_codes_tc_kernel<<<nblocks(n, 256), 256, 0, stream>>>(src.codes, at<uint32_t>(packed, pl.qw[p]),
+                                                                 K, q.d_out, q.d_in);
+      TQ_LAUNCHED();
+      pack_codes_kernel<<<nblocks(n / 4, 256), 256, 0, stream>>>(src.codes, at<uint4>(packed, pl.qf[p]),
                                                                  K, q.d_out, q.d_in);
       TQ_LAUNCHED();
     }

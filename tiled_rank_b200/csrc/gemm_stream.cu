@@ -8,10 +8,12 @@
 //
 //   AM_Q2   out[item][o] = sum_k s*(q - z)[o][k] * B[row(item)][k]
 //                          + sum_i U_m[o][i] * B[row(item)][ext + i]
-//           The exact (q - z) is decoded from the 2-bit codes straight into
-//           A-fragment registers (one AND-OR with the fp16 exponent of 1024 and
-//           one FMA per pair); each 64/128-wide scale group accumulates into a
-//           fresh fp32 fragment that is folded in with its scale.
+//           The 2-bit codes are stored per lane in the m16n8k16 A-fragment
+//           order (16 bytes per lane per 128x128 block, one shared-memory load
+//           per stage).  The exact (q - z) is decoded straight into fragment
+//           registers (one AND-OR with the fp16 exponent of 1024 and one FMA
+//           per pair); each 64/128-wide scale group accumulates into a fresh
+//           fp32 fragment that is folded in with its scale.
 //   AM_F16  A is a packed fp16 fragment matrix (V_n^T, shared expert, ...).
 //
 // One producer warp feeds eight consumer warps through a ring of shared-memory
@@ -21,6 +23,8 @@
 // the launch (NP = 2: gate and up of the same rows, SwiGLU in registers).
 // Split-K CTAs write fp32 partials; the last CTA of a tile sums them in split
 // order, so the result does not depend on scheduling.
+#include <type_traits>
+
 #include "kernels.cuh"
 
 namespace tileq {
@@ -62,6 +66,10 @@ struct SCfg {
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : (STAGES_RAW < 2 ? 2 : STAGES_RAW);
   static constexpr int BAR_OFF = STAGES * STAGE;
   static constexpr int SMEM = BAR_OFF + 2 * STAGES * 8 + 16;
+  // resident CTAs per SM the register budget is sized for (shared memory allows 3
+  // for the narrow 2-bit tiles, 1 for the fp16 ones)
+  static constexpr int MINB = (AM == AM_Q2) ? (NP * NT <= 2 ? 3 : 2) : 1;
+  static constexpr int RPL = (BN + 31) / 32;  // B rows per producer lane
 };
 
 __device__ __forceinline__ float epi_value(const GemmProblem &P, int item, int o, float v0, float v1) {
@@ -95,7 +103,8 @@ __device__ __forceinline__ void epi_store(const GemmProblem &P, int item, int o,
 }
 
 template <int AM, int NP, int BN>
-__global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_constant__ GemmBatch batch) {
+__global__ void __launch_bounds__(THREADS, SCfg<AM, NP, BN>::MINB)
+    gemm_stream_kernel(const __grid_constant__ GemmBatch batch) {
   using C = SCfg<AM, NP, BN>;
   const GemmProblem &P = batch.p[blockIdx.y];
   extern __shared__ __align__(128) uint8_t smem[];
@@ -176,6 +185,13 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
 
   if (warp == W) {
     // ------------------------------------------------------------ producer warp
+    // the B rows of this tile, looked up once (lane l copies items l, l+32, ..)
+    int brow[C::RPL];
+#pragma unroll
+    for (int j = 0; j < C::RPL; ++j) {
+      const int n = lane + 32 * j;
+      brow[j] = n < nitems ? (P.b_row ? P.b_row[item0 + n] : item0 + n) : 0;
+    }
     int issued = 0;
     for (int it = 0; it < nst; ++it) {
       const int s = it % C::STAGES;
@@ -207,10 +223,12 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
           const size_t zoff = (((size_t)ablk * n128 + ob) * G + (kb * BK) / g) * 128;
           bulk_g2s(stage_sz(s, p), P.sz[p] + zoff, gps * 512, &full[s]);
         }
-        for (int n = lane; n < nitems; n += 32) {
-          const int item = item0 + n;
-          const int row = P.b_row ? P.b_row[item] : item;
-          bulk_g2s(stage_b(s, 0) + n * BROW, P.b + (size_t)row * P.ldb + (size_t)kb * BK, kvalid * 2, &full[s]);
+#pragma unroll
+        for (int j = 0; j < C::RPL; ++j) {
+          const int n = lane + 32 * j;
+          if (n < nitems)
+            bulk_g2s(stage_b(s, 0) + n * BROW, P.b + (size_t)brow[j] * P.ldb + (size_t)kb * BK, kvalid * 2,
+                     &full[s]);
         }
       } else {
         // low-rank extension: B columns ext_col[p] + e*128 .. for each projection
@@ -219,11 +237,12 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
         if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)NP * nitems * rlen * 2);
         __syncwarp();
         for (int p = 0; p < NP; ++p)
-          for (int n = lane; n < nitems; n += 32) {
-            const int item = item0 + n;
-            const int row = P.b_row ? P.b_row[item] : item;
-            bulk_g2s(stage_b(s, p) + n * BROW, P.b + (size_t)row * P.ldb + P.ext_col[p] + e * BK, rlen * 2,
-                     &full[s]);
+#pragma unroll
+          for (int j = 0; j < C::RPL; ++j) {
+            const int n = lane + 32 * j;
+            if (n < nitems)
+              bulk_g2s(stage_b(s, p) + n * BROW, P.b + (size_t)brow[j] * P.ldb + P.ext_col[p] + e * BK,
+                       rlen * 2, &full[s]);
           }
       }
       issued = it + 1;
@@ -237,131 +256,148 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
     // ------------------------------------------------------------ consumer warps
     const int r0 = lane >> 2;
     const int rw = warp * 16 + r0;  // fragment rows rw and rw + 8 of the 128-row block
-    // per-lane decode constants: this lane's fragment columns 2*(lane%4) (+1) sit at
-    // bit 2*(lane%4) of each 16-bit half, so the AND-OR gives 1024 + 4^(lane%4) * q
-    const uint32_t lmask = 0x00030003u << (2 * (lane & 3));
-    const float lbase = 1024.f / (float)(1 << (2 * (lane & 3)));
-    const __half2 lmul = __float2half2_rn(1.f / (float)(1 << (2 * (lane & 3))));
+
+    // B fragments of k16 step ks for every projection (the extension reads each
+    // projection's own tile; otherwise all projections share tile 0)
+    auto load_b = [&](int s, int ks, bool ext, uint32_t (&bf)[NP][C::NT][2]) {
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        if (p > 0 && !(AM == AM_Q2 && ext)) {
+#pragma unroll
+          for (int j = 0; j < C::NT; ++j) {
+            bf[p][j][0] = bf[0][j][0];
+            bf[p][j][1] = bf[0][j][1];
+          }
+          continue;
+        }
+        const __half *bs = stage_b(s, p);
+        if constexpr (C::NT == 1) {
+          uint32_t r[2];
+          ldmatrix_x2(r, bs + (lane & 7) * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
+          bf[p][0][0] = r[0];
+          bf[p][0][1] = r[1];
+        } else {
+#pragma unroll
+          for (int j = 0; j < C::NT; j += 2) {
+            uint32_t r[4];
+            const int row = (j + (lane >> 4)) * 8 + (lane & 7);
+            ldmatrix_x4(r, bs + row * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
+            bf[p][j][0] = r[0];
+            bf[p][j][1] = r[1];
+            bf[p][j + 1][0] = r[2];
+            bf[p][j + 1][1] = r[3];
+          }
+        }
+      }
+    };
+
+    // One stage of fp16 A (packed fragments, or the rows of U_m for the
+    // extension); FULL stages run all eight k16 steps without a bound check.
+    auto stage_f16 = [&](int s, int it, bool ext, int kvalid, auto full_tag) {
+      constexpr bool FULL = decltype(full_tag)::value;
+#pragma unroll
+      for (int ks = 0; ks < BK / 16; ++ks) {
+        if (!FULL && ks * 16 >= kvalid) break;
+        uint32_t bf[NP][C::NT][2];
+        load_b(s, ks, ext, bf);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          uint32_t af[4];
+          if (AM == AM_F16) {
+            const uint4 v =
+                reinterpret_cast<const uint4 *>(stage_a(s) + p * W * C::A_WARP * 16)[(warp * 8 + ks) * 32 + lane];
+            af[0] = v.x;
+            af[1] = v.y;
+            af[2] = v.z;
+            af[3] = v.w;
+          } else {
+            // A = rows of U_m (fp16), columns e*128 + ks*16 ..
+            const int e = it - nmain;
+            const __half *ur = P.u[p] + (((size_t)P.u_blk[p][grp] * n128 + ob) * 128 + rw) * P.rank + e * BK +
+                               ks * 16 + (lane & 3) * 2;
+            af[0] = __ldg(reinterpret_cast<const unsigned int *>(ur));
+            af[1] = __ldg(reinterpret_cast<const unsigned int *>(ur + 8 * P.rank));
+            af[2] = __ldg(reinterpret_cast<const unsigned int *>(ur + 8));
+            af[3] = __ldg(reinterpret_cast<const unsigned int *>(ur + 8 * P.rank + 8));
+          }
+#pragma unroll
+          for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[p][j][0], bf[p][j][1]);
+        }
+      }
+    };
+
+    // One full stage of the 2-bit residual: 128 rows x 128 K per projection.
+    auto stage_q2 = [&](int s, int it) {
+      uint4 cw[NP];
+#pragma unroll
+      for (int p = 0; p < NP; ++p) cw[p] = reinterpret_cast<const uint4 *>(stage_a(s) + p * 4096)[warp * 32 + lane];
+      float part[NP][C::NT][4];
+      __half2 nz[NP][4];
+      float sc0[NP], sc8[NP];
+      // scale group of k16 step ks: 64-wide groups start a new one at ks 4
+      auto group_consts = [&](int ks) {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const uint32_t *szs = stage_sz(s, p) + (ks == 4 ? 128 : 0);
+          const __half2 w0 = u32_as_h2(szs[rw]), w8 = u32_as_h2(szs[rw + 8]);
+          const __half2 z0 = __high2half2(w0), z8 = __high2half2(w8);
+          nz[p][0] = __hsub2(u32_as_h2(0xE400E400u), z0);  // -(1024 + z)
+          nz[p][1] = __hsub2(u32_as_h2(0xDC00DC00u), z8);  // -(256 + z)
+          nz[p][2] = __hsub2(u32_as_h2(0xD400D400u), z0);  // -(64 + z)
+          nz[p][3] = __hsub2(u32_as_h2(0xCC00CC00u), z8);  // -(16 + z)
+          sc0[p] = __low2float(w0);
+          sc8[p] = __low2float(w8);
+        }
+      };
+      auto fold = [&]() {
+#pragma unroll
+        for (int p = 0; p < NP; ++p)
+#pragma unroll
+          for (int j = 0; j < C::NT; ++j)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) acc[p][j][v] = fmaf(v < 2 ? sc0[p] : sc8[p], part[p][j][v], acc[p][j][v]);
+      };
+      group_consts(0);
+#pragma unroll
+      for (int ks = 0; ks < BK / 16; ++ks) {
+        const bool gstart = ks == 0 || (g == 64 && ks == 4);
+        if (ks == 4 && g == 64) {
+          fold();
+          group_consts(4);
+        }
+        uint32_t bf[NP][C::NT][2];
+        load_b(s, ks, false, bf);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const uint32_t word = (ks >> 1) == 0 ? cw[p].x : (ks >> 1) == 1 ? cw[p].y : (ks >> 1) == 2 ? cw[p].z : cw[p].w;
+          uint32_t af[4];
+          dequant_qz_k16((ks & 1) ? (word >> 8) : word, nz[p], af);
+          if (gstart) {
+#pragma unroll
+            for (int j = 0; j < C::NT; ++j) mma_f16_16816_z(part[p][j], af, bf[p][j][0], bf[p][j][1]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < C::NT; ++j) mma_f16_16816(part[p][j], af, bf[p][j][0], bf[p][j][1]);
+          }
+        }
+      }
+      fold();
+    };
+
     for (int it = 0; it < nst; ++it) {
       const int s = it % C::STAGES;
       if (lane == 0 && (warp == 0 || warp == 7)) ST_TRACE(warp == 0 ? 1 : 3, it);
       if (!mbar_wait(&full[s], (it / C::STAGES) & 1, P.status)) break;
       if (lane == 0 && warp == 0) ST_TRACE(2, it);
       const bool ext = it >= nmain;
-      const int kvalid = ext ? min(BK, P.rank - (it - nmain) * BK) : min(BK, P.d_in - (kb0 + it) * BK);
-      // partial sums of the current scale group (R chains, folded with the scale)
-      constexpr int R = 1;
-      float part[R][NP][C::NT][4];
-      __half2 nz0[NP], nz8[NP];
-      float sc0[NP], sc8[NP];
-      uint2 wr0[NP], wr8[NP];
-      // acc += s_row * (sum of the chains) for one projection's finished scale group
-      auto fold = [&](int p) {
-#pragma unroll
-        for (int j = 0; j < C::NT; ++j)
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            float t = part[0][p][j][v];
-#pragma unroll
-            for (int r = 1; r < R; ++r) t += part[r][p][j][v];
-            acc[p][j][v] = fmaf(v < 2 ? sc0[p] : sc8[p], t, acc[p][j][v]);
-          }
-      };
-#pragma unroll
-      for (int ks = 0; ks < BK / 16; ++ks) {
-        if (ks * 16 >= kvalid) break;
-        // B fragments of this k16 step (the extension reads each projection's own tile)
-        uint32_t bf[NP][C::NT][2];
-#pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          if (p > 0 && !(AM == AM_Q2 && ext)) {
-#pragma unroll
-            for (int j = 0; j < C::NT; ++j) {
-              bf[p][j][0] = bf[0][j][0];
-              bf[p][j][1] = bf[0][j][1];
-            }
-            continue;
-          }
-          const __half *bs = stage_b(s, p);
-          if constexpr (C::NT == 1) {
-            uint32_t r[2];
-            ldmatrix_x2(r, bs + (lane & 7) * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
-            bf[p][0][0] = r[0];
-            bf[p][0][1] = r[1];
-          } else {
-#pragma unroll
-            for (int j = 0; j < C::NT; j += 2) {
-              uint32_t r[4];
-              const int row = (j + (lane >> 4)) * 8 + (lane & 7);
-              ldmatrix_x4(r, bs + row * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
-              bf[p][j][0] = r[0];
-              bf[p][j][1] = r[1];
-              bf[p][j + 1][0] = r[2];
-              bf[p][j + 1][1] = r[3];
-            }
-          }
-        }
-#pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          uint32_t af[4];
-          if (AM == AM_F16) {
-            const uint4 v = reinterpret_cast<const uint4 *>(stage_a(s) + p * W * C::A_WARP * 16)[(warp * 8 + ks) * 32 + lane];
-            af[0] = v.x;
-            af[1] = v.y;
-            af[2] = v.z;
-            af[3] = v.w;
-#pragma unroll
-            for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[p][j][0], bf[p][j][1]);
-          } else if (ext) {
-            // A = rows of U_m (fp16), columns e*128 + ks*16 ..
-            const int e = it - nmain;
-            const __half *ur = P.u[p] + (((size_t)P.u_blk[p][grp] * n128 + ob) * 128 + rw) * P.rank +
-                               e * BK + ks * 16 + (lane & 3) * 2;
-            af[0] = *reinterpret_cast<const uint32_t *>(ur);
-            af[1] = *reinterpret_cast<const uint32_t *>(ur + 8 * P.rank);
-            af[2] = *reinterpret_cast<const uint32_t *>(ur + 8);
-            af[3] = *reinterpret_cast<const uint32_t *>(ur + 8 * P.rank + 8);
-#pragma unroll
-            for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[p][j][0], bf[p][j][1]);
-          } else {
-            // new scale group at ks 0 (and at ks 4 for groups of 64)
-            const bool gstart = ks == 0 || (g == 64 && ks == 4);
-            const int gbase = (g == 64 && ks >= 4) ? 4 : 0;
-            if (gstart) {
-              if (ks == 4) fold(p);
-              const uint32_t *szs = stage_sz(s, p) + (ks == 4 ? 128 : 0);
-              const __half2 w0 = u32_as_h2(szs[rw]), w8 = u32_as_h2(szs[rw + 8]);
-              nz0[p] = __float2half2_rn(-(lbase + __high2float(w0)));
-              nz8[p] = __float2half2_rn(-(lbase + __high2float(w8)));
-              sc0[p] = __low2float(w0);
-              sc8[p] = __low2float(w8);
-            }
-            if ((ks & 1) == 0) {  // the two 16-wide halves of a 32-wide K slice share one load
-              const uint8_t *cb = stage_a(s) + p * 4096;
-              wr0[p] = *reinterpret_cast<const uint2 *>(cb + ((ks >> 1) * 128 + rw) * 8);
-              wr8[p] = *reinterpret_cast<const uint2 *>(cb + ((ks >> 1) * 128 + rw + 8) * 8);
-            }
-            const uint32_t w0 = (ks & 1) ? wr0[p].y : wr0[p].x;
-            const uint32_t w8 = (ks & 1) ? wr8[p].y : wr8[p].x;
-            const uint32_t kMagic = 0x64006400u;
-            af[0] = h2_as_u32(__hfma2(u32_as_h2(and_or(w0, lmask, kMagic)), lmul, nz0[p]));
-            af[1] = h2_as_u32(__hfma2(u32_as_h2(and_or(w8, lmask, kMagic)), lmul, nz8[p]));
-            af[2] = h2_as_u32(__hfma2(u32_as_h2(and_or(w0 >> 8, lmask, kMagic)), lmul, nz0[p]));
-            af[3] = h2_as_u32(__hfma2(u32_as_h2(and_or(w8 >> 8, lmask, kMagic)), lmul, nz8[p]));
-            if (ks - gbase < R) {  // first step of chain ks % R in this group
-#pragma unroll
-              for (int j = 0; j < C::NT; ++j) mma_f16_16816_z(part[ks % R][p][j], af, bf[p][j][0], bf[p][j][1]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < C::NT; ++j) mma_f16_16816(part[ks % R][p][j], af, bf[p][j][0], bf[p][j][1]);
-            }
-          }
-        }
-      }
       if (AM == AM_Q2 && !ext) {
-        // fold the last group of the stage: acc += s_row * sum_k (q - z) x
-#pragma unroll
-        for (int p = 0; p < NP; ++p) fold(p);
+        stage_q2(s, it);  // d_in is a multiple of 128: main stages are always full
+      } else {
+        const int kvalid = ext ? min(BK, P.rank - (it - nmain) * BK) : min(BK, P.d_in - (kb0 + it) * BK);
+        if (kvalid == BK)
+          stage_f16(s, it, ext, kvalid, std::true_type{});
+        else
+          stage_f16(s, it, ext, kvalid, std::false_type{});
       }
       __syncwarp();
       if (lane == 0 && warp == 0) ST_TRACE(4, it);

@@ -54,10 +54,10 @@ enum Epi { EPI_SWIGLU_H = 0, EPI_STORE_F32 = 1, EPI_STORE_F16 = 2, EPI_ACCUM_F32
 // low-rank K extension), items grouped by tiles (group, item0, nitems).  A rows
 // are output features; items are tokens / slots / (token, column) pairs.
 //   AM_F16: A = packed fp16 fragments [blk][R/128][K/128][8 warps][8 k16][32 lanes].
-//   AM_Q2:  A = 2-bit residual of expert `group` in the row layout of the
-//           tensor-core kernel ([4 K slices][128 rows][2 words] per 128x128
-//           block) with scale/zero words; the extension adds U_m (fp16 rows)
-//           times B columns ext_col[p] .. ext_col[p] + rank.
+//   AM_Q2:  A = 2-bit residual of expert `group` in the per-lane fragment
+//           layout ([8 warps][32 lanes] uint4 per 128x128 block, see
+//           pack_codes_kernel) with scale/zero words; the extension adds U_m
+//           (fp16 rows) times B columns ext_col[p] .. ext_col[p] + rank.
 struct GemmProblem {
   const int4 *tiles;
   const int *tile_count;
