@@ -31,7 +31,7 @@ struct ProjInfo {
 };
 
 struct LayerInfo {
-  int nproj;
+  int nproj, K;
   ProjInfo p[3];
   int d_x, d_y;
 };
@@ -42,6 +42,7 @@ tileq_status validate_layer(const tileq_layer *L, LayerInfo *li, bool need_devic
   if (L->K < 1 || L->M < 1 || L->N < 1 || (long long)L->M * L->N < L->K) return TILEQ_ERR_INVALID_ARG;
   if (L->K > kMaxExperts || L->M > kMaxExperts || L->N > kMaxExperts) return TILEQ_ERR_UNSUPPORTED;
   li->nproj = L->kind == TILEQ_LINEAR ? 1 : 3;
+  li->K = L->K;
   for (int pi = 0; pi < li->nproj; ++pi) {
     const tileq_proj &p = L->proj[pi];
     ProjInfo &q = li->p[pi];
@@ -399,8 +400,8 @@ GemmProblem problem(const GemmPlan &g, void *ws, const WsLayout &w) {
   return p;
 }
 
-tileq_status gemm(const GemmBatch &b, int nprob, int am, int np, const GemmPlan &g, cudaStream_t s) {
-  if (launch_gemm(b, nprob, GemmShape{am, np, g.bn}, g.slots, s) != cudaSuccess)
+tileq_status gemm(const GemmBatch &b, int nprob, int np, const GemmPlan &g, cudaStream_t s) {
+  if (launch_gemm(b, nprob, GemmShape{np, g.bn}, g.slots, s) != cudaSuccess)
     return TILEQ_ERR_CUDA;
   return TILEQ_OK;
 }
@@ -440,6 +441,7 @@ tileq_status tc_args(TcArgs *a, const GemmPlan &g, const LayerInfo &li, const Pa
   a->d_out = q.d_out;
   a->d_in = q.d_in;
   a->group = q.group;
+  a->n_experts = li.K;
   a->codes[0] = at<uint4>(packed, pl.qw[p]);
   a->sz[0] = at<uint32_t>(packed, pl.sz[p]);
   a->part = at<float>(ws, w.part);
@@ -480,50 +482,22 @@ struct Residual {
 
 tileq_status run_residual(const Residual &r, const GemmPlan &g, const LayerInfo &li, const PackedLayout &pl,
                           const void *packed, void *ws, const WsLayout &w, cudaStream_t stream) {
-  const ProjInfo &q = li.p[r.proj[0]];
-  if (g.tc) {
-    TcArgs a;
-    tileq_status st = tc_args(&a, g, li, pl, packed, r.proj[0], ws, w, r.b, r.ldb, r.ldb);
-    if (st != TILEQ_OK) return st;
-    for (int i = 0; i < r.np; ++i) {
-      a.codes[i] = at<uint4>(packed, pl.qw[r.proj[i]]);
-      a.sz[i] = at<uint32_t>(packed, pl.sz[r.proj[i]]);
-      if (r.ext) tc_ext(&a, i, li, pl, packed, r.proj[i], r.ext_col[i]);
-    }
-    a.epi = r.epi;
-    a.out[0] = r.out[0];
-    a.out[1] = r.out[1];
-    a.ldo = r.ldo;
-    a.row_scale = r.row_scale;
-    return tc_launch(a, r.np, g, stream);
-  }
-  GemmBatch b;
-  b.p[0] = problem(g, ws, w);
-  GemmProblem &p = b.p[0];
-  p.tiles = at<int4>(ws, w.tiles_main);
-  p.tile_count = at<int>(ws, w.tile_counts);
-  p.d_out = q.d_out;
-  p.d_in = q.d_in;
-  p.group_size = q.group;
+  TcArgs a;
+  tileq_status st = tc_args(&a, g, li, pl, packed, r.proj[0], ws, w, r.b, r.ldb, r.ldb);
+  if (st != TILEQ_OK) return st;
   for (int i = 0; i < r.np; ++i) {
-    p.a[i] = at<uint4>(packed, pl.qf[r.proj[i]]);
-    p.sz[i] = at<uint32_t>(packed, pl.sz[r.proj[i]]);
-    if (r.ext) {
-      const ProjInfo &qi = li.p[r.proj[i]];
-      p.rank = qi.rank;
-      p.ext_col[i] = r.ext_col[i];
-      p.u[i] = at<__half>(packed, pl.uf[r.proj[i]]);
-      std::memcpy(p.u_blk[i], qi.m_of, kMaxExperts);
-    }
+    // tcgen05 reads the row layout of the codes, warp MMA the fragment layout
+    a.codes[i] = at<uint4>(packed, g.tc ? pl.qw[r.proj[i]] : pl.qf[r.proj[i]]);
+    a.sz[i] = at<uint32_t>(packed, pl.sz[r.proj[i]]);
+    if (r.ext) tc_ext(&a, i, li, pl, packed, r.proj[i], r.ext_col[i]);
   }
-  p.b = r.b;
-  p.ldb = r.ldb;
-  p.epi = r.epi;
-  p.out[0] = r.out[0];
-  p.out[1] = r.out[1];
-  p.ldo = r.ldo;
-  p.row_scale = r.row_scale;
-  return gemm(b, 1, AM_Q2, r.np, g, stream);
+  a.epi = r.epi;
+  a.out[0] = r.out[0];
+  a.out[1] = r.out[1];
+  a.ldo = r.ldo;
+  a.row_scale = r.row_scale;
+  if (g.tc) return tc_launch(a, r.np, g, stream);
+  return launch_gemm_q2(a, r.np, g.bn, g.slots, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
 }
 
 tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const WsLayout &w,
@@ -625,7 +599,7 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
     g.epi = EPI_SWIGLU_H;
     g.out[0] = at<__half>(ws, w.hs);
     g.ldo = Fs;
-    if (gemm(b, 1, AM_F16, 2, w.plan.sh_gu, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
+    if (gemm(b, 1, 2, w.plan.sh_gu, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
     b.p[0] = problem(w.plan.sh_down, ws, w);
     GemmProblem &d = b.p[0];
     d.static_items = T;
@@ -637,7 +611,7 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
     d.epi = EPI_STORE_F32;
     d.out[0] = at<float>(ws, w.ys);
     d.ldo = D;
-    if (gemm(b, 1, AM_F16, 1, w.plan.sh_down, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
+    if (gemm(b, 1, 1, w.plan.sh_down, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
     yshared = at<float>(ws, w.ys);
   }
   mark(ST_SHARED, stream);
@@ -714,7 +688,7 @@ tileq_status run_zproj(const tileq_layer *layer, const LayerInfo &li, const Pack
     z.ldo = q.rank;
     z.part = at<float>(ws, w.part) + (size_t)p * w.part_zstride;
   }
-  return gemm(b, nz, AM_F16, 1, w.plan.zproj, stream);
+  return gemm(b, nz, 1, w.plan.zproj, stream);
 }
 
 }  // namespace
@@ -925,7 +899,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       z.col_scale = layer->proj[2].Sigma;
       z.out[0] = at<float>(ws, w.zs);
       z.ldo = qd.rank;
-      if ((st = gemm(b, 1, AM_F16, 1, plan.zdown, stream)) != TILEQ_OK) return st;
+      if ((st = gemm(b, 1, 1, plan.zdown, stream)) != TILEQ_OK) return st;
       mark(ST_ZDOWN, stream);
       LrAccArgs la = lracc_args(qd, w, ws, top_k, hext, w.ld_h, F);
       la.zslot = at<float>(ws, w.zs);
@@ -1056,8 +1030,8 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
         u.out[0] = outs[i];
         u.ldo = ldo;
       }
-      if ((st = gemm(zb, np, AM_F16, 1, gp, stream)) != TILEQ_OK) return st;
-      if ((st = gemm(ub, np, AM_F16, 1, gp, stream)) != TILEQ_OK) return st;
+      if ((st = gemm(zb, np, 1, gp, stream)) != TILEQ_OK) return st;
+      if ((st = gemm(ub, np, 1, gp, stream)) != TILEQ_OK) return st;
     }
     return TILEQ_OK;
   };

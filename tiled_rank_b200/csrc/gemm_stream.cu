@@ -1,20 +1,11 @@
 // Streaming grouped GEMM on warp-level tensor-core MMA (m16n8k16, fp16 in, fp32
-// accumulate) for the narrow products of the TileQ forward: the residual GEMMs
-// when an expert sees few tokens (decode), the column projection
-// z = Sigma*(V_n^T x), the down-side projection z' = Sigma*(V_n^T h), the
-// shared expert and the per-expert launches of the unfused path.  (A tcgen05
-// instruction costs the same tensor-core time for any N up to 256, so with a
-// handful of tokens per expert the warp-level MMA has the higher throughput.)
+// accumulate) for the narrow fp16 products of the TileQ forward: the column
+// projection z = Sigma*(V_n^T x), the down-side projection z' = Sigma*(V_n^T h),
+// the shared expert and the per-expert launches of the unfused path.  A is a
+// packed fp16 fragment matrix, streamed as one bulk copy per stage (32 KB per
+// projection); B rows are gathered by row index into the same stage.
 //
-//   AM_Q2   out[item][o] = sum_k s*(q - z)[o][k] * B[row(item)][k]
-//                          + sum_i U_m[o][i] * B[row(item)][ext + i]
-//           The 2-bit codes are stored per lane in the m16n8k16 A-fragment
-//           order (16 bytes per lane per 128x128 block, one shared-memory load
-//           per stage).  The exact (q - z) is decoded straight into fragment
-//           registers (one AND-OR with the fp16 exponent of 1024 and one FMA
-//           per pair); each 64/128-wide scale group accumulates into a fresh
-//           fp32 fragment that is folded in with its scale.
-//   AM_F16  A is a packed fp16 fragment matrix (V_n^T, shared expert, ...).
+//   out[item][o] = epi( sum_k A[o][k] * B[row(item)][k] )
 //
 // One producer warp feeds eight consumer warps through a ring of shared-memory
 // stages filled by bulk copies (cp.async.bulk) and handed over with mbarriers,
@@ -30,11 +21,12 @@
 namespace tileq {
 
 #ifdef TILEQ_TRACE
-// Debug builds only: clock64 time stamps of pipeline events of CTA 0.
-__device__ unsigned long long g_st_trace[6][1024];
+// Debug builds only: clock64 time stamps of pipeline events of CTA 0, kept
+// separately for one- and two-projection launches.
+__device__ unsigned long long g_st_trace[2][6][1024];
 #define ST_TRACE(kind, idx) \
   do {                      \
-    if (blockIdx.x == 0 && blockIdx.y == 0 && (idx) < 1024) g_st_trace[kind][idx] = clock64(); \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && (idx) < 1024) g_st_trace[NP - 1][kind][idx] = clock64(); \
   } while (0)
 extern "C" int tileq_debug_st_trace(unsigned long long *host) {
   return (int)cudaMemcpyFromSymbol(host, g_st_trace, sizeof(g_st_trace));
@@ -52,23 +44,18 @@ constexpr int THREADS = (W + 1) * 32;    // + one producer warp
 constexpr int BK = 128;                  // K per stage
 constexpr int BROW = BK + 8;             // padded smem row of B (halves)
 
-template <int AM, int NP, int BN>
+template <int NP, int BN>
 struct SCfg {
   static constexpr int NT = BN / 8;
-  static constexpr int A_WARP = (AM == AM_Q2) ? 0 : 8 * 32;  // uint4 per warp per projection (F16)
-  static constexpr int A_BYTES = (AM == AM_Q2) ? NP * 4096 : NP * W * A_WARP * 16;
-  static constexpr int SZ_BYTES = (AM == AM_Q2) ? NP * 2 * 512 : 0;
-  static constexpr int B_ONE = BN * BROW * 2;
-  static constexpr int B_BYTES = (AM == AM_Q2 ? NP : 1) * B_ONE;  // Q2: one B tile per projection for the extension
-  static constexpr int STAGE = A_BYTES + SZ_BYTES + B_BYTES;
-  static constexpr int BUDGET = (AM == AM_Q2 && BN <= 32) ? 74 * 1024 : 200 * 1024;
+  static constexpr int A_WARP = 8 * 32;  // uint4 per warp per projection and stage
+  static constexpr int A_BYTES = NP * W * A_WARP * 16;
+  static constexpr int B_BYTES = BN * BROW * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int BUDGET = 200 * 1024;
   static constexpr int STAGES_RAW = BUDGET / STAGE;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : (STAGES_RAW < 2 ? 2 : STAGES_RAW);
   static constexpr int BAR_OFF = STAGES * STAGE;
   static constexpr int SMEM = BAR_OFF + 2 * STAGES * 8 + 16;
-  // resident CTAs per SM the register budget is sized for (shared memory allows 3
-  // for the narrow 2-bit tiles, 1 for the fp16 ones)
-  static constexpr int MINB = (AM == AM_Q2) ? (NP * NT <= 2 ? 3 : 2) : 1;
   static constexpr int RPL = (BN + 31) / 32;  // B rows per producer lane
 };
 
@@ -102,10 +89,9 @@ __device__ __forceinline__ void epi_store(const GemmProblem &P, int item, int o,
   }
 }
 
-template <int AM, int NP, int BN>
-__global__ void __launch_bounds__(THREADS, SCfg<AM, NP, BN>::MINB)
-    gemm_stream_kernel(const __grid_constant__ GemmBatch batch) {
-  using C = SCfg<AM, NP, BN>;
+template <int NP, int BN>
+__global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_constant__ GemmBatch batch) {
+  using C = SCfg<NP, BN>;
   const GemmProblem &P = batch.p[blockIdx.y];
   extern __shared__ __align__(128) uint8_t smem[];
 
@@ -139,29 +125,19 @@ __global__ void __launch_bounds__(THREADS, SCfg<AM, NP, BN>::MINB)
   const int nkb = (P.d_in + BK - 1) / BK;
   const int per = (nkb + P.ksplit - 1) / P.ksplit;
   const int kb0 = min(nkb, split * per), kb1 = min(nkb, kb0 + per);
-  const int nmain = kb1 - kb0;
-  const int next = (AM == AM_Q2 && split == 0 && P.rank > 0) ? (P.rank + BK - 1) / BK : 0;
-  const int nst = nmain + next;
+  const int nst = kb1 - kb0;
   const int n128 = P.m_tiles;
-  const int g = P.group_size;
-  const int G = (AM == AM_Q2) ? P.d_in / g : 1;
-  const int gps = (AM == AM_Q2 && g == 64) ? 2 : 1;
 
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   uint64_t *empty = full + C::STAGES;
   int *sflag = reinterpret_cast<int *>(empty + C::STAGES);
   auto stage_a = [&](int st) { return smem + st * C::STAGE; };
-  auto stage_sz = [&](int st, int p) {
-    return reinterpret_cast<uint32_t *>(smem + st * C::STAGE + C::A_BYTES) + p * 2 * 128;
-  };
-  auto stage_b = [&](int st, int p) {
-    return reinterpret_cast<__half *>(smem + st * C::STAGE + C::A_BYTES + C::SZ_BYTES + p * C::B_ONE);
-  };
+  auto stage_b = [&](int st) { return reinterpret_cast<__half *>(smem + st * C::STAGE + C::A_BYTES); };
 
   // B rows past the end of K (ragged last stage) must read as zeros: clear once
   for (int i = threadIdx.x; i < C::STAGES * (C::B_BYTES / 16); i += THREADS) {
     const int st = i / (C::B_BYTES / 16), j = i % (C::B_BYTES / 16);
-    reinterpret_cast<uint4 *>(stage_b(st, 0))[j] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4 *>(stage_b(st))[j] = make_uint4(0, 0, 0, 0);
   }
   // order the generic zero stores before the bulk copies (async proxy) into the same buffers
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
@@ -202,48 +178,23 @@ __global__ void __launch_bounds__(THREADS, SCfg<AM, NP, BN>::MINB)
         if (!ok) break;
       }
       if (lane == 0) ST_TRACE(0, it);
-      if (it < nmain) {
-        const int kb = kb0 + it;
-        const int kvalid = min(BK, P.d_in - kb * BK);
-        uint32_t bytes = (uint32_t)C::A_BYTES + (uint32_t)nitems * kvalid * 2;
-        if (AM == AM_Q2) bytes += NP * gps * 512;
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
-        __syncwarp();
-        if (lane < NP) {
-          const int p = lane;
-          const size_t blk = ((size_t)ablk * n128 + ob) * nkb + kb;
-          if (AM == AM_Q2) {
-            bulk_g2s(stage_a(s) + p * 4096, reinterpret_cast<const uint8_t *>(P.a[p]) + blk * 4096, 4096, &full[s]);
-          } else {
-            bulk_g2s(stage_a(s) + p * W * C::A_WARP * 16, P.a[p] + blk * W * C::A_WARP, W * C::A_WARP * 16,
-                     &full[s]);
-          }
-        } else if (AM == AM_Q2 && lane < 2 * NP) {
-          const int p = lane - NP;
-          const size_t zoff = (((size_t)ablk * n128 + ob) * G + (kb * BK) / g) * 128;
-          bulk_g2s(stage_sz(s, p), P.sz[p] + zoff, gps * 512, &full[s]);
-        }
+      const int kb = kb0 + it;
+      const int kvalid = min(BK, P.d_in - kb * BK);
+      const uint32_t bytes = (uint32_t)C::A_BYTES + (uint32_t)nitems * kvalid * 2;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
+      __syncwarp();
+      if (lane < NP) {
+        const int p = lane;
+        const size_t blk = ((size_t)ablk * n128 + ob) * nkb + kb;
+        bulk_g2s(stage_a(s) + p * W * C::A_WARP * 16, P.a[p] + blk * W * C::A_WARP, W * C::A_WARP * 16,
+                 &full[s]);
+      }
 #pragma unroll
-        for (int j = 0; j < C::RPL; ++j) {
-          const int n = lane + 32 * j;
-          if (n < nitems)
-            bulk_g2s(stage_b(s, 0) + n * BROW, P.b + (size_t)brow[j] * P.ldb + (size_t)kb * BK, kvalid * 2,
-                     &full[s]);
-        }
-      } else {
-        // low-rank extension: B columns ext_col[p] + e*128 .. for each projection
-        const int e = it - nmain;
-        const int rlen = min(BK, P.rank - e * BK);
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)NP * nitems * rlen * 2);
-        __syncwarp();
-        for (int p = 0; p < NP; ++p)
-#pragma unroll
-          for (int j = 0; j < C::RPL; ++j) {
-            const int n = lane + 32 * j;
-            if (n < nitems)
-              bulk_g2s(stage_b(s, p) + n * BROW, P.b + (size_t)brow[j] * P.ldb + P.ext_col[p] + e * BK,
-                       rlen * 2, &full[s]);
-          }
+      for (int j = 0; j < C::RPL; ++j) {
+        const int n = lane + 32 * j;
+        if (n < nitems)
+          bulk_g2s(stage_b(s) + n * BROW, P.b + (size_t)brow[j] * P.ldb + (size_t)kb * BK, kvalid * 2,
+                   &full[s]);
       }
       issued = it + 1;
     }
@@ -255,133 +206,41 @@ __global__ void __launch_bounds__(THREADS, SCfg<AM, NP, BN>::MINB)
   } else {
     // ------------------------------------------------------------ consumer warps
     const int r0 = lane >> 2;
-    const int rw = warp * 16 + r0;  // fragment rows rw and rw + 8 of the 128-row block
 
-    // B fragments of k16 step ks for every projection (the extension reads each
-    // projection's own tile; otherwise all projections share tile 0)
-    auto load_b = [&](int s, int ks, bool ext, uint32_t (&bf)[NP][C::NT][2]) {
+    // One stage; FULL stages run all eight k16 steps without a bound check.
+    auto stage = [&](int s, int kvalid, auto full_tag) {
+      constexpr bool FULL = decltype(full_tag)::value;
+      const __half *bs = stage_b(s);
 #pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        if (p > 0 && !(AM == AM_Q2 && ext)) {
-#pragma unroll
-          for (int j = 0; j < C::NT; ++j) {
-            bf[p][j][0] = bf[0][j][0];
-            bf[p][j][1] = bf[0][j][1];
-          }
-          continue;
-        }
-        const __half *bs = stage_b(s, p);
+      for (int ks = 0; ks < BK / 16; ++ks) {
+        if (!FULL && ks * 16 >= kvalid) break;
+        uint32_t bf[C::NT][2];
         if constexpr (C::NT == 1) {
           uint32_t r[2];
           ldmatrix_x2(r, bs + (lane & 7) * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
-          bf[p][0][0] = r[0];
-          bf[p][0][1] = r[1];
+          bf[0][0] = r[0];
+          bf[0][1] = r[1];
         } else {
 #pragma unroll
           for (int j = 0; j < C::NT; j += 2) {
             uint32_t r[4];
             const int row = (j + (lane >> 4)) * 8 + (lane & 7);
             ldmatrix_x4(r, bs + row * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
-            bf[p][j][0] = r[0];
-            bf[p][j][1] = r[1];
-            bf[p][j + 1][0] = r[2];
-            bf[p][j + 1][1] = r[3];
+            bf[j][0] = r[0];
+            bf[j][1] = r[1];
+            bf[j + 1][0] = r[2];
+            bf[j + 1][1] = r[3];
           }
         }
-      }
-    };
-
-    // One stage of fp16 A (packed fragments, or the rows of U_m for the
-    // extension); FULL stages run all eight k16 steps without a bound check.
-    auto stage_f16 = [&](int s, int it, bool ext, int kvalid, auto full_tag) {
-      constexpr bool FULL = decltype(full_tag)::value;
-#pragma unroll
-      for (int ks = 0; ks < BK / 16; ++ks) {
-        if (!FULL && ks * 16 >= kvalid) break;
-        uint32_t bf[NP][C::NT][2];
-        load_b(s, ks, ext, bf);
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-          uint32_t af[4];
-          if (AM == AM_F16) {
-            const uint4 v =
-                reinterpret_cast<const uint4 *>(stage_a(s) + p * W * C::A_WARP * 16)[(warp * 8 + ks) * 32 + lane];
-            af[0] = v.x;
-            af[1] = v.y;
-            af[2] = v.z;
-            af[3] = v.w;
-          } else {
-            // A = rows of U_m (fp16), columns e*128 + ks*16 ..
-            const int e = it - nmain;
-            const __half *ur = P.u[p] + (((size_t)P.u_blk[p][grp] * n128 + ob) * 128 + rw) * P.rank + e * BK +
-                               ks * 16 + (lane & 3) * 2;
-            af[0] = __ldg(reinterpret_cast<const unsigned int *>(ur));
-            af[1] = __ldg(reinterpret_cast<const unsigned int *>(ur + 8 * P.rank));
-            af[2] = __ldg(reinterpret_cast<const unsigned int *>(ur + 8));
-            af[3] = __ldg(reinterpret_cast<const unsigned int *>(ur + 8 * P.rank + 8));
-          }
+          const uint4 v =
+              reinterpret_cast<const uint4 *>(stage_a(s) + p * W * C::A_WARP * 16)[(warp * 8 + ks) * 32 + lane];
+          const uint32_t af[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[p][j][0], bf[p][j][1]);
+          for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[j][0], bf[j][1]);
         }
       }
-    };
-
-    // One full stage of the 2-bit residual: 128 rows x 128 K per projection.
-    auto stage_q2 = [&](int s, int it) {
-      uint4 cw[NP];
-#pragma unroll
-      for (int p = 0; p < NP; ++p) cw[p] = reinterpret_cast<const uint4 *>(stage_a(s) + p * 4096)[warp * 32 + lane];
-      float part[NP][C::NT][4];
-      __half2 nz[NP][4];
-      float sc0[NP], sc8[NP];
-      // scale group of k16 step ks: 64-wide groups start a new one at ks 4
-      auto group_consts = [&](int ks) {
-#pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          const uint32_t *szs = stage_sz(s, p) + (ks == 4 ? 128 : 0);
-          const __half2 w0 = u32_as_h2(szs[rw]), w8 = u32_as_h2(szs[rw + 8]);
-          const __half2 z0 = __high2half2(w0), z8 = __high2half2(w8);
-          nz[p][0] = __hsub2(u32_as_h2(0xE400E400u), z0);  // -(1024 + z)
-          nz[p][1] = __hsub2(u32_as_h2(0xDC00DC00u), z8);  // -(256 + z)
-          nz[p][2] = __hsub2(u32_as_h2(0xD400D400u), z0);  // -(64 + z)
-          nz[p][3] = __hsub2(u32_as_h2(0xCC00CC00u), z8);  // -(16 + z)
-          sc0[p] = __low2float(w0);
-          sc8[p] = __low2float(w8);
-        }
-      };
-      auto fold = [&]() {
-#pragma unroll
-        for (int p = 0; p < NP; ++p)
-#pragma unroll
-          for (int j = 0; j < C::NT; ++j)
-#pragma unroll
-            for (int v = 0; v < 4; ++v) acc[p][j][v] = fmaf(v < 2 ? sc0[p] : sc8[p], part[p][j][v], acc[p][j][v]);
-      };
-      group_consts(0);
-#pragma unroll
-      for (int ks = 0; ks < BK / 16; ++ks) {
-        const bool gstart = ks == 0 || (g == 64 && ks == 4);
-        if (ks == 4 && g == 64) {
-          fold();
-          group_consts(4);
-        }
-        uint32_t bf[NP][C::NT][2];
-        load_b(s, ks, false, bf);
-#pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          const uint32_t word = (ks >> 1) == 0 ? cw[p].x : (ks >> 1) == 1 ? cw[p].y : (ks >> 1) == 2 ? cw[p].z : cw[p].w;
-          uint32_t af[4];
-          dequant_qz_k16((ks & 1) ? (word >> 8) : word, nz[p], af);
-          if (gstart) {
-#pragma unroll
-            for (int j = 0; j < C::NT; ++j) mma_f16_16816_z(part[p][j], af, bf[p][j][0], bf[p][j][1]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < C::NT; ++j) mma_f16_16816(part[p][j], af, bf[p][j][0], bf[p][j][1]);
-          }
-        }
-      }
-      fold();
     };
 
     for (int it = 0; it < nst; ++it) {
@@ -389,16 +248,11 @@ __global__ void __launch_bounds__(THREADS, SCfg<AM, NP, BN>::MINB)
       if (lane == 0 && (warp == 0 || warp == 7)) ST_TRACE(warp == 0 ? 1 : 3, it);
       if (!mbar_wait(&full[s], (it / C::STAGES) & 1, P.status)) break;
       if (lane == 0 && warp == 0) ST_TRACE(2, it);
-      const bool ext = it >= nmain;
-      if (AM == AM_Q2 && !ext) {
-        stage_q2(s, it);  // d_in is a multiple of 128: main stages are always full
-      } else {
-        const int kvalid = ext ? min(BK, P.rank - (it - nmain) * BK) : min(BK, P.d_in - (kb0 + it) * BK);
-        if (kvalid == BK)
-          stage_f16(s, it, ext, kvalid, std::true_type{});
-        else
-          stage_f16(s, it, ext, kvalid, std::false_type{});
-      }
+      const int kvalid = min(BK, P.d_in - (kb0 + it) * BK);
+      if (kvalid == BK)
+        stage(s, kvalid, std::true_type{});
+      else
+        stage(s, kvalid, std::false_type{});
       __syncwarp();
       if (lane == 0 && warp == 0) ST_TRACE(4, it);
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -467,10 +321,10 @@ __global__ void __launch_bounds__(THREADS, SCfg<AM, NP, BN>::MINB)
   if (threadIdx.x == 0) P.counters[tile_id] = 0;
 }
 
-template <int AM, int NP, int BN>
+template <int NP, int BN>
 cudaError_t launch_one(const GemmBatch &batch, int nprob, int n_tile_slots, cudaStream_t stream) {
-  using C = SCfg<AM, NP, BN>;
-  auto kern = gemm_stream_kernel<AM, NP, BN>;
+  using C = SCfg<NP, BN>;
+  auto kern = gemm_stream_kernel<NP, BN>;
   static bool configured = false;  // one attribute call per instantiation and process
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -491,40 +345,6 @@ cudaError_t launch_one(const GemmBatch &batch, int nprob, int n_tile_slots, cuda
   return cudaGetLastError();
 }
 
-template <int AM>
-cudaError_t launch_am(const GemmBatch &batch, int nprob, GemmShape shape, int slots, cudaStream_t stream) {
-  if constexpr (AM == AM_Q2) {
-    // the 2-bit path serves narrow tiles only (wider ones run on tcgen05)
-    switch (shape.bn * 4 + shape.np) {
-      case 8 * 4 + 1: return launch_one<AM, 1, 8>(batch, nprob, slots, stream);
-      case 16 * 4 + 1: return launch_one<AM, 1, 16>(batch, nprob, slots, stream);
-      case 32 * 4 + 1: return launch_one<AM, 1, 32>(batch, nprob, slots, stream);
-      case 8 * 4 + 2: return launch_one<AM, 2, 8>(batch, nprob, slots, stream);
-      case 16 * 4 + 2: return launch_one<AM, 2, 16>(batch, nprob, slots, stream);
-      case 32 * 4 + 2: return launch_one<AM, 2, 32>(batch, nprob, slots, stream);
-      default: return cudaErrorInvalidValue;
-    }
-  } else {
-  if (shape.np == 1) {
-    switch (shape.bn) {
-      case 8: return launch_one<AM, 1, 8>(batch, nprob, slots, stream);
-      case 16: return launch_one<AM, 1, 16>(batch, nprob, slots, stream);
-      case 32: return launch_one<AM, 1, 32>(batch, nprob, slots, stream);
-      case 64: return launch_one<AM, 1, 64>(batch, nprob, slots, stream);
-      case 128: return launch_one<AM, 1, 128>(batch, nprob, slots, stream);
-      default: return cudaErrorInvalidValue;
-    }
-  }
-  switch (shape.bn) {
-    case 8: return launch_one<AM, 2, 8>(batch, nprob, slots, stream);
-    case 16: return launch_one<AM, 2, 16>(batch, nprob, slots, stream);
-    case 32: return launch_one<AM, 2, 32>(batch, nprob, slots, stream);
-    case 64: return launch_one<AM, 2, 64>(batch, nprob, slots, stream);
-    default: return cudaErrorInvalidValue;
-  }
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_gemm(const GemmBatch &batch, int nprob, GemmShape shape, int n_tile_slots,
@@ -532,8 +352,23 @@ cudaError_t launch_gemm(const GemmBatch &batch, int nprob, GemmShape shape, int 
   if (n_tile_slots <= 0 || nprob <= 0) return cudaSuccess;
   for (int i = 0; i < nprob; ++i)
     if (batch.p[i].m_tiles <= 0 || batch.p[i].ksplit <= 0) return cudaErrorInvalidValue;
-  if (shape.am == AM_Q2) return launch_am<AM_Q2>(batch, nprob, shape, n_tile_slots, stream);
-  return launch_am<AM_F16>(batch, nprob, shape, n_tile_slots, stream);
+  if (shape.np == 1) {
+    switch (shape.bn) {
+      case 8: return launch_one<1, 8>(batch, nprob, n_tile_slots, stream);
+      case 16: return launch_one<1, 16>(batch, nprob, n_tile_slots, stream);
+      case 32: return launch_one<1, 32>(batch, nprob, n_tile_slots, stream);
+      case 64: return launch_one<1, 64>(batch, nprob, n_tile_slots, stream);
+      case 128: return launch_one<1, 128>(batch, nprob, n_tile_slots, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (shape.bn) {
+    case 8: return launch_one<2, 8>(batch, nprob, n_tile_slots, stream);
+    case 16: return launch_one<2, 16>(batch, nprob, n_tile_slots, stream);
+    case 32: return launch_one<2, 32>(batch, nprob, n_tile_slots, stream);
+    case 64: return launch_one<2, 64>(batch, nprob, n_tile_slots, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace tileq

@@ -46,18 +46,13 @@ struct PermuteArgs {
 };
 
 // ---------------------------------------------------------------- GEMM
-enum AMode { AM_Q2 = 0, AM_F16 = 1 };
 enum Epi { EPI_SWIGLU_H = 0, EPI_STORE_F32 = 1, EPI_STORE_F16 = 2, EPI_ACCUM_F32 = 3,
            EPI_STORE2_F32 = 4 };
 
-// One grouped GEMM  out[item][o] = sum_k A_g[o][k] * B[row(item)][k]  (+ a
-// low-rank K extension), items grouped by tiles (group, item0, nitems).  A rows
-// are output features; items are tokens / slots / (token, column) pairs.
-//   AM_F16: A = packed fp16 fragments [blk][R/128][K/128][8 warps][8 k16][32 lanes].
-//   AM_Q2:  A = 2-bit residual of expert `group` in the per-lane fragment
-//           layout ([8 warps][32 lanes] uint4 per 128x128 block, see
-//           pack_codes_kernel) with scale/zero words; the extension adds U_m
-//           (fp16 rows) times B columns ext_col[p] .. ext_col[p] + rank.
+// One grouped fp16 GEMM  out[item][o] = sum_k A_g[o][k] * B[row(item)][k],
+// items grouped by tiles (group, item0, nitems).  A rows are output features
+// (packed fp16 fragments [blk][R/128][K/128][8 warps][8 k16][32 lanes]); items
+// are tokens / slots / (token, column) pairs.
 struct GemmProblem {
   const int4 *tiles;
   const int *tile_count;
@@ -66,17 +61,11 @@ struct GemmProblem {
   const int *group_first_tile;
   int d_out, d_in;
   const uint4 *a[2];
-  const uint32_t *sz[2];
-  int group_size;
   int use_a_blk;
   int8_t a_blk[kMaxExperts];
   const __half *b;
   int ldb;
   const int *b_row;
-  int rank;
-  int ext_col[2];
-  const __half *u[2];     // [M][pad128(d_out)][rank] fp16
-  int8_t u_blk[2][kMaxExperts];
   int epi;
   void *out[2];
   int ldo;
@@ -98,7 +87,7 @@ struct GemmBatch {
 };
 
 struct GemmShape {
-  int am, np, bn;
+  int np, bn;
 };
 
 // Process-wide count of kernel launches issued by the library.
@@ -119,8 +108,10 @@ struct TcArgs {
   const int4 *tiles;
   const int *tile_count;
   int m_tiles, ksplit, d_out, d_in, group, rank;
+  int n_experts;             // experts (blocks) in codes / sz
   int ext_col[2];            // first B column of the K extension of projection p
-  const uint4 *codes[2];     // [K][d_out/128][d_in/128][4 slices][128 rows][8 B]
+  const uint4 *codes[2];     // tcgen05: [K][d_out/128][d_in/128][4 slices][128 rows][8 B]
+                             // warp MMA: [K][d_out/128][d_in/128][8 warps][32 lanes][16 B]
   const uint32_t *sz[2];     // [K][d_out/128][G][128 rows] {fp16 scale, fp16 zero}
   const __half *u[2];        // [M][pad128(d_out)][rank] fp16
   int8_t u_blk[2][kMaxExperts];
@@ -135,6 +126,11 @@ struct TcArgs {
 };
 
 cudaError_t launch_gemm_tc(const TcArgs &a, int np, int bn, int grid, cudaStream_t stream);
+
+// The same residual GEMM for narrow tiles (bn 8, 16 or 32) on warp-level MMA:
+// codes[p] in the per-lane fragment layout of pack_codes_kernel, B through
+// bmap (box 64 x bn); one CTA per (tile slot, 128-row block, K split).
+cudaError_t launch_gemm_q2(const TcArgs &a, int np, int bn, int n_tile_slots, cudaStream_t stream);
 int tc_smem_bytes(int np, int bn);
 
 // ---------------------------------------------------------------- misc
