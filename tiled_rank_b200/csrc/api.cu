@@ -97,8 +97,10 @@ size_t frag_bytes(int nblk, int R, int C, int kb) {
 
 // qw: codes in the row layout of the tcgen05 kernel; qf: the same codes in the
 // per-lane A-fragment order of the warp-MMA streaming kernel.
+// sig: Sigma repeated per grid column ([N][pad128(rank)] fp32), the column
+// scales of the projection onto all grid columns at once.
 struct PackedLayout {
-  size_t qw[3], qf[3], sz[3], uf[3], vf[3], sh[3], total;
+  size_t qw[3], qf[3], sz[3], uf[3], vf[3], sig[3], sh[3], total;
 };
 
 PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
@@ -116,6 +118,8 @@ PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
     if (q.rank > 0) off += align_up((size_t)L->M * pad128(q.d_out) * q.rank * 2);
     pl.vf[p] = off;
     if (q.rank > 0) off += align_up(frag_bytes(L->N, q.rank, q.d_in, 8));
+    pl.sig[p] = off;
+    if (q.rank > 0) off += align_up((size_t)L->N * pad128(q.rank) * 4);
   }
   for (int i = 0; i < 3; ++i) {
     pl.sh[i] = off;
@@ -173,11 +177,11 @@ int choose_bn_tc(long long avg) {
 
 // Split K until the grid covers about `per_sm` CTAs (or work items) per SM,
 // keeping >= 2 k-blocks per split.
-int choose_ksplit(long long ctas, int d_in, int per_sm = 4) {
+int choose_ksplit(long long ctas, int d_in, int per_sm = 4, int cap = 8) {
   const int nkb = cdiv(d_in, 128);
   int ks = (int)std::max(1LL, ((long long)per_sm * kNumSMs + ctas - 1) / std::max(1LL, ctas));
   ks = std::min(ks, std::max(1, nkb / 2));
-  return std::max(1, std::min(ks, 8));
+  return std::max(1, std::min(ks, cap));
 }
 
 struct Plan {
@@ -200,9 +204,6 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   pl.bn_main = use_tc ? choose_bn_tc(avg) : choose_bn(avg);
   pl.slots_main = cdiv(P, pl.bn_main) + L->K;
   const long long est_main = std::min(L->K, P) + P / pl.bn_main;
-  const int bn_z = choose_bn(P / std::max(1, L->N));
-  const int slots_z = cdiv(P, bn_z) + L->N;
-  const long long est_z = std::min(L->N, P) + P / bn_z;
   auto tc_plan = [&](int d_out, int d_in, int np) {
     GemmPlan g;
     g.tc = use_tc;
@@ -227,17 +228,19 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
       z.slots = pl.slots_main;
       z.m_tiles = cdiv(li.p[2].rank, 128);
       z.items = P;
-      z.ksplit = choose_ksplit(est_main * z.m_tiles, L->d_ff);
+      z.ksplit = choose_ksplit(est_main * z.m_tiles, L->d_ff, 4, 16);
       pl.zdown = z;
     }
   }
   if (q0.rank > 0) {
+    // z = Sigma*(V_n^T x_t) for every token and grid column: one dense product
+    // [T, d_in] x [d_in, N*rank] (TileQ paper, section 2.2: the projected [T, N, r] tensor)
     GemmPlan z;
-    z.bn = bn_z;
-    z.slots = slots_z;
-    z.m_tiles = cdiv(q0.rank, 128);
-    z.items = P;
-    z.ksplit = choose_ksplit(est_z * z.m_tiles * (L->kind == TILEQ_SWIGLU ? 2 : 1), q0.d_in);
+    z.bn = choose_bn(T);
+    z.slots = cdiv(T, z.bn);
+    z.m_tiles = L->N * (pad128(q0.rank) / 128);
+    z.items = T;
+    z.ksplit = choose_ksplit((long long)z.slots * z.m_tiles * (L->kind == TILEQ_SWIGLU ? 2 : 1), q0.d_in, 4, 16);
     pl.zproj = z;
   }
   if (L->shared_d_ff > 0) {
@@ -269,8 +272,8 @@ struct WsLayout {
       dest, tiles_main, tile_first, tile_counts, counters, part;
   int n_counters;
   size_t part_zstride;
-  size_t col_offsets[2], colpair_tok[2], zidx[2], tiles_z[2];
-  size_t row_offsets, rowpair_tok, rowpair_row, aidx;
+  size_t zidx[2];
+  size_t aidx;
   size_t x16, xext, hext, zc[2], zs, ybuf, hs, ys, g32, u32, zpe[2];
   int ld_x, ld_h;
   size_t total;
@@ -315,15 +318,7 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   for (const GemmPlan *g : {&pl.gateup, &pl.zdown, &pl.down, &pl.linear, &pl.sh_gu, &pl.sh_down})
     pf = std::max(pf, g->part_floats());
   w.part = take(pf * 4);
-  for (int z = 0; z < 2; ++z) {
-    w.col_offsets[z] = take((L->N + 1) * 4);
-    w.colpair_tok[z] = take(Pz * 4);
-    w.zidx[z] = take(Pz * 4);
-    w.tiles_z[z] = take((size_t)(pl.zproj.slots + 1) * 16);
-  }
-  w.row_offsets = take((L->M + 1) * 4);
-  w.rowpair_tok = take(Pz * 4);
-  w.rowpair_row = take(Pz * 4);
+  for (int z = 0; z < 2; ++z) w.zidx[z] = take(Pz * 4);
   w.aidx = take(Pz * 4);
   w.x16 = take((size_t)std::max(T, 1) * li.d_x * 2);
   const int rmax = std::max(std::max(li.p[0].rank, li.nproj > 1 ? li.p[1].rank : 0),
@@ -331,14 +326,14 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   if (L->kind == TILEQ_LINEAR) {
     w.ld_x = li.d_x + li.p[0].rank;
     w.xext = take(Pz * w.ld_x * 2);
-    w.zc[0] = take(Pz * li.p[0].rank * 2);
+    w.zc[0] = take((size_t)std::max(T, 1) * L->N * pad128(li.p[0].rank) * 2);
   } else {
     w.ld_x = L->d_model + 2 * li.p[0].rank;
     w.ld_h = L->d_ff + li.p[2].rank;
     w.xext = take(Pz * w.ld_x * 2);
     w.hext = take(Pz * w.ld_h * 2);
-    w.zc[0] = take(Pz * li.p[0].rank * 2);
-    w.zc[1] = take(Pz * li.p[1].rank * 2);
+    w.zc[0] = take((size_t)std::max(T, 1) * L->N * pad128(li.p[0].rank) * 2);
+    w.zc[1] = take((size_t)std::max(T, 1) * L->N * pad128(li.p[1].rank) * 2);
     w.zs = take(Pz * li.p[2].rank * 4);
     w.g32 = take(Pz * L->d_ff * 4);
     w.u32 = take(Pz * L->d_ff * 4);
@@ -517,7 +512,11 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   ra.zero = at<int>(ws, w.counters);
   ra.nzero = w.n_counters;
   mark(ST_BEGIN, stream);
-  route_kernel<<<nblocks(T, 8), 256, 0, stream>>>(ra);
+  // one warp per token for the top-k; enough blocks that the x conversion has
+  // at most four 16-byte chunks per thread
+  const long long xchunks = x ? (long long)T * li.d_x / 8 : 0;
+  const unsigned rblocks = std::max(nblocks(T, 8), std::min(nblocks(xchunks, 256 * 4), (unsigned)(8 * kNumSMs)));
+  route_kernel<<<rblocks, 256, 0, stream>>>(ra);
   TQ_LAUNCHED();
   mark(ST_ROUTE, stream);
 
@@ -529,7 +528,6 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   pa.M = L->M;
   pa.N = L->N;
   pa.bn = w.plan.bn_main;
-  pa.bn_z = w.plan.zproj.bn;
   pa.topk_idx = ra.topk_idx;
   pa.topk_w = ra.topk_w;
   pa.dest = at<int>(ws, w.dest);
@@ -544,16 +542,10 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   pa.n_zproj = n_zproj;
   for (int z = 0; z < 2; ++z) {
     if (z < n_zproj) std::memcpy(pa.n_of[z], li.p[zproj_ids[z]].n_of, kMaxExperts);
-    pa.col_offsets[z] = at<int>(ws, w.col_offsets[z]);
-    pa.colpair_tok[z] = at<int>(ws, w.colpair_tok[z]);
     pa.zidx[z] = at<int>(ws, w.zidx[z]);
-    pa.tiles_z[z] = at<int4>(ws, w.tiles_z[z]);
   }
   pa.row_proj = row_proj;
   if (row_proj >= 0) std::memcpy(pa.m_of_row, li.p[row_proj].m_of, kMaxExperts);
-  pa.row_offsets = at<int>(ws, w.row_offsets);
-  pa.rowpair_tok = at<int>(ws, w.rowpair_tok);
-  pa.rowpair_row = at<int>(ws, w.rowpair_row);
   pa.aidx = at<int>(ws, w.aidx);
   permute_kernel<<<1, 1024, 0, stream>>>(pa);
   TQ_LAUNCHED();
@@ -674,18 +666,16 @@ tileq_status run_zproj(const tileq_layer *layer, const LayerInfo &li, const Pack
     const ProjInfo &q = li.p[p];
     b.p[p] = problem(w.plan.zproj, ws, w);
     GemmProblem &z = b.p[p];
-    z.tiles = at<int4>(ws, w.tiles_z[p]);
-    z.tile_count = at<int>(ws, w.tile_counts) + 1 + p;
-    z.d_out = q.rank;
+    z.static_items = w.plan.T;
+    z.d_out = layer->N * pad128(q.rank);
     z.d_in = q.d_in;
     z.a[0] = at<uint4>(packed, pl.vf[p]);
     z.b = at<__half>(ws, w.x16);
     z.ldb = q.d_in;
-    z.b_row = at<int>(ws, w.colpair_tok[p]);
     z.epi = EPI_STORE_F16;
-    z.col_scale = layer->proj[p].Sigma;
+    z.col_scale = at<float>(packed, pl.sig[p]);
     z.out[0] = at<__half>(ws, w.zc[p]);
-    z.ldo = q.rank;
+    z.ldo = z.d_out;
     z.part = at<float>(ws, w.part) + (size_t)p * w.part_zstride;
   }
   return gemm(b, nz, 1, w.plan.zproj, stream);
@@ -759,6 +749,10 @@ tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_by
                                                              layer->N, q.rank, q.d_in, 8,
                                                              at<uint4>(packed, pl.vf[p]));
       TQ_LAUNCHED();
+      const int ns = layer->N * pad128(q.rank);
+      expand_sigma_kernel<<<nblocks(ns, 256), 256, 0, stream>>>(src.Sigma, q.rank, pad128(q.rank), layer->N,
+                                                                at<float>(packed, pl.sig[p]));
+      TQ_LAUNCHED();
     }
   }
   if (layer->shared_d_ff > 0) {
@@ -817,6 +811,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       LrAccArgs la = lracc_args(q, w, ws, top_k, xext, w.ld_x, q.d_in);
       la.zcol = at<__half>(ws, w.zc[0]);
       la.zidx = at<int>(ws, w.zidx[0]);
+      la.zld = pad128(q.rank);
       lr_accumulate_kernel<<<nblocks((long long)plan.P * q.rank, 256), 256, 0, stream>>>(la);
       TQ_LAUNCHED();
     } else {
@@ -857,6 +852,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       ga.z[1] = lr_gu ? at<__half>(ws, w.zc[1]) : nullptr;
       ga.zidx[0] = at<int>(ws, w.zidx[0]);
       ga.zidx[1] = at<int>(ws, w.zidx[1]);
+      ga.zld = pad128(qg.rank);
       ga.out = xext;
       const long long chunks = (long long)plan.P * (D / 8 + (lr_gu ? 2 * qg.rank / 8 : 0));
       gather_ext_kernel<<<nblocks(chunks, 256), 256, 0, stream>>>(ga);

@@ -48,8 +48,7 @@ namespace {
 
 constexpr int QW = 8;                    // consumer warps (16 rows each)
 constexpr int QTHREADS = (QW + 1) * 32;  // + one producer warp
-constexpr int QBLK = 128;                // K of one packed code block
-constexpr int QBK = 2 * QBLK;            // K per main stage (two blocks)
+constexpr int QBLK = 128;                // K of one packed code block; a main stage covers two
 
 template <int NP, int BN>
 struct QCfg {

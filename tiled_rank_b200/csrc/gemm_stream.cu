@@ -305,18 +305,41 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
   __syncthreads();
   if (!*sflag) return;
   __threadfence();
+  // four consecutive rows per thread and step (16-byte loads), all splits of
+  // one step issued before they are summed in split order
   const int ldp = n128 * kRowsPerCta;
-  for (int idx = threadIdx.x; idx < BN * kRowsPerCta; idx += THREADS) {
-    const int n = idx / kRowsPerCta;
-    const int o = ob * kRowsPerCta + idx % kRowsPerCta;
+  const size_t pstride = (size_t)P.part_items * ldp;  // one (split, projection) slab
+  for (int idx = threadIdx.x; idx < BN * (kRowsPerCta / 4); idx += THREADS) {
+    const int n = idx / (kRowsPerCta / 4);
+    const int o = ob * kRowsPerCta + (idx % (kRowsPerCta / 4)) * 4;
     if (n >= nitems || o >= P.d_out) continue;
     const int item = item0 + n;
-    float v[2] = {0.f, 0.f};
-    for (int sp = 0; sp < P.ksplit; ++sp)
+    const float *src = P.part + (size_t)item * ldp + o;
+    float4 v[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    for (int sp0 = 0; sp0 < P.ksplit; sp0 += 8) {
+      float4 t[8][NP];
 #pragma unroll
-      for (int p = 0; p < NP; ++p)
-        v[p] += __ldcg(&P.part[(((size_t)sp * NP + p) * P.part_items + item) * ldp + o]);
-    epi_store(P, item, o, v[0], v[NP - 1]);
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int p = 0; p < NP; ++p)
+          t[u][p] = sp0 + u < P.ksplit
+                        ? __ldcg(reinterpret_cast<const float4 *>(src + ((size_t)(sp0 + u) * NP + p) * pstride))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          v[p].x += t[u][p].x;
+          v[p].y += t[u][p].y;
+          v[p].z += t[u][p].z;
+          v[p].w += t[u][p].w;
+        }
+    }
+    const float r0v[4] = {v[0].x, v[0].y, v[0].z, v[0].w};
+    const float r1v[4] = {v[NP - 1].x, v[NP - 1].y, v[NP - 1].z, v[NP - 1].w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      if (o + c < P.d_out) epi_store(P, item, o + c, r0v[c], r1v[c]);
   }
   if (threadIdx.x == 0) P.counters[tile_id] = 0;
 }

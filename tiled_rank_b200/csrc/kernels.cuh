@@ -19,7 +19,7 @@ struct RouteArgs {
 };
 
 struct PermuteArgs {
-  int T, k, K, M, N, bn, bn_z;
+  int T, k, K, M, N, bn;
   const int32_t *topk_idx;
   const float *topk_w;
   int *dest;               // scratch [P]
@@ -30,19 +30,13 @@ struct PermuteArgs {
   float *slot_w;           // [P]
   int4 *tiles_main;        // [P/bn + K]
   int *tile_first_main;    // [K+1] first tile of each expert
-  int *tile_counts;        // [4]: main, z0, z1, rows
+  int *tile_counts;        // [1]: main tiles
   int n_zproj;             // 0, 1 or 2
   int8_t n_of[2][kMaxExperts];
-  int *col_offsets[2];     // [N+1]
-  int *colpair_tok[2];     // [P]
-  int *zidx[2];            // slot -> colpair
-  int4 *tiles_z[2];        // [P/bn + N]
-  int row_proj;            // -1 = no row sort
+  int *zidx[2];            // slot -> t*N + n (row of the projected [T, N, r] tensor)
+  int row_proj;            // -1 = no row designation
   int8_t m_of_row[kMaxExperts];
-  int *row_offsets;        // [M+1]
-  int *rowpair_tok;        // [P]
-  int *rowpair_row;        // [P]
-  int *aidx;               // slot -> rowpair (or -1 when not the designated pair)
+  int *aidx;               // slot -> 1 for the token's first slot in its grid row, else -1
 };
 
 // ---------------------------------------------------------------- GEMM
@@ -136,6 +130,7 @@ int tc_smem_bytes(int np, int bn);
 // ---------------------------------------------------------------- misc
 struct GatherExtArgs {
   int P, d, r, ld;            // x_ext[s] = [x16[tok(s)] (d) | z0[zidx0[s]] (r) | z1[zidx1[s]] (r)]
+  int zld;                    // row stride of z0 / z1 (elements)
   const int *slot_tok;
   const __half *x16;
   const __half *z[2];
@@ -149,15 +144,17 @@ struct GatherExtArgs {
 struct LrAccArgs {
   int P, k, r;
   const int32_t *sorted_pairs;
-  const int *aidx;         // slot -> rowpair (designated) or -1
+  const int *aidx;         // slot -> >= 0 for the token's first slot in its grid row, else -1
   const int32_t *topk_idx;
   const float *topk_w;
   int8_t m_of[kMaxExperts];
   const int *slot_of_pair;
-  // source: per-slot fp32 z' (weights already applied) or per-colpair fp16 z times w
+  // source: per-slot fp32 z' (weights already applied) or fp16 rows of the
+  // projected [T, N, r] tensor (stride zld) times w
   const float *zslot;
   const __half *zcol;
   const int *zidx;
+  int zld;
   __half *out;             // [P][ld], columns col .. col+r-1
   int ld, col;
 };
@@ -213,6 +210,7 @@ __global__ void pack_frag_kernel(const __nv_bfloat16 *src, long long bs, long lo
 // reading one slice of 32 consecutive rows touches 256 contiguous bytes.
 __global__ void pack_codes_tc_kernel(const uint32_t *codes, uint32_t *out, int K, int d_out, int d_in);
 // bf16 [nblk][R][C] -> fp16 [nblk][pad128(R)][C] (zero rows appended).
+__global__ void expand_sigma_kernel(const float *sigma, int r, int rp, int n, float *out);
 __global__ void pack_rows_f16_kernel(const __nv_bfloat16 *src, int nblk, int R, int C, __half *out);
 
 __host__ __device__ inline int pad128(int x) { return (x + 127) / 128 * 128; }

@@ -30,7 +30,7 @@ __global__ void lr_accumulate_kernel(LrAccArgs a) {
       if (a.zslot)
         acc += a.zslot[(size_t)slot * a.r + i];
       else
-        acc += a.topk_w[p] * __half2float(a.zcol[(size_t)a.zidx[slot] * a.r + i]);
+        acc += a.topk_w[p] * __half2float(a.zcol[(size_t)a.zidx[slot] * a.zld + i]);
     }
   }
   a.out[(size_t)s * a.ld + a.col + i] = __float2half_rn(acc);
@@ -48,7 +48,7 @@ __global__ void gather_ext_kernel(GatherExtArgs a) {
     v = reinterpret_cast<const uint4 *>(a.x16 + (size_t)a.slot_tok[s] * a.d)[c];
   } else {
     const int zc = c - a.d / 8, p = zc / (a.r / 8), cc = zc % (a.r / 8);
-    v = reinterpret_cast<const uint4 *>(a.z[p] + (size_t)a.zidx[p][s] * a.r)[cc];
+    v = reinterpret_cast<const uint4 *>(a.z[p] + (size_t)a.zidx[p][s] * a.zld)[cc];
   }
   reinterpret_cast<uint4 *>(a.out + (size_t)s * a.ld)[c] = v;
 }

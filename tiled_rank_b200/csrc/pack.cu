@@ -143,6 +143,15 @@ __global__ void pack_codes_tc_kernel(const uint32_t *codes, uint32_t *out, int K
   out[gid] = acc;
 }
 
+// Sigma [r] -> [n][rp] (rp = r rounded up to 128; zeros past r): the column
+// scales of the projection onto all n grid columns at once.
+__global__ void expand_sigma_kernel(const float *sigma, int r, int rp, int n, float *out) {
+  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= n * rp) return;
+  const int i = gid % rp;
+  out[gid] = i < r ? sigma[i] : 0.f;
+}
+
 __global__ void pack_rows_f16_kernel(const __nv_bfloat16 *src, int nblk, int R, int C, __half *out) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int Rp = pad128(R);

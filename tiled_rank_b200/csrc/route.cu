@@ -3,21 +3,46 @@
 // route_kernel    : one warp per token: exact top-k of the fp32 logits (descending,
 //                   equal logits -> lower expert id), softmax over the chosen
 //                   logits, and the bf16 -> fp16 conversion of the token's x row.
-// permute_kernel  : one CTA: deterministic stable counting sorts of the
-//                   (token, slot) pairs by expert, of the distinct (token, grid
-//                   column) pairs by column (one z = Sigma*(V_n^T x) per pair,
-//                   TileQ paper section 2.2 "project the input once"), and of the
-//                   distinct (token, grid row) pairs by row (the in-place
-//                   accumulation buffer of section 2.2), plus the GEMM tile tables.
+// permute_kernel  : one CTA: deterministic stable counting sort of the
+//                   (token, slot) pairs by expert and the GEMM tile table; per
+//                   slot, the row of the projected [T, N, r] tensor it reads
+//                   (TileQ paper, section 2.2) and whether it is the token's
+//                   first slot in its grid row (the in-place accumulation).
 #include "kernels.cuh"
 
 namespace tileq {
 
 __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long gthreads = (long long)gridDim.x * blockDim.x;
+  const int warp = (int)(gtid >> 5);
   const int lane = threadIdx.x & 31;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.nzero; i += gridDim.x * blockDim.x)
-    a.zero[i] = 0;
+  for (long long i = gtid; i < a.nzero; i += gthreads) a.zero[i] = 0;
+  // bf16 -> fp16 copy of x: every thread of the grid, four 16-byte chunks in flight
+  if (a.x != nullptr) {
+    const long long nchunk = (long long)a.T * (a.d_x / 8);
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.x);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.x16);
+    for (long long c0 = gtid; c0 < nchunk; c0 += 4 * gthreads) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const long long c = c0 + u * gthreads;
+        if (c < nchunk) v[u] = src[c];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const long long c = c0 + u * gthreads;
+        if (c >= nchunk) continue;
+        const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
+        uint4 o;
+        __half2 *h = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __float22half2_rn(__bfloat1622float2(b[i]));
+        dst[c] = o;
+      }
+    }
+  }
   if (warp >= a.T) return;
   const int t = warp;
   const float NEG = -INFINITY;
@@ -57,19 +82,6 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
         a.topk_idx[t * a.k + j] = sel_i[j];
         a.topk_w[t * a.k + j] = expf(sel_v[j] - sel_v[0]) / sum;
       }
-    }
-  }
-  if (a.x != nullptr) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d_x);
-    uint4 *dst = reinterpret_cast<uint4 *>(a.x16 + (size_t)t * a.d_x);
-    for (int c = lane; c < a.d_x / 8; c += 32) {
-      uint4 v = src[c];
-      const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v);
-      uint4 o;
-      __half2 *h = reinterpret_cast<__half2 *>(&o);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) h[i] = __float22half2_rn(__bfloat1622float2(b[i]));
-      dst[c] = o;
     }
   }
 }
@@ -186,69 +198,29 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
   cta_stable_sort(P, a.K, [&](int p) { return idx[p]; }, a.dest, a.expert_offsets, s);
   for (int p = threadIdx.x; p < P; p += blockDim.x) {
     const int slot = a.dest[p];
+    const int t = p / k, j = p - t * k;
+    const int e = idx[p];
     a.sorted_pairs[slot] = p;
     a.slot_of_pair[p] = slot;
-    a.slot_tok[slot] = p / k;
+    a.slot_tok[slot] = t;
     a.slot_w[slot] = a.topk_w[p];
+    // 2. the slot's row of the projected [T, N, r] tensor, z = Sigma*(V_n^T x_t),
+    //    per z projection (TileQ paper, section 2.2: project once, select by routing)
+    for (int zp = 0; zp < a.n_zproj; ++zp) a.zidx[zp][slot] = t * a.N + a.n_of[zp][e];
+    // 3. in-place accumulation per (token, grid row): the token's first slot in
+    //    grid row m carries a_{t,m}, the others carry zeros
+    if (a.row_proj >= 0) {
+      const int8_t *mrow = a.m_of_row;
+      const int r = mrow[e];
+      bool designated = true;
+      for (int jj = 0; jj < j; ++jj)
+        if (mrow[idx[t * k + jj]] == r) designated = false;
+      a.aidx[slot] = designated ? 1 : -1;
+    }
   }
   __syncthreads();
   build_tiles(a.expert_offsets, a.K, a.bn, a.tiles_main, a.tile_counts + 0, a.tile_first_main,
               scratch);
-
-  // 2. distinct (token, grid column) pairs by column, per z projection
-  for (int zp = 0; zp < a.n_zproj; ++zp) {
-    const int8_t *ncol = a.n_of[zp];
-    auto key = [&](int p) {
-      const int t = p / k, j = p - t * k;
-      const int c = ncol[idx[p]];
-      for (int jj = 0; jj < j; ++jj)
-        if (ncol[idx[t * k + jj]] == c) return -1;
-      return c;
-    };
-    cta_stable_sort(P, a.N, key, a.dest, a.col_offsets[zp], s);
-    for (int p = threadIdx.x; p < P; p += blockDim.x) {
-      const int t = p / k, j = p - t * k;
-      const int c = ncol[idx[p]];
-      int jd = j;
-      for (int jj = 0; jj < j; ++jj)
-        if (ncol[idx[t * k + jj]] == c) { jd = jj; break; }
-      const int cp = a.dest[t * k + jd];
-      if (jd == j) a.colpair_tok[zp][cp] = t;
-      a.zidx[zp][a.slot_of_pair[p]] = cp;
-    }
-    __syncthreads();
-    build_tiles(a.col_offsets[zp], a.N, a.bn_z, a.tiles_z[zp], a.tile_counts + 1 + zp, nullptr,
-                scratch);
-  }
-
-  // 3. distinct (token, grid row) pairs by row of the combined projection
-  if (a.row_proj >= 0) {
-    const int8_t *mrow = a.m_of_row;
-    auto key = [&](int p) {
-      const int t = p / k, j = p - t * k;
-      const int r = mrow[idx[p]];
-      for (int jj = 0; jj < j; ++jj)
-        if (mrow[idx[t * k + jj]] == r) return -1;
-      return r;
-    };
-    cta_stable_sort(P, a.M, key, a.dest, a.row_offsets, s);
-    for (int p = threadIdx.x; p < P; p += blockDim.x) {
-      const int t = p / k, j = p - t * k;
-      const int r = mrow[idx[p]];
-      bool designated = true;
-      for (int jj = 0; jj < j; ++jj)
-        if (mrow[idx[t * k + jj]] == r) { designated = false; break; }
-      const int slot = a.slot_of_pair[p];
-      if (designated) {
-        const int rp = a.dest[p];
-        a.rowpair_tok[rp] = t;
-        a.rowpair_row[rp] = r;
-        a.aidx[slot] = rp;
-      } else {
-        a.aidx[slot] = -1;
-      }
-    }
-  }
 }
 
 }  // namespace tileq
