@@ -24,6 +24,10 @@ int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 unsigned nblocks(long long n, int per) { return (unsigned)((n + per - 1) / per); }
 
 constexpr int kNumSMs = 148;
+#ifndef TILEQ_Q2_PER_SM
+#define TILEQ_Q2_PER_SM 4
+#endif
+constexpr int kQ2PerSm = TILEQ_Q2_PER_SM;  // split the narrow residual GEMM until ~this many CTAs per SM
 
 struct ProjInfo {
   int d_in, d_out, rank, group, G;
@@ -153,8 +157,11 @@ PePackedLayout pe_layout(const tileq_layer *L, const LayerInfo &li) {
 // ------------------------------------------------------------------ launch plan
 struct GemmPlan {
   int bn = 8, slots = 0, ksplit = 1, m_tiles = 1, np = 1, items = 0;
-  bool tc = false;  // residual GEMM on tcgen05 (wide tiles) rather than warp-level MMA
+  bool tc = false;       // residual GEMM on tcgen05 (wide tiles) rather than warp-level MMA
+  bool q2 = false;  // residual GEMM on warp-level MMA (narrow tiles)
   size_t part_floats() const {
+    // q2: one [np][bn][128] fp32 partial per (split, tile slot, row block)
+    if (q2) return ksplit > 1 ? (size_t)ksplit * slots * m_tiles * np * bn * kRowsPerCta : 0;
     return ksplit > 1 ? (size_t)ksplit * np * std::max(items, 1) * m_tiles * kRowsPerCta : 0;
   }
   int counters(int nprob) const { return ksplit > 1 ? nprob * slots * m_tiles : 0; }
@@ -213,7 +220,8 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
     g.np = np;
     g.items = P;
     // tcgen05: persistent CTAs walk (tile, row block, split) items; warp MMA: one CTA each
-    g.ksplit = choose_ksplit(est_main * g.m_tiles, d_in, use_tc ? 2 : 4);
+    g.q2 = !use_tc;
+    g.ksplit = choose_ksplit(est_main * g.m_tiles, d_in, use_tc ? 2 : kQ2PerSm);
     return g;
   };
   const ProjInfo &q0 = li.p[0];
@@ -279,7 +287,9 @@ struct WsLayout {
   size_t total;
 };
 
-WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k) {
+// route_only: the routing and permutation arrays alone (tileq_route and
+// tileq_route_static); no GEMM scratch, no activation matrices.
+WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool route_only = false) {
   WsLayout w{};
   w.plan = make_plan(L, li, T, k);
   const Plan &pl = w.plan;
@@ -303,6 +313,15 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   w.tiles_main = take((size_t)(pl.slots_main + 1) * 16);
   w.tile_first = take((L->K + 1) * 4);
   w.tile_counts = take(16);
+  if (route_only) {
+    w.n_counters = 0;
+    w.counters = take(16);
+    w.part = take(16);
+    for (int z = 0; z < 2; ++z) w.zidx[z] = take(Pz * 4);
+    w.aidx = take(Pz * 4);
+    w.total = off;
+    return w;
+  }
   int nc = 0;
   nc = std::max(nc, pl.zproj.counters(2));
   nc = std::max(nc, pl.gateup.counters(1));
@@ -1135,7 +1154,7 @@ tileq_status tileq_route(const float *router_logits, int T, int K, int top_k, ti
   LayerInfo li;
   tileq_status st = validate_layer(&L, &li, false);
   if (st != TILEQ_OK) return st;
-  const WsLayout w = ws_layout(&L, li, T, top_k);
+  const WsLayout w = ws_layout(&L, li, T, top_k, true);
   if (ws_bytes < w.total) return TILEQ_ERR_WORKSPACE;
   const int zids[2] = {0, 0};
   st = run_route_permute(&L, li, w, nullptr, T, router_logits, top_k, ws, 0, zids, -1, stream);
@@ -1247,7 +1266,7 @@ extern "C" tileq_status tileq_route_static(const float *router_logits, int T, in
   LayerInfo li;
   tileq_status st = validate_layer(&L, &li, false);
   if (st != TILEQ_OK) return st;
-  const WsLayout w = ws_layout(&L, li, T, top_k);
+  const WsLayout w = ws_layout(&L, li, T, top_k, true);
   if (w.total > kRouteStaticBytes) return TILEQ_ERR_UNSUPPORTED;
   void *ws = nullptr;
   if ((st = route_static_scratch(&ws)) != TILEQ_OK) return st;

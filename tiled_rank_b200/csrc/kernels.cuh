@@ -123,7 +123,9 @@ cudaError_t launch_gemm_tc(const TcArgs &a, int np, int bn, int grid, cudaStream
 
 // The same residual GEMM for narrow tiles (bn 8, 16 or 32) on warp-level MMA:
 // codes[p] in the per-lane fragment layout of pack_codes_kernel, B through
-// bmap (box 64 x bn); one CTA per (tile slot, 128-row block, K split).
+// bmap (box 64 x bn).  One CTA per (tile slot, 128-row block, K split); with
+// ksplit > 1, part holds one [np][bn][128] fp32 partial per CTA and counters
+// one zeroed arrival count per (tile slot, row block).
 cudaError_t launch_gemm_q2(const TcArgs &a, int np, int bn, int n_tile_slots, cudaStream_t stream);
 int tc_smem_bytes(int np, int bn);
 
