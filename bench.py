@@ -245,8 +245,16 @@ def main():
         dl.forward(xt, lg, out=out, ws=ws)
     torch.cuda.synchronize(dev)
 
-    # ---------------- timed region: K forwards, inputs resident
+    # ---------------- timed region: K forwards, inputs resident.  The library
+    # records one event at every stage boundary of every step on the launching
+    # stream (per-kernel device times for the roofline), set per step below.
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+            for _ in range(args.steps)]
+    for sev in sevs:  # create the CUDA events (first record) before the timed region
+        for e in sev:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
     n0 = tq.tileq_launch_count()
     barrier()
     torch.cuda.synchronize(dev)
@@ -254,15 +262,18 @@ def main():
         if flush:
             for i in range(args.steps):
                 flush_buf.zero_()
+                tq.tileq_set_stage_events(sevs[i])
                 ev[2 * i].record(stream)
                 dl.forward(xt, lg, out=out, ws=ws)
                 ev[2 * i + 1].record(stream)
         else:
             ev[0].record(stream)
             for i in range(args.steps):
+                tq.tileq_set_stage_events(sevs[i])
                 dl.forward(xt, lg, out=out, ws=ws)
             ev[1].record(stream)
         torch.cuda.synchronize(dev)
+    tq.tileq_set_stage_events(None)
     barrier()
     launches = tq.tileq_launch_count() - n0
     if flush:
@@ -276,24 +287,11 @@ def main():
     ms_per_step = ms / args.steps
     value = world * T * args.steps / (ms / 1000.0)
 
-    # ---------------- per-stage device times (separate pass, same stream)
-    # forwards are queued back to back (no host sync in between), one event set each
-    nprof = max(3, min(args.steps, 50))
-    sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
-            for _ in range(nprof)]
-    for _ in range(2):
-        dl.forward(xt, lg, out=out, ws=ws)
-    for i in range(nprof):
-        if flush:
-            flush_buf.zero_()
-        tq.tileq_set_stage_events(sevs[i])
-        dl.forward(xt, lg, out=out, ws=ws)
-    tq.tileq_set_stage_events(None)
-    torch.cuda.synchronize(dev)
+    # ---------------- per-stage device times of the timed steps
     stage_ms = np.zeros(len(STAGES))
     for sev in sevs:
         stage_ms += np.array([sev[i].elapsed_time(sev[i + 1]) for i in range(len(STAGES))])
-    stage_ms /= nprof
+    stage_ms /= len(sevs)
     stage_times = {n: round(float(t), 5) for n, t in zip(STAGES, stage_ms)}
 
     peaks = measured_peaks()
@@ -359,7 +357,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(layer, x_np, logits_np, n_tokens=1)
+        cpu = cpu_baseline(layer, x_np, logits_np, n_tokens=4)
 
     if rank == 0:
         line = {
