@@ -33,6 +33,23 @@ L2_BYTES = 126 * 2**20
 STAGES = ["route", "permute", "zproj", "gateup", "zdown", "rowacc", "residual", "shared", "combine"]
 
 
+def aggregate(ms_local, world, T, steps, device="cpu"):
+    """Whole-job figures of N replicas: the slowest rank's device time (max over
+    ranks, one all-reduce) and the tokens all ranks processed in that time."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms_local)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return ms, world * T * steps / (ms / 1000.0)
+
+
+def rank_seed(seed, rank):
+    """Each replica draws its own synthetic batch (same layer weights)."""
+    return seed + 1000 * rank
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -219,7 +236,7 @@ def main():
                                 device_id=dev)
 
     layer = synth.make_layer(cfg, seed=args.seed)
-    logits_np, x_np = synth.make_inputs(cfg, T, seed=args.seed + 1000 * rank)
+    logits_np, x_np = synth.make_inputs(cfg, T, seed=rank_seed(args.seed, rank))
     dl = tq.DeviceLayer(layer, dev)
     lg = torch.from_numpy(logits_np).to(dev)
     xt = torch.from_numpy(x_np.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -280,12 +297,8 @@ def main():
         ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps))
     else:
         ms = ev[0].elapsed_time(ev[1])
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms = float(ms_t.item())
+    ms, value = aggregate(ms, world, T, args.steps, dev)
     ms_per_step = ms / args.steps
-    value = world * T * args.steps / (ms / 1000.0)
 
     # ---------------- per-stage device times of the timed steps
     stage_ms = np.zeros(len(STAGES))
