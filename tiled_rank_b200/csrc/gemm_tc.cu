@@ -25,11 +25,12 @@
 namespace tileq {
 
 #ifdef TILEQ_TRACE
-// Debug builds only: clock64 time stamps of pipeline events of CTA 0.
-__device__ unsigned long long g_tc_trace[8][2048];
+// Debug builds only: clock64 time stamps of pipeline events of CTA 0, kept
+// separately for one- and two-projection launches.
+__device__ unsigned long long g_tc_trace[2][8][2048];
 #define TC_TRACE(kind, idx) \
   do {                      \
-    if (blockIdx.x == 0 && (idx) < 2048) g_tc_trace[kind][idx] = clock64(); \
+    if (blockIdx.x == 0 && (idx) < 2048) g_tc_trace[NP - 1][kind][idx] = clock64(); \
   } while (0)
 #else
 #define TC_TRACE(kind, idx) \
@@ -40,6 +41,10 @@ __device__ unsigned long long g_tc_trace[8][2048];
 namespace {
 
 constexpr int BK = 128;  // K per stage
+#ifndef TILEQ_TC_DQW128
+#define TILEQ_TC_DQW128 16
+#endif
+constexpr int kDqw128 = TILEQ_TC_DQW128;  // dequantising warps of the 128-item tiles
 
 template <int NP, int BN, int DQW>
 struct TcCfg {
@@ -48,7 +53,7 @@ struct TcCfg {
   static constexpr int CODES = NP * 128 * 32;         // packed codes of one stage (bytes)
   static constexpr int SZ = NP * 2 * 128 * 4;         // scale/zero words, up to 2 groups per stage
   static constexpr int BATOM = BN * 128;              // one 64-wide K atom of B (bytes)
-  static constexpr int B = NP * 2 * BATOM;            // main stage uses the first 2 atoms
+  static constexpr int B = 2 * BATOM;                 // 128 K (main) or 128 extension columns of one projection
   static constexpr int QSTAGE = ((CODES + SZ + B) + 1023) / 1024 * 1024;
   static constexpr int SQ_RAW = (200 * 1024) / QSTAGE;
   static constexpr int SQ = SQ_RAW > 8 ? 8 : (SQ_RAW < 2 ? 2 : SQ_RAW);
@@ -154,7 +159,9 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
   const int g = P.group;
   const int G = P.d_in / g;
   const int gps = g == 64 ? 2 : 1;
-  const int n_ext = P.rank > 0 ? (P.rank + BK - 1) / BK : 0;
+  // the K extension runs one projection at a time: n_ext1 stages of 128 columns each
+  const int n_ext1 = P.rank > 0 ? (P.rank + BK - 1) / BK : 0;
+  const int n_ext = NP * n_ext1;
   bool ok = true;
 
   auto decode = [&](int w, int &jt, int &ob, int &split) {
@@ -195,14 +202,12 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
             for (int a = 0; a < 2; ++a)
               tc::tma_load_2d(q_b(s) + a * C::BATOM, &P.bmap, kb * BK + a * 64, item0, &q_full[s]);
           } else {
-            const int e = st - nmain;
+            const int p = (st - nmain) / n_ext1, e = (st - nmain) % n_ext1;
             const int rlen = min(BK, P.rank - e * BK);
             const int natoms = (rlen + 63) / 64;
-            mbar_arrive_expect_tx(&q_full[s], NP * natoms * C::BATOM);
-            for (int p = 0; p < NP; ++p)
-              for (int a = 0; a < natoms; ++a)
-                tc::tma_load_2d(q_b(s) + (p * 2 + a) * C::BATOM, &P.bmap, P.ext_col[p] + e * BK + a * 64,
-                                item0, &q_full[s]);
+            mbar_arrive_expect_tx(&q_full[s], natoms * C::BATOM);
+            for (int a = 0; a < natoms; ++a)
+              tc::tma_load_2d(q_b(s) + a * C::BATOM, &P.bmap, P.ext_col[p] + e * BK + a * 64, item0, &q_full[s]);
           }
         }
       }
@@ -229,16 +234,28 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
           if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
           tc::fence_after();
           const bool ext = st >= nmain;
-          const int nk = ext ? (min(BK, P.rank - (st - nmain) * BK) + 15) / 16 : BK / 16;
-          const uint32_t b_base = smem_addr(q_b(s));
-          for (int p = 0; p < NP; ++p) {
-            const uint32_t d = tmem + p * BN;
-            const uint32_t a = tmem + C::ACC_COLS + sa * C::A_COLS + p * (BK / 2);
-            for (int kk = 0; kk < nk; ++kk) {
-              const int atom = (ext ? p * 2 : 0) + kk / 4;
-              const uint64_t bd = tc::sdesc_sw128(b_base + atom * C::BATOM + (kk % 4) * 32);
-              tc::mma_ts(d, a + kk * 8, bd, idesc, (first && kk == 0) ? 0u : 1u);
+          // an extension stage feeds one projection (pe); a main stage all of them
+          const int pe = ext ? (st - nmain) / n_ext1 : 0;
+          const int nk = ext ? (min(BK, P.rank - ((st - nmain) % n_ext1) * BK) + 15) / 16 : BK / 16;
+          // the issuing thread shares its SM sub-partition with dequantising
+          // warps: keep its instruction stream short (one descriptor per stage,
+          // constant offsets: the start-address field counts 16-byte units)
+          const uint64_t bd0 = tc::sdesc_sw128(smem_addr(q_b(s)));
+          const uint32_t a0 = tmem + C::ACC_COLS + sa * C::A_COLS;
+          if (!ext) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+              const uint32_t d = tmem + p * BN, a = a0 + p * (BK / 2);
+              tc::mma_ts(d, a, bd0, idesc, first ? 0u : 1u);
+#pragma unroll
+              for (int kk = 1; kk < BK / 16; ++kk)
+                tc::mma_ts(d, a + kk * 8, bd0 + (uint64_t)(((kk / 4) * C::BATOM + (kk % 4) * 32) >> 4), idesc, 1u);
             }
+          } else {
+            const uint32_t d = tmem + pe * BN, a = a0 + pe * (BK / 2);
+            for (int kk = 0; kk < nk; ++kk)
+              tc::mma_ts(d, a + kk * 8, bd0 + (uint64_t)(((kk / 4) * C::BATOM + (kk % 4) * 32) >> 4), idesc,
+                         (first && kk == 0) ? 0u : 1u);
           }
           first = false;
           TC_TRACE(5, qi);
@@ -270,16 +287,16 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
         const int s = qi % C::SQ, sa = ai % C::SA;
         if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
         if (dw == 0 && lane == 0) TC_TRACE(1, qi);
-        if (ai >= (uint32_t)C::SA && !(ok = mbar_wait(&a_empty[sa], ((ai / C::SA) - 1) & 1, P.status))) break;
-        if (dw == 0 && lane == 0) TC_TRACE(2, qi);
-        tc::fence_after();
         const bool ext = st >= nmain;
+        const int pe = ext ? (st - nmain) / n_ext1 : 0;  // the projection of an extension stage
+        // decode into registers first: this overlaps the wait for a free A stage
+        uint32_t vv[NP][C::KPW / 32][16];
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-          const uint32_t acol = tmem + lane_addr + C::ACC_COLS + sa * C::A_COLS + p * (BK / 2) + part * (C::KPW / 2);
+          if (ext && p != pe) continue;
 #pragma unroll
           for (int c = 0; c < C::KPW / 32; ++c) {   // chunks of 32 K elements = 16 columns
-            uint32_t v[16];
+            uint32_t *v = vv[p][c];
             const int k0 = part * C::KPW + c * 32;  // K offset within the stage
             if (!ext) {
               const uint32_t *cw = reinterpret_cast<const uint32_t *>(q_codes(s, p)) + ((k0 / 32) * 128 + row) * 2;
@@ -291,7 +308,7 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
               dq_word(cw[0], nz, s2, v);
               dq_word(cw[1], nz, s2, v + 8);
             } else {
-              const int e = st - nmain;
+              const int e = (st - nmain) % n_ext1;
               const int kg = e * BK + k0;          // column of U
               const int ub = P.u_blk[p][grp];
               const __half *ur = P.u[p] + (((size_t)ub * P.m_tiles + ob) * 128 + row) * P.rank;
@@ -305,18 +322,27 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
                 v[4 * j + 3] = q4.w;
               }
             }
-            tc::st16(acol + c * 16, v);
           }
+        }
+        // the codes of this stage are consumed: the producer may refill it once the MMAs are done too
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_empty[s]);
+        if (ai >= (uint32_t)C::SA && !(ok = mbar_wait(&a_empty[sa], ((ai / C::SA) - 1) & 1, P.status))) break;
+        if (dw == 0 && lane == 0) TC_TRACE(2, qi);
+        tc::fence_after();
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          if (ext && p != pe) continue;
+          const uint32_t acol = tmem + lane_addr + C::ACC_COLS + sa * C::A_COLS + p * (BK / 2) + part * (C::KPW / 2);
+#pragma unroll
+          for (int c = 0; c < C::KPW / 32; ++c) tc::st16(acol + c * 16, vv[p][c]);
         }
         if (dw == 0 && lane == 0) TC_TRACE(3, qi);
         tc::wait_st();
         if (dw == 0 && lane == 0) TC_TRACE(6, qi);
         tc::fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&a_full[sa]);
-          mbar_arrive(&q_empty[s]);
-        }
+        if (lane == 0) mbar_arrive(&a_full[sa]);
       }
       if (!ok) break;
 
@@ -420,7 +446,7 @@ cudaError_t launch_tc_bn(const TcArgs &a, int bn, int grid, cudaStream_t s) {
     case 16: return launch_tc_one<NP, 16, 16>(a, grid, s);
     case 32: return launch_tc_one<NP, 32, 16>(a, grid, s);
     case 64: return launch_tc_one<NP, 64, 16>(a, grid, s);
-    case 128: return launch_tc_one<NP, 128, 8>(a, grid, s);
+    case 128: return launch_tc_one<NP, 128, kDqw128>(a, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -439,14 +465,14 @@ int tc_smem_bytes(int np, int bn) {
       case 16: return TcCfg<1, 16, 16>::SMEM;
       case 32: return TcCfg<1, 32, 16>::SMEM;
       case 64: return TcCfg<1, 64, 16>::SMEM;
-      default: return TcCfg<1, 128, 8>::SMEM;
+      default: return TcCfg<1, 128, kDqw128>::SMEM;
     }
   }
   switch (bn) {
     case 16: return TcCfg<2, 16, 16>::SMEM;
     case 32: return TcCfg<2, 32, 16>::SMEM;
     case 64: return TcCfg<2, 64, 16>::SMEM;
-    default: return TcCfg<2, 128, 8>::SMEM;
+    default: return TcCfg<2, 128, kDqw128>::SMEM;
   }
 }
 
