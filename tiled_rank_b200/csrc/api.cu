@@ -158,13 +158,15 @@ PePackedLayout pe_layout(const tileq_layer *L, const LayerInfo &li) {
 struct GemmPlan {
   int bn = 8, slots = 0, ksplit = 1, m_tiles = 1, np = 1, items = 0;
   bool tc = false;       // residual GEMM on tcgen05 (wide tiles) rather than warp-level MMA
-  bool q2 = false;  // residual GEMM on warp-level MMA (narrow tiles)
+  bool q2 = false;       // residual GEMM on warp-level MMA (narrow tiles)
+  bool partial = false;  // K splits store their own partials (EPI_PARTIAL_F32); no reduction scratch
   size_t part_floats() const {
+    if (partial) return 0;
     // q2: one [np][bn][128] fp32 partial per (split, tile slot, row block)
     if (q2) return ksplit > 1 ? (size_t)ksplit * slots * m_tiles * np * bn * kRowsPerCta : 0;
     return ksplit > 1 ? (size_t)ksplit * np * std::max(items, 1) * m_tiles * kRowsPerCta : 0;
   }
-  int counters(int nprob) const { return ksplit > 1 ? nprob * slots * m_tiles : 0; }
+  int counters(int nprob) const { return ksplit > 1 && !partial ? nprob * slots * m_tiles : 0; }
 };
 
 int choose_bn(long long avg) {
@@ -237,6 +239,7 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
       z.m_tiles = cdiv(li.p[2].rank, 128);
       z.items = P;
       z.ksplit = choose_ksplit(est_main * z.m_tiles, L->d_ff, 4, 16);
+      z.partial = true;
       pl.zdown = z;
     }
   }
@@ -249,6 +252,7 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
     z.m_tiles = L->N * (pad128(q0.rank) / 128);
     z.items = T;
     z.ksplit = choose_ksplit((long long)z.slots * z.m_tiles * (L->kind == TILEQ_SWIGLU ? 2 : 1), q0.d_in, 4, 16);
+    z.partial = true;
     pl.zproj = z;
   }
   if (L->shared_d_ff > 0) {
@@ -345,15 +349,16 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool
   if (L->kind == TILEQ_LINEAR) {
     w.ld_x = li.d_x + li.p[0].rank;
     w.xext = take(Pz * w.ld_x * 2);
-    w.zc[0] = take((size_t)std::max(T, 1) * L->N * pad128(li.p[0].rank) * 2);
+    w.zc[0] = take((size_t)pl.zproj.ksplit * std::max(T, 1) * L->N * pad128(li.p[0].rank) * 4);
   } else {
     w.ld_x = L->d_model + 2 * li.p[0].rank;
     w.ld_h = L->d_ff + li.p[2].rank;
     w.xext = take(Pz * w.ld_x * 2);
     w.hext = take(Pz * w.ld_h * 2);
-    w.zc[0] = take((size_t)std::max(T, 1) * L->N * pad128(li.p[0].rank) * 2);
-    w.zc[1] = take((size_t)std::max(T, 1) * L->N * pad128(li.p[1].rank) * 2);
-    w.zs = take(Pz * li.p[2].rank * 4);
+    // z for all tokens and columns, and z' per slot: fp32 partials, one per K split
+    w.zc[0] = take((size_t)pl.zproj.ksplit * std::max(T, 1) * L->N * pad128(li.p[0].rank) * 4);
+    w.zc[1] = take((size_t)pl.zproj.ksplit * std::max(T, 1) * L->N * pad128(li.p[1].rank) * 4);
+    w.zs = take((size_t)pl.zdown.ksplit * Pz * li.p[2].rank * 4);
     w.g32 = take(Pz * L->d_ff * 4);
     w.u32 = take(Pz * L->d_ff * 4);
   }
@@ -439,6 +444,17 @@ bool make_map(CUtensorMap *m, const void *base, int rows, int cols, int ld, int 
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Read the B rows of an fp16 GEMM through a TMA tensor map when they are
+// contiguous per tile (no b_row gather): one box load per 64 K instead of one
+// bulk copy per row.
+bool tma_b(GemmProblem &p, int rows, int bn) {
+  p.tma_b = 0;
+  if (p.b_row || (reinterpret_cast<uintptr_t>(p.b) & 15) || (p.ldb * 2) % 16) return false;
+  if (!make_map(&p.bmap, p.b, rows, p.ldb, p.ldb, bn)) return false;
+  p.tma_b = 1;
+  return true;
 }
 
 // Tensor-core residual GEMM of projection p over the main tile table.
@@ -610,6 +626,7 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
     g.epi = EPI_SWIGLU_H;
     g.out[0] = at<__half>(ws, w.hs);
     g.ldo = Fs;
+    tma_b(g, T, w.plan.sh_gu.bn);
     if (gemm(b, 1, 2, w.plan.sh_gu, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
     b.p[0] = problem(w.plan.sh_down, ws, w);
     GemmProblem &d = b.p[0];
@@ -622,6 +639,7 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
     d.epi = EPI_STORE_F32;
     d.out[0] = at<float>(ws, w.ys);
     d.ldo = D;
+    tma_b(d, T, w.plan.sh_down.bn);
     if (gemm(b, 1, 1, w.plan.sh_down, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
     yshared = at<float>(ws, w.ys);
   }
@@ -691,10 +709,11 @@ tileq_status run_zproj(const tileq_layer *layer, const LayerInfo &li, const Pack
     z.a[0] = at<uint4>(packed, pl.vf[p]);
     z.b = at<__half>(ws, w.x16);
     z.ldb = q.d_in;
-    z.epi = EPI_STORE_F16;
+    z.epi = EPI_PARTIAL_F32;
     z.col_scale = at<float>(packed, pl.sig[p]);
-    z.out[0] = at<__half>(ws, w.zc[p]);
+    z.out[0] = at<float>(ws, w.zc[p]);
     z.ldo = z.d_out;
+    tma_b(z, w.plan.T, w.plan.zproj.bn);
     z.part = at<float>(ws, w.part) + (size_t)p * w.part_zstride;
   }
   return gemm(b, nz, 1, w.plan.zproj, stream);
@@ -828,9 +847,11 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       mark(ST_ZDOWN, stream);
       // a_{t,m} = sum_j w_j z_{t,n_j} over the token's experts in grid row m -> columns d_in..
       LrAccArgs la = lracc_args(q, w, ws, top_k, xext, w.ld_x, q.d_in);
-      la.zcol = at<__half>(ws, w.zc[0]);
+      la.zcol = at<float>(ws, w.zc[0]);
       la.zidx = at<int>(ws, w.zidx[0]);
       la.zld = pad128(q.rank);
+      la.zks = plan.zproj.ksplit;
+      la.zsplit = (long long)T * layer->N * pad128(q.rank);
       lr_accumulate_kernel<<<nblocks((long long)plan.P * q.rank, 256), 256, 0, stream>>>(la);
       TQ_LAUNCHED();
     } else {
@@ -867,8 +888,10 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       ga.ld = w.ld_x;
       ga.slot_tok = at<int>(ws, w.slot_tok);
       ga.x16 = at<__half>(ws, w.x16);
-      ga.z[0] = lr_gu ? at<__half>(ws, w.zc[0]) : nullptr;
-      ga.z[1] = lr_gu ? at<__half>(ws, w.zc[1]) : nullptr;
+      ga.z[0] = lr_gu ? at<float>(ws, w.zc[0]) : nullptr;
+      ga.z[1] = lr_gu ? at<float>(ws, w.zc[1]) : nullptr;
+      ga.zks = plan.zproj.ksplit;
+      ga.zsplit = (long long)T * layer->N * pad128(qg.rank);
       ga.zidx[0] = at<int>(ws, w.zidx[0]);
       ga.zidx[1] = at<int>(ws, w.zidx[1]);
       ga.zld = pad128(qg.rank);
@@ -910,14 +933,17 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       std::memcpy(z.a_blk, qd.n_of, kMaxExperts);
       z.b = hext;
       z.ldb = w.ld_h;
-      z.epi = EPI_STORE_F32;
+      z.epi = EPI_PARTIAL_F32;
       z.col_scale = layer->proj[2].Sigma;
       z.out[0] = at<float>(ws, w.zs);
       z.ldo = qd.rank;
+      tma_b(z, plan.P, plan.zdown.bn);
       if ((st = gemm(b, 1, 1, plan.zdown, stream)) != TILEQ_OK) return st;
       mark(ST_ZDOWN, stream);
       LrAccArgs la = lracc_args(qd, w, ws, top_k, hext, w.ld_h, F);
       la.zslot = at<float>(ws, w.zs);
+      la.zks = plan.zdown.ksplit;
+      la.zsplit = (long long)plan.P * qd.rank;
       lr_accumulate_kernel<<<nblocks((long long)plan.P * qd.rank, 256), 256, 0, stream>>>(la);
       TQ_LAUNCHED();
     } else {

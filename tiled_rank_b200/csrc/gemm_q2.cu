@@ -80,15 +80,13 @@ struct QCfg {
   static_assert(BOX % 1024 == 0 && STAGE % 1024 == 0, "swizzled boxes need 1024-byte alignment");
 };
 
-__device__ __forceinline__ void q2_store(const TcArgs &a, int item, int o, float v0, float v1) {
+// rs: the item's row scale (SwiGLU h), loaded by the caller ahead of the stores
+__device__ __forceinline__ void q2_store(const TcArgs &a, int item, int o, float v0, float v1, float rs) {
   const size_t idx = (size_t)item * a.ldo + o;
   switch (a.epi) {
-    case EPI_SWIGLU_H: {
-      float h = silu_f(v0) * v1;
-      if (a.row_scale) h *= a.row_scale[item];
-      reinterpret_cast<__half *>(a.out[0])[idx] = __float2half_rn(h);
+    case EPI_SWIGLU_H:
+      reinterpret_cast<__half *>(a.out[0])[idx] = __float2half_rn(silu_f(v0) * v1 * rs);
       break;
-    }
     case EPI_STORE_F16:
       reinterpret_cast<__half *>(a.out[0])[idx] = __float2half_rn(v0);
       break;
@@ -366,6 +364,12 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
 
   // ---------------------------------------------------------- epilogue / partials
   if (a.ksplit == 1) {
+    float rs[C::NT][2];  // row scales first (read-only path), then the stores
+#pragma unroll
+    for (int j = 0; j < C::NT; ++j)
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc)
+        rs[j][cc] = a.row_scale ? __ldg(a.row_scale + item0 + min(j * 8 + cq + cc, nitems - 1)) : 1.f;
 #pragma unroll
     for (int j = 0; j < C::NT; ++j)
 #pragma unroll
@@ -375,7 +379,7 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int n = j * 8 + cq + cc;
-          if (n < nitems) q2_store(a, item0 + n, o, acc[0][j][2 * h + cc], acc[NP - 1][j][2 * h + cc]);
+          if (n < nitems) q2_store(a, item0 + n, o, acc[0][j][2 * h + cc], acc[NP - 1][j][2 * h + cc], rs[j][cc]);
         }
       }
   } else {
@@ -435,9 +439,10 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
     }
     const float x0[4] = {v[0].x, v[0].y, v[0].z, v[0].w};
     const float x1[4] = {v[NP - 1].x, v[NP - 1].y, v[NP - 1].z, v[NP - 1].w};
+    const float rsn = a.row_scale ? __ldg(a.row_scale + item0 + n) : 1.f;
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4)
-      if (o + c4 < a.d_out) q2_store(a, item0 + n, o + c4, x0[c4], x1[c4]);
+      if (o + c4 < a.d_out) q2_store(a, item0 + n, o + c4, x0[c4], x1[c4], rsn);
   }
   if (threadIdx.x == 0) a.counters[unit] = 0;
   Q2_CTA_TIME(1);

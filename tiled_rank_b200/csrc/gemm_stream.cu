@@ -17,6 +17,7 @@
 #include <type_traits>
 
 #include "kernels.cuh"
+#include "tc.cuh"
 
 namespace tileq {
 
@@ -49,35 +50,36 @@ struct SCfg {
   static constexpr int NT = BN / 8;
   static constexpr int A_WARP = 8 * 32;  // uint4 per warp per projection and stage
   static constexpr int A_BYTES = NP * W * A_WARP * 16;
-  static constexpr int B_BYTES = BN * BROW * 2;
+  // B stage: padded rows (row copies) or two swizzled 64-wide TMA boxes; 1024-aligned
+  static constexpr int B_BYTES = (BN * BROW * 2 + 1023) / 1024 * 1024;
+  static constexpr int BOX = BN * 128;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int BUDGET = 200 * 1024;
   static constexpr int STAGES_RAW = BUDGET / STAGE;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : (STAGES_RAW < 2 ? 2 : STAGES_RAW);
   static constexpr int BAR_OFF = STAGES * STAGE;
-  static constexpr int SMEM = BAR_OFF + 2 * STAGES * 8 + 16;
+  static constexpr int SMEM = BAR_OFF + 2 * STAGES * 8 + 16 + 1024;  // + slack to align the base
   static constexpr int RPL = (BN + 31) / 32;  // B rows per producer lane
 };
 
-__device__ __forceinline__ float epi_value(const GemmProblem &P, int item, int o, float v0, float v1) {
-  if (P.epi == EPI_SWIGLU_H) {
-    float h = silu_f(v0) * v1;
-    if (P.row_scale) h *= P.row_scale[item];
-    return h;
-  }
-  if (P.col_scale) v0 *= P.col_scale[o];
-  return v0;
-}
-
-__device__ __forceinline__ void epi_store(const GemmProblem &P, int item, int o, float v0, float v1) {
+// Epilogue of one output element.  rs = the item's row scale (SwiGLU h), cs =
+// the output feature's column scale; callers load both once, ahead of the
+// stores (a load after a store to memory it may alias would wait for it).
+__device__ __forceinline__ void epi_store(const GemmProblem &P, int item, int o, float v0, float v1, int split,
+                                          float rs, float cs) {
   const size_t idx = (size_t)item * P.ldo + o;
   switch (P.epi) {
+    case EPI_PARTIAL_F32:
+      reinterpret_cast<float *>(P.out[0])[((size_t)split * P.part_items + item) * P.ldo + o] = v0 * cs;
+      break;
     case EPI_SWIGLU_H:
+      reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(silu_f(v0) * v1 * rs);
+      break;
     case EPI_STORE_F16:
-      reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(epi_value(P, item, o, v0, v1));
+      reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(v0 * cs);
       break;
     case EPI_STORE_F32:
-      reinterpret_cast<float *>(P.out[0])[idx] = epi_value(P, item, o, v0, v1);
+      reinterpret_cast<float *>(P.out[0])[idx] = v0 * cs;
       break;
     case EPI_ACCUM_F32:
       reinterpret_cast<float *>(P.out[0])[idx] += v0;
@@ -93,7 +95,8 @@ template <int NP, int BN>
 __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_constant__ GemmBatch batch) {
   using C = SCfg<NP, BN>;
   const GemmProblem &P = batch.p[blockIdx.y];
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
 
   int bid = blockIdx.x;
   const int split = bid % P.ksplit;
@@ -134,11 +137,13 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
   auto stage_a = [&](int st) { return smem + st * C::STAGE; };
   auto stage_b = [&](int st) { return reinterpret_cast<__half *>(smem + st * C::STAGE + C::A_BYTES); };
 
-  // B rows past the end of K (ragged last stage) must read as zeros: clear once
-  for (int i = threadIdx.x; i < C::STAGES * (C::B_BYTES / 16); i += THREADS) {
-    const int st = i / (C::B_BYTES / 16), j = i % (C::B_BYTES / 16);
-    reinterpret_cast<uint4 *>(stage_b(st))[j] = make_uint4(0, 0, 0, 0);
-  }
+  // row copies of a ragged last K stage leave the rest of the row as it was:
+  // it must read as zeros, so clear once (TMA boxes fill zeros themselves)
+  if (!P.tma_b && P.d_in % BK != 0)
+    for (int i = threadIdx.x; i < C::STAGES * (C::B_BYTES / 16); i += THREADS) {
+      const int st = i / (C::B_BYTES / 16), j = i % (C::B_BYTES / 16);
+      reinterpret_cast<uint4 *>(stage_b(st))[j] = make_uint4(0, 0, 0, 0);
+    }
   // order the generic zero stores before the bulk copies (async proxy) into the same buffers
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
   if (threadIdx.x == 0) {
@@ -180,7 +185,7 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
       if (lane == 0) ST_TRACE(0, it);
       const int kb = kb0 + it;
       const int kvalid = min(BK, P.d_in - kb * BK);
-      const uint32_t bytes = (uint32_t)C::A_BYTES + (uint32_t)nitems * kvalid * 2;
+      const uint32_t bytes = (uint32_t)C::A_BYTES + (P.tma_b ? 2u * C::BOX : (uint32_t)nitems * kvalid * 2);
       if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
       __syncwarp();
       if (lane < NP) {
@@ -189,12 +194,18 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
         bulk_g2s(stage_a(s) + p * W * C::A_WARP * 16, P.a[p] + blk * W * C::A_WARP, W * C::A_WARP * 16,
                  &full[s]);
       }
+      if (P.tma_b) {
+        if (lane >= 16 && lane < 18)
+          tc::tma_load_2d(reinterpret_cast<uint8_t *>(stage_b(s)) + (lane - 16) * C::BOX, &P.bmap,
+                          kb * BK + (lane - 16) * 64, item0, &full[s]);
+      } else {
 #pragma unroll
-      for (int j = 0; j < C::RPL; ++j) {
-        const int n = lane + 32 * j;
-        if (n < nitems)
-          bulk_g2s(stage_b(s) + n * BROW, P.b + (size_t)brow[j] * P.ldb + (size_t)kb * BK, kvalid * 2,
-                   &full[s]);
+        for (int j = 0; j < C::RPL; ++j) {
+          const int n = lane + 32 * j;
+          if (n < nitems)
+            bulk_g2s(stage_b(s) + n * BROW, P.b + (size_t)brow[j] * P.ldb + (size_t)kb * BK, kvalid * 2,
+                     &full[s]);
+        }
       }
       issued = it + 1;
     }
@@ -207,25 +218,37 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
     // ------------------------------------------------------------ consumer warps
     const int r0 = lane >> 2;
 
+    // B fragment addresses: padded rows (row copies) or swizzled 64-wide boxes
+    // (TMA; 16-byte chunk c of a box row sits at chunk c ^ (row % 8), row % 8 ==
+    // lane % 8).  address(j, ks) = rbase + j * rstep + tb[ks % 4] + (ks / 4) * kstep
+    const int hh = (lane >> 3) & 1;
+    const uint32_t rbase = P.tma_b ? (uint32_t)((C::NT == 1 ? 0 : (lane >> 4) * 8) + (lane & 7)) * 128
+                                   : (uint32_t)((C::NT == 1 ? 0 : (lane >> 4) * 8) + (lane & 7)) * BROW * 2 + hh * 16;
+    const uint32_t rstep = P.tma_b ? 8 * 128 : 8 * BROW * 2;
+    const uint32_t kstep = P.tma_b ? (uint32_t)C::BOX : 4 * 32;
+    uint32_t tb[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tb[q] = P.tma_b ? (uint32_t)(((q * 2 + hh) ^ (lane & 7)) << 4) : (uint32_t)q * 32;
+
     // One stage; FULL stages run all eight k16 steps without a bound check.
     auto stage = [&](int s, int kvalid, auto full_tag) {
       constexpr bool FULL = decltype(full_tag)::value;
-      const __half *bs = stage_b(s);
+      const uint32_t bs = smem_addr(stage_b(s)) + rbase;
 #pragma unroll
       for (int ks = 0; ks < BK / 16; ++ks) {
         if (!FULL && ks * 16 >= kvalid) break;
         uint32_t bf[C::NT][2];
+        const uint32_t ba = bs + tb[ks & 3] + (ks >> 2) * kstep;
         if constexpr (C::NT == 1) {
           uint32_t r[2];
-          ldmatrix_x2(r, bs + (lane & 7) * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
+          ldmatrix_x2_a(r, ba);
           bf[0][0] = r[0];
           bf[0][1] = r[1];
         } else {
 #pragma unroll
           for (int j = 0; j < C::NT; j += 2) {
             uint32_t r[4];
-            const int row = (j + (lane >> 4)) * 8 + (lane & 7);
-            ldmatrix_x4(r, bs + row * BROW + ks * 16 + ((lane >> 3) & 1) * 8);
+            ldmatrix_x4_a(r, ba + (j / 2) * 2 * rstep);
             bf[j][0] = r[0];
             bf[j][1] = r[1];
             bf[j + 1][0] = r[2];
@@ -260,7 +283,21 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
 
     // ---------------------------------------------------------- epilogue / partials
     const int cq = (lane & 3) * 2;
-    if (P.ksplit == 1) {
+    if (P.ksplit == 1 || P.epi == EPI_PARTIAL_F32) {
+      // scales first (read-only path), then the stores
+      float cs[2], rs[C::NT][2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int o = min(ob * kRowsPerCta + warp * 16 + r0 + 8 * h, P.d_out - 1);
+        cs[h] = P.col_scale ? __ldg(P.col_scale + o) : 1.f;
+      }
+#pragma unroll
+      for (int j = 0; j < C::NT; ++j)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int n = min(j * 8 + cq + cc, nitems - 1);
+          rs[j][cc] = P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f;
+        }
 #pragma unroll
       for (int j = 0; j < C::NT; ++j)
 #pragma unroll
@@ -271,7 +308,7 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
           for (int cc = 0; cc < 2; ++cc) {
             const int n = j * 8 + cq + cc;
             if (n >= nitems) continue;
-            epi_store(P, item0 + n, o, acc[0][j][2 * h + cc], acc[NP - 1][j][2 * h + cc]);
+            epi_store(P, item0 + n, o, acc[0][j][2 * h + cc], acc[NP - 1][j][2 * h + cc], split, rs[j][cc], cs[h]);
           }
         }
     } else {
@@ -294,7 +331,7 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
     }
   }
 
-  if (P.ksplit == 1) return;
+  if (P.ksplit == 1 || P.epi == EPI_PARTIAL_F32) return;
   // ------------------------------------------------------------ split-K: last CTA reduces
   __syncthreads();
   const int tile_id = blockIdx.y * (int)(gridDim.x / (P.ksplit)) + jt * P.m_tiles + ob;
@@ -339,7 +376,9 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
     const float r1v[4] = {v[NP - 1].x, v[NP - 1].y, v[NP - 1].z, v[NP - 1].w};
 #pragma unroll
     for (int c = 0; c < 4; ++c)
-      if (o + c < P.d_out) epi_store(P, item, o + c, r0v[c], r1v[c]);
+      if (o + c < P.d_out)
+        epi_store(P, item, o + c, r0v[c], r1v[c], 0, P.row_scale ? __ldg(P.row_scale + item) : 1.f,
+                  P.col_scale ? __ldg(P.col_scale + o + c) : 1.f);
   }
   if (threadIdx.x == 0) P.counters[tile_id] = 0;
 }

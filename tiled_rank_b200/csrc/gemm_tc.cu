@@ -69,19 +69,11 @@ struct TcCfg {
   static_assert(SA >= 2, "TMEM too small for two A stages");
 };
 
-__device__ __forceinline__ float tc_epi_value(const TcArgs &P, int item, int o, float v0, float v1) {
-  if (P.epi == EPI_SWIGLU_H) {
-    float h = silu_f(v0) * v1;
-    if (P.row_scale) h *= P.row_scale[item];
-    return h;
-  }
-  return v0;
-}
-
-__device__ __forceinline__ void tc_epi_store(const TcArgs &P, int item, int o, float v0, float v1) {
+// rs: the item's row scale (SwiGLU h), loaded by the caller ahead of the stores
+__device__ __forceinline__ void tc_epi_store(const TcArgs &P, int item, int o, float v0, float v1, float rs) {
   const size_t idx = (size_t)item * P.ldo + o;
   if (P.epi == EPI_SWIGLU_H) {
-    reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(tc_epi_value(P, item, o, v0, v1));
+    reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(silu_f(v0) * v1 * rs);
   } else if (P.epi == EPI_STORE2_F32) {
     reinterpret_cast<float *>(P.out[0])[idx] = v0;
     reinterpret_cast<float *>(P.out[1])[idx] = v1;
@@ -374,12 +366,16 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
           for (int p = 0; p < NP; ++p)
 #pragma unroll
             for (int i = 0; i < CH; ++i) v[p][i] = 0.f;
+        float rs[CH];  // row scales ahead of the stores
+#pragma unroll
+        for (int i = 0; i < CH; ++i)
+          rs[i] = P.row_scale ? __ldg(P.row_scale + item0 + min(part * COLS + c + i, nitems - 1)) : 1.f;
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
           const int n = part * COLS + c + i;
           if (n >= nitems) continue;
           if (P.ksplit == 1) {
-            if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i]);
+            if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i], rs[i]);
           } else {
 #pragma unroll
             for (int p = 0; p < NP; ++p)
@@ -407,7 +403,7 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
 #pragma unroll
               for (int p = 0; p < NP; ++p)
                 r[p] += __ldcg(&P.part[(((size_t)sp * NP + p) * P.part_items + item0 + n) * ldp + oo]);
-            tc_epi_store(P, item0 + n, oo, r[0], r[NP - 1]);
+            tc_epi_store(P, item0 + n, oo, r[0], r[NP - 1], P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f);
           }
           if (dw == 0 && lane == 0) P.counters[tile_id] = 0;
         }

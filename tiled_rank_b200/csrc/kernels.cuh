@@ -40,14 +40,21 @@ struct PermuteArgs {
 };
 
 // ---------------------------------------------------------------- GEMM
+// EPI_PARTIAL_F32: each K split stores its own fp32 partial (times col_scale) at
+// out[0][(split * part_items + item) * ldo + o]; the consumer sums the splits in
+// order, so no CTA waits for another and the result stays deterministic.
 enum Epi { EPI_SWIGLU_H = 0, EPI_STORE_F32 = 1, EPI_STORE_F16 = 2, EPI_ACCUM_F32 = 3,
-           EPI_STORE2_F32 = 4 };
+           EPI_STORE2_F32 = 4, EPI_PARTIAL_F32 = 5 };
 
 // One grouped fp16 GEMM  out[item][o] = sum_k A_g[o][k] * B[row(item)][k],
 // items grouped by tiles (group, item0, nitems).  A rows are output features
 // (packed fp16 fragments [blk][R/128][K/128][8 warps][8 k16][32 lanes]); items
 // are tokens / slots / (token, column) pairs.
 struct GemmProblem {
+  // tma_b != 0: B rows item0.. are contiguous and read through bmap (fp16,
+  // box 64 x bn, 128-byte swizzle) instead of one bulk copy per row (b_row)
+  alignas(64) CUtensorMap bmap;
+  int tma_b;
   const int4 *tiles;
   const int *tile_count;
   int static_items;       // tiles == nullptr: one group 0 holding this many items
@@ -133,9 +140,11 @@ int tc_smem_bytes(int np, int bn);
 struct GatherExtArgs {
   int P, d, r, ld;            // x_ext[s] = [x16[tok(s)] (d) | z0[zidx0[s]] (r) | z1[zidx1[s]] (r)]
   int zld;                    // row stride of z0 / z1 (elements)
+  int zks;                    // z0 / z1 are fp32 partials [zks][rows][zld], summed in order
+  long long zsplit;           // elements between two partials
   const int *slot_tok;
   const __half *x16;
-  const __half *z[2];
+  const float *z[2];
   const int *zidx[2];
   __half *out;
 };
@@ -151,12 +160,15 @@ struct LrAccArgs {
   const float *topk_w;
   int8_t m_of[kMaxExperts];
   const int *slot_of_pair;
-  // source: per-slot fp32 z' (weights already applied) or fp16 rows of the
-  // projected [T, N, r] tensor (stride zld) times w
+  // source: per-slot fp32 z' (weights already applied) or fp32 rows of the
+  // projected [T, N, r] tensor (stride zld) times w; both as zks partials
+  // (zsplit elements apart) summed in order
   const float *zslot;
-  const __half *zcol;
+  const float *zcol;
   const int *zidx;
   int zld;
+  int zks;
+  long long zsplit;
   __half *out;             // [P][ld], columns col .. col+r-1
   int ld, col;
 };

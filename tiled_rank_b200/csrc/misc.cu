@@ -27,10 +27,17 @@ __global__ void lr_accumulate_kernel(LrAccArgs a) {
       const int p = t * a.k + j;
       if (a.m_of[a.topk_idx[p]] != m) continue;
       const int slot = a.slot_of_pair[p];
-      if (a.zslot)
-        acc += a.zslot[(size_t)slot * a.r + i];
-      else
-        acc += a.topk_w[p] * __half2float(a.zcol[(size_t)a.zidx[slot] * a.zld + i]);
+      const float *z = a.zslot ? a.zslot + (size_t)slot * a.r + i : a.zcol + (size_t)a.zidx[slot] * a.zld + i;
+      float zz = 0.f;
+      for (int sp0 = 0; sp0 < a.zks; sp0 += 8) {
+        // eight splits' loads in flight, then summed in split order
+        float t[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) t[u] = sp0 + u < a.zks ? z[(size_t)(sp0 + u) * a.zsplit] : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) zz += t[u];
+      }
+      acc += a.zslot ? zz : a.topk_w[p] * zz;
     }
   }
   a.out[(size_t)s * a.ld + a.col + i] = __float2half_rn(acc);
@@ -47,8 +54,31 @@ __global__ void gather_ext_kernel(GatherExtArgs a) {
   if (c < a.d / 8) {
     v = reinterpret_cast<const uint4 *>(a.x16 + (size_t)a.slot_tok[s] * a.d)[c];
   } else {
+    // eight z values: the sum of the K-split partials in split order, to fp16
     const int zc = c - a.d / 8, p = zc / (a.r / 8), cc = zc % (a.r / 8);
-    v = reinterpret_cast<const uint4 *>(a.z[p] + (size_t)a.zidx[p][s] * a.zld)[cc];
+    const float *z = a.z[p] + (size_t)a.zidx[p][s] * a.zld + cc * 8;
+    float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+    for (int sp0 = 0; sp0 < a.zks; sp0 += 8) {
+      // eight splits' loads in flight, then summed in split order
+      float4 l[8], h[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool in = sp0 + u < a.zks;
+        const float4 *q = reinterpret_cast<const float4 *>(z + (size_t)(sp0 + u) * a.zsplit);
+        l[u] = in ? q[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+        h[u] = in ? q[1] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        lo.x += l[u].x; lo.y += l[u].y; lo.z += l[u].z; lo.w += l[u].w;
+        hi.x += h[u].x; hi.y += h[u].y; hi.z += h[u].z; hi.w += h[u].w;
+      }
+    }
+    __half2 *o = reinterpret_cast<__half2 *>(&v);
+    o[0] = __floats2half2_rn(lo.x, lo.y);
+    o[1] = __floats2half2_rn(lo.z, lo.w);
+    o[2] = __floats2half2_rn(hi.x, hi.y);
+    o[3] = __floats2half2_rn(hi.z, hi.w);
   }
   reinterpret_cast<uint4 *>(a.out + (size_t)s * a.ld)[c] = v;
 }
