@@ -107,6 +107,13 @@ TINY = [
     (synth.LINEAR, 5, 2, 3, 384, 144, 16, 128, 3, 0, 1),
     (synth.LINEAR, 9, 3, 3, 128, 64, 0, 64, 2, 0, 300),
     (synth.SWIGLU, 12, 3, 4, 128, 128, 16, 128, 1, 0, 513),
+    # largest rank, groups of 256, ~25 tokens per expert (32-wide warp-MMA tiles)
+    (synth.SWIGLU, 8, 2, 4, 256, 512, 256, 256, 2, 0, 100),
+    # groups of 384 spanning three 128-blocks, a 1 x K grid, tcgen05 tiles
+    (synth.SWIGLU, 6, 1, 6, 384, 768, 16, 384, 2, 0, 300),
+    # 64 experts on a 64 x 1 grid and on a 1 x 64 grid
+    (synth.LINEAR, 64, 64, 1, 128, 128, 16, 128, 2, 0, 64),
+    (synth.LINEAR, 64, 1, 64, 128, 128, 16, 64, 4, 0, 20),
 ]
 
 
