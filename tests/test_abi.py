@@ -83,8 +83,8 @@ def _host_layer(L, cfg, rank=None, grids=None):
 def test_packed_size_closed_form(L):
     """Packed bytes: codes 2 bits/weight in two layouts (tcgen05 rows, warp-MMA
     fragments), one u32 (scale, zero) per row and group, U blocks and V_n^T
-    blocks in fp16 with rows padded to multiples of 128, and Sigma repeated per
-    grid column in fp32."""
+    blocks in fp16 with rows padded to multiples of 128 (V_n^T twice: fragment
+    order and row-major), and Sigma repeated per grid column in fp32."""
     c, layer = _host_layer(L, 0)
     p = layer.projs[0]
     pad = lambda v: (v + 127) // 128 * 128  # noqa: E731
@@ -93,7 +93,7 @@ def test_packed_size_closed_form(L):
     for nbytes in (K * pad(p.d_out) * p.d_in // 4, K * pad(p.d_out) * p.d_in // 4,
                    K * pad(p.d_out) * (p.d_in // p.group) * 4,
                    M * pad(p.d_out) * p.rank * 2, N * pad(p.rank) * pad(p.d_in) * 2,
-                   N * pad(p.rank) * 4):
+                   N * pad(p.rank) * 4, N * pad(p.rank) * p.d_in * 2):
         expect += (nbytes + 255) // 256 * 256
     assert L.tileq_packed_size(c) == expect
 

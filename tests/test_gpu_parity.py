@@ -114,6 +114,9 @@ TINY = [
     # 64 experts on a 64 x 1 grid and on a 1 x 64 grid
     (synth.LINEAR, 64, 64, 1, 128, 128, 16, 128, 2, 0, 64),
     (synth.LINEAR, 64, 1, 64, 128, 128, 16, 64, 4, 0, 20),
+    # long batches: z, z' and the shared expert on tcgen05 as well
+    (synth.SWIGLU, 8, 2, 4, 128, 256, 48, 128, 2, 256, 300),
+    (synth.LINEAR, 5, 2, 3, 384, 144, 16, 128, 3, 0, 300),
 ]
 
 

@@ -27,7 +27,8 @@ constexpr int kNumSMs = 148;
 #ifndef TILEQ_Q2_PER_SM
 #define TILEQ_Q2_PER_SM 4
 #endif
-constexpr int kQ2PerSm = TILEQ_Q2_PER_SM;  // split the narrow residual GEMM until ~this many CTAs per SM
+constexpr int kQ2PerSm = TILEQ_Q2_PER_SM;
+constexpr int kTcMinTokens = 256;  // dense fp16 products (z, shared expert) move to tcgen05 from here  // split the narrow residual GEMM until ~this many CTAs per SM
 
 struct ProjInfo {
   int d_in, d_out, rank, group, G;
@@ -102,9 +103,12 @@ size_t frag_bytes(int nblk, int R, int C, int kb) {
 // qw: codes in the row layout of the tcgen05 kernel; qf: the same codes in the
 // per-lane A-fragment order of the warp-MMA streaming kernel.
 // sig: Sigma repeated per grid column ([N][pad128(rank)] fp32), the column
-// scales of the projection onto all grid columns at once.
+// scales of the projection onto all grid columns at once.  vr: V_n^T rows in
+// fp16, row-major [N][pad128(rank)][d_in], and shr: the shared expert's
+// weights row-major fp16 [pad128(rows)][cols] (the A operands of the tcgen05
+// kernel; vf / sh hold the same values in warp-MMA fragment order).
 struct PackedLayout {
-  size_t qw[3], qf[3], sz[3], uf[3], vf[3], sig[3], sh[3], total;
+  size_t qw[3], qf[3], sz[3], uf[3], vf[3], sig[3], vr[3], sh[3], shr[3], total;
 };
 
 PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
@@ -124,12 +128,17 @@ PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
     if (q.rank > 0) off += align_up(frag_bytes(L->N, q.rank, q.d_in, 8));
     pl.sig[p] = off;
     if (q.rank > 0) off += align_up((size_t)L->N * pad128(q.rank) * 4);
+    pl.vr[p] = off;
+    if (q.rank > 0) off += align_up((size_t)L->N * pad128(q.rank) * q.d_in * 2);
   }
   for (int i = 0; i < 3; ++i) {
     pl.sh[i] = off;
+    pl.shr[i] = off;
     if (L->shared_d_ff > 0) {
       const int R = i < 2 ? L->shared_d_ff : L->d_model, C = i < 2 ? L->d_model : L->shared_d_ff;
       off += align_up(frag_bytes(1, R, C, 8));
+      pl.shr[i] = off;
+      off += align_up((size_t)pad128(R) * C * 2);
     }
   }
   pl.total = off;
@@ -240,6 +249,10 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
       z.items = P;
       z.ksplit = choose_ksplit(est_main * z.m_tiles, L->d_ff, 4, 16);
       z.partial = true;
+      if (use_tc) {  // wide tiles: the same product on tcgen05, no K split
+        z.tc = true;
+        z.ksplit = 1;
+      }
       pl.zdown = z;
     }
   }
@@ -253,6 +266,12 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
     z.items = T;
     z.ksplit = choose_ksplit((long long)z.slots * z.m_tiles * (L->kind == TILEQ_SWIGLU ? 2 : 1), q0.d_in, 4, 16);
     z.partial = true;
+    if (T >= kTcMinTokens) {  // long batches: tcgen05, 128-token tiles, no K split
+      z.tc = true;
+      z.bn = choose_bn_tc(T);
+      z.slots = cdiv(T, z.bn);
+      z.ksplit = 1;
+    }
     pl.zproj = z;
   }
   if (L->shared_d_ff > 0) {
@@ -269,6 +288,14 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
     g.m_tiles = cdiv(L->d_model, 128);
     g.ksplit = choose_ksplit((long long)g.slots * g.m_tiles, L->shared_d_ff);
     pl.sh_down = g;
+    if (T >= kTcMinTokens) {  // long batches: both products on tcgen05, no K split
+      for (GemmPlan *q : {&pl.sh_gu, &pl.sh_down}) {
+        q->tc = true;
+        q->bn = choose_bn_tc(T);
+        q->slots = cdiv(T, q->bn);
+        q->ksplit = 1;
+      }
+    }
   }
   // unfused per-expert launches: one expert per launch, grid sized for T slots, no split
   pl.pe.bn = pl.bn_main;
@@ -495,6 +522,56 @@ tileq_status tc_launch(const TcArgs &a, int np, const GemmPlan &g, cudaStream_t 
   return launch_gemm_tc(a, np, g.bn, kNumSMs, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
 }
 
+// A dense fp16 product on tcgen05: A row-major fp16 (arow[p], lda), B the fp16
+// rows [brows][ldb] read by TMA, items either a tile table or 0..static_items-1.
+struct TcF16 {
+  int np = 1;
+  const __half *arow[2] = {nullptr, nullptr};
+  int lda = 0, d_out = 0, d_in = 0;
+  const int4 *tiles = nullptr;
+  const int *tile_count = nullptr;
+  int static_items = 0;
+  const int8_t *a_blk = nullptr;
+  const __half *b = nullptr;
+  int brows = 0, ldb = 0;
+  int epi = EPI_STORE_F32;
+  void *out[2] = {nullptr, nullptr};
+  int ldo = 0;
+  const float *col_scale[2] = {nullptr, nullptr};
+  const float *row_scale = nullptr;
+};
+
+tileq_status tc_f16(const TcF16 &f, const GemmPlan &g, void *ws, const WsLayout &w, cudaStream_t stream) {
+  TcArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if (!make_map(&a.bmap, f.b, f.brows, f.ldb, f.ldb, g.bn)) return TILEQ_ERR_CUDA;
+  a.tiles = f.tiles;
+  a.tile_count = f.tile_count;
+  a.static_items = f.static_items;
+  a.m_tiles = cdiv(f.d_out, 128);
+  a.ksplit = 1;
+  a.d_out = f.d_out;
+  a.d_in = f.d_in;
+  a.a_f16 = 1;
+  a.arow[0] = f.arow[0];
+  a.arow[1] = f.arow[1];
+  a.lda = f.lda;
+  a.use_a_blk = f.a_blk != nullptr;
+  if (f.a_blk) std::memcpy(a.a_blk, f.a_blk, kMaxExperts);
+  a.epi = f.epi;
+  a.out[0] = f.out[0];
+  a.out[1] = f.out[1];
+  a.ldo = f.ldo;
+  a.row_scale = f.row_scale;
+  a.col_scale[0] = f.col_scale[0];
+  a.col_scale[1] = f.col_scale[1];
+  a.part = at<float>(ws, w.part);
+  a.part_items = 1;
+  a.counters = at<int>(ws, w.counters);
+  a.status = at<int>(ws, w.status);
+  return launch_gemm_tc(a, f.np, g.bn, kNumSMs, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
+}
+
 // One residual projection (or the gate/up pair) over the main tile table:
 //   out = epi( s*(q-z) B[:, 0:d_in]  +  U_m B[:, ext .. ext + rank] )
 struct Residual {
@@ -611,7 +688,38 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
                                     const PackedLayout &pl, const WsLayout &w, const void *packed,
                                     void *ws, int T, int top_k, void *out, cudaStream_t stream) {
   const float *yshared = nullptr;
-  if (L->shared_d_ff > 0) {
+  if (L->shared_d_ff > 0 && w.plan.sh_gu.tc) {
+    const int Fs = L->shared_d_ff, D = L->d_model;
+    TcF16 f;
+    f.np = 2;
+    f.arow[0] = at<__half>(packed, pl.shr[0]);
+    f.arow[1] = at<__half>(packed, pl.shr[1]);
+    f.lda = D;
+    f.d_out = Fs;
+    f.d_in = D;
+    f.static_items = T;
+    f.b = at<__half>(ws, w.x16);
+    f.brows = T;
+    f.ldb = D;
+    f.epi = EPI_SWIGLU_H;
+    f.out[0] = at<__half>(ws, w.hs);
+    f.ldo = Fs;
+    if (tc_f16(f, w.plan.sh_gu, ws, w, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
+    TcF16 d;
+    d.arow[0] = at<__half>(packed, pl.shr[2]);
+    d.lda = Fs;
+    d.d_out = D;
+    d.d_in = Fs;
+    d.static_items = T;
+    d.b = at<__half>(ws, w.hs);
+    d.brows = T;
+    d.ldb = Fs;
+    d.epi = EPI_STORE_F32;
+    d.out[0] = at<float>(ws, w.ys);
+    d.ldo = D;
+    if (tc_f16(d, w.plan.sh_down, ws, w, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
+    yshared = at<float>(ws, w.ys);
+  } else if (L->shared_d_ff > 0) {
     const int Fs = L->shared_d_ff, D = L->d_model;
     GemmBatch b;
     b.p[0] = problem(w.plan.sh_gu, ws, w);
@@ -698,6 +806,27 @@ LrAccArgs lracc_args(const ProjInfo &q, const WsLayout &w, void *ws, int top_k, 
 tileq_status run_zproj(const tileq_layer *layer, const LayerInfo &li, const PackedLayout &pl,
                        const void *packed, const WsLayout &w, void *ws, int nz,
                        cudaStream_t stream) {
+  if (w.plan.zproj.tc) {
+    // all projections of the launch in one tcgen05 pass (gate and up share B = x)
+    const ProjInfo &q = li.p[0];
+    TcF16 f;
+    f.np = nz;
+    for (int p = 0; p < nz; ++p) {
+      f.arow[p] = at<__half>(packed, pl.vr[p]);
+      f.out[p] = at<float>(ws, w.zc[p]);
+      f.col_scale[p] = at<float>(packed, pl.sig[p]);
+    }
+    f.lda = q.d_in;
+    f.d_out = layer->N * pad128(q.rank);
+    f.d_in = q.d_in;
+    f.static_items = w.plan.T;
+    f.b = at<__half>(ws, w.x16);
+    f.brows = w.plan.T;
+    f.ldb = q.d_in;
+    f.epi = nz == 2 ? EPI_STORE2_F32 : EPI_STORE_F32;
+    f.ldo = f.d_out;
+    return tc_f16(f, w.plan.zproj, ws, w, stream);
+  }
   GemmBatch b;
   for (int p = 0; p < nz; ++p) {
     const ProjInfo &q = li.p[p];
@@ -791,6 +920,10 @@ tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_by
       expand_sigma_kernel<<<nblocks(ns, 256), 256, 0, stream>>>(src.Sigma, q.rank, pad128(q.rank), layer->N,
                                                                 at<float>(packed, pl.sig[p]));
       TQ_LAUNCHED();
+      n = (long long)layer->N * pad128(q.rank) * q.d_in;
+      pack_vt_rows_kernel<<<nblocks(n, 256), 256, 0, stream>>>(V, layer->N, q.rank, q.d_in,
+                                                                 at<__half>(packed, pl.vr[p]));
+      TQ_LAUNCHED();
     }
   }
   if (layer->shared_d_ff > 0) {
@@ -801,6 +934,10 @@ tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_by
       pack_frag_kernel<<<nblocks(n, 256), 256, 0, stream>>>(
           static_cast<const __nv_bfloat16 *>(layer->shared_w[i]), 0, Cc, 1, 1, R, Cc, 8,
           at<uint4>(packed, pl.sh[i]));
+      TQ_LAUNCHED();
+      const long long nr = (long long)pad128(R) * Cc;
+      pack_rows_f16_kernel<<<nblocks(nr, 256), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16 *>(layer->shared_w[i]), 1, R, Cc, at<__half>(packed, pl.shr[i]));
       TQ_LAUNCHED();
     }
   }
@@ -921,6 +1058,23 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     if (lr_d) {
       // z'_slot = Sigma * (V_n^T h_slot), then the in-place accumulation
       // a_{t,m} = sum of the token's z' over its experts in grid row m -> columns F..
+      if (plan.zdown.tc) {
+        TcF16 f;
+        f.arow[0] = at<__half>(packed, pl.vr[2]);
+        f.lda = F;
+        f.d_out = qd.rank;
+        f.d_in = F;
+        f.tiles = at<int4>(ws, w.tiles_main);
+        f.tile_count = at<int>(ws, w.tile_counts);
+        f.a_blk = qd.n_of;
+        f.b = hext;
+        f.brows = plan.P;
+        f.ldb = w.ld_h;
+        f.out[0] = at<float>(ws, w.zs);
+        f.ldo = qd.rank;
+        f.col_scale[0] = layer->proj[2].Sigma;
+        if ((st = tc_f16(f, plan.zdown, ws, w, stream)) != TILEQ_OK) return st;
+      } else {
       GemmBatch b;
       b.p[0] = problem(plan.zdown, ws, w);
       GemmProblem &z = b.p[0];
@@ -939,6 +1093,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       z.ldo = qd.rank;
       tma_b(z, plan.P, plan.zdown.bn);
       if ((st = gemm(b, 1, 1, plan.zdown, stream)) != TILEQ_OK) return st;
+      }
       mark(ST_ZDOWN, stream);
       LrAccArgs la = lracc_args(qd, w, ws, top_k, hext, w.ld_h, F);
       la.zslot = at<float>(ws, w.zs);

@@ -69,16 +69,20 @@ struct TcCfg {
   static_assert(SA >= 2, "TMEM too small for two A stages");
 };
 
-// rs: the item's row scale (SwiGLU h), loaded by the caller ahead of the stores
-__device__ __forceinline__ void tc_epi_store(const TcArgs &P, int item, int o, float v0, float v1, float rs) {
+// rs: the item's row scale (SwiGLU h); c0, c1: the output row's column scales
+// of projection 0 / 1; all loaded by the caller ahead of the stores
+__device__ __forceinline__ void tc_epi_store(const TcArgs &P, int item, int o, float v0, float v1, float rs,
+                                             float c0 = 1.f, float c1 = 1.f) {
   const size_t idx = (size_t)item * P.ldo + o;
   if (P.epi == EPI_SWIGLU_H) {
     reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(silu_f(v0) * v1 * rs);
   } else if (P.epi == EPI_STORE2_F32) {
-    reinterpret_cast<float *>(P.out[0])[idx] = v0;
-    reinterpret_cast<float *>(P.out[1])[idx] = v1;
+    reinterpret_cast<float *>(P.out[0])[idx] = v0 * c0;
+    reinterpret_cast<float *>(P.out[1])[idx] = v1 * c1;
+  } else if (P.epi == EPI_STORE_F16) {
+    reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(v0 * c0);
   } else {
-    reinterpret_cast<float *>(P.out[0])[idx] = v0;
+    reinterpret_cast<float *>(P.out[0])[idx] = v0 * c0;
   }
 }
 
@@ -144,11 +148,15 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
   tc::fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int n_tiles = *P.tile_count;
+  const int n_tiles = P.tiles ? *P.tile_count : (P.static_items + BN - 1) / BN;
+  // tile jt: (group, first item, items)
+  auto tile_of = [&](int jt) {
+    return P.tiles ? P.tiles[jt] : make_int4(0, jt * BN, min(BN, P.static_items - jt * BN), 0);
+  };
   const int total = n_tiles * P.m_tiles * P.ksplit;
   const int nkb = P.d_in / BK;
   const int per = (nkb + P.ksplit - 1) / P.ksplit;
-  const int g = P.group;
+  const int g = P.a_f16 ? BK : P.group;
   const int G = P.d_in / g;
   const int gps = g == 64 ? 2 : 1;
   // the K extension runs one projection at a time: n_ext1 stages of 128 columns each
@@ -176,13 +184,19 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
         int jt, ob, split, kb0, nmain, next;
         decode(w, jt, ob, split);
         stages_of(split, kb0, nmain, next);
-        const int4 t = P.tiles[jt];
+        const int4 t = tile_of(jt);
         const int grp = t.x, item0 = t.y;
         for (int st = 0; st < nmain + next; ++st, ++qi) {
           const int s = qi % C::SQ;
           if (qi >= (uint32_t)C::SQ && !(ok = mbar_wait(&q_empty[s], ((qi / C::SQ) - 1) & 1, P.status))) break;
           TC_TRACE(0, qi);
-          if (st < nmain) {
+          if (st < nmain && P.a_f16) {
+            // fp16 A: the dequantising warps read it from global memory; B only
+            const int kb = kb0 + st;
+            mbar_arrive_expect_tx(&q_full[s], 2 * C::BATOM);
+            for (int a = 0; a < 2; ++a)
+              tc::tma_load_2d(q_b(s) + a * C::BATOM, &P.bmap, kb * BK + a * 64, item0, &q_full[s]);
+          } else if (st < nmain) {
             const int kb = kb0 + st;
             mbar_arrive_expect_tx(&q_full[s], NP * (128 * 32 + gps * 512) + 2 * C::BATOM);
             for (int p = 0; p < NP; ++p) {
@@ -273,7 +287,7 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
       int jt, ob, split, kb0, nmain, next;
       decode(w, jt, ob, split);
       stages_of(split, kb0, nmain, next);
-      const int4 t = P.tiles[jt];
+      const int4 t = tile_of(jt);
       const int grp = t.x, item0 = t.y, nitems = t.z;
       for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
         const int s = qi % C::SQ, sa = ai % C::SA;
@@ -290,7 +304,20 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
           for (int c = 0; c < C::KPW / 32; ++c) {   // chunks of 32 K elements = 16 columns
             uint32_t *v = vv[p][c];
             const int k0 = part * C::KPW + c * 32;  // K offset within the stage
-            if (!ext) {
+            if (!ext && P.a_f16) {
+              // fp16 weights, row-major: 32 K elements of this thread's row
+              const int ab = P.use_a_blk ? P.a_blk[grp] : 0;
+              const uint4 *ar = reinterpret_cast<const uint4 *>(
+                  P.arow[p] + (((size_t)ab * P.m_tiles + ob) * 128 + row) * P.lda + (size_t)(kb0 + st) * BK + k0);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint4 q4 = __ldg(ar + j);
+                v[4 * j + 0] = q4.x;
+                v[4 * j + 1] = q4.y;
+                v[4 * j + 2] = q4.z;
+                v[4 * j + 3] = q4.w;
+              }
+            } else if (!ext) {
               const uint32_t *cw = reinterpret_cast<const uint32_t *>(q_codes(s, p)) + ((k0 / 32) * 128 + row) * 2;
               const int gl = g == 64 ? (k0 >> 6) : 0;
               const __half2 sz = u32_as_h2(q_sz(s, p)[gl * 128 + row]);
@@ -347,6 +374,9 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
       constexpr int CH = COLS >= 8 ? 8 : 4;    // columns per TMEM load
       const int o = ob * 128 + row;
       const int ldp = P.m_tiles * 128;
+      const int oc = min(o, P.d_out - 1);
+      const float cs0 = P.col_scale[0] ? __ldg(P.col_scale[0] + oc) : 1.f;
+      const float cs1 = P.col_scale[1] ? __ldg(P.col_scale[1] + oc) : 1.f;
       const bool no_k = nmain + next == 0;     // a split past the end of K contributes zeros
 #pragma unroll 1
       for (int c = 0; c < COLS; c += CH) {
@@ -366,7 +396,7 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
           for (int p = 0; p < NP; ++p)
 #pragma unroll
             for (int i = 0; i < CH; ++i) v[p][i] = 0.f;
-        float rs[CH];  // row scales ahead of the stores
+        float rs[CH];  // row (and below column) scales ahead of the stores
 #pragma unroll
         for (int i = 0; i < CH; ++i)
           rs[i] = P.row_scale ? __ldg(P.row_scale + item0 + min(part * COLS + c + i, nitems - 1)) : 1.f;
@@ -375,7 +405,7 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
           const int n = part * COLS + c + i;
           if (n >= nitems) continue;
           if (P.ksplit == 1) {
-            if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i], rs[i]);
+            if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i], rs[i], cs0, cs1);
           } else {
 #pragma unroll
             for (int p = 0; p < NP; ++p)
@@ -403,7 +433,9 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
 #pragma unroll
               for (int p = 0; p < NP; ++p)
                 r[p] += __ldcg(&P.part[(((size_t)sp * NP + p) * P.part_items + item0 + n) * ldp + oo]);
-            tc_epi_store(P, item0 + n, oo, r[0], r[NP - 1], P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f);
+            tc_epi_store(P, item0 + n, oo, r[0], r[NP - 1], P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f,
+                         P.col_scale[0] ? __ldg(P.col_scale[0] + oo) : 1.f,
+                         P.col_scale[1] ? __ldg(P.col_scale[1] + oo) : 1.f);
           }
           if (dw == 0 && lane == 0) P.counters[tile_id] = 0;
         }

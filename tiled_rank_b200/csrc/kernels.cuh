@@ -110,6 +110,16 @@ struct TcArgs {
   const int *tile_count;
   int m_tiles, ksplit, d_out, d_in, group, rank;
   int n_experts;             // experts (blocks) in codes / sz
+  // fp16 A instead of 2-bit codes (tcgen05 kernel only): arow[p] is row-major
+  // [blocks][m_tiles * 128][lda]; the block of a tile is a_blk[group] when
+  // use_a_blk, else 0.  tiles == nullptr: items 0..static_items-1 in tiles of bn.
+  int a_f16;
+  const __half *arow[2];
+  int lda;
+  int use_a_blk;
+  int8_t a_blk[kMaxExperts];
+  int static_items;
+  const float *col_scale[2];  // optional per-output-row scale of projection p (store epilogues)
   int ext_col[2];            // first B column of the K extension of projection p
   const uint4 *codes[2];     // tcgen05: [K][d_out/128][d_in/128][4 slices][128 rows][8 B]
                              // warp MMA: [K][d_out/128][d_in/128][8 warps][32 lanes][16 B]
@@ -224,6 +234,7 @@ __global__ void pack_frag_kernel(const __nv_bfloat16 *src, long long bs, long lo
 // reading one slice of 32 consecutive rows touches 256 contiguous bytes.
 __global__ void pack_codes_tc_kernel(const uint32_t *codes, uint32_t *out, int K, int d_out, int d_in);
 // bf16 [nblk][R][C] -> fp16 [nblk][pad128(R)][C] (zero rows appended).
+__global__ void pack_vt_rows_kernel(const __nv_bfloat16 *V, int N, int r, int d_in, __half *out);
 __global__ void expand_sigma_kernel(const float *sigma, int r, int rp, int n, float *out);
 __global__ void pack_rows_f16_kernel(const __nv_bfloat16 *src, int nblk, int R, int C, __half *out);
 

@@ -164,4 +164,18 @@ __global__ void pack_rows_f16_kernel(const __nv_bfloat16 *src, int nblk, int R, 
   out[gid] = r < R ? __float2half_rn(__bfloat162float(src[((size_t)b * R + r) * C + c])) : __float2half_rn(0.f);
 }
 
+// V [N][d_in][r] (bf16) -> V_n^T rows in fp16, [N][pad128(r)][d_in] (zero rows
+// past r): the row-major A operand of the tensor-core product z = V_n^T x.
+__global__ void pack_vt_rows_kernel(const __nv_bfloat16 *V, int N, int r, int d_in, __half *out) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int rp = pad128(r);
+  const long long total = (long long)N * rp * d_in;
+  if (gid >= total) return;
+  const int k = (int)(gid % d_in);
+  long long rest = gid / d_in;
+  const int i = (int)(rest % rp);
+  const int n = (int)(rest / rp);
+  out[gid] = i < r ? __float2half_rn(__bfloat162float(V[((size_t)n * d_in + k) * r + i])) : __float2half_rn(0.f);
+}
+
 }  // namespace tileq
