@@ -19,6 +19,8 @@
 // z (or a) vector, accumulated into the same TMEM accumulator.
 // Split-K work items write fp32 partials; the last one of a tile reduces them
 // in split order.  Every mbarrier wait is bounded and reports TILEQ_ERR_TIMEOUT.
+#include <type_traits>
+
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -48,7 +50,13 @@ constexpr int kDqw128 = TILEQ_TC_DQW128;  // dequantising warps of the 128-item 
 
 template <int NP, int BN, int DQW>
 struct TcCfg {
-  static constexpr int THREADS = (2 + DQW) * 32;
+  // one-projection launches: eight more warps run the epilogue from a second
+  // accumulator buffer while the next unit's MMAs fill the first (two-projection
+  // accumulators fill TMEM, so there the dequantising warps run the epilogue)
+  static constexpr bool EW = NP == 1;
+  static constexpr int NACC = EW ? 2 : 1;
+  static constexpr int EPW = EW ? 8 : 0;  // two warps per TMEM lane quadrant
+  static constexpr int THREADS = (2 + DQW + EPW) * 32;
   static constexpr int KPW = BK / (DQW / 4);          // K elements per dequant warp per stage
   static constexpr int CODES = NP * 128 * 32;         // packed codes of one stage (bytes)
   static constexpr int SZ = NP * 2 * 128 * 4;         // scale/zero words, up to 2 groups per stage
@@ -59,10 +67,10 @@ struct TcCfg {
   static constexpr int SQ = SQ_RAW > 8 ? 8 : (SQ_RAW < 2 ? 2 : SQ_RAW);
   static constexpr int ACC_COLS = NP * BN;
   static constexpr int A_COLS = NP * (BK / 2);          // TMEM columns of one A stage
-  static constexpr int SA_RAW = (512 - ACC_COLS) / A_COLS;
+  static constexpr int SA_RAW = (512 - NACC * ACC_COLS) / A_COLS;
   static constexpr int SA = SA_RAW > 4 ? 4 : SA_RAW;
   static constexpr int BAR_OFF = SQ * QSTAGE;
-  static constexpr int SMEM_USED = BAR_OFF + (2 * SQ + 2 * SA + 4) * 8 + 64 + 1024;  // + align slack
+  static constexpr int SMEM_USED = BAR_OFF + (2 * SQ + 2 * SA + 8) * 8 + 64 + 1024;  // + align slack
   // at least half of the SM's shared memory: one CTA per SM, so the 512-column
   // TMEM allocation never waits for another CTA of this kernel
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
@@ -103,7 +111,7 @@ __device__ __forceinline__ void dq_word(uint32_t w, const __half2 (&nz)[4], __ha
 }
 
 template <int NP, int BN, int DQW>
-__global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid_constant__ TcArgs P) {
+__global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel(const __grid_constant__ TcArgs P) {
   using C = TcCfg<NP, BN, DQW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -111,10 +119,10 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
   uint64_t *q_empty = q_full + C::SQ;
   uint64_t *a_full = q_empty + C::SQ;
   uint64_t *a_empty = a_full + C::SA;
-  uint64_t *acc_full = a_empty + C::SA;
-  uint64_t *acc_empty = acc_full + 1;
-  uint64_t *drain = acc_full + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 4);
+  uint64_t *acc_full = a_empty + C::SA;   // [NACC]
+  uint64_t *acc_empty = acc_full + 2;     // [NACC]
+  uint64_t *drain = acc_full + 4;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 6);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -133,8 +141,10 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
       mbar_init(&a_full[s], DQW);
       mbar_init(&a_empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, DQW);
+    for (int b = 0; b < C::NACC; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], C::EW ? C::EPW : DQW);
+    }
     mbar_init(drain, 1);
     *flag = 0;
     fence_mbar_init();
@@ -174,6 +184,90 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
     kb0 = min(nkb, split * per);
     nmain = min(nkb, kb0 + per) - kb0;
     next = split == 0 ? n_ext : 0;
+  };
+
+  // ---------------------------------------------------------------- epilogue
+  // Unit wi's accumulator (buffer ab) -> outputs.  COLS columns from `part *
+  // COLS`, row `row` of the 128-row block; the group of `nthr` threads syncs on
+  // named barrier `bar_id`; `leader` takes the split-K arrival.
+  auto epilogue = [&](auto cols_c, uint32_t wi, int ab, int jt, int ob, int split, bool no_k, int item0,
+                      int nitems, int row, int part, uint32_t lane_addr, int bar_id, int nthr, int tid,
+                      bool leader) -> bool {
+    constexpr int COLS = decltype(cols_c)::value;
+    constexpr int CH = COLS >= 8 ? 8 : 4;  // columns per TMEM load
+    if (leader) TC_TRACE(7, 2 * wi);
+    if (!mbar_wait(&acc_full[ab], (wi / C::NACC) & 1, P.status)) return false;
+    if (leader) TC_TRACE(7, 2 * wi + 1);
+    tc::fence_after();
+    const int o = ob * 128 + row;
+    const int ldp = P.m_tiles * 128;
+    const int oc = min(o, P.d_out - 1);
+    const float cs0 = P.col_scale[0] ? __ldg(P.col_scale[0] + oc) : 1.f;
+    const float cs1 = P.col_scale[1] ? __ldg(P.col_scale[1] + oc) : 1.f;
+#pragma unroll 1
+    for (int c = 0; c < COLS; c += CH) {
+      float v[NP][CH];
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const uint32_t addr = tmem + lane_addr + ab * C::ACC_COLS + p * BN + part * COLS + c;
+        if constexpr (CH == 8) {
+          tc::ld8(addr, v[p]);
+        } else {
+          tc::ld4(addr, v[p]);
+        }
+      }
+      tc::wait_ld();
+      if (no_k)  // a split past the end of K contributes zeros
+#pragma unroll
+        for (int p = 0; p < NP; ++p)
+#pragma unroll
+          for (int i = 0; i < CH; ++i) v[p][i] = 0.f;
+      float rs[CH];  // row scales ahead of the stores
+#pragma unroll
+      for (int i = 0; i < CH; ++i)
+        rs[i] = P.row_scale ? __ldg(P.row_scale + item0 + min(part * COLS + c + i, nitems - 1)) : 1.f;
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        const int n = part * COLS + c + i;
+        if (n >= nitems) continue;
+        if (P.ksplit == 1) {
+          if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i], rs[i], cs0, cs1);
+        } else {
+#pragma unroll
+          for (int p = 0; p < NP; ++p)
+            P.part[(((size_t)split * NP + p) * P.part_items + item0 + n) * ldp + o] = v[p][i];
+        }
+      }
+    }
+    tc::fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&acc_empty[ab]);
+
+    if (P.ksplit > 1) {
+      __threadfence();
+      named_sync(bar_id, nthr);
+      const int tile_id = jt * P.m_tiles + ob;
+      if (leader) *flag = (atomicAdd(&P.counters[tile_id], 1) == P.ksplit - 1);
+      named_sync(bar_id, nthr);
+      if (*flag) {
+        __threadfence();
+        for (int idx = tid; idx < BN * 128; idx += nthr) {
+          const int n = idx / 128, oo = ob * 128 + idx % 128;
+          if (n >= nitems || oo >= P.d_out) continue;
+          float r[2] = {0.f, 0.f};
+          for (int sp = 0; sp < P.ksplit; ++sp)
+#pragma unroll
+            for (int p = 0; p < NP; ++p)
+              r[p] += __ldcg(&P.part[(((size_t)sp * NP + p) * P.part_items + item0 + n) * ldp + oo]);
+          tc_epi_store(P, item0 + n, oo, r[0], r[NP - 1], P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f,
+                       P.col_scale[0] ? __ldg(P.col_scale[0] + oo) : 1.f,
+                       P.col_scale[1] ? __ldg(P.col_scale[1] + oo) : 1.f);
+        }
+        if (leader) P.counters[tile_id] = 0;
+      }
+      named_sync(bar_id, nthr);
+    }
+    return true;
   };
 
   if (warp == 0) {
@@ -230,7 +324,8 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
         int jt, ob, split, kb0, nmain, next;
         decode(w, jt, ob, split);
         stages_of(split, kb0, nmain, next);
-        if (wi > 0 && !(ok = mbar_wait(acc_empty, (wi - 1) & 1, P.status))) break;
+        const int ab = wi % C::NACC;  // accumulator buffer of this unit
+        if (wi >= (uint32_t)C::NACC && !(ok = mbar_wait(&acc_empty[ab], ((wi / C::NACC) - 1) & 1, P.status))) break;
         tc::fence_after();
         bool first = true;
         for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
@@ -247,18 +342,18 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
           // warps: keep its instruction stream short (one descriptor per stage,
           // constant offsets: the start-address field counts 16-byte units)
           const uint64_t bd0 = tc::sdesc_sw128(smem_addr(q_b(s)));
-          const uint32_t a0 = tmem + C::ACC_COLS + sa * C::A_COLS;
+          const uint32_t a0 = tmem + C::NACC * C::ACC_COLS + sa * C::A_COLS;
           if (!ext) {
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
-              const uint32_t d = tmem + p * BN, a = a0 + p * (BK / 2);
+              const uint32_t d = tmem + ab * C::ACC_COLS + p * BN, a = a0 + p * (BK / 2);
               tc::mma_ts(d, a, bd0, idesc, first ? 0u : 1u);
 #pragma unroll
               for (int kk = 1; kk < BK / 16; ++kk)
                 tc::mma_ts(d, a + kk * 8, bd0 + (uint64_t)(((kk / 4) * C::BATOM + (kk % 4) * 32) >> 4), idesc, 1u);
             }
           } else {
-            const uint32_t d = tmem + pe * BN, a = a0 + pe * (BK / 2);
+            const uint32_t d = tmem + ab * C::ACC_COLS + pe * BN, a = a0 + pe * (BK / 2);
             for (int kk = 0; kk < nk; ++kk)
               tc::mma_ts(d, a + kk * 8, bd0 + (uint64_t)(((kk / 4) * C::BATOM + (kk % 4) * 32) >> 4), idesc,
                          (first && kk == 0) ? 0u : 1u);
@@ -269,14 +364,14 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
           tc::commit(&q_empty[s]);
         }
         if (!ok) break;
-        tc::commit(acc_full);
+        tc::commit(&acc_full[ab]);
       }
       // all issued MMAs have retired before TMEM is released
       tc::commit(drain);
       mbar_wait(drain, 0, P.status);
     }
-  } else {
-    // ============================================================ dequant + epilogue
+  } else if (warp < 2 + DQW) {
+    // ============================================================ dequant (+ epilogue when NP == 2)
     const int dw = warp - 2;
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int part = dw >> 2;                  // K slice (dequant) / column slice (epilogue)
@@ -352,7 +447,8 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
           if (ext && p != pe) continue;
-          const uint32_t acol = tmem + lane_addr + C::ACC_COLS + sa * C::A_COLS + p * (BK / 2) + part * (C::KPW / 2);
+          const uint32_t acol =
+              tmem + lane_addr + C::NACC * C::ACC_COLS + sa * C::A_COLS + p * (BK / 2) + part * (C::KPW / 2);
 #pragma unroll
           for (int c = 0; c < C::KPW / 32; ++c) tc::st16(acol + c * 16, vv[p][c]);
         }
@@ -365,82 +461,28 @@ __global__ void __launch_bounds__((2 + DQW) * 32, 1) gemm_tc_kernel(const __grid
       }
       if (!ok) break;
 
-      // -------------------------------------------------------- epilogue
-      if (dw == 0 && lane == 0) TC_TRACE(7, 2 * wi);
-      if (!(ok = mbar_wait(acc_full, wi & 1, P.status))) break;
-      if (dw == 0 && lane == 0) TC_TRACE(7, 2 * wi + 1);
-      tc::fence_after();
-      constexpr int COLS = BN / (DQW / 4);     // accumulator columns of this warp
-      constexpr int CH = COLS >= 8 ? 8 : 4;    // columns per TMEM load
-      const int o = ob * 128 + row;
-      const int ldp = P.m_tiles * 128;
-      const int oc = min(o, P.d_out - 1);
-      const float cs0 = P.col_scale[0] ? __ldg(P.col_scale[0] + oc) : 1.f;
-      const float cs1 = P.col_scale[1] ? __ldg(P.col_scale[1] + oc) : 1.f;
-      const bool no_k = nmain + next == 0;     // a split past the end of K contributes zeros
-#pragma unroll 1
-      for (int c = 0; c < COLS; c += CH) {
-        float v[NP][CH];
-#pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          const uint32_t addr = tmem + lane_addr + p * BN + part * COLS + c;
-          if constexpr (CH == 8) {
-            tc::ld8(addr, v[p]);
-          } else {
-            tc::ld4(addr, v[p]);
-          }
-        }
-        tc::wait_ld();
-        if (no_k)
-#pragma unroll
-          for (int p = 0; p < NP; ++p)
-#pragma unroll
-            for (int i = 0; i < CH; ++i) v[p][i] = 0.f;
-        float rs[CH];  // row (and below column) scales ahead of the stores
-#pragma unroll
-        for (int i = 0; i < CH; ++i)
-          rs[i] = P.row_scale ? __ldg(P.row_scale + item0 + min(part * COLS + c + i, nitems - 1)) : 1.f;
-#pragma unroll
-        for (int i = 0; i < CH; ++i) {
-          const int n = part * COLS + c + i;
-          if (n >= nitems) continue;
-          if (P.ksplit == 1) {
-            if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i], rs[i], cs0, cs1);
-          } else {
-#pragma unroll
-            for (int p = 0; p < NP; ++p)
-              P.part[(((size_t)split * NP + p) * P.part_items + item0 + n) * ldp + o] = v[p][i];
-          }
-        }
+      if (!C::EW) {
+        if (!(ok = epilogue(std::integral_constant<int, BN / (DQW / 4)>{}, wi, 0, jt, ob, split, nmain + next == 0,
+                            item0, nitems, row, part, lane_addr, 1, DQW * 32, dw * 32 + lane, dw == 0 && lane == 0)))
+          break;
       }
-      tc::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-
-      if (P.ksplit > 1) {
-        __threadfence();
-        named_sync(1, DQW * 32);
-        const int tile_id = jt * P.m_tiles + ob;
-        if (dw == 0 && lane == 0) *flag = (atomicAdd(&P.counters[tile_id], 1) == P.ksplit - 1);
-        named_sync(1, DQW * 32);
-        if (*flag) {
-          __threadfence();
-          for (int idx = dw * 32 + lane; idx < BN * 128; idx += DQW * 32) {
-            const int n = idx / 128, oo = ob * 128 + idx % 128;
-            if (n >= nitems || oo >= P.d_out) continue;
-            float r[2] = {0.f, 0.f};
-            for (int sp = 0; sp < P.ksplit; ++sp)
-#pragma unroll
-              for (int p = 0; p < NP; ++p)
-                r[p] += __ldcg(&P.part[(((size_t)sp * NP + p) * P.part_items + item0 + n) * ldp + oo]);
-            tc_epi_store(P, item0 + n, oo, r[0], r[NP - 1], P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f,
-                         P.col_scale[0] ? __ldg(P.col_scale[0] + oo) : 1.f,
-                         P.col_scale[1] ? __ldg(P.col_scale[1] + oo) : 1.f);
-          }
-          if (dw == 0 && lane == 0) P.counters[tile_id] = 0;
-        }
-        named_sync(1, DQW * 32);
-      }
+    }
+  } else {
+    // ============================================================ epilogue warps (NP == 1)
+    const int ew = warp - 2 - DQW;
+    const int row = (warp & 3) * 32 + lane;  // this warp's TMEM lane quadrant
+    const int epart = ew >> 2;                 // column half
+    const uint32_t lane_addr = tc::lane_base(warp);
+    uint32_t wi = 0;
+    for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++wi) {
+      int jt, ob, split, kb0, nmain, next;
+      decode(w, jt, ob, split);
+      stages_of(split, kb0, nmain, next);
+      const int4 t = tile_of(jt);
+      if (!(ok = epilogue(std::integral_constant<int, BN / (C::EW ? C::EPW / 4 : 1)>{}, wi, wi % C::NACC, jt, ob, split,
+                          nmain + next == 0, t.y, t.z, row, epart, lane_addr, 2, C::EPW * 32, ew * 32 + lane,
+                          ew == 0 && lane == 0)))
+        break;
     }
   }
 
