@@ -55,7 +55,9 @@ def check_route(route, logits, top_k, K):
 # ---------------------------------------------------------------------------
 # routing
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("T,K,k", [(1, 8, 2), (37, 4, 4), (1000, 60, 4), (4096, 8, 2), (2048, 64, 8)])
+# above 4096 pairs the sort runs on one CTA per 1024 pairs; 8194 and 20000 end in a ragged chunk
+@pytest.mark.parametrize("T,K,k", [(1, 8, 2), (37, 4, 4), (1000, 60, 4), (1024, 8, 4), (4096, 8, 2),
+                                   (4097, 8, 2), (2048, 64, 8), (5000, 60, 4)])
 def test_route_bitexact(torch_cuda, T, K, k):
     torch = torch_cuda
     from tiled_rank_b200 import tileq_route
@@ -117,6 +119,9 @@ TINY = [
     # long batches: z, z' and the shared expert on tcgen05 as well
     (synth.SWIGLU, 8, 2, 4, 128, 256, 48, 128, 2, 256, 300),
     (synth.LINEAR, 5, 2, 3, 384, 144, 16, 128, 3, 0, 300),
+    # more than 4096 pairs: the multi-CTA sort, its slot tables and grid-row flags
+    (synth.SWIGLU, 16, 4, 4, 128, 128, 16, 64, 4, 0, 1500),
+    (synth.LINEAR, 12, 3, 4, 128, 128, 16, 64, 3, 0, 1700),
 ]
 
 

@@ -308,7 +308,7 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
 struct WsLayout {
   Plan plan;
   size_t status, topk_idx, topk_w, expert_offsets, sorted_pairs, slot_of_pair, slot_tok, slot_w,
-      dest, tiles_main, tile_first, tile_counts, counters, part;
+      dest, pcounts, tiles_main, tile_first, tile_counts, counters, part;
   int n_counters;
   size_t part_zstride;
   size_t zidx[2];
@@ -341,6 +341,7 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool
   w.slot_tok = take(Pz * 4);
   w.slot_w = take(Pz * 4);
   w.dest = take(Pz * 4);
+  w.pcounts = take((size_t)cdiv(P, kPermChunk) * L->K * 4);
   w.tiles_main = take((size_t)(pl.slots_main + 1) * 16);
   w.tile_first = take((L->K + 1) * 4);
   w.tile_counts = take(16);
@@ -659,8 +660,18 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   pa.row_proj = row_proj;
   if (row_proj >= 0) std::memcpy(pa.m_of_row, li.p[row_proj].m_of, kMaxExperts);
   pa.aidx = at<int>(ws, w.aidx);
-  permute_kernel<<<1, 1024, 0, stream>>>(pa);
-  TQ_LAUNCHED();
+  pa.pcounts = at<int>(ws, w.pcounts);
+  const int P = T * top_k;
+  if (P > kPermMultiMin) {
+    const unsigned nc = (unsigned)cdiv(P, kPermChunk);
+    permute_count_kernel<<<nc, kPermChunkThreads, 0, stream>>>(pa);
+    TQ_LAUNCHED();
+    permute_scatter_kernel<<<nc, kPermChunkThreads, 0, stream>>>(pa);
+    TQ_LAUNCHED();
+  } else {
+    permute_kernel<<<1, 1024, 0, stream>>>(pa);
+    TQ_LAUNCHED();
+  }
   mark(ST_PERMUTE, stream);
   return TILEQ_OK;
 }

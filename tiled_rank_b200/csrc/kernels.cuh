@@ -37,7 +37,13 @@ struct PermuteArgs {
   int row_proj;            // -1 = no row designation
   int8_t m_of_row[kMaxExperts];
   int *aidx;               // slot -> 1 for the token's first slot in its grid row, else -1
+  int *pcounts;            // multi-CTA sort: [CTAs][K] pairs per expert in each CTA's chunk
 };
+
+// Batches of more than kPermMultiMin pairs are sorted by kPermChunk-pair CTAs.
+constexpr int kPermChunk = 1024;
+constexpr int kPermChunkThreads = 256;
+constexpr int kPermMultiMin = 4096;
 
 // ---------------------------------------------------------------- GEMM
 // EPI_PARTIAL_F32: each K split stores its own fp32 partial (times col_scale) at
@@ -210,6 +216,8 @@ struct SwigluArgs {
 
 __global__ void route_kernel(RouteArgs a);
 __global__ void permute_kernel(PermuteArgs a);
+__global__ void permute_count_kernel(PermuteArgs a);
+__global__ void permute_scatter_kernel(PermuteArgs a);
 __global__ void lr_accumulate_kernel(LrAccArgs a);
 __global__ void combine_kernel(CombineArgs a);
 __global__ void scale_gather_kernel(ScaleGatherArgs a);

@@ -8,6 +8,8 @@
 //                   slot, the row of the projected [T, N, r] tensor it reads
 //                   (TileQ paper, section 2.2) and whether it is the token's
 //                   first slot in its grid row (the in-place accumulation).
+// permute_count_kernel + permute_scatter_kernel: the same sort and tables for
+//                   long batches, one CTA per 1024 pairs.
 #include "kernels.cuh"
 
 namespace tileq {
@@ -187,40 +189,144 @@ __device__ void build_tiles(const int *off, int ngroups, int bn, int4 *tiles, in
   __syncthreads();
 }
 
+// The tables of one sorted pair p placed at slot: the pair itself, its token and
+// weight; its row of the projected [T, N, r] tensor per z projection (TileQ
+// paper, section 2.2: project once, select by routing); and for the in-place
+// accumulation per (token, grid row), whether it is the token's first slot in
+// its grid row (that slot carries a_{t,m}, the others carry zeros).
+__device__ __forceinline__ void write_slot(const PermuteArgs &a, int p, int slot) {
+  const int k = a.k;
+  const int t = p / k, j = p - t * k;
+  const int e = a.topk_idx[p];
+  a.sorted_pairs[slot] = p;
+  a.slot_of_pair[p] = slot;
+  a.slot_tok[slot] = t;
+  a.slot_w[slot] = a.topk_w[p];
+  for (int zp = 0; zp < a.n_zproj; ++zp) a.zidx[zp][slot] = t * a.N + a.n_of[zp][e];
+  if (a.row_proj >= 0) {
+    const int8_t *mrow = a.m_of_row;
+    const int r = mrow[e];
+    bool designated = true;
+    for (int jj = 0; jj < j; ++jj)
+      if (mrow[a.topk_idx[t * k + jj]] == r) designated = false;
+    a.aidx[slot] = designated ? 1 : -1;
+  }
+}
+
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
   __shared__ SortSmem s;
   __shared__ int scratch[kMaxExperts + 1];
   const int P = a.T * a.k;
-  const int k = a.k;
   const int32_t *idx = a.topk_idx;
 
-  // 1. pairs by expert
   cta_stable_sort(P, a.K, [&](int p) { return idx[p]; }, a.dest, a.expert_offsets, s);
-  for (int p = threadIdx.x; p < P; p += blockDim.x) {
-    const int slot = a.dest[p];
-    const int t = p / k, j = p - t * k;
-    const int e = idx[p];
-    a.sorted_pairs[slot] = p;
-    a.slot_of_pair[p] = slot;
-    a.slot_tok[slot] = t;
-    a.slot_w[slot] = a.topk_w[p];
-    // 2. the slot's row of the projected [T, N, r] tensor, z = Sigma*(V_n^T x_t),
-    //    per z projection (TileQ paper, section 2.2: project once, select by routing)
-    for (int zp = 0; zp < a.n_zproj; ++zp) a.zidx[zp][slot] = t * a.N + a.n_of[zp][e];
-    // 3. in-place accumulation per (token, grid row): the token's first slot in
-    //    grid row m carries a_{t,m}, the others carry zeros
-    if (a.row_proj >= 0) {
-      const int8_t *mrow = a.m_of_row;
-      const int r = mrow[e];
-      bool designated = true;
-      for (int jj = 0; jj < j; ++jj)
-        if (mrow[idx[t * k + jj]] == r) designated = false;
-      a.aidx[slot] = designated ? 1 : -1;
-    }
-  }
+  for (int p = threadIdx.x; p < P; p += blockDim.x) write_slot(a, p, a.dest[p]);
   __syncthreads();
   build_tiles(a.expert_offsets, a.K, a.bn, a.tiles_main, a.tile_counts + 0, a.tile_first_main,
               scratch);
+}
+
+// ---------------------------------------------------------------------------
+// multi-CTA stable counting sort for long batches: CTA c owns the pairs
+// [c*kPermChunk, (c+1)*kPermChunk).  permute_count_kernel stores each CTA's
+// per-expert counts; permute_scatter_kernel derives from them where the CTA's
+// pairs of each expert start and places them in pair order, so the result is
+// the same stable order as the one-CTA sort.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kPermChunkThreads) permute_count_kernel(PermuteArgs a) {
+  __shared__ int hist[kMaxExperts];
+  const int P = a.T * a.k;
+  for (int e = threadIdx.x; e < a.K; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int p0 = blockIdx.x * kPermChunk, p1 = min(P, p0 + kPermChunk);
+  for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) atomicAdd(&hist[a.topk_idx[p]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.K; e += blockDim.x) a.pcounts[blockIdx.x * a.K + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(kPermChunkThreads) permute_scatter_kernel(PermuteArgs a) {
+  constexpr int W = kPermChunkThreads / 32;
+  constexpr int kParts = kPermChunkThreads / kMaxExperts;
+  static_assert(kPermChunk % W == 0 && kParts >= 1, "chunk split");
+  __shared__ int hist[W][kMaxExperts];
+  __shared__ int red[2][kParts][kMaxExperts];
+  __shared__ int before[kMaxExperts];
+  __shared__ int start[kMaxExperts + 1];
+  __shared__ int scratch[kMaxExperts + 1];
+  const int P = a.T * a.k, K = a.K, C = gridDim.x, c = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t *idx = a.topk_idx;
+
+  // 1. per expert: pairs in all CTAs (the bucket sizes) and in the CTAs before this one
+  {
+    const int e = threadIdx.x % kMaxExperts, part = threadIdx.x / kMaxExperts;
+    int b = 0, tot = 0;
+    if (e < K) {
+      for (int cc = part; cc < C; cc += kParts) {
+        const int v = a.pcounts[cc * K + e];
+        tot += v;
+        if (cc < c) b += v;
+      }
+    }
+    red[0][part][e] = b;
+    red[1][part][e] = tot;
+  }
+  for (int i = threadIdx.x; i < W * kMaxExperts; i += blockDim.x) (&hist[0][0])[i] = 0;
+  __syncthreads();
+  if (threadIdx.x < K) {
+    int b = 0, tot = 0;
+    for (int q = 0; q < kParts; ++q) {
+      b += red[0][q][threadIdx.x];
+      tot += red[1][q][threadIdx.x];
+    }
+    before[threadIdx.x] = b;
+    start[threadIdx.x] = tot;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < K; ++e) {
+      const int n = start[e];
+      start[e] = run;
+      run += n;
+    }
+    start[K] = run;
+  }
+  __syncthreads();
+  if (c == 0) {
+    for (int e = threadIdx.x; e <= K; e += blockDim.x) a.expert_offsets[e] = start[e];
+    build_tiles(start, K, a.bn, a.tiles_main, a.tile_counts + 0, a.tile_first_main, scratch);
+  }
+
+  // 2. this CTA's pairs, split into W contiguous runs, one per warp
+  const int p0 = c * kPermChunk, p1 = min(P, p0 + kPermChunk);
+  constexpr int sub = kPermChunk / W;
+  const int w0 = min(p1, p0 + warp * sub), w1 = min(p1, w0 + sub);
+  for (int i = w0 + lane; i < w1; i += 32) atomicAdd(&hist[warp][idx[i]], 1);
+  __syncthreads();
+  if (threadIdx.x < K) {
+    int run = start[threadIdx.x] + before[threadIdx.x];
+    for (int w = 0; w < W; ++w) {
+      const int n = hist[w][threadIdx.x];
+      hist[w][threadIdx.x] = run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  // 3. stable placement: equal experts within 32 pairs ranked by lane
+  for (int base = w0; base < w1; base += 32) {
+    const int i = base + lane;
+    const int kk = i < w1 ? idx[i] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, kk);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int pos = kk >= 0 ? hist[warp][kk] + rank : 0;
+    __syncwarp();
+    if (kk >= 0) {
+      write_slot(a, i, pos);
+      if (rank == 0) hist[warp][kk] += __popc(peers);
+    }
+    __syncwarp();
+  }
 }
 
 }  // namespace tileq
