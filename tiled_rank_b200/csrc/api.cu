@@ -24,11 +24,18 @@ int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 unsigned nblocks(long long n, int per) { return (unsigned)((n + per - 1) / per); }
 
 constexpr int kNumSMs = 148;
+// gather_ext_kernel: one chunk per thread while that fits in one wave of CTAs
+// (short batches: the z sums need the parallelism), then grid-stride with
+// kGatherUnroll chunks per thread in flight
+unsigned gather_blocks(long long chunks) {
+  return std::max(1u, std::min(nblocks(chunks, 256), 8u * kNumSMs));
+}
+// split the narrow residual GEMM until ~this many CTAs per SM
 #ifndef TILEQ_Q2_PER_SM
 #define TILEQ_Q2_PER_SM 4
 #endif
 constexpr int kQ2PerSm = TILEQ_Q2_PER_SM;
-constexpr int kTcMinTokens = 256;  // dense fp16 products (z, shared expert) move to tcgen05 from here  // split the narrow residual GEMM until ~this many CTAs per SM
+constexpr int kTcMinTokens = 256;  // dense fp16 products (z, shared expert) move to tcgen05 from here
 
 struct ProjInfo {
   int d_in, d_out, rank, group, G;
@@ -523,12 +530,14 @@ tileq_status tc_launch(const TcArgs &a, int np, const GemmPlan &g, cudaStream_t 
   return launch_gemm_tc(a, np, g.bn, kNumSMs, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
 }
 
-// A dense fp16 product on tcgen05: A row-major fp16 (arow[p], lda), B the fp16
-// rows [brows][ldb] read by TMA, items either a tile table or 0..static_items-1.
+// A dense fp16 product on tcgen05 (gemm_dense.cu): A row-major fp16 (arow[p],
+// lda, arows rows; 0 = pad128(d_out)), B the fp16 rows [brows][ldb], items
+// either a tile table (of width g.bn) or 0..static_items-1.  np == 2: two
+// projections share B (pair units).
 struct TcF16 {
   int np = 1;
   const __half *arow[2] = {nullptr, nullptr};
-  int lda = 0, d_out = 0, d_in = 0;
+  int lda = 0, d_out = 0, d_in = 0, arows = 0;
   const int4 *tiles = nullptr;
   const int *tile_count = nullptr;
   int static_items = 0;
@@ -542,35 +551,56 @@ struct TcF16 {
   const float *row_scale = nullptr;
 };
 
+// Item-tile width of a dense product over `items` items with `m_units` units
+// per tile: the fewest CTA waves times the time of one unit, from the measured
+// cost of one M=128 K=16 tcgen05.mma (N=64: 48 cycles, N=128: 64, N=256: 128).
+int dense_bn(int items, int m_units) {
+  int best = 128;
+  long long best_cost = -1;
+  for (int bn : {256, 128, 64}) {
+    const long long units = (long long)cdiv(items, bn) * m_units;
+    const long long cost = cdiv(units, kNumSMs) * (bn == 64 ? 48 : bn / 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best = bn;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 tileq_status tc_f16(const TcF16 &f, const GemmPlan &g, void *ws, const WsLayout &w, cudaStream_t stream) {
-  TcArgs a;
+  DenseArgs a;
   std::memset(&a, 0, sizeof(a));
-  if (!make_map(&a.bmap, f.b, f.brows, f.ldb, f.ldb, g.bn)) return TILEQ_ERR_CUDA;
+  if (f.d_in % 64 || f.d_in <= 0) return TILEQ_ERR_UNSUPPORTED;
+  const int m_blocks = cdiv(f.d_out, 128);
+  const bool pair = f.np == 2;
+  const int mb = pair || m_blocks > 1 ? 2 : 1;
+  a.pair = pair;
+  a.m_blocks = m_blocks;
+  a.m_units = pair ? m_blocks : cdiv(m_blocks, mb);
+  const int bn = f.tiles ? g.bn : dense_bn(f.static_items, a.m_units);
+  const int arows = f.arows ? f.arows : m_blocks * 128;
+  for (int p = 0; p < f.np; ++p)
+    if (!make_map(&a.amap[p], f.arow[p], arows, f.d_in, f.lda, 128)) return TILEQ_ERR_CUDA;
+  if (!make_map(&a.bmap, f.b, f.brows, f.ldb, f.ldb, bn)) return TILEQ_ERR_CUDA;
   a.tiles = f.tiles;
   a.tile_count = f.tile_count;
   a.static_items = f.static_items;
-  a.m_tiles = cdiv(f.d_out, 128);
-  a.ksplit = 1;
-  a.d_out = f.d_out;
-  a.d_in = f.d_in;
-  a.a_f16 = 1;
-  a.arow[0] = f.arow[0];
-  a.arow[1] = f.arow[1];
-  a.lda = f.lda;
   a.use_a_blk = f.a_blk != nullptr;
   if (f.a_blk) std::memcpy(a.a_blk, f.a_blk, kMaxExperts);
+  a.d_out = f.d_out;
+  a.d_in = f.d_in;
   a.epi = f.epi;
   a.out[0] = f.out[0];
   a.out[1] = f.out[1];
   a.ldo = f.ldo;
-  a.row_scale = f.row_scale;
   a.col_scale[0] = f.col_scale[0];
   a.col_scale[1] = f.col_scale[1];
-  a.part = at<float>(ws, w.part);
-  a.part_items = 1;
-  a.counters = at<int>(ws, w.counters);
+  a.row_scale = f.row_scale;
   a.status = at<int>(ws, w.status);
-  return launch_gemm_tc(a, f.np, g.bn, kNumSMs, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
+  const long long units = f.tiles ? kNumSMs : (long long)cdiv(f.static_items, bn) * a.m_units;
+  const int grid = (int)std::min<long long>(kNumSMs, units);
+  return launch_gemm_dense(a, mb, bn, grid, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
 }
 
 // One residual projection (or the gate/up pair) over the main tile table:
@@ -1045,7 +1075,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       ga.zld = pad128(qg.rank);
       ga.out = xext;
       const long long chunks = (long long)plan.P * (D / 8 + (lr_gu ? 2 * qg.rank / 8 : 0));
-      gather_ext_kernel<<<nblocks(chunks, 256), 256, 0, stream>>>(ga);
+      gather_ext_kernel<<<gather_blocks(chunks), 256, 0, stream>>>(ga);
       TQ_LAUNCHED();
     }
     mark(ST_ZPROJ, stream);
@@ -1073,6 +1103,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
         TcF16 f;
         f.arow[0] = at<__half>(packed, pl.vr[2]);
         f.lda = F;
+        f.arows = layer->N * pad128(qd.rank);
         f.d_out = qd.rank;
         f.d_in = F;
         f.tiles = at<int4>(ws, w.tiles_main);
@@ -1275,7 +1306,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     ga.slot_tok = at<int>(ws, w.slot_tok);
     ga.x16 = at<__half>(ws, w.x16);
     ga.out = xext;
-    gather_ext_kernel<<<nblocks((long long)plan.P * (D / 8), 256), 256, 0, stream>>>(ga);
+    gather_ext_kernel<<<gather_blocks((long long)plan.P * (D / 8)), 256, 0, stream>>>(ga);
     TQ_LAUNCHED();
     Residual r;
     r.np = 2;

@@ -45,6 +45,9 @@ constexpr int kPermChunk = 1024;
 constexpr int kPermChunkThreads = 256;
 constexpr int kPermMultiMin = 4096;
 
+// 16-byte chunks per thread in flight in gather_ext_kernel.
+constexpr int kGatherUnroll = 4;
+
 // ---------------------------------------------------------------- GEMM
 // EPI_PARTIAL_F32: each K split stores its own fp32 partial (times col_scale) at
 // out[0][(split * part_items + item) * ldo + o]; the consumer sums the splits in
@@ -143,6 +146,35 @@ struct TcArgs {
 };
 
 cudaError_t launch_gemm_tc(const TcArgs &a, int np, int bn, int grid, cudaStream_t stream);
+
+// Dense fp16 GEMM on tcgen05 with both operands read by TMA (gemm_dense.cu).
+// A: fp16 row-major, tensor maps amap[j] (box 64 x 128, 128-byte swizzle);
+// B: fp16 item rows, bmap (box 64 x bn).  A work unit is MB row blocks of 128
+// against one item tile: pair != 0: block `ou` of amap[0] and of amap[1]
+// (two projections sharing B; epilogue EPI_STORE2_F32 or EPI_SWIGLU_H),
+// else blocks MB*ou .. MB*ou+MB-1 of amap[0].  The A row of block rb of a tile
+// of group g is (a_blk[g] * m_blocks + rb) * 128 when use_a_blk, else rb * 128.
+struct DenseArgs {
+  alignas(64) CUtensorMap amap[2];
+  alignas(64) CUtensorMap bmap;
+  const int4 *tiles;      // (group, first item, items) or nullptr: static_items in tiles of bn
+  const int *tile_count;
+  int static_items;
+  int pair;
+  int m_units;            // units per item tile
+  int m_blocks;           // row blocks of one A block (cdiv(d_out, 128))
+  int use_a_blk;
+  int8_t a_blk[kMaxExperts];
+  int d_out, d_in;        // d_in a multiple of 64
+  int epi;
+  void *out[2];
+  int ldo;
+  const float *col_scale[2];
+  const float *row_scale;
+  int *status;
+};
+
+cudaError_t launch_gemm_dense(const DenseArgs &a, int mb, int bn, int grid, cudaStream_t stream);
 
 // The same residual GEMM for narrow tiles (bn 8, 16 or 32) on warp-level MMA:
 // codes[p] in the per-lane fragment layout of pack_codes_kernel, B through

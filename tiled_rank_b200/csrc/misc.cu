@@ -44,60 +44,96 @@ __global__ void lr_accumulate_kernel(LrAccArgs a) {
 }
 
 // x_ext[s] = [x16[tok(s)] | z0[zidx0[s]] | z1[zidx1[s]]]  (fp16, 8-element chunks)
-__global__ void gather_ext_kernel(GatherExtArgs a) {
+// One 16-byte chunk of row s of the activation matrix: x_t, or eight z values
+// (the sum of the K-split partials in split order, to fp16).
+__device__ __forceinline__ uint4 ext_chunk(const GatherExtArgs &a, int s, int c) {
+  if (c < a.d / 8) return __ldg(reinterpret_cast<const uint4 *>(a.x16 + (size_t)a.slot_tok[s] * a.d) + c);
+  const int zc = c - a.d / 8, p = zc / (a.r / 8), cc = zc % (a.r / 8);
+  const float *z = a.z[p] + (size_t)a.zidx[p][s] * a.zld + cc * 8;
+  float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+  for (int sp0 = 0; sp0 < a.zks; sp0 += 8) {
+    // eight splits' loads in flight, then summed in split order
+    float4 l[8], h[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const bool in = sp0 + u < a.zks;
+      const float4 *q = reinterpret_cast<const float4 *>(z + (size_t)(sp0 + u) * a.zsplit);
+      l[u] = in ? q[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+      h[u] = in ? q[1] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      lo.x += l[u].x; lo.y += l[u].y; lo.z += l[u].z; lo.w += l[u].w;
+      hi.x += h[u].x; hi.y += h[u].y; hi.z += h[u].z; hi.w += h[u].w;
+    }
+  }
+  uint4 v;
+  __half2 *o = reinterpret_cast<__half2 *>(&v);
+  o[0] = __floats2half2_rn(lo.x, lo.y);
+  o[1] = __floats2half2_rn(lo.z, lo.w);
+  o[2] = __floats2half2_rn(hi.x, hi.y);
+  o[3] = __floats2half2_rn(hi.z, hi.w);
+  return v;
+}
+
+// Grid-stride over the P * chunks 16-byte chunks, kGatherUnroll of them per
+// thread in flight.
+__global__ void __launch_bounds__(256) gather_ext_kernel(GatherExtArgs a) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long G = (long long)gridDim.x * blockDim.x;
   const int nz = a.z[0] ? (a.z[1] ? 2 : 1) : 0;
   const int chunks = a.d / 8 + nz * (a.r / 8);
-  const int s = (int)(gid / chunks), c = (int)(gid % chunks);
-  if (s >= a.P) return;
-  uint4 v;
-  if (c < a.d / 8) {
-    v = reinterpret_cast<const uint4 *>(a.x16 + (size_t)a.slot_tok[s] * a.d)[c];
-  } else {
-    // eight z values: the sum of the K-split partials in split order, to fp16
-    const int zc = c - a.d / 8, p = zc / (a.r / 8), cc = zc % (a.r / 8);
-    const float *z = a.z[p] + (size_t)a.zidx[p][s] * a.zld + cc * 8;
-    float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
-    for (int sp0 = 0; sp0 < a.zks; sp0 += 8) {
-      // eight splits' loads in flight, then summed in split order
-      float4 l[8], h[8];
+  const long long total = (long long)a.P * chunks;
+  for (long long c0 = gid; c0 < total; c0 += kGatherUnroll * G) {
+    uint4 v[kGatherUnroll];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const bool in = sp0 + u < a.zks;
-        const float4 *q = reinterpret_cast<const float4 *>(z + (size_t)(sp0 + u) * a.zsplit);
-        l[u] = in ? q[0] : make_float4(0.f, 0.f, 0.f, 0.f);
-        h[u] = in ? q[1] : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const long long i = c0 + u * G;
+      if (i < total) v[u] = ext_chunk(a, (int)(i / chunks), (int)(i % chunks));
+    }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        lo.x += l[u].x; lo.y += l[u].y; lo.z += l[u].z; lo.w += l[u].w;
-        hi.x += h[u].x; hi.y += h[u].y; hi.z += h[u].z; hi.w += h[u].w;
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const long long i = c0 + u * G;
+      if (i < total) {
+        const int s = (int)(i / chunks), c = (int)(i % chunks);
+        reinterpret_cast<uint4 *>(a.out + (size_t)s * a.ld)[c] = v[u];
       }
     }
-    __half2 *o = reinterpret_cast<__half2 *>(&v);
-    o[0] = __floats2half2_rn(lo.x, lo.y);
-    o[1] = __floats2half2_rn(lo.z, lo.w);
-    o[2] = __floats2half2_rn(hi.x, hi.y);
-    o[3] = __floats2half2_rn(hi.z, hi.w);
   }
-  reinterpret_cast<uint4 *>(a.out + (size_t)s * a.ld)[c] = v;
 }
 
 // out[t][:] = yshared[t][:] + sum_j sum_split ybuf[split][slot(t,j)][:], in bf16.
 // Fixed summation order, so the result is deterministic.
-__global__ void combine_kernel(CombineArgs a) {
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int d4 = a.d / 4;
   const int t = (int)(gid / d4), c = (int)(gid % d4);
   if (t >= a.T) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (a.yshared) acc = reinterpret_cast<const float4 *>(a.yshared + (size_t)t * a.d)[c];
-  for (int j = 0; j < a.k; ++j) {
-    const int slot = a.slot_of_pair[t * a.k + j];
-    for (int s = 0; s < a.ksplit; ++s) {
-      const float4 v =
-          reinterpret_cast<const float4 *>(a.ybuf + s * a.split_stride + (size_t)slot * a.d)[c];
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  int slot[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) slot[j] = j < a.k ? __ldg(a.slot_of_pair + t * a.k + j) : 0;
+  if (a.ksplit == 1) {
+    // the token's k rows in flight together, summed in slot order
+    float4 v[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < a.k) v[j] = reinterpret_cast<const float4 *>(a.ybuf + (size_t)slot[j] * a.d)[c];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < a.k) {
+        acc.x += v[j].x; acc.y += v[j].y; acc.z += v[j].z; acc.w += v[j].w;
+      }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j >= a.k) break;
+      for (int s = 0; s < a.ksplit; ++s) {
+        const float4 v =
+            reinterpret_cast<const float4 *>(a.ybuf + s * a.split_stride + (size_t)slot[j] * a.d)[c];
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
     }
   }
   __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(a.out + (size_t)t * a.d + c * 4);
