@@ -797,14 +797,12 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
   ca.T = T;
   ca.k = top_k;
   ca.d = li.d_y;
-  ca.ksplit = 1;
-  ca.split_stride = 0;
   ca.slot_of_pair = at<int>(ws, w.slot_of_pair);
   ca.ybuf = at<float>(ws, w.ybuf);
   ca.yshared = yshared;
   ca.out = static_cast<__nv_bfloat16 *>(out);
-  combine_kernel<<<nblocks((long long)T * (li.d_y / 4), 256), 256, 0, stream>>>(ca);
-  TQ_LAUNCHED();
+  if (launch_combine(ca, stream) != cudaSuccess) return TILEQ_ERR_CUDA;
+  count_launches();
   mark(ST_COMBINE, stream);
   return TILEQ_OK;
 }

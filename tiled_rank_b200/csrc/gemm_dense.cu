@@ -13,9 +13,9 @@
 // CTA per SM:
 //   warp 0      producer: 2-D TMA loads (128-byte swizzle) of A and B tiles,
 //               64 K per stage, into a ring of shared-memory stages;
-//   warp 1      allocates tensor memory, issues tcgen05.mma (M = 128, N = BN,
-//               K = 16, both operands in shared memory) into fp32 TMEM
-//               accumulators (two buffers when they fit);
+//   warp 1      allocates tensor memory; one elected lane issues tcgen05.mma
+//               (M = 128, N = BN, K = 16, both operands in shared memory) into
+//               fp32 TMEM accumulators (two buffers when they fit);
 //   warps 2..9  epilogue: tcgen05.ld of the accumulators, scaling and stores,
 //               two warps per TMEM lane quadrant, each half of the columns.
 // Every mbarrier wait is bounded and reports TILEQ_ERR_TIMEOUT.
@@ -132,7 +132,8 @@ __global__ void __launch_bounds__(DenseCfg<MB, BN>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    if (lane == 0) {
+    // The whole warp waits; one elected lane issues the MMAs and commits.
+    {
       constexpr uint32_t idesc = tc::idesc_f16(BN);
       uint32_t qi = 0, wi = 0;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++wi) {
@@ -144,22 +145,29 @@ __global__ void __launch_bounds__(DenseCfg<MB, BN>::THREADS, 1)
           if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
           tc::fence_after();
           const uint64_t bd = tc::sdesc_sw128(smem_addr(stage_b(s)));
+          const uint64_t ad0 = tc::sdesc_sw128(smem_addr(stage_a(s, 0)));
+          if (tc::elect_one()) {
 #pragma unroll
-          for (int j = 0; j < MB; ++j) {
-            const uint64_t ad = tc::sdesc_sw128(smem_addr(stage_a(s, j)));
-            const uint32_t d = tmem + ab * C::ACC_COLS + j * BN;
-            // K steps of 16 inside the swizzle atom: +32 bytes on both start addresses
+            for (int j = 0; j < MB; ++j) {
+              // row block j sits C::A_BYTES further on; K steps of 16 inside the
+              // swizzle atom advance both start addresses by 32 bytes
+              const uint64_t ad = ad0 + (uint64_t)((j * C::A_BYTES) >> 4);
+              const uint32_t d = tmem + ab * C::ACC_COLS + j * BN;
 #pragma unroll
-            for (int kk = 0; kk < DBK / 16; ++kk)
-              mma_ss(d, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) ? 1u : 0u);
+              for (int kk = 0; kk < DBK / 16; ++kk)
+                mma_ss(d, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) ? 1u : 0u);
+            }
+            tc::commit(&q_empty[s]);
           }
-          tc::commit(&q_empty[s]);
+          __syncwarp();
         }
         if (!ok) break;
-        tc::commit(&acc_full[ab]);
+        if (tc::elect_one()) tc::commit(&acc_full[ab]);
+        __syncwarp();
       }
       // all issued MMAs have retired before TMEM is released
-      tc::commit(drain);
+      if (tc::elect_one()) tc::commit(drain);
+      __syncwarp();
       mbar_wait(drain, 0, P.status);
     }
   } else {

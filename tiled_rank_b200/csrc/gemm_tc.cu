@@ -7,8 +7,9 @@
 //   warp 0        producer: bulk copies of the packed 2-bit codes and group
 //                 scales, 2-D TMA tiles of the activation matrix B
 //                 (128-byte swizzle), into a ring of shared-memory stages;
-//   warp 1        allocates tensor memory and issues tcgen05.mma (M = 128 weight
-//                 rows, N = BN items, K = 16) with A in TMEM and B in smem;
+//   warp 1        allocates tensor memory; one elected lane issues tcgen05.mma
+//                 (M = 128 weight rows, N = BN items, K = 16) with A in TMEM and
+//                 B in smem;
 //   warps 2..     dequantisation: each thread owns one of the 128 weight rows,
 //                 decodes its codes into fp16 (w = s * (q - z)) and writes them
 //                 straight into the TMEM A stage with tcgen05.st; after the K
@@ -77,20 +78,18 @@ struct TcCfg {
   static_assert(SA >= 2, "TMEM too small for two A stages");
 };
 
-// rs: the item's row scale (SwiGLU h); c0, c1: the output row's column scales
-// of projection 0 / 1; all loaded by the caller ahead of the stores
-__device__ __forceinline__ void tc_epi_store(const TcArgs &P, int item, int o, float v0, float v1, float rs,
-                                             float c0 = 1.f, float c1 = 1.f) {
+// rs: the item's row scale (SwiGLU h), loaded by the caller ahead of the stores
+__device__ __forceinline__ void tc_epi_store(const TcArgs &P, int item, int o, float v0, float v1, float rs) {
   const size_t idx = (size_t)item * P.ldo + o;
   if (P.epi == EPI_SWIGLU_H) {
     reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(silu_f(v0) * v1 * rs);
   } else if (P.epi == EPI_STORE2_F32) {
-    reinterpret_cast<float *>(P.out[0])[idx] = v0 * c0;
-    reinterpret_cast<float *>(P.out[1])[idx] = v1 * c1;
+    reinterpret_cast<float *>(P.out[0])[idx] = v0;
+    reinterpret_cast<float *>(P.out[1])[idx] = v1;
   } else if (P.epi == EPI_STORE_F16) {
-    reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(v0 * c0);
+    reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(v0);
   } else {
-    reinterpret_cast<float *>(P.out[0])[idx] = v0 * c0;
+    reinterpret_cast<float *>(P.out[0])[idx] = v0;
   }
 }
 
@@ -158,15 +157,13 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
   tc::fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int n_tiles = P.tiles ? *P.tile_count : (P.static_items + BN - 1) / BN;
+  const int n_tiles = *P.tile_count;
   // tile jt: (group, first item, items)
-  auto tile_of = [&](int jt) {
-    return P.tiles ? P.tiles[jt] : make_int4(0, jt * BN, min(BN, P.static_items - jt * BN), 0);
-  };
+  auto tile_of = [&](int jt) { return P.tiles[jt]; };
   const int total = n_tiles * P.m_tiles * P.ksplit;
   const int nkb = P.d_in / BK;
   const int per = (nkb + P.ksplit - 1) / P.ksplit;
-  const int g = P.a_f16 ? BK : P.group;
+  const int g = P.group;
   const int G = P.d_in / g;
   const int gps = g == 64 ? 2 : 1;
   // the K extension runs one projection at a time: n_ext1 stages of 128 columns each
@@ -201,9 +198,6 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
     tc::fence_after();
     const int o = ob * 128 + row;
     const int ldp = P.m_tiles * 128;
-    const int oc = min(o, P.d_out - 1);
-    const float cs0 = P.col_scale[0] ? __ldg(P.col_scale[0] + oc) : 1.f;
-    const float cs1 = P.col_scale[1] ? __ldg(P.col_scale[1] + oc) : 1.f;
 #pragma unroll 1
     for (int c = 0; c < COLS; c += CH) {
       float v[NP][CH];
@@ -231,7 +225,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
         const int n = part * COLS + c + i;
         if (n >= nitems) continue;
         if (P.ksplit == 1) {
-          if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i], rs[i], cs0, cs1);
+          if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i], rs[i]);
         } else {
 #pragma unroll
           for (int p = 0; p < NP; ++p)
@@ -259,9 +253,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
 #pragma unroll
             for (int p = 0; p < NP; ++p)
               r[p] += __ldcg(&P.part[(((size_t)sp * NP + p) * P.part_items + item0 + n) * ldp + oo]);
-          tc_epi_store(P, item0 + n, oo, r[0], r[NP - 1], P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f,
-                       P.col_scale[0] ? __ldg(P.col_scale[0] + oo) : 1.f,
-                       P.col_scale[1] ? __ldg(P.col_scale[1] + oo) : 1.f);
+          tc_epi_store(P, item0 + n, oo, r[0], r[NP - 1], P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f);
         }
         if (leader) P.counters[tile_id] = 0;
       }
@@ -284,13 +276,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
           const int s = qi % C::SQ;
           if (qi >= (uint32_t)C::SQ && !(ok = mbar_wait(&q_empty[s], ((qi / C::SQ) - 1) & 1, P.status))) break;
           TC_TRACE(0, qi);
-          if (st < nmain && P.a_f16) {
-            // fp16 A: the dequantising warps read it from global memory; B only
-            const int kb = kb0 + st;
-            mbar_arrive_expect_tx(&q_full[s], 2 * C::BATOM);
-            for (int a = 0; a < 2; ++a)
-              tc::tma_load_2d(q_b(s) + a * C::BATOM, &P.bmap, kb * BK + a * 64, item0, &q_full[s]);
-          } else if (st < nmain) {
+          if (st < nmain) {
             const int kb = kb0 + st;
             mbar_arrive_expect_tx(&q_full[s], NP * (128 * 32 + gps * 512) + 2 * C::BATOM);
             for (int p = 0; p < NP; ++p) {
@@ -317,7 +303,9 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop and waits on the barriers; one elected lane
+    // issues the MMAs and commits, so the issuing code stays warp-uniform.
+    {
       constexpr uint32_t idesc = tc::idesc_f16(BN);
       uint32_t qi = 0, ai = 0, wi = 0;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++wi) {
@@ -331,43 +319,47 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
         for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
           const int s = qi % C::SQ, sa = ai % C::SA;
           if (!(ok = mbar_wait(&a_full[sa], (ai / C::SA) & 1, P.status))) break;
-          TC_TRACE(4, qi);
+          if (lane == 0) TC_TRACE(4, qi);
           if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
           tc::fence_after();
           const bool ext = st >= nmain;
           // an extension stage feeds one projection (pe); a main stage all of them
           const int pe = ext ? (st - nmain) / n_ext1 : 0;
           const int nk = ext ? (min(BK, P.rank - ((st - nmain) % n_ext1) * BK) + 15) / 16 : BK / 16;
-          // the issuing thread shares its SM sub-partition with dequantising
-          // warps: keep its instruction stream short (one descriptor per stage,
-          // constant offsets: the start-address field counts 16-byte units)
+          // one descriptor per stage, constant offsets (the start-address field
+          // counts 16-byte units)
           const uint64_t bd0 = tc::sdesc_sw128(smem_addr(q_b(s)));
           const uint32_t a0 = tmem + C::NACC * C::ACC_COLS + sa * C::A_COLS;
-          if (!ext) {
+          if (tc::elect_one()) {
+            if (!ext) {
 #pragma unroll
-            for (int p = 0; p < NP; ++p) {
-              const uint32_t d = tmem + ab * C::ACC_COLS + p * BN, a = a0 + p * (BK / 2);
-              tc::mma_ts(d, a, bd0, idesc, first ? 0u : 1u);
+              for (int p = 0; p < NP; ++p) {
+                const uint32_t d = tmem + ab * C::ACC_COLS + p * BN, a = a0 + p * (BK / 2);
+                tc::mma_ts(d, a, bd0, idesc, first ? 0u : 1u);
 #pragma unroll
-              for (int kk = 1; kk < BK / 16; ++kk)
-                tc::mma_ts(d, a + kk * 8, bd0 + (uint64_t)(((kk / 4) * C::BATOM + (kk % 4) * 32) >> 4), idesc, 1u);
+                for (int kk = 1; kk < BK / 16; ++kk)
+                  tc::mma_ts(d, a + kk * 8, bd0 + (uint64_t)(((kk / 4) * C::BATOM + (kk % 4) * 32) >> 4), idesc, 1u);
+              }
+            } else {
+              const uint32_t d = tmem + ab * C::ACC_COLS + pe * BN, a = a0 + pe * (BK / 2);
+              for (int kk = 0; kk < nk; ++kk)
+                tc::mma_ts(d, a + kk * 8, bd0 + (uint64_t)(((kk / 4) * C::BATOM + (kk % 4) * 32) >> 4), idesc,
+                           (first && kk == 0) ? 0u : 1u);
             }
-          } else {
-            const uint32_t d = tmem + ab * C::ACC_COLS + pe * BN, a = a0 + pe * (BK / 2);
-            for (int kk = 0; kk < nk; ++kk)
-              tc::mma_ts(d, a + kk * 8, bd0 + (uint64_t)(((kk / 4) * C::BATOM + (kk % 4) * 32) >> 4), idesc,
-                         (first && kk == 0) ? 0u : 1u);
+            TC_TRACE(5, qi);
+            tc::commit(&a_empty[sa]);
+            tc::commit(&q_empty[s]);
           }
+          __syncwarp();
           first = false;
-          TC_TRACE(5, qi);
-          tc::commit(&a_empty[sa]);
-          tc::commit(&q_empty[s]);
         }
         if (!ok) break;
-        tc::commit(&acc_full[ab]);
+        if (tc::elect_one()) tc::commit(&acc_full[ab]);
+        __syncwarp();
       }
       // all issued MMAs have retired before TMEM is released
-      tc::commit(drain);
+      if (tc::elect_one()) tc::commit(drain);
+      __syncwarp();
       mbar_wait(drain, 0, P.status);
     }
   } else if (warp < 2 + DQW) {
@@ -399,20 +391,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
           for (int c = 0; c < C::KPW / 32; ++c) {   // chunks of 32 K elements = 16 columns
             uint32_t *v = vv[p][c];
             const int k0 = part * C::KPW + c * 32;  // K offset within the stage
-            if (!ext && P.a_f16) {
-              // fp16 weights, row-major: 32 K elements of this thread's row
-              const int ab = P.use_a_blk ? P.a_blk[grp] : 0;
-              const uint4 *ar = reinterpret_cast<const uint4 *>(
-                  P.arow[p] + (((size_t)ab * P.m_tiles + ob) * 128 + row) * P.lda + (size_t)(kb0 + st) * BK + k0);
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint4 q4 = __ldg(ar + j);
-                v[4 * j + 0] = q4.x;
-                v[4 * j + 1] = q4.y;
-                v[4 * j + 2] = q4.z;
-                v[4 * j + 3] = q4.w;
-              }
-            } else if (!ext) {
+            if (!ext) {
               const uint32_t *cw = reinterpret_cast<const uint32_t *>(q_codes(s, p)) + ((k0 / 32) * 128 + row) * 2;
               const int gl = g == 64 ? (k0 >> 6) : 0;
               const __half2 sz = u32_as_h2(q_sz(s, p)[gl * 128 + row]);

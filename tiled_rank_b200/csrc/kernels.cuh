@@ -119,16 +119,6 @@ struct TcArgs {
   const int *tile_count;
   int m_tiles, ksplit, d_out, d_in, group, rank;
   int n_experts;             // experts (blocks) in codes / sz
-  // fp16 A instead of 2-bit codes (tcgen05 kernel only): arow[p] is row-major
-  // [blocks][m_tiles * 128][lda]; the block of a tile is a_blk[group] when
-  // use_a_blk, else 0.  tiles == nullptr: items 0..static_items-1 in tiles of bn.
-  int a_f16;
-  const __half *arow[2];
-  int lda;
-  int use_a_blk;
-  int8_t a_blk[kMaxExperts];
-  int static_items;
-  const float *col_scale[2];  // optional per-output-row scale of projection p (store epilogues)
   int ext_col[2];            // first B column of the K extension of projection p
   const uint4 *codes[2];     // tcgen05: [K][d_out/128][d_in/128][4 slices][128 rows][8 B]
                              // warp MMA: [K][d_out/128][d_in/128][8 warps][32 lanes][16 B]
@@ -222,10 +212,9 @@ struct LrAccArgs {
 };
 
 struct CombineArgs {
-  int T, k, d, ksplit;
-  long long split_stride;
+  int T, k, d;
   const int *slot_of_pair;
-  const float *ybuf;       // [ksplit][P][d]
+  const float *ybuf;       // [P][d]
   const float *yshared;    // [T][d] or null
   __nv_bfloat16 *out;
 };
@@ -251,7 +240,8 @@ __global__ void permute_kernel(PermuteArgs a);
 __global__ void permute_count_kernel(PermuteArgs a);
 __global__ void permute_scatter_kernel(PermuteArgs a);
 __global__ void lr_accumulate_kernel(LrAccArgs a);
-__global__ void combine_kernel(CombineArgs a);
+static_assert(kMaxTopK == 8, "launch_combine instantiates top-k 1..8");
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream);
 __global__ void scale_gather_kernel(ScaleGatherArgs a);
 __global__ void gather_ext_kernel(GatherExtArgs a);
 __global__ void swiglu_kernel(SwigluArgs a);

@@ -102,8 +102,11 @@ __global__ void __launch_bounds__(256) gather_ext_kernel(GatherExtArgs a) {
   }
 }
 
-// out[t][:] = yshared[t][:] + sum_j sum_split ybuf[split][slot(t,j)][:], in bf16.
+// out[t][:] = yshared[t][:] + sum_j ybuf[slot(t,j)][:], in bf16.
 // Fixed summation order, so the result is deterministic.
+// KT: top-k known at compile time (1..kMaxTopK), so the token's k rows are
+// loaded together without spending registers on unused slots.
+template <int KT>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int d4 = a.d / 4;
@@ -111,34 +114,34 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   if (t >= a.T) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (a.yshared) acc = reinterpret_cast<const float4 *>(a.yshared + (size_t)t * a.d)[c];
-  int slot[kMaxTopK];
+  int slot[KT];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) slot[j] = j < a.k ? __ldg(a.slot_of_pair + t * a.k + j) : 0;
-  if (a.ksplit == 1) {
-    // the token's k rows in flight together, summed in slot order
-    float4 v[kMaxTopK];
+  for (int j = 0; j < KT; ++j) slot[j] = __ldg(a.slot_of_pair + t * KT + j);
+  // the token's k rows in flight together, summed in slot order
+  float4 v[KT];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < a.k) v[j] = reinterpret_cast<const float4 *>(a.ybuf + (size_t)slot[j] * a.d)[c];
+  for (int j = 0; j < KT; ++j) v[j] = reinterpret_cast<const float4 *>(a.ybuf + (size_t)slot[j] * a.d)[c];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < a.k) {
-        acc.x += v[j].x; acc.y += v[j].y; acc.z += v[j].z; acc.w += v[j].w;
-      }
-  } else {
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j >= a.k) break;
-      for (int s = 0; s < a.ksplit; ++s) {
-        const float4 v =
-            reinterpret_cast<const float4 *>(a.ybuf + s * a.split_stride + (size_t)slot[j] * a.d)[c];
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
-    }
+  for (int j = 0; j < KT; ++j) {
+    acc.x += v[j].x; acc.y += v[j].y; acc.z += v[j].z; acc.w += v[j].w;
   }
   __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(a.out + (size_t)t * a.d + c * 4);
   o[0] = __floats2bfloat162_rn(acc.x, acc.y);
   o[1] = __floats2bfloat162_rn(acc.z, acc.w);
+}
+
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream) {
+  const unsigned grid = (unsigned)(((long long)a.T * (a.d / 4) + 255) / 256);
+  if (grid == 0) return cudaSuccess;
+  switch (a.k) {
+#define TQ_COMBINE_K(K) \
+  case K: combine_kernel<K><<<grid, 256, 0, stream>>>(a); break;
+    TQ_COMBINE_K(1) TQ_COMBINE_K(2) TQ_COMBINE_K(3) TQ_COMBINE_K(4)
+    TQ_COMBINE_K(5) TQ_COMBINE_K(6) TQ_COMBINE_K(7) TQ_COMBINE_K(8)
+#undef TQ_COMBINE_K
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
 }
 
 // xs[slot][:] = w_slot * x16[token(slot)][:]  (fp16), for the linear layer.
