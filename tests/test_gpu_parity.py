@@ -119,6 +119,8 @@ TINY = [
     # long batches: z, z' and the shared expert on tcgen05 as well
     (synth.SWIGLU, 8, 2, 4, 128, 256, 48, 128, 2, 256, 300),
     (synth.LINEAR, 5, 2, 3, 384, 144, 16, 128, 3, 0, 300),
+    # K = 4096 with ~300 tokens per expert: 256-item tcgen05 tiles and a ragged last tile
+    (synth.LINEAR, 4, 2, 2, 4096, 256, 16, 128, 2, 0, 600),
     # more than 4096 pairs: the multi-CTA sort, its slot tables and grid-row flags
     (synth.SWIGLU, 16, 4, 4, 128, 128, 16, 64, 4, 0, 1500),
     (synth.LINEAR, 12, 3, 4, 128, 128, 16, 64, 3, 0, 1700),

@@ -36,6 +36,7 @@ unsigned gather_blocks(long long chunks) {
 #endif
 constexpr int kQ2PerSm = TILEQ_Q2_PER_SM;
 constexpr int kTcMinTokens = 256;  // dense fp16 products (z, shared expert) move to tcgen05 from here
+constexpr int kWideMinK = 4096;    // 256-item tcgen05 tiles from this K (32 stages per unit) on
 
 struct ProjInfo {
   int d_in, d_out, rank, group, G;
@@ -176,6 +177,7 @@ struct GemmPlan {
   bool tc = false;       // residual GEMM on tcgen05 (wide tiles) rather than warp-level MMA
   bool q2 = false;       // residual GEMM on warp-level MMA (narrow tiles)
   bool partial = false;  // K splits store their own partials (EPI_PARTIAL_F32); no reduction scratch
+  bool wide = false;     // items from the wide tile table (tiles of Plan::bn_wide)
   size_t part_floats() const {
     if (partial) return 0;
     // q2: one [np][bn][128] fp32 partial per (split, tile slot, row block)
@@ -212,6 +214,7 @@ int choose_ksplit(long long ctas, int d_in, int per_sm = 4, int cap = 8) {
 struct Plan {
   int T, k, P;
   int bn_main, slots_main;
+  int bn_wide = 0, slots_wide = 0;  // second tile table (one-projection tcgen05 GEMMs over long K)
   GemmPlan zproj, gateup, zdown, down, linear, sh_gu, sh_down, pe;
 };
 
@@ -221,9 +224,9 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   pl.k = k;
   pl.P = T * k;
   const int P = pl.P;
-  // One tcgen05.mma costs about the same tensor time for any N <= 256, so the
-  // residual GEMMs use it only when an expert sees many tokens; narrow tiles
-  // run on warp-level MMA.
+  // Narrow tiles (<= 32 tokens per expert on average) run faster on warp-level
+  // MMA than on tcgen05 (measured: an M=128 N=16 tcgen05.mma does fewer MACs per
+  // cycle than mma.sync, and the decode then dominates); wider ones on tcgen05.
   const long long avg = P / std::max(1, L->K);
   const bool use_tc = avg > 32;
   pl.bn_main = use_tc ? choose_bn_tc(avg) : choose_bn(avg);
@@ -242,12 +245,27 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
     g.ksplit = choose_ksplit(est_main * g.m_tiles, d_in, use_tc ? 2 : kQ2PerSm);
     return g;
   };
+  // One-projection tcgen05 GEMMs over a long K take 256-item tiles (N = 256:
+  // half the MMA instructions and barrier rounds per FLOP of N = 128); the
+  // accumulator then fills half of tensor memory, so the epilogue no longer
+  // overlaps the next unit, which only pays off when a unit spans many stages.
+  auto widen = [&](GemmPlan &g, int d_in) {
+    if (!use_tc || pl.bn_main != 128 || d_in < kWideMinK) return;
+    pl.bn_wide = 256;
+    pl.slots_wide = cdiv(P, 256) + L->K;
+    g.wide = true;
+    g.bn = 256;
+    g.slots = pl.slots_wide;
+    g.ksplit = choose_ksplit(((long long)std::min(L->K, P) + P / 256) * g.m_tiles, d_in, 2);
+  };
   const ProjInfo &q0 = li.p[0];
   if (L->kind == TILEQ_LINEAR) {
     pl.linear = tc_plan(q0.d_out, q0.d_in, 1);
+    widen(pl.linear, q0.d_in);
   } else {
     pl.gateup = tc_plan(L->d_ff, L->d_model, 2);
     pl.down = tc_plan(L->d_model, L->d_ff, 1);
+    widen(pl.down, L->d_ff);
     if (li.p[2].rank > 0) {
       GemmPlan z;
       z.bn = pl.bn_main;
@@ -315,7 +333,7 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
 struct WsLayout {
   Plan plan;
   size_t status, topk_idx, topk_w, expert_offsets, sorted_pairs, slot_of_pair, slot_tok, slot_w,
-      dest, pcounts, tiles_main, tile_first, tile_counts, counters, part;
+      dest, pcounts, tiles_main, tiles_wide, tile_first, tile_counts, counters, part;
   int n_counters;
   size_t part_zstride;
   size_t zidx[2];
@@ -350,6 +368,7 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool
   w.dest = take(Pz * 4);
   w.pcounts = take((size_t)cdiv(P, kPermChunk) * L->K * 4);
   w.tiles_main = take((size_t)(pl.slots_main + 1) * 16);
+  w.tiles_wide = take((size_t)(pl.slots_wide + 1) * 16);
   w.tile_first = take((L->K + 1) * 4);
   w.tile_counts = take(16);
   if (route_only) {
@@ -499,8 +518,8 @@ tileq_status tc_args(TcArgs *a, const GemmPlan &g, const LayerInfo &li, const Pa
   const ProjInfo &q = li.p[p];
   std::memset(a, 0, sizeof(*a));
   if (!make_map(&a->bmap, bmat, w.plan.P, bcols, bld, g.bn)) return TILEQ_ERR_CUDA;
-  a->tiles = at<int4>(ws, w.tiles_main);
-  a->tile_count = at<int>(ws, w.tile_counts);
+  a->tiles = at<int4>(ws, g.wide ? w.tiles_wide : w.tiles_main);
+  a->tile_count = at<int>(ws, w.tile_counts) + (g.wide ? 1 : 0);
   a->m_tiles = g.m_tiles;
   a->ksplit = g.ksplit;
   a->d_out = q.d_out;
@@ -682,6 +701,8 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   pa.tiles_main = at<int4>(ws, w.tiles_main);
   pa.tile_first_main = at<int>(ws, w.tile_first);
   pa.tile_counts = at<int>(ws, w.tile_counts);
+  pa.bn_wide = w.plan.bn_wide;
+  pa.tiles_wide = at<int4>(ws, w.tiles_wide);
   pa.n_zproj = n_zproj;
   for (int z = 0; z < 2; ++z) {
     if (z < n_zproj) std::memcpy(pa.n_of[z], li.p[zproj_ids[z]].n_of, kMaxExperts);

@@ -214,6 +214,7 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
   const int rw = warp * 16 + r0;  // fragment rows rw and rw + 8 of the 128-row block
   const int cq = (lane & 3) * 2;
 
+  const int ntv = (nitems + 7) / 8;  // n8 blocks holding items of this tile
   float acc[NP][C::NT][4];
 #pragma unroll
   for (int p = 0; p < NP; ++p)
@@ -299,12 +300,15 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
         const uint32_t word = cw[ks >> 1];
         uint32_t af[4];
         dequant_qz_k16((ks & 1) ? (word >> 8) : word, nz, af);
+        // n8 blocks past the tile's last item are skipped (their outputs are never stored)
         if (gstart) {
 #pragma unroll
-          for (int j = 0; j < C::NT; ++j) mma_f16_16816_z(part[j], af, bf[j][0], bf[j][1]);
+          for (int j = 0; j < C::NT; ++j)
+            if (j < ntv) mma_f16_16816_z(part[j], af, bf[j][0], bf[j][1]);
         } else {
 #pragma unroll
-          for (int j = 0; j < C::NT; ++j) mma_f16_16816(part[j], af, bf[j][0], bf[j][1]);
+          for (int j = 0; j < C::NT; ++j)
+            if (j < ntv) mma_f16_16816(part[j], af, bf[j][0], bf[j][1]);
         }
       }
       fold();
@@ -331,7 +335,8 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
         af[2] = __ldg(reinterpret_cast<const unsigned int *>(ur + 8));
         af[3] = __ldg(reinterpret_cast<const unsigned int *>(ur + 8 * a.rank + 8));
 #pragma unroll
-        for (int j = 0; j < C::NT; ++j) mma_f16_16816(acc[p][j], af, bf[j][0], bf[j][1]);
+        for (int j = 0; j < C::NT; ++j)
+          if (j < ntv) mma_f16_16816(acc[p][j], af, bf[j][0], bf[j][1]);
       }
     }
   };

@@ -51,11 +51,12 @@ constexpr int kDqw128 = TILEQ_TC_DQW128;  // dequantising warps of the 128-item 
 
 template <int NP, int BN, int DQW>
 struct TcCfg {
-  // one-projection launches: eight more warps run the epilogue from a second
-  // accumulator buffer while the next unit's MMAs fill the first (two-projection
-  // accumulators fill TMEM, so there the dequantising warps run the epilogue)
+  // one-projection launches: eight more warps run the epilogue, from a second
+  // accumulator buffer while the next unit's MMAs fill the first when BN <= 128
+  // (two-projection accumulators fill TMEM, so there the dequantising warps
+  // run the epilogue)
   static constexpr bool EW = NP == 1;
-  static constexpr int NACC = EW ? 2 : 1;
+  static constexpr int NACC = EW && BN <= 128 ? 2 : 1;
   static constexpr int EPW = EW ? 8 : 0;  // two warps per TMEM lane quadrant
   static constexpr int THREADS = (2 + DQW + EPW) * 32;
   static constexpr int KPW = BK / (DQW / 4);          // K elements per dequant warp per stage
@@ -64,7 +65,7 @@ struct TcCfg {
   static constexpr int BATOM = BN * 128;              // one 64-wide K atom of B (bytes)
   static constexpr int B = 2 * BATOM;                 // 128 K (main) or 128 extension columns of one projection
   static constexpr int QSTAGE = ((CODES + SZ + B) + 1023) / 1024 * 1024;
-  static constexpr int SQ_RAW = (200 * 1024) / QSTAGE;
+  static constexpr int SQ_RAW = (212 * 1024) / QSTAGE;
   static constexpr int SQ = SQ_RAW > 8 ? 8 : (SQ_RAW < 2 ? 2 : SQ_RAW);
   static constexpr int ACC_COLS = NP * BN;
   static constexpr int A_COLS = NP * (BK / 2);          // TMEM columns of one A stage
@@ -496,6 +497,9 @@ cudaError_t launch_tc_bn(const TcArgs &a, int bn, int grid, cudaStream_t s) {
     case 32: return launch_tc_one<NP, 32, 16>(a, grid, s);
     case 64: return launch_tc_one<NP, 64, 16>(a, grid, s);
     case 128: return launch_tc_one<NP, 128, kDqw128>(a, grid, s);
+    case 256:  // one projection only: two 256-column accumulators would fill tensor memory
+      if constexpr (NP == 1) return launch_tc_one<NP, 256, kDqw128>(a, grid, s);
+      return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }
@@ -514,6 +518,7 @@ int tc_smem_bytes(int np, int bn) {
       case 16: return TcCfg<1, 16, 16>::SMEM;
       case 32: return TcCfg<1, 32, 16>::SMEM;
       case 64: return TcCfg<1, 64, 16>::SMEM;
+      case 256: return TcCfg<1, 256, kDqw128>::SMEM;
       default: return TcCfg<1, 128, kDqw128>::SMEM;
     }
   }

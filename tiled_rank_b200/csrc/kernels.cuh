@@ -30,7 +30,9 @@ struct PermuteArgs {
   float *slot_w;           // [P]
   int4 *tiles_main;        // [P/bn + K]
   int *tile_first_main;    // [K+1] first tile of each expert
-  int *tile_counts;        // [1]: main tiles
+  int *tile_counts;        // [0]: main tiles, [1]: wide tiles
+  int bn_wide;             // > 0: also a table of tiles of bn_wide items
+  int4 *tiles_wide;        // [P/bn_wide + K]
   int n_zproj;             // 0, 1 or 2
   int8_t n_of[2][kMaxExperts];
   int *zidx[2];            // slot -> t*N + n (row of the projected [T, N, r] tensor)

@@ -224,6 +224,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
   __syncthreads();
   build_tiles(a.expert_offsets, a.K, a.bn, a.tiles_main, a.tile_counts + 0, a.tile_first_main,
               scratch);
+  if (a.bn_wide > 0)
+    build_tiles(a.expert_offsets, a.K, a.bn_wide, a.tiles_wide, a.tile_counts + 1, nullptr, scratch);
 }
 
 // ---------------------------------------------------------------------------
@@ -296,6 +298,7 @@ __global__ void __launch_bounds__(kPermChunkThreads) permute_scatter_kernel(Perm
   if (c == 0) {
     for (int e = threadIdx.x; e <= K; e += blockDim.x) a.expert_offsets[e] = start[e];
     build_tiles(start, K, a.bn, a.tiles_main, a.tile_counts + 0, a.tile_first_main, scratch);
+    if (a.bn_wide > 0) build_tiles(start, K, a.bn_wide, a.tiles_wide, a.tile_counts + 1, nullptr, scratch);
   }
 
   // 2. this CTA's pairs, split into W contiguous runs, one per warp
