@@ -194,22 +194,27 @@ __global__ void __launch_bounds__(DenseCfg<MB, BN>::THREADS, 1)
         const float *c = P.col_scale[P.pair ? j : 0];
         cs[j] = c ? __ldg(c + min(o[j], P.d_out - 1)) : 1.f;
       }
+      // the TMEM loads of a batch of columns go out together and are waited for
+      // once (each wait lasts about as long as the queued MMAs take to drain)
+      constexpr int BATCH = (MB == 1 ? 32 : 16) < COLS ? (MB == 1 ? 32 : 16) : COLS;
 #pragma unroll 1
-      for (int c = 0; c < COLS; c += CH) {
-        float v[MB][CH];
+      for (int c0 = 0; c0 < COLS; c0 += BATCH) {
+        float v[MB][BATCH];
 #pragma unroll
-        for (int j = 0; j < MB; ++j) {
-          const uint32_t addr = tmem + lane_addr + ab * C::ACC_COLS + j * BN + half * COLS + c;
-          if constexpr (CH == 8) {
-            tc::ld8(addr, v[j]);
-          } else {
-            tc::ld4(addr, v[j]);
+        for (int cc = 0; cc < BATCH; cc += CH)
+#pragma unroll
+          for (int j = 0; j < MB; ++j) {
+            const uint32_t addr = tmem + lane_addr + ab * C::ACC_COLS + j * BN + half * COLS + c0 + cc;
+            if constexpr (CH == 8) {
+              tc::ld8(addr, *reinterpret_cast<float(*)[8]>(&v[j][cc]));
+            } else {
+              tc::ld4(addr, *reinterpret_cast<float(*)[4]>(&v[j][cc]));
+            }
           }
-        }
         tc::wait_ld();
 #pragma unroll
-        for (int i = 0; i < CH; ++i) {
-          const int n = half * COLS + c + i;
+        for (int i = 0; i < BATCH; ++i) {
+          const int n = half * COLS + c0 + i;
           if (n >= nitems) continue;
           const size_t ib = (size_t)(item0 + n) * P.ldo;
           if (P.epi == EPI_SWIGLU_H) {

@@ -65,13 +65,21 @@ struct TcCfg {
   static constexpr int BATOM = BN * 128;              // one 64-wide K atom of B (bytes)
   static constexpr int B = 2 * BATOM;                 // 128 K (main) or 128 extension columns of one projection
   static constexpr int QSTAGE = ((CODES + SZ + B) + 1023) / 1024 * 1024;
-  static constexpr int SQ_RAW = (212 * 1024) / QSTAGE;
+  // one-projection launches with two accumulator buffers stage the epilogue in
+  // shared memory: per column half, two buffers of EBATCH items x 128 rows of
+  // fp32, written out by bulk copies (one per item row) instead of one store
+  // instruction per item (256-item tiles keep the shared memory for a third
+  // input stage)
+  static constexpr int EBATCH = 32;
+  static constexpr int EPI_BYTES = EW && BN <= 128 ? 2 * 2 * EBATCH * 128 * 4 : 0;
+  static constexpr int SQ_RAW = (212 * 1024 - EPI_BYTES) / QSTAGE;
   static constexpr int SQ = SQ_RAW > 8 ? 8 : (SQ_RAW < 2 ? 2 : SQ_RAW);
   static constexpr int ACC_COLS = NP * BN;
   static constexpr int A_COLS = NP * (BK / 2);          // TMEM columns of one A stage
   static constexpr int SA_RAW = (512 - NACC * ACC_COLS) / A_COLS;
   static constexpr int SA = SA_RAW > 4 ? 4 : SA_RAW;
-  static constexpr int BAR_OFF = SQ * QSTAGE;
+  static constexpr int EPI_OFF = SQ * QSTAGE;
+  static constexpr int BAR_OFF = EPI_OFF + EPI_BYTES;
   static constexpr int SMEM_USED = BAR_OFF + (2 * SQ + 2 * SA + 8) * 8 + 64 + 1024;  // + align slack
   // at least half of the SM's shared memory: one CTA per SM, so the 512-column
   // TMEM allocation never waits for another CTA of this kernel
@@ -199,38 +207,47 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
     tc::fence_after();
     const int o = ob * 128 + row;
     const int ldp = P.m_tiles * 128;
+    // the TMEM loads of a batch of columns go out together and are waited for
+    // once: with the next unit's MMAs queued, each wait costs about as long as
+    // the MMA queue takes to drain
+    constexpr int BATCH = (NP == 1 ? 32 : CH) < COLS ? (NP == 1 ? 32 : CH) : COLS;
 #pragma unroll 1
-    for (int c = 0; c < COLS; c += CH) {
-      float v[NP][CH];
+    for (int c0 = 0; c0 < COLS; c0 += BATCH) {
+      float v[NP][BATCH];
 #pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        const uint32_t addr = tmem + lane_addr + ab * C::ACC_COLS + p * BN + part * COLS + c;
-        if constexpr (CH == 8) {
-          tc::ld8(addr, v[p]);
-        } else {
-          tc::ld4(addr, v[p]);
+      for (int cc = 0; cc < BATCH; cc += CH)
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const uint32_t addr = tmem + lane_addr + ab * C::ACC_COLS + p * BN + part * COLS + c0 + cc;
+          if constexpr (CH == 8) {
+            tc::ld8(addr, *reinterpret_cast<float(*)[8]>(&v[p][cc]));
+          } else {
+            tc::ld4(addr, *reinterpret_cast<float(*)[4]>(&v[p][cc]));
+          }
         }
-      }
       tc::wait_ld();
       if (no_k)  // a split past the end of K contributes zeros
 #pragma unroll
         for (int p = 0; p < NP; ++p)
 #pragma unroll
-          for (int i = 0; i < CH; ++i) v[p][i] = 0.f;
-      float rs[CH];  // row scales ahead of the stores
+          for (int i = 0; i < BATCH; ++i) v[p][i] = 0.f;
 #pragma unroll
-      for (int i = 0; i < CH; ++i)
-        rs[i] = P.row_scale ? __ldg(P.row_scale + item0 + min(part * COLS + c + i, nitems - 1)) : 1.f;
+      for (int c = 0; c < BATCH; c += CH) {
+        float rs[CH];  // row scales ahead of the stores
 #pragma unroll
-      for (int i = 0; i < CH; ++i) {
-        const int n = part * COLS + c + i;
-        if (n >= nitems) continue;
-        if (P.ksplit == 1) {
-          if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][i], v[NP - 1][i], rs[i]);
-        } else {
+        for (int i = 0; i < CH; ++i)
+          rs[i] = P.row_scale ? __ldg(P.row_scale + item0 + min(part * COLS + c0 + c + i, nitems - 1)) : 1.f;
 #pragma unroll
-          for (int p = 0; p < NP; ++p)
-            P.part[(((size_t)split * NP + p) * P.part_items + item0 + n) * ldp + o] = v[p][i];
+        for (int i = 0; i < CH; ++i) {
+          const int n = part * COLS + c0 + c + i;
+          if (n >= nitems) continue;
+          if (P.ksplit == 1) {
+            if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][c + i], v[NP - 1][c + i], rs[i]);
+          } else {
+#pragma unroll
+            for (int p = 0; p < NP; ++p)
+              P.part[(((size_t)split * NP + p) * P.part_items + item0 + n) * ldp + o] = v[p][c + i];
+          }
         }
       }
     }
@@ -259,6 +276,56 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
         if (leader) P.counters[tile_id] = 0;
       }
       named_sync(bar_id, nthr);
+    }
+    return true;
+  };
+
+  // ---------------------------------------------------------------- staged epilogue
+  // One-projection fp32 stores (ksplit == 1): the four warps of column half
+  // `part` (one per TMEM lane quadrant) move EBATCH columns at a time from TMEM
+  // to a shared buffer [item][128 rows], then lane i of the half's first warp
+  // writes item i's row segment with one bulk copy.  Two buffers per half: a
+  // buffer is refilled once the bulk copies that read it two batches earlier
+  // are done reading.
+  auto epilogue_staged = [&](uint32_t wi, int ab, int ob, bool no_k, int item0, int nitems, int row, int part,
+                             uint32_t lane_addr, bool leader) -> bool {
+    constexpr int COLS = BN / 2, EB = C::EBATCH < COLS ? C::EBATCH : COLS;
+    static_assert(EB % 8 == 0, "TMEM loads of 8 columns");
+    if (leader) TC_TRACE(7, 2 * wi);
+    if (!mbar_wait(&acc_full[ab], (wi / C::NACC) & 1, P.status)) return false;
+    if (leader) TC_TRACE(7, 2 * wi + 1);
+    tc::fence_after();
+    const bool issuer = (warp & 3) == 0;  // the half's warp of lane quadrant 0 issues the copies
+    const int rows = min(128, P.d_out - ob * 128);
+    float *out = reinterpret_cast<float *>(P.out[0]);
+#pragma unroll 1
+    for (int c0 = 0; c0 < COLS; c0 += EB) {
+      const int b = (int)((wi * (COLS / EB) + c0 / EB) & 1);
+      float *buf = reinterpret_cast<float *>(smem + C::EPI_OFF + (part * 2 + b) * EB * 128 * 4);
+      float v[EB];
+#pragma unroll
+      for (int cc = 0; cc < EB; cc += 8)
+        tc::ld8(tmem + lane_addr + ab * C::ACC_COLS + part * COLS + c0 + cc, *reinterpret_cast<float(*)[8]>(&v[cc]));
+      tc::wait_ld();
+      if (c0 + EB >= COLS) {
+        // the accumulator is in registers: hand it back to the MMA warp
+        tc::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      }
+      // the copies that last read this buffer (two batches ago) are done reading
+      if (issuer) tc::bulk_wait_read<1>();
+      named_sync(3 + part, 128);
+#pragma unroll
+      for (int i = 0; i < EB; ++i) buf[i * 128 + row] = no_k ? 0.f : v[i];
+      tc::fence_proxy_async_smem();
+      named_sync(3 + part, 128);
+      if (issuer) {
+        const int n = part * COLS + c0 + lane;
+        if (lane < EB && n < nitems)
+          tc::bulk_s2g(out + (size_t)(item0 + n) * P.ldo + ob * 128, buf + lane * 128, (uint32_t)rows * 4);
+        tc::bulk_commit();
+      }
     }
     return true;
   };
@@ -377,6 +444,14 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
       stages_of(split, kb0, nmain, next);
       const int4 t = tile_of(jt);
       const int grp = t.x, item0 = t.y, nitems = t.z;
+      // the U_m rows of this unit's extension stages, read from global memory
+      // at the end of the unit: start them towards L2 now
+      for (int e = 0; e < (next ? n_ext1 : 0); ++e)
+#pragma unroll
+        for (int p = 0; p < NP; ++p)
+          if (e * BK + part * C::KPW < P.rank)
+            prefetch_l2(P.u[p] + (((size_t)P.u_blk[p][grp] * P.m_tiles + ob) * 128 + row) * P.rank + e * BK +
+                        part * C::KPW);
       for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
         const int s = qi % C::SQ, sa = ai % C::SA;
         if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
@@ -449,6 +524,9 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
     }
   } else {
     // ============================================================ epilogue warps (NP == 1)
+    // fp32 stores without K splits go through shared memory (rows of 16-byte multiples)
+    const bool staged = C::EPI_BYTES > 0 && P.ksplit == 1 && P.epi == EPI_STORE_F32 && P.d_out % 4 == 0 && P.ldo % 4 == 0 &&
+                        (reinterpret_cast<uintptr_t>(P.out[0]) & 15) == 0;
     const int ew = warp - 2 - DQW;
     const int row = (warp & 3) * 32 + lane;  // this warp's TMEM lane quadrant
     const int epart = ew >> 2;                 // column half
@@ -459,11 +537,18 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
       decode(w, jt, ob, split);
       stages_of(split, kb0, nmain, next);
       const int4 t = tile_of(jt);
-      if (!(ok = epilogue(std::integral_constant<int, BN / (C::EW ? C::EPW / 4 : 1)>{}, wi, wi % C::NACC, jt, ob, split,
-                          nmain + next == 0, t.y, t.z, row, epart, lane_addr, 2, C::EPW * 32, ew * 32 + lane,
-                          ew == 0 && lane == 0)))
+      if (staged) {
+        if (!(ok = epilogue_staged(wi, wi % C::NACC, ob, nmain + next == 0, t.y, t.z, row, epart, lane_addr,
+                                   ew == 0 && lane == 0)))
+          break;
+      } else if (!(ok = epilogue(std::integral_constant<int, BN / (C::EW ? C::EPW / 4 : 1)>{}, wi, wi % C::NACC, jt,
+                                 ob, split, nmain + next == 0, t.y, t.z, row, epart, lane_addr, 2, C::EPW * 32,
+                                 ew * 32 + lane, ew == 0 && lane == 0))) {
         break;
+      }
     }
+    // every bulk copy of this thread has landed before the CTA exits
+    if (staged && (warp & 3) == 0) tc::bulk_wait_all();
   }
 
   __syncwarp();
