@@ -1049,7 +1049,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       la.zld = pad128(q.rank);
       la.zks = plan.zproj.ksplit;
       la.zsplit = (long long)T * layer->N * pad128(q.rank);
-      lr_accumulate_kernel<<<nblocks((long long)plan.P * q.rank, 256), 256, 0, stream>>>(la);
+      lr_accumulate_kernel<<<nblocks((long long)plan.P * 32, 256), 256, 0, stream>>>(la);
       TQ_LAUNCHED();
     } else {
       mark(ST_ZPROJ, stream);
@@ -1160,7 +1160,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       la.zslot = at<float>(ws, w.zs);
       la.zks = plan.zdown.ksplit;
       la.zsplit = (long long)plan.P * qd.rank;
-      lr_accumulate_kernel<<<nblocks((long long)plan.P * qd.rank, 256), 256, 0, stream>>>(la);
+      lr_accumulate_kernel<<<nblocks((long long)plan.P * 32, 256), 256, 0, stream>>>(la);
       TQ_LAUNCHED();
     } else {
       mark(ST_ZDOWN, stream);

@@ -14,33 +14,71 @@ namespace tileq {
 // buffer accumulates them per grid row, so that the shared left factor U_m is
 // applied once per (token, row); here the buffer lives in the K-extension
 // columns of the next GEMM's activation matrix.
-__global__ void lr_accumulate_kernel(LrAccArgs a) {
-  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const int s = (int)(gid / a.r), i = (int)(gid % a.r);
-  if (s >= a.P) return;
-  float acc = 0.f;
-  if (a.aidx[s] >= 0) {
-    const int p0 = a.sorted_pairs[s];
-    const int t = p0 / a.k;
-    const int m = a.m_of[a.topk_idx[p0]];
-    for (int j = 0; j < a.k; ++j) {
-      const int p = t * a.k + j;
-      if (a.m_of[a.topk_idx[p]] != m) continue;
-      const int slot = a.slot_of_pair[p];
-      const float *z = a.zslot ? a.zslot + (size_t)slot * a.r + i : a.zcol + (size_t)a.zidx[slot] * a.zld + i;
-      float zz = 0.f;
-      for (int sp0 = 0; sp0 < a.zks; sp0 += 8) {
-        // eight splits' loads in flight, then summed in split order
-        float t[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) t[u] = sp0 + u < a.zks ? z[(size_t)(sp0 + u) * a.zsplit] : 0.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) zz += t[u];
-      }
-      acc += a.zslot ? zz : a.topk_w[p] * zz;
+// One warp per slot.  The token's k pairs are looked up once (lane j holds
+// pair j's slot, weight and z row, or -1 outside grid row m) and broadcast;
+// each lane then sums four consecutive elements over the pairs, all pairs'
+// loads in flight, in pair order and split order.
+__global__ void __launch_bounds__(256) lr_accumulate_kernel(LrAccArgs a) {
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= a.P) return;
+  const int s = (int)gw;
+  const int r4 = a.r / 4;
+  __half2 *dst = reinterpret_cast<__half2 *>(a.out + (size_t)s * a.ld + a.col);
+  if (a.aidx[s] < 0) {
+    for (int c = lane; c < r4; c += 32) {
+      dst[2 * c] = __floats2half2_rn(0.f, 0.f);
+      dst[2 * c + 1] = __floats2half2_rn(0.f, 0.f);
+    }
+    return;
+  }
+  const int p0 = a.sorted_pairs[s];
+  const int t = p0 / a.k;
+  const int m = a.m_of[a.topk_idx[p0]];
+  int my_slot = -1, my_row = 0;
+  float my_w = 0.f;
+  if (lane < a.k) {
+    const int p = t * a.k + lane;
+    if (a.m_of[a.topk_idx[p]] == m) {
+      my_slot = a.slot_of_pair[p];
+      my_w = a.topk_w[p];
+      my_row = a.zslot ? my_slot : a.zidx[my_slot];
     }
   }
-  a.out[(size_t)s * a.ld + a.col + i] = __float2half_rn(acc);
+  int slot[kMaxTopK], zrow[kMaxTopK];
+  float w[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    slot[j] = __shfl_sync(0xffffffffu, my_slot, j);
+    zrow[j] = __shfl_sync(0xffffffffu, my_row, j);
+    w[j] = __shfl_sync(0xffffffffu, my_w, j);
+  }
+  const float *zbase = a.zslot ? a.zslot : a.zcol;
+  const size_t zstride = a.zslot ? (size_t)a.r : (size_t)a.zld;
+  for (int c = lane; c < r4; c += 32) {
+    float4 z[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      z[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < a.k && slot[j] >= 0) {
+        const float *zp = zbase + (size_t)zrow[j] * zstride + 4 * c;
+        for (int sp = 0; sp < a.zks; ++sp) {  // K-split partials in split order
+          const float4 q = *reinterpret_cast<const float4 *>(zp + (size_t)sp * a.zsplit);
+          z[j].x += q.x; z[j].y += q.y; z[j].z += q.z; z[j].w += q.w;
+        }
+      }
+    }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j < a.k && slot[j] >= 0) {
+        const float f = a.zslot ? 1.f : w[j];
+        acc.x += f * z[j].x; acc.y += f * z[j].y; acc.z += f * z[j].z; acc.w += f * z[j].w;
+      }
+    }
+    dst[2 * c] = __floats2half2_rn(acc.x, acc.y);
+    dst[2 * c + 1] = __floats2half2_rn(acc.z, acc.w);
+  }
 }
 
 // x_ext[s] = [x16[tok(s)] | z0[zidx0[s]] | z1[zidx1[s]]]  (fp16, 8-element chunks)
