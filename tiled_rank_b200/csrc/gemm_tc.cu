@@ -71,7 +71,10 @@ struct TcCfg {
   // instruction per item (256-item tiles keep the shared memory for a third
   // input stage)
   static constexpr int EBATCH = 32;
-  static constexpr int EPI_BYTES = EW && BN <= 128 ? 2 * 2 * EBATCH * 128 * 4 : 0;
+  // two-projection launches (SwiGLU h in fp16, written by the dequantising
+  // warps): per column quarter two buffers of 8 items x 128 rows of fp16
+  static constexpr int EPI_BYTES = EW ? (BN <= 128 ? 2 * 2 * EBATCH * 128 * 4 : 0)
+                                      : (BN >= 64 ? 4 * 2 * 8 * 128 * 2 : 0);
   static constexpr int SQ_RAW = (212 * 1024 - EPI_BYTES) / QSTAGE;
   static constexpr int SQ = SQ_RAW > 8 ? 8 : (SQ_RAW < 2 ? 2 : SQ_RAW);
   static constexpr int ACC_COLS = NP * BN;
@@ -330,6 +333,64 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
     return true;
   };
 
+  // Two-projection SwiGLU epilogue (ksplit == 1) by the 16 dequantising warps:
+  // the four warps of column quarter `part` move 8 columns of both
+  // accumulators at a time from TMEM, store h = silu(g) * u * w in fp16 into a
+  // shared buffer [item][128 rows], and lane i of the quarter's first warp
+  // writes item i's row segment with one bulk copy (two buffers per quarter).
+  auto epilogue_swiglu_staged = [&](uint32_t wi, int ob, bool no_k, int item0, int nitems, int row, int part,
+                                    uint32_t lane_addr, bool leader) -> bool {
+    if constexpr (C::EW || BN < 64) {
+      return false;  // not used by these instantiations
+    } else {
+    constexpr int COLS = BN / 4, EB = 8;
+    static_assert(COLS % EB == 0, "column quarter in batches of 8");
+    if (leader) TC_TRACE(7, 2 * wi);
+    if (!mbar_wait(&acc_full[0], wi & 1, P.status)) return false;
+    if (leader) TC_TRACE(7, 2 * wi + 1);
+    tc::fence_after();
+    const bool issuer = (warp & 3) == 2;  // dequantising warps 2, 6, 10, 14: lane quadrant 2
+    const int rows = min(128, P.d_out - ob * 128);
+    __half *out = reinterpret_cast<__half *>(P.out[0]);
+#pragma unroll 1
+    for (int c0 = 0; c0 < COLS; c0 += EB) {
+      const int b = (int)((wi * (COLS / EB) + c0 / EB) & 1);
+      __half *buf = reinterpret_cast<__half *>(smem + C::EPI_OFF + (part * 2 + b) * EB * 128 * 2);
+      float g[EB], u[EB];
+#pragma unroll
+      for (int cc = 0; cc < EB; cc += 8) {
+        tc::ld8(tmem + lane_addr + part * COLS + c0 + cc, *reinterpret_cast<float(*)[8]>(&g[cc]));
+        tc::ld8(tmem + lane_addr + BN + part * COLS + c0 + cc, *reinterpret_cast<float(*)[8]>(&u[cc]));
+      }
+      tc::wait_ld();
+      if (c0 + EB >= COLS) {
+        // both accumulators are in registers: the next unit's MMAs may start
+        tc::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[0]);
+      }
+      float rs[EB];
+#pragma unroll
+      for (int i = 0; i < EB; ++i)
+        rs[i] = P.row_scale ? __ldg(P.row_scale + item0 + min(part * COLS + c0 + i, nitems - 1)) : 1.f;
+      if (issuer) tc::bulk_wait_read<1>();
+      named_sync(5 + part, 128);
+#pragma unroll
+      for (int i = 0; i < EB; ++i)
+        buf[i * 128 + row] = __float2half_rn(no_k ? 0.f : silu_f(g[i]) * u[i] * rs[i]);
+      tc::fence_proxy_async_smem();
+      named_sync(5 + part, 128);
+      if (issuer) {
+        const int n = part * COLS + c0 + lane;
+        if (lane < EB && n < nitems)
+          tc::bulk_s2g(out + (size_t)(item0 + n) * P.ldo + ob * 128, buf + lane * 128, (uint32_t)rows * 2);
+        tc::bulk_commit();
+      }
+    }
+    return true;
+    }
+  };
+
   if (warp == 0) {
     // ============================================================ producer
     if (lane == 0) {
@@ -432,6 +493,9 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
     }
   } else if (warp < 2 + DQW) {
     // ============================================================ dequant (+ epilogue when NP == 2)
+    const bool swiglu_staged = !C::EW && C::EPI_BYTES > 0 && DQW == 16 && P.ksplit == 1 &&
+                               P.epi == EPI_SWIGLU_H && P.d_out % 8 == 0 && P.ldo % 8 == 0 &&
+                               (reinterpret_cast<uintptr_t>(P.out[0]) & 15) == 0;
     const int dw = warp - 2;
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int part = dw >> 2;                  // K slice (dequant) / column slice (epilogue)
@@ -517,11 +581,19 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
       if (!ok) break;
 
       if (!C::EW) {
-        if (!(ok = epilogue(std::integral_constant<int, BN / (DQW / 4)>{}, wi, 0, jt, ob, split, nmain + next == 0,
-                            item0, nitems, row, part, lane_addr, 1, DQW * 32, dw * 32 + lane, dw == 0 && lane == 0)))
+        if (swiglu_staged) {
+          if (!(ok = epilogue_swiglu_staged(wi, ob, nmain + next == 0, item0, nitems, row, part, lane_addr,
+                                            dw == 0 && lane == 0)))
+            break;
+        } else if (!(ok = epilogue(std::integral_constant<int, BN / (DQW / 4)>{}, wi, 0, jt, ob, split,
+                                   nmain + next == 0, item0, nitems, row, part, lane_addr, 1, DQW * 32,
+                                   dw * 32 + lane, dw == 0 && lane == 0))) {
           break;
+        }
       }
     }
+    // every bulk copy of this thread has landed before the CTA exits
+    if (swiglu_staged && (warp & 3) == 2) tc::bulk_wait_all();
   } else {
     // ============================================================ epilogue warps (NP == 1)
     // fp32 stores without K splits go through shared memory (rows of 16-byte multiples)
