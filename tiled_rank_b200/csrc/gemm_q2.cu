@@ -253,66 +253,73 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
   };
 
   // one 128-wide block h of a main stage: 16 rows x 128 K of every projection,
-  // one projection after the other (fewer live registers; B fragments are
-  // re-read from shared memory for the second projection)
+  // the projections interleaved per k16 step (one B fragment load serves both,
+  // and their MMA chains are independent)
   auto block_main = [&](int s, int h) {
     const uint32_t bs = smem_addr(st_b(s));
+    uint32_t cw[NP][4];
+    float part[NP][C::NT][4];
+    __half2 nz[NP][4];
+    float sc0[NP], sc8[NP];
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-      uint32_t cw[4];
       const uint32_t sa = smem_addr(st_a(s, p, h)) + (warp * 32 + lane) * 16;
       asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
-                   : "=r"(cw[0]), "=r"(cw[1]), "=r"(cw[2]), "=r"(cw[3])
+                   : "=r"(cw[p][0]), "=r"(cw[p][1]), "=r"(cw[p][2]), "=r"(cw[p][3])
                    : "r"(sa));
-      float part[C::NT][4];
-      __half2 nz[4];
-      float sc0, sc8;
+    }
+    auto group_consts = [&](int p, int sub) {
       const uint32_t zs = smem_addr(st_z(s, p, h)) + rw * 4;
-      auto group_consts = [&](int sub) {
-        uint32_t u0, u8;
-        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(u0) : "r"(zs + sub * 512));
-        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(u8) : "r"(zs + sub * 512 + 32));
-        const __half2 w0 = u32_as_h2(u0), w8 = u32_as_h2(u8);
-        const __half2 z0 = __high2half2(w0), z8 = __high2half2(w8);
-        nz[0] = __hsub2(u32_as_h2(0xE400E400u), z0);  // -(1024 + z)
-        nz[1] = __hsub2(u32_as_h2(0xDC00DC00u), z8);  // -(256 + z)
-        nz[2] = __hsub2(u32_as_h2(0xD400D400u), z0);  // -(64 + z)
-        nz[3] = __hsub2(u32_as_h2(0xCC00CC00u), z8);  // -(16 + z)
-        sc0 = __low2float(w0);
-        sc8 = __low2float(w8);
-      };
-      auto fold = [&]() {
+      uint32_t u0, u8;
+      asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(u0) : "r"(zs + sub * 512));
+      asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(u8) : "r"(zs + sub * 512 + 32));
+      const __half2 w0 = u32_as_h2(u0), w8 = u32_as_h2(u8);
+      const __half2 z0 = __high2half2(w0), z8 = __high2half2(w8);
+      nz[p][0] = __hsub2(u32_as_h2(0xE400E400u), z0);
+      nz[p][1] = __hsub2(u32_as_h2(0xDC00DC00u), z8);
+      nz[p][2] = __hsub2(u32_as_h2(0xD400D400u), z0);
+      nz[p][3] = __hsub2(u32_as_h2(0xCC00CC00u), z8);
+      sc0[p] = __low2float(w0);
+      sc8[p] = __low2float(w8);
+    };
+    auto fold = [&](int p) {
 #pragma unroll
-        for (int j = 0; j < C::NT; ++j)
+      for (int j = 0; j < C::NT; ++j)
 #pragma unroll
-          for (int v = 0; v < 4; ++v) acc[p][j][v] = fmaf(v < 2 ? sc0 : sc8, part[j][v], acc[p][j][v]);
-      };
-      group_consts(0);
+        for (int v = 0; v < 4; ++v) acc[p][j][v] = fmaf(v < 2 ? sc0[p] : sc8[p], part[p][j][v], acc[p][j][v]);
+    };
 #pragma unroll
-      for (int ks = 0; ks < QBLK / 16; ++ks) {
-        const bool gstart = ks == 0 || (g64 && ks == 4);
-        if (ks == 4 && g64) {
-          fold();
-          group_consts(1);
+    for (int p = 0; p < NP; ++p) group_consts(p, 0);
+#pragma unroll
+    for (int ks = 0; ks < QBLK / 16; ++ks) {
+      const bool gstart = ks == 0 || (g64 && ks == 4);
+      if (ks == 4 && g64) {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          fold(p);
+          group_consts(p, 1);
         }
-        uint32_t bf[C::NT][2];
-        load_b(bs, 2 * h, ks, bf);
-        const uint32_t word = cw[ks >> 1];
+      }
+      uint32_t bf[C::NT][2];
+      load_b(bs, 2 * h, ks, bf);
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const uint32_t word = cw[p][ks >> 1];
         uint32_t af[4];
-        dequant_qz_k16((ks & 1) ? (word >> 8) : word, nz, af);
-        // n8 blocks past the tile's last item are skipped (their outputs are never stored)
+        dequant_qz_k16((ks & 1) ? (word >> 8) : word, nz[p], af);
         if (gstart) {
 #pragma unroll
           for (int j = 0; j < C::NT; ++j)
-            if (j < ntv) mma_f16_16816_z(part[j], af, bf[j][0], bf[j][1]);
+            if (j < ntv) mma_f16_16816_z(part[p][j], af, bf[j][0], bf[j][1]);
         } else {
 #pragma unroll
           for (int j = 0; j < C::NT; ++j)
-            if (j < ntv) mma_f16_16816(part[j], af, bf[j][0], bf[j][1]);
+            if (j < ntv) mma_f16_16816(part[p][j], af, bf[j][0], bf[j][1]);
         }
       }
-      fold();
     }
+#pragma unroll
+    for (int p = 0; p < NP; ++p) fold(p);
   };
 
   // one extension stage: A = rows of U_m (fp16, read from global), B = 128
