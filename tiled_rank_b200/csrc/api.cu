@@ -1093,7 +1093,10 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       ga.zidx[1] = at<int>(ws, w.zidx[1]);
       ga.zld = pad128(qg.rank);
       ga.out = xext;
-      const long long chunks = (long long)plan.P * (D / 8 + (lr_gu ? 2 * qg.rank / 8 : 0));
+      ga.T = T;
+      ga.k = top_k;
+      ga.slot_of_pair = at<int>(ws, w.slot_of_pair);
+      const long long chunks = (long long)T * (D / 8) + (long long)plan.P * (lr_gu ? 2 * qg.rank / 8 : 0);
       gather_ext_kernel<<<gather_blocks(chunks), 256, 0, stream>>>(ga);
       TQ_LAUNCHED();
     }
@@ -1325,7 +1328,10 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     ga.slot_tok = at<int>(ws, w.slot_tok);
     ga.x16 = at<__half>(ws, w.x16);
     ga.out = xext;
-    gather_ext_kernel<<<gather_blocks((long long)plan.P * (D / 8)), 256, 0, stream>>>(ga);
+    ga.T = T;
+    ga.k = top_k;
+    ga.slot_of_pair = at<int>(ws, w.slot_of_pair);
+    gather_ext_kernel<<<gather_blocks((long long)T * (D / 8)), 256, 0, stream>>>(ga);
     TQ_LAUNCHED();
     Residual r;
     r.np = 2;

@@ -179,6 +179,8 @@ int tc_smem_bytes(int np, int bn);
 // ---------------------------------------------------------------- misc
 struct GatherExtArgs {
   int P, d, r, ld;            // x_ext[s] = [x16[tok(s)] (d) | z0[zidx0[s]] (r) | z1[zidx1[s]] (r)]
+  int T, k;                   // x part token-major: row t read once, written to its k slots
+  const int *slot_of_pair;    // [T*k]
   int zld;                    // row stride of z0 / z1 (elements)
   int zks;                    // z0 / z1 are fp32 partials [zks][rows][zld], summed in order
   long long zsplit;           // elements between two partials

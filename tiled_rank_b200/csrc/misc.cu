@@ -82,11 +82,9 @@ __global__ void __launch_bounds__(256) lr_accumulate_kernel(LrAccArgs a) {
 }
 
 // x_ext[s] = [x16[tok(s)] | z0[zidx0[s]] | z1[zidx1[s]]]  (fp16, 8-element chunks)
-// One 16-byte chunk of row s of the activation matrix: x_t, or eight z values
-// (the sum of the K-split partials in split order, to fp16).
-__device__ __forceinline__ uint4 ext_chunk(const GatherExtArgs &a, int s, int c) {
-  if (c < a.d / 8) return __ldg(reinterpret_cast<const uint4 *>(a.x16 + (size_t)a.slot_tok[s] * a.d) + c);
-  const int zc = c - a.d / 8, p = zc / (a.r / 8), cc = zc % (a.r / 8);
+// Eight z values of row s: the sum of the K-split partials in split order, to fp16.
+__device__ __forceinline__ uint4 z_chunk(const GatherExtArgs &a, int s, int zc) {
+  const int p = zc / (a.r / 8), cc = zc % (a.r / 8);
   const float *z = a.z[p] + (size_t)a.zidx[p][s] * a.zld + cc * 8;
   float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
   for (int sp0 = 0; sp0 < a.zks; sp0 += 8) {
@@ -114,26 +112,41 @@ __device__ __forceinline__ uint4 ext_chunk(const GatherExtArgs &a, int s, int c)
   return v;
 }
 
-// Grid-stride over the P * chunks 16-byte chunks, kGatherUnroll of them per
-// thread in flight.
+// Grid-stride over T * (d/8) token-major x chunks (each read once and written
+// to the token's k slot rows), then P * (nz*r/8) slot-major z chunks;
+// kGatherUnroll items per thread in flight.
 __global__ void __launch_bounds__(256) gather_ext_kernel(GatherExtArgs a) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long G = (long long)gridDim.x * blockDim.x;
   const int nz = a.z[0] ? (a.z[1] ? 2 : 1) : 0;
-  const int chunks = a.d / 8 + nz * (a.r / 8);
-  const long long total = (long long)a.P * chunks;
+  const int xc = a.d / 8, zcn = nz * (a.r / 8);
+  const long long nx = (long long)a.T * xc;
+  const long long total = nx + (long long)a.P * zcn;
   for (long long c0 = gid; c0 < total; c0 += kGatherUnroll * G) {
     uint4 v[kGatherUnroll];
 #pragma unroll
     for (int u = 0; u < kGatherUnroll; ++u) {
       const long long i = c0 + u * G;
-      if (i < total) v[u] = ext_chunk(a, (int)(i / chunks), (int)(i % chunks));
+      if (i < nx) {
+        const int t = (int)(i / xc), c = (int)(i % xc);
+        v[u] = __ldg(reinterpret_cast<const uint4 *>(a.x16 + (size_t)t * a.d) + c);
+      } else if (i < total) {
+        const long long iz = i - nx;
+        v[u] = z_chunk(a, (int)(iz / zcn), (int)(iz % zcn));
+      }
     }
 #pragma unroll
     for (int u = 0; u < kGatherUnroll; ++u) {
       const long long i = c0 + u * G;
-      if (i < total) {
-        const int s = (int)(i / chunks), c = (int)(i % chunks);
+      if (i < nx) {
+        const int t = (int)(i / xc), c = (int)(i % xc);
+        for (int j = 0; j < a.k; ++j) {
+          const int s = a.slot_of_pair[t * a.k + j];
+          reinterpret_cast<uint4 *>(a.out + (size_t)s * a.ld)[c] = v[u];
+        }
+      } else if (i < total) {
+        const long long iz = i - nx;
+        const int s = (int)(iz / zcn), c = xc + (int)(iz % zcn);
         reinterpret_cast<uint4 *>(a.out + (size_t)s * a.ld)[c] = v[u];
       }
     }
