@@ -201,6 +201,44 @@ tileq_status tileq_route_static(const float *router_logits, int T, int K, int to
 
 /* Synchronously read (and clear) the device status word in `ws`.
  * *status receives TILEQ_OK or the first device error recorded. */
+/* ---------------------------------------------------------------------------
+ * Global low-rank decomposition of W_big by Gaussian sketching (TileQ summary,
+ * section 2.1, step 5 "Quantization": the large tiled matrix W_big undergoes a
+ * global low-rank decomposition approximated via Gaussian sketching; its
+ * shared factors U, Sigma, V are what tileq_moe_forward reads).
+ *
+ * W_big [M*d_out, N*d_in] holds expert k's weights in grid block
+ * (m, n) = (grid_assign[k] / N, grid_assign[k] % N).  Steps (randomised range
+ * finder, then the SVD of the projected matrix):
+ *   Y = W_big Omega;  Q = an orthonormal basis of range(Y);  B = Q^T W_big;
+ *   B = U_B diag(s) V_B^T;  U = Q U_B[:, :r], Sigma = s[:r], V = V_B[:, :r].
+ * U diag(Sigma) V^T is the rank-r truncated SVD of Q Q^T W_big.  The GPU
+ * computes the basis and the SVD from fp64 Jacobi eigen-decompositions of the
+ * l x l Gram matrices Y^T Y and B B^T; products are fp32.
+ * ------------------------------------------------------------------------- */
+#define TILEQ_SKETCH_MAX_L 160
+
+typedef struct {
+  int K, M, N;                  /* K == M * N <= 64: every grid cell holds one expert */
+  int d_out, d_in;
+  const void *w;                /* device, bf16 [K][d_out][d_in], expert k's weights */
+  const int32_t *grid_assign;   /* host, [K], a bijection onto the cells 0..K-1 */
+} tileq_wbig;
+
+/* Workspace bytes of tileq_sketch_lowrank.  l: sketch width (even, 2..
+ * TILEQ_SKETCH_MAX_L), r: rank (1..l).  TILEQ_ERR_UNSUPPORTED for shapes outside
+ * these limits, TILEQ_ERR_INVALID_ARG for a grid_assign that is not a bijection. */
+tileq_status tileq_sketch_workspace_size(const tileq_wbig *w, int l, int r, size_t *bytes);
+
+/* omega: device fp32 [N*d_in][l], the Gaussian test matrix (the caller draws
+ * it).  Outputs (device, overwritten): U fp32 [M*d_out][r], sigma fp32 [r]
+ * (descending), V fp32 [N*d_in][r]; the columns of U and V pair up (the sign
+ * of each pair is arbitrary).  ws: device workspace of at least the queried
+ * size.  Asynchronous on stream; the host validates before any launch. */
+tileq_status tileq_sketch_lowrank(const tileq_wbig *w, const float *omega, int l, int r, float *U,
+                                  float *sigma, float *V, void *ws, size_t ws_bytes,
+                                  tileq_stream_t stream);
+
 tileq_status tileq_device_status(void *ws, int *status, tileq_stream_t stream);
 
 /* Self-test of the bounded device wait: launches one block that waits on an

@@ -174,3 +174,45 @@ def test_route_static_scratch_covers_max_pairs(L):
         for k in (1, 2, 4, 8):
             if k <= K:
                 assert L.tileq_workspace_size(c, max_pairs // k, k) <= 6 << 20, (K, k)
+
+
+def test_wbig_layout_matches_c(L, tmp_path):
+    src = tmp_path / "wbig.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "tileq.h"\n'
+                   'int main(void){printf("%zu %zu %zu %d\\n", sizeof(tileq_wbig), offsetof(tileq_wbig, w),'
+                   'offsetof(tileq_wbig, grid_assign), TILEQ_SKETCH_MAX_L); return 0;}\n')
+    exe = tmp_path / "wbig"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
+    assert got == [ctypes.sizeof(L.tileq_wbig), L.tileq_wbig.w.offset, L.tileq_wbig.grid_assign.offset,
+                   L.TILEQ_SKETCH_MAX_L]
+
+
+def _wbig(L, M, N, d_out, d_in, grid=None):
+    K = M * N
+    g = np.ascontiguousarray(np.arange(K) if grid is None else grid, dtype=np.int32)
+    w = L.tileq_wbig()
+    w.K, w.M, w.N, w.d_out, w.d_in = K, M, N, d_out, d_in
+    w.w = 16  # never dereferenced by the host checks
+    w.grid_assign = g.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    w._keep = g
+    return w
+
+
+def test_sketch_workspace_and_validation(L):
+    w = _wbig(L, 2, 4, 256, 128)
+    n = L.tileq_sketch_workspace_size(w, 24, 16)
+    R, C, l, r = 2 * 256, 4 * 128, 24, 16
+    assert n >= (2 * R * l + C * l) * 4 + 16 * l * l * 8
+    with pytest.raises(L.TileQError):
+        L.tileq_sketch_workspace_size(w, 23, 16)          # odd sketch width
+    with pytest.raises(L.TileQError):
+        L.tileq_sketch_workspace_size(w, L.TILEQ_SKETCH_MAX_L + 2, 16)
+    with pytest.raises(L.TileQError):
+        L.tileq_sketch_workspace_size(w, 24, 25)          # rank above the sketch width
+    with pytest.raises(L.TileQError):
+        L.tileq_sketch_workspace_size(_wbig(L, 2, 2, 64, 64, grid=[0, 1, 1, 3]), 8, 4)  # not a bijection
+    bad = _wbig(L, 2, 2, 64, 64)
+    bad.K = 3
+    with pytest.raises(L.TileQError):
+        L.tileq_sketch_workspace_size(bad, 8, 4)          # K != M*N

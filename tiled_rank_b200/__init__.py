@@ -9,5 +9,6 @@ from ._lib import (  # noqa: F401
     tileq_packed_per_expert_size, tileq_packed_size, tileq_route, tileq_route_static,
     tileq_selftest_bounded_wait,
     tileq_workspace_size, tileq_set_stage_events, tileq_launch_count,
+    tileq_wbig, tileq_sketch_workspace_size, tileq_sketch_lowrank,
 )
 from .layer import DeviceLayer  # noqa: F401

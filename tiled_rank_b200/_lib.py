@@ -29,7 +29,9 @@ EXPORTS = (
     "tileq_moe_forward", "tileq_packed_per_expert_size", "tileq_pack_per_expert",
     "tileq_moe_forward_unfused", "tileq_route", "tileq_route_static", "tileq_device_status",
     "tileq_selftest_bounded_wait", "tileq_set_stage_events", "tileq_launch_count",
+    "tileq_sketch_workspace_size", "tileq_sketch_lowrank",
 )
+TILEQ_SKETCH_MAX_L = 160
 
 
 class TileQError(RuntimeError):
@@ -63,6 +65,14 @@ class tileq_route_out(ctypes.Structure):
                 ("expert_offsets", ctypes.c_void_p), ("sorted_pairs", ctypes.c_void_p)]
 
 
+class tileq_wbig(ctypes.Structure):
+    _fields_ = [
+        ("K", ctypes.c_int), ("M", ctypes.c_int), ("N", ctypes.c_int),
+        ("d_out", ctypes.c_int), ("d_in", ctypes.c_int),
+        ("w", ctypes.c_void_p), ("grid_assign", ctypes.POINTER(ctypes.c_int32)),
+    ]
+
+
 class tileq_per_expert_lr(ctypes.Structure):
     _fields_ = [("U_pe", ctypes.c_void_p * 3), ("V_pe", ctypes.c_void_p * 3)]
 
@@ -90,6 +100,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tileq_selftest_bounded_wait": ([vp, c_size, c_int, vp], c_int),
         "tileq_set_stage_events": ([P(vp), c_int], c_int),
         "tileq_launch_count": ([P(ctypes.c_ulonglong)], c_int),
+        "tileq_sketch_workspace_size": ([P(tileq_wbig), c_int, c_int, P(c_size)], c_int),
+        "tileq_sketch_lowrank": ([P(tileq_wbig), vp, c_int, c_int, vp, vp, vp, vp, c_size, vp], c_int),
     }
     for name, (argtypes, restype) in sigs.items():
         fn = getattr(lib, name)
@@ -230,3 +242,16 @@ def tileq_launch_count() -> int:
     n = ctypes.c_ulonglong()
     _check(lib().tileq_launch_count(ctypes.byref(n)), "tileq_launch_count")
     return n.value
+
+
+def tileq_sketch_workspace_size(wbig: tileq_wbig, l: int, r: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().tileq_sketch_workspace_size(ctypes.byref(wbig), l, r, ctypes.byref(n)),
+           "tileq_sketch_workspace_size")
+    return n.value
+
+
+def tileq_sketch_lowrank(wbig: tileq_wbig, omega, l: int, r: int, U, sigma, V, ws, stream=None):
+    _check(lib().tileq_sketch_lowrank(ctypes.byref(wbig), _ptr(omega), l, r, _ptr(U), _ptr(sigma),
+                                      _ptr(V), _ptr(ws), ws.numel() * ws.element_size(),
+                                      _stream(stream)), "tileq_sketch_lowrank")

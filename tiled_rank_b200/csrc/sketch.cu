@@ -1,0 +1,445 @@
+// Gaussian-sketch global low-rank decomposition of a projection's tiled matrix
+// W_big [M*d_out, N*d_in] (expert k's bf16 weights in block (m, n) of the grid):
+// TileQ summary, section 2.1, step 5 (global low-rank decomposition of W_big,
+// approximated by Gaussian sketching instead of a full SVD).  The randomised
+// range finder with an SVD of the projected matrix, computed as:
+//
+//   Y  = W_big Omega                     [R, l]   fp32 SIMT GEMM, W_big read blockwise
+//   G  = Y^T Y                           [l, l]   fp64 accumulation
+//   G  = E diag(lam) E^T                 Jacobi, fp64, one CTA
+//   Q  = Y E lam^-1/2  (lam > tol)       [R, l]   orthonormal basis of range(Y)
+//   Bt = W_big^T Q                       [C, l]   (B = Q^T W_big)
+//   C2 = Bt^T Bt = B B^T = Ub diag(s^2) Ub^T      Jacobi again
+//   U  = Q Ub[:, :r],  Sigma = s[:r],  V = Bt Ub[:, :r] diag(1/s)
+//
+// so U diag(Sigma) V^T is the rank-r truncated SVD of Q Q^T W_big, the same
+// quantity as the QR + SVD formulation.  The two eigen-decompositions of the
+// small Gram matrices replace a tall QR and an SVD of B; both see fp64.
+#include <cstring>
+
+#include "kernels.cuh"
+
+namespace tileq {
+namespace {
+
+constexpr int kSketchMaxL = TILEQ_SKETCH_MAX_L;  // sketch width: the l x l Gram matrix fits shared memory in fp64
+constexpr int kSketchGramSplits = 16;             // row splits of a Gram matrix (partials summed in order)
+constexpr double kSketchBasisTol = 1e-10;         // eigenvalues of Y^T Y below this times the largest are dropped
+
+// ---------------------------------------------------------------- operands
+// Element (i, k) of the left operand and (k, j) of the right one.
+struct DenseF32 {
+  const float *p;
+  long long ld0, ld1;  // element (a, b) at p[a*ld0 + b*ld1]
+  __device__ __forceinline__ float at(long long a, long long b) const { return p[a * ld0 + b * ld1]; }
+};
+// W_big (T = false) or its transpose (T = true), read blockwise from the
+// experts' bf16 weights [K][d_out][d_in]; expert_of[m*N + n] is the expert in
+// grid block (m, n).
+template <bool T>
+struct WBig {
+  const __nv_bfloat16 *w;
+  int N, d_out, d_in;
+  int8_t expert_of[kMaxExperts];  // grid cell m*N + n -> expert
+  __device__ __forceinline__ float at(long long a, long long b) const {
+    const long long row = T ? b : a, col = T ? a : b;
+    const int m = (int)(row / d_out), n = (int)(col / d_in);
+    const int e = expert_of[m * N + n];
+    return __bfloat162float(w[((size_t)e * d_out + (row - (long long)m * d_out)) * d_in + (col - (long long)n * d_in)]);
+  }
+};
+
+// C[i][j] = cs[j] * sum_k A(i, k) B(k, j), fp32 accumulation.  64x64 tiles, K
+// steps of 16 through shared memory, 4x4 outputs per thread.  A is loaded with
+// consecutive threads along k (row-major W_big, dense row-major) or along i
+// (transposed W_big), whichever is contiguous in memory.
+constexpr int GT = 64, GK = 16;
+
+template <typename AOp, bool A_ALONG_I>
+__global__ void __launch_bounds__(256) sk_gemm_kernel(AOp A, DenseF32 B, float *C, long long ldc, int Mr, int Nc,
+                                                      long long Kd, const float *cs) {
+  __shared__ float as[GK][GT + 4];
+  __shared__ float bs[GK][GT + 4];
+  const int tid = threadIdx.x;
+  const long long i0 = (long long)blockIdx.y * GT, j0 = (long long)blockIdx.x * GT;
+  const int ti = (tid / 16) * 4, tj = (tid % 16) * 4;
+  float acc[4][4] = {};
+  for (long long k0 = 0; k0 < Kd; k0 += GK) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = tid + u * 256;  // 1024 elements of each 64 x 16 tile
+      int ii, kk;
+      if (A_ALONG_I) {
+        ii = e % GT;
+        kk = e / GT;
+      } else {
+        kk = e % GK;
+        ii = e / GK;
+      }
+      const long long gi = i0 + ii, gk = k0 + kk;
+      as[kk][ii] = (gi < Mr && gk < Kd) ? A.at(gi, gk) : 0.f;
+      const int jj = e % GT, kb = e / GT;
+      const long long gj = j0 + jj, gkb = k0 + kb;
+      bs[kb][jj] = (gj < Nc && gkb < Kd) ? B.at(gkb, gj) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < GK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        a[u] = as[kk][ti + u];
+        b[u] = bs[kk][tj + u];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const long long gi = i0 + ti + u, gj = j0 + tj + v;
+      if (gi < Mr && gj < Nc) C[gi * ldc + gj] = acc[u][v] * (cs ? cs[gj] : 1.f);
+    }
+}
+
+// Gram partial: part[s][a][b] = sum over rows of split s of X[row][a] * X[row][b]
+// in fp64 (X fp32 [rows][l]); one CTA per (32x32 tile of the l x l result, split).
+constexpr int GR = 32;
+
+__global__ void __launch_bounds__(256) sk_gram_kernel(const float *X, long long rows, int l, int splits,
+                                                      double *part) {
+  __shared__ float xa[GR][GR + 1];
+  __shared__ float xb[GR][GR + 1];
+  const int ta = blockIdx.x % ((l + GR - 1) / GR), tb = blockIdx.x / ((l + GR - 1) / GR);
+  const int s = blockIdx.y;
+  const long long per = (rows + splits - 1) / splits;
+  const long long r0 = s * per, r1 = min(rows, r0 + per);
+  const int a0 = ta * GR, b0 = tb * GR;
+  const int tid = threadIdx.x;
+  const int oa = tid / 8, ob = (tid % 8) * 4;  // this thread: row oa, columns ob..ob+3 of the tile
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (long long rr = r0; rr < r1; rr += GR) {
+    for (int e = tid; e < GR * GR; e += 256) {
+      const int rw = e / GR, c = e % GR;
+      const long long row = rr + rw;
+      xa[rw][c] = (row < r1 && a0 + c < l) ? X[row * l + a0 + c] : 0.f;
+      xb[rw][c] = (row < r1 && b0 + c < l) ? X[row * l + b0 + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int rw = 0; rw < GR; ++rw) {
+      const double va = xa[rw][oa];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[v] += va * (double)xb[rw][ob + v];
+    }
+    __syncthreads();
+  }
+  double *out = part + (size_t)s * l * l;
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    if (a0 + oa < l && b0 + ob + v < l) out[(size_t)(a0 + oa) * l + b0 + ob + v] = acc[v];
+}
+
+// G[a][b] = sum of the splits' partials in split order.
+__global__ void sk_gram_reduce_kernel(const double *part, int l, int splits, double *G) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= l * l) return;
+  double v = 0.0;
+  for (int s = 0; s < splits; ++s) v += part[(size_t)s * l * l + e];
+  G[e] = v;
+}
+
+// Cyclic Jacobi eigen-decomposition of the symmetric l x l matrix G (fp64, l
+// even, l <= kSketchMaxL), one CTA.  Each round rotates l/2 disjoint index
+// pairs of the round-robin schedule (index 0 fixed, the others rotating), the
+// rotation of Golub and Van Loan's symmetric Schur step annihilating G[p][q];
+// sweeps of l-1 rounds until the off-diagonal mass is below (1e-15 ||G||)^2 or
+// kJacobiSweeps sweeps.  E (global, [l][l]) accumulates the rotations.  Then
+// lam[i] = the i-th largest eigenvalue and perm[i] its column of E.
+constexpr int kJacobiSweeps = 40;
+
+__global__ void __launch_bounds__(1024) sk_jacobi_kernel(const double *Gin, int l, double *E, double *lam,
+                                                        int *perm) {
+  extern __shared__ double G[];  // [l][l]
+  __shared__ double rc[kSketchMaxL / 2], rs[kSketchMaxL / 2];
+  __shared__ int rp[kSketchMaxL / 2], rq[kSketchMaxL / 2];
+  __shared__ double red[32];
+  __shared__ int done;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int h = l / 2;
+  for (int e = tid; e < l * l; e += nt) {
+    G[e] = Gin[e];
+    E[e] = (e / l == e % l) ? 1.0 : 0.0;
+  }
+  if (tid == 0) done = 0;
+  __syncthreads();
+  auto block_sum = [&](double v) -> double {
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((tid & 31) == 0) red[tid >> 5] = v;
+    __syncthreads();
+    double t = 0.0;
+    if (tid < 32) {
+      t = tid < (nt >> 5) ? red[tid] : 0.0;
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    }
+    __syncthreads();
+    return t;  // valid in warp 0
+  };
+  for (int sweep = 0; sweep < kJacobiSweeps; ++sweep) {
+    // convergence: off-diagonal mass against the Frobenius mass
+    double off = 0.0, all = 0.0;
+    for (int e = tid; e < l * l; e += nt) {
+      const double g = G[e];
+      all += g * g;
+      if (e / l != e % l) off += g * g;
+    }
+    const double off_s = block_sum(off);
+    const double all_s = block_sum(all);
+    if (tid == 0) done = !(off_s > 1e-30 * all_s);
+    __syncthreads();
+    if (done) break;
+    for (int t = 0; t < l - 1; ++t) {
+      if (tid < h) {
+        // round-robin pair i: positions i and l-1-i of [0, rotation of 1..l-1]
+        auto player = [&](int pos) { return pos == 0 ? 0 : ((pos - 1 + t) % (l - 1)) + 1; };
+        int p = player(tid), q = player(l - 1 - tid);
+        if (p > q) {
+          const int x = p;
+          p = q;
+          q = x;
+        }
+        const double apq = G[p * l + q];
+        double c = 1.0, sn = 0.0;
+        if (apq != 0.0) {
+          const double tau = (G[q * l + q] - G[p * l + p]) / (2.0 * apq);
+          const double tt = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+          c = 1.0 / sqrt(1.0 + tt * tt);
+          sn = tt * c;
+        }
+        rc[tid] = c;
+        rs[tid] = sn;
+        rp[tid] = p;
+        rq[tid] = q;
+      }
+      __syncthreads();
+      // rows p, q of every pair: J^T G
+      for (int e = tid; e < h * l; e += nt) {
+        const int i = e / l, j = e % l;
+        const int p = rp[i], q = rq[i];
+        const double c = rc[i], sn = rs[i];
+        const double gp = G[p * l + j], gq = G[q * l + j];
+        G[p * l + j] = c * gp - sn * gq;
+        G[q * l + j] = sn * gp + c * gq;
+      }
+      __syncthreads();
+      // columns p, q of every pair: (J^T G) J, and E J
+      for (int e = tid; e < h * l; e += nt) {
+        const int i = e / l, j = e % l;
+        const int p = rp[i], q = rq[i];
+        const double c = rc[i], sn = rs[i];
+        const double gp = G[j * l + p], gq = G[j * l + q];
+        G[j * l + p] = c * gp - sn * gq;
+        G[j * l + q] = sn * gp + c * gq;
+        const double ep = E[(size_t)j * l + p], eq = E[(size_t)j * l + q];
+        E[(size_t)j * l + p] = c * ep - sn * eq;
+        E[(size_t)j * l + q] = sn * ep + c * eq;
+      }
+      __syncthreads();
+    }
+  }
+  // descending order of the eigenvalues; equal ones keep their index order
+  for (int i = tid; i < l; i += nt) {
+    const double li = G[i * l + i];
+    int rank = 0;
+    for (int j = 0; j < l; ++j) {
+      const double lj = G[j * l + j];
+      rank += (lj > li || (lj == li && j < i)) ? 1 : 0;
+    }
+    lam[rank] = li;
+    perm[rank] = i;
+  }
+}
+
+// Wsmall[j][i] = E[j][perm[i]] / sqrt(lam[i]) for eigenvalues above tol * lam[0]
+// (an orthonormal basis Q = Y Wsmall of range(Y)), zero columns otherwise.
+__global__ void sk_basis_kernel(const double *E, const double *lam, const int *perm, int l, double tol,
+                                float *Wsmall) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= l * l) return;
+  const int j = e / l, i = e % l;
+  const double li = lam[i];
+  Wsmall[e] = (li > tol * lam[0] && li > 0.0) ? (float)(E[(size_t)j * l + perm[i]] / sqrt(li)) : 0.f;
+}
+
+// Ur[j][i] = E[j][perm[i]] (i < r), sigma[i] = sqrt(lam[i]), inv_sigma[i] = 1/sigma[i] (0 if sigma = 0).
+__global__ void sk_select_kernel(const double *E, const double *lam, const int *perm, int l, int r, float *Ur,
+                                 float *sigma, float *inv_sigma) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < l * r) {
+    const int j = e / r, i = e % r;
+    Ur[e] = (float)E[(size_t)j * l + perm[i]];
+  }
+  if (e < r) {
+    const double s = sqrt(fmax(lam[e], 0.0));
+    sigma[e] = (float)s;
+    inv_sigma[e] = s > 0.0 ? (float)(1.0 / s) : 0.f;
+  }
+}
+
+template <typename AOp, bool A_ALONG_I>
+cudaError_t gemm(const AOp &A, const DenseF32 &B, float *C, long long ldc, long long Mr, int Nc, long long Kd,
+                 const float *cs, cudaStream_t st) {
+  const dim3 grid((unsigned)((Nc + GT - 1) / GT), (unsigned)((Mr + GT - 1) / GT));
+  sk_gemm_kernel<AOp, A_ALONG_I><<<grid, 256, 0, st>>>(A, B, C, ldc, (int)Mr, Nc, Kd, cs);
+  count_launches();
+  return cudaGetLastError();
+}
+
+cudaError_t gram(const float *X, long long rows, int l, double *part, int splits, double *G, cudaStream_t st) {
+  const int tiles = ((l + GR - 1) / GR) * ((l + GR - 1) / GR);
+  sk_gram_kernel<<<dim3(tiles, splits), 256, 0, st>>>(X, rows, l, splits, part);
+  count_launches();
+  sk_gram_reduce_kernel<<<(l * l + 255) / 256, 256, 0, st>>>(part, l, splits, G);
+  count_launches();
+  return cudaGetLastError();
+}
+
+cudaError_t jacobi(const double *G, int l, double *E, double *lam, int *perm, cudaStream_t st) {
+  const int smem = l * l * (int)sizeof(double);
+  static int configured = 0;
+  if (smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(sk_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSketchMaxL * kSketchMaxL * (int)sizeof(double));
+    if (e != cudaSuccess) return e;
+    configured = kSketchMaxL * kSketchMaxL * (int)sizeof(double);
+  }
+  sk_jacobi_kernel<<<1, 1024, smem, st>>>(G, l, E, lam, perm);
+  count_launches();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Workspace layout of the sketch (byte offsets, 256-byte aligned).
+struct SketchWs {
+  size_t y, q, bt, part, g, e, lam, perm, wsmall, ur, inv_sigma, total;
+};
+
+static size_t sk_align(size_t x) { return (x + 255) / 256 * 256; }
+
+static SketchWs sketch_ws(long long R, long long C, int l, int r) {
+  SketchWs w{};
+  size_t off = 0;
+  auto take = [&](size_t b) {
+    const size_t o = off;
+    off += sk_align(b > 0 ? b : 16);
+    return o;
+  };
+  w.y = take((size_t)R * l * 4);
+  w.q = take((size_t)R * l * 4);
+  w.bt = take((size_t)C * l * 4);
+  w.part = take((size_t)kSketchGramSplits * l * l * 8);
+  w.g = take((size_t)l * l * 8);
+  w.e = take((size_t)l * l * 8);
+  w.lam = take((size_t)l * 8);
+  w.perm = take((size_t)l * 4);
+  w.wsmall = take((size_t)l * l * 4);
+  w.ur = take((size_t)l * r * 4);
+  w.inv_sigma = take((size_t)r * 4);
+  w.total = off;
+  return w;
+}
+
+static tileq_status sketch_check(const tileq_wbig *wb, int l, int r) {
+  if (!wb || !wb->w || !wb->grid_assign) return TILEQ_ERR_INVALID_ARG;
+  if (wb->M <= 0 || wb->N <= 0 || wb->K != wb->M * wb->N || wb->K > kMaxExperts) return TILEQ_ERR_UNSUPPORTED;
+  if (wb->d_out <= 0 || wb->d_in <= 0) return TILEQ_ERR_INVALID_ARG;
+  if (l < 2 || l > kSketchMaxL || (l & 1) || r < 1 || r > l) return TILEQ_ERR_UNSUPPORTED;
+  bool seen[kMaxExperts] = {};
+  for (int k = 0; k < wb->K; ++k) {
+    const int c = wb->grid_assign[k];
+    if (c < 0 || c >= wb->K || seen[c]) return TILEQ_ERR_INVALID_ARG;
+    seen[c] = true;
+  }
+  return TILEQ_OK;
+}
+
+}  // namespace tileq
+
+using namespace tileq;
+
+extern "C" tileq_status tileq_sketch_workspace_size(const tileq_wbig *wb, int l, int r, size_t *bytes) {
+  if (!bytes) return TILEQ_ERR_INVALID_ARG;
+  const tileq_status st = sketch_check(wb, l, r);
+  if (st != TILEQ_OK) return st;
+  *bytes = sketch_ws((long long)wb->M * wb->d_out, (long long)wb->N * wb->d_in, l, r).total;
+  return TILEQ_OK;
+}
+
+extern "C" tileq_status tileq_sketch_lowrank(const tileq_wbig *wb, const float *omega, int l, int r, float *U,
+                                             float *sigma, float *V, void *ws, size_t ws_bytes,
+                                             tileq_stream_t stream_) {
+  tileq_status st = sketch_check(wb, l, r);
+  if (st != TILEQ_OK) return st;
+  if (!omega || !U || !sigma || !V || !ws) return TILEQ_ERR_INVALID_ARG;
+  const long long R = (long long)wb->M * wb->d_out, C = (long long)wb->N * wb->d_in;
+  const SketchWs w = sketch_ws(R, C, l, r);
+  if (ws_bytes < w.total) return TILEQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  char *base = static_cast<char *>(ws);
+  float *Y = reinterpret_cast<float *>(base + w.y);
+  float *Q = reinterpret_cast<float *>(base + w.q);
+  float *Bt = reinterpret_cast<float *>(base + w.bt);
+  double *part = reinterpret_cast<double *>(base + w.part);
+  double *G = reinterpret_cast<double *>(base + w.g);
+  double *E = reinterpret_cast<double *>(base + w.e);
+  double *lam = reinterpret_cast<double *>(base + w.lam);
+  int *perm = reinterpret_cast<int *>(base + w.perm);
+  float *Wsmall = reinterpret_cast<float *>(base + w.wsmall);
+  float *Ur = reinterpret_cast<float *>(base + w.ur);
+  float *inv_sigma = reinterpret_cast<float *>(base + w.inv_sigma);
+
+  WBig<false> wbig;
+  wbig.w = static_cast<const __nv_bfloat16 *>(wb->w);
+  wbig.N = wb->N;
+  wbig.d_out = wb->d_out;
+  wbig.d_in = wb->d_in;
+  for (int k = 0; k < wb->K; ++k) wbig.expert_of[wb->grid_assign[k]] = (int8_t)k;
+  WBig<true> wbig_t;
+  wbig_t.w = wbig.w;
+  wbig_t.N = wbig.N;
+  wbig_t.d_out = wbig.d_out;
+  wbig_t.d_in = wbig.d_in;
+  std::memcpy(wbig_t.expert_of, wbig.expert_of, sizeof(wbig.expert_of));
+
+#define SK(call)                                          \
+  do {                                                    \
+    if ((call) != cudaSuccess) return TILEQ_ERR_CUDA;     \
+  } while (0)
+  // Y = W_big Omega
+  SK((gemm<WBig<false>, false>(wbig, DenseF32{omega, l, 1}, Y, l, R, l, C, nullptr, s)));
+  // orthonormal basis of range(Y) from the eigen-decomposition of Y^T Y
+  SK(gram(Y, R, l, part, kSketchGramSplits, G, s));
+  SK(jacobi(G, l, E, lam, perm, s));
+  sk_basis_kernel<<<(l * l + 255) / 256, 256, 0, s>>>(E, lam, perm, l, kSketchBasisTol, Wsmall);
+  count_launches();
+  SK(cudaGetLastError());
+  SK((gemm<DenseF32, false>(DenseF32{Y, l, 1}, DenseF32{Wsmall, l, 1}, Q, l, R, l, l, nullptr, s)));
+  // Bt = W_big^T Q, then the eigen-decomposition of B B^T
+  SK((gemm<WBig<true>, true>(wbig_t, DenseF32{Q, l, 1}, Bt, l, C, l, R, nullptr, s)));
+  SK(gram(Bt, C, l, part, kSketchGramSplits, G, s));
+  SK(jacobi(G, l, E, lam, perm, s));
+  sk_select_kernel<<<(l * r + 255) / 256, 256, 0, s>>>(E, lam, perm, l, r, Ur, sigma, inv_sigma);
+  count_launches();
+  SK(cudaGetLastError());
+  // U = Q Ub_r, V = Bt Ub_r diag(1/sigma)
+  SK((gemm<DenseF32, false>(DenseF32{Q, l, 1}, DenseF32{Ur, r, 1}, U, r, R, r, l, nullptr, s)));
+  SK((gemm<DenseF32, false>(DenseF32{Bt, l, 1}, DenseF32{Ur, r, 1}, V, r, C, r, l, inv_sigma, s)));
+#undef SK
+  return TILEQ_OK;
+}
