@@ -230,12 +230,15 @@ typedef struct {
  * these limits, TILEQ_ERR_INVALID_ARG for a grid_assign that is not a bijection. */
 tileq_status tileq_sketch_workspace_size(const tileq_wbig *w, int l, int r, size_t *bytes);
 
-/* omega: device fp32 [N*d_in][l], the Gaussian test matrix (the caller draws
- * it).  Outputs (device, overwritten): U fp32 [M*d_out][r], sigma fp32 [r]
- * (descending), V fp32 [N*d_in][r]; the columns of U and V pair up (the sign
- * of each pair is arbitrary).  ws: device workspace of at least the queried
- * size.  Asynchronous on stream; the host validates before any launch. */
-tileq_status tileq_sketch_lowrank(const tileq_wbig *w, const float *omega, int l, int r, float *U,
+/* omega_t: device bf16 [l][N*d_in], the transpose of the Gaussian test matrix
+ * Omega (the caller draws it).  Outputs (device, overwritten): U fp32
+ * [M*d_out][r], sigma fp32 [r] (descending), V fp32 [N*d_in][r]; the columns of
+ * U and V pair up (the sign of each pair is arbitrary).  ws: device workspace
+ * of at least the queried size (it holds, among others, a transposed copy of
+ * the experts' weights).  d_out and d_in must be multiples of 128
+ * (TILEQ_ERR_UNSUPPORTED).  Asynchronous on stream; the host validates before
+ * any launch. */
+tileq_status tileq_sketch_lowrank(const tileq_wbig *w, const void *omega_t, int l, int r, float *U,
                                   float *sigma, float *V, void *ws, size_t ws_bytes,
                                   tileq_stream_t stream);
 

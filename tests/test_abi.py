@@ -203,7 +203,7 @@ def test_sketch_workspace_and_validation(L):
     w = _wbig(L, 2, 4, 256, 128)
     n = L.tileq_sketch_workspace_size(w, 24, 16)
     R, C, l, r = 2 * 256, 4 * 128, 24, 16
-    assert n >= (2 * R * l + C * l) * 4 + 16 * l * l * 8
+    assert n >= 8 * 256 * 128 * 2 + (2 * R * l + 2 * C * l) * 4 + 2 * l * R * 2 + 16 * l * l * 8
     with pytest.raises(L.TileQError):
         L.tileq_sketch_workspace_size(w, 23, 16)          # odd sketch width
     with pytest.raises(L.TileQError):
@@ -211,8 +211,10 @@ def test_sketch_workspace_and_validation(L):
     with pytest.raises(L.TileQError):
         L.tileq_sketch_workspace_size(w, 24, 25)          # rank above the sketch width
     with pytest.raises(L.TileQError):
-        L.tileq_sketch_workspace_size(_wbig(L, 2, 2, 64, 64, grid=[0, 1, 1, 3]), 8, 4)  # not a bijection
-    bad = _wbig(L, 2, 2, 64, 64)
+        L.tileq_sketch_workspace_size(_wbig(L, 2, 2, 128, 128, grid=[0, 1, 1, 3]), 8, 4)  # not a bijection
+    with pytest.raises(L.TileQError):
+        L.tileq_sketch_workspace_size(_wbig(L, 2, 2, 192, 128), 8, 4)  # d_out not a multiple of 128
+    bad = _wbig(L, 2, 2, 128, 128)
     bad.K = 3
     with pytest.raises(L.TileQError):
         L.tileq_sketch_workspace_size(bad, 8, 4)          # K != M*N

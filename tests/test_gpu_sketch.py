@@ -27,15 +27,16 @@ def _bf16_bits(a):
     return ((f + np.uint32(0x7FFF) + ((f >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
 
 
-def run_sketch(torch, w_bits, grid, M, N, omega, r):
-    """GPU sketch of the experts' bf16 weights w_bits [K][d_out][d_in]; omega fp32 [N*d_in][l]."""
+def run_sketch(torch, w_bits, grid, M, N, omega_t_bits, r):
+    """GPU sketch of the experts' bf16 weights w_bits [K][d_out][d_in]; omega_t_bits: the
+    transposed Gaussian test matrix, bf16 bits [l][N*d_in]."""
     import ctypes
     from tiled_rank_b200 import _lib as L
     K, d_out, d_in = w_bits.shape
-    l = omega.shape[1]
+    l = omega_t_bits.shape[0]
     dev = torch.device("cuda:0")
     w = torch.from_numpy(w_bits.view(np.int16)).to(dev)
-    om = torch.from_numpy(np.ascontiguousarray(omega, dtype=np.float32)).to(dev)
+    om = torch.from_numpy(np.ascontiguousarray(omega_t_bits).view(np.int16)).to(dev)
     g = np.ascontiguousarray(grid, dtype=np.int32)
     wb = L.tileq_wbig()
     wb.K, wb.M, wb.N, wb.d_out, wb.d_in = K, M, N, d_out, d_in
@@ -50,6 +51,12 @@ def run_sketch(torch, w_bits, grid, M, N, omega, r):
     return U.cpu().numpy().astype(np.float64), S.cpu().numpy().astype(np.float64), V.cpu().numpy().astype(np.float64)
 
 
+def gaussian_sketch(rng, C, l):
+    """The transposed test matrix as bf16 bits [l][C] and its exact float64 value [C][l]."""
+    bits = _bf16_bits(rng.standard_normal((l, C)))
+    return bits, oracle.widen_bf16(bits).T
+
+
 def check(gpu, ref, w_big, rtol_s, tol_prod):
     (u, s, v), (uo, so, vo) = gpu, ref
     np.testing.assert_allclose(s, so, rtol=rtol_s, atol=rtol_s * so[0])
@@ -60,8 +67,8 @@ def check(gpu, ref, w_big, rtol_s, tol_prod):
     np.testing.assert_allclose(v.T @ v, np.eye(r), atol=1e-3)
 
 
-@pytest.mark.parametrize("M,N,d_out,d_in,r,l", [(2, 2, 192, 128, 8, 8), (2, 3, 128, 64, 12, 20),
-                                               (3, 2, 64, 192, 16, 24)])
+@pytest.mark.parametrize("M,N,d_out,d_in,r,l", [(2, 2, 256, 128, 8, 8), (2, 3, 128, 128, 12, 20),
+                                               (3, 2, 128, 256, 16, 24)])
 def test_planted_rank(torch_cuda, M, N, d_out, d_in, r, l):
     """A rank-r W_big (rounded to bf16: a rank-r part plus a tiny full-rank rest)."""
     rng = np.random.default_rng(M * 100 + N * 10 + r)
@@ -76,9 +83,9 @@ def test_planted_rank(torch_cuda, M, N, d_out, d_in, r, l):
         w[k] = big[m * d_out:(m + 1) * d_out, n * d_in:(n + 1) * d_in]
     w_bits = _bf16_bits(w)
     w_big = osk.assemble_wbig(w_bits, grid, M, N)
-    omega = rng.standard_normal((C, l)).astype(np.float32)
-    ref = osk.sketch_lowrank(w_big, omega.astype(np.float64), r)
-    gpu = run_sketch(torch_cuda, w_bits, grid, M, N, omega, r)
+    om_bits, omega = gaussian_sketch(rng, C, l)
+    ref = osk.sketch_lowrank(w_big, omega, r)
+    gpu = run_sketch(torch_cuda, w_bits, grid, M, N, om_bits, r)
     check(gpu, ref, w_big, 1e-4, 1e-4)
 
 
@@ -96,9 +103,9 @@ def test_decaying_spectrum(torch_cuda):
                   for k in range(M * N)])
     w_bits = _bf16_bits(w)
     w_big = osk.assemble_wbig(w_bits, grid, M, N)
-    omega = rng.standard_normal((C, l)).astype(np.float32)
-    ref = osk.sketch_lowrank(w_big, omega.astype(np.float64), r)
-    gpu = run_sketch(torch_cuda, w_bits, grid, M, N, omega, r)
+    om_bits, omega = gaussian_sketch(rng, C, l)
+    ref = osk.sketch_lowrank(w_big, omega, r)
+    gpu = run_sketch(torch_cuda, w_bits, grid, M, N, om_bits, r)
     check(gpu, ref, w_big, 1e-3, 1e-3)
 
 
@@ -114,8 +121,8 @@ def test_mixtral_shaped_gate(torch_cuda):
     del w
     r, l = 128, 136
     rng = np.random.default_rng(11)
-    omega = rng.standard_normal((layer.N * p.d_in, l)).astype(np.float32)
+    om_bits, omega = gaussian_sketch(rng, layer.N * p.d_in, l)
     w_big = osk.assemble_wbig(w_bits, p.grid_assign, layer.M, layer.N)
-    ref = osk.sketch_lowrank(w_big, omega.astype(np.float64), r)
-    gpu = run_sketch(torch_cuda, w_bits, p.grid_assign, layer.M, layer.N, omega, r)
+    ref = osk.sketch_lowrank(w_big, omega, r)
+    gpu = run_sketch(torch_cuda, w_bits, p.grid_assign, layer.M, layer.N, om_bits, r)
     check(gpu, ref, w_big, 1e-3, 2e-3)

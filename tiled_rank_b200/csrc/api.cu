@@ -1526,4 +1526,8 @@ extern "C" tileq_status tileq_route_static(const float *router_logits, int T, in
 
 namespace tileq {
 void count_launches(int n) { g_launches.fetch_add((unsigned long long)n); }
+bool tensor_map_2b(CUtensorMap *m, const void *base, int rows, int cols, int ld, int box_rows) {
+  return make_map(m, base, rows, cols, ld, box_rows);
+}
+int dense_tile_items(int items, int m_units) { return dense_bn(items, m_units); }
 }  // namespace tileq

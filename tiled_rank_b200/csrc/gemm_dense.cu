@@ -121,8 +121,18 @@ __global__ void __launch_bounds__(DenseCfg<MB, BN>::THREADS, 1)
           if (qi >= (uint32_t)C::SQ && !(ok = mbar_wait(&q_empty[s], ((qi / C::SQ) - 1) & 1, P.status))) break;
           mbar_arrive_expect_tx(&q_full[s], C::STAGE);
 #pragma unroll
-          for (int j = 0; j < MB; ++j)
-            tc::tma_load_2d(stage_a(s, j), &P.amap[P.pair ? j : 0], kb * DBK, a_row(t.x, ou, j), &q_full[s]);
+          for (int j = 0; j < MB; ++j) {
+            int ax = kb * DBK, ay = a_row(t.x, ou, j);
+            if (P.kblk) {
+              // grid mode: output rows ay and K column ax fall in block (bi, bk)
+              // (rows past the last block, padding of an odd row-block count, reuse the
+              // last block: the epilogue drops them)
+              const int bi = min(ay / P.blk_rows, P.grid_i - 1), bk = ax / P.kblk;
+              ay = P.a_blk[bi * P.cell_i + bk * P.cell_k] * P.blk_rows + (ay - bi * P.blk_rows);
+              ax -= bk * P.kblk;
+            }
+            tc::tma_load_2d(stage_a(s, j), &P.amap[P.pair ? j : 0], ax, ay, &q_full[s]);
+          }
           tc::tma_load_2d(stage_b(s), &P.bmap, kb * DBK, t.y, &q_full[s]);
         }
       }
@@ -134,7 +144,8 @@ __global__ void __launch_bounds__(DenseCfg<MB, BN>::THREADS, 1)
     // ============================================================ MMA issuer
     // The whole warp waits; one elected lane issues the MMAs and commits.
     {
-      constexpr uint32_t idesc = tc::idesc_f16(BN);
+      // kind::f16 with both operands fp16, or both bf16 (A and B formats at bits 7 and 10)
+      const uint32_t idesc = tc::idesc_f16(BN) | (P.bf16 ? ((1u << 7) | (1u << 10)) : 0u);
       uint32_t qi = 0, wi = 0;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++wi) {
         const int ab = wi % C::NACC;

@@ -157,6 +157,11 @@ struct DenseArgs {
   int m_blocks;           // row blocks of one A block (cdiv(d_out, 128))
   int use_a_blk;
   int8_t a_blk[kMaxExperts];
+  // grid mode (kblk > 0): A is a grid of blocks of blk_rows output rows x kblk
+  // K columns, block (i, k) stored as the matrix a_blk[i * cell_i + k * cell_k]
+  // of the array [blocks][blk_rows][kblk] (blk_rows a multiple of 128, kblk of 64)
+  int kblk, blk_rows, cell_i, cell_k, grid_i;  // grid_i: blocks along the output rows
+  int bf16;               // operands bf16 instead of fp16
   int d_out, d_in;        // d_in a multiple of 64
   int epi;
   void *out[2];
@@ -167,6 +172,10 @@ struct DenseArgs {
 };
 
 cudaError_t launch_gemm_dense(const DenseArgs &a, int mb, int bn, int grid, cudaStream_t stream);
+// 2-D tensor map over 2-byte elements [rows][ld] (cols used), box 64 x box_rows,
+// 128-byte swizzle (api.cu), and the item-tile width the dense products use.
+bool tensor_map_2b(CUtensorMap *m, const void *base, int rows, int cols, int ld, int box_rows);
+int dense_tile_items(int items, int m_units);
 
 // The same residual GEMM for narrow tiles (bn 8, 16 or 32) on warp-level MMA:
 // codes[p] in the per-lane fragment layout of pack_codes_kernel, B through

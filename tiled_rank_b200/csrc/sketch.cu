@@ -4,13 +4,14 @@
 // approximated by Gaussian sketching instead of a full SVD).  The randomised
 // range finder with an SVD of the projected matrix, computed as:
 //
-//   Y  = W_big Omega                     [R, l]   fp32 SIMT GEMM, W_big read blockwise
-//   G  = Y^T Y                           [l, l]   fp64 accumulation
-//   G  = E diag(lam) E^T                 Jacobi, fp64, one CTA
-//   Q  = Y E lam^-1/2  (lam > tol)       [R, l]   orthonormal basis of range(Y)
-//   Bt = W_big^T Q                       [C, l]   (B = Q^T W_big)
-//   C2 = Bt^T Bt = B B^T = Ub diag(s^2) Ub^T      Jacobi again
-//   U  = Q Ub[:, :r],  Sigma = s[:r],  V = Bt Ub[:, :r] diag(1/s)
+//   Y^T = Omega^T W_big^T                [l, R]   tcgen05 (bf16 in, fp32 out), W_big read by blocks
+//   G   = Y^T Y                          [l, l]   fp64 accumulation
+//   G   = E diag(lam) E^T                Jacobi, fp64, one CTA
+//   Q^T = (E lam^-1/2)^T Y^T (lam > tol) [l, R]   orthonormal basis of range(Y), fp32
+//   B   = Q^T W_big                      [l, C]   tcgen05 on the experts' transposes, Q^T
+//                                                 split into two bf16 terms (hi + lo)
+//   B B^T = Ub diag(s^2) Ub^T            Jacobi again
+//   U  = Q Ub[:, :r],  Sigma = s[:r],  V = B^T Ub[:, :r] diag(1/s)
 //
 // so U diag(Sigma) V^T is the rank-r truncated SVD of Q Q^T W_big, the same
 // quantity as the QR + SVD formulation.  The two eigen-decompositions of the
@@ -145,6 +146,76 @@ __global__ void __launch_bounds__(256) sk_gram_kernel(const float *X, long long 
     if (a0 + oa < l && b0 + ob + v < l) out[(size_t)(a0 + oa) * l + b0 + ob + v] = acc[v];
 }
 
+// The same Gram partial of a row-major [l][rows] matrix (Y^T, B): rows along
+// the contiguous dimension.
+__global__ void __launch_bounds__(256) sk_gram_t_kernel(const float *Xt, long long rows, int l, int splits,
+                                                        double *part) {
+  __shared__ float xa[GR][GR + 1];
+  __shared__ float xb[GR][GR + 1];
+  const int ta = blockIdx.x % ((l + GR - 1) / GR), tb = blockIdx.x / ((l + GR - 1) / GR);
+  const int s = blockIdx.y;
+  const long long per = (rows + splits - 1) / splits;
+  const long long r0 = s * per, r1 = min(rows, r0 + per);
+  const int a0 = ta * GR, b0 = tb * GR;
+  const int tid = threadIdx.x;
+  const int oa = tid / 8, ob = (tid % 8) * 4;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (long long rr = r0; rr < r1; rr += GR) {
+    for (int e = tid; e < GR * GR; e += 256) {
+      const int c = e / GR, rw = e % GR;  // consecutive threads along the rows
+      const long long row = rr + rw;
+      xa[rw][c] = (row < r1 && a0 + c < l) ? Xt[(size_t)(a0 + c) * rows + row] : 0.f;
+      xb[rw][c] = (row < r1 && b0 + c < l) ? Xt[(size_t)(b0 + c) * rows + row] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int rw = 0; rw < GR; ++rw) {
+      const double va = xa[rw][oa];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[v] += va * (double)xb[rw][ob + v];
+    }
+    __syncthreads();
+  }
+  double *out = part + (size_t)s * l * l;
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    if (a0 + oa < l && b0 + ob + v < l) out[(size_t)(a0 + oa) * l + b0 + ob + v] = acc[v];
+}
+
+// wt[k][c][r] = w[k][r][c] (bf16, 32 x 32 tiles through shared memory).
+__global__ void sk_transpose_kernel(const __nv_bfloat16 *w, int d_out, int d_in, __nv_bfloat16 *wt) {
+  __shared__ __nv_bfloat16 t[32][33];
+  const int k = blockIdx.z;
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  const __nv_bfloat16 *src = w + (size_t)k * d_out * d_in;
+  __nv_bfloat16 *dst = wt + (size_t)k * d_out * d_in;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < d_out && c < d_in) t[i][threadIdx.x] = src[(size_t)r * d_in + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < d_out && c < d_in) dst[(size_t)c * d_out + r] = t[threadIdx.x][i];
+  }
+}
+
+// q (fp32) = hi + lo with hi = bf16(q), lo = bf16(q - hi): hl[0:n] = hi, hl[n:2n] = lo.
+__global__ void sk_split_kernel(const float *q, long long n, __nv_bfloat16 *hl) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float v = q[i];
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  hl[i] = hi;
+  hl[n + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
+// b[i] += b[n + i]: the hi and lo products summed.
+__global__ void sk_sum_halves_kernel(float *b, long long n) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) b[i] += b[n + i];
+}
+
 // G[a][b] = sum of the splits' partials in split order.
 __global__ void sk_gram_reduce_kernel(const double *part, int l, int splits, double *G) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -158,23 +229,27 @@ __global__ void sk_gram_reduce_kernel(const double *part, int l, int splits, dou
 // even, l <= kSketchMaxL), one CTA.  Each round rotates l/2 disjoint index
 // pairs of the round-robin schedule (index 0 fixed, the others rotating), the
 // rotation of Golub and Van Loan's symmetric Schur step annihilating G[p][q];
-// sweeps of l-1 rounds until the off-diagonal mass is below (1e-15 ||G||)^2 or
-// kJacobiSweeps sweeps.  E (global, [l][l]) accumulates the rotations.  Then
-// lam[i] = the i-th largest eigenvalue and perm[i] its column of E.
+// sweeps of l-1 rounds until the off-diagonal mass is below (1e-13 ||G||)^2 or
+// kJacobiSweeps sweeps.  G lives in shared memory with a row stride of l + 1
+// (its columns are read too).  The eigenvectors accumulate transposed in
+// global memory, Et[q][j] = E[j][q], so that rotating columns p, q of E moves
+// two contiguous rows.  Then lam[i] = the i-th largest eigenvalue and perm[i]
+// the row of Et holding its eigenvector.
 constexpr int kJacobiSweeps = 40;
+constexpr int kJacobiThreads = 512;
 
-__global__ void __launch_bounds__(1024) sk_jacobi_kernel(const double *Gin, int l, double *E, double *lam,
-                                                        int *perm) {
-  extern __shared__ double G[];  // [l][l]
+__global__ void __launch_bounds__(kJacobiThreads) sk_jacobi_kernel(const double *Gin, int l, double *Et, double *lam,
+                                                                  int *perm) {
+  extern __shared__ double G[];  // [l][l + 1]
   __shared__ double rc[kSketchMaxL / 2], rs[kSketchMaxL / 2];
   __shared__ int rp[kSketchMaxL / 2], rq[kSketchMaxL / 2];
   __shared__ double red[32];
   __shared__ int done;
   const int tid = threadIdx.x, nt = blockDim.x;
-  const int h = l / 2;
+  const int h = l / 2, ld = l + 1;
   for (int e = tid; e < l * l; e += nt) {
-    G[e] = Gin[e];
-    E[e] = (e / l == e % l) ? 1.0 : 0.0;
+    G[(e / l) * ld + e % l] = Gin[e];
+    Et[e] = (e / l == e % l) ? 1.0 : 0.0;
   }
   if (tid == 0) done = 0;
   __syncthreads();
@@ -194,13 +269,13 @@ __global__ void __launch_bounds__(1024) sk_jacobi_kernel(const double *Gin, int 
     // convergence: off-diagonal mass against the Frobenius mass
     double off = 0.0, all = 0.0;
     for (int e = tid; e < l * l; e += nt) {
-      const double g = G[e];
+      const double g = G[(e / l) * ld + e % l];
       all += g * g;
       if (e / l != e % l) off += g * g;
     }
     const double off_s = block_sum(off);
     const double all_s = block_sum(all);
-    if (tid == 0) done = !(off_s > 1e-30 * all_s);
+    if (tid == 0) done = !(off_s > 1e-26 * all_s);
     __syncthreads();
     if (done) break;
     for (int t = 0; t < l - 1; ++t) {
@@ -213,10 +288,10 @@ __global__ void __launch_bounds__(1024) sk_jacobi_kernel(const double *Gin, int 
           p = q;
           q = x;
         }
-        const double apq = G[p * l + q];
+        const double apq = G[p * ld + q];
         double c = 1.0, sn = 0.0;
         if (apq != 0.0) {
-          const double tau = (G[q * l + q] - G[p * l + p]) / (2.0 * apq);
+          const double tau = (G[q * ld + q] - G[p * ld + p]) / (2.0 * apq);
           const double tt = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
           c = 1.0 / sqrt(1.0 + tt * tt);
           sn = tt * c;
@@ -227,37 +302,37 @@ __global__ void __launch_bounds__(1024) sk_jacobi_kernel(const double *Gin, int 
         rq[tid] = q;
       }
       __syncthreads();
-      // rows p, q of every pair: J^T G
+      // rows p, q of every pair: J^T G; rows p, q of Et: (E J)^T
       for (int e = tid; e < h * l; e += nt) {
         const int i = e / l, j = e % l;
         const int p = rp[i], q = rq[i];
         const double c = rc[i], sn = rs[i];
-        const double gp = G[p * l + j], gq = G[q * l + j];
-        G[p * l + j] = c * gp - sn * gq;
-        G[q * l + j] = sn * gp + c * gq;
+        const double gp = G[p * ld + j], gq = G[q * ld + j];
+        G[p * ld + j] = c * gp - sn * gq;
+        G[q * ld + j] = sn * gp + c * gq;
+        const double ep = Et[(size_t)p * l + j], eq = Et[(size_t)q * l + j];
+        Et[(size_t)p * l + j] = c * ep - sn * eq;
+        Et[(size_t)q * l + j] = sn * ep + c * eq;
       }
       __syncthreads();
-      // columns p, q of every pair: (J^T G) J, and E J
+      // columns p, q of every pair: (J^T G) J
       for (int e = tid; e < h * l; e += nt) {
         const int i = e / l, j = e % l;
         const int p = rp[i], q = rq[i];
         const double c = rc[i], sn = rs[i];
-        const double gp = G[j * l + p], gq = G[j * l + q];
-        G[j * l + p] = c * gp - sn * gq;
-        G[j * l + q] = sn * gp + c * gq;
-        const double ep = E[(size_t)j * l + p], eq = E[(size_t)j * l + q];
-        E[(size_t)j * l + p] = c * ep - sn * eq;
-        E[(size_t)j * l + q] = sn * ep + c * eq;
+        const double gp = G[j * ld + p], gq = G[j * ld + q];
+        G[j * ld + p] = c * gp - sn * gq;
+        G[j * ld + q] = sn * gp + c * gq;
       }
       __syncthreads();
     }
   }
   // descending order of the eigenvalues; equal ones keep their index order
   for (int i = tid; i < l; i += nt) {
-    const double li = G[i * l + i];
+    const double li = G[i * ld + i];
     int rank = 0;
     for (int j = 0; j < l; ++j) {
-      const double lj = G[j * l + j];
+      const double lj = G[j * ld + j];
       rank += (lj > li || (lj == li && j < i)) ? 1 : 0;
     }
     lam[rank] = li;
@@ -267,22 +342,22 @@ __global__ void __launch_bounds__(1024) sk_jacobi_kernel(const double *Gin, int 
 
 // Wsmall[j][i] = E[j][perm[i]] / sqrt(lam[i]) for eigenvalues above tol * lam[0]
 // (an orthonormal basis Q = Y Wsmall of range(Y)), zero columns otherwise.
-__global__ void sk_basis_kernel(const double *E, const double *lam, const int *perm, int l, double tol,
+__global__ void sk_basis_kernel(const double *Et, const double *lam, const int *perm, int l, double tol,
                                 float *Wsmall) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= l * l) return;
   const int j = e / l, i = e % l;
   const double li = lam[i];
-  Wsmall[e] = (li > tol * lam[0] && li > 0.0) ? (float)(E[(size_t)j * l + perm[i]] / sqrt(li)) : 0.f;
+  Wsmall[e] = (li > tol * lam[0] && li > 0.0) ? (float)(Et[(size_t)perm[i] * l + j] / sqrt(li)) : 0.f;
 }
 
 // Ur[j][i] = E[j][perm[i]] (i < r), sigma[i] = sqrt(lam[i]), inv_sigma[i] = 1/sigma[i] (0 if sigma = 0).
-__global__ void sk_select_kernel(const double *E, const double *lam, const int *perm, int l, int r, float *Ur,
+__global__ void sk_select_kernel(const double *Et, const double *lam, const int *perm, int l, int r, float *Ur,
                                  float *sigma, float *inv_sigma) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e < l * r) {
     const int j = e / r, i = e % r;
-    Ur[e] = (float)E[(size_t)j * l + perm[i]];
+    Ur[e] = (float)Et[(size_t)perm[i] * l + j];
   }
   if (e < r) {
     const double s = sqrt(fmax(lam[e], 0.0));
@@ -300,9 +375,13 @@ cudaError_t gemm(const AOp &A, const DenseF32 &B, float *C, long long ldc, long 
   return cudaGetLastError();
 }
 
-cudaError_t gram(const float *X, long long rows, int l, double *part, int splits, double *G, cudaStream_t st) {
+cudaError_t gram(const float *X, bool xt, long long rows, int l, double *part, int splits, double *G,
+                 cudaStream_t st) {
   const int tiles = ((l + GR - 1) / GR) * ((l + GR - 1) / GR);
-  sk_gram_kernel<<<dim3(tiles, splits), 256, 0, st>>>(X, rows, l, splits, part);
+  if (xt)
+    sk_gram_t_kernel<<<dim3(tiles, splits), 256, 0, st>>>(X, rows, l, splits, part);
+  else
+    sk_gram_kernel<<<dim3(tiles, splits), 256, 0, st>>>(X, rows, l, splits, part);
   count_launches();
   sk_gram_reduce_kernel<<<(l * l + 255) / 256, 256, 0, st>>>(part, l, splits, G);
   count_launches();
@@ -310,29 +389,64 @@ cudaError_t gram(const float *X, long long rows, int l, double *part, int splits
 }
 
 cudaError_t jacobi(const double *G, int l, double *E, double *lam, int *perm, cudaStream_t st) {
-  const int smem = l * l * (int)sizeof(double);
+  const int smem = l * (l + 1) * (int)sizeof(double);
   static int configured = 0;
   if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(sk_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSketchMaxL * kSketchMaxL * (int)sizeof(double));
+    const int most = kSketchMaxL * (kSketchMaxL + 1) * (int)sizeof(double);
+    cudaError_t e = cudaFuncSetAttribute(sk_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
     if (e != cudaSuccess) return e;
-    configured = kSketchMaxL * kSketchMaxL * (int)sizeof(double);
+    configured = most;
   }
-  sk_jacobi_kernel<<<1, 1024, smem, st>>>(G, l, E, lam, perm);
+  sk_jacobi_kernel<<<1, kJacobiThreads, smem, st>>>(G, l, E, lam, perm);
   count_launches();
   return cudaGetLastError();
+}
+
+// out[item][o] = sum_k A(o, k) Bop[item][k] on tcgen05 (bf16 operands, fp32 out):
+// A is the grid of expert blocks in `a_arr` ([K][blk_rows][kblk], block of cell
+// bi * cell_i + bk * cell_k), Bop the row-major bf16 [items][kd] matrix.
+cudaError_t tc_grid_product(const __nv_bfloat16 *a_arr, int K, int blk_rows, int kblk, int grid_i, int cell_i,
+                            int cell_k, const int8_t *blk_of, const __nv_bfloat16 *bop, int items, long long rows,
+                            long long kd, float *out, cudaStream_t st) {
+  DenseArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const int m_blocks = (int)(rows / 128);
+  const int mb = m_blocks > 1 ? 2 : 1;
+  a.pair = 0;
+  a.m_blocks = m_blocks;
+  a.m_units = (m_blocks + mb - 1) / mb;
+  const int bn = dense_tile_items(items, a.m_units);
+  if (!tensor_map_2b(&a.amap[0], a_arr, K * blk_rows, kblk, kblk, 128)) return cudaErrorInvalidValue;
+  if (!tensor_map_2b(&a.bmap, bop, items, (int)kd, (int)kd, bn)) return cudaErrorInvalidValue;
+  a.static_items = items;
+  a.kblk = kblk;
+  a.blk_rows = blk_rows;
+  a.cell_i = cell_i;
+  a.cell_k = cell_k;
+  a.grid_i = grid_i;
+  std::memcpy(a.a_blk, blk_of, kMaxExperts);
+  a.bf16 = 1;
+  a.d_out = (int)rows;
+  a.d_in = (int)kd;
+  a.epi = EPI_STORE_F32;
+  a.out[0] = out;
+  a.ldo = (int)rows;
+  a.status = nullptr;
+  const long long units = (long long)((items + bn - 1) / bn) * a.m_units;
+  const int grid = (int)(units < 148 ? units : 148);
+  return launch_gemm_dense(a, mb, bn, grid, st);
 }
 
 }  // namespace
 
 // Workspace layout of the sketch (byte offsets, 256-byte aligned).
 struct SketchWs {
-  size_t y, q, bt, part, g, e, lam, perm, wsmall, ur, inv_sigma, total;
+  size_t wt, yt, qt, qhl, bo, part, g, e, lam, perm, wsmall, ur, inv_sigma, total;
 };
 
 static size_t sk_align(size_t x) { return (x + 255) / 256 * 256; }
 
-static SketchWs sketch_ws(long long R, long long C, int l, int r) {
+static SketchWs sketch_ws(int K, long long R, long long C, int d_out, int d_in, int l, int r) {
   SketchWs w{};
   size_t off = 0;
   auto take = [&](size_t b) {
@@ -340,9 +454,11 @@ static SketchWs sketch_ws(long long R, long long C, int l, int r) {
     off += sk_align(b > 0 ? b : 16);
     return o;
   };
-  w.y = take((size_t)R * l * 4);
-  w.q = take((size_t)R * l * 4);
-  w.bt = take((size_t)C * l * 4);
+  w.wt = take((size_t)K * d_out * d_in * 2);
+  w.yt = take((size_t)l * R * 4);
+  w.qt = take((size_t)l * R * 4);
+  w.qhl = take((size_t)2 * l * R * 2);
+  w.bo = take((size_t)2 * l * C * 4);
   w.part = take((size_t)kSketchGramSplits * l * l * 8);
   w.g = take((size_t)l * l * 8);
   w.e = take((size_t)l * l * 8);
@@ -359,6 +475,7 @@ static tileq_status sketch_check(const tileq_wbig *wb, int l, int r) {
   if (!wb || !wb->w || !wb->grid_assign) return TILEQ_ERR_INVALID_ARG;
   if (wb->M <= 0 || wb->N <= 0 || wb->K != wb->M * wb->N || wb->K > kMaxExperts) return TILEQ_ERR_UNSUPPORTED;
   if (wb->d_out <= 0 || wb->d_in <= 0) return TILEQ_ERR_INVALID_ARG;
+  if (wb->d_out % 128 || wb->d_in % 128) return TILEQ_ERR_UNSUPPORTED;  // 128-row tiles of W_big and W_big^T
   if (l < 2 || l > kSketchMaxL || (l & 1) || r < 1 || r > l) return TILEQ_ERR_UNSUPPORTED;
   bool seen[kMaxExperts] = {};
   for (int k = 0; k < wb->K; ++k) {
@@ -377,24 +494,28 @@ extern "C" tileq_status tileq_sketch_workspace_size(const tileq_wbig *wb, int l,
   if (!bytes) return TILEQ_ERR_INVALID_ARG;
   const tileq_status st = sketch_check(wb, l, r);
   if (st != TILEQ_OK) return st;
-  *bytes = sketch_ws((long long)wb->M * wb->d_out, (long long)wb->N * wb->d_in, l, r).total;
+  *bytes = sketch_ws(wb->K, (long long)wb->M * wb->d_out, (long long)wb->N * wb->d_in, wb->d_out, wb->d_in, l, r).total;
   return TILEQ_OK;
 }
 
-extern "C" tileq_status tileq_sketch_lowrank(const tileq_wbig *wb, const float *omega, int l, int r, float *U,
+extern "C" tileq_status tileq_sketch_lowrank(const tileq_wbig *wb, const void *omega_t, int l, int r, float *U,
                                              float *sigma, float *V, void *ws, size_t ws_bytes,
                                              tileq_stream_t stream_) {
   tileq_status st = sketch_check(wb, l, r);
   if (st != TILEQ_OK) return st;
-  if (!omega || !U || !sigma || !V || !ws) return TILEQ_ERR_INVALID_ARG;
-  const long long R = (long long)wb->M * wb->d_out, C = (long long)wb->N * wb->d_in;
-  const SketchWs w = sketch_ws(R, C, l, r);
+  if (!omega_t || !U || !sigma || !V || !ws) return TILEQ_ERR_INVALID_ARG;
+  const int M = wb->M, N = wb->N, K = wb->K, d_out = wb->d_out, d_in = wb->d_in;
+  const long long R = (long long)M * d_out, C = (long long)N * d_in;
+  const SketchWs w = sketch_ws(K, R, C, d_out, d_in, l, r);
   if (ws_bytes < w.total) return TILEQ_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream_);
   char *base = static_cast<char *>(ws);
-  float *Y = reinterpret_cast<float *>(base + w.y);
-  float *Q = reinterpret_cast<float *>(base + w.q);
-  float *Bt = reinterpret_cast<float *>(base + w.bt);
+  const __nv_bfloat16 *W = static_cast<const __nv_bfloat16 *>(wb->w);
+  __nv_bfloat16 *Wt = reinterpret_cast<__nv_bfloat16 *>(base + w.wt);
+  float *Yt = reinterpret_cast<float *>(base + w.yt);
+  float *Qt = reinterpret_cast<float *>(base + w.qt);
+  __nv_bfloat16 *Qhl = reinterpret_cast<__nv_bfloat16 *>(base + w.qhl);
+  float *Bo = reinterpret_cast<float *>(base + w.bo);
   double *part = reinterpret_cast<double *>(base + w.part);
   double *G = reinterpret_cast<double *>(base + w.g);
   double *E = reinterpret_cast<double *>(base + w.e);
@@ -403,43 +524,46 @@ extern "C" tileq_status tileq_sketch_lowrank(const tileq_wbig *wb, const float *
   float *Wsmall = reinterpret_cast<float *>(base + w.wsmall);
   float *Ur = reinterpret_cast<float *>(base + w.ur);
   float *inv_sigma = reinterpret_cast<float *>(base + w.inv_sigma);
-
-  WBig<false> wbig;
-  wbig.w = static_cast<const __nv_bfloat16 *>(wb->w);
-  wbig.N = wb->N;
-  wbig.d_out = wb->d_out;
-  wbig.d_in = wb->d_in;
-  for (int k = 0; k < wb->K; ++k) wbig.expert_of[wb->grid_assign[k]] = (int8_t)k;
-  WBig<true> wbig_t;
-  wbig_t.w = wbig.w;
-  wbig_t.N = wbig.N;
-  wbig_t.d_out = wbig.d_out;
-  wbig_t.d_in = wbig.d_in;
-  std::memcpy(wbig_t.expert_of, wbig.expert_of, sizeof(wbig.expert_of));
+  int8_t cell_expert[kMaxExperts] = {};
+  for (int k = 0; k < K; ++k) cell_expert[wb->grid_assign[k]] = (int8_t)k;
 
 #define SK(call)                                          \
   do {                                                    \
     if ((call) != cudaSuccess) return TILEQ_ERR_CUDA;     \
   } while (0)
-  // Y = W_big Omega
-  SK((gemm<WBig<false>, false>(wbig, DenseF32{omega, l, 1}, Y, l, R, l, C, nullptr, s)));
+  // Y^T = Omega^T W_big^T: output rows = rows of W_big (blocks of d_out, grid
+  // row m), K = columns of W_big (blocks of d_in, grid column n)
+  SK(tc_grid_product(W, K, d_out, d_in, M, N, 1, cell_expert, static_cast<const __nv_bfloat16 *>(omega_t), l, R, C,
+                     Yt, s));
   // orthonormal basis of range(Y) from the eigen-decomposition of Y^T Y
-  SK(gram(Y, R, l, part, kSketchGramSplits, G, s));
+  SK(gram(Yt, true, R, l, part, kSketchGramSplits, G, s));
   SK(jacobi(G, l, E, lam, perm, s));
   sk_basis_kernel<<<(l * l + 255) / 256, 256, 0, s>>>(E, lam, perm, l, kSketchBasisTol, Wsmall);
   count_launches();
   SK(cudaGetLastError());
-  SK((gemm<DenseF32, false>(DenseF32{Y, l, 1}, DenseF32{Wsmall, l, 1}, Q, l, R, l, l, nullptr, s)));
-  // Bt = W_big^T Q, then the eigen-decomposition of B B^T
-  SK((gemm<WBig<true>, true>(wbig_t, DenseF32{Q, l, 1}, Bt, l, C, l, R, nullptr, s)));
-  SK(gram(Bt, C, l, part, kSketchGramSplits, G, s));
+  // Q^T[i][row] = sum_j Wsmall[j][i] Y^T[j][row]
+  SK((gemm<DenseF32, true>(DenseF32{Wsmall, 1, l}, DenseF32{Yt, R, 1}, Qt, R, l, (int)R, l, nullptr, s)));
+  // B = Q^T W_big with Q^T = hi + lo (bf16 each): products on the experts' transposes,
+  // output rows = columns of W_big (blocks of d_in, grid column n), K = rows of
+  // W_big (blocks of d_out, grid row m)
+  sk_transpose_kernel<<<dim3((d_in + 31) / 32, (d_out + 31) / 32, K), dim3(32, 8), 0, s>>>(W, d_out, d_in, Wt);
+  count_launches();
+  sk_split_kernel<<<(unsigned)((l * R + 255) / 256), 256, 0, s>>>(Qt, (long long)l * R, Qhl);
+  count_launches();
+  SK(cudaGetLastError());
+  SK(tc_grid_product(Wt, K, d_in, d_out, N, 1, N, cell_expert, Qhl, 2 * l, C, R, Bo, s));
+  sk_sum_halves_kernel<<<(unsigned)((l * C + 255) / 256), 256, 0, s>>>(Bo, (long long)l * C);
+  count_launches();
+  SK(cudaGetLastError());
+  // eigen-decomposition of B B^T
+  SK(gram(Bo, true, C, l, part, kSketchGramSplits, G, s));
   SK(jacobi(G, l, E, lam, perm, s));
   sk_select_kernel<<<(l * r + 255) / 256, 256, 0, s>>>(E, lam, perm, l, r, Ur, sigma, inv_sigma);
   count_launches();
   SK(cudaGetLastError());
-  // U = Q Ub_r, V = Bt Ub_r diag(1/sigma)
-  SK((gemm<DenseF32, false>(DenseF32{Q, l, 1}, DenseF32{Ur, r, 1}, U, r, R, r, l, nullptr, s)));
-  SK((gemm<DenseF32, false>(DenseF32{Bt, l, 1}, DenseF32{Ur, r, 1}, V, r, C, r, l, inv_sigma, s)));
+  // U[row][i] = sum_j Q^T[j][row] Ur[j][i];  V[c][i] = sum_j B[j][c] Ur[j][i] / sigma[i]
+  SK((gemm<DenseF32, true>(DenseF32{Qt, 1, R}, DenseF32{Ur, r, 1}, U, r, R, r, l, nullptr, s)));
+  SK((gemm<DenseF32, true>(DenseF32{Bo, 1, C}, DenseF32{Ur, r, 1}, V, r, C, r, l, inv_sigma, s)));
 #undef SK
   return TILEQ_OK;
 }
