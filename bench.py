@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-compare", action="store_true", help="skip the unfused / rank-0 comparisons")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sketch", action="store_true",
+                    help="time the Gaussian-sketch global low-rank decomposition of one projection's W_big "
+                         "(the configuration's gate projection) instead of the forward")
     return ap.parse_args()
 
 
@@ -210,10 +213,82 @@ def workload_config(cfg, T, args, l2):
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
+def run_sketch(args, cfg):
+    """Gaussian-sketch decomposition of the configuration's gate W_big [M*F, N*D] at rank r with
+    8 columns of oversampling; synthetic bf16 expert weights and sketch drawn on the device."""
+    import ctypes
+    import torch
+    from tiled_rank_b200 import _lib as L
+    if int(os.environ.get("RANK", "0")) != 0:
+        return  # one decomposition: replicas would only repeat it
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    K, M, N = cfg.K, cfg.M, cfg.N
+    d_out, d_in = cfg.d_ff, cfg.d_model
+    r = cfg.rank
+    l = r + 8
+    gen = torch.Generator(device=dev).manual_seed(args.seed)
+    w = (torch.randn((K, d_out, d_in), generator=gen, device=dev) * (d_in ** -0.5)).to(torch.bfloat16)
+    om = torch.randn((l, N * d_in), generator=gen, device=dev).to(torch.bfloat16)
+    grid = np.arange(K, dtype=np.int32)
+    wb = L.tileq_wbig()
+    wb.K, wb.M, wb.N, wb.d_out, wb.d_in = K, M, N, d_out, d_in
+    wb.w = w.data_ptr()
+    wb.grid_assign = grid.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    ws = torch.empty(L.tileq_sketch_workspace_size(wb, l, r), dtype=torch.uint8, device=dev)
+    U = torch.empty((M * d_out, r), device=dev)
+    S = torch.empty((r,), device=dev)
+    V = torch.empty((N * d_in, r), device=dev)
+    for _ in range(args.warmup):
+        L.tileq_sketch_lowrank(wb, om, l, r, U, S, V, ws)
+    torch.cuda.synchronize()
+    n0 = L.tileq_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        L.tileq_sketch_lowrank(wb, om, l, r, U, S, V, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    launches = L.tileq_launch_count() - n0
+    ms = e0.elapsed_time(e1) / args.steps
+    R, C = M * d_out, N * d_in
+    flops = 2.0 * 2 * R * C * l  # W_big Omega and Q^T W_big
+    peaks = measured_peaks()
+    t_roof = flops / (peaks["bf16_tflops"] * 1e12)
+    cpu = None
+    if not args.no_cpu_baseline:
+        from oracle import sketch as osk
+        t0 = time.perf_counter()
+        w_bits = w.view(torch.int16).cpu().numpy().view(np.uint16)
+        big = osk.assemble_wbig(w_bits, grid, M, N)
+        omega = osk.widen_bf16(om.view(torch.int16).cpu().numpy().view(np.uint16)).T
+        osk.sketch_lowrank(big, omega, r)
+        dt = time.perf_counter() - t0
+        cpu = {"value": 1.0 / dt, "unit": "sketch/s", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": f"the whole decomposition ({R} x {C}, rank {r}, l {l}) through the fp64 oracle, {dt:.1f} s"}
+    line = {
+        "metric": "TileQ Gaussian-sketch global low-rank decompositions/s", "value": 1000.0 / ms,
+        "unit": "sketch/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "replicas only", "vs_baseline": None, "dtype": "bf16/f32/f64",
+        "data": "synthetic (Gaussian bf16 expert weights and sketch, seeded)",
+        "config": {"workload": f"{cfg.name} gate W_big sketch", "rows": R, "cols": C, "rank": r, "sketch": l,
+                   "experts": K, "grid": f"{M}x{N}", "l2": "working set above L2"},
+        "roofline": {"bound": "tensor", "achieved": flops / (ms / 1000.0) / 1e12, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": t_roof / (ms / 1000.0), "traffic": None,
+                     "note": "large products only; the two l x l Jacobi eigen-decompositions (one CTA, "
+                             "latency-bound) take most of the time"},
+        "gpu_launches": launches, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     cfg = synth.CONFIGS[args.config]
     T = args.batch or (64 if args.config == 1 else cfg.batches[-1])
+    if args.sketch:
+        run_sketch(args, cfg)
+        return
     if args.impl == "reference":
         run_reference(args, cfg, T)
         return

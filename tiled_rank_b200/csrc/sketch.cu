@@ -236,7 +236,8 @@ __global__ void sk_gram_reduce_kernel(const double *part, int l, int splits, dou
 // two contiguous rows.  Then lam[i] = the i-th largest eigenvalue and perm[i]
 // the row of Et holding its eigenvector.
 constexpr int kJacobiSweeps = 40;
-constexpr int kJacobiThreads = 512;
+constexpr int kJacobiThreads = 1024;
+constexpr int kJacobiLaneCols = (kSketchMaxL + 31) / 32;  // row elements per lane
 
 __global__ void __launch_bounds__(kJacobiThreads) sk_jacobi_kernel(const double *Gin, int l, double *Et, double *lam,
                                                                   int *perm) {
@@ -246,6 +247,7 @@ __global__ void __launch_bounds__(kJacobiThreads) sk_jacobi_kernel(const double 
   __shared__ double red[32];
   __shared__ int done;
   const int tid = threadIdx.x, nt = blockDim.x;
+  const int warp = tid >> 5, lane = tid & 31, nwarp = nt >> 5;
   const int h = l / 2, ld = l + 1;
   for (int e = tid; e < l * l; e += nt) {
     G[(e / l) * ld + e % l] = Gin[e];
@@ -302,27 +304,47 @@ __global__ void __launch_bounds__(kJacobiThreads) sk_jacobi_kernel(const double 
         rq[tid] = q;
       }
       __syncthreads();
-      // rows p, q of every pair: J^T G; rows p, q of Et: (E J)^T
-      for (int e = tid; e < h * l; e += nt) {
-        const int i = e / l, j = e % l;
+      // rows p, q of every pair: J^T G; rows p, q of Et: (E J)^T.  One warp per
+      // pair, the lanes along the row (contiguous in G and in Et), the Et loads
+      // of the whole row out before its stores.
+      for (int i = warp; i < h; i += nwarp) {
         const int p = rp[i], q = rq[i];
         const double c = rc[i], sn = rs[i];
-        const double gp = G[p * ld + j], gq = G[q * ld + j];
-        G[p * ld + j] = c * gp - sn * gq;
-        G[q * ld + j] = sn * gp + c * gq;
-        const double ep = Et[(size_t)p * l + j], eq = Et[(size_t)q * l + j];
-        Et[(size_t)p * l + j] = c * ep - sn * eq;
-        Et[(size_t)q * l + j] = sn * ep + c * eq;
+        double ep[kJacobiLaneCols], eq[kJacobiLaneCols];
+#pragma unroll
+        for (int u = 0; u < kJacobiLaneCols; ++u) {
+          const int j = lane + 32 * u;
+          if (j < l) {
+            ep[u] = Et[(size_t)p * l + j];
+            eq[u] = Et[(size_t)q * l + j];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kJacobiLaneCols; ++u) {
+          const int j = lane + 32 * u;
+          if (j < l) {
+            const double gp = G[p * ld + j], gq = G[q * ld + j];
+            G[p * ld + j] = c * gp - sn * gq;
+            G[q * ld + j] = sn * gp + c * gq;
+            Et[(size_t)p * l + j] = c * ep[u] - sn * eq[u];
+            Et[(size_t)q * l + j] = sn * ep[u] + c * eq[u];
+          }
+        }
       }
       __syncthreads();
-      // columns p, q of every pair: (J^T G) J
-      for (int e = tid; e < h * l; e += nt) {
-        const int i = e / l, j = e % l;
+      // columns p, q of every pair: (J^T G) J (odd row stride: conflict-free)
+      for (int i = warp; i < h; i += nwarp) {
         const int p = rp[i], q = rq[i];
         const double c = rc[i], sn = rs[i];
-        const double gp = G[j * ld + p], gq = G[j * ld + q];
-        G[j * ld + p] = c * gp - sn * gq;
-        G[j * ld + q] = sn * gp + c * gq;
+#pragma unroll
+        for (int u = 0; u < kJacobiLaneCols; ++u) {
+          const int j = lane + 32 * u;
+          if (j < l) {
+            const double gp = G[j * ld + p], gq = G[j * ld + q];
+            G[j * ld + p] = c * gp - sn * gq;
+            G[j * ld + q] = sn * gp + c * gq;
+          }
+        }
       }
       __syncthreads();
     }
