@@ -678,7 +678,7 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   // at most four 16-byte chunks per thread
   const long long xchunks = x ? (long long)T * li.d_x / 8 : 0;
   const unsigned rblocks = std::max(nblocks(T, 8), std::min(nblocks(xchunks, 256 * 4), (unsigned)(8 * kNumSMs)));
-  route_kernel<<<rblocks, 256, 0, stream>>>(ra);
+  TQ_CUDA(launch_pdl(route_kernel, dim3(rblocks), dim3(256), 0, stream, ra));
   TQ_LAUNCHED();
   mark(ST_ROUTE, stream);
 
@@ -715,12 +715,12 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   const int P = T * top_k;
   if (P > kPermMultiMin) {
     const unsigned nc = (unsigned)cdiv(P, kPermChunk);
-    permute_count_kernel<<<nc, kPermChunkThreads, 0, stream>>>(pa);
+    TQ_CUDA(launch_pdl(permute_count_kernel, dim3(nc), dim3(kPermChunkThreads), 0, stream, pa));
     TQ_LAUNCHED();
-    permute_scatter_kernel<<<nc, kPermChunkThreads, 0, stream>>>(pa);
+    TQ_CUDA(launch_pdl(permute_scatter_kernel, dim3(nc), dim3(kPermChunkThreads), 0, stream, pa));
     TQ_LAUNCHED();
   } else {
-    permute_kernel<<<1, 1024, 0, stream>>>(pa);
+    TQ_CUDA(launch_pdl(permute_kernel, dim3(1), dim3(1024), 0, stream, pa));
     TQ_LAUNCHED();
   }
   mark(ST_PERMUTE, stream);
@@ -1035,7 +1035,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     // x' = w * x per slot in the first d_in columns of the activation matrix
     ScaleGatherArgs sg{plan.P, q.d_in, w.ld_x, at<int>(ws, w.slot_tok), at<float>(ws, w.slot_w),
                        at<__half>(ws, w.x16), xext};
-    scale_gather_kernel<<<nblocks((long long)plan.P * (q.d_in / 2), 256), 256, 0, stream>>>(sg);
+    TQ_CUDA(launch_pdl(scale_gather_kernel, dim3(nblocks((long long)plan.P * (q.d_in / 2), 256)), dim3(256), 0, stream, sg));
     TQ_LAUNCHED();
     if (q.rank > 0) {
       if ((st = run_zproj(layer, li, pl, packed, w, ws, 1, stream)) != TILEQ_OK) return st;
@@ -1049,7 +1049,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       la.zld = pad128(q.rank);
       la.zks = plan.zproj.ksplit;
       la.zsplit = (long long)T * layer->N * pad128(q.rank);
-      lr_accumulate_kernel<<<nblocks((long long)plan.P * 32, 256), 256, 0, stream>>>(la);
+      TQ_CUDA(launch_pdl(lr_accumulate_kernel, dim3(nblocks((long long)plan.P * 32, 256)), dim3(256), 0, stream, la));
       TQ_LAUNCHED();
     } else {
       mark(ST_ZPROJ, stream);
@@ -1097,7 +1097,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       ga.k = top_k;
       ga.slot_of_pair = at<int>(ws, w.slot_of_pair);
       const long long chunks = (long long)T * (D / 8) + (long long)plan.P * (lr_gu ? 2 * qg.rank / 8 : 0);
-      gather_ext_kernel<<<gather_blocks(chunks), 256, 0, stream>>>(ga);
+      TQ_CUDA(launch_pdl(gather_ext_kernel, dim3(gather_blocks(chunks)), dim3(256), 0, stream, ga));
       TQ_LAUNCHED();
     }
     mark(ST_ZPROJ, stream);
@@ -1163,7 +1163,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       la.zslot = at<float>(ws, w.zs);
       la.zks = plan.zdown.ksplit;
       la.zsplit = (long long)plan.P * qd.rank;
-      lr_accumulate_kernel<<<nblocks((long long)plan.P * 32, 256), 256, 0, stream>>>(la);
+      TQ_CUDA(launch_pdl(lr_accumulate_kernel, dim3(nblocks((long long)plan.P * 32, 256)), dim3(256), 0, stream, la));
       TQ_LAUNCHED();
     } else {
       mark(ST_ZDOWN, stream);
@@ -1300,7 +1300,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     const ProjInfo &q = li.p[0];
     ScaleGatherArgs sg{plan.P, q.d_in, w.ld_x, at<int>(ws, w.slot_tok), at<float>(ws, w.slot_w),
                        at<__half>(ws, w.x16), xext};
-    scale_gather_kernel<<<nblocks((long long)plan.P * (q.d_in / 2), 256), 256, 0, stream>>>(sg);
+    TQ_CUDA(launch_pdl(scale_gather_kernel, dim3(nblocks((long long)plan.P * (q.d_in / 2), 256)), dim3(256), 0, stream, sg));
     TQ_LAUNCHED();
     Residual r;
     r.b = xext;
@@ -1331,7 +1331,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     ga.T = T;
     ga.k = top_k;
     ga.slot_of_pair = at<int>(ws, w.slot_of_pair);
-    gather_ext_kernel<<<gather_blocks((long long)T * (D / 8)), 256, 0, stream>>>(ga);
+    TQ_CUDA(launch_pdl(gather_ext_kernel, dim3(gather_blocks((long long)T * (D / 8))), dim3(256), 0, stream, ga));
     TQ_LAUNCHED();
     Residual r;
     r.np = 2;
@@ -1352,7 +1352,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     mark(ST_ZPROJ, stream);
     SwigluArgs sa{(long long)plan.P * F, F, w.ld_h, at<float>(ws, w.g32), at<float>(ws, w.u32),
                   at<float>(ws, w.slot_w), hext};
-    swiglu_kernel<<<nblocks(sa.n, 256), 256, 0, stream>>>(sa);
+    TQ_CUDA(launch_pdl(swiglu_kernel, dim3(nblocks(sa.n, 256)), dim3(256), 0, stream, sa));
     TQ_LAUNCHED();
     mark(ST_GATEUP, stream);
     Residual rd;

@@ -190,6 +190,15 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
+// Programmatic dependent launch (the forward's kernels are launched with the
+// programmatic stream serialization attribute): wait until the previous kernel
+// in the stream has completed and its writes are visible, then let the next one
+// start its prologue.  Every CTA calls this before its first global memory
+// access, so a kernel never completes before its predecessor.
+__device__ __forceinline__ void pdl_wait_and_release() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
 // Hint: bring the line holding `p` into L2.
 __device__ __forceinline__ void prefetch_l2(const void *p) {
   asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p));

@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(DenseCfg<MB, BN>::THREADS, 1)
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the prologue above (barriers, TMEM) overlaps the previous kernel's tail
+  pdl_wait_and_release();
 
   const int n_tiles = P.tiles ? *P.tile_count : (P.static_items + BN - 1) / BN;
   auto tile_of = [&](int jt) {
@@ -271,7 +273,8 @@ cudaError_t launch_dense_one(const DenseArgs &a, int grid, cudaStream_t stream) 
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  kern<<<grid, C::THREADS, C::SMEM, stream>>>(a);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, stream, a);
+  if (e != cudaSuccess) return e;
   count_launches();
   return cudaGetLastError();
 }

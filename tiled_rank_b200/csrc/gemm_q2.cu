@@ -105,6 +105,7 @@ __device__ __forceinline__ void q2_store(const TcArgs &a, int item, int o, float
 
 template <int NP, int BN>
 __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(const __grid_constant__ TcArgs a) {
+  pdl_wait_and_release();
   using C = QCfg<NP, BN>;
   constexpr int SLOT = NP * BN * kRowsPerCta;  // floats of one fp32 partial
   extern __shared__ uint8_t smem_raw[];
@@ -470,7 +471,9 @@ cudaError_t launch_q2(const TcArgs &a, int n_tile_slots, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  kern<<<(unsigned)n_tile_slots * a.m_tiles * a.ksplit, QTHREADS, C::SMEM, stream>>>(a);
+  const cudaError_t e = launch_pdl(kern, dim3((unsigned)n_tile_slots * a.m_tiles * a.ksplit), dim3(QTHREADS), C::SMEM,
+                                   stream, a);
+  if (e != cudaSuccess) return e;
   count_launches();
   return cudaGetLastError();
 }

@@ -93,6 +93,7 @@ __device__ __forceinline__ void epi_store(const GemmProblem &P, int item, int o,
 
 template <int NP, int BN>
 __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_constant__ GemmBatch batch) {
+  pdl_wait_and_release();
   using C = SCfg<NP, BN>;
   const GemmProblem &P = batch.p[blockIdx.y];
   extern __shared__ uint8_t smem_raw[];
@@ -402,7 +403,8 @@ cudaError_t launch_one(const GemmBatch &batch, int nprob, int n_tile_slots, cuda
     if (batch.p[i].ksplit > 1 && (batch.p[i].m_tiles != mt || batch.p[i].ksplit != ks))
       return cudaErrorInvalidValue;
   const dim3 grid((unsigned)n_tile_slots * mt * ks, nprob);
-  kern<<<grid, THREADS, C::SMEM, stream>>>(batch);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(THREADS), C::SMEM, stream, batch);
+  if (e != cudaSuccess) return e;
   count_launches();
   return cudaGetLastError();
 }

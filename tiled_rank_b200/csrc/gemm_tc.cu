@@ -168,6 +168,8 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the prologue above (barriers, TMEM) overlaps the previous kernel's tail
+  pdl_wait_and_release();
 
   const int n_tiles = *P.tile_count;
   // tile jt: (group, first item, items)
@@ -642,7 +644,8 @@ cudaError_t launch_tc_one(const TcArgs &a, int grid, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  kern<<<grid, C::THREADS, C::SMEM, stream>>>(a);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, stream, a);
+  if (e != cudaSuccess) return e;
   count_launches();
   return cudaGetLastError();
 }

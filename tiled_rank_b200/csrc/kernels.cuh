@@ -105,6 +105,25 @@ struct GemmShape {
 // Process-wide count of kernel launches issued by the library.
 void count_launches(int n = 1);
 
+// Launch `kern` with programmatic stream serialization: it may be scheduled
+// while the previous kernel of the stream is still running and waits for it
+// in the kernel (pdl_wait_and_release).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Rows of A per CTA of the streaming GEMM (eight m16 consumer warps).
 constexpr int kRowsPerCta = 128;
 

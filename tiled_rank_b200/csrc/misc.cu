@@ -19,6 +19,7 @@ namespace tileq {
 // each lane then sums four consecutive elements over the pairs, all pairs'
 // loads in flight, in pair order and split order.
 __global__ void __launch_bounds__(256) lr_accumulate_kernel(LrAccArgs a) {
+  pdl_wait_and_release();
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= a.P) return;
@@ -116,6 +117,7 @@ __device__ __forceinline__ uint4 z_chunk(const GatherExtArgs &a, int s, int zc) 
 // to the token's k slot rows), then P * (nz*r/8) slot-major z chunks;
 // kGatherUnroll items per thread in flight.
 __global__ void __launch_bounds__(256) gather_ext_kernel(GatherExtArgs a) {
+  pdl_wait_and_release();
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long G = (long long)gridDim.x * blockDim.x;
   const int nz = a.z[0] ? (a.z[1] ? 2 : 1) : 0;
@@ -159,6 +161,7 @@ __global__ void __launch_bounds__(256) gather_ext_kernel(GatherExtArgs a) {
 // loaded together without spending registers on unused slots.
 template <int KT>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  pdl_wait_and_release();
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int d4 = a.d / 4;
   const int t = (int)(gid / d4), c = (int)(gid % d4);
@@ -186,7 +189,7 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream) {
   if (grid == 0) return cudaSuccess;
   switch (a.k) {
 #define TQ_COMBINE_K(K) \
-  case K: combine_kernel<K><<<grid, 256, 0, stream>>>(a); break;
+  case K: return launch_pdl(combine_kernel<K>, dim3(grid), dim3(256), 0, stream, a);
     TQ_COMBINE_K(1) TQ_COMBINE_K(2) TQ_COMBINE_K(3) TQ_COMBINE_K(4)
     TQ_COMBINE_K(5) TQ_COMBINE_K(6) TQ_COMBINE_K(7) TQ_COMBINE_K(8)
 #undef TQ_COMBINE_K
@@ -197,6 +200,7 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream) {
 
 // xs[slot][:] = w_slot * x16[token(slot)][:]  (fp16), for the linear layer.
 __global__ void scale_gather_kernel(ScaleGatherArgs a) {
+  pdl_wait_and_release();
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int d2 = a.d / 2;
   const int s = (int)(gid / d2), c = (int)(gid % d2);
@@ -209,6 +213,7 @@ __global__ void scale_gather_kernel(ScaleGatherArgs a) {
 
 // h[slot][f] = w_slot * silu(g) * u  (unfused path: activation after the per-expert adds)
 __global__ void swiglu_kernel(SwigluArgs a) {
+  pdl_wait_and_release();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.n) return;
   const int slot = (int)(i / a.F), f = (int)(i % a.F);

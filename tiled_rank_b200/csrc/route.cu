@@ -15,6 +15,7 @@
 namespace tileq {
 
 __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
+  pdl_wait_and_release();
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long gthreads = (long long)gridDim.x * blockDim.x;
   const int warp = (int)(gtid >> 5);
@@ -214,6 +215,7 @@ __device__ __forceinline__ void write_slot(const PermuteArgs &a, int p, int slot
 }
 
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
+  pdl_wait_and_release();
   __shared__ SortSmem s;
   __shared__ int scratch[kMaxExperts + 1];
   const int P = a.T * a.k;
@@ -236,6 +238,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
 // the same stable order as the one-CTA sort.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kPermChunkThreads) permute_count_kernel(PermuteArgs a) {
+  pdl_wait_and_release();
   __shared__ int hist[kMaxExperts];
   const int P = a.T * a.k;
   for (int e = threadIdx.x; e < a.K; e += blockDim.x) hist[e] = 0;
@@ -247,6 +250,7 @@ __global__ void __launch_bounds__(kPermChunkThreads) permute_count_kernel(Permut
 }
 
 __global__ void __launch_bounds__(kPermChunkThreads) permute_scatter_kernel(PermuteArgs a) {
+  pdl_wait_and_release();
   constexpr int W = kPermChunkThreads / 32;
   constexpr int kParts = kPermChunkThreads / kMaxExperts;
   static_assert(kPermChunk % W == 0 && kParts >= 1, "chunk split");
