@@ -26,7 +26,8 @@ PINS (what each function is checked against, in tests/test_oracle.py):
   unpack_codes / unpack_zeros / dequant ... hand-decoded golden fixture
       tests/golden/dequant_16x2.txt, plus a test-side packer
   route ... hand cases (tests/golden/route_cases.txt), softmax closed form,
-      brute-force top-k property on tiny inputs
+      brute-force top-k property on tiny inputs; the full-softmax variant
+      against the closed form (chosen mass = renormalised weights x that mass)
   permute ... brute-force stable sort definition on tiny inputs
   lowrank_block / expert_weight ... factored == reconstructed (1e-9),
       block of the global product U diag(Sigma) V^T (W_big), singular values of
@@ -63,12 +64,15 @@ def widen_fp16(h) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # routing (implicit on the pages; the plainest reading, see module docstring)
 # ---------------------------------------------------------------------------
-def route(logits, top_k: int):
-    """Exact top-k by a full sort and softmax weights over the chosen logits.
+def route(logits, top_k: int, full_softmax: bool = False):
+    """Exact top-k by a full sort and softmax weights.
 
     Order: descending logit; equal logits -> lower expert index first.
-    w_j = exp(l_j - l_max) / sum_{chosen} exp(l - l_max), in float64.
-    Returns (idx int32 [T, k], w float64 [T, k]).
+    Default: softmax over the chosen logits,
+        w_j = exp(l_j - l_max) / sum_{chosen} exp(l - l_max);
+    full_softmax: the chosen entries of the softmax over all K logits, not
+    renormalised, w_j = exp(l_j - l_max) / sum_{all K} exp(l - l_max).
+    Both in float64.  Returns (idx int32 [T, k], w float64 [T, k]).
     """
     lg = np.asarray(logits, dtype=np.float32)
     T, K = lg.shape
@@ -82,7 +86,11 @@ def route(logits, top_k: int):
         vals = np.array([float(lg[t, e]) for e in chosen], dtype=np.float64)
         ex = np.exp(vals - vals.max())
         idx[t] = chosen
-        w[t] = ex / ex.sum()
+        if full_softmax:
+            every = np.exp(lg[t].astype(np.float64) - vals.max())
+            w[t] = ex / every.sum()
+        else:
+            w[t] = ex / ex.sum()
     return idx, w
 
 
@@ -215,7 +223,7 @@ def forward(layer, x_bits, logits, tokens=None, return_h: bool = False):
     lg = np.asarray(logits, dtype=np.float32)
     T = x.shape[0]
     toks = list(range(T)) if tokens is None else [int(t) for t in tokens]
-    idx, w = route(lg[toks], layer.top_k)
+    idx, w = route(lg[toks], layer.top_k, getattr(layer, "route_mode", 0) == 1)
     cache = _WeightCache(layer)
     d_y = layer.projs[-1].d_out
     out = np.zeros((len(toks), d_y), dtype=np.float64)
@@ -249,7 +257,7 @@ def forward_batched(layer, x_bits, logits):
     """
     x = widen_bf16(x_bits)
     T = x.shape[0]
-    idx, w = route(logits, layer.top_k)
+    idx, w = route(logits, layer.top_k, getattr(layer, "route_mode", 0) == 1)
     d_y = layer.projs[-1].d_out
     out = np.zeros((T, d_y), dtype=np.float64)
     for e in range(layer.K):

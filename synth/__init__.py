@@ -97,6 +97,7 @@ class Layer:
     top_k: int
     projs: list              # LINEAR: [proj]; SWIGLU: [gate, up, down]
     shared: Optional[dict] = None  # {"gate","up": uint16 [Fs, D], "down": uint16 [D, Fs]}
+    route_mode: int = 0      # 0: softmax over the chosen logits; 1: chosen entries of the softmax over all K
 
     @property
     def d_x(self) -> int:

@@ -377,3 +377,24 @@ def test_memory_closed_form():
         tiled = oracle.lowrank_bytes_tiled(M, N, 1024, 1024, 64)
         per = oracle.lowrank_bytes_per_expert(M * N, 1024, 1024, 64)
         assert abs(per / tiled - expect) < 1e-12
+
+
+def test_route_full_softmax_variant():
+    """The chosen entries of the softmax over all K logits (not renormalised):
+    the same order as the default; weights = renormalised weights times the
+    chosen share of the full softmax mass; hand case below."""
+    rng = np.random.default_rng(4)
+    lg = (rng.standard_normal((20, 9)) * 2).astype(np.float32)
+    i0, w0 = oracle.route(lg, 3)
+    i1, w1 = oracle.route(lg, 3, full_softmax=True)
+    assert np.array_equal(i0, i1)
+    full = np.exp(lg.astype(np.float64) - lg.max(axis=1, keepdims=True))
+    full /= full.sum(axis=1, keepdims=True)
+    chosen = np.take_along_axis(full, i1.astype(np.int64), axis=1)
+    np.testing.assert_allclose(w1, chosen, rtol=1e-13)
+    np.testing.assert_allclose(w1, w0 * chosen.sum(axis=1, keepdims=True), rtol=1e-13)
+    assert np.all(w1.sum(axis=1) < 1.0)
+    # hand case: logits (0, ln 2, ln 3), top-2 -> 3/6 and 2/6
+    i, w = oracle.route(np.log(np.array([[1.0, 2.0, 3.0]], dtype=np.float32)), 2, full_softmax=True)
+    assert list(i[0]) == [2, 1]
+    np.testing.assert_allclose(w[0], [0.5, 1.0 / 3.0], rtol=1e-6)
