@@ -18,7 +18,10 @@
  *
  *   Routing (implicit on the pages: only a few experts are active per token):
  *   top-k of the fp32 router logits in descending order, equal logits -> the
- *   lower expert index first; weights = softmax over the k chosen logits.
+ *   lower expert index first; weights = softmax over the k chosen logits
+ *   (route_mode TILEQ_ROUTE_TOPK_SOFTMAX), or the k chosen entries of the
+ *   softmax over all K logits, not renormalised (TILEQ_ROUTE_FULL_SOFTMAX,
+ *   the routing variant of the TileQ summary's design notes).
  *   LINEAR layer:  out_t = sum_j w_j W_{e_j} x_t
  *   SWIGLU layer:  out_t = sum_j w_j W^down_{e_j} (silu(W^gate_{e_j} x_t) * (W^up_{e_j} x_t))
  *                  (+ an optional always-on dense bf16 SwiGLU shared expert, weight 1)
@@ -92,7 +95,12 @@ typedef struct {
  *                        proj[2] = down (d_model x d_ff); x and out are [T, d_model].
  *   shared_d_ff > 0 adds a dense SwiGLU shared expert (SWIGLU only):
  *   shared_w[0] gate, shared_w[1] up: device bf16 [shared_d_ff, d_model];
- *   shared_w[2] down: device bf16 [d_model, shared_d_ff]; shared_d_ff % 128 == 0. */
+ *   shared_w[2] down: device bf16 [d_model, shared_d_ff]; shared_d_ff % 128 == 0.
+ *   route_mode: TILEQ_ROUTE_TOPK_SOFTMAX (0, a zero-initialised struct) or
+ *   TILEQ_ROUTE_FULL_SOFTMAX; any other value -> TILEQ_ERR_INVALID_ARG.
+ *   tileq_route and tileq_route_static always route with mode 0. */
+#define TILEQ_ROUTE_TOPK_SOFTMAX 0
+#define TILEQ_ROUTE_FULL_SOFTMAX 1
 typedef struct {
   int kind;
   int K, M, N;            /* experts and grid; K <= M*N; K, M, N <= 64 */
@@ -100,12 +108,13 @@ typedef struct {
   tileq_proj proj[3];
   int shared_d_ff;
   const void *shared_w[3];
+  int route_mode;
 } tileq_layer;
 
 /* Optional copies of the routing results (device pointers, each may be NULL). */
 typedef struct {
   int32_t *topk_idx;        /* [T, top_k] expert ids, descending logit               */
-  float *topk_w;            /* [T, top_k] softmax weights over the chosen logits      */
+  float *topk_w;            /* [T, top_k] routing weights (per the layer's route_mode) */
   int32_t *expert_offsets;  /* [K+1] range of each expert in sorted_pairs             */
   int32_t *sorted_pairs;    /* [T*top_k] pair ids t*top_k+j, stably sorted by expert  */
 } tileq_route_out;

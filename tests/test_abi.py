@@ -48,17 +48,17 @@ def test_library_exports_every_declared_symbol(L):
 def test_struct_layout_matches_c(L, tmp_path):
     src = tmp_path / "layout.c"
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "tileq.h"\n'
-                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\\n",'
+                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n",'
                    'sizeof(tileq_proj), offsetof(tileq_proj, grid_assign), offsetof(tileq_proj, zeros),'
                    'sizeof(tileq_layer), offsetof(tileq_layer, proj), offsetof(tileq_layer, shared_d_ff),'
-                   'offsetof(tileq_layer, shared_w), sizeof(tileq_route_out), sizeof(tileq_per_expert_lr));'
+                   'offsetof(tileq_layer, shared_w), offsetof(tileq_layer, route_mode), sizeof(tileq_route_out), sizeof(tileq_per_expert_lr));'
                    'return 0;}\n')
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
     want = [ctypes.sizeof(L.tileq_proj), L.tileq_proj.grid_assign.offset, L.tileq_proj.zeros.offset,
             ctypes.sizeof(L.tileq_layer), L.tileq_layer.proj.offset, L.tileq_layer.shared_d_ff.offset,
-            L.tileq_layer.shared_w.offset, ctypes.sizeof(L.tileq_route_out),
+            L.tileq_layer.shared_w.offset, L.tileq_layer.route_mode.offset, ctypes.sizeof(L.tileq_route_out),
             ctypes.sizeof(L.tileq_per_expert_lr)]
     assert got == want
 
@@ -122,6 +122,13 @@ def test_validation_rejects_bad_layers(L):
     c.proj[0].d_in = 256
     with pytest.raises(L.TileQError) as e:
         L.tileq_workspace_size(c, 4, 5)                           # top_k > K
+    assert e.value.status == L.TILEQ_ERR_INVALID_ARG
+    c4, _ = _host_layer(L, 0)
+    c4.route_mode = L.TILEQ_ROUTE_FULL_SOFTMAX
+    assert L.tileq_packed_size(c4) == L.tileq_packed_size(_host_layer(L, 0)[0])
+    c4.route_mode = 2                                             # no such routing
+    with pytest.raises(L.TileQError) as e:
+        L.tileq_packed_size(c4)
     assert e.value.status == L.TILEQ_ERR_INVALID_ARG
 
 

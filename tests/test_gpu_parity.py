@@ -43,10 +43,11 @@ def run_gpu(torch, layer, logits, x, unfused=False, per_expert=None, dl=None):
     return to_numpy(out), {k: to_numpy(v) for k, v in route.items()}, dl
 
 
-def check_route(route, logits, top_k, K):
-    idx, w = oracle.route(logits, top_k)
+def check_route(route, logits, top_k, K, full_softmax=False):
+    idx, w = oracle.route(logits, top_k, full_softmax)
     assert np.array_equal(route["topk_idx"], idx)
-    np.testing.assert_allclose(route["topk_w"], w, rtol=2e-6, atol=1e-7)
+    # fp32 exp and a sum of up to 64 terms (full softmax) against fp64
+    np.testing.assert_allclose(route["topk_w"], w, rtol=1e-5 if full_softmax else 2e-6, atol=1e-7)
     off, sp = oracle.permute(idx, K)
     assert np.array_equal(route["expert_offsets"], off)
     assert np.array_equal(route["sorted_pairs"], sp)
@@ -141,6 +142,27 @@ def test_tiny_layers(torch_cuda, case):
         zr = zero_residual(layer)
         out, _, _ = run_gpu(torch_cuda, zr, logits, x)
         assert_parity(out, oracle.forward(zr, x, logits), f"{case} zero residual")
+
+
+# the routing variant: chosen entries of the softmax over all K logits; K = 60
+# takes the second logit per lane
+@pytest.mark.parametrize("case", [TINY[0], TINY[2], TINY[3],
+                                  (synth.SWIGLU, 60, 6, 10, 128, 128, 16, 64, 4, 0, 700)],
+                         ids=["swiglu", "shared", "linear", "k60"])
+def test_full_softmax_routing(torch_cuda, case):
+    import dataclasses
+    kind, K, M, N, dm, dff, r, g, k, sh, T = case
+    cfg = synth.tiny_config(kind=kind, K=K, M=M, N=N, d_model=dm, d_ff=dff, rank=r, group=g,
+                            top_k=k, shared_d_ff=sh)
+    layer = dataclasses.replace(synth.make_layer(cfg, seed=T + 1), route_mode=1)
+    logits, x = synth.make_inputs(cfg, T, seed=T + 1)
+    out, route, _ = run_gpu(torch_cuda, layer, logits, x)
+    check_route(route, logits, k, K, full_softmax=True)
+    ref = oracle.forward(layer, x, logits)
+    assert_parity(out, ref, f"full softmax {case}")
+    # the output follows the variant, not the default routing
+    default = oracle.forward(dataclasses.replace(layer, route_mode=0), x, logits)
+    assert np.abs(out - ref).max() < 0.25 * np.abs(out - default).max()
 
 
 @pytest.mark.parametrize("case", [TINY[0], TINY[3], TINY[2]], ids=["swiglu", "linear", "shared"])

@@ -22,6 +22,8 @@ TILEQ_ERR_CUDA = -4
 TILEQ_ERR_TIMEOUT = -5
 TILEQ_LINEAR = 0
 TILEQ_SWIGLU = 1
+TILEQ_ROUTE_TOPK_SOFTMAX = 0
+TILEQ_ROUTE_FULL_SOFTMAX = 1
 
 # every symbol include/tileq.h declares
 EXPORTS = (
@@ -57,6 +59,7 @@ class tileq_layer(ctypes.Structure):
         ("proj", tileq_proj * 3),
         ("shared_d_ff", ctypes.c_int),
         ("shared_w", ctypes.c_void_p * 3),
+        ("route_mode", ctypes.c_int),
     ]
 
 

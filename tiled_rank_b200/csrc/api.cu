@@ -52,6 +52,8 @@ struct LayerInfo {
 tileq_status validate_layer(const tileq_layer *L, LayerInfo *li, bool need_device_ptrs = true) {
   if (!L) return TILEQ_ERR_INVALID_ARG;
   if (L->kind != TILEQ_LINEAR && L->kind != TILEQ_SWIGLU) return TILEQ_ERR_INVALID_ARG;
+  if (L->route_mode != TILEQ_ROUTE_TOPK_SOFTMAX && L->route_mode != TILEQ_ROUTE_FULL_SOFTMAX)
+    return TILEQ_ERR_INVALID_ARG;
   if (L->K < 1 || L->M < 1 || L->N < 1 || (long long)L->M * L->N < L->K) return TILEQ_ERR_INVALID_ARG;
   if (L->K > kMaxExperts || L->M > kMaxExperts || L->N > kMaxExperts) return TILEQ_ERR_UNSUPPORTED;
   li->nproj = L->kind == TILEQ_LINEAR ? 1 : 3;
@@ -669,6 +671,7 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   ra.T = T;
   ra.K = L->K;
   ra.k = top_k;
+  ra.full_softmax = L->route_mode == TILEQ_ROUTE_FULL_SOFTMAX;
   ra.topk_idx = at<int32_t>(ws, w.topk_idx);
   ra.topk_w = at<float>(ws, w.topk_w);
   ra.zero = at<int>(ws, w.counters);

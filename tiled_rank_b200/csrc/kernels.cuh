@@ -12,6 +12,7 @@ struct RouteArgs {
   const __nv_bfloat16 *x;  // may be null (route only)
   __half *x16;
   int d_x, T, K, k;
+  int full_softmax;        // 1: the chosen entries of the softmax over all K logits
   int32_t *topk_idx;
   float *topk_w;
   int *zero;               // split-K arrival counters, cleared for this forward

@@ -2,7 +2,8 @@
 //
 // route_kernel    : one warp per token: exact top-k of the fp32 logits (descending,
 //                   equal logits -> lower expert id), softmax over the chosen
-//                   logits, and the bf16 -> fp16 conversion of the token's x row.
+//                   logits (or, full_softmax, their entries of the softmax over
+//                   all K logits), and the bf16 -> fp16 conversion of x.
 // permute_kernel  : one CTA: deterministic stable counting sort of the
 //                   (token, slot) pairs by expert and the GEMM tile table; per
 //                   slot, the row of the projected [T, N, r] tensor it reads
@@ -78,6 +79,13 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j)
     if (j < a.k) sum += expf(sel_v[j] - sel_v[0]);
+  if (a.full_softmax) {
+    // the denominator runs over every logit; sel_v[0] is the row maximum
+    float s = (lane < a.K ? expf(v0 - sel_v[0]) : 0.f) + (lane + 32 < a.K ? expf(v1 - sel_v[0]) : 0.f);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    sum = s;
+  }
   if (lane == 0) {
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {

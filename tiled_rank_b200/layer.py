@@ -64,6 +64,7 @@ class DeviceLayer:
             cp.U = L._ptr(tens.get("U"))
             cp.V = L._ptr(tens.get("V"))
             cp.Sigma = L._ptr(tens.get("Sigma"))
+        c.route_mode = int(getattr(layer, "route_mode", 0))
         c.shared_d_ff = 0
         if layer.shared is not None:
             c.shared_d_ff = int(layer.shared["gate"].shape[0])
