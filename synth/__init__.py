@@ -240,3 +240,31 @@ def tiny_config(kind=SWIGLU, K=4, M=2, N=2, d_model=64, d_ff=128, rank=8, group=
     """A small configuration for tests (oracle runs it in milliseconds)."""
     return Config(f"tiny-{kind}-{K}e", kind, K, M, N, d_model, d_ff, rank, group, top_k, (16,),
                   logit_std=logit_std, zipf_s=zipf_s, shared_d_ff=shared_d_ff)
+
+
+def planted_factors(K: int, M: int, N: int, d_u: int, d_v: int, r0: int, noise: float = 0.05,
+                    seed: int = 0):
+    """Per-expert rank-r0 factors with a planted grid structure.
+
+    A seeded injective expert -> cell map (the planted grid_assign) puts expert
+    k in cell (m_k, n_k); its left factor is an orthonormal basis of
+    A_{m_k} + noise * G_k and its right factor one of B_{n_k} + noise * H_k
+    (A_m [d_u, r0], B_n [d_v, r0], G_k, H_k standard normal), each column then
+    multiplied by a random sign, as an SVD would return it.  Experts of one
+    grid row thus have nearby left subspaces, experts of one column nearby
+    right subspaces.  Returns (u fp32 [K, d_u, r0], v fp32 [K, d_v, r0],
+    planted grid_assign int32 [K]).
+    """
+    rng = np.random.default_rng([seed, 5])
+    cells = rng.permutation(M * N)[:K].astype(np.int32)
+    A = rng.standard_normal((M, d_u, r0))
+    B = rng.standard_normal((N, d_v, r0))
+    u = np.empty((K, d_u, r0), dtype=np.float32)
+    v = np.empty((K, d_v, r0), dtype=np.float32)
+    for k in range(K):
+        m, n = divmod(int(cells[k]), N)
+        qu, _ = np.linalg.qr(A[m] + noise * rng.standard_normal((d_u, r0)))
+        qv, _ = np.linalg.qr(B[n] + noise * rng.standard_normal((d_v, r0)))
+        u[k] = qu * rng.choice([-1.0, 1.0], size=r0)[None, :]
+        v[k] = qv * rng.choice([-1.0, 1.0], size=r0)[None, :]
+    return u, v, cells
