@@ -208,8 +208,6 @@ tileq_status tileq_route(const float *router_logits, int T, int K, int top_k,
 tileq_status tileq_route_static(const float *router_logits, int T, int K, int top_k,
                                 tileq_route_out *route, tileq_stream_t stream);
 
-/* Synchronously read (and clear) the device status word in `ws`.
- * *status receives TILEQ_OK or the first device error recorded. */
 /* ---------------------------------------------------------------------------
  * Global low-rank decomposition of W_big by Gaussian sketching (TileQ summary,
  * section 2.1, step 5 "Quantization": the large tiled matrix W_big undergoes a
@@ -251,6 +249,64 @@ tileq_status tileq_sketch_lowrank(const tileq_wbig *w, const void *omega_t, int 
                                   float *sigma, float *V, void *ws, size_t ws_bytes,
                                   tileq_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Expert placement on the M x N grid (TileQ summary, section 2.1, steps 2-4:
+ * "Extracting" -- the rank-r0 SVD factors (U_k, V_k) of each expert,
+ * vectorised and normalised into feature embeddings; "Clustering" -- a
+ * biclustering by K-Means gives each expert an ideal grid coordinate (m, n);
+ * "2D-Tiling Placement" -- a greedy spatial allocation resolves experts that
+ * want the same tile, minimising the distance between ideal and actual tile).
+ * The result is the grid_assign that W_big, tileq_sketch_lowrank and
+ * tileq_pack take.
+ *
+ * Steps (the pages give no more detail; these are the plainest readings):
+ *   embedding: each factor column is multiplied by the sign of its entry of
+ *     largest magnitude (the first such row on ties), the factor is flattened
+ *     row-major and divided by its L2 norm (a zero factor stays zero);
+ *   rows: K-Means on the U-embeddings with min(M, K) clusters; columns:
+ *     K-Means on the V-embeddings with min(N, K) clusters (rows of the grid
+ *     share the left basis, columns the right basis);
+ *   K-Means: Lloyd's algorithm on squared Euclidean distance; first centre =
+ *     expert 0, each further centre = the expert farthest from the centres
+ *     so far (ties -> lowest index); assignment to the nearest centre (ties
+ *     -> lowest centre index); a centre with no experts keeps its place; stop
+ *     when an update changes no assignment or after max_iter updates;
+ *   greedy: repeatedly place the (unplaced expert, free cell) pair with the
+ *     smallest squared grid distance (m - m*)^2 + (n - n*)^2 to the expert's
+ *     ideal (m*, n*), ties -> lower expert index, then lower cell m*N + n.
+ * The GPU evaluates the K-Means distances from the fp64 Gram matrix of the
+ * embeddings, which it builds in one pass over the factors.
+ * ------------------------------------------------------------------------- */
+#define TILEQ_PLACE_MAX_R0 256
+#define TILEQ_PLACE_MAX_ITER 65536
+
+typedef struct {
+  int K, M, N;          /* experts and grid: 1 <= K <= M*N; K, M, N <= 64 */
+  int d_u, d_v, r0;     /* factor shapes: U_k [d_u][r0], V_k [d_v][r0]; 1 <= r0 <= TILEQ_PLACE_MAX_R0 */
+  const float *u;       /* device fp32 [K][d_u][r0], row-major: the left (output-space) factors */
+  const float *v;       /* device fp32 [K][d_v][r0]: the right (input-space) factors */
+  int max_iter;         /* cap on the K-Means centre updates, 1..TILEQ_PLACE_MAX_ITER */
+} tileq_place_in;
+
+typedef struct {
+  int32_t *grid_assign; /* device [K]: cell m*N + n of expert k (required) */
+  int32_t *ideal;       /* device [K][2]: the ideal (m, n) from the two K-Means, or NULL */
+  int32_t *iterations;  /* device [2]: centre updates run on the U side and the V side, or NULL */
+} tileq_place_out;
+
+/* Workspace bytes of tileq_place_experts (host only). */
+tileq_status tileq_place_workspace_size(const tileq_place_in *in, size_t *bytes);
+
+/* Embeddings, both K-Means and the greedy placement, asynchronous on stream.
+ * Shapes outside the limits above -> TILEQ_ERR_UNSUPPORTED, NULL pointers or
+ * max_iter < 1 -> TILEQ_ERR_INVALID_ARG, a short workspace ->
+ * TILEQ_ERR_WORKSPACE; all checked on the host before any launch.  The factors
+ * must stay valid until the stream reaches the call. */
+tileq_status tileq_place_experts(const tileq_place_in *in, tileq_place_out *out, void *ws,
+                                 size_t ws_bytes, tileq_stream_t stream);
+
+/* Synchronously read (and clear) the device status word in `ws`.
+ * *status receives TILEQ_OK or the first device error recorded. */
 tileq_status tileq_device_status(void *ws, int *status, tileq_stream_t stream);
 
 /* Self-test of the bounded device wait: launches one block that waits on an

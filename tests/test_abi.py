@@ -225,3 +225,48 @@ def test_sketch_workspace_and_validation(L):
     bad.K = 3
     with pytest.raises(L.TileQError):
         L.tileq_sketch_workspace_size(bad, 8, 4)          # K != M*N
+
+
+def test_place_layout_matches_c(L, tmp_path):
+    src = tmp_path / "place.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "tileq.h"\n'
+                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %d\\n", sizeof(tileq_place_in),'
+                   'offsetof(tileq_place_in, u), offsetof(tileq_place_in, max_iter), sizeof(tileq_place_out),'
+                   'offsetof(tileq_place_out, ideal), offsetof(tileq_place_out, iterations),'
+                   'TILEQ_PLACE_MAX_R0); return 0;}\n')
+    exe = tmp_path / "place"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
+    assert got == [ctypes.sizeof(L.tileq_place_in), L.tileq_place_in.u.offset, L.tileq_place_in.max_iter.offset,
+                   ctypes.sizeof(L.tileq_place_out), L.tileq_place_out.ideal.offset,
+                   L.tileq_place_out.iterations.offset, L.TILEQ_PLACE_MAX_R0]
+
+
+def _place(L, K, M, N, d_u=64, d_v=32, r0=8, max_iter=100):
+    c = L.tileq_place_in()
+    c.K, c.M, c.N, c.d_u, c.d_v, c.r0, c.max_iter = K, M, N, d_u, d_v, r0, max_iter
+    c.u = c.v = 16   # never dereferenced by the host checks
+    return c
+
+
+def test_place_workspace_and_validation(L):
+    """Errors are returned on the host, before any launch (no device needed)."""
+    n = L.tileq_place_workspace_size(_place(L, 64, 8, 8, r0=16))
+    assert n >= 2 * 148 * 64 * 64 * 8 + 2 * 64 * 64 * 8 + 2 * 64 * 16 * 12
+    for bad, want in [((65, 8, 9), L.TILEQ_ERR_UNSUPPORTED), ((9, 2, 4), L.TILEQ_ERR_INVALID_ARG),
+                      ((4, 2, 65), L.TILEQ_ERR_UNSUPPORTED), ((0, 2, 2), L.TILEQ_ERR_INVALID_ARG)]:
+        with pytest.raises(L.TileQError) as e:
+            L.tileq_place_workspace_size(_place(L, *bad))
+        assert e.value.status == want, bad
+    for kw, want in [(dict(r0=257), L.TILEQ_ERR_UNSUPPORTED), (dict(r0=0), L.TILEQ_ERR_INVALID_ARG),
+                     (dict(max_iter=0), L.TILEQ_ERR_INVALID_ARG), (dict(d_v=0), L.TILEQ_ERR_INVALID_ARG),
+                     (dict(max_iter=65537), L.TILEQ_ERR_UNSUPPORTED)]:
+        with pytest.raises(L.TileQError) as e:
+            L.tileq_place_workspace_size(_place(L, 4, 2, 2, **kw))
+        assert e.value.status == want, kw
+    out = L.tileq_place_out(None, None, None)      # grid_assign is required
+    st = L.lib().tileq_place_experts(ctypes.byref(_place(L, 4, 2, 2)), ctypes.byref(out), 16, 1 << 30, None)
+    assert st == L.TILEQ_ERR_INVALID_ARG
+    out = L.tileq_place_out(16, None, None)
+    st = L.lib().tileq_place_experts(ctypes.byref(_place(L, 4, 2, 2)), ctypes.byref(out), 16, 8, None)
+    assert st == L.TILEQ_ERR_WORKSPACE

@@ -32,8 +32,10 @@ EXPORTS = (
     "tileq_moe_forward_unfused", "tileq_route", "tileq_route_static", "tileq_device_status",
     "tileq_selftest_bounded_wait", "tileq_set_stage_events", "tileq_launch_count",
     "tileq_sketch_workspace_size", "tileq_sketch_lowrank",
+    "tileq_place_workspace_size", "tileq_place_experts",
 )
 TILEQ_SKETCH_MAX_L = 160
+TILEQ_PLACE_MAX_R0 = 256
 
 
 class TileQError(RuntimeError):
@@ -76,6 +78,19 @@ class tileq_wbig(ctypes.Structure):
     ]
 
 
+class tileq_place_in(ctypes.Structure):
+    _fields_ = [
+        ("K", ctypes.c_int), ("M", ctypes.c_int), ("N", ctypes.c_int),
+        ("d_u", ctypes.c_int), ("d_v", ctypes.c_int), ("r0", ctypes.c_int),
+        ("u", ctypes.c_void_p), ("v", ctypes.c_void_p), ("max_iter", ctypes.c_int),
+    ]
+
+
+class tileq_place_out(ctypes.Structure):
+    _fields_ = [("grid_assign", ctypes.c_void_p), ("ideal", ctypes.c_void_p),
+                ("iterations", ctypes.c_void_p)]
+
+
 class tileq_per_expert_lr(ctypes.Structure):
     _fields_ = [("U_pe", ctypes.c_void_p * 3), ("V_pe", ctypes.c_void_p * 3)]
 
@@ -105,6 +120,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "tileq_launch_count": ([P(ctypes.c_ulonglong)], c_int),
         "tileq_sketch_workspace_size": ([P(tileq_wbig), c_int, c_int, P(c_size)], c_int),
         "tileq_sketch_lowrank": ([P(tileq_wbig), vp, c_int, c_int, vp, vp, vp, vp, c_size, vp], c_int),
+        "tileq_place_workspace_size": ([P(tileq_place_in), P(c_size)], c_int),
+        "tileq_place_experts": ([P(tileq_place_in), P(tileq_place_out), vp, c_size, vp], c_int),
     }
     for name, (argtypes, restype) in sigs.items():
         fn = getattr(lib, name)
@@ -258,3 +275,27 @@ def tileq_sketch_lowrank(wbig: tileq_wbig, omega, l: int, r: int, U, sigma, V, w
     _check(lib().tileq_sketch_lowrank(ctypes.byref(wbig), _ptr(omega), l, r, _ptr(U), _ptr(sigma),
                                       _ptr(V), _ptr(ws), ws.numel() * ws.element_size(),
                                       _stream(stream)), "tileq_sketch_lowrank")
+
+
+def place_in(u, v, M: int, N: int, max_iter: int = 100) -> tileq_place_in:
+    """The placement input for device fp32 factors u [K, d_u, r0], v [K, d_v, r0]."""
+    K, d_u, r0 = (int(x) for x in u.shape)
+    if tuple(v.shape[::2]) != (K, r0):
+        raise ValueError("u and v must share K and r0")
+    c = tileq_place_in()
+    c.K, c.M, c.N, c.d_u, c.d_v, c.r0 = K, M, N, d_u, int(v.shape[1]), r0
+    c.u, c.v, c.max_iter = _ptr(u), _ptr(v), max_iter
+    return c
+
+
+def tileq_place_workspace_size(pin: tileq_place_in) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().tileq_place_workspace_size(ctypes.byref(pin), ctypes.byref(n)), "tileq_place_workspace_size")
+    return n.value
+
+
+def tileq_place_experts(pin: tileq_place_in, grid_assign, ws, ideal=None, iterations=None, stream=None):
+    out = tileq_place_out(_ptr(grid_assign), _ptr(ideal), _ptr(iterations))
+    _check(lib().tileq_place_experts(ctypes.byref(pin), ctypes.byref(out), _ptr(ws),
+                                     ws.numel() * ws.element_size() if ws is not None else 0,
+                                     _stream(stream)), "tileq_place_experts")
