@@ -64,6 +64,10 @@ def parse():
     ap.add_argument("--sketch", action="store_true",
                     help="time the Gaussian-sketch global low-rank decomposition of one projection's W_big "
                          "(the configuration's gate projection) instead of the forward")
+    ap.add_argument("--place", action="store_true",
+                    help="time the expert placement (embeddings, K-Means biclustering, greedy 2D placement) "
+                         "of the configuration's gate projection instead of the forward")
+    ap.add_argument("--r0", type=int, default=16, help="rank of the per-expert factors for --place")
     return ap.parse_args()
 
 
@@ -282,12 +286,125 @@ def run_sketch(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+FP64_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12   # SMs x fp64 FMA/clk/SM x 2 x max SM clock
+
+
+def run_place(args, cfg):
+    """Expert placement of the configuration's gate projection: per-expert rank-r0
+    factors U_k [d_ff, r0] and V_k [d_model, r0] with a planted grid (synthetic,
+    seeded), embeddings + both K-Means + greedy placement per step."""
+    import torch
+    from tiled_rank_b200 import _lib as L
+    if int(os.environ.get("RANK", "0")) != 0:
+        return  # one placement: replicas would only repeat it
+    if args.warmup < 3:
+        raise SystemExit("at least 3 warm-up steps")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    K, M, N, r0 = cfg.K, cfg.M, cfg.N, args.r0
+    d_u, d_v = cfg.d_ff, cfg.d_model
+    u_np, v_np, _ = synth.planted_factors(K, M, N, d_u, d_v, r0, noise=0.1, seed=args.seed)
+    u = torch.from_numpy(u_np).to(dev)
+    v = torch.from_numpy(v_np).to(dev)
+    pin = L.place_in(u, v, M, N, 100)
+    ws = torch.empty(L.tileq_place_workspace_size(pin), dtype=torch.uint8, device=dev)
+    grid = torch.empty((K,), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush_buf = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)   # 2x L2: inputs are smaller
+    for _ in range(args.warmup):
+        L.tileq_place_experts(pin, grid, ws)
+    torch.cuda.synchronize()
+    nst = 5
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
+    for sev in sevs:
+        for e in sev:
+            e.record(stream)
+    torch.cuda.synchronize()
+    n0 = L.tileq_launch_count()
+    with ClockSampler(0) as clocks:
+        for i in range(args.steps):
+            flush_buf.zero_()
+            ev[2 * i].record(stream)
+            L.tileq_place_experts(pin, grid, ws)
+            ev[2 * i + 1].record(stream)
+        torch.cuda.synchronize()
+    launches = L.tileq_launch_count() - n0
+    # per-stage device times from a second pass of the same steps, with the
+    # library's stage-boundary events on (kept out of the timed pass above)
+    for i in range(args.steps):
+        flush_buf.zero_()
+        L.tileq_set_stage_events(sevs[i])
+        L.tileq_place_experts(pin, grid, ws)
+    torch.cuda.synchronize()
+    L.tileq_set_stage_events(None)
+    ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps)) / args.steps
+    names = ["sign", "gram", "cluster", "greedy"]
+    stage_ms = {n: sum(sevs[i][j].elapsed_time(sevs[i][j + 1]) for i in range(args.steps)) / args.steps
+                for j, n in enumerate(names)}
+    # end to end through the C ABI: factors from pinned host memory, grid_assign back to the host
+    u_h = torch.from_numpy(u_np).pin_memory()
+    v_h = torch.from_numpy(v_np).pin_memory()
+    g_h = torch.empty((K,), dtype=torch.int32).pin_memory()
+    u_d, v_d = torch.empty_like(u), torch.empty_like(v)
+    pin_e = L.place_in(u_d, v_d, M, N, 100)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for i in range(args.warmup + args.steps):
+        flush_buf.zero_()
+        e0.record(stream)
+        u_d.copy_(u_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        L.tileq_place_experts(pin_e, grid, ws)
+        g_h.copy_(grid, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms += e0.elapsed_time(e1)
+    e2e_ms /= args.steps
+    D = (d_u + d_v) * r0
+    gram_flops = 2.0 * K * (K + 1) / 2 * D        # the symmetric half of E E^T, both sides
+    in_bytes = K * D * 4
+    cpu = None
+    if not args.no_cpu_baseline:
+        from oracle import placement as opl
+        t0 = time.perf_counter()
+        opl.place_experts(u_np, v_np, M, N, 100)
+        dt = time.perf_counter() - t0
+        cpu = {"value": 1.0 / dt, "unit": "placements/s", "cores": len(os.sched_getaffinity(0)),
+               "kind": "oracle", "sample": f"one whole placement ({K} experts, factors {d_u}+{d_v} x {r0}) "
+                                           f"through the fp64 oracle, {dt:.2f} s"}
+    line = {
+        "metric": "TileQ expert placements/s (embeddings + K-Means biclustering + greedy 2D placement)",
+        "value": 1000.0 / ms, "unit": "placements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "replicas only", "vs_baseline": None,
+        "dtype": "f32 in, f64", "data": "synthetic (planted-grid orthonormal factors with random column signs, "
+                                        "seeded)",
+        "config": {"workload": f"{cfg.name} gate-projection expert placement", "experts": K, "grid": f"{M}x{N}",
+                   "d_u": d_u, "d_v": d_v, "r0": r0, "l2": "flushed between steps (inputs smaller than L2)"},
+        "stages_ms": stage_ms,
+        "roofline": {"bound": "alu", "achieved": gram_flops / (stage_ms["gram"] / 1000.0) / 1e12,
+                     "peak": FP64_TFLOPS, "unit": "TFLOP/s",
+                     "frac": gram_flops / (stage_ms["gram"] / 1000.0) / 1e12 / FP64_TFLOPS, "traffic": None,
+                     "kernel": "pl_gram_kernel (fp64 Gram of the embeddings, symmetric half counted)",
+                     "hbm_floor_us": in_bytes / (measured_peaks()["hbm_gbs"] * 1e9) * 1e6,
+                     "note": "peak derived: 148 SMs x 64 fp64 FMA/clk x 2 x 1965 MHz"},
+        "e2e": {"value": 1000.0 / e2e_ms, "unit": "placements/s", "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": K * 4},
+        "gpu_launches": launches, "clocks": clocks.report(), "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     cfg = synth.CONFIGS[args.config]
     T = args.batch or (64 if args.config == 1 else cfg.batches[-1])
     if args.sketch:
         run_sketch(args, cfg)
+        return
+    if args.place:
+        run_place(args, cfg)
         return
     if args.impl == "reference":
         run_reference(args, cfg, T)

@@ -322,7 +322,10 @@ tileq_status tileq_selftest_bounded_wait(void *ws, size_t ws_bytes, int max_poll
  * permutation, 3 after the column projection z = Sigma*(V_n^T x), 4 after the
  * gate/up (or linear residual input) GEMM, 5 after the down-side projection,
  * 6 after the row accumulation, 7 after the combined residual GEMM, 8 after
- * the shared expert, 9 after the combine.  Events past n_events are skipped.
+ * the shared expert, 9 after the combine.  tileq_place_experts records 0
+ * before its first launch, 1 after the sign pass, 2 after the Gram pass, 3
+ * after both K-Means, 4 after the greedy placement.  Events past n_events are
+ * skipped.
  * Process-wide, not thread-safe; host only. */
 tileq_status tileq_set_stage_events(void **events, int n_events);
 

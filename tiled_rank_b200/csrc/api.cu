@@ -1529,6 +1529,7 @@ extern "C" tileq_status tileq_route_static(const float *router_logits, int T, in
 
 namespace tileq {
 void count_launches(int n) { g_launches.fetch_add((unsigned long long)n); }
+void mark_stage(int stage, cudaStream_t stream) { mark(stage, stream); }
 bool tensor_map_2b(CUtensorMap *m, const void *base, int rows, int cols, int ld, int box_rows) {
   return make_map(m, base, rows, cols, ld, box_rows);
 }

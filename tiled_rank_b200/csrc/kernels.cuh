@@ -105,6 +105,8 @@ struct GemmShape {
 
 // Process-wide count of kernel launches issued by the library.
 void count_launches(int n = 1);
+// Record stage-boundary event `stage` of the timing hook (no-op while it is off).
+void mark_stage(int stage, cudaStream_t stream);
 
 // Launch `kern` with programmatic stream serialization: it may be scheduled
 // while the previous kernel of the stream is still running and waits for it
