@@ -23,7 +23,9 @@ top-k is an exact full sort: no blocking, fusion or reordering.
 
 PINS (what each function is checked against, in tests/test_oracle.py):
   widen_bf16 / widen_fp16 ... exact bit patterns of known values
-  unpack_codes / unpack_zeros / dequant ... hand-decoded golden fixture
+  unpack_codes / unpack_zeros / dequant ... hand-decoded golden fixture (2-bit);
+      3-bit: hand-decoded case, a zero high plane reduces to the 2-bit result,
+      and the residual range |q - z| <= 7
       tests/golden/dequant_16x2.txt, plus a test-side packer
   route ... hand cases (tests/golden/route_cases.txt), softmax closed form,
       brute-force top-k property on tiny inputs; the full-softmax variant
@@ -40,7 +42,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "widen_bf16", "widen_fp16", "route", "permute", "unpack_codes", "unpack_zeros",
+    "widen_bf16", "widen_fp16", "route", "permute", "unpack_codes", "unpack_zeros", "unpack_codes_hi",
     "dequant", "grid_cell", "lowrank_block", "expert_weight", "silu", "forward",
     "forward_batched", "assemble_wbig_lowrank", "lowrank_bytes_tiled",
     "lowrank_bytes_per_expert",
@@ -126,20 +128,35 @@ def unpack_codes(codes, d_in: int) -> np.ndarray:
     return q.reshape(c.shape[:-1] + (c.shape[-1] * 16,))[..., :d_in].astype(np.uint8)
 
 
-def unpack_zeros(zeros, n_groups: int) -> np.ndarray:
-    """uint8 [..., ceil(G/4)] -> zero points uint8 [..., G]; group j at bits 2*(j%4) of byte j//4."""
+def unpack_zeros(zeros, n_groups: int, bits: int = 2) -> np.ndarray:
+    """Zero points uint8 [..., G].  2-bit: uint8 [..., ceil(G/4)], group j at bits
+    2*(j%4) of byte j//4.  3-bit: uint8 [..., ceil(G/2)], group j at bits 4*(j%2)
+    of byte j//2 (values 0..7)."""
     zb = np.asarray(zeros, dtype=np.uint8)
-    shifts = (2 * np.arange(4, dtype=np.uint8))
-    z = (zb[..., None] >> shifts) & np.uint8(3)
-    return z.reshape(zb.shape[:-1] + (zb.shape[-1] * 4,))[..., :n_groups]
+    per, width, mask = (4, 2, 3) if bits != 3 else (2, 4, 7)
+    shifts = (width * np.arange(per, dtype=np.uint8))
+    z = (zb[..., None] >> shifts) & np.uint8(mask)
+    return z.reshape(zb.shape[:-1] + (zb.shape[-1] * per,))[..., :n_groups]
+
+
+def unpack_codes_hi(codes_hi, d_in: int) -> np.ndarray:
+    """3-bit codes' high bits: uint32 [..., d_in/32] -> uint8 [..., d_in]; element j at bit j%32."""
+    c = np.asarray(codes_hi, dtype=np.uint32)
+    q = (c[..., None] >> np.arange(32, dtype=np.uint32)) & np.uint32(1)
+    return q.reshape(c.shape[:-1] + (c.shape[-1] * 32,))[..., :d_in].astype(np.uint8)
 
 
 def dequant(proj, e: int) -> np.ndarray:
-    """deq(Q_e) float64 [d_out, d_in]: w[o, i] = s[o, i//g] * (q[o, i] - z[o, i//g])."""
+    """deq(Q_e) float64 [d_out, d_in]: w[o, i] = s[o, i//g] * (q[o, i] - z[o, i//g]).
+    2-bit: q from `codes`; 3-bit (proj.bits == 3): q = codes + 4 * codes_hi bit."""
     g = proj.group
     G = proj.d_in // g
-    q = unpack_codes(proj.codes[e], proj.d_in).reshape(proj.d_out, G, g)
-    z = unpack_zeros(proj.zeros[e], G).astype(np.float64)
+    bits = getattr(proj, "bits", 2)
+    q = unpack_codes(proj.codes[e], proj.d_in).astype(np.int64)
+    if bits == 3:
+        q = q + 4 * unpack_codes_hi(proj.codes_hi[e], proj.d_in)
+    q = q.reshape(proj.d_out, G, g)
+    z = unpack_zeros(proj.zeros[e], G, bits).astype(np.float64)
     s = widen_fp16(proj.scales[e])
     # group j of row o covers inputs j*g .. j*g+g-1
     w = (q - z[:, :, None]) * s[:, :, None]

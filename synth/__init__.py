@@ -79,7 +79,9 @@ class Proj:
     V: np.ndarray            # uint16 (bf16 bits) [N*d_in, r]
     codes: np.ndarray        # uint32 [K, d_out, d_in/16]
     scales: np.ndarray       # float16 [K, d_out, d_in/g]
-    zeros: np.ndarray        # uint8 [K, d_out, ceil(d_in/g/4)]
+    zeros: np.ndarray        # uint8 [K, d_out, ceil(G/4)] (2-bit) or [K, d_out, ceil(G/2)] (3-bit)
+    bits: int = 2            # 2 or 3 (3: q = codes + 4 * bit of codes_hi)
+    codes_hi: Optional[np.ndarray] = None  # 3-bit: uint32 [K, d_out, d_in/32], element j at bit j%32
 
     @property
     def n_groups(self) -> int:
@@ -129,6 +131,7 @@ class Config:
     zipf_s: float = 0.0
     shared_d_ff: int = 0
     per_expert_layout: bool = False
+    bits: int = 2
 
 
 CONFIGS = {
@@ -155,7 +158,7 @@ def proj_shapes(kind: int, d_model: int, d_ff: int):
     return [(d_model, d_ff), (d_model, d_ff), (d_ff, d_model)]
 
 
-def _make_proj(rng, K, M, N, d_in, d_out, rank, group) -> Proj:
+def _make_proj(rng, K, M, N, d_in, d_out, rank, group, bits=2) -> Proj:
     if d_in % 16 or d_in % group:
         raise ValueError("d_in must be a multiple of 16 and of the group size")
     G = d_in // group
@@ -171,7 +174,16 @@ def _make_proj(rng, K, M, N, d_in, d_out, rank, group) -> Proj:
         zeros[..., -1] &= np.uint8(keep)
     grid = rng.permutation(M * N)[:K].astype(np.int32)
     sigma = (1.0 / (1.0 + np.arange(rank, dtype=np.float64))).astype(np.float32)
-    return Proj(d_in, d_out, rank, group, grid, U, sigma, V, codes, scales, zeros)
+    if bits != 3:
+        return Proj(d_in, d_out, rank, group, grid, U, sigma, V, codes, scales, zeros)
+    # 3-bit: a high-bit plane and zero points 0..7, two per byte (drawn after the
+    # 2-bit arrays, so the other draws of the layer are unchanged)
+    codes_hi = rng.integers(0, 2**32, size=(K, d_out, d_in // 32), dtype=np.uint32)
+    z3 = rng.integers(0, 8, size=(K, d_out, G), dtype=np.uint8)
+    if G % 2:
+        z3 = np.concatenate([z3, np.zeros((K, d_out, 1), np.uint8)], axis=-1)
+    zeros3 = (z3[..., 0::2] | (z3[..., 1::2] << 4)).astype(np.uint8)
+    return Proj(d_in, d_out, rank, group, grid, U, sigma, V, codes, scales, zeros3, 3, codes_hi)
 
 
 def make_layer(cfg: Config | int, seed: int = 0, rank: Optional[int] = None) -> Layer:
@@ -184,7 +196,7 @@ def make_layer(cfg: Config | int, seed: int = 0, rank: Optional[int] = None) -> 
         cfg = CONFIGS[cfg]
     r = cfg.rank if rank is None else rank
     rng = np.random.default_rng([seed, 1])
-    projs = [_make_proj(rng, cfg.K, cfg.M, cfg.N, di, do, r, cfg.group)
+    projs = [_make_proj(rng, cfg.K, cfg.M, cfg.N, di, do, r, cfg.group, cfg.bits)
              for (di, do) in proj_shapes(cfg.kind, cfg.d_model, cfg.d_ff)]
     shared = None
     if cfg.shared_d_ff:
@@ -236,10 +248,10 @@ def per_expert_lowrank(layer: Layer, p: Proj):
 
 
 def tiny_config(kind=SWIGLU, K=4, M=2, N=2, d_model=64, d_ff=128, rank=8, group=32, top_k=2,
-                shared_d_ff=0, zipf_s=0.0, logit_std=1.0) -> Config:
+                shared_d_ff=0, zipf_s=0.0, logit_std=1.0, bits=2) -> Config:
     """A small configuration for tests (oracle runs it in milliseconds)."""
     return Config(f"tiny-{kind}-{K}e", kind, K, M, N, d_model, d_ff, rank, group, top_k, (16,),
-                  logit_std=logit_std, zipf_s=zipf_s, shared_d_ff=shared_d_ff)
+                  logit_std=logit_std, zipf_s=zipf_s, shared_d_ff=shared_d_ff, bits=bits)
 
 
 def planted_factors(K: int, M: int, N: int, d_u: int, d_v: int, r0: int, noise: float = 0.05,

@@ -398,3 +398,39 @@ def test_route_full_softmax_variant():
     i, w = oracle.route(np.log(np.array([[1.0, 2.0, 3.0]], dtype=np.float32)), 2, full_softmax=True)
     assert list(i[0]) == [2, 1]
     np.testing.assert_allclose(w[0], [0.5, 1.0 / 3.0], rtol=1e-6)
+
+
+def test_dequant_3bit_hand_case():
+    """3-bit residual, hand-packed: q_j = j % 8 for j < 32, group 16, zeros (5, 2),
+    scales (0.5, 0.25).  Low 2 bits (0, 1, 2, 3, ...) at bits 2*(j%16): 0xE4 per
+    byte; high bits (q >= 4 for j % 8 in 4..7) at bit j: 0xF0 per byte; zeros
+    5 | 2 << 4 = 0x25."""
+    import dataclasses
+    p = synth.Proj(32, 1, 0, 16, np.zeros(1, np.int32), np.zeros((1, 0), np.uint16),
+                   np.zeros(0, np.float32), np.zeros((1, 0), np.uint16),
+                   np.array([[[0xE4E4E4E4, 0xE4E4E4E4]]], np.uint32),
+                   np.array([[[0.5, 0.25]]], np.float16), np.array([[[0x25]]], np.uint8),
+                   3, np.array([[[0xF0F0F0F0]]], np.uint32))
+    j = np.arange(32)
+    want = np.where(j < 16, 0.5 * (j % 8 - 5), 0.25 * (j % 8 - 2))
+    assert np.array_equal(oracle.dequant(p, 0)[0], want)
+    assert list(oracle.unpack_zeros(np.array([0x25, 0x07], np.uint8), 3, bits=3)) == [5, 2, 7]
+    # a zero high plane with the same zero points is the 2-bit residual
+    two = dataclasses.replace(p, bits=2, codes_hi=None, zeros=np.array([[[0x09]]], np.uint8))  # 1 | 2 << 2
+    three = dataclasses.replace(p, codes_hi=np.zeros((1, 1, 1), np.uint32), zeros=np.array([[[0x21]]], np.uint8))
+    assert np.array_equal(oracle.dequant(two, 0), oracle.dequant(three, 0))
+
+
+def test_dequant_3bit_range():
+    cfg = synth.tiny_config(K=3, M=2, N=2, d_model=128, d_ff=64, rank=0, group=64, bits=3)
+    layer = synth.make_layer(cfg, seed=5)
+    for p in layer.projs:
+        assert p.bits == 3 and p.codes_hi.shape == (3, p.d_out, p.d_in // 32)
+        G = p.d_in // p.group
+        z = oracle.unpack_zeros(p.zeros, G, 3)
+        assert z.max() <= 7 and z.shape[-1] == G
+        s = oracle.widen_fp16(p.scales)
+        for e in range(3):
+            w = oracle.dequant(p, e)
+            ratio = np.abs(w).reshape(p.d_out, G, p.group) / s[e][:, :, None]
+            assert ratio.max() <= 7.0 and ratio.max() >= 6.0   # q and z span 0..7
