@@ -73,11 +73,18 @@ enum { TILEQ_LINEAR = 0, TILEQ_SWIGLU = 1 };
  *   scales       device fp16 [K, d_out, d_in/group]
  *   zeros        device uint8 [K, d_out, ceil(d_in/group/4)]; group j at bits 2*(j%4)
  *                of byte j/4
+ *   bits         2 (or 0: a zero-initialised struct) or 3.  The summary evaluates
+ *                2-bit and 3-bit residuals.  For 3: q = codes + 4 * (bit of codes_hi),
+ *                zeros are device uint8 [K, d_out, ceil(d_in/group/2)] with group j
+ *                at bits 4*(j%2) of byte j/2 (values 0..7), and
+ *   codes_hi     device uint32 [K, d_out, d_in/32], element j at bit j%32 (3-bit only).
+ *                3-bit projections run the residual on warp-level MMA at every
+ *                batch size (the tcgen05 residual kernel reads 2-bit codes only).
  *   Residual: w[o,i] = scales[o,i/group] * (q[o,i] - z[o,i/group]).
  * Supported: d_out % 16 == 0, d_in % 128 == 0, group == 64 or a multiple of 128,
  * d_in % group == 0,
- * 0 <= rank <= 256 and rank % 16 == 0 (rank 0 = residual only); otherwise
- * TILEQ_ERR_UNSUPPORTED. */
+ * 0 <= rank <= 256 and rank % 16 == 0 (rank 0 = residual only), bits in {0, 2, 3};
+ * otherwise TILEQ_ERR_UNSUPPORTED. */
 typedef struct {
   int d_in, d_out, rank, group;
   const int32_t *grid_assign;
@@ -87,6 +94,8 @@ typedef struct {
   const uint32_t *codes;
   const void *scales;
   const uint8_t *zeros;
+  int bits;
+  const uint32_t *codes_hi;
 } tileq_proj;
 
 /* A TileQ MoE layer.

@@ -54,12 +54,19 @@ def zero_residual(layer: synth.Layer, lr_gain: float = 1.0) -> synth.Layer:
     for p in layer.projs:
         G = p.d_in // p.group
         zb = p.zeros
-        z = np.stack([(zb[..., j // 4] >> (2 * (j % 4))) & 3 for j in range(G)], axis=-1)
+        if p.bits == 3:   # zero points 0..7, two per byte; q = low 2 bits + 4 * high bit
+            z = np.stack([(zb[..., j // 2] >> (4 * (j % 2))) & 7 for j in range(G)], axis=-1)
+        else:
+            z = np.stack([(zb[..., j // 4] >> (2 * (j % 4))) & 3 for j in range(G)], axis=-1)
         words_per_group = p.group // 16
-        zw = np.repeat(z.astype(np.uint32), words_per_group, axis=-1) * np.uint32(0x55555555)
+        zw = np.repeat((z & 3).astype(np.uint32), words_per_group, axis=-1) * np.uint32(0x55555555)
+        extra = {}
+        if p.bits == 3:
+            hw = np.repeat((z >> 2).astype(np.uint32), p.group // 32, axis=-1) * np.uint32(0xFFFFFFFF)
+            extra["codes_hi"] = np.ascontiguousarray(hw)
         U = p.U
         if lr_gain != 1.0 and p.rank > 0:
             U = synth.to_bf16_bits(synth.bf16_bits_to_f32(p.U) * np.float32(lr_gain))
-        projs.append(synth.Proj(**{**p.__dict__, "codes": np.ascontiguousarray(zw), "U": U}))
+        projs.append(synth.Proj(**{**p.__dict__, "codes": np.ascontiguousarray(zw), "U": U, **extra}))
     return synth.Layer(layer.kind, layer.K, layer.M, layer.N, layer.d_model, layer.d_ff,
-                       layer.top_k, projs, layer.shared)
+                       layer.top_k, projs, layer.shared, layer.route_mode)

@@ -48,8 +48,9 @@ def test_library_exports_every_declared_symbol(L):
 def test_struct_layout_matches_c(L, tmp_path):
     src = tmp_path / "layout.c"
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "tileq.h"\n'
-                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n",'
+                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n",'
                    'sizeof(tileq_proj), offsetof(tileq_proj, grid_assign), offsetof(tileq_proj, zeros),'
+                   'offsetof(tileq_proj, bits), offsetof(tileq_proj, codes_hi),'
                    'sizeof(tileq_layer), offsetof(tileq_layer, proj), offsetof(tileq_layer, shared_d_ff),'
                    'offsetof(tileq_layer, shared_w), offsetof(tileq_layer, route_mode), sizeof(tileq_route_out), sizeof(tileq_per_expert_lr));'
                    'return 0;}\n')
@@ -57,6 +58,7 @@ def test_struct_layout_matches_c(L, tmp_path):
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
     want = [ctypes.sizeof(L.tileq_proj), L.tileq_proj.grid_assign.offset, L.tileq_proj.zeros.offset,
+            L.tileq_proj.bits.offset, L.tileq_proj.codes_hi.offset,
             ctypes.sizeof(L.tileq_layer), L.tileq_layer.proj.offset, L.tileq_layer.shared_d_ff.offset,
             L.tileq_layer.shared_w.offset, L.tileq_layer.route_mode.offset, ctypes.sizeof(L.tileq_route_out),
             ctypes.sizeof(L.tileq_per_expert_lr)]
@@ -270,3 +272,29 @@ def test_place_workspace_and_validation(L):
     out = L.tileq_place_out(16, None, None)
     st = L.lib().tileq_place_experts(ctypes.byref(_place(L, 4, 2, 2)), ctypes.byref(out), 16, 8, None)
     assert st == L.TILEQ_ERR_WORKSPACE
+
+
+def test_3bit_validation_and_packed_size(L):
+    """3-bit projections: bits in {0, 2, 3}; the packed copy drops the tcgen05
+    row layout (2 bits/weight) and adds the high-bit plane (1 bit/weight)."""
+    c2, layer = _host_layer(L, 0)
+    n2 = L.tileq_packed_size(c2)
+    cfg3 = synth.Config(**{**synth.CONFIGS[0].__dict__, "bits": 3})
+    c3, _ = _host_layer(L, cfg3)
+    for i in range(1):
+        c3.proj[i].bits = 3
+    n3 = L.tileq_packed_size(c3)
+    p = layer.projs[0]
+    assert n3 - n2 == -layer.K * p.d_out * p.d_in // 4 + layer.K * p.d_out * p.d_in // 8
+    c3.proj[0].bits = 4
+    with pytest.raises(L.TileQError) as e:
+        L.tileq_packed_size(c3)
+    assert e.value.status == L.TILEQ_ERR_UNSUPPORTED
+    # gate and up share one residual kernel: their bits must agree
+    cs, _ = _host_layer(L, synth.tiny_config(K=4, M=2, N=2, d_model=128, d_ff=128, rank=16, group=64))
+    cs.proj[0].bits = 3
+    with pytest.raises(L.TileQError) as e:
+        L.tileq_packed_size(cs)
+    assert e.value.status == L.TILEQ_ERR_UNSUPPORTED
+    cs.proj[1].bits = 3
+    assert L.tileq_packed_size(cs) > 0

@@ -165,6 +165,47 @@ def test_full_softmax_routing(torch_cuda, case):
     assert np.abs(out - ref).max() < 0.25 * np.abs(out - default).max()
 
 
+# 3-bit residuals (q = codes + 4 * high bit; zeros 0..7).  They run the warp-MMA
+# residual kernel at every batch size: 300 tokens over 8 experts would take
+# tcgen05 tiles with 2-bit codes.
+TINY3 = [
+    (synth.SWIGLU, 8, 2, 4, 256, 512, 32, 128, 2, 0, 16),
+    (synth.SWIGLU, 8, 2, 4, 256, 512, 32, 128, 2, 256, 300),
+    (synth.LINEAR, 5, 2, 3, 384, 144, 16, 64, 3, 0, 200),
+    (synth.SWIGLU, 16, 4, 4, 128, 128, 16, 64, 4, 0, 1500),
+]
+
+
+@pytest.mark.parametrize("case", TINY3, ids=[f"q3_{i}" for i in range(len(TINY3))])
+def test_tiny_layers_3bit(torch_cuda, case):
+    kind, K, M, N, dm, dff, r, g, k, sh, T = case
+    cfg = synth.tiny_config(kind=kind, K=K, M=M, N=N, d_model=dm, d_ff=dff, rank=r, group=g,
+                            top_k=k, shared_d_ff=sh, bits=3)
+    layer = synth.make_layer(cfg, seed=T + 7)
+    assert all(p.bits == 3 for p in layer.projs)
+    logits, x = synth.make_inputs(cfg, T, seed=T + 7)
+    out, route, _ = run_gpu(torch_cuda, layer, logits, x)
+    check_route(route, logits, k, K)
+    assert_parity(out, oracle.forward(layer, x, logits), f"3-bit {case}")
+    zr = zero_residual(layer)
+    out, _, _ = run_gpu(torch_cuda, zr, logits, x)
+    assert_parity(out, oracle.forward(zr, x, logits), f"3-bit {case} zero residual")
+    r0 = synth.make_layer(cfg, seed=T + 7, rank=0)
+    out, _, _ = run_gpu(torch_cuda, r0, logits, x)
+    assert_parity(out, oracle.forward(r0, x, logits), f"3-bit {case} rank 0")
+
+
+def test_unfused_path_3bit(torch_cuda):
+    kind, K, M, N, dm, dff, r, g, k, sh, T = TINY3[1]
+    cfg = synth.tiny_config(kind=kind, K=K, M=M, N=N, d_model=dm, d_ff=dff, rank=r, group=g,
+                            top_k=k, shared_d_ff=sh, bits=3)
+    layer = synth.make_layer(cfg, seed=5)
+    logits, x = synth.make_inputs(cfg, T, seed=5)
+    pe = [synth.per_expert_lowrank(layer, p) for p in layer.projs]
+    out_u, _, _ = run_gpu(torch_cuda, layer, logits, x, unfused=True, per_expert=pe)
+    assert_parity(out_u, oracle.forward(layer, x, logits), "unfused 3-bit")
+
+
 @pytest.mark.parametrize("case", [TINY[0], TINY[3], TINY[2]], ids=["swiglu", "linear", "shared"])
 def test_unfused_path(torch_cuda, case):
     kind, K, M, N, dm, dff, r, g, k, sh, T = case

@@ -51,6 +51,7 @@ class tileq_proj(ctypes.Structure):
         ("grid_assign", ctypes.POINTER(ctypes.c_int32)),
         ("U", ctypes.c_void_p), ("Sigma", ctypes.c_void_p), ("V", ctypes.c_void_p),
         ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p),
+        ("bits", ctypes.c_int), ("codes_hi", ctypes.c_void_p),
     ]
 
 

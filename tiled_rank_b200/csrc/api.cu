@@ -40,6 +40,7 @@ constexpr int kWideMinK = 4096;    // 256-item tcgen05 tiles from this K (32 sta
 
 struct ProjInfo {
   int d_in, d_out, rank, group, G;
+  int bits;   // 2 or 3
   int8_t m_of[kMaxExperts], n_of[kMaxExperts];
 };
 
@@ -62,6 +63,7 @@ tileq_status validate_layer(const tileq_layer *L, LayerInfo *li, bool need_devic
     const tileq_proj &p = L->proj[pi];
     ProjInfo &q = li->p[pi];
     if (p.d_in <= 0 || p.d_out <= 0 || p.rank < 0 || p.group <= 0) return TILEQ_ERR_INVALID_ARG;
+    if (p.bits != 0 && p.bits != 2 && p.bits != 3) return TILEQ_ERR_UNSUPPORTED;
     if (p.d_out % 16 || p.d_in % 128 || (p.group != 64 && p.group % 128) || p.d_in % p.group ||
         p.rank % 16 ||
         p.rank > 256)
@@ -69,6 +71,7 @@ tileq_status validate_layer(const tileq_layer *L, LayerInfo *li, bool need_devic
     if (!p.grid_assign) return TILEQ_ERR_INVALID_ARG;
     if (need_device_ptrs) {
       if (!p.codes || !p.scales || !p.zeros) return TILEQ_ERR_INVALID_ARG;
+      if (p.bits == 3 && !p.codes_hi) return TILEQ_ERR_INVALID_ARG;
       if (p.rank > 0 && (!p.U || !p.V || !p.Sigma)) return TILEQ_ERR_INVALID_ARG;
     }
     std::vector<char> seen((size_t)L->M * L->N, 0);
@@ -84,6 +87,7 @@ tileq_status validate_layer(const tileq_layer *L, LayerInfo *li, bool need_devic
     q.rank = p.rank;
     q.group = p.group;
     q.G = p.d_in / p.group;
+    q.bits = p.bits == 3 ? 3 : 2;
   }
   if (L->kind == TILEQ_SWIGLU) {
     const ProjInfo &g = li->p[0], &u = li->p[1], &d = li->p[2];
@@ -91,6 +95,7 @@ tileq_status validate_layer(const tileq_layer *L, LayerInfo *li, bool need_devic
         d.d_in != L->d_ff || d.d_out != L->d_model)
       return TILEQ_ERR_INVALID_ARG;
     if (g.rank != u.rank) return TILEQ_ERR_UNSUPPORTED;
+    if (g.bits != u.bits) return TILEQ_ERR_UNSUPPORTED;   // gate and up share one residual kernel
     if (L->shared_d_ff < 0) return TILEQ_ERR_INVALID_ARG;
     if (L->shared_d_ff > 0) {
       if (L->shared_d_ff % 128) return TILEQ_ERR_UNSUPPORTED;
@@ -118,7 +123,7 @@ size_t frag_bytes(int nblk, int R, int C, int kb) {
 // weights row-major fp16 [pad128(rows)][cols] (the A operands of the tcgen05
 // kernel; vf / sh hold the same values in warp-MMA fragment order).
 struct PackedLayout {
-  size_t qw[3], qf[3], sz[3], uf[3], vf[3], sig[3], vr[3], sh[3], shr[3], total;
+  size_t qw[3], qf[3], qfh[3], sz[3], uf[3], vf[3], sig[3], vr[3], sh[3], shr[3], total;
 };
 
 PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
@@ -126,10 +131,12 @@ PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
   size_t off = 0;
   for (int p = 0; p < li.nproj; ++p) {
     const ProjInfo &q = li.p[p];
-    pl.qw[p] = off;
-    off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 4);
+    pl.qw[p] = off;   // tcgen05 row layout (2-bit only: 3-bit runs on warp MMA)
+    if (q.bits == 2) off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 4);
     pl.qf[p] = off;
     off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 4);
+    pl.qfh[p] = off;  // 3-bit high-bit plane, fragment layout
+    if (q.bits == 3) off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 8);
     pl.sz[p] = off;
     off += align_up((size_t)L->K * pad128(q.d_out) * q.G * 4);
     pl.uf[p] = off;
@@ -230,8 +237,11 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   // MMA than on tcgen05 (measured: an M=128 N=16 tcgen05.mma does fewer MACs per
   // cycle than mma.sync, and the decode then dominates); wider ones on tcgen05.
   const long long avg = P / std::max(1, L->K);
-  const bool use_tc = avg > 32;
-  pl.bn_main = use_tc ? choose_bn_tc(avg) : choose_bn(avg);
+  bool any3 = false;   // the tcgen05 residual kernel reads 2-bit codes only
+  for (int p = 0; p < li.nproj; ++p) any3 = any3 || li.p[p].bits == 3;
+  const bool use_tc = avg > 32 && !any3;
+  // warp-MMA tiles hold at most 32 items (3-bit layers keep them at any batch)
+  pl.bn_main = use_tc ? choose_bn_tc(avg) : std::min(choose_bn(avg), 32);
   pl.slots_main = cdiv(P, pl.bn_main) + L->K;
   const long long est_main = std::min(L->K, P) + P / pl.bn_main;
   auto tc_plan = [&](int d_out, int d_in, int np) {
@@ -647,6 +657,7 @@ tileq_status run_residual(const Residual &r, const GemmPlan &g, const LayerInfo 
   for (int i = 0; i < r.np; ++i) {
     // tcgen05 reads the row layout of the codes, warp MMA the fragment layout
     a.codes[i] = at<uint4>(packed, g.tc ? pl.qw[r.proj[i]] : pl.qf[r.proj[i]]);
+    a.codes_hi[i] = li.p[r.proj[i]].bits == 3 ? at<uint2>(packed, pl.qfh[r.proj[i]]) : nullptr;
     a.sz[i] = at<uint32_t>(packed, pl.sz[r.proj[i]]);
     if (r.ext) tc_ext(&a, i, li, pl, packed, r.proj[i], r.ext_col[i]);
   }
@@ -951,18 +962,25 @@ tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_by
     const ProjInfo &q = li.p[p];
     {
       const long long n = (long long)K * (pad128(q.d_out) / 128) * (q.d_in / 128) * 128 * 8;
-      pack_codes_tc_kernel<<<nblocks(n, 256), 256, 0, stream>>>(src.codes, at<uint32_t>(packed, pl.qw[p]),
-                                                                 K, q.d_out, q.d_in);
-      TQ_LAUNCHED();
+      if (q.bits == 2) {
+        pack_codes_tc_kernel<<<nblocks(n, 256), 256, 0, stream>>>(src.codes, at<uint32_t>(packed, pl.qw[p]),
+                                                                   K, q.d_out, q.d_in);
+        TQ_LAUNCHED();
+      }
       pack_codes_kernel<<<nblocks(n / 4, 256), 256, 0, stream>>>(src.codes, at<uint4>(packed, pl.qf[p]),
                                                                  K, q.d_out, q.d_in);
       TQ_LAUNCHED();
+      if (q.bits == 3) {
+        pack_codes_hi_kernel<<<nblocks(n / 4, 256), 256, 0, stream>>>(src.codes_hi, at<uint2>(packed, pl.qfh[p]),
+                                                                      K, q.d_out, q.d_in);
+        TQ_LAUNCHED();
+      }
     }
     {
       const long long n = (long long)K * pad128(q.d_out) * q.G;
       pack_sz_kernel<<<nblocks(n, 256), 256, 0, stream>>>(static_cast<const __half *>(src.scales),
                                                            src.zeros, at<uint32_t>(packed, pl.sz[p]),
-                                                           K, q.d_out, q.G);
+                                                           K, q.d_out, q.G, q.bits);
       TQ_LAUNCHED();
     }
     if (q.rank > 0) {

@@ -126,6 +126,23 @@ __device__ __forceinline__ void dequant_qz_k16(uint32_t w, const __half2 (&nz)[4
   a[3] = h2_as_u32(__hfma2(v3, u32_as_h2(0x24002400u), nz[3]));
 }
 
+// 3-bit codes: as dequant_qz_k16, with the high bit of register i's codes at
+// bits 2i+2 and 18+2i of `h` (just above the 2-bit field, which is masked to
+// zero there): one more AND-OR places it, and the fp16 value becomes
+// 1024 + 4^i*(q_lo + 4*q_hi) = 1024 + 4^i*q, still exact (q <= 7).
+__device__ __forceinline__ void dequant_qz3_k16(uint32_t w, uint32_t h, const __half2 (&nz)[4],
+                                                uint32_t (&a)[4]) {
+  const uint32_t kMagic = 0x64006400u;
+  const __half2 v0 = u32_as_h2(and_or(w, 0x00030003u, and_or(h, 0x00040004u, kMagic)));
+  const __half2 v1 = u32_as_h2(and_or(w, 0x000C000Cu, and_or(h, 0x00100010u, kMagic)));
+  const __half2 v2 = u32_as_h2(and_or(w, 0x00300030u, and_or(h, 0x00400040u, kMagic)));
+  const __half2 v3 = u32_as_h2(and_or(w, 0x00C000C0u, and_or(h, 0x01000100u, kMagic)));
+  a[0] = h2_as_u32(__hfma2(v0, u32_as_h2(0x3C003C00u), nz[0]));
+  a[1] = h2_as_u32(__hfma2(v1, u32_as_h2(0x34003400u), nz[1]));
+  a[2] = h2_as_u32(__hfma2(v2, u32_as_h2(0x2C002C00u), nz[2]));
+  a[3] = h2_as_u32(__hfma2(v3, u32_as_h2(0x24002400u), nz[3]));
+}
+
 // D = A * B (C = 0), fp16 inputs, fp32 result.
 __device__ __forceinline__ void mma_f16_16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                                 uint32_t b1) {

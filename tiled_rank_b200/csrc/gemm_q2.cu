@@ -61,7 +61,7 @@ constexpr int QW = 8;                    // consumer warps (16 rows each)
 constexpr int QTHREADS = (QW + 1) * 32;  // + one producer warp
 constexpr int QBLK = 128;                // K of one packed code block; a main stage covers two
 
-template <int NP, int BN>
+template <int NP, int BN, bool Q3>
 struct QCfg {
   static constexpr int NT = BN / 8;
   static constexpr int MINB = NP * NT <= 2 ? 3 : (NP * NT <= 4 ? 2 : 1);  // resident CTAs per SM
@@ -71,7 +71,8 @@ struct QCfg {
   static constexpr int B_BYTES = 4 * BOX;
   static constexpr int A_BYTES = NP * 2 * 4096;  // codes: two 128x128 blocks per projection
   static constexpr int SZ_BYTES = NP * 2 * 1024;  // (scale, zero): per block up to two 64-wide groups
-  static constexpr int STAGE = B_BYTES + A_BYTES + SZ_BYTES;
+  static constexpr int H_BYTES = Q3 ? NP * 2 * 2048 : 0;  // 3-bit codes: the high-bit plane
+  static constexpr int STAGE = B_BYTES + A_BYTES + SZ_BYTES + H_BYTES;
   static constexpr int S_RAW = (BUDGET - 1024 - 64) / STAGE;
   static constexpr int S = S_RAW > 8 ? 8 : S_RAW;  // ring stages
   static constexpr int BAR_OFF = S * STAGE;
@@ -103,10 +104,10 @@ __device__ __forceinline__ void q2_store(const TcArgs &a, int item, int o, float
   }
 }
 
-template <int NP, int BN>
-__global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(const __grid_constant__ TcArgs a) {
+template <int NP, int BN, bool Q3>
+__global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN, Q3>::MINB) gemm_q2_kernel(const __grid_constant__ TcArgs a) {
   pdl_wait_and_release();
-  using C = QCfg<NP, BN>;
+  using C = QCfg<NP, BN, Q3>;
   constexpr int SLOT = NP * BN * kRowsPerCta;  // floats of one fp32 partial
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -153,6 +154,9 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
   auto st_z = [&](int s, int p, int h) {
     return smem + s * C::STAGE + C::B_BYTES + C::A_BYTES + (p * 2 + h) * 1024;
   };
+  auto st_h = [&](int s, int p, int h) {
+    return smem + s * C::STAGE + C::B_BYTES + C::A_BYTES + C::SZ_BYTES + (p * 2 + h) * 2048;
+  };
 
   if (warp == QW) {
     // ------------------------------------------------------------ producer
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
         const int nh = kb + 1 < nkb ? 2 : 1;  // blocks in this stage
         const uint32_t zb = g64 ? 1024 : 512;   // (scale, zero) bytes of one block
         if (lane == 0)
-          mbar_arrive_expect_tx(&full[s], (uint32_t)(nh * 2 * C::BOX + NP * nh * (4096 + zb)));
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(nh * 2 * C::BOX + NP * nh * (4096 + zb + (Q3 ? 2048 : 0))));
         __syncwarp();
         if (lane < 2 * nh) {
           tc::tma_load_2d(bs + lane * C::BOX, &a.bmap, kb * QBLK + lane * 64, item0, &full[s]);
@@ -187,6 +191,11 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
             const int gi = g64 ? 2 * (kb + h) : ((kb + h) * QBLK) / a.group;
             bulk_g2s(st_z(s, p, h), a.sz[p] + (((size_t)grp * n128 + ob) * G + gi) * 128, zb, &full[s]);
           }
+        } else if (Q3 && lane >= 24 && lane < 24 + NP) {
+          const int p = lane - 24;
+          const size_t blk = ((size_t)grp * n128 + ob) * nkb + kb;
+          bulk_g2s(st_h(s, p, 0), reinterpret_cast<const uint8_t *>(a.codes_hi[p]) + blk * 2048,
+                   (uint32_t)(nh * 2048), &full[s]);
         }
       } else {
         // low-rank extension: 128 K-extension columns of each projection
@@ -259,6 +268,7 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
   auto block_main = [&](int s, int h) {
     const uint32_t bs = smem_addr(st_b(s));
     uint32_t cw[NP][4];
+    uint32_t hw[NP][2];   // 3-bit: high-bit words (each covers two of cw)
     float part[NP][C::NT][4];
     __half2 nz[NP][4];
     float sc0[NP], sc8[NP];
@@ -268,6 +278,10 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
       asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
                    : "=r"(cw[p][0]), "=r"(cw[p][1]), "=r"(cw[p][2]), "=r"(cw[p][3])
                    : "r"(sa));
+      if constexpr (Q3) {
+        const uint32_t sh = smem_addr(st_h(s, p, h)) + (warp * 32 + lane) * 8;
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(hw[p][0]), "=r"(hw[p][1]) : "r"(sh));
+      }
     }
     auto group_consts = [&](int p, int sub) {
       const uint32_t zs = smem_addr(st_z(s, p, h)) + rw * 4;
@@ -307,7 +321,15 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
       for (int p = 0; p < NP; ++p) {
         const uint32_t word = cw[p][ks >> 1];
         uint32_t af[4];
-        dequant_qz_k16((ks & 1) ? (word >> 8) : word, nz[p], af);
+        if constexpr (Q3) {
+          // high bits of word ks/2: half (ks/2)&1 of hw, rotated into place; k16 step ks&1 one bit up
+          uint32_t hword = hw[p][ks >> 2];
+          if ((ks >> 1) & 1) hword = __funnelshift_r(hword, hword, 8);
+          if (ks & 1) hword >>= 1;
+          dequant_qz3_k16((ks & 1) ? (word >> 8) : word, hword, nz[p], af);
+        } else {
+          dequant_qz_k16((ks & 1) ? (word >> 8) : word, nz[p], af);
+        }
         if (gstart) {
 #pragma unroll
           for (int j = 0; j < C::NT; ++j)
@@ -461,10 +483,10 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN>::MINB) gemm_q2_kernel(c
   Q2_CTA_TIME(1);
 }
 
-template <int NP, int BN>
+template <int NP, int BN, bool Q3>
 cudaError_t launch_q2(const TcArgs &a, int n_tile_slots, cudaStream_t stream) {
-  using C = QCfg<NP, BN>;
-  auto kern = gemm_q2_kernel<NP, BN>;
+  using C = QCfg<NP, BN, Q3>;
+  auto kern = gemm_q2_kernel<NP, BN, Q3>;
   static bool configured = false;  // one attribute call per instantiation and process
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -483,13 +505,24 @@ cudaError_t launch_q2(const TcArgs &a, int n_tile_slots, cudaStream_t stream) {
 cudaError_t launch_gemm_q2(const TcArgs &a, int np, int bn, int n_tile_slots, cudaStream_t stream) {
   if (n_tile_slots <= 0) return cudaSuccess;
   if (a.m_tiles <= 0 || a.ksplit <= 0 || (a.group != 64 && a.group % 128 != 0)) return cudaErrorInvalidValue;
+  if (a.codes_hi[0] != nullptr) {   // 3-bit codes
+    switch (bn * 4 + np) {
+      case 8 * 4 + 1: return launch_q2<1, 8, true>(a, n_tile_slots, stream);
+      case 16 * 4 + 1: return launch_q2<1, 16, true>(a, n_tile_slots, stream);
+      case 32 * 4 + 1: return launch_q2<1, 32, true>(a, n_tile_slots, stream);
+      case 8 * 4 + 2: return launch_q2<2, 8, true>(a, n_tile_slots, stream);
+      case 16 * 4 + 2: return launch_q2<2, 16, true>(a, n_tile_slots, stream);
+      case 32 * 4 + 2: return launch_q2<2, 32, true>(a, n_tile_slots, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (bn * 4 + np) {
-    case 8 * 4 + 1: return launch_q2<1, 8>(a, n_tile_slots, stream);
-    case 16 * 4 + 1: return launch_q2<1, 16>(a, n_tile_slots, stream);
-    case 32 * 4 + 1: return launch_q2<1, 32>(a, n_tile_slots, stream);
-    case 8 * 4 + 2: return launch_q2<2, 8>(a, n_tile_slots, stream);
-    case 16 * 4 + 2: return launch_q2<2, 16>(a, n_tile_slots, stream);
-    case 32 * 4 + 2: return launch_q2<2, 32>(a, n_tile_slots, stream);
+    case 8 * 4 + 1: return launch_q2<1, 8, false>(a, n_tile_slots, stream);
+    case 16 * 4 + 1: return launch_q2<1, 16, false>(a, n_tile_slots, stream);
+    case 32 * 4 + 1: return launch_q2<1, 32, false>(a, n_tile_slots, stream);
+    case 8 * 4 + 2: return launch_q2<2, 8, false>(a, n_tile_slots, stream);
+    case 16 * 4 + 2: return launch_q2<2, 16, false>(a, n_tile_slots, stream);
+    case 32 * 4 + 2: return launch_q2<2, 32, false>(a, n_tile_slots, stream);
     default: return cudaErrorInvalidValue;
   }
 }

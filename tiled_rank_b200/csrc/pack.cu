@@ -47,11 +47,55 @@ __global__ void pack_codes_kernel(const uint32_t *codes, uint4 *out, int K, int 
   out[gid] = make_uint4(words[0], words[1], words[2], words[3]);
 }
 
-// scales fp16 [K][d_out][G], zeros [K][d_out][ceil(G/4)] ->
+// 3-bit codes' high bits [K][d_out][d_in/32] (element j at bit j%32) ->
+// [K][R/128][d_in/128][8 warps][32 lanes] uint2, beside pack_codes_kernel's
+// layout: word p of a lane holds the high bits of its code words 2p and 2p+1.
+// For code word 2p, k16 step s and fragment register i, the (lo, hi) codes'
+// bits sit at (2 + 2i + s, 18 + 2i + s): after the decoder's shift by s, bit
+// 2i+2 lies just above the 2-bit field of register i.  Code word 2p+1 uses the
+// same positions rotated left by 8 (the 32 positions are all distinct).
+__global__ void pack_codes_hi_kernel(const uint32_t *hi, uint2 *out, int K, int d_out, int d_in) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nkb = d_in / 128, n128 = pad128(d_out) / 128, wpr = d_in / 32;
+  const long long total = (long long)K * n128 * nkb * 8 * 32;
+  if (gid >= total) return;
+  const int lane = (int)(gid % 32);
+  long long rest = gid / 32;
+  const int w8 = (int)(rest % 8);
+  rest /= 8;
+  const int kb = (int)(rest % nkb);
+  rest /= nkb;
+  const int ob = (int)(rest % n128);
+  const int e = (int)(rest / n128);
+  const int r0 = lane >> 2, c = (lane & 3) * 2;
+  auto bit = [&](int row, int col) -> uint32_t {
+    if (row >= d_out) return 0u;
+    return (hi[((size_t)e * d_out + row) * wpr + col / 32] >> (col % 32)) & 1u;
+  };
+  uint32_t words[2] = {0u, 0u};
+  for (int w = 0; w < 4; ++w) {
+    uint32_t acc = 0;
+    for (int s = 0; s < 2; ++s) {
+      const int ks = kb * 128 + w * 32 + s * 16;
+      for (int i = 0; i < 4; ++i) {
+        const int row = ob * 128 + w8 * 16 + r0 + 8 * (i & 1);
+        const int col = ks + c + 8 * (i >> 1);
+        acc |= bit(row, col) << (2 + 2 * i + s);
+        acc |= bit(row, col + 1) << (18 + 2 * i + s);
+      }
+    }
+    if (w & 1) acc = (acc << 8) | (acc >> 24);
+    words[w >> 1] |= acc;
+  }
+  out[gid] = make_uint2(words[0], words[1]);
+}
+
+// scales fp16 [K][d_out][G], zeros [K][d_out][ceil(G/4)] (2-bit; 3-bit:
+// [K][d_out][ceil(G/2)], 4-bit fields) ->
 // [K][R/128][G][8 warps][16 rows] u32 = {low half: scale bits, high half: fp16(z)};
 // rows past d_out hold scale 0.
 __global__ void pack_sz_kernel(const __half *scales, const uint8_t *zeros, uint32_t *out, int K,
-                               int d_out, int G) {
+                               int d_out, int G, int bits) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int n128 = pad128(d_out) / 128;
   const long long total = (long long)K * n128 * G * 128;
@@ -69,9 +113,15 @@ __global__ void pack_sz_kernel(const __half *scales, const uint8_t *zeros, uint3
     out[gid] = 0u;
     return;
   }
-  const int zb = (G + 3) / 4;
   const __half s = scales[((size_t)e * d_out + row) * G + grp];
-  const uint32_t z = (zeros[((size_t)e * d_out + row) * zb + grp / 4] >> (2 * (grp % 4))) & 3u;
+  uint32_t z;
+  if (bits == 3) {
+    const int zb = (G + 1) / 2;
+    z = (zeros[((size_t)e * d_out + row) * zb + grp / 2] >> (4 * (grp % 2))) & 7u;
+  } else {
+    const int zb = (G + 3) / 4;
+    z = (zeros[((size_t)e * d_out + row) * zb + grp / 4] >> (2 * (grp % 4))) & 3u;
+  }
   const __half zh = __uint2half_rn(z);
   const uint32_t lo = *reinterpret_cast<const uint16_t *>(&s);
   const uint32_t hi = *reinterpret_cast<const uint16_t *>(&zh);

@@ -53,6 +53,9 @@ class DeviceLayer:
                 "scales": _dev(p.scales, self.device),
                 "zeros": _dev(p.zeros, self.device),
             }
+            bits = int(getattr(p, "bits", 2))
+            if bits == 3:
+                tens["codes_hi"] = _dev(p.codes_hi, self.device)
             if p.rank > 0:
                 tens["U"] = _dev(p.U, self.device)
                 tens["V"] = _dev(p.V, self.device)
@@ -61,6 +64,8 @@ class DeviceLayer:
             cp.codes = L._ptr(tens["codes"])
             cp.scales = L._ptr(tens["scales"])
             cp.zeros = L._ptr(tens["zeros"])
+            cp.bits = bits
+            cp.codes_hi = L._ptr(tens.get("codes_hi"))
             cp.U = L._ptr(tens.get("U"))
             cp.V = L._ptr(tens.get("V"))
             cp.Sigma = L._ptr(tens.get("Sigma"))
