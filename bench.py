@@ -15,6 +15,7 @@ scaling, no data-path collective (the forward has no exchange step).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -68,6 +69,7 @@ def parse():
                     help="time the expert placement (embeddings, K-Means biclustering, greedy 2D placement) "
                          "of the configuration's gate projection instead of the forward")
     ap.add_argument("--r0", type=int, default=16, help="rank of the per-expert factors for --place")
+    ap.add_argument("--bits", type=int, default=2, choices=[2, 3], help="residual code width of the layer")
     return ap.parse_args()
 
 
@@ -211,7 +213,7 @@ def workload_config(cfg, T, args, l2):
     return {"workload": f"{cfg.name} T={T}", "experts": cfg.K, "grid": f"{cfg.M}x{cfg.N}",
             "d_model": cfg.d_model, "d_ff": cfg.d_ff, "rank": cfg.rank, "group": cfg.group,
             "top_k": cfg.top_k, "tokens_per_gpu": T, "shared_d_ff": cfg.shared_d_ff,
-            "residual_bits": 2, "parallelism": f"replicas x{args.gpus}", "l2": l2}
+            "residual_bits": cfg.bits, "parallelism": f"replicas x{args.gpus}", "l2": l2}
 
 
 # ---------------------------------------------------------------------------
@@ -399,6 +401,8 @@ def run_place(args, cfg):
 def main():
     args = parse()
     cfg = synth.CONFIGS[args.config]
+    if args.bits != cfg.bits:
+        cfg = dataclasses.replace(cfg, bits=args.bits, name=f"{cfg.name}-{args.bits}bit")
     T = args.batch or (64 if args.config == 1 else cfg.batches[-1])
     if args.sketch:
         run_sketch(args, cfg)

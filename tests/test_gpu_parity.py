@@ -256,10 +256,12 @@ def _sample(T, n, seed):
     return np.sort(rng.choice(T, size=min(n, T), replace=False))
 
 
-def _full_config_check(torch, cfg_ids, samples, variants=("normal", "zero_residual", "rank0")):
+def _full_config_check(torch, cfg_ids, samples, variants=("normal", "zero_residual", "rank0"), bits=2):
     """One oracle pass per layer variant over the sampled tokens of every batch."""
+    import dataclasses
     from tiled_rank_b200 import DeviceLayer
-    cfg0 = synth.CONFIGS[cfg_ids[0]]
+    cfgs = {c: dataclasses.replace(synth.CONFIGS[c], bits=bits) for c in cfg_ids}
+    cfg0 = cfgs[cfg_ids[0]]
     base = synth.make_layer(cfg0)
     for variant in variants:
         if variant == "normal":
@@ -272,7 +274,7 @@ def _full_config_check(torch, cfg_ids, samples, variants=("normal", "zero_residu
         dl = DeviceLayer(layer, torch.device("cuda:0"))
         xs, ls, gpu_rows = [], [], []
         for cid in cfg_ids:
-            cfg = synth.CONFIGS[cid]
+            cfg = cfgs[cid]
             for T in cfg.batches:
                 logits, x = synth.make_inputs(cfg, T)
                 out, route, _ = run_gpu(torch, layer, logits, x, dl=dl)
@@ -291,6 +293,12 @@ def _full_config_check(torch, cfg_ids, samples, variants=("normal", "zero_residu
 @pytest.mark.slow
 def test_mixtral_shaped_decode_and_prefill(torch_cuda):
     _full_config_check(torch_cuda, (1, 2), samples=3)
+
+
+@pytest.mark.slow
+def test_mixtral_shaped_3bit(torch_cuda):
+    """The Mixtral-shaped layer with 3-bit residual codes, decode and prefill."""
+    _full_config_check(torch_cuda, (1, 2), samples=3, bits=3)
 
 
 @pytest.mark.slow

@@ -1,7 +1,8 @@
 """Algorithmic work of the TileQ MoE forward: bytes the method must touch and
 FLOPs it must do, from the realised routing (host logic, no GPU).
 
-Bytes: the stored residual (2-bit codes, fp16 group scales, 2-bit zero points)
+Bytes: the stored residual (2- or 3-bit codes, fp16 group scales, 2- or 3-bit
+zero points, the latter stored in 4-bit fields)
 of every active expert once per projection; the shared low-rank blocks U_m of
 active grid rows and V_n of active grid columns once; x, router logits and the
 output once; the shared expert's bf16 weights.
@@ -18,9 +19,11 @@ import math
 import numpy as np
 
 
-def residual_bytes(d_out: int, d_in: int, group: int) -> int:
+def residual_bytes(d_out: int, d_in: int, group: int, bits: int = 2) -> int:
     """Stored bytes of one expert's residual in one projection."""
     G = d_in // group
+    if bits == 3:
+        return d_out * d_in * 3 // 8 + d_out * G * 2 + d_out * math.ceil(G / 2)
     return d_out * d_in // 4 + d_out * G * 2 + d_out * math.ceil(G / 4)
 
 
@@ -63,7 +66,7 @@ def work(layer, topk_idx: np.ndarray) -> dict:
         return len(s["rows"]) * p.d_out * p.rank * 2
 
     def res(p, s):
-        return len(s["experts"]) * residual_bytes(p.d_out, p.d_in, p.group)
+        return len(s["experts"]) * residual_bytes(p.d_out, p.d_in, p.group, getattr(p, "bits", 2))
 
     if layer.kind == 0:
         p, s = layer.projs[0], sets[0]
