@@ -78,8 +78,6 @@ enum { TILEQ_LINEAR = 0, TILEQ_SWIGLU = 1 };
  *                zeros are device uint8 [K, d_out, ceil(d_in/group/2)] with group j
  *                at bits 4*(j%2) of byte j/2 (values 0..7), and
  *   codes_hi     device uint32 [K, d_out, d_in/32], element j at bit j%32 (3-bit only).
- *                3-bit projections run the residual on warp-level MMA at every
- *                batch size (the tcgen05 residual kernel reads 2-bit codes only).
  *   Residual: w[o,i] = scales[o,i/group] * (q[o,i] - z[o,i/group]).
  * Supported: d_out % 16 == 0, d_in % 128 == 0, group == 64 or a multiple of 128,
  * d_in % group == 0,

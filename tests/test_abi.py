@@ -275,8 +275,8 @@ def test_place_workspace_and_validation(L):
 
 
 def test_3bit_validation_and_packed_size(L):
-    """3-bit projections: bits in {0, 2, 3}; the packed copy drops the tcgen05
-    row layout (2 bits/weight) and adds the high-bit plane (1 bit/weight)."""
+    """3-bit projections: bits in {0, 2, 3}; the packed copy adds the high-bit
+    plane beside each of the two code layouts (1 bit/weight each)."""
     c2, layer = _host_layer(L, 0)
     n2 = L.tileq_packed_size(c2)
     cfg3 = synth.Config(**{**synth.CONFIGS[0].__dict__, "bits": 3})
@@ -285,7 +285,7 @@ def test_3bit_validation_and_packed_size(L):
         c3.proj[i].bits = 3
     n3 = L.tileq_packed_size(c3)
     p = layer.projs[0]
-    assert n3 - n2 == -layer.K * p.d_out * p.d_in // 4 + layer.K * p.d_out * p.d_in // 8
+    assert n3 - n2 == 2 * (layer.K * p.d_out * p.d_in // 8)
     c3.proj[0].bits = 4
     with pytest.raises(L.TileQError) as e:
         L.tileq_packed_size(c3)

@@ -125,6 +125,9 @@ TINY = [
     # more than 4096 pairs: the multi-CTA sort, its slot tables and grid-row flags
     (synth.SWIGLU, 16, 4, 4, 128, 128, 16, 64, 4, 0, 1500),
     (synth.LINEAR, 12, 3, 4, 128, 128, 16, 64, 3, 0, 1700),
+    # groups of 256 (one (scale, zero) word per two 128-wide K blocks), warp MMA and tcgen05
+    (synth.SWIGLU, 4, 2, 2, 512, 256, 16, 256, 2, 0, 12),
+    (synth.LINEAR, 4, 2, 2, 512, 128, 16, 256, 2, 0, 200),
 ]
 
 
@@ -165,14 +168,15 @@ def test_full_softmax_routing(torch_cuda, case):
     assert np.abs(out - ref).max() < 0.25 * np.abs(out - default).max()
 
 
-# 3-bit residuals (q = codes + 4 * high bit; zeros 0..7).  They run the warp-MMA
-# residual kernel at every batch size: 300 tokens over 8 experts would take
-# tcgen05 tiles with 2-bit codes.
+# 3-bit residuals (q = codes + 4 * high bit; zeros 0..7): short batches on
+# warp-level MMA, longer ones (more than 32 items per expert) on tcgen05
 TINY3 = [
     (synth.SWIGLU, 8, 2, 4, 256, 512, 32, 128, 2, 0, 16),
     (synth.SWIGLU, 8, 2, 4, 256, 512, 32, 128, 2, 256, 300),
     (synth.LINEAR, 5, 2, 3, 384, 144, 16, 64, 3, 0, 200),
     (synth.SWIGLU, 16, 4, 4, 128, 128, 16, 64, 4, 0, 1500),
+    (synth.LINEAR, 4, 2, 2, 512, 128, 16, 256, 2, 0, 200),
+    (synth.LINEAR, 4, 2, 2, 4096, 256, 16, 128, 2, 0, 600),
 ]
 
 

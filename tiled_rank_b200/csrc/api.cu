@@ -123,7 +123,7 @@ size_t frag_bytes(int nblk, int R, int C, int kb) {
 // weights row-major fp16 [pad128(rows)][cols] (the A operands of the tcgen05
 // kernel; vf / sh hold the same values in warp-MMA fragment order).
 struct PackedLayout {
-  size_t qw[3], qf[3], qfh[3], sz[3], uf[3], vf[3], sig[3], vr[3], sh[3], shr[3], total;
+  size_t qw[3], qwh[3], qf[3], qfh[3], sz[3], uf[3], vf[3], sig[3], vr[3], sh[3], shr[3], total;
 };
 
 PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
@@ -131,8 +131,10 @@ PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
   size_t off = 0;
   for (int p = 0; p < li.nproj; ++p) {
     const ProjInfo &q = li.p[p];
-    pl.qw[p] = off;   // tcgen05 row layout (2-bit only: 3-bit runs on warp MMA)
-    if (q.bits == 2) off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 4);
+    pl.qw[p] = off;   // tcgen05 row layout
+    off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 4);
+    pl.qwh[p] = off;  // 3-bit high-bit plane, row layout
+    if (q.bits == 3) off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 8);
     pl.qf[p] = off;
     off += align_up((size_t)L->K * pad128(q.d_out) * q.d_in / 4);
     pl.qfh[p] = off;  // 3-bit high-bit plane, fragment layout
@@ -237,11 +239,8 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   // MMA than on tcgen05 (measured: an M=128 N=16 tcgen05.mma does fewer MACs per
   // cycle than mma.sync, and the decode then dominates); wider ones on tcgen05.
   const long long avg = P / std::max(1, L->K);
-  bool any3 = false;   // the tcgen05 residual kernel reads 2-bit codes only
-  for (int p = 0; p < li.nproj; ++p) any3 = any3 || li.p[p].bits == 3;
-  const bool use_tc = avg > 32 && !any3;
-  // warp-MMA tiles hold at most 32 items (3-bit layers keep them at any batch)
-  pl.bn_main = use_tc ? choose_bn_tc(avg) : std::min(choose_bn(avg), 32);
+  const bool use_tc = avg > 32;
+  pl.bn_main = use_tc ? choose_bn_tc(avg) : choose_bn(avg);
   pl.slots_main = cdiv(P, pl.bn_main) + L->K;
   const long long est_main = std::min(L->K, P) + P / pl.bn_main;
   auto tc_plan = [&](int d_out, int d_in, int np) {
@@ -657,7 +656,9 @@ tileq_status run_residual(const Residual &r, const GemmPlan &g, const LayerInfo 
   for (int i = 0; i < r.np; ++i) {
     // tcgen05 reads the row layout of the codes, warp MMA the fragment layout
     a.codes[i] = at<uint4>(packed, g.tc ? pl.qw[r.proj[i]] : pl.qf[r.proj[i]]);
-    a.codes_hi[i] = li.p[r.proj[i]].bits == 3 ? at<uint2>(packed, pl.qfh[r.proj[i]]) : nullptr;
+    const bool q3 = li.p[r.proj[i]].bits == 3;
+    a.codes_hi[i] = q3 && !g.tc ? at<uint2>(packed, pl.qfh[r.proj[i]]) : nullptr;
+    a.codes_hi_rows[i] = q3 && g.tc ? at<uint32_t>(packed, pl.qwh[r.proj[i]]) : nullptr;
     a.sz[i] = at<uint32_t>(packed, pl.sz[r.proj[i]]);
     if (r.ext) tc_ext(&a, i, li, pl, packed, r.proj[i], r.ext_col[i]);
   }
@@ -962,17 +963,18 @@ tileq_status tileq_pack(const tileq_layer *layer, void *packed, size_t packed_by
     const ProjInfo &q = li.p[p];
     {
       const long long n = (long long)K * (pad128(q.d_out) / 128) * (q.d_in / 128) * 128 * 8;
-      if (q.bits == 2) {
-        pack_codes_tc_kernel<<<nblocks(n, 256), 256, 0, stream>>>(src.codes, at<uint32_t>(packed, pl.qw[p]),
-                                                                   K, q.d_out, q.d_in);
-        TQ_LAUNCHED();
-      }
+      pack_codes_tc_kernel<<<nblocks(n, 256), 256, 0, stream>>>(src.codes, at<uint32_t>(packed, pl.qw[p]),
+                                                                 K, q.d_out, q.d_in);
+      TQ_LAUNCHED();
       pack_codes_kernel<<<nblocks(n / 4, 256), 256, 0, stream>>>(src.codes, at<uint4>(packed, pl.qf[p]),
                                                                  K, q.d_out, q.d_in);
       TQ_LAUNCHED();
       if (q.bits == 3) {
         pack_codes_hi_kernel<<<nblocks(n / 4, 256), 256, 0, stream>>>(src.codes_hi, at<uint2>(packed, pl.qfh[p]),
                                                                       K, q.d_out, q.d_in);
+        TQ_LAUNCHED();
+        pack_codes_tc_hi_kernel<<<nblocks(n / 2, 256), 256, 0, stream>>>(
+            src.codes_hi, at<uint32_t>(packed, pl.qwh[p]), K, q.d_out, q.d_in);
         TQ_LAUNCHED();
       }
     }

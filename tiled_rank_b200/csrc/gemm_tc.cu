@@ -49,7 +49,7 @@ constexpr int BK = 128;  // K per stage
 #endif
 constexpr int kDqw128 = TILEQ_TC_DQW128;  // dequantising warps of the 128-item tiles
 
-template <int NP, int BN, int DQW>
+template <int NP, int BN, int DQW, bool Q3 = false>
 struct TcCfg {
   // one-projection launches: eight more warps run the epilogue, from a second
   // accumulator buffer while the next unit's MMAs fill the first when BN <= 128
@@ -62,9 +62,11 @@ struct TcCfg {
   static constexpr int KPW = BK / (DQW / 4);          // K elements per dequant warp per stage
   static constexpr int CODES = NP * 128 * 32;         // packed codes of one stage (bytes)
   static constexpr int SZ = NP * 2 * 128 * 4;         // scale/zero words, up to 2 groups per stage
+  static constexpr int HI = Q3 ? NP * 128 * 16 : 0;   // 3-bit codes: the high-bit plane of the stage
   static constexpr int BATOM = BN * 128;              // one 64-wide K atom of B (bytes)
   static constexpr int B = 2 * BATOM;                 // 128 K (main) or 128 extension columns of one projection
-  static constexpr int QSTAGE = ((CODES + SZ + B) + 1023) / 1024 * 1024;
+  static constexpr int QSTAGE = ((CODES + SZ + HI + B) + 1023) / 1024 * 1024;
+  static_assert((CODES + SZ + HI) % 1024 == 0, "B atoms need 1024-byte alignment");
   // one-projection launches with two accumulator buffers stage the epilogue in
   // shared memory: per column half, two buffers of EBATCH items x 128 rows of
   // fp32, written out by bulk copies (one per item row) instead of one store
@@ -105,6 +107,26 @@ __device__ __forceinline__ void tc_epi_store(const TcArgs &P, int item, int o, f
   }
 }
 
+// 3-bit codes: as dq_word, with the high bit of pair (hb, i) at bits
+// 2 + 2i + hb and 18 + 2i + hb of `h`, just above the 2-bit field once shifted
+// by hb: the fp16 value becomes 1024 + 4^i*q (q <= 7), still exact.
+__device__ __forceinline__ void dq_word3(uint32_t w, uint32_t h, const __half2 (&nz)[4], __half2 s2,
+                                         uint32_t *out) {
+  const uint32_t kMagic = 0x64006400u;
+  const __half2 m[4] = {u32_as_h2(0x3C003C00u), u32_as_h2(0x34003400u), u32_as_h2(0x2C002C00u),
+                        u32_as_h2(0x24002400u)};
+#pragma unroll
+  for (int hb = 0; hb < 2; ++hb) {
+    const uint32_t v = hb ? (w >> 8) : w;
+    const uint32_t hv = hb ? (h >> 1) : h;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 x = u32_as_h2(and_or(v, 0x00030003u << (2 * i), and_or(hv, 0x00040004u << (2 * i), kMagic)));
+      out[4 * hb + i] = h2_as_u32(__hmul2(__hfma2(x, m[i], nz[i]), s2));
+    }
+  }
+}
+
 // Decode 16 codes (one packed word) into 8 fp16x2 of s * (q - z).
 __device__ __forceinline__ void dq_word(uint32_t w, const __half2 (&nz)[4], __half2 s2, uint32_t *out) {
   const uint32_t kMagic = 0x64006400u;
@@ -121,9 +143,9 @@ __device__ __forceinline__ void dq_word(uint32_t w, const __half2 (&nz)[4], __ha
   }
 }
 
-template <int NP, int BN, int DQW>
-__global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel(const __grid_constant__ TcArgs P) {
-  using C = TcCfg<NP, BN, DQW>;
+template <int NP, int BN, int DQW, bool Q3>
+__global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_kernel(const __grid_constant__ TcArgs P) {
+  using C = TcCfg<NP, BN, DQW, Q3>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *q_full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
@@ -141,7 +163,10 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
   auto q_sz = [&](int s, int p) {
     return reinterpret_cast<uint32_t *>(smem + s * C::QSTAGE + C::CODES) + p * 2 * 128;
   };
-  auto q_b = [&](int s) { return smem + s * C::QSTAGE + C::CODES + C::SZ; };
+  auto q_hi = [&](int s, int p) {
+    return reinterpret_cast<const uint32_t *>(smem + s * C::QSTAGE + C::CODES + C::SZ) + p * 4 * 128;
+  };
+  auto q_b = [&](int s) { return smem + s * C::QSTAGE + C::CODES + C::SZ + C::HI; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::SQ; ++s) {
@@ -409,10 +434,13 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
           TC_TRACE(0, qi);
           if (st < nmain) {
             const int kb = kb0 + st;
-            mbar_arrive_expect_tx(&q_full[s], NP * (128 * 32 + gps * 512) + 2 * C::BATOM);
+            mbar_arrive_expect_tx(&q_full[s], NP * (128 * 32 + gps * 512) + C::HI + 2 * C::BATOM);
             for (int p = 0; p < NP; ++p) {
               const size_t cblk = (((size_t)grp * P.m_tiles + ob) * nkb + kb) * (128 * 32);
               bulk_g2s(q_codes(s, p), reinterpret_cast<const uint8_t *>(P.codes[p]) + cblk, 128 * 32, &q_full[s]);
+              if constexpr (Q3)
+                bulk_g2s(const_cast<uint32_t *>(q_hi(s, p)),
+                         reinterpret_cast<const uint8_t *>(P.codes_hi_rows[p]) + cblk / 2, 128 * 16, &q_full[s]);
               const size_t zoff = (((size_t)grp * P.m_tiles + ob) * G + (kb * BK) / g) * 128;
               bulk_g2s(q_sz(s, p), P.sz[p] + zoff, gps * 512, &q_full[s]);
             }
@@ -540,8 +568,15 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
               const __half2 z2 = __high2half2(sz), s2 = __low2half2(sz);
               const __half2 nz[4] = {__hsub2(__float2half2_rn(-1024.f), z2), __hsub2(__float2half2_rn(-256.f), z2),
                                      __hsub2(__float2half2_rn(-64.f), z2), __hsub2(__float2half2_rn(-16.f), z2)};
-              dq_word(cw[0], nz, s2, v);
-              dq_word(cw[1], nz, s2, v + 8);
+              if constexpr (Q3) {
+                // one high-bit word per (K slice, row): code word 1's bits rotated by 8
+                const uint32_t hw = q_hi(s, p)[(k0 / 32) * 128 + row];
+                dq_word3(cw[0], hw, nz, s2, v);
+                dq_word3(cw[1], __funnelshift_r(hw, hw, 8), nz, s2, v + 8);
+              } else {
+                dq_word(cw[0], nz, s2, v);
+                dq_word(cw[1], nz, s2, v + 8);
+              }
             } else {
               const int e = (st - nmain) % n_ext1;
               const int kg = e * BK + k0;          // column of U
@@ -634,10 +669,10 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW>::THREADS, 1) gemm_tc_kernel
   }
 }
 
-template <int NP, int BN, int DQW>
+template <int NP, int BN, int DQW, bool Q3>
 cudaError_t launch_tc_one(const TcArgs &a, int grid, cudaStream_t stream) {
-  using C = TcCfg<NP, BN, DQW>;
-  auto kern = gemm_tc_kernel<NP, BN, DQW>;
+  using C = TcCfg<NP, BN, DQW, Q3>;
+  auto kern = gemm_tc_kernel<NP, BN, DQW, Q3>;
   static bool configured = false;  // one attribute call per instantiation and process
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -650,15 +685,15 @@ cudaError_t launch_tc_one(const TcArgs &a, int grid, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <int NP>
+template <int NP, bool Q3>
 cudaError_t launch_tc_bn(const TcArgs &a, int bn, int grid, cudaStream_t s) {
   switch (bn) {
-    case 16: return launch_tc_one<NP, 16, 16>(a, grid, s);
-    case 32: return launch_tc_one<NP, 32, 16>(a, grid, s);
-    case 64: return launch_tc_one<NP, 64, 16>(a, grid, s);
-    case 128: return launch_tc_one<NP, 128, kDqw128>(a, grid, s);
+    case 16: return launch_tc_one<NP, 16, 16, Q3>(a, grid, s);
+    case 32: return launch_tc_one<NP, 32, 16, Q3>(a, grid, s);
+    case 64: return launch_tc_one<NP, 64, 16, Q3>(a, grid, s);
+    case 128: return launch_tc_one<NP, 128, kDqw128, Q3>(a, grid, s);
     case 256:  // one projection only: two 256-column accumulators would fill tensor memory
-      if constexpr (NP == 1) return launch_tc_one<NP, 256, kDqw128>(a, grid, s);
+      if constexpr (NP == 1) return launch_tc_one<NP, 256, kDqw128, Q3>(a, grid, s);
       return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
@@ -692,7 +727,9 @@ int tc_smem_bytes(int np, int bn) {
 
 cudaError_t launch_gemm_tc(const TcArgs &a, int np, int bn, int grid, cudaStream_t stream) {
   if (grid <= 0) return cudaSuccess;
-  return np == 1 ? launch_tc_bn<1>(a, bn, grid, stream) : launch_tc_bn<2>(a, bn, grid, stream);
+  if (a.codes_hi_rows[0] != nullptr)   // 3-bit codes
+    return np == 1 ? launch_tc_bn<1, true>(a, bn, grid, stream) : launch_tc_bn<2, true>(a, bn, grid, stream);
+  return np == 1 ? launch_tc_bn<1, false>(a, bn, grid, stream) : launch_tc_bn<2, false>(a, bn, grid, stream);
 }
 
 }  // namespace tileq

@@ -147,8 +147,10 @@ struct TcArgs {
   const uint4 *codes[2];     // tcgen05: [K][d_out/128][d_in/128][4 slices][128 rows][8 B]
                              // warp MMA: [K][d_out/128][d_in/128][8 warps][32 lanes][16 B]
   const uint32_t *sz[2];     // [K][d_out/128][G][128 rows] {fp16 scale, fp16 zero}
-  const uint2 *codes_hi[2];  // 3-bit high plane, warp MMA only: [K][d_out/128][d_in/128][8 warps][32 lanes][8 B];
+  const uint2 *codes_hi[2];  // 3-bit high plane, warp MMA: [K][d_out/128][d_in/128][8 warps][32 lanes][8 B];
                              // null for 2-bit codes
+  const uint32_t *codes_hi_rows[2];  // 3-bit high plane, tcgen05: [K][d_out/128][d_in/128][4 slices][128 rows]
+                                     // u32; null for 2-bit codes
   const __half *u[2];        // [M][pad128(d_out)][rank] fp16
   int8_t u_blk[2][kMaxExperts];
   int epi;
@@ -291,6 +293,7 @@ __global__ void bounded_wait_kernel(int *status, int max_polls);
 //   frag   [blk][R/128][C/(16*kb)][8 warps][kb k16 steps][32 lanes] uint4 (fp16 A fragments)
 __global__ void pack_codes_kernel(const uint32_t *codes, uint4 *out, int K, int d_out, int d_in);
 __global__ void pack_codes_hi_kernel(const uint32_t *hi, uint2 *out, int K, int d_out, int d_in);
+__global__ void pack_codes_tc_hi_kernel(const uint32_t *hi, uint32_t *out, int K, int d_out, int d_in);
 __global__ void pack_sz_kernel(const __half *scales, const uint8_t *zeros, uint32_t *out, int K,
                                int d_out, int G, int bits);
 // Element (i, j) of block b of a bf16 matrix S[R][C] is src[b*bs + i*rs + j*cs].

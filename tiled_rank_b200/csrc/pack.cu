@@ -193,6 +193,42 @@ __global__ void pack_codes_tc_kernel(const uint32_t *codes, uint32_t *out, int K
   out[gid] = acc;
 }
 
+// 3-bit codes' high bits [K][d_out][d_in/32] -> [K][R/128][d_in/128][4 slices][128 rows]
+// u32, beside pack_codes_tc_kernel's layout: the word of (slice, row) holds
+// the high bits of its two code words (16-element halves wi = 0, 1).  Pair p,
+// half h of code word 0 at bit (h ? 16 : 0) + 2 + 2*(p%4) + p/4, just above the
+// 2-bit field once the decoder has shifted by p/4; code word 1's bits rotated
+// left by 8.
+__global__ void pack_codes_tc_hi_kernel(const uint32_t *hi, uint32_t *out, int K, int d_out, int d_in) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nkb = d_in / 128, n128 = pad128(d_out) / 128, wpr = d_in / 32;
+  const long long total = (long long)K * n128 * nkb * 4 * 128;
+  if (gid >= total) return;
+  const int r = (int)(gid % 128);
+  const int part = (int)((gid / 128) % 4);
+  long long rest = gid / 512;
+  const int kb = (int)(rest % nkb);
+  rest /= nkb;
+  const int ob = (int)(rest % n128);
+  const int e = (int)(rest / n128);
+  const int row = ob * 128 + r;
+  uint32_t acc = 0;
+  if (row < d_out) {
+    for (int wi = 0; wi < 2; ++wi) {
+      uint32_t a = 0;
+      for (int p = 0; p < 8; ++p)
+        for (int h = 0; h < 2; ++h) {
+          const int col = kb * 128 + (part * 2 + wi) * 16 + 2 * p + h;
+          const uint32_t b = (hi[((size_t)e * d_out + row) * wpr + col / 32] >> (col % 32)) & 1u;
+          a |= b << ((h ? 16 : 0) + 2 + 2 * (p % 4) + p / 4);
+        }
+      if (wi) a = (a << 8) | (a >> 24);
+      acc |= a;
+    }
+  }
+  out[gid] = acc;
+}
+
 // Sigma [r] -> [n][rp] (rp = r rounded up to 128; zeros past r): the column
 // scales of the projection onto all n grid columns at once.
 __global__ void expand_sigma_kernel(const float *sigma, int r, int rp, int n, float *out) {
