@@ -120,3 +120,42 @@ def test_place_experts_recovers_planted_grid(K, M, N, d_u, d_v, r0):
     # a full grid of distinct (row, column) clusters: every expert gets its ideal cell
     assert np.array_equal(g, lm * N + ln)
     assert all(1 <= i <= 100 for i in its)
+
+
+def _greedy_rounds(im, inn, M, N):
+    """The greedy order restated as the GPU runs it: first every distance-0
+    pair whose expert is the lowest index wanting that cell, then one round
+    per remaining expert, each placing the smallest (distance, expert, cell)
+    key over the unplaced experts' best free cells."""
+    K = len(im)
+    grid = [-1] * K
+    free = [True] * (M * N)
+    for k in range(K):
+        c = int(im[k]) * N + int(inn[k])
+        if all(int(im[j]) * N + int(inn[j]) != c for j in range(k)):
+            grid[k] = c
+            free[c] = False
+    while any(g < 0 for g in grid):
+        best = None
+        for k in range(K):
+            if grid[k] >= 0:
+                continue
+            for c in range(M * N):
+                if free[c]:
+                    key = ((c // N - im[k]) ** 2 + (c % N - inn[k]) ** 2, k, c)
+                    best = key if best is None or key < best else best
+        _, k, c = best
+        grid[k] = c
+        free[c] = False
+    return np.array(grid, dtype=np.int32)
+
+
+@pytest.mark.parametrize("K,M,N,spread,seed", [(64, 8, 8, 3, 0), (60, 6, 10, 2, 1), (8, 2, 4, 1, 2),
+                                               (33, 4, 9, 4, 3), (5, 3, 3, 1, 4), (64, 8, 8, 1, 5)])
+def test_greedy_round_form_matches_sorted_scan(K, M, N, spread, seed):
+    """Ideal coordinates crowded into a corner (many conflicts): the round-by-
+    round form with the distance-0 head gives the sorted-scan result."""
+    rng = np.random.default_rng(seed)
+    im = rng.integers(0, min(M, spread), K)
+    inn = rng.integers(0, min(N, spread), K)
+    assert np.array_equal(_greedy_rounds(im, inn, M, N), P.greedy_place(im, inn, M, N))
