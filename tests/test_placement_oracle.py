@@ -159,3 +159,52 @@ def test_greedy_round_form_matches_sorted_scan(K, M, N, spread, seed):
     im = rng.integers(0, min(M, spread), K)
     inn = rng.integers(0, min(N, spread), K)
     assert np.array_equal(_greedy_rounds(im, inn, M, N), P.greedy_place(im, inn, M, N))
+
+
+def _kmeans_gram_form(E, C, max_iter):
+    """Lloyd K-Means evaluated as the GPU does: only the normalised Gram
+    matrix G of the embeddings, every centre as weights a_j over the points,
+    |e_i - c_j|^2 = G_ii - 2 (G a_j)_i + a_j^T G a_j."""
+    G = E @ E.T
+    n = np.sqrt(np.diag(G))
+    inv = np.where(n > 0, 1.0 / np.where(n > 0, n, 1.0), 0.0)
+    G = G * inv[:, None] * inv[None, :]
+    P_ = len(E)
+    alpha = np.zeros((C, P_))
+    mind = None
+    p = 0
+    for j in range(C):
+        if j > 0:
+            p = int(np.argmax(mind))
+        alpha[j, p] = 1.0
+        d = np.diag(G) - 2 * G[:, p] + G[p, p]
+        mind = d if j == 0 else np.minimum(mind, d)
+
+    def assign():
+        H = alpha @ G                                   # [C, P]
+        q = np.einsum("jp,jp->j", alpha, H)
+        return np.argmin(np.diag(G)[:, None] - 2 * H.T + q[None, :], axis=1)
+
+    labels = assign()
+    it = 0
+    while it < max_iter:
+        for j in range(C):
+            m = labels == j
+            if m.any():
+                alpha[j] = m / m.sum()
+        it += 1
+        new = assign()
+        if np.array_equal(new, labels):
+            break
+        labels = new
+    return labels, it
+
+
+@pytest.mark.parametrize("P_,D,C,seed", [(64, 3, 8, 0), (60, 2, 6, 1), (64, 40, 8, 2), (33, 7, 4, 3)])
+def test_kmeans_gram_form_matches_direct(P_, D, C, seed):
+    rng = np.random.default_rng(seed)
+    E = rng.standard_normal((P_, D))
+    E /= np.linalg.norm(E, axis=1, keepdims=True)
+    lab, _, it = P.kmeans(E, C, 100)
+    lab2, it2 = _kmeans_gram_form(E, C, 100)
+    assert np.array_equal(lab, lab2) and it == it2
