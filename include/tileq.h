@@ -20,8 +20,9 @@
  *   top-k of the fp32 router logits in descending order, equal logits -> the
  *   lower expert index first; weights = softmax over the k chosen logits
  *   (route_mode TILEQ_ROUTE_TOPK_SOFTMAX), or the k chosen entries of the
- *   softmax over all K logits, not renormalised (TILEQ_ROUTE_FULL_SOFTMAX,
- *   the routing variant of the TileQ summary's design notes).
+ *   softmax over all K logits, not renormalised (TILEQ_ROUTE_FULL_SOFTMAX).
+ *   Section 2.2 ("Mechanism") only says that routing weights select the
+ *   active tiles; both normalisations are readings of it.
  *   LINEAR layer:  out_t = sum_j w_j W_{e_j} x_t
  *   SWIGLU layer:  out_t = sum_j w_j W^down_{e_j} (silu(W^gate_{e_j} x_t) * (W^up_{e_j} x_t))
  *                  (+ an optional always-on dense bf16 SwiGLU shared expert, weight 1)
