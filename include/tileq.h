@@ -74,8 +74,8 @@ enum { TILEQ_LINEAR = 0, TILEQ_SWIGLU = 1 };
  *   scales       device fp16 [K, d_out, d_in/group]
  *   zeros        device uint8 [K, d_out, ceil(d_in/group/4)]; group j at bits 2*(j%4)
  *                of byte j/4
- *   bits         2 (or 0: a zero-initialised struct) or 3.  The summary evaluates
- *                2-bit and 3-bit residuals.  For 3: q = codes + 4 * (bit of codes_hi),
+ *   bits         2 (or 0: a zero-initialised struct) or 3 (the summary's section 4,
+ *                "Experimental Results", evaluates 2-bit and 3-bit TileQ).  For 3: q = codes + 4 * (bit of codes_hi),
  *                zeros are device uint8 [K, d_out, ceil(d_in/group/2)] with group j
  *                at bits 4*(j%2) of byte j/2 (values 0..7), and
  *   codes_hi     device uint32 [K, d_out, d_in/32], element j at bit j%32 (3-bit only).

@@ -148,7 +148,8 @@ def unpack_codes_hi(codes_hi, d_in: int) -> np.ndarray:
 
 def dequant(proj, e: int) -> np.ndarray:
     """deq(Q_e) float64 [d_out, d_in]: w[o, i] = s[o, i//g] * (q[o, i] - z[o, i//g]).
-    2-bit: q from `codes`; 3-bit (proj.bits == 3): q = codes + 4 * codes_hi bit."""
+    2-bit: q from `codes`; 3-bit (proj.bits == 3; the TileQ summary's section 4,
+    "Experimental Results", evaluates 2-bit and 3-bit): q = codes + 4 * codes_hi bit."""
     g = proj.group
     G = proj.d_in // g
     bits = getattr(proj, "bits", 2)
