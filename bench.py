@@ -250,11 +250,12 @@ def run_sketch(args, cfg):
     torch.cuda.synchronize()
     n0 = L.tileq_launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        L.tileq_sketch_lowrank(wb, om, l, r, U, S, V, ws)
-    e1.record()
-    torch.cuda.synchronize()
+    with ClockSampler(0) as clocks:
+        e0.record()
+        for _ in range(args.steps):
+            L.tileq_sketch_lowrank(wb, om, l, r, U, S, V, ws)
+        e1.record()
+        torch.cuda.synchronize()
     launches = L.tileq_launch_count() - n0
     ms = e0.elapsed_time(e1) / args.steps
     R, C = M * d_out, N * d_in
@@ -283,7 +284,7 @@ def run_sketch(args, cfg):
                      "unit": "TFLOP/s", "frac": t_roof / (ms / 1000.0), "traffic": None,
                      "note": "large products only; the two l x l Jacobi eigen-decompositions (one CTA, "
                              "latency-bound) take most of the time"},
-        "gpu_launches": launches, "cpu_baseline": cpu,
+        "gpu_launches": launches, "clocks": clocks.report(), "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
 
