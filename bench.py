@@ -7,8 +7,12 @@
 A step is one full forward (routing, permutation, column projection, gate/up,
 down-side projection, row accumulation, down/combine) over one batch of T
 synthetic tokens with every input already resident in HBM.  Default workload:
-the Mixtral-8x7B-shaped decode layer (8 experts on a 2x4 grid, d_model 4096,
-d_ff 14336, rank 128, 2-bit residual in groups of 128, top-2) at T=64.
+the largest single-GPU configuration, the fine-grained 64-expert layer (8x8
+grid, d_model 4096, d_ff 1536, rank 128, 2-bit residual in groups of 128,
+top-8) at T=16384 (prefill, tensor-bound).  The default run also times, each
+with its own roofline, the Mixtral-8x7B-shaped layer (8 experts on 2x4,
+d_model 4096, d_ff 14336, rank 128, top-2) at decode batches of 1, 8, 32 and
+64 tokens (HBM-bound) and at a 4096-token prefill (``extra_workloads``).
 With N > 1 (torchrun), every rank runs its own batch on its own GPU: weak
 scaling, no data-path collective (the forward has no exchange step).
 """
@@ -31,6 +35,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 L2_BYTES = 126 * 2**20
+DEFAULT_CONFIG = 4   # the largest single-GPU configuration: 64 experts on 8x8, 16384 tokens
 STAGES = ["route", "permute", "zproj", "gateup", "zdown", "rowacc", "residual", "shared", "combine"]
 
 
@@ -57,11 +62,13 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="tileq", choices=["tileq", "reference"])
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG)
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-compare", action="store_true", help="skip the unfused / rank-0 comparisons")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the extra decode / Mixtral-prefill workloads of the default run")
     ap.add_argument("--sketch", action="store_true",
                     help="time the Gaussian-sketch global low-rank decomposition of one projection's W_big "
                          "(the configuration's gate projection) instead of the forward")
@@ -162,6 +169,11 @@ def blas_threads():
         return 1
 
 
+def host_cores():
+    """Host cores this process may run on (the oracle's BLAS uses them)."""
+    return len(os.sched_getaffinity(0))
+
+
 def oracle_step(layer, x, logits, tok):
     import oracle
     return oracle.forward(layer, x, logits, tokens=[tok])
@@ -173,9 +185,10 @@ def cpu_baseline(layer, x, logits, n_tokens=1):
     for t in range(n_tokens):
         oracle_step(layer, x, logits, t)
     dt = time.perf_counter() - t0
-    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": host_cores(), "blas_threads": blas_threads(),
+            "kind": "oracle",
             "sample": f"{n_tokens} token(s) of the batch through the fp64 oracle "
-                      f"(dense reconstruction of each routed expert's 3 projections), {dt:.1f} s"}
+                      f"(dense reconstruction of each routed expert's projections), {dt:.1f} s"}
 
 
 def run_reference(args, cfg, T):
@@ -197,7 +210,8 @@ def run_reference(args, cfg, T):
         "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(cfg, T, args, "host"),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(),
+                         "blas_threads": blas_threads(),
                          "kind": "oracle",
                          "sample": "each step: one token of the batch through the fp64 oracle"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -399,39 +413,24 @@ def run_place(args, cfg):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    args = parse()
-    cfg = synth.CONFIGS[args.config]
-    if args.bits != cfg.bits:
-        cfg = dataclasses.replace(cfg, bits=args.bits, name=f"{cfg.name}-{args.bits}bit")
-    T = args.batch or (64 if args.config == 1 else cfg.batches[-1])
-    if args.sketch:
-        run_sketch(args, cfg)
-        return
-    if args.place:
-        run_place(args, cfg)
-        return
-    if args.impl == "reference":
-        run_reference(args, cfg, T)
-        return
-    if args.warmup < 3:
-        raise SystemExit("at least 3 warm-up steps")
+def default_batch(cid, cfg):
+    return 64 if cid == 1 else cfg.batches[-1]
 
+
+# Extra workloads timed in the default run, each with its own roofline: the
+# Mixtral-shaped decode batches (HBM-bound) and the Mixtral-shaped prefill
+# (tensor-bound); the headline is the largest single-GPU configuration.
+EXTRAS = [(1, 1), (1, 8), (1, 32), (1, 64), (2, 4096)]
+
+
+def measure(args, cfg, T, dev, world, rank, e2e=True, compare=True, cpu=True):
+    """Time K forwards of one workload; returns the fields of its JSON line."""
     import torch
     import torch.distributed as dist
     import tiled_rank_b200 as tq
     from tiled_rank_b200 import roofline
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-
+    local = dev.index
     layer = synth.make_layer(cfg, seed=args.seed)
     logits_np, x_np = synth.make_inputs(cfg, T, seed=rank_seed(args.seed, rank))
     dl = tq.DeviceLayer(layer, dev)
@@ -530,61 +529,110 @@ def main():
              "t_roof_ms": 1000 * max(wk["bytes"] / (peaks["hbm_gbs"] * 1e9),
                                      wk["flops"] / (peaks["bf16_tflops"] * 1e12))}
     whole["frac_of_roofline"] = whole["t_roof_ms"] / ms_per_step
+    res = {"ms_per_step": ms_per_step, "value": value, "roofline": roof, "whole_step": whole,
+           "stage_ms": stage_times, "gpu_launches": launches, "clocks": clocks.report(),
+           "config": workload_config(cfg, T, args,
+                                     "L2 flushed (256 MB write) between steps" if flush else
+                                     f"working set {footprint / 2**20:.0f} MB > 3x L2, no flush")}
 
     # ---------------- end to end through the public API with host buffers
-    x_h = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
-    lg_h = torch.from_numpy(logits_np).pin_memory()
-    out_h = torch.empty((T, dl.d_y), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(xt)
-    lgd = torch.empty_like(lg)
-    for _ in range(3):
-        xd.copy_(x_h, non_blocking=True)
-        lgd.copy_(lg_h, non_blocking=True)
-        dl.forward(xd, lgd, out=out, ws=ws)
-        out_h.copy_(out, non_blocking=True)
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(args.steps):
-        xd.copy_(x_h, non_blocking=True)
-        lgd.copy_(lg_h, non_blocking=True)
-        dl.forward(xd, lgd, out=out, ws=ws)
-        out_h.copy_(out, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
-    e2e = {"value": world * T * args.steps / (e2e_ms / 1000.0), "unit": "tokens/s",
-           "h2d_bytes_per_step": x_h.numel() * 2 + lg_h.numel() * 4,
-           "d2h_bytes_per_step": out_h.numel() * 2}
+    if e2e:
+        x_h = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+        lg_h = torch.from_numpy(logits_np).pin_memory()
+        out_h = torch.empty((T, dl.d_y), dtype=torch.bfloat16).pin_memory()
+        xd = torch.empty_like(xt)
+        lgd = torch.empty_like(lg)
+        for _ in range(3):
+            xd.copy_(x_h, non_blocking=True)
+            lgd.copy_(lg_h, non_blocking=True)
+            dl.forward(xd, lgd, out=out, ws=ws)
+            out_h.copy_(out, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(args.steps):
+            xd.copy_(x_h, non_blocking=True)
+            lgd.copy_(lg_h, non_blocking=True)
+            dl.forward(xd, lgd, out=out, ws=ws)
+            out_h.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        e2e_ms = float(e2e_ms.item())
+        res["e2e"] = {"value": world * T * args.steps / (e2e_ms / 1000.0), "unit": "tokens/s",
+                      "h2d_bytes_per_step": x_h.numel() * 2 + lg_h.numel() * 4,
+                      "d2h_bytes_per_step": out_h.numel() * 2}
 
     # ---------------- in-run comparisons (rank 0, N = 1)
-    extra = {}
-    if rank == 0 and world == 1 and not args.no_compare:
-        extra = compare_paths(cfg, layer, dl, xt, lg, out, T, args, flush_buf, ms_per_step)
+    if compare and rank == 0 and world == 1 and not args.no_compare:
+        res.update(compare_paths(cfg, layer, dl, xt, lg, out, T, args, flush_buf, ms_per_step))
+    if cpu and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(layer, x_np, logits_np, n_tokens=4)
+    del dl, ws, route, out, flush_buf
+    torch.cuda.empty_cache()
+    return res
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(layer, x_np, logits_np, n_tokens=4)
+
+def main():
+    args = parse()
+    cid = args.config
+    cfg = synth.CONFIGS[cid]
+    if args.bits != cfg.bits:
+        cfg = dataclasses.replace(cfg, bits=args.bits, name=f"{cfg.name}-{args.bits}bit")
+    T = args.batch or default_batch(cid, cfg)
+    if args.sketch:
+        run_sketch(args, cfg)
+        return
+    if args.place:
+        run_place(args, cfg)
+        return
+    if args.impl == "reference":
+        run_reference(args, cfg, T)
+        return
+    if args.warmup < 3:
+        raise SystemExit("at least 3 warm-up steps")
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    head = measure(args, cfg, T, dev, world, rank)
+    extras = {}
+    if world == 1 and not args.no_extras and args.batch is None and cid == DEFAULT_CONFIG and args.bits == 2:
+        for ec, eT in EXTRAS:
+            ecfg = synth.CONFIGS[ec]
+            r = measure(args, ecfg, eT, dev, world, rank, e2e=False, compare=False, cpu=False)
+            extras[f"{ecfg.name} T={eT}"] = {k: r[k] for k in ("ms_per_step", "value", "roofline", "whole_step",
+                                                               "stage_ms", "clocks")}
 
     if rank == 0:
         line = {
-            "metric": metric_name(cfg, T), "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "metric": metric_name(cfg, T), "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic (seeded numpy draws in the stored TileQ format)",
-            "config": workload_config(cfg, T, args,
-                                      "L2 flushed (256 MB write) between steps" if flush else
-                                      f"working set {footprint / 2**20:.0f} MB > 3x L2, no flush"),
-            "roofline": roof, "whole_step": whole, "stage_ms": stage_times,
-            "e2e": e2e, "gpu_launches": launches, "cpu_baseline": cpu,
-            "clocks": clocks.report(),
+            "config": head["config"], "roofline": head["roofline"], "whole_step": head["whole_step"],
+            "stage_ms": head["stage_ms"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+            "cpu_baseline": head.get("cpu_baseline"), "clocks": head["clocks"],
         }
-        line.update(extra)
+        for k in ("unfused", "rank0"):
+            if k in head:
+                line[k] = head[k]
+        if extras:
+            line["extra_workloads"] = extras
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

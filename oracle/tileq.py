@@ -75,8 +75,12 @@ def route(logits, top_k: int, full_softmax: bool = False):
     full_softmax: the chosen entries of the softmax over all K logits, not
     renormalised, w_j = exp(l_j - l_max) / sum_{all K} exp(l - l_max).
     Both in float64.  Returns (idx int32 [T, k], w float64 [T, k]).
+    Non-finite logits (the pages only meet finite ones; this is the reading
+    taken): a NaN ranks as -inf; when every chosen logit is -inf the weights are
+    equal (1/k, or 1/K for the full softmax), the limit of equal logits.
     """
-    lg = np.asarray(logits, dtype=np.float32)
+    lg = np.asarray(logits, dtype=np.float32).astype(np.float64)
+    lg = np.where(np.isnan(lg), -np.inf, lg)
     T, K = lg.shape
     if not 1 <= top_k <= K:
         raise ValueError("top_k out of range")
@@ -86,10 +90,13 @@ def route(logits, top_k: int, full_softmax: bool = False):
         order = sorted(range(K), key=lambda e: (-float(lg[t, e]), e))
         chosen = order[:top_k]
         vals = np.array([float(lg[t, e]) for e in chosen], dtype=np.float64)
-        ex = np.exp(vals - vals.max())
         idx[t] = chosen
+        if vals.max() == -np.inf:
+            w[t] = 1.0 / (K if full_softmax else top_k)
+            continue
+        ex = np.exp(vals - vals.max())
         if full_softmax:
-            every = np.exp(lg[t].astype(np.float64) - vals.max())
+            every = np.exp(lg[t] - vals.max())
             w[t] = ex / every.sum()
         else:
             w[t] = ex / ex.sum()
@@ -267,15 +274,23 @@ def forward(layer, x_bits, logits, tokens=None, return_h: bool = False):
     return out
 
 
-def forward_batched(layer, x_bits, logits):
+def forward_batched(layer, x_bits, logits, tokens=None):
     """Whole-batch forward, one dense float64 matmul per (expert, projection).
 
     Same definition as ``forward``; the tokens routed to an expert are stacked
-    so each reconstructed W_e is applied once.  Used for full-size outputs.
+    so each reconstructed W_e is applied once, and only one W_e is held at a
+    time.  ``tokens`` restricts the batch to a subset of token indices (their
+    own logits route them), returned in the given order.  Used for full-size
+    outputs.
     """
     x = widen_bf16(x_bits)
+    lg = np.asarray(logits, dtype=np.float32)
+    if tokens is not None:
+        sel = np.asarray(tokens, dtype=np.int64)
+        x = x[sel]
+        lg = lg[sel]
     T = x.shape[0]
-    idx, w = route(logits, layer.top_k, getattr(layer, "route_mode", 0) == 1)
+    idx, w = route(lg, layer.top_k, getattr(layer, "route_mode", 0) == 1)
     d_y = layer.projs[-1].d_out
     out = np.zeros((T, d_y), dtype=np.float64)
     for e in range(layer.K):
@@ -289,6 +304,7 @@ def forward_batched(layer, x_bits, logits):
             G = Xe @ expert_weight(layer.projs[0], e, layer.N).T
             Uu = Xe @ expert_weight(layer.projs[1], e, layer.N).T
             H = silu(G) * Uu
+            del G, Uu
             Y = H @ expert_weight(layer.projs[2], e, layer.N).T
         np.add.at(out, rows, w[rows, slots][:, None] * Y)
     if layer.shared is not None:

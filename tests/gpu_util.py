@@ -3,6 +3,7 @@ from __future__ import annotations
 
 import numpy as np
 
+import oracle
 import synth
 
 # parity bar: max|gpu - ref| <= 1e-2 * max|ref| and sum|gpu - ref| / sum|ref| <= 2e-3
@@ -70,3 +71,34 @@ def zero_residual(layer: synth.Layer, lr_gain: float = 1.0) -> synth.Layer:
         projs.append(synth.Proj(**{**p.__dict__, "codes": np.ascontiguousarray(zw), "U": U, **extra}))
     return synth.Layer(layer.kind, layer.K, layer.M, layer.N, layer.d_model, layer.d_ff,
                        layer.top_k, projs, layer.shared, layer.route_mode)
+
+
+N_DENSE = 256
+
+
+def dense_tokens(logits, top_k, K, seed, n_min=N_DENSE, route_mode=0):
+    """Tokens to compare at full size: every token when T <= n_min; otherwise the
+    tokens holding each active expert's first and last slot and the first and
+    last slot of every 128-slot run of each expert (so every 128- and 256-item
+    tile of the GEMMs, its ragged tail and every K split of it are covered),
+    topped up with seeded random tokens to at least n_min."""
+    T = logits.shape[0]
+    if T <= n_min:
+        return np.arange(T)
+    idx, _ = oracle.route(logits, top_k, route_mode == 1)
+    off, sp = oracle.permute(idx, K)
+    slots = []
+    for e in range(K):
+        a, b = int(off[e]), int(off[e + 1])
+        if b <= a:
+            continue
+        for t0 in range(a, b, 128):
+            slots += [t0, min(t0 + 127, b - 1)]
+    toks = set(int(sp[s]) // top_k for s in slots)
+    rng = np.random.default_rng(seed)
+    rest = rng.permutation(T)
+    i = 0
+    while len(toks) < n_min:
+        toks.add(int(rest[i]))
+        i += 1
+    return np.array(sorted(toks))

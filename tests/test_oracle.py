@@ -369,6 +369,9 @@ def test_batched_matches_per_token_loop():
     assert rel_err(b, a) < 1e-12
     sub = oracle.forward(layer, x, logits, tokens=[7, 2])
     assert rel_err(sub, a[[7, 2]]) < 1e-12
+    # the token subset of the batched form, in the given order, with a repeat
+    subb = oracle.forward_batched(layer, x, logits, tokens=[8, 0, 3, 0])
+    assert rel_err(subb, a[[8, 0, 3, 0]]) < 1e-12
 
 
 def test_memory_closed_form():
@@ -434,3 +437,22 @@ def test_dequant_3bit_range():
             w = oracle.dequant(p, e)
             ratio = np.abs(w).reshape(p.d_out, G, p.group) / s[e][:, :, None]
             assert ratio.max() <= 7.0 and ratio.max() >= 6.0   # q and z span 0..7
+
+
+def test_route_nonfinite_logits():
+    """A NaN logit ranks as -inf (below every finite logit; among -inf and NaN the
+    lower index first); a token whose chosen logits are all -inf gets equal weights."""
+    nan, inf = np.float32(np.nan), np.float32(np.inf)
+    lg = np.array([[0.5, nan, -1.0, 2.0],
+                   [nan, nan, 1.0, nan],
+                   [-inf, nan, -inf, nan]], dtype=np.float32)
+    idx, w = oracle.route(lg, 2)
+    assert idx.tolist() == [[3, 0], [2, 0], [0, 1]]
+    e = np.exp(0.5 - 2.0)
+    np.testing.assert_allclose(w[0], [1 / (1 + e), e / (1 + e)], rtol=1e-15)
+    np.testing.assert_allclose(w[1], [1.0, 0.0], atol=0)
+    np.testing.assert_allclose(w[2], [0.5, 0.5], atol=0)
+    idx_f, w_f = oracle.route(lg, 2, full_softmax=True)
+    assert np.array_equal(idx_f, idx)
+    np.testing.assert_allclose(w_f[1], [1.0, 0.0], atol=0)   # NaN entries add nothing to the mass
+    np.testing.assert_allclose(w_f[2], [0.25, 0.25], atol=0)

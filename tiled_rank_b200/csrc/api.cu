@@ -31,10 +31,7 @@ unsigned gather_blocks(long long chunks) {
   return std::max(1u, std::min(nblocks(chunks, 256), 8u * kNumSMs));
 }
 // split the narrow residual GEMM until ~this many CTAs per SM
-#ifndef TILEQ_Q2_PER_SM
-#define TILEQ_Q2_PER_SM 4
-#endif
-constexpr int kQ2PerSm = TILEQ_Q2_PER_SM;
+constexpr int kQ2PerSm = 4;
 constexpr int kTcMinTokens = 256;  // dense fp16 products (z, shared expert) move to tcgen05 from here
 constexpr int kWideMinK = 4096;    // 256-item tcgen05 tiles from this K (32 stages per unit) on
 

@@ -25,36 +25,6 @@
 
 namespace tileq {
 
-#ifdef TILEQ_TRACE
-// Debug builds only: clock64 time stamps of pipeline events of CTA 0, kept
-// separately for one- and two-projection launches.
-__device__ unsigned long long g_q2_trace[2][6][1024];
-#define Q2_TRACE(kind, idx) \
-  do {                      \
-    if (blockIdx.x == 0 && (idx) < 1024) g_q2_trace[NP - 1][kind][idx] = clock64(); \
-  } while (0)
-// per CTA: global nanosecond timer at start and at the end of the consumer loop
-__device__ unsigned long long g_q2_cta[2][1024][2];
-#define Q2_CTA_TIME(k)                                                                        \
-  do {                                                                                        \
-    unsigned long long t_;                                                                    \
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                     \
-    if (threadIdx.x == 0 && blockIdx.x < 1024) g_q2_cta[NP - 1][blockIdx.x][k] = t_;           \
-  } while (0)
-extern "C" int tileq_debug_q2_trace(unsigned long long *host) {
-  int e = (int)cudaMemcpyFromSymbol(host, g_q2_trace, sizeof(g_q2_trace));
-  if (e) return e;
-  return (int)cudaMemcpyFromSymbol(host + sizeof(g_q2_trace) / 8, g_q2_cta, sizeof(g_q2_cta));
-}
-#else
-#define Q2_TRACE(kind, idx) \
-  do {                      \
-  } while (0)
-#define Q2_CTA_TIME(k) \
-  do {                 \
-  } while (0)
-#endif
-
 namespace {
 
 constexpr int QW = 8;                    // consumer warps (16 rows each)
@@ -120,7 +90,6 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN, Q3>::MINB) gemm_q2_kern
   const int G = a.d_in / a.group;        // scale groups per row
   const bool g64 = a.group == 64;
 
-  Q2_CTA_TIME(0);
   // one CTA per (tile, 128-row block, K split)
   int bid = blockIdx.x;
   const int split = bid % a.ksplit;
@@ -168,7 +137,6 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN, Q3>::MINB) gemm_q2_kern
         if (lane == 0) ok = mbar_wait(&empty[s], par ^ 1u, a.status);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
-      if (lane == 0) Q2_TRACE(0, it);
       uint8_t *bs = st_b(s);
       if (it < nmain) {
         const int kb = 2 * (st0 + it);
@@ -374,9 +342,7 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN, Q3>::MINB) gemm_q2_kern
   int s = 0;
   uint32_t par = 0;
   for (int it = 0; it < nst; ++it) {
-    if (lane == 0 && (warp == 0 || warp == 7)) Q2_TRACE(warp == 0 ? 1 : 3, it);
     if (!mbar_wait(&full[s], par, a.status)) break;
-    if (lane == 0 && warp == 0) Q2_TRACE(2, it);
     if (it < nmain) {
       block_main(s, 0);
       if (2 * (st0 + it) + 1 < nkb) block_main(s, 1);
@@ -389,7 +355,6 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN, Q3>::MINB) gemm_q2_kern
         stage_ext(e, s, grp, ob, kvalid, std::false_type{});
     }
     __syncwarp();
-    if (lane == 0 && warp == 0) Q2_TRACE(4, it);
     if (lane == 0) mbar_arrive(&empty[s]);
     if (++s == C::S) {
       s = 0;
@@ -434,7 +399,6 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN, Q3>::MINB) gemm_q2_kern
   }  // consumer warps
 
   if (a.ksplit == 1) {
-    Q2_CTA_TIME(1);
     return;
   }
   // ------------------------------------------------------------ split-K: last CTA reduces
@@ -480,7 +444,6 @@ __global__ void __launch_bounds__(QTHREADS, QCfg<NP, BN, Q3>::MINB) gemm_q2_kern
       if (o + c4 < a.d_out) q2_store(a, item0 + n, o + c4, x0[c4], x1[c4], rsn);
   }
   if (threadIdx.x == 0) a.counters[unit] = 0;
-  Q2_CTA_TIME(1);
 }
 
 template <int NP, int BN, bool Q3>

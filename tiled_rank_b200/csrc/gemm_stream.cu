@@ -21,23 +21,6 @@
 
 namespace tileq {
 
-#ifdef TILEQ_TRACE
-// Debug builds only: clock64 time stamps of pipeline events of CTA 0, kept
-// separately for one- and two-projection launches.
-__device__ unsigned long long g_st_trace[2][6][1024];
-#define ST_TRACE(kind, idx) \
-  do {                      \
-    if (blockIdx.x == 0 && blockIdx.y == 0 && (idx) < 1024) g_st_trace[NP - 1][kind][idx] = clock64(); \
-  } while (0)
-extern "C" int tileq_debug_st_trace(unsigned long long *host) {
-  return (int)cudaMemcpyFromSymbol(host, g_st_trace, sizeof(g_st_trace));
-}
-#else
-#define ST_TRACE(kind, idx) \
-  do {                      \
-  } while (0)
-#endif
-
 namespace {
 
 constexpr int W = 8;                     // consumer warps
@@ -183,7 +166,6 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
       }
-      if (lane == 0) ST_TRACE(0, it);
       const int kb = kb0 + it;
       const int kvalid = min(BK, P.d_in - kb * BK);
       const uint32_t bytes = (uint32_t)C::A_BYTES + (P.tma_b ? 2u * C::BOX : (uint32_t)nitems * kvalid * 2);
@@ -269,16 +251,13 @@ __global__ void __launch_bounds__(THREADS) gemm_stream_kernel(const __grid_const
 
     for (int it = 0; it < nst; ++it) {
       const int s = it % C::STAGES;
-      if (lane == 0 && (warp == 0 || warp == 7)) ST_TRACE(warp == 0 ? 1 : 3, it);
       if (!mbar_wait(&full[s], (it / C::STAGES) & 1, P.status)) break;
-      if (lane == 0 && warp == 0) ST_TRACE(2, it);
       const int kvalid = min(BK, P.d_in - (kb0 + it) * BK);
       if (kvalid == BK)
         stage(s, kvalid, std::true_type{});
       else
         stage(s, kvalid, std::false_type{});
       __syncwarp();
-      if (lane == 0 && warp == 0) ST_TRACE(4, it);
       if (lane == 0) mbar_arrive(&empty[s]);
     }
 

@@ -27,27 +27,10 @@
 
 namespace tileq {
 
-#ifdef TILEQ_TRACE
-// Debug builds only: clock64 time stamps of pipeline events of CTA 0, kept
-// separately for one- and two-projection launches.
-__device__ unsigned long long g_tc_trace[2][8][2048];
-#define TC_TRACE(kind, idx) \
-  do {                      \
-    if (blockIdx.x == 0 && (idx) < 2048) g_tc_trace[NP - 1][kind][idx] = clock64(); \
-  } while (0)
-#else
-#define TC_TRACE(kind, idx) \
-  do {                      \
-  } while (0)
-#endif
-
 namespace {
 
 constexpr int BK = 128;  // K per stage
-#ifndef TILEQ_TC_DQW128
-#define TILEQ_TC_DQW128 16
-#endif
-constexpr int kDqw128 = TILEQ_TC_DQW128;  // dequantising warps of the 128-item tiles
+constexpr int kDqw128 = 16;  // dequantising warps of the 128-item tiles
 
 template <int NP, int BN, int DQW, bool Q3 = false>
 struct TcCfg {
@@ -231,9 +214,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
                       bool leader) -> bool {
     constexpr int COLS = decltype(cols_c)::value;
     constexpr int CH = COLS >= 8 ? 8 : 4;  // columns per TMEM load
-    if (leader) TC_TRACE(7, 2 * wi);
     if (!mbar_wait(&acc_full[ab], (wi / C::NACC) & 1, P.status)) return false;
-    if (leader) TC_TRACE(7, 2 * wi + 1);
     tc::fence_after();
     const int o = ob * 128 + row;
     const int ldp = P.m_tiles * 128;
@@ -321,9 +302,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
                              uint32_t lane_addr, bool leader) -> bool {
     constexpr int COLS = BN / 2, EB = C::EBATCH < COLS ? C::EBATCH : COLS;
     static_assert(EB % 8 == 0, "TMEM loads of 8 columns");
-    if (leader) TC_TRACE(7, 2 * wi);
     if (!mbar_wait(&acc_full[ab], (wi / C::NACC) & 1, P.status)) return false;
-    if (leader) TC_TRACE(7, 2 * wi + 1);
     tc::fence_after();
     const bool issuer = (warp & 3) == 0;  // the half's warp of lane quadrant 0 issues the copies
     const int rows = min(128, P.d_out - ob * 128);
@@ -372,9 +351,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
     } else {
     constexpr int COLS = BN / 4, EB = 8;
     static_assert(COLS % EB == 0, "column quarter in batches of 8");
-    if (leader) TC_TRACE(7, 2 * wi);
     if (!mbar_wait(&acc_full[0], wi & 1, P.status)) return false;
-    if (leader) TC_TRACE(7, 2 * wi + 1);
     tc::fence_after();
     const bool issuer = (warp & 3) == 2;  // dequantising warps 2, 6, 10, 14: lane quadrant 2
     const int rows = min(128, P.d_out - ob * 128);
@@ -431,7 +408,6 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
         for (int st = 0; st < nmain + next; ++st, ++qi) {
           const int s = qi % C::SQ;
           if (qi >= (uint32_t)C::SQ && !(ok = mbar_wait(&q_empty[s], ((qi / C::SQ) - 1) & 1, P.status))) break;
-          TC_TRACE(0, qi);
           if (st < nmain) {
             const int kb = kb0 + st;
             mbar_arrive_expect_tx(&q_full[s], NP * (128 * 32 + gps * 512) + C::HI + 2 * C::BATOM);
@@ -478,7 +454,6 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
         for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
           const int s = qi % C::SQ, sa = ai % C::SA;
           if (!(ok = mbar_wait(&a_full[sa], (ai / C::SA) & 1, P.status))) break;
-          if (lane == 0) TC_TRACE(4, qi);
           if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
           tc::fence_after();
           const bool ext = st >= nmain;
@@ -505,7 +480,6 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
                 tc::mma_ts(d, a + kk * 8, bd0 + (uint64_t)(((kk / 4) * C::BATOM + (kk % 4) * 32) >> 4), idesc,
                            (first && kk == 0) ? 0u : 1u);
             }
-            TC_TRACE(5, qi);
             tc::commit(&a_empty[sa]);
             tc::commit(&q_empty[s]);
           }
@@ -549,7 +523,6 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
       for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
         const int s = qi % C::SQ, sa = ai % C::SA;
         if (!(ok = mbar_wait(&q_full[s], (qi / C::SQ) & 1, P.status))) break;
-        if (dw == 0 && lane == 0) TC_TRACE(1, qi);
         const bool ext = st >= nmain;
         const int pe = ext ? (st - nmain) / n_ext1 : 0;  // the projection of an extension stage
         // decode into registers first: this overlaps the wait for a free A stage
@@ -598,7 +571,6 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
         __syncwarp();
         if (lane == 0) mbar_arrive(&q_empty[s]);
         if (ai >= (uint32_t)C::SA && !(ok = mbar_wait(&a_empty[sa], ((ai / C::SA) - 1) & 1, P.status))) break;
-        if (dw == 0 && lane == 0) TC_TRACE(2, qi);
         tc::fence_after();
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
@@ -608,9 +580,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
 #pragma unroll
           for (int c = 0; c < C::KPW / 32; ++c) tc::st16(acol + c * 16, vv[p][c]);
         }
-        if (dw == 0 && lane == 0) TC_TRACE(3, qi);
         tc::wait_st();
-        if (dw == 0 && lane == 0) TC_TRACE(6, qi);
         tc::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[sa]);
@@ -701,11 +671,6 @@ cudaError_t launch_tc_bn(const TcArgs &a, int bn, int grid, cudaStream_t s) {
 
 }  // namespace
 
-#ifdef TILEQ_TRACE
-extern "C" int tileq_debug_tc_trace(unsigned long long *host) {
-  return (int)cudaMemcpyFromSymbol(host, g_tc_trace, sizeof(g_tc_trace));
-}
-#endif
 
 int tc_smem_bytes(int np, int bn) {
   if (np == 1) {

@@ -51,8 +51,12 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
   const int t = warp;
   const float NEG = -INFINITY;
   const float *lg = a.logits + (size_t)t * a.K;
+  // a NaN logit ranks as -inf: every comparison below is then a total order,
+  // so all lanes agree on the winners
   float v0 = lane < a.K ? lg[lane] : NEG;
   float v1 = lane + 32 < a.K ? lg[lane + 32] : NEG;
+  if (isnan(v0)) v0 = NEG;
+  if (isnan(v1)) v1 = NEG;
   bool used0 = lane >= a.K, used1 = lane + 32 >= a.K;
   float sel_v[kMaxTopK];
   int sel_i[kMaxTopK];
@@ -86,12 +90,14 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     sum = s;
   }
+  // every chosen logit -inf (or NaN): equal weights, the limit of equal logits
+  const bool none = sel_v[0] == NEG;
   if (lane == 0) {
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
       if (j < a.k) {
         a.topk_idx[t * a.k + j] = sel_i[j];
-        a.topk_w[t * a.k + j] = expf(sel_v[j] - sel_v[0]) / sum;
+        a.topk_w[t * a.k + j] = none ? 1.0f / (a.full_softmax ? a.K : a.k) : expf(sel_v[j] - sel_v[0]) / sum;
       }
     }
   }
