@@ -36,7 +36,7 @@ import synth  # noqa: E402
 
 L2_BYTES = 126 * 2**20
 DEFAULT_CONFIG = 4   # the largest single-GPU configuration: 64 experts on 8x8, 16384 tokens
-STAGES = ["route", "permute", "zproj", "gateup", "zdown", "rowacc", "residual", "shared", "combine"]
+STAGES = ["route", "permute", "zproj", "gateup", "zdown", "shared", "residual", "combine"]
 
 
 def aggregate(ms_local, world, T, steps, device="cpu"):

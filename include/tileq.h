@@ -39,6 +39,15 @@
  *   - Outputs are overwritten, never accumulated into.
  *   - Bounded device waits that give up write TILEQ_ERR_TIMEOUT into the
  *     workspace status word (read it with tileq_device_status).
+ *   - Numeric range.  The forward computes in fp16 operands with fp32
+ *     accumulation: x (bf16) is converted to fp16, and the projected vectors
+ *     z and z', and the SwiGLU activation h = w * silu(g) * u, are stored in
+ *     fp16.  fp16's finite range is |v| <= 65504 (normal down to 6.1e-5,
+ *     subnormal to 6.0e-8).  Any of these values outside the finite range
+ *     (including a NaN or infinite input) records TILEQ_ERR_RANGE in the
+ *     workspace status word; the output of that forward is then not valid.
+ *     Values below the normal range lose relative precision gradually, as
+ *     fp16 subnormals.  The output is bf16 (fp32 range).
  */
 #ifndef TILEQ_H_
 #define TILEQ_H_
@@ -59,7 +68,9 @@ typedef enum {
   TILEQ_ERR_UNSUPPORTED = -2,  /* shape outside the supported tiling (see tileq_proj)     */
   TILEQ_ERR_WORKSPACE = -3,    /* workspace or packed buffer smaller than the query says  */
   TILEQ_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed             */
-  TILEQ_ERR_TIMEOUT = -5       /* a bounded device wait gave up (device status word)      */
+  TILEQ_ERR_TIMEOUT = -5,      /* a bounded device wait gave up (device status word)      */
+  TILEQ_ERR_RANGE = -6         /* an fp16 internal value left fp16's finite range (device
+                                  status word): the output of that forward is not valid  */
 } tileq_status;
 
 enum { TILEQ_LINEAR = 0, TILEQ_SWIGLU = 1 };

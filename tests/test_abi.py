@@ -158,6 +158,7 @@ def test_forward_validation_before_launch(L):
     st = lib.tileq_route(fake, 4, 4, 2, ctypes.byref(r), fake, 1 << 20, None)
     assert st == L.TILEQ_ERR_INVALID_ARG                          # route outputs missing
     assert L.status_string(L.TILEQ_ERR_TIMEOUT) == "TILEQ_ERR_TIMEOUT"
+    assert L.status_string(L.TILEQ_ERR_RANGE) == "TILEQ_ERR_RANGE"
 
 
 def test_route_static_validation_before_launch(L):

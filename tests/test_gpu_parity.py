@@ -248,6 +248,66 @@ def test_unfused_path(torch_cuda, case):
     assert_parity(out_z, oracle.forward(zr, x, logits), f"unfused zero residual {case}")
 
 
+def _range_run(torch, layer, logits, x):
+    from tiled_rank_b200 import DeviceLayer, tileq_device_status
+    dl = DeviceLayer(layer, torch.device("cuda:0"))
+    lg, xt = device_inputs(logits, x, torch.device("cuda:0"))
+    out = dl.forward(xt, lg)
+    torch.cuda.synchronize()
+    return to_numpy(out), tileq_device_status(dl.workspace(x.shape[0]))
+
+
+def test_wide_dynamic_range(torch_cuda):
+    """Outlier channels at 1e3 and 4e3 and whole tokens scaled down to ~1e-3: every
+    fp16 intermediate stays in range, the status word stays clear and the output
+    matches the oracle."""
+    torch = torch_cuda
+    cfg = synth.tiny_config(K=8, M=2, N=4, d_model=512, d_ff=1024, rank=64, group=128, top_k=2)
+    layer = synth.make_layer(cfg, seed=21)
+    logits, x = synth.make_inputs(cfg, 48, seed=21)
+    xf = synth.bf16_bits_to_f32(x).copy()
+    xf[:, 7] *= 1.0e3
+    xf[::3, 300] = 4.0e3
+    xf[1::4] *= 1.0e-3
+    xb = synth.to_bf16_bits(xf)
+    out, status = _range_run(torch, layer, logits, xb)
+    assert status == 0
+    assert_parity(out, oracle.forward(layer, xb, logits), "wide dynamic range")
+
+
+def test_lowrank_only_unit_factors(torch_cuda):
+    """Low-rank term alone with unit-norm factors (no gain): outputs near 1e-4,
+    intermediates far below 1 (fp16 subnormals for the smallest z')."""
+    torch = torch_cuda
+    cfg = synth.tiny_config(K=8, M=2, N=4, d_model=1024, d_ff=2048, rank=64, group=128, top_k=2)
+    layer = zero_residual(synth.make_layer(cfg, seed=22))
+    logits, x = synth.make_inputs(cfg, 40, seed=22)
+    out, status = _range_run(torch, layer, logits, x)
+    assert status == 0
+    assert_parity(out, oracle.forward(layer, x, logits), "low-rank only, unit factors")
+
+
+@pytest.mark.parametrize("case", ["x_above_fp16", "h_above_fp16"])
+def test_range_error_reported(torch_cuda, case):
+    """Values that leave fp16's finite range are reported in the status word
+    (TILEQ_ERR_RANGE), never passed on silently: an input above 65504, or
+    outliers at 3e4 whose SwiGLU activations exceed it (checked on the oracle's h)."""
+    torch = torch_cuda
+    from tiled_rank_b200 import TILEQ_ERR_RANGE
+    cfg = synth.tiny_config(K=8, M=2, N=4, d_model=512, d_ff=1024, rank=64, group=128, top_k=2)
+    layer = synth.make_layer(cfg, seed=23)
+    logits, x = synth.make_inputs(cfg, 24, seed=23)
+    xf = synth.bf16_bits_to_f32(x).copy()
+    if case == "x_above_fp16":
+        xf[5, 17] = 1.0e5
+    else:
+        xf[:4, :8] = 3.0e4
+        _, h = oracle.forward(layer, synth.to_bf16_bits(xf), logits, return_h=True)
+        assert np.abs(h).max() > 1e5   # the true activations leave fp16's range
+    _, status = _range_run(torch, layer, logits, synth.to_bf16_bits(xf))
+    assert status == TILEQ_ERR_RANGE
+
+
 def test_empty_batch_and_status(torch_cuda):
     torch = torch_cuda
     from tiled_rank_b200 import DeviceLayer, tileq_device_status, tileq_selftest_bounded_wait

@@ -5,6 +5,7 @@ its thin ctypes binding plus a helper that keeps a layer's device tensors.
 """
 from ._lib import (  # noqa: F401
     TILEQ_LINEAR, TILEQ_SWIGLU, TILEQ_ROUTE_FULL_SOFTMAX, TILEQ_ROUTE_TOPK_SOFTMAX, TileQError,
+    TILEQ_ERR_TIMEOUT, TILEQ_ERR_RANGE,
     status_string, tileq_device_status,
     tileq_moe_forward, tileq_moe_forward_unfused, tileq_pack, tileq_pack_per_expert,
     tileq_packed_per_expert_size, tileq_packed_size, tileq_route, tileq_route_static,

@@ -20,6 +20,7 @@ TILEQ_ERR_UNSUPPORTED = -2
 TILEQ_ERR_WORKSPACE = -3
 TILEQ_ERR_CUDA = -4
 TILEQ_ERR_TIMEOUT = -5
+TILEQ_ERR_RANGE = -6
 TILEQ_LINEAR = 0
 TILEQ_SWIGLU = 1
 TILEQ_ROUTE_TOPK_SOFTMAX = 0

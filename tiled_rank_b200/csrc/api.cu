@@ -186,19 +186,34 @@ struct GemmPlan {
   bool q2 = false;       // residual GEMM on warp-level MMA (narrow tiles)
   bool partial = false;  // K splits store their own partials (EPI_PARTIAL_F32); no reduction scratch
   bool wide = false;     // items from the wide tile table (tiles of Plan::bn_wide)
+  bool dq = false;       // residual GEMM on the decode-regime tcgen05 kernel (gemm_dq.cu, stream-K)
+  bool row_pair = false; // one projection on the two-projection tcgen05 kernel, two row blocks per unit
   size_t part_floats() const {
+    if (dq) return (size_t)dq_grid() * 2 * np * bn * kRowsPerCta;
     if (partial) return 0;
     // q2: one [np][bn][128] fp32 partial per (split, tile slot, row block)
     if (q2) return ksplit > 1 ? (size_t)ksplit * slots * m_tiles * np * bn * kRowsPerCta : 0;
     return ksplit > 1 ? (size_t)ksplit * np * std::max(items, 1) * m_tiles * kRowsPerCta : 0;
   }
-  int counters(int nprob) const { return ksplit > 1 && !partial ? nprob * slots * m_tiles : 0; }
+  int counters(int nprob) const {
+    if (dq) return slots * m_tiles;  // one per (tile, row block) unit
+    return ksplit > 1 && !partial ? nprob * slots * m_tiles : 0;
+  }
 };
 
 int choose_bn(long long avg) {
   if (avg <= 8) return 8;
   if (avg <= 16) return 16;
   if (avg <= 32) return 32;
+  return 64;
+}
+
+// Items per tile of the decode-regime tcgen05 GEMM: wide enough that most
+// experts fit one tile (an expert spilling into a second tile streams its
+// weights twice).
+int choose_bn_dq(long long avg) {
+  if (avg <= 6) return 16;
+  if (avg <= 16) return 32;
   return 64;
 }
 
@@ -237,7 +252,11 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   // cycle than mma.sync, and the decode then dominates); wider ones on tcgen05.
   const long long avg = P / std::max(1, L->K);
   const bool use_tc = avg > 32;
-  pl.bn_main = use_tc ? choose_bn_tc(avg) : choose_bn(avg);
+  // narrow tiles on the decode-regime tcgen05 kernel where every projection
+  // has 2-bit codes in groups of a multiple of 128; otherwise warp-level MMA
+  bool dq_ok = !use_tc;
+  for (int p = 0; p < li.nproj; ++p) dq_ok = dq_ok && li.p[p].bits == 2 && li.p[p].group % 128 == 0;
+  pl.bn_main = use_tc ? choose_bn_tc(avg) : (dq_ok ? choose_bn_dq(avg) : choose_bn(avg));
   pl.slots_main = cdiv(P, pl.bn_main) + L->K;
   const long long est_main = std::min(L->K, P) + P / pl.bn_main;
   auto tc_plan = [&](int d_out, int d_in, int np) {
@@ -249,8 +268,9 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
     g.np = np;
     g.items = P;
     // tcgen05: persistent CTAs walk (tile, row block, split) items; warp MMA: one CTA each
-    g.q2 = !use_tc;
-    g.ksplit = choose_ksplit(est_main * g.m_tiles, d_in, use_tc ? 2 : kQ2PerSm);
+    g.q2 = !use_tc && !dq_ok;
+    g.dq = dq_ok;
+    g.ksplit = dq_ok ? 1 : choose_ksplit(est_main * g.m_tiles, d_in, use_tc ? 2 : kQ2PerSm);
     return g;
   };
   // One-projection tcgen05 GEMMs over a long K take 256-item tiles (N = 256:
@@ -266,14 +286,25 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
     g.slots = pl.slots_wide;
     g.ksplit = choose_ksplit(((long long)std::min(L->K, P) + P / 256) * g.m_tiles, d_in, 2);
   };
+  // A one-projection tcgen05 GEMM over a short K that is not widened runs as
+  // row pairs: two 128-row blocks of the projection share each activation
+  // tile (half the activation reads per FLOP) and each barrier round of the
+  // MMA warp covers twice the tensor work.
+  auto pair_rows = [&](GemmPlan &g, int d_out) {
+    if (!g.tc || g.wide || g.ksplit != 1 || pl.bn_main != 128 || d_out <= 128) return;
+    g.row_pair = true;
+    g.m_tiles = cdiv(d_out, 256);
+  };
   const ProjInfo &q0 = li.p[0];
   if (L->kind == TILEQ_LINEAR) {
     pl.linear = tc_plan(q0.d_out, q0.d_in, 1);
     widen(pl.linear, q0.d_in);
+    pair_rows(pl.linear, q0.d_out);
   } else {
     pl.gateup = tc_plan(L->d_ff, L->d_model, 2);
     pl.down = tc_plan(L->d_model, L->d_ff, 1);
     widen(pl.down, L->d_ff);
+    pair_rows(pl.down, L->d_model);
     if (li.p[2].rank > 0) {
       GemmPlan z;
       z.bn = pl.bn_main;
@@ -281,7 +312,9 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
       z.m_tiles = cdiv(li.p[2].rank, 128);
       z.items = P;
       z.ksplit = choose_ksplit(est_main * z.m_tiles, L->d_ff, 4, 16);
-      z.partial = true;
+      // K splits reduced by the last CTA of a tile, which writes z' in fp16
+      // straight into the K-extension columns of the down GEMM's activations
+      z.partial = false;
       if (use_tc) {  // wide tiles: the same product on tcgen05, no K split
         z.tc = true;
         z.ksplit = 1;
@@ -347,6 +380,7 @@ struct WsLayout {
   size_t zidx[2];
   size_t aidx;
   size_t x16, xext, hext, zc[2], zs, ybuf, hs, ys, g32, u32, zpe[2];
+  size_t tokcnt;
   int ld_x, ld_h;
   size_t total;
 };
@@ -396,8 +430,12 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool
   nc = std::max(nc, pl.linear.counters(1));
   nc = std::max(nc, pl.sh_gu.counters(1));
   nc = std::max(nc, pl.sh_down.counters(1));
-  w.n_counters = nc;
-  w.counters = take((size_t)nc * 4);
+  // + one arrival count per (token, output row block) for the combine fused
+  // into the decode-regime down GEMM
+  const int ntok = (pl.down.dq || pl.linear.dq) ? std::max(T, 1) * cdiv(li.d_y, 128) : 0;
+  w.n_counters = nc + ntok;
+  w.counters = take((size_t)(nc + ntok) * 4);
+  w.tokcnt = w.counters + (size_t)nc * 4;
   size_t pf = 2 * pl.zproj.part_floats();
   w.part_zstride = pl.zproj.part_floats();
   for (const GemmPlan *g : {&pl.gateup, &pl.zdown, &pl.down, &pl.linear, &pl.sh_gu, &pl.sh_down})
@@ -420,7 +458,6 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool
     // z for all tokens and columns, and z' per slot: fp32 partials, one per K split
     w.zc[0] = take((size_t)pl.zproj.ksplit * std::max(T, 1) * L->N * pad128(li.p[0].rank) * 4);
     w.zc[1] = take((size_t)pl.zproj.ksplit * std::max(T, 1) * L->N * pad128(li.p[1].rank) * 4);
-    w.zs = take((size_t)pl.zdown.ksplit * Pz * li.p[2].rank * 4);
     w.g32 = take(Pz * L->d_ff * 4);
     w.u32 = take(Pz * L->d_ff * 4);
   }
@@ -460,8 +497,8 @@ cudaEvent_t g_stage_events[16];
 int g_n_stage_events = 0;
 
 // Stage boundaries of one forward (see tileq_set_stage_events).
-enum Stage { ST_BEGIN = 0, ST_ROUTE, ST_PERMUTE, ST_ZPROJ, ST_GATEUP, ST_ZDOWN, ST_ROWACC,
-             ST_RESIDUAL, ST_SHARED, ST_COMBINE };
+enum Stage { ST_BEGIN = 0, ST_ROUTE, ST_PERMUTE, ST_ZPROJ, ST_GATEUP, ST_ZDOWN, ST_SHARED, ST_RESIDUAL,
+             ST_COMBINE };
 
 void mark(int stage, cudaStream_t stream) {
   if (stage < g_n_stage_events) cudaEventRecord(g_stage_events[stage], stream);
@@ -529,6 +566,7 @@ tileq_status tc_args(TcArgs *a, const GemmPlan &g, const LayerInfo &li, const Pa
   a->tiles = at<int4>(ws, g.wide ? w.tiles_wide : w.tiles_main);
   a->tile_count = at<int>(ws, w.tile_counts) + (g.wide ? 1 : 0);
   a->m_tiles = g.m_tiles;
+  a->m_rows = g.m_tiles;
   a->ksplit = g.ksplit;
   a->d_out = q.d_out;
   a->d_in = q.d_in;
@@ -643,10 +681,60 @@ struct Residual {
   void *out[2] = {nullptr, nullptr};
   int ldo = 0;
   const float *row_scale = nullptr;
+  // decode-regime kernel, one projection: fuse the weighted top-k combine
+  // (out_tok = bf16 layer output, yshared = the shared expert or null)
+  bool combine = false;
+  int top_k = 0;
+  const float *yshared = nullptr;
+  void *out_tok = nullptr;
 };
+
+tileq_status run_residual_dq(const Residual &r, const GemmPlan &g, const LayerInfo &li, const PackedLayout &pl,
+                             const void *packed, void *ws, const WsLayout &w, cudaStream_t stream) {
+  DqArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const ProjInfo &q = li.p[r.proj[0]];
+  if (!make_map(&a.bmap, r.b, w.plan.P, r.ldb, r.ldb, g.bn)) return TILEQ_ERR_CUDA;
+  a.tiles = at<int4>(ws, w.tiles_main);
+  a.tile_count = at<int>(ws, w.tile_counts);
+  a.m_tiles = g.m_tiles;
+  a.d_out = q.d_out;
+  a.d_in = q.d_in;
+  a.group = q.group;
+  a.rank = r.ext ? q.rank : 0;
+  for (int i = 0; i < r.np; ++i) {
+    const ProjInfo &qi = li.p[r.proj[i]];
+    a.codes[i] = at<uint32_t>(packed, pl.qw[r.proj[i]]);
+    a.sz[i] = at<uint32_t>(packed, pl.sz[r.proj[i]]);
+    if (r.ext) {
+      a.ext_col[i] = r.ext_col[i];
+      a.u[i] = at<__half>(packed, pl.uf[r.proj[i]]);
+      std::memcpy(a.u_blk[i], qi.m_of, kMaxExperts);
+    }
+  }
+  a.epi = r.epi;
+  a.out = r.out[0];
+  a.out2 = r.out[1];
+  a.ldo = r.ldo;
+  a.row_scale = r.row_scale;
+  a.part = at<float>(ws, w.part);
+  a.counters = at<int>(ws, w.counters);
+  a.status = at<int>(ws, w.status);
+  if (r.combine) {
+    a.combine = 1;
+    a.top_k = r.top_k;
+    a.slot_tok = at<int>(ws, w.slot_tok);
+    a.slot_of_pair = at<int>(ws, w.slot_of_pair);
+    a.yshared = r.yshared;
+    a.out_tok = static_cast<__nv_bfloat16 *>(r.out_tok);
+    a.tok_counters = at<int>(ws, w.tokcnt);
+  }
+  return launch_gemm_dq(a, r.np, g.bn, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
+}
 
 tileq_status run_residual(const Residual &r, const GemmPlan &g, const LayerInfo &li, const PackedLayout &pl,
                           const void *packed, void *ws, const WsLayout &w, cudaStream_t stream) {
+  if (g.dq) return run_residual_dq(r, g, li, pl, packed, ws, w, stream);
   TcArgs a;
   tileq_status st = tc_args(&a, g, li, pl, packed, r.proj[0], ws, w, r.b, r.ldb, r.ldb);
   if (st != TILEQ_OK) return st;
@@ -664,6 +752,18 @@ tileq_status run_residual(const Residual &r, const GemmPlan &g, const LayerInfo 
   a.out[1] = r.out[1];
   a.ldo = r.ldo;
   a.row_scale = r.row_scale;
+  if (g.row_pair) {
+    // both halves of the pair read projection r.proj[0]
+    a.row_pair = 1;
+    a.m_rows = cdiv(li.p[r.proj[0]].d_out, 128);
+    a.codes[1] = a.codes[0];
+    a.codes_hi_rows[1] = a.codes_hi_rows[0];
+    a.sz[1] = a.sz[0];
+    a.u[1] = a.u[0];
+    a.ext_col[1] = a.ext_col[0];
+    std::memcpy(a.u_blk[1], a.u_blk[0], kMaxExperts);
+    return tc_launch(a, 2, g, stream);
+  }
   if (g.tc) return tc_launch(a, r.np, g, stream);
   return launch_gemm_q2(a, r.np, g.bn, g.slots, stream) == cudaSuccess ? TILEQ_OK : TILEQ_ERR_CUDA;
 }
@@ -685,14 +785,10 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   ra.topk_w = at<float>(ws, w.topk_w);
   ra.zero = at<int>(ws, w.counters);
   ra.nzero = w.n_counters;
+  ra.status = at<int>(ws, w.status);
   mark(ST_BEGIN, stream);
-  // one warp per token for the top-k; enough blocks that the x conversion has
-  // at most four 16-byte chunks per thread
   const long long xchunks = x ? (long long)T * li.d_x / 8 : 0;
-  const unsigned rblocks = std::max(nblocks(T, 8), std::min(nblocks(xchunks, 256 * 4), (unsigned)(8 * kNumSMs)));
-  TQ_CUDA(launch_pdl(route_kernel, dim3(rblocks), dim3(256), 0, stream, ra));
-  TQ_LAUNCHED();
-  mark(ST_ROUTE, stream);
+  const int P = T * top_k;
 
   PermuteArgs pa;
   std::memset(&pa, 0, sizeof(pa));
@@ -724,15 +820,28 @@ tileq_status run_route_permute(const tileq_layer *L, const LayerInfo &li, const 
   if (row_proj >= 0) std::memcpy(pa.m_of_row, li.p[row_proj].m_of, kMaxExperts);
   pa.aidx = at<int>(ws, w.aidx);
   pa.pcounts = at<int>(ws, w.pcounts);
-  const int P = T * top_k;
-  if (P > kPermMultiMin) {
+  if (P <= kPermMultiMin) {
+    // one launch: CTA 0 routes and sorts, the others zero the counters and
+    // convert x (at most four 16-byte chunks per thread of 1024-thread CTAs)
+    const unsigned cblocks = std::min(std::max(nblocks(xchunks, 1024 * 4), nblocks(w.n_counters, 1024)),
+                                      (unsigned)(2 * kNumSMs));
+    TQ_CUDA(launch_pdl(route_permute_kernel, dim3(1 + cblocks), dim3(1024), 0, stream, ra, pa));
+    TQ_LAUNCHED();
+    mark(ST_ROUTE, stream);
+    mark(ST_PERMUTE, stream);
+    return TILEQ_OK;
+  }
+  // one warp per token for the top-k; enough blocks that the x conversion has
+  // at most four 16-byte chunks per thread
+  const unsigned rblocks = std::max(nblocks(T, 8), std::min(nblocks(xchunks, 256 * 4), (unsigned)(8 * kNumSMs)));
+  TQ_CUDA(launch_pdl(route_kernel, dim3(rblocks), dim3(256), 0, stream, ra));
+  TQ_LAUNCHED();
+  mark(ST_ROUTE, stream);
+  {
     const unsigned nc = (unsigned)cdiv(P, kPermChunk);
     TQ_CUDA(launch_pdl(permute_count_kernel, dim3(nc), dim3(kPermChunkThreads), 0, stream, pa));
     TQ_LAUNCHED();
     TQ_CUDA(launch_pdl(permute_scatter_kernel, dim3(nc), dim3(kPermChunkThreads), 0, stream, pa));
-    TQ_LAUNCHED();
-  } else {
-    TQ_CUDA(launch_pdl(permute_kernel, dim3(1), dim3(1024), 0, stream, pa));
     TQ_LAUNCHED();
   }
   mark(ST_PERMUTE, stream);
@@ -758,9 +867,10 @@ tileq_status copy_route_out(const tileq_layer *L, const WsLayout &w, void *ws, i
   return TILEQ_OK;
 }
 
-tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
-                                    const PackedLayout &pl, const WsLayout &w, const void *packed,
-                                    void *ws, int T, int top_k, void *out, cudaStream_t stream) {
+// The always-on shared expert (dense fp16 SwiGLU) into the fp32 buffer ys;
+// *yshared = ys, or null without a shared expert.
+tileq_status run_shared(const tileq_layer *L, const PackedLayout &pl, const WsLayout &w, const void *packed,
+                        void *ws, int T, const float **yshared_out, cudaStream_t stream) {
   const float *yshared = nullptr;
   if (L->shared_d_ff > 0 && w.plan.sh_gu.tc) {
     const int Fs = L->shared_d_ff, D = L->d_model;
@@ -826,6 +936,14 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
     yshared = at<float>(ws, w.ys);
   }
   mark(ST_SHARED, stream);
+  *yshared_out = yshared;
+  return TILEQ_OK;
+}
+
+// The weighted top-k combine / unpermute of the per-slot outputs (the slot
+// weights are already applied), plus the shared expert.
+tileq_status run_combine(const LayerInfo &li, const WsLayout &w, void *ws, int T, int top_k, const float *yshared,
+                         void *out, cudaStream_t stream) {
   CombineArgs ca;
   ca.T = T;
   ca.k = top_k;
@@ -836,7 +954,6 @@ tileq_status run_shared_and_combine(const tileq_layer *L, const LayerInfo &li,
   ca.out = static_cast<__nv_bfloat16 *>(out);
   if (launch_combine(ca, stream) != cudaSuccess) return TILEQ_ERR_CUDA;
   count_launches();
-  mark(ST_COMBINE, stream);
   return TILEQ_OK;
 }
 
@@ -870,6 +987,7 @@ LrAccArgs lracc_args(const ProjInfo &q, const WsLayout &w, void *ws, int top_k, 
   la.out = out;
   la.ld = ld;
   la.col = col;
+  la.status = at<int>(ws, w.status);
   return la;
 }
 
@@ -932,6 +1050,7 @@ const char *tileq_status_string(tileq_status s) {
     case TILEQ_ERR_WORKSPACE: return "TILEQ_ERR_WORKSPACE";
     case TILEQ_ERR_CUDA: return "TILEQ_ERR_CUDA";
     case TILEQ_ERR_TIMEOUT: return "TILEQ_ERR_TIMEOUT";
+    case TILEQ_ERR_RANGE: return "TILEQ_ERR_RANGE";
   }
   return "TILEQ_UNKNOWN_STATUS";
 }
@@ -1061,7 +1180,6 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       if ((st = run_zproj(layer, li, pl, packed, w, ws, 1, stream)) != TILEQ_OK) return st;
       mark(ST_ZPROJ, stream);
       mark(ST_GATEUP, stream);
-      mark(ST_ZDOWN, stream);
       // a_{t,m} = sum_j w_j z_{t,n_j} over the token's experts in grid row m -> columns d_in..
       LrAccArgs la = lracc_args(q, w, ws, top_k, xext, w.ld_x, q.d_in);
       la.zcol = at<float>(ws, w.zc[0]);
@@ -1071,12 +1189,13 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       la.zsplit = (long long)T * layer->N * pad128(q.rank);
       TQ_CUDA(launch_pdl(lr_accumulate_kernel, dim3(nblocks((long long)plan.P * 32, 256)), dim3(256), 0, stream, la));
       TQ_LAUNCHED();
+      mark(ST_ZDOWN, stream);
     } else {
       mark(ST_ZPROJ, stream);
       mark(ST_GATEUP, stream);
       mark(ST_ZDOWN, stream);
     }
-    mark(ST_ROWACC, stream);
+    mark(ST_SHARED, stream);
     Residual r;
     r.ext = q.rank > 0;
     r.ext_col[0] = q.d_in;
@@ -1084,14 +1203,18 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     r.ldb = w.ld_x;
     r.out[0] = at<float>(ws, w.ybuf);
     r.ldo = q.d_out;
+    r.combine = plan.linear.dq;
+    r.top_k = top_k;
+    r.out_tok = out;
     if ((st = run_residual(r, plan.linear, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     mark(ST_RESIDUAL, stream);
+    if (!r.combine && (st = run_combine(li, w, ws, T, top_k, nullptr, out, stream)) != TILEQ_OK) return st;
+    mark(ST_COMBINE, stream);
   } else {
     const ProjInfo &qg = li.p[0], &qd = li.p[2];
     const int zids[2] = {0, 1};
     const bool lr_gu = qg.rank > 0, lr_d = qd.rank > 0;
-    st = run_route_permute(layer, li, w, x, T, router_logits, top_k, ws, lr_gu ? 2 : 0, zids,
-                           lr_d ? 2 : -1, stream);
+    st = run_route_permute(layer, li, w, x, T, router_logits, top_k, ws, lr_gu ? 2 : 0, zids, -1, stream);
     if (st != TILEQ_OK) return st;
     const int D = layer->d_model, F = layer->d_ff;
     __half *hext = at<__half>(ws, w.hext);
@@ -1116,6 +1239,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       ga.T = T;
       ga.k = top_k;
       ga.slot_of_pair = at<int>(ws, w.slot_of_pair);
+      ga.status = at<int>(ws, w.status);
       const long long chunks = (long long)T * (D / 8) + (long long)plan.P * (lr_gu ? 2 * qg.rank / 8 : 0);
       TQ_CUDA(launch_pdl(gather_ext_kernel, dim3(gather_blocks(chunks)), dim3(256), 0, stream, ga));
       TQ_LAUNCHED();
@@ -1139,8 +1263,11 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     }
     mark(ST_GATEUP, stream);
     if (lr_d) {
-      // z'_slot = Sigma * (V_n^T h_slot), then the in-place accumulation
-      // a_{t,m} = sum of the token's z' over its experts in grid row m -> columns F..
+      // z'_slot = Sigma * (V_n^T h_slot) in fp16 into the K-extension columns
+      // F .. F + r of the slot's row of h: the down GEMM then adds U_m z'_slot
+      // per slot, and the combine's sum over the token's slots carries out the
+      // accumulation per grid row (TileQ paper, section 2.2, the in-place
+      // accumulation buffer), with the routing weight already inside h
       if (plan.zdown.tc) {
         TcF16 f;
         f.arow[0] = at<__half>(packed, pl.vr[2]);
@@ -1154,8 +1281,9 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
         f.b = hext;
         f.brows = plan.P;
         f.ldb = w.ld_h;
-        f.out[0] = at<float>(ws, w.zs);
-        f.ldo = qd.rank;
+        f.epi = EPI_STORE_F16;
+        f.out[0] = hext + F;
+        f.ldo = w.ld_h;
         f.col_scale[0] = layer->proj[2].Sigma;
         if ((st = tc_f16(f, plan.zdown, ws, w, stream)) != TILEQ_OK) return st;
       } else {
@@ -1171,39 +1299,36 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       std::memcpy(z.a_blk, qd.n_of, kMaxExperts);
       z.b = hext;
       z.ldb = w.ld_h;
-      z.epi = EPI_PARTIAL_F32;
+      z.epi = EPI_STORE_F16;
       z.col_scale = layer->proj[2].Sigma;
-      z.out[0] = at<float>(ws, w.zs);
-      z.ldo = qd.rank;
+      z.out[0] = hext + F;
+      z.ldo = w.ld_h;
       tma_b(z, plan.P, plan.zdown.bn);
       if ((st = gemm(b, 1, 1, plan.zdown, stream)) != TILEQ_OK) return st;
       }
       mark(ST_ZDOWN, stream);
-      LrAccArgs la = lracc_args(qd, w, ws, top_k, hext, w.ld_h, F);
-      la.zslot = at<float>(ws, w.zs);
-      la.zks = plan.zdown.ksplit;
-      la.zsplit = (long long)plan.P * qd.rank;
-      TQ_CUDA(launch_pdl(lr_accumulate_kernel, dim3(nblocks((long long)plan.P * 32, 256)), dim3(256), 0, stream, la));
-      TQ_LAUNCHED();
     } else {
       mark(ST_ZDOWN, stream);
     }
-    mark(ST_ROWACC, stream);
-    {
-      Residual r;
-      r.proj[0] = 2;
-      r.ext = lr_d;
-      r.ext_col[0] = F;
-      r.b = hext;
-      r.ldb = w.ld_h;
-      r.out[0] = at<float>(ws, w.ybuf);
-      r.ldo = D;
-      if ((st = run_residual(r, plan.down, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
-    }
+    const float *yshared = nullptr;
+    if ((st = run_shared(layer, pl, w, packed, ws, T, &yshared, stream)) != TILEQ_OK) return st;
+    Residual r;
+    r.proj[0] = 2;
+    r.ext = lr_d;
+    r.ext_col[0] = F;
+    r.b = hext;
+    r.ldb = w.ld_h;
+    r.out[0] = at<float>(ws, w.ybuf);
+    r.ldo = D;
+    r.combine = plan.down.dq;
+    r.top_k = top_k;
+    r.yshared = yshared;
+    r.out_tok = out;
+    if ((st = run_residual(r, plan.down, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     mark(ST_RESIDUAL, stream);
+    if (!r.combine && (st = run_combine(li, w, ws, T, top_k, yshared, out, stream)) != TILEQ_OK) return st;
+    mark(ST_COMBINE, stream);
   }
-  st = run_shared_and_combine(layer, li, pl, w, packed, ws, T, top_k, out, stream);
-  if (st != TILEQ_OK) return st;
   return copy_route_out(layer, w, ws, T, top_k, route, stream);
 }
 
@@ -1334,7 +1459,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
       st = per_expert_lr(1, projs, xext, w.ld_x, nullptr, outs, q.d_out);
       if (st != TILEQ_OK) return st;
     }
-    for (int sidx = ST_ZPROJ; sidx <= ST_RESIDUAL; ++sidx) mark(sidx, stream);
+    for (int sidx = ST_ZPROJ; sidx <= ST_ZDOWN; ++sidx) mark(sidx, stream);
   } else {
     const ProjInfo &qg = li.p[0], &qd = li.p[2];
     const int D = layer->d_model, F = layer->d_ff;
@@ -1351,6 +1476,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     ga.T = T;
     ga.k = top_k;
     ga.slot_of_pair = at<int>(ws, w.slot_of_pair);
+    ga.status = at<int>(ws, w.status);
     TQ_CUDA(launch_pdl(gather_ext_kernel, dim3(gather_blocks((long long)T * (D / 8))), dim3(256), 0, stream, ga));
     TQ_LAUNCHED();
     Residual r;
@@ -1371,7 +1497,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     }
     mark(ST_ZPROJ, stream);
     SwigluArgs sa{(long long)plan.P * F, F, w.ld_h, at<float>(ws, w.g32), at<float>(ws, w.u32),
-                  at<float>(ws, w.slot_w), hext};
+                  at<float>(ws, w.slot_w), hext, at<int>(ws, w.status)};
     TQ_CUDA(launch_pdl(swiglu_kernel, dim3(nblocks(sa.n, 256)), dim3(256), 0, stream, sa));
     TQ_LAUNCHED();
     mark(ST_GATEUP, stream);
@@ -1389,11 +1515,12 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
       if (st != TILEQ_OK) return st;
     }
     mark(ST_ZDOWN, stream);
-    mark(ST_ROWACC, stream);
-    mark(ST_RESIDUAL, stream);
   }
-  st = run_shared_and_combine(layer, li, pl, w, packed, ws, T, top_k, out, stream);
-  if (st != TILEQ_OK) return st;
+  const float *yshared = nullptr;
+  if ((st = run_shared(layer, pl, w, packed, ws, T, &yshared, stream)) != TILEQ_OK) return st;
+  mark(ST_RESIDUAL, stream);
+  if ((st = run_combine(li, w, ws, T, top_k, yshared, out, stream)) != TILEQ_OK) return st;
+  mark(ST_COMBINE, stream);
   return copy_route_out(layer, w, ws, T, top_k, route, stream);
 }
 

@@ -159,6 +159,17 @@ __device__ __forceinline__ void set_status(int *status, int code) {
 
 __device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
 
+// fp16 of an internal activation (x, z, z', h); a value outside fp16's finite
+// range, NaN included, records TILEQ_ERR_RANGE in the device status word.
+__device__ __forceinline__ __half half_checked(float v, int *status) {
+  if (!(fabsf(v) <= 65504.f)) set_status(status, TILEQ_ERR_RANGE);
+  return __float2half_rn(v);
+}
+__device__ __forceinline__ __half2 half2_checked(float a, float b, int *status) {
+  if (!(fmaxf(fabsf(a), fabsf(b)) <= 65504.f) || a != a || b != b) set_status(status, TILEQ_ERR_RANGE);
+  return __floats2half2_rn(a, b);
+}
+
 // ------------------------------------------------------------------ mbarrier / bulk copy
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count) : "memory");

@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(DenseCfg<MB, BN>::THREADS, 1)
           if (P.epi == EPI_SWIGLU_H) {
             if (o[0] < P.d_out) {
               const float rs = P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f;
-              reinterpret_cast<__half *>(P.out[0])[ib + o[0]] = __float2half_rn(silu_f(v[0][i]) * v[MB - 1][i] * rs);
+              reinterpret_cast<__half *>(P.out[0])[ib + o[0]] = half_checked(silu_f(v[0][i]) * v[MB - 1][i] * rs, P.status);
             }
             continue;
           }
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(DenseCfg<MB, BN>::THREADS, 1)
             if (o[j] >= P.d_out) continue;
             void *dst = P.out[P.pair ? j : 0];
             if (P.epi == EPI_STORE_F16)
-              reinterpret_cast<__half *>(dst)[ib + o[j]] = __float2half_rn(v[j][i] * cs[j]);
+              reinterpret_cast<__half *>(dst)[ib + o[j]] = half_checked(v[j][i] * cs[j], P.status);
             else
               reinterpret_cast<float *>(dst)[ib + o[j]] = v[j][i] * cs[j];
           }

@@ -56,10 +56,10 @@ __device__ __forceinline__ void q2_store(const TcArgs &a, int item, int o, float
   const size_t idx = (size_t)item * a.ldo + o;
   switch (a.epi) {
     case EPI_SWIGLU_H:
-      reinterpret_cast<__half *>(a.out[0])[idx] = __float2half_rn(silu_f(v0) * v1 * rs);
+      reinterpret_cast<__half *>(a.out[0])[idx] = half_checked(silu_f(v0) * v1 * rs, a.status);
       break;
     case EPI_STORE_F16:
-      reinterpret_cast<__half *>(a.out[0])[idx] = __float2half_rn(v0);
+      reinterpret_cast<__half *>(a.out[0])[idx] = half_checked(v0, a.status);
       break;
     case EPI_STORE_F32:
       reinterpret_cast<float *>(a.out[0])[idx] = v0;

@@ -56,10 +56,10 @@ __device__ __forceinline__ void epi_store(const GemmProblem &P, int item, int o,
       reinterpret_cast<float *>(P.out[0])[((size_t)split * P.part_items + item) * P.ldo + o] = v0 * cs;
       break;
     case EPI_SWIGLU_H:
-      reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(silu_f(v0) * v1 * rs);
+      reinterpret_cast<__half *>(P.out[0])[idx] = half_checked(silu_f(v0) * v1 * rs, P.status);
       break;
     case EPI_STORE_F16:
-      reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(v0 * cs);
+      reinterpret_cast<__half *>(P.out[0])[idx] = half_checked(v0 * cs, P.status);
       break;
     case EPI_STORE_F32:
       reinterpret_cast<float *>(P.out[0])[idx] = v0 * cs;

@@ -79,12 +79,12 @@ struct TcCfg {
 __device__ __forceinline__ void tc_epi_store(const TcArgs &P, int item, int o, float v0, float v1, float rs) {
   const size_t idx = (size_t)item * P.ldo + o;
   if (P.epi == EPI_SWIGLU_H) {
-    reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(silu_f(v0) * v1 * rs);
+    reinterpret_cast<__half *>(P.out[0])[idx] = half_checked(silu_f(v0) * v1 * rs, P.status);
   } else if (P.epi == EPI_STORE2_F32) {
     reinterpret_cast<float *>(P.out[0])[idx] = v0;
     reinterpret_cast<float *>(P.out[1])[idx] = v1;
   } else if (P.epi == EPI_STORE_F16) {
-    reinterpret_cast<__half *>(P.out[0])[idx] = __float2half_rn(v0);
+    reinterpret_cast<__half *>(P.out[0])[idx] = half_checked(v0, P.status);
   } else {
     reinterpret_cast<float *>(P.out[0])[idx] = v0;
   }
@@ -193,6 +193,10 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
   const int n_ext = NP * n_ext1;
   bool ok = true;
 
+  // the 128-row block of "projection" p of unit row index ob (row pairs: two
+  // row blocks of one projection; past the last block it repeats the last one,
+  // whose rows the epilogue then drops)
+  auto rb_of = [&](int ob, int p) { return P.row_pair ? min(2 * ob + p, P.m_rows - 1) : ob; };
   auto decode = [&](int w, int &jt, int &ob, int &split) {
     split = w % P.ksplit;
     w /= P.ksplit;
@@ -252,7 +256,13 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
         for (int i = 0; i < CH; ++i) {
           const int n = part * COLS + c0 + c + i;
           if (n >= nitems) continue;
-          if (P.ksplit == 1) {
+          if (P.row_pair) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+              const int op = (2 * ob + p) * 128 + row;
+              if (op < P.d_out) reinterpret_cast<float *>(P.out[0])[(size_t)(item0 + n) * P.ldo + op] = v[p][c + i];
+            }
+          } else if (P.ksplit == 1) {
             if (o < P.d_out) tc_epi_store(P, item0 + n, o, v[0][c + i], v[NP - 1][c + i], rs[i]);
           } else {
 #pragma unroll
@@ -381,7 +391,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
       named_sync(5 + part, 128);
 #pragma unroll
       for (int i = 0; i < EB; ++i)
-        buf[i * 128 + row] = __float2half_rn(no_k ? 0.f : silu_f(g[i]) * u[i] * rs[i]);
+        buf[i * 128 + row] = half_checked(no_k ? 0.f : silu_f(g[i]) * u[i] * rs[i], P.status);
       tc::fence_proxy_async_smem();
       named_sync(5 + part, 128);
       if (issuer) {
@@ -412,12 +422,12 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
             const int kb = kb0 + st;
             mbar_arrive_expect_tx(&q_full[s], NP * (128 * 32 + gps * 512) + C::HI + 2 * C::BATOM);
             for (int p = 0; p < NP; ++p) {
-              const size_t cblk = (((size_t)grp * P.m_tiles + ob) * nkb + kb) * (128 * 32);
+              const size_t cblk = (((size_t)grp * P.m_rows + rb_of(ob, p)) * nkb + kb) * (128 * 32);
               bulk_g2s(q_codes(s, p), reinterpret_cast<const uint8_t *>(P.codes[p]) + cblk, 128 * 32, &q_full[s]);
               if constexpr (Q3)
                 bulk_g2s(const_cast<uint32_t *>(q_hi(s, p)),
                          reinterpret_cast<const uint8_t *>(P.codes_hi_rows[p]) + cblk / 2, 128 * 16, &q_full[s]);
-              const size_t zoff = (((size_t)grp * P.m_tiles + ob) * G + (kb * BK) / g) * 128;
+              const size_t zoff = (((size_t)grp * P.m_rows + rb_of(ob, p)) * G + (kb * BK) / g) * 128;
               bulk_g2s(q_sz(s, p), P.sz[p] + zoff, gps * 512, &q_full[s]);
             }
             for (int a = 0; a < 2; ++a)
@@ -518,7 +528,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
 #pragma unroll
         for (int p = 0; p < NP; ++p)
           if (e * BK + part * C::KPW < P.rank)
-            prefetch_l2(P.u[p] + (((size_t)P.u_blk[p][grp] * P.m_tiles + ob) * 128 + row) * P.rank + e * BK +
+            prefetch_l2(P.u[p] + (((size_t)P.u_blk[p][grp] * P.m_rows + rb_of(ob, p)) * 128 + row) * P.rank + e * BK +
                         part * C::KPW);
       for (int st = 0; st < nmain + next; ++st, ++qi, ++ai) {
         const int s = qi % C::SQ, sa = ai % C::SA;
@@ -554,7 +564,7 @@ __global__ void __launch_bounds__(TcCfg<NP, BN, DQW, Q3>::THREADS, 1) gemm_tc_ke
               const int e = (st - nmain) % n_ext1;
               const int kg = e * BK + k0;          // column of U
               const int ub = P.u_blk[p][grp];
-              const __half *ur = P.u[p] + (((size_t)ub * P.m_tiles + ob) * 128 + row) * P.rank;
+              const __half *ur = P.u[p] + (((size_t)ub * P.m_rows + rb_of(ob, p)) * 128 + row) * P.rank;
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 uint4 q4 = make_uint4(0, 0, 0, 0);

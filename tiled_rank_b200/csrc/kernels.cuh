@@ -17,6 +17,7 @@ struct RouteArgs {
   float *topk_w;
   int *zero;               // split-K arrival counters, cleared for this forward
   int nzero;
+  int *status;             // device status word (TILEQ_ERR_RANGE)
 };
 
 struct PermuteArgs {
@@ -142,6 +143,11 @@ struct TcArgs {
   const int4 *tiles;
   const int *tile_count;
   int m_tiles, ksplit, d_out, d_in, group, rank;
+  // row_pair (two-projection kernel, ksplit 1, fp32 stores): the two
+  // "projections" are row blocks 2 ob and 2 ob + 1 of one projection, which
+  // share each activation tile; m_tiles counts row-block pairs and m_rows the
+  // 128-row blocks of the packed layout (m_rows == m_tiles otherwise)
+  int row_pair, m_rows;
   int n_experts;             // experts (blocks) in codes / sz
   int ext_col[2];            // first B column of the K extension of projection p
   const uint4 *codes[2];     // tcgen05: [K][d_out/128][d_in/128][4 slices][128 rows][8 B]
@@ -164,6 +170,49 @@ struct TcArgs {
 };
 
 cudaError_t launch_gemm_tc(const TcArgs &a, int np, int bn, int grid, cudaStream_t stream);
+
+// Residual GEMM of the decode regime on tcgen05 (gemm_dq.cu): narrow item
+// tiles (16, 32 or 64 items), the exact q - z of each 2-bit code in fp16 as
+// the A operand in tensor memory, one fp32 accumulator per 128-wide K block
+// (scale group) folded into registers with its scale, and stream-K work
+// division: the (tile, row block, round) space is cut into gridDim.x equal
+// ranges; a (tile, row block) unit split between CTAs is summed, in CTA
+// order, by the CTA that finishes it last.  Groups are multiples of 128.
+// A round covers two slices: gate and up of one 128-wide K block (np = 2) or
+// two consecutive K blocks of one projection (np = 1); the low-rank K
+// extension follows the residual rounds of each unit.
+struct DqArgs {
+  alignas(64) CUtensorMap bmap;  // B: fp16 activation rows [items][ldb], box 64 x bn, 128-byte swizzle
+  const int4 *tiles;             // (expert, first item, items)
+  const int *tile_count;
+  int m_tiles, d_out, d_in, group, rank;
+  int ext_col[2];                // first B column of projection p's K extension
+  const uint32_t *codes[2];      // tcgen05 row layout of the codes (qw)
+  const uint32_t *sz[2];         // [K][d_out/128][G][128 rows] {fp16 scale, fp16 zero}
+  const __half *u[2];            // [M][pad128(d_out)][rank] fp16
+  int8_t u_blk[2][kMaxExperts];
+  int epi;                       // np = 2: EPI_SWIGLU_H (fp16 h) or EPI_STORE2_F32 (gate, up in fp32);
+                                 // np = 1: EPI_STORE_F32
+  void *out;
+  void *out2;                    // EPI_STORE2_F32: the up projection
+  int ldo;
+  const float *row_scale;        // per item (SwiGLU h)
+  float *part;                   // split units: [gridDim.x][2][np][bn][128] fp32
+  int *counters;                 // one zeroed arrival count per (tile, row block)
+  int *status;
+  // np = 1 with combine: out is the fp32 per-slot buffer [items][ldo]; the
+  // last of a token's top_k slots to finish a row block writes
+  // out_tok[t][o] = bf16(sum over the token's slots in slot order (+ yshared[t][o]))
+  int combine;
+  int top_k;
+  const int *slot_tok;           // [items] token of each slot
+  const int *slot_of_pair;       // [T * top_k]
+  const float *yshared;          // [T][ldo] or null
+  __nv_bfloat16 *out_tok;        // [T][ldo]
+  int *tok_counters;             // [T][m_tiles], zeroed
+};
+cudaError_t launch_gemm_dq(const DqArgs &a, int np, int bn, cudaStream_t stream);
+int dq_grid();
 
 // Dense fp16 GEMM on tcgen05 with both operands read by TMA (gemm_dense.cu).
 // A: fp16 row-major, tensor maps amap[j] (box 64 x 128, 128-byte swizzle);
@@ -224,6 +273,7 @@ struct GatherExtArgs {
   const float *z[2];
   const int *zidx[2];
   __half *out;
+  int *status;
 };
 
 // Row accumulation, written per slot into the K-extension columns of the
@@ -248,6 +298,7 @@ struct LrAccArgs {
   long long zsplit;
   __half *out;             // [P][ld], columns col .. col+r-1
   int ld, col;
+  int *status;
 };
 
 struct CombineArgs {
@@ -272,10 +323,11 @@ struct SwigluArgs {
   const float *g, *u;
   const float *slot_w;
   __half *h;               // [P][ldh]
+  int *status;
 };
 
 __global__ void route_kernel(RouteArgs a);
-__global__ void permute_kernel(PermuteArgs a);
+__global__ void route_permute_kernel(RouteArgs ra, PermuteArgs a);
 __global__ void permute_count_kernel(PermuteArgs a);
 __global__ void permute_scatter_kernel(PermuteArgs a);
 __global__ void lr_accumulate_kernel(LrAccArgs a);

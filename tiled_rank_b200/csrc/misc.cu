@@ -77,8 +77,8 @@ __global__ void __launch_bounds__(256) lr_accumulate_kernel(LrAccArgs a) {
         acc.x += f * z[j].x; acc.y += f * z[j].y; acc.z += f * z[j].z; acc.w += f * z[j].w;
       }
     }
-    dst[2 * c] = __floats2half2_rn(acc.x, acc.y);
-    dst[2 * c + 1] = __floats2half2_rn(acc.z, acc.w);
+    dst[2 * c] = half2_checked(acc.x, acc.y, a.status);
+    dst[2 * c + 1] = half2_checked(acc.z, acc.w, a.status);
   }
 }
 
@@ -106,10 +106,10 @@ __device__ __forceinline__ uint4 z_chunk(const GatherExtArgs &a, int s, int zc) 
   }
   uint4 v;
   __half2 *o = reinterpret_cast<__half2 *>(&v);
-  o[0] = __floats2half2_rn(lo.x, lo.y);
-  o[1] = __floats2half2_rn(lo.z, lo.w);
-  o[2] = __floats2half2_rn(hi.x, hi.y);
-  o[3] = __floats2half2_rn(hi.z, hi.w);
+  o[0] = half2_checked(lo.x, lo.y, a.status);
+  o[1] = half2_checked(lo.z, lo.w, a.status);
+  o[2] = half2_checked(hi.x, hi.y, a.status);
+  o[3] = half2_checked(hi.z, hi.w, a.status);
   return v;
 }
 
@@ -217,7 +217,7 @@ __global__ void swiglu_kernel(SwigluArgs a) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.n) return;
   const int slot = (int)(i / a.F), f = (int)(i % a.F);
-  a.h[(size_t)slot * a.ldh + f] = __float2half_rn(a.slot_w[slot] * silu_f(a.g[i]) * a.u[i]);
+  a.h[(size_t)slot * a.ldh + f] = half_checked(a.slot_w[slot] * silu_f(a.g[i]) * a.u[i], a.status);
 }
 
 // Bounded wait on an mbarrier that nothing arrives on: gives up after

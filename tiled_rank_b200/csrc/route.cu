@@ -4,51 +4,53 @@
 //                   equal logits -> lower expert id), softmax over the chosen
 //                   logits (or, full_softmax, their entries of the softmax over
 //                   all K logits), and the bf16 -> fp16 conversion of x.
-// permute_kernel  : one CTA: deterministic stable counting sort of the
-//                   (token, slot) pairs by expert and the GEMM tile table; per
-//                   slot, the row of the projected [T, N, r] tensor it reads
-//                   (TileQ paper, section 2.2) and whether it is the token's
-//                   first slot in its grid row (the in-place accumulation).
+// route_permute_kernel: up to 4096 pairs, routing and, in CTA 0, the
+//                   deterministic stable counting sort of the (token, slot)
+//                   pairs by expert and the GEMM tile tables; per slot, the
+//                   row of the projected [T, N, r] tensor it reads (TileQ
+//                   paper, section 2.2) and, for the linear layer, whether it
+//                   is the token's first slot in its grid row (the in-place
+//                   accumulation).
 // permute_count_kernel + permute_scatter_kernel: the same sort and tables for
 //                   long batches, one CTA per 1024 pairs.
 #include "kernels.cuh"
 
 namespace tileq {
 
-__global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
-  pdl_wait_and_release();
-  const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long gthreads = (long long)gridDim.x * blockDim.x;
-  const int warp = (int)(gtid >> 5);
-  const int lane = threadIdx.x & 31;
-  for (long long i = gtid; i < a.nzero; i += gthreads) a.zero[i] = 0;
-  // bf16 -> fp16 copy of x: every thread of the grid, four 16-byte chunks in flight
-  if (a.x != nullptr) {
-    const long long nchunk = (long long)a.T * (a.d_x / 8);
-    const uint4 *src = reinterpret_cast<const uint4 *>(a.x);
-    uint4 *dst = reinterpret_cast<uint4 *>(a.x16);
-    for (long long c0 = gtid; c0 < nchunk; c0 += 4 * gthreads) {
-      uint4 v[4];
+// Zero the split-K arrival counters and copy x from bf16 to fp16; thread tid
+// of nthreads, four 16-byte chunks in flight per thread.
+__device__ __forceinline__ void zero_and_convert(const RouteArgs &a, long long tid, long long nthreads) {
+  for (long long i = tid; i < a.nzero; i += nthreads) a.zero[i] = 0;
+  if (a.x == nullptr) return;
+  const long long nchunk = (long long)a.T * (a.d_x / 8);
+  const uint4 *src = reinterpret_cast<const uint4 *>(a.x);
+  uint4 *dst = reinterpret_cast<uint4 *>(a.x16);
+  for (long long c0 = tid; c0 < nchunk; c0 += 4 * nthreads) {
+    uint4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const long long c = c0 + u * gthreads;
-        if (c < nchunk) v[u] = src[c];
+    for (int u = 0; u < 4; ++u) {
+      const long long c = c0 + u * nthreads;
+      if (c < nchunk) v[u] = src[c];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long c = c0 + u * nthreads;
+      if (c >= nchunk) continue;
+      const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
+      uint4 o;
+      __half2 *h = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(b[i]);
+        h[i] = half2_checked(f.x, f.y, a.status);
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const long long c = c0 + u * gthreads;
-        if (c >= nchunk) continue;
-        const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
-        uint4 o;
-        __half2 *h = reinterpret_cast<__half2 *>(&o);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) h[i] = __float22half2_rn(__bfloat1622float2(b[i]));
-        dst[c] = o;
-      }
+      dst[c] = o;
     }
   }
-  if (warp >= a.T) return;
-  const int t = warp;
+}
+
+// Top-k and weights of token t by one warp.
+__device__ __forceinline__ void route_token(const RouteArgs &a, int t, int lane) {
   const float NEG = -INFINITY;
   const float *lg = a.logits + (size_t)t * a.K;
   // a NaN logit ranks as -inf: every comparison below is then a total order,
@@ -101,6 +103,14 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
       }
     }
   }
+}
+
+__global__ void __launch_bounds__(256) route_kernel(RouteArgs a) {
+  pdl_wait_and_release();
+  const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  zero_and_convert(a, gtid, (long long)gridDim.x * blockDim.x);
+  const int warp = (int)(gtid >> 5);
+  if (warp < a.T) route_token(a, warp, threadIdx.x & 31);
 }
 
 // ---------------------------------------------------------------------------
@@ -228,18 +238,27 @@ __device__ __forceinline__ void write_slot(const PermuteArgs &a, int p, int slot
   }
 }
 
-__global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteArgs a) {
+// Routing and the one-CTA permutation in one launch (batches of at most
+// kPermMultiMin pairs): CTA 0 routes every token (one warp per token) and
+// sorts the pairs; the other CTAs zero the counters and convert x.  The top-k
+// results CTA 0 writes are visible to its own threads after the barrier.
+__global__ void __launch_bounds__(kPermThreads) route_permute_kernel(RouteArgs ra, PermuteArgs a) {
   pdl_wait_and_release();
+  if (blockIdx.x != 0 || gridDim.x == 1)
+    zero_and_convert(ra, (long long)(blockIdx.x - (gridDim.x > 1)) * blockDim.x + threadIdx.x,
+                     (long long)(gridDim.x - (gridDim.x > 1)) * blockDim.x);
+  if (blockIdx.x != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = warp; t < ra.T; t += kPermWarps) route_token(ra, t, lane);
+  __syncthreads();
   __shared__ SortSmem s;
   __shared__ int scratch[kMaxExperts + 1];
   const int P = a.T * a.k;
   const int32_t *idx = a.topk_idx;
-
   cta_stable_sort(P, a.K, [&](int p) { return idx[p]; }, a.dest, a.expert_offsets, s);
   for (int p = threadIdx.x; p < P; p += blockDim.x) write_slot(a, p, a.dest[p]);
   __syncthreads();
-  build_tiles(a.expert_offsets, a.K, a.bn, a.tiles_main, a.tile_counts + 0, a.tile_first_main,
-              scratch);
+  build_tiles(a.expert_offsets, a.K, a.bn, a.tiles_main, a.tile_counts + 0, a.tile_first_main, scratch);
   if (a.bn_wide > 0)
     build_tiles(a.expert_offsets, a.K, a.bn_wide, a.tiles_wide, a.tile_counts + 1, nullptr, scratch);
 }
