@@ -161,8 +161,12 @@ PackedLayout packed_layout(const tileq_layer *L, const LayerInfo &li) {
   return pl;
 }
 
+// Per-expert factors of the unfused comparison path: warp-MMA fragment order
+// (uf, vf) for short batches and row-major fp16 (ur = U_pe rows
+// [K][pad128(d_out)][rank], vr = V_pe^T rows [K][pad128(rank)][d_in]) for the
+// dense tcgen05 kernel on long ones, the same split as the fused path.
 struct PePackedLayout {
-  size_t uf[3], vf[3], total;
+  size_t uf[3], vf[3], ur[3], vr[3], total;
 };
 
 PePackedLayout pe_layout(const tileq_layer *L, const LayerInfo &li) {
@@ -174,6 +178,10 @@ PePackedLayout pe_layout(const tileq_layer *L, const LayerInfo &li) {
     if (q.rank > 0) off += align_up(frag_bytes(L->K, q.d_out, q.rank, 8));
     pl.vf[p] = off;
     if (q.rank > 0) off += align_up(frag_bytes(L->K, q.rank, q.d_in, 8));
+    pl.ur[p] = off;
+    if (q.rank > 0) off += align_up((size_t)L->K * pad128(q.d_out) * q.rank * 2);
+    pl.vr[p] = off;
+    if (q.rank > 0) off += align_up((size_t)L->K * pad128(q.rank) * q.d_in * 2);
   }
   pl.total = off;
   return pl;
@@ -238,7 +246,11 @@ struct Plan {
   int T, k, P;
   int bn_main, slots_main;
   int bn_wide = 0, slots_wide = 0;  // second tile table (one-projection tcgen05 GEMMs over long K)
-  GemmPlan zproj, gateup, zdown, down, linear, sh_gu, sh_down, pe;
+  GemmPlan zproj, gateup, zdown, down, linear, sh_gu, sh_down;
+  // unfused comparison path: the per-expert z products (gate/up or linear, and
+  // down) and the U-side products, grouped over all experts' tiles like the
+  // fused path's own projections (split-K below 256 tokens, tcgen05 above)
+  GemmPlan pe_zx, pe_zd, pe_u;
 };
 
 Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
@@ -363,10 +375,21 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
       }
     }
   }
-  // unfused per-expert launches: one expert per launch, grid sized for T slots, no split
-  pl.pe.bn = pl.bn_main;
-  pl.pe.slots = cdiv(T, pl.bn_main);
-  pl.pe.items = P;
+  auto pe_plan = [&](int rank, int d_in, int np) {
+    GemmPlan g;
+    g.bn = pl.bn_main;
+    g.slots = pl.slots_main;
+    g.items = P;
+    g.np = np;
+    g.m_tiles = std::max(1, cdiv(rank, 128));
+    g.tc = T >= kTcMinTokens;
+    g.ksplit = g.tc ? 1 : choose_ksplit(est_main * g.m_tiles * np, d_in, 4, 16);
+    return g;
+  };
+  pl.pe_zx = pe_plan(q0.rank, q0.d_in, L->kind == TILEQ_SWIGLU ? 2 : 1);
+  if (L->kind == TILEQ_SWIGLU) pl.pe_zd = pe_plan(li.p[2].rank, L->d_ff, 1);
+  pl.pe_u = pe_plan(0, 128, 1);
+  pl.pe_u.ksplit = 1;
   return pl;
 }
 
@@ -381,6 +404,7 @@ struct WsLayout {
   size_t aidx;
   size_t x16, xext, hext, zc[2], zs, ybuf, hs, ys, g32, u32, zpe[2];
   size_t tokcnt;
+  size_t x8, xs;
   int ld_x, ld_h;
   size_t total;
 };
@@ -430,6 +454,8 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool
   nc = std::max(nc, pl.linear.counters(1));
   nc = std::max(nc, pl.sh_gu.counters(1));
   nc = std::max(nc, pl.sh_down.counters(1));
+  nc = std::max(nc, pl.pe_zx.counters(pl.pe_zx.np));
+  nc = std::max(nc, pl.pe_zd.counters(1));
   // + one arrival count per (token, output row block) for the combine fused
   // into the decode-regime down GEMM
   const int ntok = (pl.down.dq || pl.linear.dq) ? std::max(T, 1) * cdiv(li.d_y, 128) : 0;
@@ -438,7 +464,8 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool
   w.tokcnt = w.counters + (size_t)nc * 4;
   size_t pf = 2 * pl.zproj.part_floats();
   w.part_zstride = pl.zproj.part_floats();
-  for (const GemmPlan *g : {&pl.gateup, &pl.zdown, &pl.down, &pl.linear, &pl.sh_gu, &pl.sh_down})
+  for (const GemmPlan *g : {&pl.gateup, &pl.zdown, &pl.down, &pl.linear, &pl.sh_gu, &pl.sh_down, &pl.pe_zx,
+                            &pl.pe_zd})
     pf = std::max(pf, g->part_floats());
   w.part = take(pf * 4);
   for (int z = 0; z < 2; ++z) w.zidx[z] = take(Pz * 4);
@@ -455,6 +482,10 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool
     w.ld_h = L->d_ff + li.p[2].rank;
     w.xext = take(Pz * w.ld_x * 2);
     w.hext = take(Pz * w.ld_h * 2);
+    if (pl.gateup.dq) {  // e4m3 pieces of x per slot and the per-slot scales
+      w.x8 = take(Pz * 2 * L->d_model);
+      w.xs = take(Pz * 4);
+    }
     // z for all tokens and columns, and z' per slot: fp32 partials, one per K split
     w.zc[0] = take((size_t)pl.zproj.ksplit * std::max(T, 1) * L->N * pad128(li.p[0].rank) * 4);
     w.zc[1] = take((size_t)pl.zproj.ksplit * std::max(T, 1) * L->N * pad128(li.p[1].rank) * 4);
@@ -541,6 +572,27 @@ bool make_map(CUtensorMap *m, const void *base, int rows, int cols, int ld, int 
   const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D tensor map over a byte matrix [rows][cols] (row stride cols bytes, a
+// multiple of 16), box 128 x box_rows, 128-byte swizzle, zero fill outside.
+bool make_map_u8(CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)std::max(rows, 1)};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols};
+  const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -684,6 +736,9 @@ struct Residual {
   // decode-regime kernel, one projection: fuse the weighted top-k combine
   // (out_tok = bf16 layer output, yshared = the shared expert or null)
   bool combine = false;
+  // decode-regime kernel, gate/up: fp8 mode, B = the e4m3 pieces (ws.x8, per-item
+  // scales ws.xs), the extension columns from b
+  bool f8 = false;
   int top_k = 0;
   const float *yshared = nullptr;
   void *out_tok = nullptr;
@@ -694,7 +749,14 @@ tileq_status run_residual_dq(const Residual &r, const GemmPlan &g, const LayerIn
   DqArgs a;
   std::memset(&a, 0, sizeof(a));
   const ProjInfo &q = li.p[r.proj[0]];
-  if (!make_map(&a.bmap, r.b, w.plan.P, r.ldb, r.ldb, g.bn)) return TILEQ_ERR_CUDA;
+  if (r.f8) {
+    a.f8 = 1;
+    a.xs = at<float>(ws, w.xs);
+    if (!make_map_u8(&a.bmap, at<uint8_t>(ws, w.x8), w.plan.P, 2 * q.d_in, g.bn)) return TILEQ_ERR_CUDA;
+    if (!make_map(&a.bmap_ext, r.b, w.plan.P, r.ldb, r.ldb, g.bn)) return TILEQ_ERR_CUDA;
+  } else if (!make_map(&a.bmap, r.b, w.plan.P, r.ldb, r.ldb, g.bn)) {
+    return TILEQ_ERR_CUDA;
+  }
   a.tiles = at<int4>(ws, w.tiles_main);
   a.tile_count = at<int>(ws, w.tile_counts);
   a.m_tiles = g.m_tiles;
@@ -1240,9 +1302,35 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       ga.k = top_k;
       ga.slot_of_pair = at<int>(ws, w.slot_of_pair);
       ga.status = at<int>(ws, w.status);
-      const long long chunks = (long long)T * (D / 8) + (long long)plan.P * (lr_gu ? 2 * qg.rank / 8 : 0);
-      TQ_CUDA(launch_pdl(gather_ext_kernel, dim3(gather_blocks(chunks)), dim3(256), 0, stream, ga));
-      TQ_LAUNCHED();
+      if (plan.gateup.dq) {
+        // fp8 decode GEMM: e4m3 pieces of each slot's x (and its z columns, scaled alike)
+        GatherX8Args g8;
+        std::memset(&g8, 0, sizeof(g8));
+        g8.T = T;
+        g8.k = top_k;
+        g8.d = D;
+        g8.r = qg.rank;
+        g8.ld = w.ld_x;
+        g8.slot_of_pair = ga.slot_of_pair;
+        g8.x16 = ga.x16;
+        g8.x8 = at<uint8_t>(ws, w.x8);
+        g8.xs = at<float>(ws, w.xs);
+        g8.z[0] = ga.z[0];
+        g8.z[1] = ga.z[1];
+        g8.zidx[0] = ga.zidx[0];
+        g8.zidx[1] = ga.zidx[1];
+        g8.zld = ga.zld;
+        g8.zks = ga.zks;
+        g8.zsplit = ga.zsplit;
+        g8.xext = xext;
+        g8.status = ga.status;
+        TQ_CUDA(launch_pdl(gather_x8_kernel, dim3(T), dim3(256), 0, stream, g8));
+        TQ_LAUNCHED();
+      } else {
+        const long long chunks = (long long)T * (D / 8) + (long long)plan.P * (lr_gu ? 2 * qg.rank / 8 : 0);
+        TQ_CUDA(launch_pdl(gather_ext_kernel, dim3(gather_blocks(chunks)), dim3(256), 0, stream, ga));
+        TQ_LAUNCHED();
+      }
     }
     mark(ST_ZPROJ, stream);
     {
@@ -1259,6 +1347,7 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
       r.out[0] = hext;
       r.ldo = w.ld_h;
       r.row_scale = at<float>(ws, w.slot_w);
+      r.f8 = plan.gateup.dq;
       if ((st = run_residual(r, plan.gateup, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     }
     mark(ST_GATEUP, stream);
@@ -1365,6 +1454,14 @@ tileq_status tileq_pack_per_expert(const tileq_layer *layer, const tileq_per_exp
         static_cast<const __nv_bfloat16 *>(pe->V_pe[p]), (long long)q.d_in * q.rank, 1, q.rank, K,
         q.rank, q.d_in, 8, at<uint4>(packed_pe, pl.vf[p]));
     TQ_LAUNCHED();
+    n = (long long)K * pad128(q.d_out) * q.rank;
+    pack_rows_f16_kernel<<<nblocks(n, 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(pe->U_pe[p]), K,
+                                                               q.d_out, q.rank, at<__half>(packed_pe, pl.ur[p]));
+    TQ_LAUNCHED();
+    n = (long long)K * pad128(q.rank) * q.d_in;
+    pack_vt_rows_kernel<<<nblocks(n, 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(pe->V_pe[p]), K,
+                                                               q.rank, q.d_in, at<__half>(packed_pe, pl.vr[p]));
+    TQ_LAUNCHED();
   }
   return TILEQ_OK;
 }
@@ -1389,56 +1486,94 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
   st = run_route_permute(layer, li, w, x, T, router_logits, top_k, ws, 0, zids, -1, stream);
   if (st != TILEQ_OK) return st;
 
-  // Per-expert low-rank pass of projection(s) over the expert's slots:
+  // Per-expert low-rank pass of projection(s) over every slot, from the
+  // independent per-expert factors (no sharing across grid rows or columns):
   //   zpe = Sigma * (V_pe[e]^T B[slot])   then   out[slot] += U_pe[e] zpe
-  // The tiles of one expert are contiguous in the main table from
-  // tile_first[e]; their number is known only on the device, so each
-  // per-expert launch covers the largest possible expert (T slots) and its
-  // surplus CTAs return at once.
+  // Both products are grouped over all experts' tiles in one launch each, with
+  // the fused path's tuning: split-K warp-level MMA below 256 tokens (the z
+  // splits reduced by the last CTA of a tile), the dense tcgen05 kernel above.
   auto per_expert_lr = [&](int np, const int *projs, const __half *bsrc, int ldb, const int *b_row,
-                           float *const *outs, int ldo) -> tileq_status {
-    const GemmPlan &gp = plan.pe;
-    for (int e = 0; e < K; ++e) {
-      GemmBatch zb, ub;
+                           float *const *outs, int ldo, const GemmPlan &zp) -> tileq_status {
+    const GemmPlan &up = plan.pe_u;
+    if (zp.tc) {
       for (int i = 0; i < np; ++i) {
         const ProjInfo &q = li.p[projs[i]];
-        zb.p[i] = problem(gp, ws, w);
-        GemmProblem &z = zb.p[i];
-        z.m_tiles = cdiv(q.rank, 128);
-        z.tiles = at<int4>(ws, w.tiles_main);
-        z.tile_count = at<int>(ws, w.tile_counts);
-        z.only_group = e;
-        z.group_first_tile = at<int>(ws, w.tile_first);
+        int8_t ident[kMaxExperts];
+        for (int e = 0; e < kMaxExperts; ++e) ident[e] = (int8_t)e;
+        TcF16 z;
+        z.arow[0] = at<__half>(packed_pe, ppl.vr[projs[i]]);
+        z.lda = q.d_in;
+        z.arows = K * pad128(q.rank);
         z.d_out = q.rank;
         z.d_in = q.d_in;
-        z.a[0] = at<uint4>(packed_pe, ppl.vf[projs[i]]);
+        z.tiles = at<int4>(ws, w.tiles_main);
+        z.tile_count = at<int>(ws, w.tile_counts);
+        z.a_blk = ident;
         z.b = bsrc;
+        z.brows = plan.P;
         z.ldb = ldb;
-        z.b_row = b_row;
         z.epi = EPI_STORE_F16;
-        z.col_scale = layer->proj[projs[i]].Sigma;
         z.out[0] = at<__half>(ws, w.zpe[i]);
         z.ldo = q.rank;
-        ub.p[i] = problem(gp, ws, w);
-        GemmProblem &u = ub.p[i];
-        u.m_tiles = cdiv(q.d_out, 128);
-        u.tiles = z.tiles;
-        u.tile_count = z.tile_count;
-        u.only_group = e;
-        u.group_first_tile = z.group_first_tile;
+        z.col_scale[0] = layer->proj[projs[i]].Sigma;
+        if ((st = tc_f16(z, zp, ws, w, stream)) != TILEQ_OK) return st;
+        TcF16 u;
+        u.arow[0] = at<__half>(packed_pe, ppl.ur[projs[i]]);
+        u.lda = q.rank;
+        u.arows = K * pad128(q.d_out);
         u.d_out = q.d_out;
         u.d_in = q.rank;
-        u.a[0] = at<uint4>(packed_pe, ppl.uf[projs[i]]);
+        u.tiles = z.tiles;
+        u.tile_count = z.tile_count;
+        u.a_blk = ident;
         u.b = at<__half>(ws, w.zpe[i]);
+        u.brows = plan.P;
         u.ldb = q.rank;
         u.epi = EPI_ACCUM_F32;
         u.out[0] = outs[i];
         u.ldo = ldo;
+        if ((st = tc_f16(u, up, ws, w, stream)) != TILEQ_OK) return st;
       }
-      if ((st = gemm(zb, np, 1, gp, stream)) != TILEQ_OK) return st;
-      if ((st = gemm(ub, np, 1, gp, stream)) != TILEQ_OK) return st;
+      return TILEQ_OK;
     }
-    return TILEQ_OK;
+    GemmBatch zb, ub;
+    const int ncnt = zp.slots * zp.m_tiles;  // split-K arrival counters of one problem
+    for (int i = 0; i < np; ++i) {
+      const ProjInfo &q = li.p[projs[i]];
+      zb.p[i] = problem(zp, ws, w);
+      GemmProblem &z = zb.p[i];
+      z.tiles = at<int4>(ws, w.tiles_main);
+      z.tile_count = at<int>(ws, w.tile_counts);
+      z.d_out = q.rank;
+      z.d_in = q.d_in;
+      z.a[0] = at<uint4>(packed_pe, ppl.vf[projs[i]]);
+      z.b = bsrc;
+      z.ldb = ldb;
+      z.b_row = b_row;
+      z.epi = EPI_STORE_F16;
+      z.col_scale = layer->proj[projs[i]].Sigma;
+      z.out[0] = at<__half>(ws, w.zpe[i]);
+      z.ldo = q.rank;
+      z.counters = at<int>(ws, w.counters) + i * ncnt;
+      z.part = at<float>(ws, w.part) + (size_t)i * (zp.part_floats() / std::max(1, zp.np));
+      if (!b_row) tma_b(z, plan.P, zp.bn);
+      ub.p[i] = problem(up, ws, w);
+      GemmProblem &u = ub.p[i];
+      u.m_tiles = cdiv(q.d_out, 128);
+      u.tiles = z.tiles;
+      u.tile_count = z.tile_count;
+      u.d_out = q.d_out;
+      u.d_in = q.rank;
+      u.a[0] = at<uint4>(packed_pe, ppl.uf[projs[i]]);
+      u.b = at<__half>(ws, w.zpe[i]);
+      u.ldb = q.rank;
+      u.epi = EPI_ACCUM_F32;
+      u.out[0] = outs[i];
+      u.ldo = ldo;
+      tma_b(u, plan.P, up.bn);
+    }
+    if ((st = gemm(zb, np, 1, zp, stream)) != TILEQ_OK) return st;
+    return gemm(ub, np, 1, up, stream);
   };
 
   if (layer->kind == TILEQ_LINEAR) {
@@ -1456,7 +1591,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     if (q.rank > 0) {
       const int projs[1] = {0};
       float *outs[1] = {at<float>(ws, w.ybuf)};
-      st = per_expert_lr(1, projs, xext, w.ld_x, nullptr, outs, q.d_out);
+      st = per_expert_lr(1, projs, xext, w.ld_x, nullptr, outs, q.d_out, plan.pe_zx);
       if (st != TILEQ_OK) return st;
     }
     for (int sidx = ST_ZPROJ; sidx <= ST_ZDOWN; ++sidx) mark(sidx, stream);
@@ -1492,7 +1627,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     if (qg.rank > 0) {
       const int projs[2] = {0, 1};
       float *outs[2] = {at<float>(ws, w.g32), at<float>(ws, w.u32)};
-      st = per_expert_lr(2, projs, at<__half>(ws, w.x16), D, at<int>(ws, w.slot_tok), outs, F);
+      st = per_expert_lr(2, projs, xext, w.ld_x, nullptr, outs, F, plan.pe_zx);
       if (st != TILEQ_OK) return st;
     }
     mark(ST_ZPROJ, stream);
@@ -1511,7 +1646,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
     if (qd.rank > 0) {
       const int projs[1] = {2};
       float *outs[1] = {at<float>(ws, w.ybuf)};
-      st = per_expert_lr(1, projs, hext, w.ld_h, nullptr, outs, D);
+      st = per_expert_lr(1, projs, hext, w.ld_h, nullptr, outs, D, plan.pe_zd);
       if (st != TILEQ_OK) return st;
     }
     mark(ST_ZDOWN, stream);

@@ -243,6 +243,8 @@ __global__ void __launch_bounds__(DenseCfg<MB, BN>::THREADS, 1)
             void *dst = P.out[P.pair ? j : 0];
             if (P.epi == EPI_STORE_F16)
               reinterpret_cast<__half *>(dst)[ib + o[j]] = half_checked(v[j][i] * cs[j], P.status);
+            else if (P.epi == EPI_ACCUM_F32)
+              reinterpret_cast<float *>(dst)[ib + o[j]] += v[j][i] * cs[j];
             else
               reinterpret_cast<float *>(dst)[ib + o[j]] = v[j][i] * cs[j];
           }

@@ -127,8 +127,9 @@ __device__ __forceinline__ void dq_qz_word(uint32_t w, const __half2 (&nz)[4], u
   }
 }
 
-template <int NP, int BN>
+template <int NP, int BN, bool F8>
 __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_constant__ DqArgs P) {
+  static_assert(!F8 || NP == 2, "fp8 mode: gate/up");
   using C = DqCfg<NP, BN>;
   constexpr int HC = BN / 2;  // accumulator columns per decode warp
   extern __shared__ uint8_t smem_raw[];
@@ -213,9 +214,15 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
             bulk_g2s(st_codes(s, sl), reinterpret_cast<const uint8_t *>(P.codes[p]) + blk * 4096, 4096, &full[s]);
             const size_t zoff = (((size_t)grp * P.m_tiles + rd.ob) * G + (kb * 128) / P.group) * 128;
             bulk_g2s(const_cast<uint32_t *>(st_sz(s, sl)), P.sz[p] + zoff, 512, &full[s]);
-            if (NP == 1 || sl == 0)
+            if (F8) {
+              // the two e4m3 pieces of the 128 K of this block (one 128-byte box each)
+              if (sl == 0)
+                for (int pc = 0; pc < 2; ++pc)
+                  tc::tma_load_2d(bs + pc * C::ATOM, &P.bmap, pc * P.d_in + kb * 128, item0, &full[s]);
+            } else if (NP == 1 || sl == 0) {
               for (int a = 0; a < 2; ++a)
                 tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, &P.bmap, kb * 128 + a * 64, item0, &full[s]);
+            }
           }
         } else {
           int na = 0;
@@ -227,8 +234,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
             const int p = NP == 2 ? sl : 0;
             const int len = min(128, P.rank - rd.chunk[sl] * 128);
             for (int a = 0; a * 64 < len; ++a)
-              tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, &P.bmap, P.ext_col[p] + rd.chunk[sl] * 128 + a * 64,
-                              item0, &full[s]);
+              tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, F8 ? &P.bmap_ext : &P.bmap,
+                              P.ext_col[p] + rd.chunk[sl] * 128 + a * 64, item0, &full[s]);
           }
         }
       }
@@ -249,6 +256,15 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
           if (!rd.valid[sl]) continue;
+          if (F8 && !rd.ext) {
+            // e4m3: four K = 32 steps over 128 K; both pieces of B into the same accumulator
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+              for (int pc = 0; pc < 2; ++pc)
+                tc::mma_ts_f8(d0 + sl * BN, a0 + sl * 64 + kk * 8,
+                              bd0 + (uint64_t)((pc * C::ATOM + kk * 32) >> 4), idesc, (kk | pc) ? 1u : 0u);
+            continue;
+          }
           // B atoms of this slice: main rounds of a two-projection launch share atoms 0, 1
           const int atom0 = (NP == 2 && !rd.ext) ? 0 : 2 * sl;
           for (int kk = 0; kk < rd.nk[sl]; ++kk)
@@ -274,7 +290,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
     float acc[HC];
 #pragma unroll
     for (int c = 0; c < HC; ++c) acc[c] = 0.f;
-    float sc0 = 0.f, sc1 = 0.f;  // scale of this warp's slice in the rounds of even / odd index (0: nothing)
+    float sc0 = 0.f, sc1 = 0.f;  // this row's scale of the warp's slice in the rounds of even / odd index
+    bool v0 = false, v1 = false;  // the warp's slice was valid in the last round of even / odd index
 
     // ---- end of a unit's rounds in this CTA: combine the two slices, then
     // store the result (whole unit) or a piece (unit cut between CTAs)
@@ -295,6 +312,11 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
         auto store = [&](int c, float g, float u) {
           const int n = part * HC + c;
           if (n >= nitems || o >= P.d_out) return;
+          if (F8) {  // the activations were scaled by 2^e per item
+            const float xs = __ldg(P.xs + item0 + n);
+            g *= xs;
+            u *= xs;
+          }
           if (NP == 2 && P.epi == EPI_STORE2_F32) {
             reinterpret_cast<float *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = g;
             reinterpret_cast<float *>(P.out2)[(size_t)(item0 + n) * P.ldo + o] = u;
@@ -387,7 +409,9 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
       if (!mbar_wait(&mma_done[j & 1], (j >> 1) & 1, P.status)) return false;
       tc::fence_after();
       const float sc = (j & 1) ? sc1 : sc0;
-      if (sc != 0.f) {
+      // tcgen05.ld is warp-collective: the decision is the warp's (its slice
+      // was valid in round j), never a lane's (padding rows have scale 0)
+      if ((j & 1) ? v1 : v0) {
         const uint32_t base = tmem + lane_addr + C::ACC0 + (j & 1) * C::ACC_COLS + sl * BN + part * HC;
 #pragma unroll
         for (int c0 = 0; c0 < HC; c0 += 16) {
@@ -434,11 +458,25 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
                      : "=r"(w[2]), "=r"(w[3])
                      : "r"(smem_addr(cb + (2 * part + 1) * 1024 + row * 8)));
         const __half2 szw = u32_as_h2(st_sz(s, sl)[row]);
-        const __half2 z2 = __high2half2(szw);
-        const __half2 nz[4] = {__hsub2(__float2half2_rn(-1024.f), z2), __hsub2(__float2half2_rn(-256.f), z2),
-                               __hsub2(__float2half2_rn(-64.f), z2), __hsub2(__float2half2_rn(-16.f), z2)};
+        if constexpr (F8) {
+          // e4m3 (q - z) through a 4-entry byte table per zero point: one PRMT per 4 weights
+          const int zi = (int)__high2float(szw);
+          const uint32_t tab = zi == 0 ? 0x44403800u : zi == 1 ? 0x403800B8u : zi == 2 ? 0x3800B8C0u : 0x00B8C0C4u;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) dq_qz_word(w[q], nz, v + 8 * q);
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t c0 = w[q] & 0x33333333u, c1 = (w[q] >> 2) & 0x33333333u;
+            v[4 * q + 0] = __byte_perm(tab, 0, c0);
+            v[4 * q + 1] = __byte_perm(tab, 0, c0 >> 16);
+            v[4 * q + 2] = __byte_perm(tab, 0, c1);
+            v[4 * q + 3] = __byte_perm(tab, 0, c1 >> 16);
+          }
+        } else {
+          const __half2 z2 = __high2half2(szw);
+          const __half2 nz[4] = {__hsub2(__float2half2_rn(-1024.f), z2), __hsub2(__float2half2_rn(-256.f), z2),
+                                 __hsub2(__float2half2_rn(-64.f), z2), __hsub2(__float2half2_rn(-16.f), z2)};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dq_qz_word(w[q], nz, v + 8 * q);
+        }
         sc = __low2float(szw);
       } else if (mine) {
         // rows of U_m: rank columns chunk * 128 + part * 64 ..
@@ -459,10 +497,20 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
         sc = 1.f;
       }
       if (mine) {
-        tc::st32(tmem + lane_addr + (i & 1) * 128 + sl * 64 + part * 32, v);
+        if (F8 && !rd.ext) {
+          tc::st16(tmem + lane_addr + (i & 1) * 128 + sl * 64 + part * 16, *reinterpret_cast<uint32_t(*)[16]>(v));
+        } else {
+          tc::st32(tmem + lane_addr + (i & 1) * 128 + sl * 64 + part * 32, v);
+        }
         tc::wait_st();
       }
-      if (i & 1) sc1 = sc; else sc0 = sc;
+      if (i & 1) {
+        sc1 = sc;
+        v1 = mine;
+      } else {
+        sc0 = sc;
+        v0 = mine;
+      }
       tc::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&a_full[i & 1]);
@@ -481,10 +529,10 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
   }
 }
 
-template <int NP, int BN>
+template <int NP, int BN, bool F8 = false>
 cudaError_t launch_dq(const DqArgs &a, cudaStream_t stream) {
   using C = DqCfg<NP, BN>;
-  auto kern = gemm_dq_kernel<NP, BN>;
+  auto kern = gemm_dq_kernel<NP, BN, F8>;
   static bool configured = false;  // one attribute call per instantiation and process
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -504,6 +552,15 @@ int dq_grid() { return DQ_GRID; }
 cudaError_t launch_gemm_dq(const DqArgs &a, int np, int bn, cudaStream_t stream) {
   if (a.m_tiles <= 0 || a.group % 128 != 0 || a.d_in % 128 != 0 || a.rank < 0 || a.rank > 256)
     return cudaErrorInvalidValue;
+  if (a.f8) {
+    if (np != 2) return cudaErrorInvalidValue;
+    switch (bn) {
+      case 16: return launch_dq<2, 16, true>(a, stream);
+      case 32: return launch_dq<2, 32, true>(a, stream);
+      case 64: return launch_dq<2, 64, true>(a, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (bn * 4 + np) {
     case 16 * 4 + 1: return launch_dq<1, 16>(a, stream);
     case 32 * 4 + 1: return launch_dq<1, 32>(a, stream);

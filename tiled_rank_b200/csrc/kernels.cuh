@@ -182,7 +182,11 @@ cudaError_t launch_gemm_tc(const TcArgs &a, int np, int bn, int grid, cudaStream
 // two consecutive K blocks of one projection (np = 1); the low-rank K
 // extension follows the residual rounds of each unit.
 struct DqArgs {
-  alignas(64) CUtensorMap bmap;  // B: fp16 activation rows [items][ldb], box 64 x bn, 128-byte swizzle
+  alignas(64) CUtensorMap bmap;  // B: fp16 activation rows [items][ldb], box 64 x bn, 128-byte swizzle;
+                                 // fp8 mode: the e4m3 pieces [items][2][d_in] bytes, box 128 x bn
+  alignas(64) CUtensorMap bmap_ext;  // fp8 mode: the fp16 rows holding the extension columns
+  int f8;                        // fp8 mode (np = 2): A = e4m3 (q - z), B = two e4m3 pieces of x * 2^e
+  const float *xs;               // fp8 mode: per item 2^-e
   const int4 *tiles;             // (expert, first item, items)
   const int *tile_count;
   int m_tiles, d_out, d_in, group, rank;
@@ -276,6 +280,28 @@ struct GatherExtArgs {
   int *status;
 };
 
+// The activations of the fp8 decode GEMM (gate/up), one CTA per token t:
+// with e_t the power of two that puts max|x_t| in [128, 256), each slot of the
+// token gets x * 2^e_t as two e4m3 pieces (x8[slot][0][k] + x8[slot][1][k]:
+// the rounded value and its rounded remainder; exact for every element within
+// 2^-9 of the row maximum), the elements of each 16-wide block stored in the
+// order k = 4*(s%4) + s/4 of the decoded weights (the block's 4 x 4 transpose),
+// xs[slot] = 2^-e_t, and its z rows (sum of the K-split partials) times 2^e_t
+// in fp16 into the extension columns d .. d + nz*r of xext.
+struct GatherX8Args {
+  int T, k, d, r, ld;
+  const int *slot_of_pair;   // [T*k]
+  const __half *x16;         // [T][d]
+  uint8_t *x8;               // [P][2][d]
+  float *xs;                 // [P]
+  const float *z[2];         // fp32 partials [zks][rows][zld], or null
+  const int *zidx[2];        // slot -> row of the projected [T, N, r] tensor
+  int zld, zks;
+  long long zsplit;
+  __half *xext;              // [P][ld]
+  int *status;
+};
+
 // Row accumulation, written per slot into the K-extension columns of the
 // activation matrix: the designated slot of each (token, grid row) gets a_{t,m},
 // every other slot zeros.
@@ -335,6 +361,7 @@ static_assert(kMaxTopK == 8, "launch_combine instantiates top-k 1..8");
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream);
 __global__ void scale_gather_kernel(ScaleGatherArgs a);
 __global__ void gather_ext_kernel(GatherExtArgs a);
+__global__ void gather_x8_kernel(GatherX8Args a);
 __global__ void swiglu_kernel(SwigluArgs a);
 __global__ void bounded_wait_kernel(int *status, int max_polls);
 

@@ -1,6 +1,8 @@
 // Small element-wise kernels of the TileQ forward: the in-place accumulation
 // of the low-rank projections per (token, grid row), the weighted top-k
 // combine / unpermute, and the helpers of the unfused comparison path.
+#include <cuda_fp8.h>
+
 #include "kernels.cuh"
 
 namespace tileq {
@@ -152,6 +154,105 @@ __global__ void __launch_bounds__(256) gather_ext_kernel(GatherExtArgs a) {
         reinterpret_cast<uint4 *>(a.out + (size_t)s * a.ld)[c] = v[u];
       }
     }
+  }
+}
+
+// e4m3 pieces of one 16-element block of a scaled activation row: p0 + p1.
+__device__ __forceinline__ void e4m3_pieces(const float (&v)[16], uint4 &p0, uint4 &p1) {
+  uint32_t w0[4], w1[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // stored position 4j + b holds element j + 4b (the order of the decoded weights)
+    float f0[4], f1[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const float x = v[j + 4 * b];
+      const __nv_fp8_storage_t h = __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+      const float hx = __half2float(__half(__nv_cvt_fp8_to_halfraw(h, __NV_E4M3)));
+      f0[b] = hx;
+      f1[b] = x - hx;
+    }
+    const __nv_fp8x2_storage_t a01 = __nv_cvt_float2_to_fp8x2(make_float2(f0[0], f0[1]), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t a23 = __nv_cvt_float2_to_fp8x2(make_float2(f0[2], f0[3]), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t b01 = __nv_cvt_float2_to_fp8x2(make_float2(f1[0], f1[1]), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t b23 = __nv_cvt_float2_to_fp8x2(make_float2(f1[2], f1[3]), __NV_SATFINITE, __NV_E4M3);
+    w0[j] = (uint32_t)a01 | ((uint32_t)a23 << 16);
+    w1[j] = (uint32_t)b01 | ((uint32_t)b23 << 16);
+  }
+  p0 = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+  p1 = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+}
+
+__global__ void __launch_bounds__(256) gather_x8_kernel(GatherX8Args a) {
+  pdl_wait_and_release();
+  __shared__ float red[8];
+  const int t = blockIdx.x;
+  if (t >= a.T) return;
+  const __half *xr = a.x16 + (size_t)t * a.d;
+  const int nb = a.d / 16;
+  // the row maximum of |x|
+  float m = 0.f;
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(xr + b * 16);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 u = __ldg(q + h);
+      const __half2 *hh = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(hh[i]);
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+  int ex = 0;
+  if (m > 0.f) frexpf(m, &ex);            // m = f * 2^ex, f in [0.5, 1)
+  const int e = m > 0.f ? 8 - ex : 0;     // m * 2^e in [128, 256)
+  const float up = ldexpf(1.f, e), down = ldexpf(1.f, -e);
+  int slots[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) slots[j] = j < a.k ? __ldg(a.slot_of_pair + t * a.k + j) : 0;
+  if (threadIdx.x < a.k) a.xs[slots[threadIdx.x]] = down;
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+    float v[16];
+    const uint4 *q = reinterpret_cast<const uint4 *>(xr + b * 16);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 u = __ldg(q + h);
+      const __half2 *hh = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(hh[i]);
+        v[8 * h + 2 * i] = f.x * up;
+        v[8 * h + 2 * i + 1] = f.y * up;
+      }
+    }
+    uint4 p0, p1;
+    e4m3_pieces(v, p0, p1);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j >= a.k) break;
+      uint8_t *row = a.x8 + (size_t)slots[j] * 2 * a.d;
+      reinterpret_cast<uint4 *>(row)[b] = p0;
+      reinterpret_cast<uint4 *>(row + a.d)[b] = p1;
+    }
+  }
+  // z rows of the token's slots, scaled like x, into the extension columns
+  const int nz = a.z[0] ? (a.z[1] ? 2 : 1) : 0;
+  const int per = nz * a.r;
+  for (int idx = threadIdx.x; idx < a.k * per; idx += blockDim.x) {
+    const int j = idx / per, c = idx % per, p = c / a.r, i = c % a.r;
+    const int s = slots[j];
+    const float *zp = a.z[p] + (size_t)a.zidx[p][s] * a.zld + i;
+    float acc = 0.f;
+    for (int sp = 0; sp < a.zks; ++sp) acc += zp[(size_t)sp * a.zsplit];
+    a.xext[(size_t)s * a.ld + a.d + c] = half_checked(acc * up, a.status);
   }
 }
 

@@ -116,6 +116,18 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// kind::f8f6f4: D[tmem] (+)= A[tmem] * B[smem] with A and B both e4m3 (the
+// instruction descriptor's type fields are 0 for e4m3, as for fp16 in
+// kind::f16), K = 32 per instruction.
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // True in exactly one active lane of the (converged) warp.
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred;
