@@ -1495,7 +1495,9 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
   auto per_expert_lr = [&](int np, const int *projs, const __half *bsrc, int ldb, const int *b_row,
                            float *const *outs, int ldo, const GemmPlan &zp) -> tileq_status {
     const GemmPlan &up = plan.pe_u;
-    if (zp.tc) {
+    bool tc = zp.tc;  // the dense tcgen05 kernel takes K in multiples of 64 (the U side: K = rank)
+    for (int i = 0; i < np; ++i) tc = tc && li.p[projs[i]].rank % 64 == 0;
+    if (tc) {
       for (int i = 0; i < np; ++i) {
         const ProjInfo &q = li.p[projs[i]];
         int8_t ident[kMaxExperts];

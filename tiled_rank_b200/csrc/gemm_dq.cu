@@ -72,31 +72,58 @@ struct Round {
   int nk[2];     // 16-wide K steps of each slice
 };
 
+// Walks the rounds of a CTA's range in order without divisions: one division
+// places it at the range's first round, then each advance is a few compares.
 template <int NP>
-__device__ __forceinline__ Round round_of(long long r, int R, int nmain, int nkb, int m_tiles, int rank) {
-  Round o;
-  o.unit = (int)(r / R);
-  o.rr = (int)(r % R);
-  o.jt = o.unit / m_tiles;
-  o.ob = o.unit % m_tiles;
-  o.ext = o.rr >= nmain;
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    if (!o.ext) {
-      o.kb[s] = NP == 2 ? o.rr : 2 * o.rr + s;
-      o.valid[s] = o.kb[s] < nkb;
-      o.chunk[s] = 0;
-      o.nk[s] = 8;
-    } else {
-      const int e = o.rr - nmain;
-      o.chunk[s] = NP == 2 ? e : 2 * e + s;
-      o.valid[s] = o.chunk[s] * 128 < rank;
-      o.kb[s] = 0;
-      o.nk[s] = o.valid[s] ? (min(128, rank - o.chunk[s] * 128) + 15) / 16 : 0;
+struct RoundCursor {
+  int unit, rr, jt, ob;
+  int R, nmain, nkb, m_tiles, rank;
+  __device__ __forceinline__ void init(long long r, int R_, int nmain_, int nkb_, int m_tiles_, int rank_) {
+    R = R_;
+    nmain = nmain_;
+    nkb = nkb_;
+    m_tiles = m_tiles_;
+    rank = rank_;
+    unit = (int)(r / R);
+    rr = (int)(r - (long long)unit * R);
+    jt = unit / m_tiles;
+    ob = unit - jt * m_tiles;
+  }
+  __device__ __forceinline__ void advance() {
+    if (++rr == R) {
+      rr = 0;
+      ++unit;
+      if (++ob == m_tiles) {
+        ob = 0;
+        ++jt;
+      }
     }
   }
-  return o;
-}
+  __device__ __forceinline__ Round get() const {
+    Round o;
+    o.unit = unit;
+    o.rr = rr;
+    o.jt = jt;
+    o.ob = ob;
+    o.ext = rr >= nmain;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      if (!o.ext) {
+        o.kb[s] = NP == 2 ? rr : 2 * rr + s;
+        o.valid[s] = o.kb[s] < nkb;
+        o.chunk[s] = 0;
+        o.nk[s] = 8;
+      } else {
+        const int e = rr - nmain;
+        o.chunk[s] = NP == 2 ? e : 2 * e + s;
+        o.valid[s] = o.chunk[s] * 128 < rank;
+        o.kb[s] = 0;
+        o.nk[s] = o.valid[s] ? (min(128, rank - o.chunk[s] * 128) + 15) / 16 : 0;
+      }
+    }
+    return o;
+  }
+};
 
 // First round of CTA c's range of `total` rounds over `g` CTAs.
 __device__ __forceinline__ long long range_begin(long long total, int c, int g) { return total * c / g; }
@@ -191,10 +218,12 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
     // ============================================================ producer
     if (lane == 0) {
       int i = 0;
-      for (; i < nr; ++i) {
+      RoundCursor<NP> cur;
+      cur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
+      for (; i < nr; ++i, cur.advance()) {
         const int s = i % C::NS;
         if (i >= C::NS && !(ok = mbar_wait(&empty[s], ((i / C::NS) - 1) & 1, P.status))) break;
-        const Round rd = round_of<NP>(r0 + i, R, nmain, nkb, P.m_tiles, P.rank);
+        const Round rd = cur.get();
         const int4 t = P.tiles[rd.jt];
         const int grp = t.x, item0 = t.y;
         uint8_t *bs = st_b(s);
@@ -245,11 +274,13 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
   } else if (warp == 1) {
     // ============================================================ MMA issuer
     constexpr uint32_t idesc = tc::idesc_f16(BN);
-    for (int i = 0; i < nr; ++i) {
+    RoundCursor<NP> cur;
+    cur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
+    for (int i = 0; i < nr; ++i, cur.advance()) {
       const int as = i & 1;
       if (!(ok = mbar_wait(&a_full[as], (i >> 1) & 1, P.status))) break;
       tc::fence_after();
-      const Round rd = round_of<NP>(r0 + i, R, nmain, nkb, P.m_tiles, P.rank);
+      const Round rd = cur.get();
       if (tc::elect_one()) {
         const uint64_t bd0 = tc::sdesc_sw128(smem_addr(st_b(i % C::NS)));
         const uint32_t a0 = tmem + as * 128, d0 = tmem + C::ACC0 + as * C::ACC_COLS;
@@ -405,6 +436,9 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
     };
 
     // ---- fold round j's accumulator (slot j & 1) into registers; release its stage
+    // (rounds are finished in order: fcur is at round j)
+    RoundCursor<NP> fcur;
+    fcur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
     auto finish = [&](int j) -> bool {
       if (!mbar_wait(&mma_done[j & 1], (j >> 1) & 1, P.status)) return false;
       tc::fence_after();
@@ -432,17 +466,20 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
       tc::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[j % C::NS]);
-      const Round rd = round_of<NP>(r0 + j, R, nmain, nkb, P.m_tiles, P.rank);
+      const Round rd = fcur.get();  // round j
+      fcur.advance();
       if (rd.rr == R - 1 || j == nr - 1) unit_end(rd);
       return true;
     };
 
-    for (int i = 0; i < nr && ok; ++i) {
+    RoundCursor<NP> cur;
+    cur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
+    for (int i = 0; i < nr && ok; ++i, cur.advance()) {
       const int s = i % C::NS;
       if (!(ok = mbar_wait(&full[s], (i / C::NS) & 1, P.status))) break;
       // round i - 2: fold its accumulator; its A slot is then free for round i
       if (i >= 2 && !(ok = finish(i - 2))) break;
-      const Round rd = round_of<NP>(r0 + i, R, nmain, nkb, P.m_tiles, P.rank);
+      const Round rd = cur.get();
       const bool mine = sl ? rd.valid[1] : rd.valid[0];
       const int chunk = sl ? rd.chunk[1] : rd.chunk[0];
       uint32_t v[32];
