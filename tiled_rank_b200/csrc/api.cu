@@ -219,11 +219,7 @@ int choose_bn(long long avg) {
 // Items per tile of the decode-regime tcgen05 GEMM: wide enough that most
 // experts fit one tile (an expert spilling into a second tile streams its
 // weights twice).
-int choose_bn_dq(long long avg) {
-  if (avg <= 6) return 16;
-  if (avg <= 16) return 32;
-  return 64;
-}
+int choose_bn_dq(long long avg) { return avg <= 6 ? 16 : 32; }
 
 // Items per tile of the tensor-core GEMM (N of one tcgen05.mma: 16..128).
 int choose_bn_tc(long long avg) {

@@ -25,11 +25,14 @@
 // slot holds rows of the grid row's U_m (fp16, read from global memory) and B
 // the matching z (or a) columns of the item rows, with scale 1.
 //
-// Warp roles (18 warps): warp 0 producer (bulk copies of the codes and their
-// (scale, zero) words, 2-D TMA boxes of B into a ring of stages), warp 1 MMA
+// Warp roles (6 warps): warp 0 producer (bulk copies of the codes and their
+// (scale, zero) words in chunks of up to 8 K blocks per projection into a
+// ring of chunk slots, 2-D TMA boxes of B per round into a ring of its own), warp 1 MMA
 // issuer (the whole warp waits, one elected lane issues and commits), warps
-// 2..17 decode and epilogue: warp w works on TMEM lane quadrant w % 4 (32
-// weight rows), slice ((w - 2) / 4) / 2 and K half / column half (w - 2) / 4 % 2.
+// 2..5 decode and epilogue: warp w works on TMEM lane quadrant w % 4 (32
+// weight rows) and both slices of every round (256 weights per thread and
+// round, so that each barrier round amortises over enough decode work), with
+// both slices' accumulators in its registers.
 // Every wait is bounded and reports TILEQ_ERR_TIMEOUT.
 #include "kernels.cuh"
 #include "tc.cuh"
@@ -38,7 +41,7 @@ namespace tileq {
 
 namespace {
 
-constexpr int DQ_DW = 16;                     // decode / epilogue warps
+constexpr int DQ_DW = 4;                      // decode / epilogue warps (one per TMEM lane quadrant)
 constexpr int DQ_THREADS = (2 + DQ_DW) * 32;  // + producer + MMA issuer
 constexpr int DQ_GRID = 148;                  // one CTA per SM
 
@@ -46,20 +49,49 @@ template <int NP, int BN>
 struct DqCfg {
   static constexpr int ATOM = BN * 128;                // one 64-wide fp16 K atom of B: BN rows x 128 B
   static constexpr int B_BYTES = 4 * ATOM;             // up to four atoms per round
-  static constexpr int CODES = 2 * 4096;               // two 128 x 128 blocks of 2-bit codes
-  static constexpr int SZ = 2 * 512;                   // their (scale, zero) words
-  static constexpr int STAGE = (B_BYTES + CODES + SZ + 1023) / 1024 * 1024;
-  static constexpr int XBUF = 128 * BN * 4;            // unit-end exchange between the two slices
-  static constexpr int NS_RAW = (200 * 1024 - XBUF) / STAGE;
-  static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;   // ring stages
-  static constexpr int XBUF_OFF = NS * STAGE;
-  static constexpr int BAR_OFF = XBUF_OFF + XBUF;
-  static constexpr int SMEM = BAR_OFF + (2 * NS + 5) * 8 + 16 + BN * 4 + 1024;  // + slack to align the base
+  // The codes stream from HBM in chunks of up to CB consecutive 128-wide K
+  // blocks per projection (one bulk copy of up to 32 KB each, with the
+  // (scale, zero) words of their groups): a few large copies in flight keep
+  // the weight stream at the HBM rate, where one 4 KB copy per block does not.
+  static constexpr int CB = 8;
+  static constexpr int RPC = NP == 2 ? CB : CB / 2;     // main rounds per chunk
+  static constexpr int CODE_SLOT = NP * CB * (4096 + 512);
+  static constexpr int NB = 4;                         // activation ring (per round, from L2)
+  static constexpr int NC_RAW = (210 * 1024 - NB * B_BYTES) / CODE_SLOT;
+  static constexpr int NC = NC_RAW > 4 ? 4 : NC_RAW;   // code chunk ring
+  static constexpr int CODE_OFF = NB * B_BYTES;
+  static constexpr int BAR_OFF = CODE_OFF + NC * CODE_SLOT;
+  static constexpr int SMEM = BAR_OFF + (2 * NB + 2 * NC + 5) * 8 + 16 + BN * 4 + 1024;  // + slack to align the base
   static constexpr int ACC_COLS = 2 * BN;             // one accumulator slot: two slices
   static constexpr int ACC0 = 256;                     // TMEM: A slots at 0 and 128, accumulators from 256
-  static_assert(NS >= 3, "ring too shallow");
+  static_assert(NC >= 2, "code ring too shallow");
   static_assert(ACC0 + 2 * ACC_COLS <= 512, "tensor memory");
   static_assert(ATOM % 1024 == 0, "swizzled atoms need 1024-byte alignment");
+};
+
+// Where a CTA's main rounds of one unit start new code chunks: chunks hold
+// RPC consecutive main rounds from the first main round the CTA processes in
+// the unit, up to its last one.  Producer and consumers step it the same way.
+struct ChunkTrack {
+  int rr_lo = 0, rr_hi = 0;  // main rounds [rr_lo, rr_hi) of the current unit in this CTA
+  int n = 0;                 // chunks started so far
+  template <int RPC>
+  __device__ __forceinline__ void on_round(bool first_of_unit, int rr, int unit, int R, int nmain, long long r1) {
+    if (first_of_unit) {
+      rr_lo = rr;
+      rr_hi = (int)min((long long)nmain, r1 - (long long)unit * R);
+    }
+  }
+  template <int RPC>
+  __device__ __forceinline__ bool starts(int rr) const { return rr < rr_hi && (rr - rr_lo) % RPC == 0; }
+  template <int RPC>
+  __device__ __forceinline__ bool ends(int rr) const {
+    return rr < rr_hi && ((rr - rr_lo) % RPC == RPC - 1 || rr == rr_hi - 1);
+  }
+  template <int RPC>
+  __device__ __forceinline__ int first_round(int rr) const { return rr - (rr - rr_lo) % RPC; }
+  template <int RPC>
+  __device__ __forceinline__ int last_round(int rr) const { return min(first_round<RPC>(rr) + RPC, rr_hi) - 1; }
 };
 
 // The work of round r (global index) of a launch.
@@ -157,31 +189,37 @@ __device__ __forceinline__ void dq_qz_word(uint32_t w, const __half2 (&nz)[4], u
 template <int NP, int BN, bool F8>
 __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_constant__ DqArgs P) {
   static_assert(!F8 || NP == 2, "fp8 mode: gate/up");
+  static_assert(BN == 16 || BN == 32, "16 or 32 items per tile");
   using C = DqCfg<NP, BN>;
-  constexpr int HC = BN / 2;  // accumulator columns per decode warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
-  uint64_t *empty = full + C::NS;
-  uint64_t *a_full = empty + C::NS;   // [2]
+  uint64_t *b_full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);  // [NB] activations of a round
+  uint64_t *b_empty = b_full + C::NB;
+  uint64_t *c_full = b_empty + C::NB;  // [NC] code chunks
+  uint64_t *c_empty = c_full + C::NC;
+  uint64_t *a_full = c_empty + C::NC;  // [2]
   uint64_t *mma_done = a_full + 2;    // [2]
   uint64_t *drain = mma_done + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
-  int *fin = flag + 1;  // [BN]: combine, this CTA's slot was its token's last of the row block
-  float *xbuf = reinterpret_cast<float *>(smem + C::XBUF_OFF);
+  int *fin_tok = flag + 1;  // [BN]: combine, this CTA's slot was its token's last of the row block
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  auto st_b = [&](int s) { return smem + s * C::STAGE; };
-  auto st_codes = [&](int s, int sl) { return smem + s * C::STAGE + C::B_BYTES + sl * 4096; };
-  auto st_sz = [&](int s, int sl) {
-    return reinterpret_cast<const uint32_t *>(smem + s * C::STAGE + C::B_BYTES + C::CODES) + sl * 128;
+  auto st_b = [&](int s) { return smem + s * C::B_BYTES; };
+  // code chunk slot c: [projection][CB blocks of 4 KB], then [projection][CB groups of 128 (scale, zero) words]
+  auto ch_codes = [&](int c, int p) { return smem + C::CODE_OFF + c * C::CODE_SLOT + p * C::CB * 4096; };
+  auto ch_sz = [&](int c, int p) {
+    return reinterpret_cast<uint32_t *>(smem + C::CODE_OFF + c * C::CODE_SLOT + NP * C::CB * 4096) + p * C::CB * 128;
   };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], DQ_DW);
+    for (int s = 0; s < C::NB; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], DQ_DW);
+    }
+    for (int c = 0; c < C::NC; ++c) {
+      mbar_init(&c_full[c], 1);
+      mbar_init(&c_empty[c], DQ_DW);
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(&a_full[j], DQ_DW);
@@ -220,56 +258,75 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
       int i = 0;
       RoundCursor<NP> cur;
       cur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
+      ChunkTrack ck;
+      int cur_jt = -1;
+      int4 cur_tile = make_int4(0, 0, 0, 0);
       for (; i < nr; ++i, cur.advance()) {
-        const int s = i % C::NS;
-        if (i >= C::NS && !(ok = mbar_wait(&empty[s], ((i / C::NS) - 1) & 1, P.status))) break;
         const Round rd = cur.get();
-        const int4 t = P.tiles[rd.jt];
-        const int grp = t.x, item0 = t.y;
+        ck.on_round<C::RPC>(i == 0 || rd.rr == 0, rd.rr, rd.unit, R, nmain, r1);
+        if (rd.jt != cur_jt) {  // the tile changes with the unit only
+          cur_jt = rd.jt;
+          cur_tile = P.tiles[rd.jt];
+        }
+        const int grp = cur_tile.x, item0 = cur_tile.y;
+        if (!rd.ext && ck.starts<C::RPC>(rd.rr)) {
+          // the next code chunk: rounds first .. last of this unit
+          const int c = ck.n % C::NC;
+          if (ck.n >= C::NC && !(ok = mbar_wait(&c_empty[c], ((ck.n / C::NC) - 1) & 1, P.status))) break;
+          const int r_a = rd.rr, r_b = ck.last_round<C::RPC>(rd.rr) + 1;
+          const int kb_a = NP == 2 ? r_a : 2 * r_a, kb_b = NP == 2 ? r_b : min(nkb, 2 * r_b);
+          const int g_a = (kb_a * 128) / P.group, g_b = ((kb_b - 1) * 128) / P.group;
+          const uint32_t cbytes = (uint32_t)(kb_b - kb_a) * 4096, zbytes = (uint32_t)(g_b - g_a + 1) * 512;
+          mbar_arrive_expect_tx(&c_full[c], NP * (cbytes + zbytes));
+          for (int p = 0; p < NP; ++p) {
+            const size_t blk = ((size_t)grp * P.m_tiles + rd.ob) * nkb + kb_a;
+            bulk_g2s(ch_codes(c, p), reinterpret_cast<const uint8_t *>(P.codes[p]) + blk * 4096, cbytes, &c_full[c]);
+            const size_t zoff = (((size_t)grp * P.m_tiles + rd.ob) * G + g_a) * 128;
+            bulk_g2s(ch_sz(c, p), P.sz[p] + zoff, zbytes, &c_full[c]);
+          }
+          ++ck.n;
+        }
+        // the round's activation tile
+        const int s = i % C::NB;
+        if (i >= C::NB && !(ok = mbar_wait(&b_empty[s], ((i / C::NB) - 1) & 1, P.status))) break;
         uint8_t *bs = st_b(s);
         if (!rd.ext) {
-          uint32_t bytes = 0;
           int na = 0;
           for (int sl = 0; sl < 2; ++sl)
-            if (rd.valid[sl]) {
-              bytes += 4096 + 512;
-              na += NP == 2 ? (sl == 0 ? 2 : 0) : 2;
-            }
-          mbar_arrive_expect_tx(&full[s], bytes + (uint32_t)na * C::ATOM);
+            if (rd.valid[sl]) na += (NP == 2 || F8) ? (sl == 0 ? 2 : 0) : 2;
+          mbar_arrive_expect_tx(&b_full[s], (uint32_t)na * C::ATOM);
           for (int sl = 0; sl < 2; ++sl) {
             if (!rd.valid[sl]) continue;
-            const int p = NP == 2 ? sl : 0, kb = rd.kb[sl];
-            const size_t blk = ((size_t)grp * P.m_tiles + rd.ob) * nkb + kb;
-            bulk_g2s(st_codes(s, sl), reinterpret_cast<const uint8_t *>(P.codes[p]) + blk * 4096, 4096, &full[s]);
-            const size_t zoff = (((size_t)grp * P.m_tiles + rd.ob) * G + (kb * 128) / P.group) * 128;
-            bulk_g2s(const_cast<uint32_t *>(st_sz(s, sl)), P.sz[p] + zoff, 512, &full[s]);
+            const int kb = rd.kb[sl];
             if (F8) {
               // the two e4m3 pieces of the 128 K of this block (one 128-byte box each)
               if (sl == 0)
                 for (int pc = 0; pc < 2; ++pc)
-                  tc::tma_load_2d(bs + pc * C::ATOM, &P.bmap, pc * P.d_in + kb * 128, item0, &full[s]);
+                  tc::tma_load_2d(bs + pc * C::ATOM, &P.bmap, pc * P.d_in + kb * 128, item0, &b_full[s]);
             } else if (NP == 1 || sl == 0) {
               for (int a = 0; a < 2; ++a)
-                tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, &P.bmap, kb * 128 + a * 64, item0, &full[s]);
+                tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, &P.bmap, kb * 128 + a * 64, item0, &b_full[s]);
             }
           }
         } else {
           int na = 0;
           for (int sl = 0; sl < 2; ++sl)
             if (rd.valid[sl]) na += (min(128, P.rank - rd.chunk[sl] * 128) + 63) / 64;
-          mbar_arrive_expect_tx(&full[s], (uint32_t)na * C::ATOM);
+          mbar_arrive_expect_tx(&b_full[s], (uint32_t)na * C::ATOM);
           for (int sl = 0; sl < 2; ++sl) {
             if (!rd.valid[sl]) continue;
             const int p = NP == 2 ? sl : 0;
             const int len = min(128, P.rank - rd.chunk[sl] * 128);
             for (int a = 0; a * 64 < len; ++a)
               tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, F8 ? &P.bmap_ext : &P.bmap,
-                              P.ext_col[p] + rd.chunk[sl] * 128 + a * 64, item0, &full[s]);
+                              P.ext_col[p] + rd.chunk[sl] * 128 + a * 64, item0, &b_full[s]);
           }
         }
       }
       // no copy may still be landing in shared memory when the CTA exits
-      for (int j = i > C::NS ? i - C::NS : 0; j < i; ++j) mbar_wait(&full[j % C::NS], (j / C::NS) & 1, P.status);
+      for (int j = i > C::NB ? i - C::NB : 0; j < i; ++j) mbar_wait(&b_full[j % C::NB], (j / C::NB) & 1, P.status);
+      for (int j = ck.n > C::NC ? ck.n - C::NC : 0; j < ck.n; ++j)
+        mbar_wait(&c_full[j % C::NC], (j / C::NC) & 1, P.status);
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
@@ -279,10 +336,11 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
     for (int i = 0; i < nr; ++i, cur.advance()) {
       const int as = i & 1;
       if (!(ok = mbar_wait(&a_full[as], (i >> 1) & 1, P.status))) break;
+      if (!(ok = mbar_wait(&b_full[i % C::NB], (i / C::NB) & 1, P.status))) break;
       tc::fence_after();
       const Round rd = cur.get();
       if (tc::elect_one()) {
-        const uint64_t bd0 = tc::sdesc_sw128(smem_addr(st_b(i % C::NS)));
+        const uint64_t bd0 = tc::sdesc_sw128(smem_addr(st_b(i % C::NB)));
         const uint32_t a0 = tmem + as * 128, d0 = tmem + C::ACC0 + as * C::ACC_COLS;
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
@@ -312,241 +370,265 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
     mbar_wait(drain, 0, P.status);
   } else {
     // ============================================================ decode + epilogue
+    // One warp per TMEM lane quadrant (32 weight rows): it decodes both slices
+    // of every round (256 weights per thread) and holds both accumulators in
+    // registers, so a unit's two slices meet in the same thread.
     const int dw = warp - 2;
-    const int sub = dw >> 2;            // 0..3
-    const int sl = sub >> 1;            // slice
-    const int part = sub & 1;           // K half (decode) / column half (epilogue)
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = tc::lane_base(warp);
-    float acc[HC];
+    float acc0[BN], acc1[BN];  // np = 2: gate, up; np = 1: the two slices' partial sums
 #pragma unroll
-    for (int c = 0; c < HC; ++c) acc[c] = 0.f;
-    float sc0 = 0.f, sc1 = 0.f;  // this row's scale of the warp's slice in the rounds of even / odd index
-    bool v0 = false, v1 = false;  // the warp's slice was valid in the last round of even / odd index
+    for (int c = 0; c < BN; ++c) {
+      acc0[c] = 0.f;
+      acc1[c] = 0.f;
+    }
+    // per round parity (e: even index, o: odd): this row's scale of each slice and whether the slice was valid
+    float sce0 = 0.f, sce1 = 0.f, sco0 = 0.f, sco1 = 0.f;
+    bool vde0 = false, vde1 = false, vdo0 = false, vdo1 = false;
 
-    // ---- end of a unit's rounds in this CTA: combine the two slices, then
-    // store the result (whole unit) or a piece (unit cut between CTAs)
+    // ---- end of a unit's rounds in this CTA: store the result (whole unit) or
+    // a piece (unit cut between CTAs; the CTA finishing last sums them)
     auto unit_end = [&](const Round &rd) -> void {
       const long long ustart = (long long)rd.unit * R, uend = ustart + R;
       const bool whole = ustart >= r0 && uend <= r1;
       const int4 t = P.tiles[rd.jt];
       const int item0 = t.y, nitems = t.z;
       const int o = rd.ob * 128 + row;
-      named_sync(1, DQ_DW * 32);  // the previous unit's readers are done with xbuf
-      if (sl == 1)
-#pragma unroll
-        for (int c = 0; c < HC; ++c) xbuf[(part * HC + c) * 128 + row] = acc[c];
-      named_sync(1, DQ_DW * 32);
-      if (sl == 0) {
-        // the final result of item column n = part * HC + c: np = 2: silu(gate) * up * row scale (fp16),
-        // np = 1: the sum of both slices (fp32)
-        auto store = [&](int c, float g, float u) {
-          const int n = part * HC + c;
-          if (n >= nitems || o >= P.d_out) return;
-          if (F8) {  // the activations were scaled by 2^e per item
-            const float xs = __ldg(P.xs + item0 + n);
-            g *= xs;
-            u *= xs;
-          }
-          if (NP == 2 && P.epi == EPI_STORE2_F32) {
-            reinterpret_cast<float *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = g;
-            reinterpret_cast<float *>(P.out2)[(size_t)(item0 + n) * P.ldo + o] = u;
-          } else if (NP == 2) {
-            const float rs = P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f;
-            reinterpret_cast<__half *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = half_checked(silu_f(g) * u * rs, P.status);
-          } else {
-            reinterpret_cast<float *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = g;
-          }
-        };
-        if (whole) {
-#pragma unroll
-          for (int c = 0; c < HC; ++c) {
-            const float x = xbuf[(part * HC + c) * 128 + row];
-            store(c, NP == 2 ? acc[c] : acc[c] + x, x);
-          }
-        } else {
-          // piece of this CTA: slot 0 if the unit is the first of its range, else slot 1
-          const int slot = (ustart <= r0) ? 0 : 1;
-          float *pc = P.part + ((size_t)blockIdx.x * 2 + slot) * NP * BN * 128;
-#pragma unroll
-          for (int c = 0; c < HC; ++c) {
-            const int col = part * HC + c;
-            const float x = xbuf[col * 128 + row];
-            pc[col * 128 + row] = NP == 2 ? acc[c] : acc[c] + x;
-            if (NP == 2) pc[(BN + col) * 128 + row] = x;
-          }
-          __threadfence();
-          named_sync(2, DQ_DW * 16);
-          const int c_first = cta_of(ustart, total, gridDim.x), c_last = cta_of(uend - 1, total, gridDim.x);
-          // CTAs with an empty range (fewer rounds than CTAs) leave no piece
-          int pieces = 0;
-          for (int cc = c_first; cc <= c_last; ++cc)
-            pieces += range_begin(total, cc + 1, gridDim.x) > range_begin(total, cc, gridDim.x);
-          if (dw == 0 && lane == 0) *flag = atomicAdd(&P.counters[rd.unit], 1) == pieces - 1;
-          named_sync(2, DQ_DW * 16);
-          if (*flag) {
-            // the last piece in: sum all pieces of the unit in CTA order
-            __threadfence();
-#pragma unroll 1
-            for (int c = 0; c < HC; ++c) {
-              const int col = part * HC + c;
-              float g = 0.f, u = 0.f;
-              for (int cc = c_first; cc <= c_last; ++cc) {
-                const long long b = range_begin(total, cc, gridDim.x);
-                if (range_begin(total, cc + 1, gridDim.x) == b) continue;
-                const int s2 = (b / R == rd.unit) ? 0 : 1;  // the unit is cta cc's first (slot 0) or last
-                const float *q = P.part + ((size_t)cc * 2 + s2) * NP * BN * 128;
-                g += __ldcg(q + col * 128 + row);
-                if (NP == 2) u += __ldcg(q + (BN + col) * 128 + row);
-              }
-              store(c, g, u);
-            }
-            if (dw == 0 && lane == 0) P.counters[rd.unit] = 0;
-          }
+      // the final result of item column n: np = 2: silu(gate) * up * row scale (fp16) or both in
+      // fp32; np = 1: the sum of both slices (fp32)
+      auto store = [&](int n, float g, float u) {
+        if (n >= nitems || o >= P.d_out) return;
+        if (F8) {  // the activations were scaled by 2^e per item
+          const float xs = __ldg(P.xs + item0 + n);
+          g *= xs;
+          u *= xs;
         }
-        // weighted top-k combine: the slot weights are inside h, so the layer
-        // output of a token is the plain sum of its slots' rows
-        if (NP == 1 && P.combine && (whole || *flag)) {
+        if (NP == 2 && P.epi == EPI_STORE2_F32) {
+          reinterpret_cast<float *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = g;
+          reinterpret_cast<float *>(P.out2)[(size_t)(item0 + n) * P.ldo + o] = u;
+        } else if (NP == 2) {
+          const float rs = P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f;
+          reinterpret_cast<__half *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = half_checked(silu_f(g) * u * rs, P.status);
+        } else {
+          reinterpret_cast<float *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = g;
+        }
+      };
+      bool fin = whole;
+      if (whole) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) store(c, NP == 2 ? acc0[c] : acc0[c] + acc1[c], acc1[c]);
+      } else {
+        // piece of this CTA: slot 0 if the unit is the first of its range, else slot 1
+        const int slot = (ustart <= r0) ? 0 : 1;
+        float *pc = P.part + ((size_t)blockIdx.x * 2 + slot) * NP * BN * 128;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          pc[c * 128 + row] = NP == 2 ? acc0[c] : acc0[c] + acc1[c];
+          if (NP == 2) pc[(BN + c) * 128 + row] = acc1[c];
+        }
+        __threadfence();
+        named_sync(1, DQ_DW * 32);
+        const int c_first = cta_of(ustart, total, gridDim.x), c_last = cta_of(uend - 1, total, gridDim.x);
+        // CTAs with an empty range (fewer rounds than CTAs) leave no piece
+        int pieces = 0;
+        for (int cc = c_first; cc <= c_last; ++cc)
+          pieces += range_begin(total, cc + 1, gridDim.x) > range_begin(total, cc, gridDim.x);
+        if (dw == 0 && lane == 0) *flag = atomicAdd(&P.counters[rd.unit], 1) == pieces - 1;
+        named_sync(1, DQ_DW * 32);
+        fin = *flag != 0;
+        if (fin) {
+          // the last piece in: sum all pieces of the unit in CTA order
           __threadfence();
-          named_sync(2, DQ_DW * 16);
-          const int tid = dw * 32 + lane;  // 0 .. 255 over the slice-0 warps
-          if (tid < nitems) {
-            const int tok = __ldg(P.slot_tok + item0 + tid);
-            fin[tid] = atomicAdd(&P.tok_counters[tok * P.m_tiles + rd.ob], 1) == P.top_k - 1;
-          }
-          named_sync(2, DQ_DW * 16);
-          __threadfence();
-          const float *yb = reinterpret_cast<const float *>(P.out);
-          for (int n = 0; n < nitems; ++n) {
-            if (!fin[n]) continue;
-            const int tok = __ldg(P.slot_tok + item0 + n);
-            for (int r = tid; r < 128; r += DQ_DW * 16) {
-              const int oo = rd.ob * 128 + r;
-              if (oo >= P.d_out) continue;
-              float y = P.yshared ? __ldg(P.yshared + (size_t)tok * P.ldo + oo) : 0.f;
-              for (int j = 0; j < P.top_k; ++j)
-                y += __ldcg(yb + (size_t)__ldg(P.slot_of_pair + tok * P.top_k + j) * P.ldo + oo);
-              P.out_tok[(size_t)tok * P.ldo + oo] = __float2bfloat16_rn(y);
+#pragma unroll 1
+          for (int c = 0; c < BN; ++c) {
+            float g = 0.f, u = 0.f;
+            for (int cc = c_first; cc <= c_last; ++cc) {
+              const long long b = range_begin(total, cc, gridDim.x);
+              if (range_begin(total, cc + 1, gridDim.x) == b) continue;
+              const int s2 = (b / R == rd.unit) ? 0 : 1;  // the unit is cta cc's first (slot 0) or last
+              const float *q = P.part + ((size_t)cc * 2 + s2) * NP * BN * 128;
+              g += __ldcg(q + c * 128 + row);
+              if (NP == 2) u += __ldcg(q + (BN + c) * 128 + row);
             }
+            store(c, g, u);
           }
+          if (dw == 0 && lane == 0) P.counters[rd.unit] = 0;
         }
       }
+      // weighted top-k combine: the slot weights are inside h, so the layer
+      // output of a token is the plain sum of its slots' rows
+      if (NP == 1 && P.combine && fin) {
+        __threadfence();
+        named_sync(1, DQ_DW * 32);
+        const int tid = dw * 32 + lane;  // 0 .. 127
+        if (tid < nitems) {
+          const int tok = __ldg(P.slot_tok + item0 + tid);
+          fin_tok[tid] = atomicAdd(&P.tok_counters[tok * P.m_tiles + rd.ob], 1) == P.top_k - 1;
+        }
+        named_sync(1, DQ_DW * 32);
+        __threadfence();
+        const float *yb = reinterpret_cast<const float *>(P.out);
+        for (int n = 0; n < nitems; ++n) {
+          if (!fin_tok[n]) continue;
+          const int tok = __ldg(P.slot_tok + item0 + n);
+          const int oo = rd.ob * 128 + tid;
+          if (oo >= P.d_out) continue;
+          float y = P.yshared ? __ldg(P.yshared + (size_t)tok * P.ldo + oo) : 0.f;
+          for (int j = 0; j < P.top_k; ++j)
+            y += __ldcg(yb + (size_t)__ldg(P.slot_of_pair + tok * P.top_k + j) * P.ldo + oo);
+          P.out_tok[(size_t)tok * P.ldo + oo] = __float2bfloat16_rn(y);
+        }
+        named_sync(1, DQ_DW * 32);  // fin_tok is reused by the next unit
+      }
 #pragma unroll
-      for (int c = 0; c < HC; ++c) acc[c] = 0.f;
+      for (int c = 0; c < BN; ++c) {
+        acc0[c] = 0.f;
+        acc1[c] = 0.f;
+      }
     };
 
-    // ---- fold round j's accumulator (slot j & 1) into registers; release its stage
+    // fold one slice's accumulator (BN columns at TMEM column base) into acc
+    auto fold = [&](uint32_t base, float s, float (&acc)[BN]) {
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t d[16];
+        tc::ld16_nowait(base + c0, d);
+        tc::wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) acc[c0 + c] = fmaf(__uint_as_float(d[c]), s, acc[c0 + c]);
+      }
+    };
+
+    // ---- fold round j's accumulators (slot j & 1) into registers; release its stage
     // (rounds are finished in order: fcur is at round j)
     RoundCursor<NP> fcur;
     fcur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
     auto finish = [&](int j) -> bool {
       if (!mbar_wait(&mma_done[j & 1], (j >> 1) & 1, P.status)) return false;
       tc::fence_after();
-      const float sc = (j & 1) ? sc1 : sc0;
-      // tcgen05.ld is warp-collective: the decision is the warp's (its slice
+      const uint32_t base = tmem + lane_addr + C::ACC0 + (j & 1) * C::ACC_COLS;
+      // tcgen05.ld is warp-collective: the decision is the warp's (the slice
       // was valid in round j), never a lane's (padding rows have scale 0)
-      if ((j & 1) ? v1 : v0) {
-        const uint32_t base = tmem + lane_addr + C::ACC0 + (j & 1) * C::ACC_COLS + sl * BN + part * HC;
-#pragma unroll
-        for (int c0 = 0; c0 < HC; c0 += 16) {
-          uint32_t d[16];
-          if constexpr (HC >= 16) {
-            tc::ld16_nowait(base + c0, d);
-          } else {
-            float f[8];
-            tc::ld8(base, f);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) d[c] = __float_as_uint(f[c]);
-          }
-          tc::wait_ld();
-#pragma unroll
-          for (int c = 0; c < (HC < 16 ? HC : 16); ++c) acc[c0 + c] = fmaf(__uint_as_float(d[c]), sc, acc[c0 + c]);
-        }
-      }
+      const bool odd = j & 1;
+      if (odd ? vdo0 : vde0) fold(base, odd ? sco0 : sce0, acc0);
+      if (odd ? vdo1 : vde1) fold(base + BN, odd ? sco1 : sce1, acc1);
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[j % C::NS]);
+      if (lane == 0) mbar_arrive(&b_empty[j % C::NB]);
       const Round rd = fcur.get();  // round j
       fcur.advance();
       if (rd.rr == R - 1 || j == nr - 1) unit_end(rd);
       return true;
     };
 
-    RoundCursor<NP> cur;
-    cur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
-    for (int i = 0; i < nr && ok; ++i, cur.advance()) {
-      const int s = i % C::NS;
-      if (!(ok = mbar_wait(&full[s], (i / C::NS) & 1, P.status))) break;
-      // round i - 2: fold its accumulator; its A slot is then free for round i
-      if (i >= 2 && !(ok = finish(i - 2))) break;
-      const Round rd = cur.get();
-      const bool mine = sl ? rd.valid[1] : rd.valid[0];
-      const int chunk = sl ? rd.chunk[1] : rd.chunk[0];
-      uint32_t v[32];
-      float sc = 0.f;
-      if (mine && !rd.ext) {
-        // codes of this slice's K half: K slices 2 part and 2 part + 1 of the 4 x 32 layout
-        const uint8_t *cb = st_codes(s, sl);
-        uint32_t w[4];
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n"
-                     : "=r"(w[0]), "=r"(w[1])
-                     : "r"(smem_addr(cb + (2 * part) * 1024 + row * 8)));
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n"
-                     : "=r"(w[2]), "=r"(w[3])
-                     : "r"(smem_addr(cb + (2 * part + 1) * 1024 + row * 8)));
-        const __half2 szw = u32_as_h2(st_sz(s, sl)[row]);
+    // ---- one slice of round i into the A slot: decode (main) or U_m rows (extension)
+    auto load_slice = [&](const Round &rd, int c, int kb_a, int g_a, int sl, int i, float &scale) {
+      const uint32_t acol = tmem + lane_addr + (i & 1) * 128 + sl * 64;
+      if (!rd.ext) {
+        const int p = NP == 2 ? sl : 0, kb = sl ? rd.kb[1] : rd.kb[0];
+        const uint8_t *cb = ch_codes(c, p) + (kb - kb_a) * 4096;
+        const __half2 szw = u32_as_h2(ch_sz(c, p)[((kb * 128) / P.group - g_a) * 128 + row]);
+        scale = __low2float(szw);
         if constexpr (F8) {
           // e4m3 (q - z) through a 4-entry byte table per zero point: one PRMT per 4 weights
           const int zi = (int)__high2float(szw);
           const uint32_t tab = zi == 0 ? 0x44403800u : zi == 1 ? 0x403800B8u : zi == 2 ? 0x3800B8C0u : 0x00B8C0C4u;
+          uint32_t v[32];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t c0 = w[q] & 0x33333333u, c1 = (w[q] >> 2) & 0x33333333u;
-            v[4 * q + 0] = __byte_perm(tab, 0, c0);
-            v[4 * q + 1] = __byte_perm(tab, 0, c0 >> 16);
-            v[4 * q + 2] = __byte_perm(tab, 0, c1);
-            v[4 * q + 3] = __byte_perm(tab, 0, c1 >> 16);
+          for (int ks = 0; ks < 4; ++ks) {  // the four K slices of 32 (two words of 16 codes each)
+            uint32_t w0, w1;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(w0), "=r"(w1) : "r"(smem_addr(cb + ks * 1024 + row * 8)));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t w = h ? w1 : w0;
+              const uint32_t c0 = w & 0x33333333u, c1 = (w >> 2) & 0x33333333u;
+              uint32_t *o = v + 8 * ks + 4 * h;
+              o[0] = __byte_perm(tab, 0, c0);
+              o[1] = __byte_perm(tab, 0, c0 >> 16);
+              o[2] = __byte_perm(tab, 0, c1);
+              o[3] = __byte_perm(tab, 0, c1 >> 16);
+            }
           }
+          tc::st32(acol, v);
         } else {
           const __half2 z2 = __high2half2(szw);
           const __half2 nz[4] = {__hsub2(__float2half2_rn(-1024.f), z2), __hsub2(__float2half2_rn(-256.f), z2),
                                  __hsub2(__float2half2_rn(-64.f), z2), __hsub2(__float2half2_rn(-16.f), z2)};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) dq_qz_word(w[q], nz, v + 8 * q);
+          for (int hk = 0; hk < 2; ++hk) {  // K halves of 64: 32 TMEM columns each
+            uint32_t v[32];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              uint32_t w0, w1;
+              asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n"
+                           : "=r"(w0), "=r"(w1)
+                           : "r"(smem_addr(cb + (2 * hk + q) * 1024 + row * 8)));
+              dq_qz_word(w0, nz, v + 16 * q);
+              dq_qz_word(w1, nz, v + 16 * q + 8);
+            }
+            tc::st32(acol + hk * 32, v);
+          }
         }
-        sc = __low2float(szw);
-      } else if (mine) {
-        // rows of U_m: rank columns chunk * 128 + part * 64 ..
+      } else {
+        // rows of U_m: rank columns chunk * 128 ..
         const int4 t = P.tiles[rd.jt];
         const int p = NP == 2 ? sl : 0;
-        const __half *ur =
-            P.u[p] + (((size_t)P.u_blk[p][t.x] * P.m_tiles + rd.ob) * 128 + row) * P.rank + chunk * 128 + part * 64;
-        const int kmax = P.rank - chunk * 128 - part * 64;
+        const int chunk = sl ? rd.chunk[1] : rd.chunk[0];
+        const __half *ur = P.u[p] + (((size_t)P.u_blk[p][t.x] * P.m_tiles + rd.ob) * 128 + row) * P.rank + chunk * 128;
+        const int kmax = P.rank - chunk * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint4 q4 = make_uint4(0, 0, 0, 0);
-          if (j * 8 < kmax) q4 = __ldg(reinterpret_cast<const uint4 *>(ur + j * 8));
-          v[4 * j + 0] = q4.x;
-          v[4 * j + 1] = q4.y;
-          v[4 * j + 2] = q4.z;
-          v[4 * j + 3] = q4.w;
+        for (int hk = 0; hk < 2; ++hk) {
+          uint32_t v[32];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint4 q4 = make_uint4(0, 0, 0, 0);
+            if (hk * 64 + j * 8 < kmax) q4 = __ldg(reinterpret_cast<const uint4 *>(ur + hk * 64 + j * 8));
+            v[4 * j + 0] = q4.x;
+            v[4 * j + 1] = q4.y;
+            v[4 * j + 2] = q4.z;
+            v[4 * j + 3] = q4.w;
+          }
+          tc::st32(acol + hk * 32, v);
         }
-        sc = 1.f;
+        scale = 1.f;
       }
-      if (mine) {
-        if (F8 && !rd.ext) {
-          tc::st16(tmem + lane_addr + (i & 1) * 128 + sl * 64 + part * 16, *reinterpret_cast<uint32_t(*)[16]>(v));
-        } else {
-          tc::st32(tmem + lane_addr + (i & 1) * 128 + sl * 64 + part * 32, v);
-        }
-        tc::wait_st();
+    };
+
+    RoundCursor<NP> cur;
+    cur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
+    ChunkTrack ck;
+    int c = 0, kb_a = 0, g_a = 0;  // the current code chunk: ring slot, first block, first group
+    for (int i = 0; i < nr && ok; ++i, cur.advance()) {
+      const Round rd = cur.get();
+      ck.on_round<C::RPC>(i == 0 || rd.rr == 0, rd.rr, rd.unit, R, nmain, r1);
+      if (!rd.ext && ck.starts<C::RPC>(rd.rr)) {
+        c = ck.n % C::NC;
+        kb_a = NP == 2 ? rd.rr : 2 * rd.rr;
+        g_a = (kb_a * 128) / P.group;
+        if (!(ok = mbar_wait(&c_full[c], (ck.n / C::NC) & 1, P.status))) break;
+        ++ck.n;
       }
+      // round i - 2: fold its accumulators; its A slot is then free for round i
+      if (i >= 2 && !(ok = finish(i - 2))) break;
+      float s0 = 0.f, s1 = 0.f;
+      if (rd.valid[0]) load_slice(rd, c, kb_a, g_a, 0, i, s0);
+      if (rd.valid[1]) load_slice(rd, c, kb_a, g_a, 1, i, s1);
+      // the chunk's codes are decoded: the producer may refill its slot
+      if (!rd.ext && ck.ends<C::RPC>(rd.rr)) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c_empty[c]);
+      }
+      tc::wait_st();
       if (i & 1) {
-        sc1 = sc;
-        v1 = mine;
+        sco0 = s0;
+        sco1 = s1;
+        vdo0 = rd.valid[0];
+        vdo1 = rd.valid[1];
       } else {
-        sc0 = sc;
-        v0 = mine;
+        sce0 = s0;
+        sce1 = s1;
+        vde0 = rd.valid[0];
+        vde1 = rd.valid[1];
       }
       tc::fence_before();
       __syncwarp();
@@ -594,17 +676,14 @@ cudaError_t launch_gemm_dq(const DqArgs &a, int np, int bn, cudaStream_t stream)
     switch (bn) {
       case 16: return launch_dq<2, 16, true>(a, stream);
       case 32: return launch_dq<2, 32, true>(a, stream);
-      case 64: return launch_dq<2, 64, true>(a, stream);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (bn * 4 + np) {
     case 16 * 4 + 1: return launch_dq<1, 16>(a, stream);
     case 32 * 4 + 1: return launch_dq<1, 32>(a, stream);
-    case 64 * 4 + 1: return launch_dq<1, 64>(a, stream);
     case 16 * 4 + 2: return launch_dq<2, 16>(a, stream);
     case 32 * 4 + 2: return launch_dq<2, 32>(a, stream);
-    case 64 * 4 + 2: return launch_dq<2, 64>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }
