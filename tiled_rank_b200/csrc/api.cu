@@ -264,6 +264,11 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   // has 2-bit codes in groups of a multiple of 128; otherwise warp-level MMA
   bool dq_ok = !use_tc;
   for (int p = 0; p < li.nproj; ++p) dq_ok = dq_ok && li.p[p].bits == 2 && li.p[p].group % 128 == 0;
+  if (dq_ok) {
+    const int bn = choose_bn_dq(avg), slots = cdiv(P, bn) + L->K;
+    for (int p = 0; p < li.nproj; ++p)
+      dq_ok = dq_ok && dq_fits(slots, cdiv(li.p[p].d_out, 128), li.p[p].d_in, li.p[p].rank);
+  }
   pl.bn_main = use_tc ? choose_bn_tc(avg) : (dq_ok ? choose_bn_dq(avg) : choose_bn(avg));
   pl.slots_main = cdiv(P, pl.bn_main) + L->K;
   const long long est_main = std::min(L->K, P) + P / pl.bn_main;
@@ -755,6 +760,7 @@ tileq_status run_residual_dq(const Residual &r, const GemmPlan &g, const LayerIn
   }
   a.tiles = at<int4>(ws, w.tiles_main);
   a.tile_count = at<int>(ws, w.tile_counts);
+  a.max_tiles = g.slots;
   a.m_tiles = g.m_tiles;
   a.d_out = q.d_out;
   a.d_in = q.d_in;

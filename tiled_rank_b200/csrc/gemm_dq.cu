@@ -10,12 +10,10 @@
 //     to tensor memory; the tensor cores do every multiply (TS-form
 //     tcgen05.mma, M = 128 weight rows, N = 16..64 items);
 //   * every 128-wide K block (one scale group, or part of one) accumulates
-//     into its own fp32 accumulator in tensor memory; the decoding warps fold
-//     it into registers with the group scale two rounds later (w = s*(q - z)
-//     is never rounded);
+//     into its own fp32 accumulator in tensor memory; the fold warps add it
+//     into registers with the group scale (w = s*(q - z) is never rounded);
 //   * a round = two slices of 128 K: gate and up of one K block (np = 2) or
-//     two consecutive K blocks of one projection (np = 1); the MMA warp waits
-//     on one barrier and commits once per round;
+//     two consecutive K blocks of one projection (np = 1);
 //   * stream-K: the (tile, row block, round) space is cut into gridDim.x equal
 //     contiguous ranges, one per CTA (one CTA per SM).  A (tile, row block)
 //     unit cut between CTAs leaves fp32 pieces that the CTA finishing last
@@ -25,14 +23,19 @@
 // slot holds rows of the grid row's U_m (fp16, read from global memory) and B
 // the matching z (or a) columns of the item rows, with scale 1.
 //
-// Warp roles (6 warps): warp 0 producer (bulk copies of the codes and their
-// (scale, zero) words in chunks of up to 8 K blocks per projection into a
-// ring of chunk slots, 2-D TMA boxes of B per round into a ring of its own), warp 1 MMA
-// issuer (the whole warp waits, one elected lane issues and commits), warps
-// 2..5 decode and epilogue: warp w works on TMEM lane quadrant w % 4 (32
-// weight rows) and both slices of every round (256 weights per thread and
-// round, so that each barrier round amortises over enough decode work), with
-// both slices' accumulators in its registers.
+// Warp roles (14 warps), each a pipeline stage with its own ring, so that a
+// round costs the slowest stage rather than the sum of all of them:
+//   warp 0      producer: bulk copies of the codes and their (scale, zero)
+//               words in chunks of 4 K blocks per projection (code ring), 2-D
+//               TMA boxes of B per round (activation ring);
+//   warp 1      MMA issuer: waits for a round's operand slot; one elected lane
+//               issues and commits to the operand slot, the activation stage
+//               and the accumulator;
+//   warps 2..9  decode: two warps per TMEM lane quadrant (32 weight rows), one
+//               per slice, write every round into its operand slot once its
+//               activations have landed and its accumulator slot is free;
+//   warps 10..13 fold + epilogue: one warp per lane quadrant folds every
+//               round's accumulators with the group scales and stores units.
 // Every wait is bounded and reports TILEQ_ERR_TIMEOUT.
 #include "kernels.cuh"
 #include "tc.cuh"
@@ -41,121 +44,101 @@ namespace tileq {
 
 namespace {
 
-constexpr int DQ_DW = 4;                      // decode / epilogue warps (one per TMEM lane quadrant)
-constexpr int DQ_THREADS = (2 + DQ_DW) * 32;  // + producer + MMA issuer
-constexpr int DQ_GRID = 148;                  // one CTA per SM
+constexpr int DQ_DEC = 8;                             // decode warps: two per TMEM lane quadrant (one per slice)
+constexpr int DQ_FW = 4;                              // fold / epilogue warps: one per lane quadrant
+constexpr int DQ_THREADS = (2 + DQ_DEC + DQ_FW) * 32;  // + producer + MMA issuer
+constexpr int DQ_GRID = 148;                          // one CTA per SM
+constexpr int DQ_MAX_ROUNDS = 1024;                   // rounds of one CTA (its descriptor table)
 
 template <int NP, int BN>
 struct DqCfg {
   static constexpr int ATOM = BN * 128;                // one 64-wide fp16 K atom of B: BN rows x 128 B
   static constexpr int B_BYTES = 4 * ATOM;             // up to four atoms per round
-  // The codes stream from HBM in chunks of up to CB consecutive 128-wide K
-  // blocks per projection (one bulk copy of up to 32 KB each, with the
-  // (scale, zero) words of their groups): a few large copies in flight keep
-  // the weight stream at the HBM rate, where one 4 KB copy per block does not.
-  static constexpr int CB = 8;
+  // The codes stream from HBM in chunks of CB consecutive 128-wide K blocks
+  // per projection (one bulk copy each, with the (scale, zero) words of their
+  // groups), several chunks in flight.
+  static constexpr int CB = 4;
   static constexpr int RPC = NP == 2 ? CB : CB / 2;     // main rounds per chunk
   static constexpr int CODE_SLOT = NP * CB * (4096 + 512);
   static constexpr int NB = 4;                         // activation ring (per round, from L2)
-  static constexpr int NC_RAW = (210 * 1024 - NB * B_BYTES) / CODE_SLOT;
-  static constexpr int NC = NC_RAW > 4 ? 4 : NC_RAW;   // code chunk ring
+  static constexpr int NC_RAW = (200 * 1024 - NB * B_BYTES) / CODE_SLOT;
+  static constexpr int NC = NC_RAW > 6 ? 6 : NC_RAW;   // code chunk ring
   static constexpr int CODE_OFF = NB * B_BYTES;
-  static constexpr int BAR_OFF = CODE_OFF + NC * CODE_SLOT;
-  static constexpr int SMEM = BAR_OFF + (2 * NB + 2 * NC + 5) * 8 + 16 + BN * 4 + 1024;  // + slack to align the base
-  static constexpr int ACC_COLS = 2 * BN;             // one accumulator slot: two slices
-  static constexpr int ACC0 = 256;                     // TMEM: A slots at 0 and 128, accumulators from 256
-  static_assert(NC >= 2, "code ring too shallow");
-  static_assert(ACC0 + 2 * ACC_COLS <= 512, "tensor memory");
+  static constexpr int MAX_KB = 256;                   // K blocks of 128 (d_in up to 32768)
+  static constexpr int GIDX_OFF = CODE_OFF + NC * CODE_SLOT;  // [MAX_KB] scale group of each K block
+  static constexpr int TAB_OFF = GIDX_OFF + MAX_KB * 4;  // [DQ_MAX_ROUNDS] round descriptors
+  static constexpr int BAR_OFF = TAB_OFF + DQ_MAX_ROUNDS * 8;
+  // Tensor memory: NA operand slots of one round (two slices of 64 columns),
+  // then NT accumulator slots of one round (two slices of BN columns).
+  static constexpr int NT = 4;
+  static constexpr int ACC_COLS = 2 * BN;
+  static constexpr int A_COLS = 128;
+  static constexpr int NA_RAW = (512 - NT * ACC_COLS) / A_COLS;
+  static constexpr int NA = NA_RAW > 4 ? 4 : NA_RAW;
+  static constexpr int ACC0 = NA * A_COLS;
+  static constexpr int NBAR = 2 * NB + 2 * NC + 2 * NA + 2 * NT + 1;
+  static constexpr int SMEM = BAR_OFF + NBAR * 8 + 16 + BN * 4 + 1024;  // + slack to align the base
+  static_assert(NC >= 3, "code ring too shallow");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(NA >= 2, "operand ring too shallow");
+  static_assert(ACC0 + NT * ACC_COLS <= 512, "tensor memory");
   static_assert(ATOM % 1024 == 0, "swizzled atoms need 1024-byte alignment");
 };
 
-// Where a CTA's main rounds of one unit start new code chunks: chunks hold
-// RPC consecutive main rounds from the first main round the CTA processes in
-// the unit, up to its last one.  Producer and consumers step it the same way.
-struct ChunkTrack {
-  int rr_lo = 0, rr_hi = 0;  // main rounds [rr_lo, rr_hi) of the current unit in this CTA
-  int n = 0;                 // chunks started so far
-  template <int RPC>
-  __device__ __forceinline__ void on_round(bool first_of_unit, int rr, int unit, int R, int nmain, long long r1) {
-    if (first_of_unit) {
-      rr_lo = rr;
-      rr_hi = (int)min((long long)nmain, r1 - (long long)unit * R);
+// Bounded wait that lets the hardware suspend the warp until the phase
+// completes (or the hint elapses) instead of spinning on the issue slots the
+// decoding warps need.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, int *status) {
+  auto try_once = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(0x100000u)
+        : "memory");
+    return ok != 0;
+  };
+  if (try_once()) return true;
+  const long long t0 = clock64();
+  while (!try_once()) {
+    if (clock64() - t0 > kWaitLimitCycles) {
+      set_status(status, TILEQ_ERR_TIMEOUT);
+      return false;
     }
   }
-  template <int RPC>
-  __device__ __forceinline__ bool starts(int rr) const { return rr < rr_hi && (rr - rr_lo) % RPC == 0; }
-  template <int RPC>
-  __device__ __forceinline__ bool ends(int rr) const {
-    return rr < rr_hi && ((rr - rr_lo) % RPC == RPC - 1 || rr == rr_hi - 1);
-  }
-  template <int RPC>
-  __device__ __forceinline__ int first_round(int rr) const { return rr - (rr - rr_lo) % RPC; }
-  template <int RPC>
-  __device__ __forceinline__ int last_round(int rr) const { return min(first_round<RPC>(rr) + RPC, rr_hi) - 1; }
-};
+  return true;
+}
 
-// The work of round r (global index) of a launch.
-struct Round {
-  int unit, rr, jt, ob;
-  bool ext;
-  bool valid[2];
-  int kb[2];     // main rounds: the K block of each slice
-  int chunk[2];  // extension rounds: the 128-wide rank chunk of each slice
-  int nk[2];     // 16-wide K steps of each slice
-};
+// Non-blocking probe of a phase (the result is consumed later, so its latency
+// overlaps other work).
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 
-// Walks the rounds of a CTA's range in order without divisions: one division
-// places it at the range's first round, then each advance is a few compares.
-template <int NP>
-struct RoundCursor {
-  int unit, rr, jt, ob;
-  int R, nmain, nkb, m_tiles, rank;
-  __device__ __forceinline__ void init(long long r, int R_, int nmain_, int nkb_, int m_tiles_, int rank_) {
-    R = R_;
-    nmain = nmain_;
-    nkb = nkb_;
-    m_tiles = m_tiles_;
-    rank = rank_;
-    unit = (int)(r / R);
-    rr = (int)(r - (long long)unit * R);
-    jt = unit / m_tiles;
-    ob = unit - jt * m_tiles;
-  }
-  __device__ __forceinline__ void advance() {
-    if (++rr == R) {
-      rr = 0;
-      ++unit;
-      if (++ob == m_tiles) {
-        ob = 0;
-        ++jt;
-      }
-    }
-  }
-  __device__ __forceinline__ Round get() const {
-    Round o;
-    o.unit = unit;
-    o.rr = rr;
-    o.jt = jt;
-    o.ob = ob;
-    o.ext = rr >= nmain;
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      if (!o.ext) {
-        o.kb[s] = NP == 2 ? rr : 2 * rr + s;
-        o.valid[s] = o.kb[s] < nkb;
-        o.chunk[s] = 0;
-        o.nk[s] = 8;
-      } else {
-        const int e = rr - nmain;
-        o.chunk[s] = NP == 2 ? e : 2 * e + s;
-        o.valid[s] = o.chunk[s] * 128 < rank;
-        o.kb[s] = 0;
-        o.nk[s] = o.valid[s] ? (min(128, rank - o.chunk[s] * 128) + 15) / 16 : 0;
-      }
-    }
-    return o;
-  }
+// Per-round descriptor, one table per CTA built before the pipeline starts
+// (x: flags below; y: unit << 9 | round within the unit), so that no warp
+// walks the round space or waits for a descriptor.
+enum : uint32_t {
+  RD_EXT = 1u,         // U_m extension round
+  RD_V0 = 2u,          // slice 0 valid
+  RD_V1 = 4u,          // slice 1 valid
+  RD_CSTART = 8u,      // first round of a code chunk
+  RD_CEND = 16u,       // last round of a code chunk
+  RD_UEND = 32u,       // last round of the unit in this CTA
+  // bits 8..10 chunk ring slot, bit 11 its fill parity; bits 12..15 / 16..19:
+  // 16-wide K steps of each slice (extension); bits 20..23: K block of each
+  // slice within the chunk; bits 24..27: scale group of each slice within the
+  // chunk; bits 28..29 / 30..31: rank chunk of each slice (extension)
 };
+__device__ __forceinline__ uint32_t rd_field(uint32_t f, int lo, int bits) { return (f >> lo) & ((1u << bits) - 1u); }
 
 // First round of CTA c's range of `total` rounds over `g` CTAs.
 __device__ __forceinline__ long long range_begin(long long total, int c, int g) { return total * c / g; }
@@ -197,12 +180,16 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
   uint64_t *b_empty = b_full + C::NB;
   uint64_t *c_full = b_empty + C::NB;  // [NC] code chunks
   uint64_t *c_empty = c_full + C::NC;
-  uint64_t *a_full = c_empty + C::NC;  // [2]
-  uint64_t *mma_done = a_full + 2;    // [2]
-  uint64_t *drain = mma_done + 2;
+  uint64_t *a_full = c_empty + C::NC;  // [NA] operand slots
+  uint64_t *a_free = a_full + C::NA;
+  uint64_t *acc_full = a_free + C::NA;  // [NT] accumulator slots
+  uint64_t *acc_free = acc_full + C::NT;
+  uint64_t *drain = acc_free + C::NT;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
   int *fin_tok = flag + 1;  // [BN]: combine, this CTA's slot was its token's last of the row block
+  int *gidx = reinterpret_cast<int *>(smem + C::GIDX_OFF);
+  int2 *tab = reinterpret_cast<int2 *>(smem + C::TAB_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto st_b = [&](int s) { return smem + s * C::B_BYTES; };
@@ -212,18 +199,27 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
     return reinterpret_cast<uint32_t *>(smem + C::CODE_OFF + c * C::CODE_SLOT + NP * C::CB * 4096) + p * C::CB * 128;
   };
 
+  const int nkb = P.d_in / 128;
+  const int nmain = NP == 2 ? nkb : (nkb + 1) / 2;
+  const int n_ext = P.rank > 0 ? (NP == 2 ? (P.rank + 127) / 128 : (P.rank + 255) / 256) : 0;
+  const int R = nmain + n_ext;  // rounds per unit
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NB; ++s) {
       mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], DQ_DW);
+      mbar_init(&b_empty[s], 1);
     }
     for (int c = 0; c < C::NC; ++c) {
       mbar_init(&c_full[c], 1);
-      mbar_init(&c_empty[c], DQ_DW);
+      mbar_init(&c_empty[c], DQ_DEC + DQ_FW);
     }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(&a_full[j], DQ_DW);
-      mbar_init(&mma_done[j], 1);
+    for (int j = 0; j < C::NA; ++j) {
+      mbar_init(&a_full[j], DQ_DEC);
+      mbar_init(&a_free[j], 1);
+    }
+    for (int j = 0; j < C::NT; ++j) {
+      mbar_init(&acc_full[j], 1);
+      mbar_init(&acc_free[j], DQ_FW);
     }
     mbar_init(drain, 1);
     *flag = 0;
@@ -233,147 +229,322 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
     tc::alloc(tmem_slot, 512);
     tc::relinquish();
   }
+  for (int k = threadIdx.x; k < nkb; k += blockDim.x) gidx[k] = (k * 128) / P.group;
+  // the prologue above (barriers, TMEM, group table) overlaps the previous kernel's tail
+  pdl_wait_and_release();
+
+  const int n_tiles = *P.tile_count;
+  const long long total = (long long)n_tiles * P.m_tiles * R;
+  const long long r0 = range_begin(total, blockIdx.x, gridDim.x);
+  const long long r1 = range_begin(total, blockIdx.x + 1, gridDim.x);
+  const int nr_all = (int)(r1 - r0);
+  // (the host keeps every CTA within the table; a launch outside it does nothing but report)
+  const int nr = nr_all <= DQ_MAX_ROUNDS ? nr_all : 0;
+  if (nr_all > DQ_MAX_ROUNDS && threadIdx.x == 0) set_status(P.status, TILEQ_ERR_UNSUPPORTED);
+
+  // ---- the round table.  Code chunks hold C::RPC consecutive main rounds of a
+  // unit from the first main round this CTA processes in it; units strictly
+  // inside the range are whole, so the chunks before a unit have a closed form.
+  {
+    const long long u0 = r0 / R;
+    const int rr0 = (int)(r0 - u0 * R);
+    auto rr_hi_of = [&](long long u) { return (int)min((long long)nmain, r1 - u * R); };
+    auto nch = [&](long long u, int lo) {
+      const int hi = rr_hi_of(u);
+      return hi > lo ? (hi - lo + C::RPC - 1) / C::RPC : 0;
+    };
+    const int nch0 = nch(u0, rr0), nch_full = (nmain + C::RPC - 1) / C::RPC;
+    for (int i = threadIdx.x; i < nr; i += blockDim.x) {
+      const long long r = r0 + i;
+      const long long unit = r / R;
+      const int rr = (int)(r - unit * R);
+      uint32_t f = (rr == R - 1 || i == nr - 1) ? RD_UEND : 0u;
+      if (rr < nmain) {
+        const int lo = unit == u0 ? rr0 : 0, hi = rr_hi_of(unit);
+        const int idx = (unit == u0 ? 0 : nch0 + (int)(unit - u0 - 1) * nch_full) + (rr - lo) / C::RPC;
+        const int pos = (rr - lo) % C::RPC;
+        const int kb_a = NP == 2 ? rr - pos : 2 * (rr - pos);
+        const int kb0 = NP == 2 ? rr : 2 * rr, kb1 = NP == 2 ? rr : 2 * rr + 1;
+        const int ga = (kb_a * 128) / P.group;
+        f |= RD_V0 | (pos == 0 ? RD_CSTART : 0u) | (pos == C::RPC - 1 || rr == hi - 1 ? RD_CEND : 0u);
+        f |= (uint32_t)(idx % C::NC) << 8 | (uint32_t)((idx / C::NC) & 1) << 11;
+        f |= (uint32_t)(kb0 - kb_a) << 20 | (uint32_t)((kb0 * 128) / P.group - ga) << 24;
+        if (kb1 < nkb) f |= RD_V1 | (uint32_t)(kb1 - kb_a) << 22 | (uint32_t)((kb1 * 128) / P.group - ga) << 26;
+      } else {
+        const int e = rr - nmain;
+        f |= RD_EXT;
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          const int ch = NP == 2 ? e : 2 * e + sl;
+          if (ch * 128 < P.rank) {
+            f |= (sl ? RD_V1 : RD_V0) | (uint32_t)((min(128, P.rank - ch * 128) + 15) / 16) << (sl ? 16 : 12) |
+                 (uint32_t)ch << (sl ? 30 : 28);
+          }
+        }
+      }
+      tab[i] = make_int2((int)f, (int)(unit << 9 | rr));
+    }
+  }
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = *tmem_slot;
-  // the prologue above (barriers, TMEM) overlaps the previous kernel's tail
-  pdl_wait_and_release();
-
-  const int n_tiles = *P.tile_count;
-  const int nkb = P.d_in / 128;
-  const int G = P.d_in / P.group;
-  const int nmain = NP == 2 ? nkb : (nkb + 1) / 2;
-  const int n_ext = P.rank > 0 ? (NP == 2 ? (P.rank + 127) / 128 : (P.rank + 255) / 256) : 0;
-  const int R = nmain + n_ext;  // rounds per unit
-  const long long total = (long long)n_tiles * P.m_tiles * R;
-  const long long r0 = range_begin(total, blockIdx.x, gridDim.x);
-  const long long r1 = range_begin(total, blockIdx.x + 1, gridDim.x);
-  const int nr = (int)(r1 - r0);
   bool ok = true;
 
   if (warp == 0) {
     // ============================================================ producer
     if (lane == 0) {
-      int i = 0;
-      RoundCursor<NP> cur;
-      cur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
-      ChunkTrack ck;
-      int cur_jt = -1;
-      int4 cur_tile = make_int4(0, 0, 0, 0);
-      for (; i < nr; ++i, cur.advance()) {
-        const Round rd = cur.get();
-        ck.on_round<C::RPC>(i == 0 || rd.rr == 0, rd.rr, rd.unit, R, nmain, r1);
-        if (rd.jt != cur_jt) {  // the tile changes with the unit only
-          cur_jt = rd.jt;
-          cur_tile = P.tiles[rd.jt];
+      int i = 0, nch_issued = 0;
+      long long cur_unit = -1;
+      int grp = 0, item0 = 0, ob = 0;
+      for (; i < nr; ++i) {
+        const int2 t = tab[i];
+        const uint32_t f = (uint32_t)t.x;
+        const long long unit = (unsigned)t.y >> 9;
+        const int rr = t.y & 511;
+        if (unit != cur_unit) {  // the tile changes with the unit only
+          cur_unit = unit;
+          const int jt = (int)(unit / P.m_tiles);
+          ob = (int)(unit - (long long)jt * P.m_tiles);
+          const int4 tl = P.tiles[jt];
+          grp = tl.x;
+          item0 = tl.y;
         }
-        const int grp = cur_tile.x, item0 = cur_tile.y;
-        if (!rd.ext && ck.starts<C::RPC>(rd.rr)) {
-          // the next code chunk: rounds first .. last of this unit
-          const int c = ck.n % C::NC;
-          if (ck.n >= C::NC && !(ok = mbar_wait(&c_empty[c], ((ck.n / C::NC) - 1) & 1, P.status))) break;
-          const int r_a = rd.rr, r_b = ck.last_round<C::RPC>(rd.rr) + 1;
-          const int kb_a = NP == 2 ? r_a : 2 * r_a, kb_b = NP == 2 ? r_b : min(nkb, 2 * r_b);
-          const int g_a = (kb_a * 128) / P.group, g_b = ((kb_b - 1) * 128) / P.group;
+        if (f & RD_CSTART) {
+          // the next code chunk: main rounds rr .. min(rr + RPC, this CTA's last of the unit) - 1
+          const int c = (int)rd_field(f, 8, 3);
+          if (nch_issued >= C::NC && !(ok = mbar_wait_sleep(&c_empty[c], rd_field(f, 11, 1) ^ 1u, P.status))) break;
+          const int r_b = min(rr + C::RPC, (int)min((long long)nmain, r1 - unit * R));
+          const int kb_a = NP == 2 ? rr : 2 * rr, kb_b = NP == 2 ? r_b : min(nkb, 2 * r_b);
+          const int g_a = gidx[kb_a], g_b = gidx[kb_b - 1];
           const uint32_t cbytes = (uint32_t)(kb_b - kb_a) * 4096, zbytes = (uint32_t)(g_b - g_a + 1) * 512;
           mbar_arrive_expect_tx(&c_full[c], NP * (cbytes + zbytes));
           for (int p = 0; p < NP; ++p) {
-            const size_t blk = ((size_t)grp * P.m_tiles + rd.ob) * nkb + kb_a;
+            const size_t blk = ((size_t)grp * P.m_tiles + ob) * nkb + kb_a;
             bulk_g2s(ch_codes(c, p), reinterpret_cast<const uint8_t *>(P.codes[p]) + blk * 4096, cbytes, &c_full[c]);
-            const size_t zoff = (((size_t)grp * P.m_tiles + rd.ob) * G + g_a) * 128;
+            const size_t zoff = (((size_t)grp * P.m_tiles + ob) * (nkb * 128 / P.group) + g_a) * 128;
             bulk_g2s(ch_sz(c, p), P.sz[p] + zoff, zbytes, &c_full[c]);
           }
-          ++ck.n;
+          ++nch_issued;
         }
         // the round's activation tile
         const int s = i % C::NB;
-        if (i >= C::NB && !(ok = mbar_wait(&b_empty[s], ((i / C::NB) - 1) & 1, P.status))) break;
+        if (i >= C::NB && !(ok = mbar_wait_sleep(&b_empty[s], ((i / C::NB) - 1) & 1, P.status))) break;
         uint8_t *bs = st_b(s);
-        if (!rd.ext) {
-          int na = 0;
-          for (int sl = 0; sl < 2; ++sl)
-            if (rd.valid[sl]) na += (NP == 2 || F8) ? (sl == 0 ? 2 : 0) : 2;
-          mbar_arrive_expect_tx(&b_full[s], (uint32_t)na * C::ATOM);
-          for (int sl = 0; sl < 2; ++sl) {
-            if (!rd.valid[sl]) continue;
-            const int kb = rd.kb[sl];
-            if (F8) {
-              // the two e4m3 pieces of the 128 K of this block (one 128-byte box each)
-              if (sl == 0)
-                for (int pc = 0; pc < 2; ++pc)
-                  tc::tma_load_2d(bs + pc * C::ATOM, &P.bmap, pc * P.d_in + kb * 128, item0, &b_full[s]);
-            } else if (NP == 1 || sl == 0) {
+        if (!(f & RD_EXT)) {
+          const int kb0 = NP == 2 ? rr : 2 * rr;
+          if (F8) {
+            // the two e4m3 pieces of the 128 K of this block (one 128-byte box each)
+            mbar_arrive_expect_tx(&b_full[s], 2u * C::ATOM);
+            for (int pc = 0; pc < 2; ++pc)
+              tc::tma_load_2d(bs + pc * C::ATOM, &P.bmap, pc * P.d_in + kb0 * 128, item0, &b_full[s]);
+          } else {
+            const int nsl = (NP == 1 && (f & RD_V1)) ? 2 : 1;
+            mbar_arrive_expect_tx(&b_full[s], (uint32_t)(2 * nsl) * C::ATOM);
+            for (int sl = 0; sl < nsl; ++sl)
               for (int a = 0; a < 2; ++a)
-                tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, &P.bmap, kb * 128 + a * 64, item0, &b_full[s]);
-            }
+                tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, &P.bmap, (kb0 + sl) * 128 + a * 64, item0, &b_full[s]);
           }
         } else {
           int na = 0;
           for (int sl = 0; sl < 2; ++sl)
-            if (rd.valid[sl]) na += (min(128, P.rank - rd.chunk[sl] * 128) + 63) / 64;
+            if (f & (sl ? RD_V1 : RD_V0)) na += ((int)rd_field(f, sl ? 16 : 12, 4) + 3) / 4;
           mbar_arrive_expect_tx(&b_full[s], (uint32_t)na * C::ATOM);
           for (int sl = 0; sl < 2; ++sl) {
-            if (!rd.valid[sl]) continue;
+            if (!(f & (sl ? RD_V1 : RD_V0))) continue;
             const int p = NP == 2 ? sl : 0;
-            const int len = min(128, P.rank - rd.chunk[sl] * 128);
-            for (int a = 0; a * 64 < len; ++a)
-              tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, F8 ? &P.bmap_ext : &P.bmap,
-                              P.ext_col[p] + rd.chunk[sl] * 128 + a * 64, item0, &b_full[s]);
+            const int ch = (int)rd_field(f, sl ? 30 : 28, 2);
+            const int nat = ((int)rd_field(f, sl ? 16 : 12, 4) + 3) / 4;
+            for (int a = 0; a < nat; ++a)
+              tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, F8 ? &P.bmap_ext : &P.bmap, P.ext_col[p] + ch * 128 + a * 64,
+                              item0, &b_full[s]);
           }
         }
       }
       // no copy may still be landing in shared memory when the CTA exits
-      for (int j = i > C::NB ? i - C::NB : 0; j < i; ++j) mbar_wait(&b_full[j % C::NB], (j / C::NB) & 1, P.status);
-      for (int j = ck.n > C::NC ? ck.n - C::NC : 0; j < ck.n; ++j)
-        mbar_wait(&c_full[j % C::NC], (j / C::NC) & 1, P.status);
+      for (int j = i > C::NB ? i - C::NB : 0; j < i; ++j)
+        mbar_wait_sleep(&b_full[j % C::NB], (j / C::NB) & 1, P.status);
+      for (int j = nch_issued > C::NC ? nch_issued - C::NC : 0; j < nch_issued; ++j)
+        mbar_wait_sleep(&c_full[j % C::NC], (j / C::NC) & 1, P.status);
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
+    // One decode warp arrives on a round's operand slot only once the round's
+    // activations have landed and its accumulator slot is free, so this warp
+    // waits on one barrier per round.
     constexpr uint32_t idesc = tc::idesc_f16(BN);
-    RoundCursor<NP> cur;
-    cur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
-    for (int i = 0; i < nr; ++i, cur.advance()) {
-      const int as = i & 1;
-      if (!(ok = mbar_wait(&a_full[as], (i >> 1) & 1, P.status))) break;
-      if (!(ok = mbar_wait(&b_full[i % C::NB], (i / C::NB) & 1, P.status))) break;
+    for (int i = 0; i < nr; ++i) {
+      const int as = i % C::NA, bs = i % C::NB, ts = i % C::NT;
+      if (!(ok = mbar_wait_sleep(&a_full[as], (i / C::NA) & 1, P.status))) break;
       tc::fence_after();
-      const Round rd = cur.get();
+      const uint32_t f = (uint32_t)tab[i].x;
       if (tc::elect_one()) {
-        const uint64_t bd0 = tc::sdesc_sw128(smem_addr(st_b(i % C::NB)));
-        const uint32_t a0 = tmem + as * 128, d0 = tmem + C::ACC0 + as * C::ACC_COLS;
+        const uint64_t bd0 = tc::sdesc_sw128(smem_addr(st_b(bs)));
+        const uint32_t a0 = tmem + as * C::A_COLS, d0 = tmem + C::ACC0 + ts * C::ACC_COLS;
+        if (!(f & RD_EXT) && F8) {
+          // e4m3: four K = 32 steps over 128 K per slice, both pieces of B into the same accumulator
 #pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-          if (!rd.valid[sl]) continue;
-          if (F8 && !rd.ext) {
-            // e4m3: four K = 32 steps over 128 K; both pieces of B into the same accumulator
+          for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
             for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
               for (int pc = 0; pc < 2; ++pc)
-                tc::mma_ts_f8(d0 + sl * BN, a0 + sl * 64 + kk * 8,
-                              bd0 + (uint64_t)((pc * C::ATOM + kk * 32) >> 4), idesc, (kk | pc) ? 1u : 0u);
-            continue;
+                tc::mma_ts_f8(d0 + sl * BN, a0 + sl * 64 + kk * 8, bd0 + (uint64_t)((pc * C::ATOM + kk * 32) >> 4), idesc,
+                              (kk | pc) ? 1u : 0u);
+        } else if (!(f & RD_EXT)) {
+          // fp16: eight K = 16 steps per slice; the two projections of np = 2 share B atoms 0, 1
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl) {
+            if (NP == 1 && sl == 1 && !(f & RD_V1)) break;
+            const int atom0 = NP == 2 ? 0 : 2 * sl;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tc::mma_ts(d0 + sl * BN, a0 + sl * 64 + kk * 8,
+                         bd0 + (uint64_t)((((atom0 + kk / 4) * C::ATOM) + (kk % 4) * 32) >> 4), idesc, kk ? 1u : 0u);
           }
-          // B atoms of this slice: main rounds of a two-projection launch share atoms 0, 1
-          const int atom0 = (NP == 2 && !rd.ext) ? 0 : 2 * sl;
-          for (int kk = 0; kk < rd.nk[sl]; ++kk)
-            tc::mma_ts(d0 + sl * BN, a0 + sl * 64 + kk * 8,
-                       bd0 + (uint64_t)((((atom0 + kk / 4) * C::ATOM) + (kk % 4) * 32) >> 4), idesc, kk ? 1u : 0u);
+        } else {
+          for (int sl = 0; sl < 2; ++sl) {
+            if (!(f & (sl ? RD_V1 : RD_V0))) continue;
+            const int nk = (int)rd_field(f, sl ? 16 : 12, 4);
+            for (int kk = 0; kk < nk; ++kk)
+              tc::mma_ts(d0 + sl * BN, a0 + sl * 64 + kk * 8,
+                         bd0 + (uint64_t)((((2 * sl + kk / 4) * C::ATOM) + (kk % 4) * 32) >> 4), idesc, kk ? 1u : 0u);
+          }
         }
-        tc::commit(&mma_done[as]);
+        // the operand slot and the activation stage are free once these MMAs
+        // have read them; the accumulators are then ready to fold
+        tc::commit(&a_free[as]);
+        tc::commit(&b_empty[bs]);
+        tc::commit(&acc_full[ts]);
       }
       __syncwarp();
     }
     // all issued MMAs have retired before TMEM is released
     if (tc::elect_one()) tc::commit(drain);
     __syncwarp();
-    mbar_wait(drain, 0, P.status);
-  } else {
-    // ============================================================ decode + epilogue
-    // One warp per TMEM lane quadrant (32 weight rows): it decodes both slices
-    // of every round (256 weights per thread) and holds both accumulators in
-    // registers, so a unit's two slices meet in the same thread.
+    mbar_wait_sleep(drain, 0, P.status);
+  } else if (warp < 2 + DQ_DEC) {
+    // ============================================================ decode
+    // Two warps per TMEM lane quadrant (32 weight rows): warps 2..5 decode
+    // slice 0 and warps 6..9 slice 1 of every round into its operand slot.
+    // The slot's release is probed before the decode and awaited after it, so
+    // the barrier's latency overlaps the decoding.
     const int dw = warp - 2;
+    const int sl = dw / 4;
+    const bool gate = dw == 0;  // this warp also stands for the MMA warp's other conditions
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_addr = tc::lane_base(warp);
+    for (int i = 0; i < nr && ok; ++i) {
+      const int2 t = tab[i];
+      const uint32_t f = (uint32_t)t.x;
+      const int c = (int)rd_field(f, 8, 3);
+      const int as = i % C::NA;
+      const uint32_t free_par = ((i / C::NA) - 1) & 1;
+      bool slot_free = i < C::NA || mbar_test(&a_free[as], free_par);
+      if ((f & RD_CSTART) && !(ok = mbar_wait_sleep(&c_full[c], rd_field(f, 11, 1), P.status))) break;
+      const uint32_t acol = tmem + lane_addr + as * C::A_COLS + sl * 64;
+      auto ensure_free = [&]() -> bool {
+        if (!slot_free && !mbar_wait_sleep(&a_free[as], free_par, P.status)) return false;
+        slot_free = true;
+        tc::fence_after();
+        return true;
+      };
+      if (f & (sl ? RD_V1 : RD_V0)) {
+        if (!(f & RD_EXT)) {
+          const int p = NP == 2 ? sl : 0;
+          const uint8_t *cb = ch_codes(c, p) + rd_field(f, 20 + 2 * sl, 2) * 4096;
+          const uint32_t szw = ch_sz(c, p)[rd_field(f, 24 + 2 * sl, 2) * 128 + row];
+          uint2 wv[4];
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) wv[ks] = *reinterpret_cast<const uint2 *>(cb + ks * 1024 + row * 8);
+          if constexpr (F8) {
+            // e4m3 (q - z) through a 4-entry byte table per zero point: one PRMT per 4 weights.
+            // The table for zero point z is bytes 3 - z .. 6 - z of e4m3(-3 .. 3); z comes out of
+            // its fp16 bits by adding 1024 (ulp 1 there).
+            const uint32_t zi = __half_as_ushort(__hadd(__ushort_as_half((unsigned short)(szw >> 16)),
+                                                        __ushort_as_half((unsigned short)0x6400))) & 3u;
+            const uint32_t tb = __byte_perm(0x00B8C0C4u, 0x00444038u, 0x6543u - zi * 0x1111u);
+            uint32_t v[32];
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {  // the four K slices of 32 (two words of 16 codes each)
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const uint32_t w = h ? wv[ks].y : wv[ks].x;
+                const uint32_t c0 = w & 0x33333333u, c1 = (w >> 2) & 0x33333333u;
+                uint32_t *o = v + 8 * ks + 4 * h;
+                o[0] = __byte_perm(tb, 0, c0);
+                o[1] = __byte_perm(tb, 0, c0 >> 16);
+                o[2] = __byte_perm(tb, 0, c1);
+                o[3] = __byte_perm(tb, 0, c1 >> 16);
+              }
+            }
+            if (!(ok = ensure_free())) break;
+            tc::st32(acol, v);
+          } else {
+            const __half2 z2 = __high2half2(u32_as_h2(szw));
+            const __half2 nz[4] = {__hsub2(__float2half2_rn(-1024.f), z2), __hsub2(__float2half2_rn(-256.f), z2),
+                                   __hsub2(__float2half2_rn(-64.f), z2), __hsub2(__float2half2_rn(-16.f), z2)};
+#pragma unroll
+            for (int hk = 0; hk < 2; ++hk) {  // K halves of 64: 32 TMEM columns each
+              uint32_t v[32];
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                dq_qz_word(wv[2 * hk + q].x, nz, v + 16 * q);
+                dq_qz_word(wv[2 * hk + q].y, nz, v + 16 * q + 8);
+              }
+              if (hk == 0 && !(ok = ensure_free())) break;
+              tc::st32(acol + hk * 32, v);
+            }
+            if (!ok) break;
+          }
+        } else {
+          // rows of U_m: rank columns chunk * 128 ..
+          const long long unit = (unsigned)t.y >> 9;
+          const int jt = (int)(unit / P.m_tiles), ob = (int)(unit - (long long)jt * P.m_tiles);
+          const int p = NP == 2 ? sl : 0;
+          const int chunk = (int)rd_field(f, 28 + 2 * sl, 2);
+          const __half *ur =
+              P.u[p] + (((size_t)P.u_blk[p][P.tiles[jt].x] * P.m_tiles + ob) * 128 + row) * P.rank + chunk * 128;
+          const int kmax = P.rank - chunk * 128;
+#pragma unroll
+          for (int hk = 0; hk < 2; ++hk) {
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              uint4 q4 = make_uint4(0, 0, 0, 0);
+              if (hk * 64 + j * 8 < kmax) q4 = __ldg(reinterpret_cast<const uint4 *>(ur + hk * 64 + j * 8));
+              v[4 * j + 0] = q4.x;
+              v[4 * j + 1] = q4.y;
+              v[4 * j + 2] = q4.z;
+              v[4 * j + 3] = q4.w;
+            }
+            if (hk == 0 && !(ok = ensure_free())) break;
+            tc::st32(acol + hk * 32, v);
+          }
+          if (!ok) break;
+        }
+      }
+      // (a warp with nothing to write for the round still waits for the slot:
+      // its arrival must not run ahead into the slot's previous phase)
+      if (!(ok = ensure_free())) break;
+      if (gate) {
+        // the round's activations have landed and its accumulator slot is free
+        if (!(ok = mbar_wait_sleep(&b_full[i % C::NB], (i / C::NB) & 1, P.status))) break;
+        if (i >= C::NT && !(ok = mbar_wait_sleep(&acc_free[i % C::NT], ((i / C::NT) - 1) & 1, P.status))) break;
+      }
+      tc::wait_st();
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[as]);
+      // the chunk's codes are decoded: the producer may refill its slot
+      if ((f & RD_CEND) && lane == 0) mbar_arrive(&c_empty[c]);
+    }
+  } else {
+    // ============================================================ fold + epilogue
+    // One warp per TMEM lane quadrant (32 weight rows): it folds both slices'
+    // accumulators of every round into registers with the group scale, so a
+    // unit's two slices meet in the same thread, and stores the unit's result.
+    const int fw = warp - 2 - DQ_DEC;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = tc::lane_base(warp);
     float acc0[BN], acc1[BN];  // np = 2: gate, up; np = 1: the two slices' partial sums
@@ -382,24 +553,24 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
       acc0[c] = 0.f;
       acc1[c] = 0.f;
     }
-    // per round parity (e: even index, o: odd): this row's scale of each slice and whether the slice was valid
-    float sce0 = 0.f, sce1 = 0.f, sco0 = 0.f, sco1 = 0.f;
-    bool vde0 = false, vde1 = false, vdo0 = false, vdo1 = false;
 
     // ---- end of a unit's rounds in this CTA: store the result (whole unit) or
     // a piece (unit cut between CTAs; the CTA finishing last sums them)
-    auto unit_end = [&](const Round &rd) -> void {
-      const long long ustart = (long long)rd.unit * R, uend = ustart + R;
+    auto unit_end = [&](const int unit, const int jt, const int ob) -> void {
+      const long long ustart = (long long)unit * R, uend = ustart + R;
       const bool whole = ustart >= r0 && uend <= r1;
-      const int4 t = P.tiles[rd.jt];
+      const int4 t = P.tiles[jt];
       const int item0 = t.y, nitems = t.z;
-      const int o = rd.ob * 128 + row;
+      const int o = ob * 128 + row;
+      // per-item factors, one per lane (items < 32), handed out by shuffles
+      const float xs_l = (F8 && lane < nitems) ? __ldg(P.xs + item0 + lane) : 1.f;
+      const float rs_l = (NP == 2 && P.row_scale && lane < nitems) ? __ldg(P.row_scale + item0 + lane) : 1.f;
       // the final result of item column n: np = 2: silu(gate) * up * row scale (fp16) or both in
-      // fp32; np = 1: the sum of both slices (fp32)
+      // fp32; np = 1: the sum of both slices (fp32).  Called by the whole warp with the same n.
       auto store = [&](int n, float g, float u) {
+        const float xs = __shfl_sync(0xffffffffu, xs_l, n), rs = __shfl_sync(0xffffffffu, rs_l, n);
         if (n >= nitems || o >= P.d_out) return;
         if (F8) {  // the activations were scaled by 2^e per item
-          const float xs = __ldg(P.xs + item0 + n);
           g *= xs;
           u *= xs;
         }
@@ -407,7 +578,6 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
           reinterpret_cast<float *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = g;
           reinterpret_cast<float *>(P.out2)[(size_t)(item0 + n) * P.ldo + o] = u;
         } else if (NP == 2) {
-          const float rs = P.row_scale ? __ldg(P.row_scale + item0 + n) : 1.f;
           reinterpret_cast<__half *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = half_checked(silu_f(g) * u * rs, P.status);
         } else {
           reinterpret_cast<float *>(P.out)[(size_t)(item0 + n) * P.ldo + o] = g;
@@ -427,14 +597,14 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
           if (NP == 2) pc[(BN + c) * 128 + row] = acc1[c];
         }
         __threadfence();
-        named_sync(1, DQ_DW * 32);
+        named_sync(1, DQ_FW * 32);
         const int c_first = cta_of(ustart, total, gridDim.x), c_last = cta_of(uend - 1, total, gridDim.x);
         // CTAs with an empty range (fewer rounds than CTAs) leave no piece
         int pieces = 0;
         for (int cc = c_first; cc <= c_last; ++cc)
           pieces += range_begin(total, cc + 1, gridDim.x) > range_begin(total, cc, gridDim.x);
-        if (dw == 0 && lane == 0) *flag = atomicAdd(&P.counters[rd.unit], 1) == pieces - 1;
-        named_sync(1, DQ_DW * 32);
+        if (fw == 0 && lane == 0) *flag = atomicAdd(&P.counters[unit], 1) == pieces - 1;
+        named_sync(1, DQ_FW * 32);
         fin = *flag != 0;
         if (fin) {
           // the last piece in: sum all pieces of the unit in CTA order
@@ -445,40 +615,40 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
             for (int cc = c_first; cc <= c_last; ++cc) {
               const long long b = range_begin(total, cc, gridDim.x);
               if (range_begin(total, cc + 1, gridDim.x) == b) continue;
-              const int s2 = (b / R == rd.unit) ? 0 : 1;  // the unit is cta cc's first (slot 0) or last
+              const int s2 = (b / R == unit) ? 0 : 1;  // the unit is cta cc's first (slot 0) or last
               const float *q = P.part + ((size_t)cc * 2 + s2) * NP * BN * 128;
               g += __ldcg(q + c * 128 + row);
               if (NP == 2) u += __ldcg(q + (BN + c) * 128 + row);
             }
             store(c, g, u);
           }
-          if (dw == 0 && lane == 0) P.counters[rd.unit] = 0;
+          if (fw == 0 && lane == 0) P.counters[unit] = 0;
         }
       }
       // weighted top-k combine: the slot weights are inside h, so the layer
       // output of a token is the plain sum of its slots' rows
       if (NP == 1 && P.combine && fin) {
         __threadfence();
-        named_sync(1, DQ_DW * 32);
-        const int tid = dw * 32 + lane;  // 0 .. 127
+        named_sync(1, DQ_FW * 32);
+        const int tid = ((warp & 3) * 32) + lane;  // 0 .. 127
         if (tid < nitems) {
           const int tok = __ldg(P.slot_tok + item0 + tid);
-          fin_tok[tid] = atomicAdd(&P.tok_counters[tok * P.m_tiles + rd.ob], 1) == P.top_k - 1;
+          fin_tok[tid] = atomicAdd(&P.tok_counters[tok * P.m_tiles + ob], 1) == P.top_k - 1;
         }
-        named_sync(1, DQ_DW * 32);
+        named_sync(1, DQ_FW * 32);
         __threadfence();
         const float *yb = reinterpret_cast<const float *>(P.out);
         for (int n = 0; n < nitems; ++n) {
           if (!fin_tok[n]) continue;
           const int tok = __ldg(P.slot_tok + item0 + n);
-          const int oo = rd.ob * 128 + tid;
+          const int oo = ob * 128 + tid;
           if (oo >= P.d_out) continue;
           float y = P.yshared ? __ldg(P.yshared + (size_t)tok * P.ldo + oo) : 0.f;
           for (int j = 0; j < P.top_k; ++j)
             y += __ldcg(yb + (size_t)__ldg(P.slot_of_pair + tok * P.top_k + j) * P.ldo + oo);
           P.out_tok[(size_t)tok * P.ldo + oo] = __float2bfloat16_rn(y);
         }
-        named_sync(1, DQ_DW * 32);  // fin_tok is reused by the next unit
+        named_sync(1, DQ_FW * 32);  // fin_tok is reused by the next unit
       }
 #pragma unroll
       for (int c = 0; c < BN; ++c) {
@@ -489,156 +659,47 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
 
     // fold one slice's accumulator (BN columns at TMEM column base) into acc
     auto fold = [&](uint32_t base, float s, float (&acc)[BN]) {
-#pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t d[16];
-        tc::ld16_nowait(base + c0, d);
-        tc::wait_ld();
-#pragma unroll
-        for (int c = 0; c < 16; ++c) acc[c0 + c] = fmaf(__uint_as_float(d[c]), s, acc[c0 + c]);
+      uint32_t d[BN];
+      if constexpr (BN == 32) {
+        tc::ld32_nowait(base, d);
+      } else {
+        tc::ld16_nowait(base, d);
       }
+      tc::wait_ld();
+#pragma unroll
+      for (int c = 0; c < BN; ++c) acc[c] = fmaf(__uint_as_float(d[c]), s, acc[c]);
     };
 
-    // ---- fold round j's accumulators (slot j & 1) into registers; release its stage
-    // (rounds are finished in order: fcur is at round j)
-    RoundCursor<NP> fcur;
-    fcur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
-    auto finish = [&](int j) -> bool {
-      if (!mbar_wait(&mma_done[j & 1], (j >> 1) & 1, P.status)) return false;
+    for (int i = 0; i < nr && ok; ++i) {
+      const int ts = i % C::NT;
+      const int2 t = tab[i];
+      const uint32_t f = (uint32_t)t.x;
+      const int c = (int)rd_field(f, 8, 3);
+      // this row's scale of each slice (1 for the U_m extension); the chunk's
+      // codes were awaited by the decode warps before this round's MMAs
+      float s0 = 1.f, s1 = 1.f;
+      if (!(ok = mbar_wait_sleep(&acc_full[ts], (i / C::NT) & 1, P.status))) break;
       tc::fence_after();
-      const uint32_t base = tmem + lane_addr + C::ACC0 + (j & 1) * C::ACC_COLS;
+      if (!(f & RD_EXT)) {
+        s0 = __low2float(u32_as_h2(ch_sz(c, 0)[rd_field(f, 24, 2) * 128 + row]));
+        s1 = __low2float(u32_as_h2(ch_sz(c, NP == 2 ? 1 : 0)[rd_field(f, 26, 2) * 128 + row]));
+      }
       // tcgen05.ld is warp-collective: the decision is the warp's (the slice
-      // was valid in round j), never a lane's (padding rows have scale 0)
-      const bool odd = j & 1;
-      if (odd ? vdo0 : vde0) fold(base, odd ? sco0 : sce0, acc0);
-      if (odd ? vdo1 : vde1) fold(base + BN, odd ? sco1 : sce1, acc1);
+      // was valid in round i), never a lane's (padding rows have scale 0)
+      const uint32_t base = tmem + lane_addr + C::ACC0 + ts * C::ACC_COLS;
+      if (f & RD_V0) fold(base, s0, acc0);
+      if (f & RD_V1) fold(base + BN, s1, acc1);
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&b_empty[j % C::NB]);
-      const Round rd = fcur.get();  // round j
-      fcur.advance();
-      if (rd.rr == R - 1 || j == nr - 1) unit_end(rd);
-      return true;
-    };
-
-    // ---- one slice of round i into the A slot: decode (main) or U_m rows (extension)
-    auto load_slice = [&](const Round &rd, int c, int kb_a, int g_a, int sl, int i, float &scale) {
-      const uint32_t acol = tmem + lane_addr + (i & 1) * 128 + sl * 64;
-      if (!rd.ext) {
-        const int p = NP == 2 ? sl : 0, kb = sl ? rd.kb[1] : rd.kb[0];
-        const uint8_t *cb = ch_codes(c, p) + (kb - kb_a) * 4096;
-        const __half2 szw = u32_as_h2(ch_sz(c, p)[((kb * 128) / P.group - g_a) * 128 + row]);
-        scale = __low2float(szw);
-        if constexpr (F8) {
-          // e4m3 (q - z) through a 4-entry byte table per zero point: one PRMT per 4 weights
-          const int zi = (int)__high2float(szw);
-          const uint32_t tab = zi == 0 ? 0x44403800u : zi == 1 ? 0x403800B8u : zi == 2 ? 0x3800B8C0u : 0x00B8C0C4u;
-          uint32_t v[32];
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {  // the four K slices of 32 (two words of 16 codes each)
-            uint32_t w0, w1;
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(w0), "=r"(w1) : "r"(smem_addr(cb + ks * 1024 + row * 8)));
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t w = h ? w1 : w0;
-              const uint32_t c0 = w & 0x33333333u, c1 = (w >> 2) & 0x33333333u;
-              uint32_t *o = v + 8 * ks + 4 * h;
-              o[0] = __byte_perm(tab, 0, c0);
-              o[1] = __byte_perm(tab, 0, c0 >> 16);
-              o[2] = __byte_perm(tab, 0, c1);
-              o[3] = __byte_perm(tab, 0, c1 >> 16);
-            }
-          }
-          tc::st32(acol, v);
-        } else {
-          const __half2 z2 = __high2half2(szw);
-          const __half2 nz[4] = {__hsub2(__float2half2_rn(-1024.f), z2), __hsub2(__float2half2_rn(-256.f), z2),
-                                 __hsub2(__float2half2_rn(-64.f), z2), __hsub2(__float2half2_rn(-16.f), z2)};
-#pragma unroll
-          for (int hk = 0; hk < 2; ++hk) {  // K halves of 64: 32 TMEM columns each
-            uint32_t v[32];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              uint32_t w0, w1;
-              asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n"
-                           : "=r"(w0), "=r"(w1)
-                           : "r"(smem_addr(cb + (2 * hk + q) * 1024 + row * 8)));
-              dq_qz_word(w0, nz, v + 16 * q);
-              dq_qz_word(w1, nz, v + 16 * q + 8);
-            }
-            tc::st32(acol + hk * 32, v);
-          }
-        }
-      } else {
-        // rows of U_m: rank columns chunk * 128 ..
-        const int4 t = P.tiles[rd.jt];
-        const int p = NP == 2 ? sl : 0;
-        const int chunk = sl ? rd.chunk[1] : rd.chunk[0];
-        const __half *ur = P.u[p] + (((size_t)P.u_blk[p][t.x] * P.m_tiles + rd.ob) * 128 + row) * P.rank + chunk * 128;
-        const int kmax = P.rank - chunk * 128;
-#pragma unroll
-        for (int hk = 0; hk < 2; ++hk) {
-          uint32_t v[32];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            uint4 q4 = make_uint4(0, 0, 0, 0);
-            if (hk * 64 + j * 8 < kmax) q4 = __ldg(reinterpret_cast<const uint4 *>(ur + hk * 64 + j * 8));
-            v[4 * j + 0] = q4.x;
-            v[4 * j + 1] = q4.y;
-            v[4 * j + 2] = q4.z;
-            v[4 * j + 3] = q4.w;
-          }
-          tc::st32(acol + hk * 32, v);
-        }
-        scale = 1.f;
+      if (lane == 0) mbar_arrive(&acc_free[ts]);
+      if ((f & RD_CEND) && lane == 0) mbar_arrive(&c_empty[c]);
+      if (f & RD_UEND) {
+        const long long unit = (unsigned)t.y >> 9;
+        const int jt = (int)(unit / P.m_tiles);
+        unit_end((int)unit, jt, (int)(unit - (long long)jt * P.m_tiles));
       }
-    };
-
-    RoundCursor<NP> cur;
-    cur.init(r0, R, nmain, nkb, P.m_tiles, P.rank);
-    ChunkTrack ck;
-    int c = 0, kb_a = 0, g_a = 0;  // the current code chunk: ring slot, first block, first group
-    for (int i = 0; i < nr && ok; ++i, cur.advance()) {
-      const Round rd = cur.get();
-      ck.on_round<C::RPC>(i == 0 || rd.rr == 0, rd.rr, rd.unit, R, nmain, r1);
-      if (!rd.ext && ck.starts<C::RPC>(rd.rr)) {
-        c = ck.n % C::NC;
-        kb_a = NP == 2 ? rd.rr : 2 * rd.rr;
-        g_a = (kb_a * 128) / P.group;
-        if (!(ok = mbar_wait(&c_full[c], (ck.n / C::NC) & 1, P.status))) break;
-        ++ck.n;
-      }
-      // round i - 2: fold its accumulators; its A slot is then free for round i
-      if (i >= 2 && !(ok = finish(i - 2))) break;
-      float s0 = 0.f, s1 = 0.f;
-      if (rd.valid[0]) load_slice(rd, c, kb_a, g_a, 0, i, s0);
-      if (rd.valid[1]) load_slice(rd, c, kb_a, g_a, 1, i, s1);
-      // the chunk's codes are decoded: the producer may refill its slot
-      if (!rd.ext && ck.ends<C::RPC>(rd.rr)) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c_empty[c]);
-      }
-      tc::wait_st();
-      if (i & 1) {
-        sco0 = s0;
-        sco1 = s1;
-        vdo0 = rd.valid[0];
-        vdo1 = rd.valid[1];
-      } else {
-        sce0 = s0;
-        sce1 = s1;
-        vde0 = rd.valid[0];
-        vde1 = rd.valid[1];
-      }
-      tc::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[i & 1]);
     }
-    // the last two rounds' accumulators
-    if (ok)
-      for (int j = nr >= 2 ? nr - 2 : 0; j < nr && ok; ++j) ok = finish(j);
   }
-
   __syncwarp();
   tc::fence_before();
   __syncthreads();
@@ -668,8 +729,16 @@ cudaError_t launch_dq(const DqArgs &a, cudaStream_t stream) {
 
 int dq_grid() { return DQ_GRID; }
 
+bool dq_fits(int max_tiles, int m_tiles, int d_in, int rank) {
+  // the most rounds a unit can have (two-projection launches: one K block per round)
+  const long long R = d_in / 128 + (rank + 127) / 128;
+  const long long total = (long long)max_tiles * m_tiles * R;
+  return (total + DQ_GRID - 1) / DQ_GRID <= DQ_MAX_ROUNDS;
+}
+
 cudaError_t launch_gemm_dq(const DqArgs &a, int np, int bn, cudaStream_t stream) {
-  if (a.m_tiles <= 0 || a.group % 128 != 0 || a.d_in % 128 != 0 || a.rank < 0 || a.rank > 256)
+  if (a.m_tiles <= 0 || a.group % 128 != 0 || a.d_in % 128 != 0 || a.d_in > 128 * 256 || a.rank < 0 || a.rank > 256 ||
+      !dq_fits(a.max_tiles, a.m_tiles, a.d_in, a.rank))
     return cudaErrorInvalidValue;
   if (a.f8) {
     if (np != 2) return cudaErrorInvalidValue;

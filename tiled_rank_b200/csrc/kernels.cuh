@@ -189,6 +189,7 @@ struct DqArgs {
   const float *xs;               // fp8 mode: per item 2^-e
   const int4 *tiles;             // (expert, first item, items)
   const int *tile_count;
+  int max_tiles;                 // capacity of tiles (bounds the rounds of a CTA)
   int m_tiles, d_out, d_in, group, rank;
   int ext_col[2];                // first B column of projection p's K extension
   const uint32_t *codes[2];      // tcgen05 row layout of the codes (qw)
@@ -217,6 +218,9 @@ struct DqArgs {
 };
 cudaError_t launch_gemm_dq(const DqArgs &a, int np, int bn, cudaStream_t stream);
 int dq_grid();
+// Whether every CTA's rounds of a launch over at most max_tiles tiles fit the
+// kernel's per-CTA round table.
+bool dq_fits(int max_tiles, int m_tiles, int d_in, int rank);
 
 // Dense fp16 GEMM on tcgen05 with both operands read by TMA (gemm_dense.cu).
 // A: fp16 row-major, tensor maps amap[j] (box 64 x 128, 128-byte swizzle);
