@@ -57,10 +57,12 @@ struct DqCfg {
   // The codes stream from HBM in chunks of CB consecutive 128-wide K blocks
   // per projection (one bulk copy each, with the (scale, zero) words of their
   // groups), several chunks in flight.
-  static constexpr int CB = 4;
+  static constexpr int CB = NP == 2 ? 2 : 4;
   static constexpr int RPC = NP == 2 ? CB : CB / 2;     // main rounds per chunk
   static constexpr int CODE_SLOT = NP * CB * (4096 + 512);
-  static constexpr int NB = 4;                         // activation ring (per round, from L2)
+  // activation ring (per round): its tiles come from L2 with a latency of a few
+  // rounds, so the ring runs deep
+  static constexpr int NB = 8;
   static constexpr int NC_RAW = (200 * 1024 - NB * B_BYTES) / CODE_SLOT;
   static constexpr int NC = NC_RAW > 6 ? 6 : NC_RAW;   // code chunk ring
   static constexpr int CODE_OFF = NB * B_BYTES;
@@ -78,7 +80,7 @@ struct DqCfg {
   static constexpr int ACC0 = NA * A_COLS;
   static constexpr int NBAR = 2 * NB + 2 * NC + 2 * NA + 2 * NT + 1;
   static constexpr int SMEM = BAR_OFF + NBAR * 8 + 16 + BN * 4 + 1024;  // + slack to align the base
-  static_assert(NC >= 3, "code ring too shallow");
+  static_assert(NC >= 4, "code ring too shallow");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(NA >= 2, "operand ring too shallow");
   static_assert(ACC0 + NT * ACC_COLS <= 512, "tensor memory");
@@ -607,21 +609,27 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
         named_sync(1, DQ_FW * 32);
         fin = *flag != 0;
         if (fin) {
-          // the last piece in: sum all pieces of the unit in CTA order
+          // the last piece in: sum all pieces of the unit in CTA order (the
+          // range arithmetic once per piece, not per column)
           __threadfence();
-#pragma unroll 1
+#pragma unroll
           for (int c = 0; c < BN; ++c) {
-            float g = 0.f, u = 0.f;
-            for (int cc = c_first; cc <= c_last; ++cc) {
-              const long long b = range_begin(total, cc, gridDim.x);
-              if (range_begin(total, cc + 1, gridDim.x) == b) continue;
-              const int s2 = (b / R == unit) ? 0 : 1;  // the unit is cta cc's first (slot 0) or last
-              const float *q = P.part + ((size_t)cc * 2 + s2) * NP * BN * 128;
-              g += __ldcg(q + c * 128 + row);
-              if (NP == 2) u += __ldcg(q + (BN + c) * 128 + row);
-            }
-            store(c, g, u);
+            acc0[c] = 0.f;
+            acc1[c] = 0.f;
           }
+          for (int cc = c_first; cc <= c_last; ++cc) {
+            const long long b = range_begin(total, cc, gridDim.x);
+            if (range_begin(total, cc + 1, gridDim.x) == b) continue;
+            const int s2 = (b / R == unit) ? 0 : 1;  // the unit is cta cc's first (slot 0) or last
+            const float *q = P.part + ((size_t)cc * 2 + s2) * NP * BN * 128;
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+              acc0[c] += __ldcg(q + c * 128 + row);
+              if (NP == 2) acc1[c] += __ldcg(q + (BN + c) * 128 + row);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < BN; ++c) store(c, acc0[c], acc1[c]);
           if (fw == 0 && lane == 0) P.counters[unit] = 0;
         }
       }
