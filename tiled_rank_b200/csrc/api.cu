@@ -3,6 +3,7 @@
 // launch sequence of the fused and of the unfused (per-expert) forward.
 #include <algorithm>
 #include <atomic>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -260,9 +261,15 @@ Plan make_plan(const tileq_layer *L, const LayerInfo &li, int T, int k) {
   // cycle than mma.sync, and the decode then dominates); wider ones on tcgen05.
   const long long avg = P / std::max(1, L->K);
   const bool use_tc = avg > 32;
-  // narrow tiles on the decode-regime tcgen05 kernel where every projection
-  // has 2-bit codes in groups of a multiple of 128; otherwise warp-level MMA
-  bool dq_ok = !use_tc;
+  // Narrow tiles run on warp-level MMA.  The decode-regime tcgen05 kernel
+  // (2-bit codes in groups of a multiple of 128) is measured slower at every
+  // decode shape: its per-round pipeline synchronisation outweighs the tensor
+  // core rate at N <= 32, so it runs only when TILEQ_DECODE_TC=1 asks for it.
+  static const bool dq_requested = [] {
+    const char *v = std::getenv("TILEQ_DECODE_TC");
+    return v != nullptr && v[0] == '1';
+  }();
+  bool dq_ok = !use_tc && dq_requested;
   for (int p = 0; p < li.nproj; ++p) dq_ok = dq_ok && li.p[p].bits == 2 && li.p[p].group % 128 == 0;
   if (dq_ok) {
     const int bn = choose_bn_dq(avg), slots = cdiv(P, bn) + L->K;

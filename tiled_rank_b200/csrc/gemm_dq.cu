@@ -28,12 +28,11 @@
 //   warp 0      producer: bulk copies of the codes and their (scale, zero)
 //               words in chunks of 4 K blocks per projection (code ring), 2-D
 //               TMA boxes of B per round (activation ring);
-//   warp 1      MMA issuer: waits for a round's operand slot; one elected lane
-//               issues and commits to the operand slot, the activation stage
-//               and the accumulator;
+//   warp 1      MMA issuer: waits for a round's operand slot, activations and
+//               accumulator slot; one elected lane issues and commits to the
+//               operand slot, the activation stage and the accumulator;
 //   warps 2..9  decode: two warps per TMEM lane quadrant (32 weight rows), one
-//               per slice, write every round into its operand slot once its
-//               activations have landed and its accumulator slot is free;
+//               per slice, write every round into its operand slot;
 //   warps 10..13 fold + epilogue: one warp per lane quadrant folds every
 //               round's accumulators with the group scales and stores units.
 // Every wait is bounded and reports TILEQ_ERR_TIMEOUT.
@@ -50,41 +49,52 @@ constexpr int DQ_THREADS = (2 + DQ_DEC + DQ_FW) * 32;  // + producer + MMA issue
 constexpr int DQ_GRID = 148;                          // one CTA per SM
 constexpr int DQ_MAX_ROUNDS = 1024;                   // rounds of one CTA (its descriptor table)
 
-template <int NP, int BN>
+template <int NP, int BN, bool F8>
 struct DqCfg {
-  static constexpr int ATOM = BN * 128;                // one 64-wide fp16 K atom of B: BN rows x 128 B
-  static constexpr int B_BYTES = 4 * ATOM;             // up to four atoms per round
-  // The codes stream from HBM in chunks of CB consecutive 128-wide K blocks
-  // per projection (one bulk copy each, with the (scale, zero) words of their
-  // groups), several chunks in flight.
+  static constexpr int ATOM = BN * 128;  // one 128-byte-wide K atom of B: BN rows x 128 B
+  // B atoms per round: fp8 mode two (the two e4m3 pieces of 128 K, or one
+  // 64-wide fp16 extension atom per slice), else up to four
+  static constexpr int B_ROUND = (F8 ? 2 : 4) * ATOM;
+  // A chunk is RPC consecutive rounds of one kind (residual or extension) of
+  // a unit: the codes of CB K blocks per projection, their (scale, zero)
+  // words and the rounds' activation tiles, loaded together by one warp
+  // instruction with one copy per lane.  (A single thread completes about one
+  // bulk copy per memory latency, so the copies of a chunk go out in parallel.)
   static constexpr int CB = NP == 2 ? 2 : 4;
-  static constexpr int RPC = NP == 2 ? CB : CB / 2;     // main rounds per chunk
-  static constexpr int CODE_SLOT = NP * CB * (4096 + 512);
-  // activation ring (per round): its tiles come from L2 with a latency of a few
-  // rounds, so the ring runs deep
-  static constexpr int NB = 8;
-  static constexpr int NC_RAW = (200 * 1024 - NB * B_BYTES) / CODE_SLOT;
-  static constexpr int NC = NC_RAW > 6 ? 6 : NC_RAW;   // code chunk ring
-  static constexpr int CODE_OFF = NB * B_BYTES;
-  static constexpr int MAX_KB = 256;                   // K blocks of 128 (d_in up to 32768)
-  static constexpr int GIDX_OFF = CODE_OFF + NC * CODE_SLOT;  // [MAX_KB] scale group of each K block
+  static constexpr int RPC = 2;
+  static constexpr int SZ_OFF = NP * CB * 4096;
+  static constexpr int B_OFF = (SZ_OFF + NP * CB * 512 + 1023) / 1024 * 1024;
+  static constexpr int SLOT = B_OFF + RPC * B_ROUND;
+  static constexpr int NC_RAW = 196 * 1024 / SLOT;
+  static constexpr int NC = NC_RAW > 8 ? 8 : NC_RAW;  // chunk ring
+  static constexpr int MAX_KB = 256;                  // K blocks of 128 (d_in up to 32768)
+  static constexpr int GIDX_OFF = NC * SLOT;          // [MAX_KB] scale group of each K block
   static constexpr int TAB_OFF = GIDX_OFF + MAX_KB * 4;  // [DQ_MAX_ROUNDS] round descriptors
-  static constexpr int BAR_OFF = TAB_OFF + DQ_MAX_ROUNDS * 8;
-  // Tensor memory: NA operand slots of one round (two slices of 64 columns),
-  // then NT accumulator slots of one round (two slices of BN columns).
+  // the decode warps hand each row's group scale to the fold warps through a
+  // ring of NS rounds, so that a chunk is free once decoded
+  static constexpr int NS = 16;
+  static constexpr int SBUF_OFF = TAB_OFF + DQ_MAX_ROUNDS * 8;  // [NS][2 slices][128 rows] fp16
+  static constexpr int BAR_OFF = SBUF_OFF + NS * 2 * 128 * 2;
+  // Tensor memory: NA operand slots of one round (two slices: 128 K of e4m3
+  // or 64 fp16 in fp8 mode, 128 fp16 otherwise), then NT accumulator slots of
+  // one round (two slices of BN columns).
+  static constexpr int EXT_W = F8 ? 64 : 128;  // rank columns of a slice in an extension round
   static constexpr int NT = 4;
   static constexpr int ACC_COLS = 2 * BN;
-  static constexpr int A_COLS = 128;
+  static constexpr int A_COLS = F8 ? 64 : 128;
+  static constexpr int SCOLS = A_COLS / 2;
   static constexpr int NA_RAW = (512 - NT * ACC_COLS) / A_COLS;
   static constexpr int NA = NA_RAW > 4 ? 4 : NA_RAW;
   static constexpr int ACC0 = NA * A_COLS;
-  static constexpr int NBAR = 2 * NB + 2 * NC + 2 * NA + 2 * NT + 1;
+  static constexpr int NBAR = 2 * NC + 2 * NA + 2 * NT + NS + 1;
   static constexpr int SMEM = BAR_OFF + NBAR * 8 + 16 + BN * 4 + 1024;  // + slack to align the base
-  static_assert(NC >= 4, "code ring too shallow");
+  static_assert(NC >= 3, "chunk ring too shallow");
+  static_assert(2 * NP + RPC * 4 <= 32, "one copy per lane");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(NA >= 2, "operand ring too shallow");
+  static_assert(NS > NA + NT, "scale ring: the decode runs at most NA + NT rounds ahead of the fold");
   static_assert(ACC0 + NT * ACC_COLS <= 512, "tensor memory");
-  static_assert(ATOM % 1024 == 0, "swizzled atoms need 1024-byte alignment");
+  static_assert(ATOM % 1024 == 0 && B_OFF % 1024 == 0 && SLOT % 1024 == 0, "swizzled atoms need 1024-byte alignment");
 };
 
 // Bounded wait that lets the hardware suspend the warp until the phase
@@ -175,45 +185,40 @@ template <int NP, int BN, bool F8>
 __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_constant__ DqArgs P) {
   static_assert(!F8 || NP == 2, "fp8 mode: gate/up");
   static_assert(BN == 16 || BN == 32, "16 or 32 items per tile");
-  using C = DqCfg<NP, BN>;
+  using C = DqCfg<NP, BN, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *b_full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);  // [NB] activations of a round
-  uint64_t *b_empty = b_full + C::NB;
-  uint64_t *c_full = b_empty + C::NB;  // [NC] code chunks
+  uint64_t *c_full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);  // [NC] chunks
   uint64_t *c_empty = c_full + C::NC;
   uint64_t *a_full = c_empty + C::NC;  // [NA] operand slots
   uint64_t *a_free = a_full + C::NA;
   uint64_t *acc_full = a_free + C::NA;  // [NT] accumulator slots
   uint64_t *acc_free = acc_full + C::NT;
-  uint64_t *drain = acc_free + C::NT;
+  uint64_t *s_full = acc_free + C::NT;  // [NS] scales of a round written
+  uint64_t *drain = s_full + C::NS;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
   int *fin_tok = flag + 1;  // [BN]: combine, this CTA's slot was its token's last of the row block
   int *gidx = reinterpret_cast<int *>(smem + C::GIDX_OFF);
   int2 *tab = reinterpret_cast<int2 *>(smem + C::TAB_OFF);
+  unsigned short *sbuf = reinterpret_cast<unsigned short *>(smem + C::SBUF_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  auto st_b = [&](int s) { return smem + s * C::B_BYTES; };
-  // code chunk slot c: [projection][CB blocks of 4 KB], then [projection][CB groups of 128 (scale, zero) words]
-  auto ch_codes = [&](int c, int p) { return smem + C::CODE_OFF + c * C::CODE_SLOT + p * C::CB * 4096; };
-  auto ch_sz = [&](int c, int p) {
-    return reinterpret_cast<uint32_t *>(smem + C::CODE_OFF + c * C::CODE_SLOT + NP * C::CB * 4096) + p * C::CB * 128;
-  };
+  // chunk slot c: [projection][CB blocks of 4 KB] codes, [projection][CB groups of 128] (scale, zero)
+  // words, then the activation tiles of its rounds
+  auto ch_codes = [&](int c, int p) { return smem + c * C::SLOT + p * C::CB * 4096; };
+  auto ch_sz = [&](int c, int p) { return reinterpret_cast<uint32_t *>(smem + c * C::SLOT + C::SZ_OFF) + p * C::CB * 128; };
+  auto ch_b = [&](int c, int pos) { return smem + c * C::SLOT + C::B_OFF + pos * C::B_ROUND; };
 
   const int nkb = P.d_in / 128;
   const int nmain = NP == 2 ? nkb : (nkb + 1) / 2;
-  const int n_ext = P.rank > 0 ? (NP == 2 ? (P.rank + 127) / 128 : (P.rank + 255) / 256) : 0;
+  const int n_ext = P.rank > 0 ? (NP == 2 ? (P.rank + C::EXT_W - 1) / C::EXT_W : (P.rank + 255) / 256) : 0;
   const int R = nmain + n_ext;  // rounds per unit
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NB; ++s) {
-      mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
-    }
     for (int c = 0; c < C::NC; ++c) {
       mbar_init(&c_full[c], 1);
-      mbar_init(&c_empty[c], DQ_DEC + DQ_FW);
+      mbar_init(&c_empty[c], DQ_DEC + 1);  // the decode warps (codes) and the MMA warp (activations)
     }
     for (int j = 0; j < C::NA; ++j) {
       mbar_init(&a_full[j], DQ_DEC);
@@ -223,6 +228,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
       mbar_init(&acc_full[j], 1);
       mbar_init(&acc_free[j], DQ_FW);
     }
+    for (int j = 0; j < C::NS; ++j) mbar_init(&s_full[j], DQ_DEC);
     mbar_init(drain, 1);
     *flag = 0;
     fence_mbar_init();
@@ -244,46 +250,63 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
   const int nr = nr_all <= DQ_MAX_ROUNDS ? nr_all : 0;
   if (nr_all > DQ_MAX_ROUNDS && threadIdx.x == 0) set_status(P.status, TILEQ_ERR_UNSUPPORTED);
 
-  // ---- the round table.  Code chunks hold C::RPC consecutive main rounds of a
-  // unit from the first main round this CTA processes in it; units strictly
-  // inside the range are whole, so the chunks before a unit have a closed form.
+  // ---- the round table.  A chunk holds up to RPC consecutive rounds of one
+  // kind (residual, then extension) of a unit, counted from the first round of
+  // that kind this CTA processes in the unit.  Units strictly inside the range
+  // are whole, so the chunks before a unit have a closed form.
   {
     const long long u0 = r0 / R;
     const int rr0 = (int)(r0 - u0 * R);
-    auto rr_hi_of = [&](long long u) { return (int)min((long long)nmain, r1 - u * R); };
-    auto nch = [&](long long u, int lo) {
-      const int hi = rr_hi_of(u);
-      return hi > lo ? (hi - lo + C::RPC - 1) / C::RPC : 0;
+    auto cdv = [](int a, int b) { return (a + b - 1) / b; };
+    // rounds [lo, hi) of unit u in this CTA, split into residual and extension runs
+    auto lo_of = [&](long long u) { return u == u0 ? rr0 : 0; };
+    auto hi_of = [&](long long u) { return (int)min((long long)R, r1 - u * R); };
+    auto n_main_ch = [&](long long u) {
+      const int lo = lo_of(u), hi = min(hi_of(u), nmain);
+      return hi > lo ? cdv(hi - lo, C::RPC) : 0;
     };
-    const int nch0 = nch(u0, rr0), nch_full = (nmain + C::RPC - 1) / C::RPC;
+    auto n_ext_ch = [&](long long u) {
+      const int lo = max(lo_of(u), nmain), hi = hi_of(u);
+      return hi > lo ? cdv(hi - lo, C::RPC) : 0;
+    };
+    const int nch0 = n_main_ch(u0) + n_ext_ch(u0);
+    const int nch_full = cdv(nmain, C::RPC) + cdv(n_ext, C::RPC);
     for (int i = threadIdx.x; i < nr; i += blockDim.x) {
       const long long r = r0 + i;
       const long long unit = r / R;
       const int rr = (int)(r - unit * R);
+      const int lo = lo_of(unit), hi = hi_of(unit);
+      const int before = unit == u0 ? 0 : nch0 + (int)(unit - u0 - 1) * nch_full;
       uint32_t f = (rr == R - 1 || i == nr - 1) ? RD_UEND : 0u;
+      int idx, pos, last;
       if (rr < nmain) {
-        const int lo = unit == u0 ? rr0 : 0, hi = rr_hi_of(unit);
-        const int idx = (unit == u0 ? 0 : nch0 + (int)(unit - u0 - 1) * nch_full) + (rr - lo) / C::RPC;
-        const int pos = (rr - lo) % C::RPC;
+        idx = before + (rr - lo) / C::RPC;
+        pos = (rr - lo) % C::RPC;
+        last = min(hi, nmain) - 1;
         const int kb_a = NP == 2 ? rr - pos : 2 * (rr - pos);
         const int kb0 = NP == 2 ? rr : 2 * rr, kb1 = NP == 2 ? rr : 2 * rr + 1;
         const int ga = (kb_a * 128) / P.group;
-        f |= RD_V0 | (pos == 0 ? RD_CSTART : 0u) | (pos == C::RPC - 1 || rr == hi - 1 ? RD_CEND : 0u);
-        f |= (uint32_t)(idx % C::NC) << 8 | (uint32_t)((idx / C::NC) & 1) << 11;
+        f |= RD_V0;
         f |= (uint32_t)(kb0 - kb_a) << 20 | (uint32_t)((kb0 * 128) / P.group - ga) << 24;
         if (kb1 < nkb) f |= RD_V1 | (uint32_t)(kb1 - kb_a) << 22 | (uint32_t)((kb1 * 128) / P.group - ga) << 26;
       } else {
+        const int lo_e = max(lo, nmain);
+        idx = before + n_main_ch(unit) + (rr - lo_e) / C::RPC;
+        pos = (rr - lo_e) % C::RPC;
+        last = hi - 1;
         const int e = rr - nmain;
         f |= RD_EXT;
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
           const int ch = NP == 2 ? e : 2 * e + sl;
-          if (ch * 128 < P.rank) {
-            f |= (sl ? RD_V1 : RD_V0) | (uint32_t)((min(128, P.rank - ch * 128) + 15) / 16) << (sl ? 16 : 12) |
+          if (ch * C::EXT_W < P.rank) {
+            f |= (sl ? RD_V1 : RD_V0) | (uint32_t)((min(C::EXT_W, P.rank - ch * C::EXT_W) + 15) / 16) << (sl ? 16 : 12) |
                  (uint32_t)ch << (sl ? 30 : 28);
           }
         }
       }
+      f |= (pos == 0 ? RD_CSTART : 0u) | (pos == C::RPC - 1 || rr == last ? RD_CEND : 0u) | (uint32_t)pos << 6;
+      f |= (uint32_t)(idx % C::NC) << 8 | (uint32_t)((idx / C::NC) & 1) << 11;
       tab[i] = make_int2((int)f, (int)(unit << 9 | rr));
     }
   }
@@ -295,93 +318,124 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
 
   if (warp == 0) {
     // ============================================================ producer
-    if (lane == 0) {
-      int i = 0, nch_issued = 0;
-      long long cur_unit = -1;
-      int grp = 0, item0 = 0, ob = 0;
-      for (; i < nr; ++i) {
-        const int2 t = tab[i];
-        const uint32_t f = (uint32_t)t.x;
-        const long long unit = (unsigned)t.y >> 9;
-        const int rr = t.y & 511;
-        if (unit != cur_unit) {  // the tile changes with the unit only
-          cur_unit = unit;
-          const int jt = (int)(unit / P.m_tiles);
-          ob = (int)(unit - (long long)jt * P.m_tiles);
-          const int4 tl = P.tiles[jt];
-          grp = tl.x;
-          item0 = tl.y;
-        }
-        if (f & RD_CSTART) {
-          // the next code chunk: main rounds rr .. min(rr + RPC, this CTA's last of the unit) - 1
-          const int c = (int)rd_field(f, 8, 3);
-          if (nch_issued >= C::NC && !(ok = mbar_wait_sleep(&c_empty[c], rd_field(f, 11, 1) ^ 1u, P.status))) break;
-          const int r_b = min(rr + C::RPC, (int)min((long long)nmain, r1 - unit * R));
-          const int kb_a = NP == 2 ? rr : 2 * rr, kb_b = NP == 2 ? r_b : min(nkb, 2 * r_b);
-          const int g_a = gidx[kb_a], g_b = gidx[kb_b - 1];
-          const uint32_t cbytes = (uint32_t)(kb_b - kb_a) * 4096, zbytes = (uint32_t)(g_b - g_a + 1) * 512;
-          mbar_arrive_expect_tx(&c_full[c], NP * (cbytes + zbytes));
-          for (int p = 0; p < NP; ++p) {
-            const size_t blk = ((size_t)grp * P.m_tiles + ob) * nkb + kb_a;
-            bulk_g2s(ch_codes(c, p), reinterpret_cast<const uint8_t *>(P.codes[p]) + blk * 4096, cbytes, &c_full[c]);
-            const size_t zoff = (((size_t)grp * P.m_tiles + ob) * (nkb * 128 / P.group) + g_a) * 128;
-            bulk_g2s(ch_sz(c, p), P.sz[p] + zoff, zbytes, &c_full[c]);
-          }
-          ++nch_issued;
-        }
-        // the round's activation tile
-        const int s = i % C::NB;
-        if (i >= C::NB && !(ok = mbar_wait_sleep(&b_empty[s], ((i / C::NB) - 1) & 1, P.status))) break;
-        uint8_t *bs = st_b(s);
-        if (!(f & RD_EXT)) {
-          const int kb0 = NP == 2 ? rr : 2 * rr;
-          if (F8) {
-            // the two e4m3 pieces of the 128 K of this block (one 128-byte box each)
-            mbar_arrive_expect_tx(&b_full[s], 2u * C::ATOM);
-            for (int pc = 0; pc < 2; ++pc)
-              tc::tma_load_2d(bs + pc * C::ATOM, &P.bmap, pc * P.d_in + kb0 * 128, item0, &b_full[s]);
-          } else {
-            const int nsl = (NP == 1 && (f & RD_V1)) ? 2 : 1;
-            mbar_arrive_expect_tx(&b_full[s], (uint32_t)(2 * nsl) * C::ATOM);
-            for (int sl = 0; sl < nsl; ++sl)
-              for (int a = 0; a < 2; ++a)
-                tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, &P.bmap, (kb0 + sl) * 128 + a * 64, item0, &b_full[s]);
-          }
+    // The whole warp walks the chunks; lane k issues the chunk's k-th copy.
+    int n_issued = 0;
+    long long cur_unit = -1;
+    int grp = 0, item0 = 0, ob = 0;
+    for (int i = 0; i < nr; ++i) {
+      const uint32_t f = (uint32_t)tab[i].x;
+      if (!(f & RD_CSTART)) continue;
+      int cnt = 1;
+      while (!((uint32_t)tab[i + cnt - 1].x & RD_CEND)) ++cnt;
+      const long long unit = (unsigned)tab[i].y >> 9;
+      const int rr = tab[i].y & 511;
+      if (unit != cur_unit) {  // the tile changes with the unit only
+        cur_unit = unit;
+        const int jt = (int)(unit / P.m_tiles);
+        ob = (int)(unit - (long long)jt * P.m_tiles);
+        const int4 tl = P.tiles[jt];
+        grp = tl.x;
+        item0 = tl.y;
+      }
+      const int c = (int)rd_field(f, 8, 3);
+      if (n_issued >= C::NC) {
+        if (lane == 0) ok = mbar_wait_sleep(&c_empty[c], rd_field(f, 11, 1) ^ 1u, P.status);
+        if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+      }
+      // this lane's copy: destination, source (bulk) or coordinates (TMA), bytes
+      uint32_t bytes = 0;
+      int kind = 0;  // 1 bulk, 2 TMA (bmap), 3 TMA (bmap_ext)
+      void *dst = nullptr;
+      const void *src = nullptr;
+      int tx = 0;
+      int k = lane;
+      if (!(f & RD_EXT)) {
+        const int kb_a = NP == 2 ? rr : 2 * rr;
+        const int kb_b = NP == 2 ? rr + cnt : min(nkb, 2 * (rr + cnt));
+        const int g_a = gidx[kb_a], g_b = gidx[kb_b - 1];
+        if (k < NP) {
+          kind = 1;
+          bytes = (uint32_t)(kb_b - kb_a) * 4096;
+          dst = ch_codes(c, k);
+          src = reinterpret_cast<const uint8_t *>(P.codes[k]) + (((size_t)grp * P.m_tiles + ob) * nkb + kb_a) * 4096;
+        } else if (k < 2 * NP) {
+          const int p = k - NP;
+          kind = 1;
+          bytes = (uint32_t)(g_b - g_a + 1) * 512;
+          dst = ch_sz(c, p);
+          src = P.sz[p] + (((size_t)grp * P.m_tiles + ob) * (nkb * 128 / P.group) + g_a) * 128;
         } else {
-          int na = 0;
-          for (int sl = 0; sl < 2; ++sl)
-            if (f & (sl ? RD_V1 : RD_V0)) na += ((int)rd_field(f, sl ? 16 : 12, 4) + 3) / 4;
-          mbar_arrive_expect_tx(&b_full[s], (uint32_t)na * C::ATOM);
-          for (int sl = 0; sl < 2; ++sl) {
-            if (!(f & (sl ? RD_V1 : RD_V0))) continue;
+          k -= 2 * NP;
+          if (F8) {  // the two e4m3 pieces of each round's 128 K (one 128-byte box each)
+            const int pos = k / 2, pc = k % 2;
+            if (pos < cnt) {
+              kind = 2;
+              dst = ch_b(c, pos) + pc * C::ATOM;
+              tx = pc * P.d_in + (rr + pos) * 128;
+            }
+          } else if (NP == 2) {  // fp16: two 64-wide atoms per round, shared by both projections
+            const int pos = k / 2, a = k % 2;
+            if (pos < cnt) {
+              kind = 2;
+              dst = ch_b(c, pos) + a * C::ATOM;
+              tx = (rr + pos) * 128 + a * 64;
+            }
+          } else {  // one projection: two K blocks per round, two atoms each
+            const int pos = k / 4, sl = (k / 2) % 2, a = k % 2;
+            if (pos < cnt && 2 * (rr + pos) + sl < nkb) {
+              kind = 2;
+              dst = ch_b(c, pos) + (2 * sl + a) * C::ATOM;
+              tx = (2 * (rr + pos) + sl) * 128 + a * 64;
+            }
+          }
+          if (kind) bytes = C::ATOM;
+        }
+      } else {
+        // extension rounds: the item rows' z (or a) columns of each valid slice
+        constexpr int APS = C::EXT_W / 64;  // atoms per slice
+        const int pos = k / (2 * APS), sl = (k / APS) % 2, a = k % APS;
+        if (pos < cnt) {
+          const uint32_t fp = (uint32_t)tab[i + pos].x;
+          const int nat = ((int)rd_field(fp, sl ? 16 : 12, 4) + 3) / 4;
+          if ((fp & (sl ? RD_V1 : RD_V0)) && a < nat) {
             const int p = NP == 2 ? sl : 0;
-            const int ch = (int)rd_field(f, sl ? 30 : 28, 2);
-            const int nat = ((int)rd_field(f, sl ? 16 : 12, 4) + 3) / 4;
-            for (int a = 0; a < nat; ++a)
-              tc::tma_load_2d(bs + (2 * sl + a) * C::ATOM, F8 ? &P.bmap_ext : &P.bmap, P.ext_col[p] + ch * 128 + a * 64,
-                              item0, &b_full[s]);
+            kind = F8 ? 3 : 2;
+            bytes = C::ATOM;
+            dst = ch_b(c, pos) + (sl * APS + a) * C::ATOM;
+            tx = P.ext_col[p] + (int)rd_field(fp, sl ? 30 : 28, 2) * C::EXT_W + a * 64;
           }
         }
       }
-      // no copy may still be landing in shared memory when the CTA exits
-      for (int j = i > C::NB ? i - C::NB : 0; j < i; ++j)
-        mbar_wait_sleep(&b_full[j % C::NB], (j / C::NB) & 1, P.status);
-      for (int j = nch_issued > C::NC ? nch_issued - C::NC : 0; j < nch_issued; ++j)
-        mbar_wait_sleep(&c_full[j % C::NC], (j / C::NC) & 1, P.status);
+      const uint32_t total_bytes = __reduce_add_sync(0xffffffffu, bytes);
+      if (lane == 0) mbar_arrive_expect_tx(&c_full[c], total_bytes);
+      __syncwarp();
+      if (kind == 1) {
+        bulk_g2s(dst, src, bytes, &c_full[c]);
+      } else if (kind == 2) {
+        tc::tma_load_2d(dst, &P.bmap, tx, item0, &c_full[c]);
+      } else if (kind == 3) {
+        tc::tma_load_2d(dst, &P.bmap_ext, tx, item0, &c_full[c]);
+      }
+      ++n_issued;
     }
+    // no copy may still be landing in shared memory when the CTA exits
+    if (lane == 0)
+      for (int j = n_issued > C::NC ? n_issued - C::NC : 0; j < n_issued; ++j)
+        mbar_wait_sleep(&c_full[j % C::NC], (j / C::NC) & 1, P.status);
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    // One decode warp arrives on a round's operand slot only once the round's
-    // activations have landed and its accumulator slot is free, so this warp
-    // waits on one barrier per round.
     constexpr uint32_t idesc = tc::idesc_f16(BN);
     for (int i = 0; i < nr; ++i) {
-      const int as = i % C::NA, bs = i % C::NB, ts = i % C::NT;
-      if (!(ok = mbar_wait_sleep(&a_full[as], (i / C::NA) & 1, P.status))) break;
-      tc::fence_after();
       const uint32_t f = (uint32_t)tab[i].x;
+      const int as = i % C::NA, ts = i % C::NT, c = (int)rd_field(f, 8, 3);
+      const uint32_t acc_par = ((i / C::NT) - 1) & 1;
+      const bool acc_ready = i < C::NT || mbar_test(&acc_free[ts], acc_par);
+      if ((f & RD_CSTART) && !(ok = mbar_wait_sleep(&c_full[c], rd_field(f, 11, 1), P.status))) break;
+      if (!(ok = mbar_wait_sleep(&a_full[as], (i / C::NA) & 1, P.status))) break;
+      if (!acc_ready && !(ok = mbar_wait_sleep(&acc_free[ts], acc_par, P.status))) break;
+      tc::fence_after();
       if (tc::elect_one()) {
-        const uint64_t bd0 = tc::sdesc_sw128(smem_addr(st_b(bs)));
+        const uint64_t bd0 = tc::sdesc_sw128(smem_addr(ch_b(c, (int)rd_field(f, 6, 2))));
         const uint32_t a0 = tmem + as * C::A_COLS, d0 = tmem + C::ACC0 + ts * C::ACC_COLS;
         if (!(f & RD_EXT) && F8) {
           // e4m3: four K = 32 steps over 128 K per slice, both pieces of B into the same accumulator
@@ -391,8 +445,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
             for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
               for (int pc = 0; pc < 2; ++pc)
-                tc::mma_ts_f8(d0 + sl * BN, a0 + sl * 64 + kk * 8, bd0 + (uint64_t)((pc * C::ATOM + kk * 32) >> 4), idesc,
-                              (kk | pc) ? 1u : 0u);
+                tc::mma_ts_f8(d0 + sl * BN, a0 + sl * C::SCOLS + kk * 8, bd0 + (uint64_t)((pc * C::ATOM + kk * 32) >> 4),
+                              idesc, (kk | pc) ? 1u : 0u);
         } else if (!(f & RD_EXT)) {
           // fp16: eight K = 16 steps per slice; the two projections of np = 2 share B atoms 0, 1
 #pragma unroll
@@ -401,7 +455,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
             const int atom0 = NP == 2 ? 0 : 2 * sl;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              tc::mma_ts(d0 + sl * BN, a0 + sl * 64 + kk * 8,
+              tc::mma_ts(d0 + sl * BN, a0 + sl * C::SCOLS + kk * 8,
                          bd0 + (uint64_t)((((atom0 + kk / 4) * C::ATOM) + (kk % 4) * 32) >> 4), idesc, kk ? 1u : 0u);
           }
         } else {
@@ -409,15 +463,17 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
             if (!(f & (sl ? RD_V1 : RD_V0))) continue;
             const int nk = (int)rd_field(f, sl ? 16 : 12, 4);
             for (int kk = 0; kk < nk; ++kk)
-              tc::mma_ts(d0 + sl * BN, a0 + sl * 64 + kk * 8,
-                         bd0 + (uint64_t)((((2 * sl + kk / 4) * C::ATOM) + (kk % 4) * 32) >> 4), idesc, kk ? 1u : 0u);
+              tc::mma_ts(d0 + sl * BN, a0 + sl * C::SCOLS + kk * 8,
+                         bd0 + (uint64_t)((((sl * (C::EXT_W / 64) + kk / 4) * C::ATOM) + (kk % 4) * 32) >> 4), idesc,
+                         kk ? 1u : 0u);
           }
         }
-        // the operand slot and the activation stage are free once these MMAs
-        // have read them; the accumulators are then ready to fold
+        // the operand slot is free once these MMAs have read it, the
+        // accumulators are then ready to fold, and the chunk's activations are
+        // done with after its last round
         tc::commit(&a_free[as]);
-        tc::commit(&b_empty[bs]);
         tc::commit(&acc_full[ts]);
+        if (f & RD_CEND) tc::commit(&c_empty[c]);
       }
       __syncwarp();
     }
@@ -433,9 +489,22 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
     // the barrier's latency overlaps the decoding.
     const int dw = warp - 2;
     const int sl = dw / 4;
-    const bool gate = dw == 0;  // this warp also stands for the MMA warp's other conditions
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = tc::lane_base(warp);
+    // a round's stores complete while the warp decodes the next round: its
+    // operand slot is then published (one round late)
+    int prev_as = -1, prev_s = 0;
+    auto arrive_prev = [&]() {
+      if (prev_as < 0) return;
+      tc::wait_st();
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&a_full[prev_as]);
+        mbar_arrive(&s_full[prev_s]);
+      }
+      prev_as = -1;
+    };
     for (int i = 0; i < nr && ok; ++i) {
       const int2 t = tab[i];
       const uint32_t f = (uint32_t)t.x;
@@ -444,8 +513,9 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
       const uint32_t free_par = ((i / C::NA) - 1) & 1;
       bool slot_free = i < C::NA || mbar_test(&a_free[as], free_par);
       if ((f & RD_CSTART) && !(ok = mbar_wait_sleep(&c_full[c], rd_field(f, 11, 1), P.status))) break;
-      const uint32_t acol = tmem + lane_addr + as * C::A_COLS + sl * 64;
+      const uint32_t acol = tmem + lane_addr + as * C::A_COLS + sl * C::SCOLS;
       auto ensure_free = [&]() -> bool {
+        arrive_prev();  // the previous round's stores landed while this round decoded
         if (!slot_free && !mbar_wait_sleep(&a_free[as], free_par, P.status)) return false;
         slot_free = true;
         tc::fence_after();
@@ -456,6 +526,9 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
           const int p = NP == 2 ? sl : 0;
           const uint8_t *cb = ch_codes(c, p) + rd_field(f, 20 + 2 * sl, 2) * 4096;
           const uint32_t szw = ch_sz(c, p)[rd_field(f, 24 + 2 * sl, 2) * 128 + row];
+          // (the scale slot is written once the operand slot is free: the fold of
+          // the slot's previous round is then done)
+          auto put_scale = [&]() { sbuf[((i % C::NS) * 2 + sl) * 128 + row] = (unsigned short)(szw & 0xFFFFu); };
           uint2 wv[4];
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) wv[ks] = *reinterpret_cast<const uint2 *>(cb + ks * 1024 + row * 8);
@@ -481,6 +554,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
               }
             }
             if (!(ok = ensure_free())) break;
+            put_scale();
             tc::st32(acol, v);
           } else {
             const __half2 z2 = __high2half2(u32_as_h2(szw));
@@ -494,22 +568,25 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
                 dq_qz_word(wv[2 * hk + q].x, nz, v + 16 * q);
                 dq_qz_word(wv[2 * hk + q].y, nz, v + 16 * q + 8);
               }
-              if (hk == 0 && !(ok = ensure_free())) break;
+              if (hk == 0) {
+                if (!(ok = ensure_free())) break;
+                put_scale();
+              }
               tc::st32(acol + hk * 32, v);
             }
             if (!ok) break;
           }
         } else {
-          // rows of U_m: rank columns chunk * 128 ..
+          // rows of U_m: rank columns chunk * EXT_W ..
           const long long unit = (unsigned)t.y >> 9;
           const int jt = (int)(unit / P.m_tiles), ob = (int)(unit - (long long)jt * P.m_tiles);
           const int p = NP == 2 ? sl : 0;
           const int chunk = (int)rd_field(f, 28 + 2 * sl, 2);
-          const __half *ur =
-              P.u[p] + (((size_t)P.u_blk[p][P.tiles[jt].x] * P.m_tiles + ob) * 128 + row) * P.rank + chunk * 128;
-          const int kmax = P.rank - chunk * 128;
+          const __half *ur = P.u[p] + (((size_t)P.u_blk[p][P.tiles[jt].x] * P.m_tiles + ob) * 128 + row) * P.rank +
+                             chunk * C::EXT_W;
+          const int kmax = P.rank - chunk * C::EXT_W;
 #pragma unroll
-          for (int hk = 0; hk < 2; ++hk) {
+          for (int hk = 0; hk < C::EXT_W / 64; ++hk) {
             uint32_t v[32];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -529,18 +606,13 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
       // (a warp with nothing to write for the round still waits for the slot:
       // its arrival must not run ahead into the slot's previous phase)
       if (!(ok = ensure_free())) break;
-      if (gate) {
-        // the round's activations have landed and its accumulator slot is free
-        if (!(ok = mbar_wait_sleep(&b_full[i % C::NB], (i / C::NB) & 1, P.status))) break;
-        if (i >= C::NT && !(ok = mbar_wait_sleep(&acc_free[i % C::NT], ((i / C::NT) - 1) & 1, P.status))) break;
-      }
-      tc::wait_st();
-      tc::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[as]);
+      // the round's arrival waits for its stores, after the next round's decode
+      prev_as = as;
+      prev_s = i % C::NS;
       // the chunk's codes are decoded: the producer may refill its slot
       if ((f & RD_CEND) && lane == 0) mbar_arrive(&c_empty[c]);
     }
+    if (ok) arrive_prev();
   } else {
     // ============================================================ fold + epilogue
     // One warp per TMEM lane quadrant (32 weight rows): it folds both slices'
@@ -683,14 +755,16 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
       const int2 t = tab[i];
       const uint32_t f = (uint32_t)t.x;
       const int c = (int)rd_field(f, 8, 3);
-      // this row's scale of each slice (1 for the U_m extension); the chunk's
-      // codes were awaited by the decode warps before this round's MMAs
-      float s0 = 1.f, s1 = 1.f;
+      // this row's scale of each slice (1 for the U_m extension), handed over by the decode warps
+      const uint32_t s_par = (i / C::NS) & 1;
+      const bool s_ready = mbar_test(&s_full[i % C::NS], s_par);
       if (!(ok = mbar_wait_sleep(&acc_full[ts], (i / C::NT) & 1, P.status))) break;
+      if (!s_ready && !(ok = mbar_wait_sleep(&s_full[i % C::NS], s_par, P.status))) break;
       tc::fence_after();
+      float s0 = 1.f, s1 = 1.f;
       if (!(f & RD_EXT)) {
-        s0 = __low2float(u32_as_h2(ch_sz(c, 0)[rd_field(f, 24, 2) * 128 + row]));
-        s1 = __low2float(u32_as_h2(ch_sz(c, NP == 2 ? 1 : 0)[rd_field(f, 26, 2) * 128 + row]));
+        s0 = __half2float(__ushort_as_half(sbuf[((i % C::NS) * 2 + 0) * 128 + row]));
+        s1 = __half2float(__ushort_as_half(sbuf[((i % C::NS) * 2 + 1) * 128 + row]));
       }
       // tcgen05.ld is warp-collective: the decision is the warp's (the slice
       // was valid in round i), never a lane's (padding rows have scale 0)
@@ -700,7 +774,6 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
       tc::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_free[ts]);
-      if ((f & RD_CEND) && lane == 0) mbar_arrive(&c_empty[c]);
       if (f & RD_UEND) {
         const long long unit = (unsigned)t.y >> 9;
         const int jt = (int)(unit / P.m_tiles);
@@ -719,7 +792,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) gemm_dq_kernel(const __grid_con
 
 template <int NP, int BN, bool F8 = false>
 cudaError_t launch_dq(const DqArgs &a, cudaStream_t stream) {
-  using C = DqCfg<NP, BN>;
+  using C = DqCfg<NP, BN, F8>;
   auto kern = gemm_dq_kernel<NP, BN, F8>;
   static bool configured = false;  // one attribute call per instantiation and process
   if (!configured) {
