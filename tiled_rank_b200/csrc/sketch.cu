@@ -6,7 +6,8 @@
 //
 //   Y^T = Omega^T W_big^T                [l, R]   tcgen05 (bf16 in, fp32 out), W_big read by blocks
 //   G   = Y^T Y                          [l, l]   fp64 accumulation
-//   G   = E diag(lam) E^T                Jacobi, fp64, one CTA
+//   G   = E diag(lam) E^T                Jacobi, fp64: the rotations on one CTA (G in shared
+//                                        memory), then E from the logged rotations, rows in parallel
 //   Q^T = (E lam^-1/2)^T Y^T (lam > tol) [l, R]   orthonormal basis of range(Y), fp32
 //   B   = Q^T W_big                      [l, C]   tcgen05 on the experts' transposes, Q^T
 //                                                 split into two bf16 terms (hi + lo)
@@ -226,34 +227,34 @@ __global__ void sk_gram_reduce_kernel(const double *part, int l, int splits, dou
 }
 
 // Cyclic Jacobi eigen-decomposition of the symmetric l x l matrix G (fp64, l
-// even, l <= kSketchMaxL), one CTA.  Each round rotates l/2 disjoint index
-// pairs of the round-robin schedule (index 0 fixed, the others rotating), the
-// rotation of Golub and Van Loan's symmetric Schur step annihilating G[p][q];
-// sweeps of l-1 rounds until the off-diagonal mass is below (1e-13 ||G||)^2 or
-// kJacobiSweeps sweeps.  G lives in shared memory with a row stride of l + 1
-// (its columns are read too).  The eigenvectors accumulate transposed in
-// global memory, Et[q][j] = E[j][q], so that rotating columns p, q of E moves
-// two contiguous rows.  Then lam[i] = the i-th largest eigenvalue and perm[i]
-// the row of Et holding its eigenvector.
+// even, l <= kSketchMaxL).  Each round rotates l/2 disjoint index pairs of the
+// round-robin schedule (index 0 fixed, the others rotating), the rotation of
+// Golub and Van Loan's symmetric Schur step annihilating G[p][q]; sweeps of
+// l-1 rounds until the off-diagonal mass is below (1e-13 ||G||)^2 or
+// kJacobiSweeps sweeps.  One CTA applies the rotations to G, which lives in
+// shared memory with a row stride of l + 1 (its columns are read too), and
+// logs each round's (c, s, p, q); the eigenvectors E = J_1 J_2 ... are then
+// formed from the log by sk_jacobi_vectors_kernel, whose rows are independent
+// (a rotation of columns p, q of E changes each row on its own), so they run
+// in parallel instead of adding a global-memory round trip to every round.
+// lam[i] = the i-th largest eigenvalue and perm[i] the row of Et (= E^T)
+// holding its eigenvector.
 constexpr int kJacobiSweeps = 40;
 constexpr int kJacobiThreads = 1024;
-constexpr int kJacobiLaneCols = (kSketchMaxL + 31) / 32;  // row elements per lane
 
-__global__ void __launch_bounds__(kJacobiThreads) sk_jacobi_kernel(const double *Gin, int l, double *Et, double *lam,
-                                                                  int *perm) {
+__global__ void __launch_bounds__(kJacobiThreads) sk_jacobi_kernel(const double *Gin, int l, double *lam, int *perm,
+                                                                  double *log_c, double *log_s, int *log_pq,
+                                                                  int *n_rounds) {
   extern __shared__ double G[];  // [l][l + 1]
   __shared__ double rc[kSketchMaxL / 2], rs[kSketchMaxL / 2];
   __shared__ int rp[kSketchMaxL / 2], rq[kSketchMaxL / 2];
   __shared__ double red[32];
   __shared__ int done;
   const int tid = threadIdx.x, nt = blockDim.x;
-  const int warp = tid >> 5, lane = tid & 31, nwarp = nt >> 5;
   const int h = l / 2, ld = l + 1;
-  for (int e = tid; e < l * l; e += nt) {
-    G[(e / l) * ld + e % l] = Gin[e];
-    Et[e] = (e / l == e % l) ? 1.0 : 0.0;
-  }
+  for (int e = tid; e < l * l; e += nt) G[(e / l) * ld + e % l] = Gin[e];
   if (tid == 0) done = 0;
+  int rounds = 0;
   __syncthreads();
   auto block_sum = [&](double v) -> double {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -283,68 +284,53 @@ __global__ void __launch_bounds__(kJacobiThreads) sk_jacobi_kernel(const double 
     for (int t = 0; t < l - 1; ++t) {
       if (tid < h) {
         // round-robin pair i: positions i and l-1-i of [0, rotation of 1..l-1]
-        auto player = [&](int pos) { return pos == 0 ? 0 : ((pos - 1 + t) % (l - 1)) + 1; };
+        auto player = [&](int pos) {
+          if (pos == 0) return 0;
+          const int v = pos - 1 + t;  // < 2 (l - 1)
+          return (v >= l - 1 ? v - (l - 1) : v) + 1;
+        };
         int p = player(tid), q = player(l - 1 - tid);
         if (p > q) {
           const int x = p;
           p = q;
           q = x;
         }
+        // the symmetric Schur rotation annihilating G[p][q], in the form with
+        // one division: t = 2 a sign(d) / (|d| + sqrt(d^2 + 4 a^2)), d = G[q][q] - G[p][p]
         const double apq = G[p * ld + q];
         double c = 1.0, sn = 0.0;
         if (apq != 0.0) {
-          const double tau = (G[q * ld + q] - G[p * ld + p]) / (2.0 * apq);
-          const double tt = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
-          c = 1.0 / sqrt(1.0 + tt * tt);
+          const double d = G[q * ld + q] - G[p * ld + p];
+          const double tt = (d >= 0.0 ? 2.0 : -2.0) * apq / (fabs(d) + sqrt(d * d + 4.0 * apq * apq));
+          c = rsqrt(1.0 + tt * tt);
           sn = tt * c;
         }
         rc[tid] = c;
         rs[tid] = sn;
         rp[tid] = p;
         rq[tid] = q;
+        const size_t at = (size_t)rounds * h + tid;
+        log_c[at] = c;
+        log_s[at] = sn;
+        log_pq[at] = p | (q << 16);
       }
+      ++rounds;
       __syncthreads();
-      // rows p, q of every pair: J^T G; rows p, q of Et: (E J)^T.  One warp per
-      // pair, the lanes along the row (contiguous in G and in Et), the Et loads
-      // of the whole row out before its stores.
-      for (int i = warp; i < h; i += nwarp) {
-        const int p = rp[i], q = rq[i];
-        const double c = rc[i], sn = rs[i];
-        double ep[kJacobiLaneCols], eq[kJacobiLaneCols];
-#pragma unroll
-        for (int u = 0; u < kJacobiLaneCols; ++u) {
-          const int j = lane + 32 * u;
-          if (j < l) {
-            ep[u] = Et[(size_t)p * l + j];
-            eq[u] = Et[(size_t)q * l + j];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kJacobiLaneCols; ++u) {
-          const int j = lane + 32 * u;
-          if (j < l) {
-            const double gp = G[p * ld + j], gq = G[q * ld + j];
-            G[p * ld + j] = c * gp - sn * gq;
-            G[q * ld + j] = sn * gp + c * gq;
-            Et[(size_t)p * l + j] = c * ep[u] - sn * eq[u];
-            Et[(size_t)q * l + j] = sn * ep[u] + c * eq[u];
-          }
-        }
-      }
-      __syncthreads();
-      // columns p, q of every pair: (J^T G) J (odd row stride: conflict-free)
-      for (int i = warp; i < h; i += nwarp) {
-        const int p = rp[i], q = rq[i];
-        const double c = rc[i], sn = rs[i];
-#pragma unroll
-        for (int u = 0; u < kJacobiLaneCols; ++u) {
-          const int j = lane + 32 * u;
-          if (j < l) {
-            const double gp = G[j * ld + p], gq = G[j * ld + q];
-            G[j * ld + p] = c * gp - sn * gq;
-            G[j * ld + q] = sn * gp + c * gq;
-          }
-        }
+      // G <- J^T G J in one pass: the pairs partition the indices, so every
+      // 2 x 2 block (rows p_i, q_i; columns p_j, q_j) becomes J_i^T G_ij J_j on its own
+      for (int b = tid; b < h * h; b += nt) {
+        const int bi = b / h, bj = b - bi * h;
+        const int pi = rp[bi], qi = rq[bi], pj = rp[bj], qj = rq[bj];
+        const double ci = rc[bi], si = rs[bi], cj = rc[bj], sj = rs[bj];
+        const double g00 = G[pi * ld + pj], g01 = G[pi * ld + qj], g10 = G[qi * ld + pj], g11 = G[qi * ld + qj];
+        // rows: [c -s; s c] applied as in the two-pass form (row p <- c p - s q, row q <- s p + c q)
+        const double r00 = ci * g00 - si * g10, r01 = ci * g01 - si * g11;
+        const double r10 = si * g00 + ci * g10, r11 = si * g01 + ci * g11;
+        // columns: column p <- c p - s q, column q <- s p + c q
+        G[pi * ld + pj] = cj * r00 - sj * r01;
+        G[pi * ld + qj] = sj * r00 + cj * r01;
+        G[qi * ld + pj] = cj * r10 - sj * r11;
+        G[qi * ld + qj] = sj * r10 + cj * r11;
       }
       __syncthreads();
     }
@@ -360,6 +346,56 @@ __global__ void __launch_bounds__(kJacobiThreads) sk_jacobi_kernel(const double 
     lam[rank] = li;
     perm[rank] = i;
   }
+  if (tid == 0) *n_rounds = rounds;
+}
+
+// E = J_1 J_2 ... J_n from the rotation log, written transposed (Et[q][j] =
+// E[j][q]).  A CTA holds `rpb` rows of E in shared memory, starting from the
+// identity; in every round its thread (pair i, row r) rotates entries p_i, q_i
+// of row r (the round's pairs are disjoint), with the same arithmetic as a
+// column rotation of E.  The next round's (c, s, p, q) is loaded before the
+// round's barrier.
+__global__ void __launch_bounds__(1024) sk_jacobi_vectors_kernel(const double *log_c, const double *log_s,
+                                                               const int *log_pq, const int *n_rounds, int l, int rpb,
+                                                               double *Et) {
+  extern __shared__ double Er[];  // [rpb][l]
+  const int h = l / 2, tid = threadIdx.x;
+  const int row0 = blockIdx.x * rpb;
+  const int rows = min(rpb, l - row0);
+  for (int e = tid; e < rows * l; e += blockDim.x) Er[e] = (row0 + e / l == e % l) ? 1.0 : 0.0;
+  const int i = tid % h, r = tid / h;
+  const bool active = r < rows;
+  const int nr = *n_rounds;
+  double c = 0.0, sn = 0.0;
+  int pq = 0;
+  if (nr > 0) {
+    c = log_c[i];
+    sn = log_s[i];
+    pq = log_pq[i];
+  }
+  __syncthreads();
+  for (int t = 0; t < nr; ++t) {
+    double cn = 0.0, snn = 0.0;
+    int pqn = 0;
+    if (t + 1 < nr) {
+      const size_t at = (size_t)(t + 1) * h + i;
+      cn = log_c[at];
+      snn = log_s[at];
+      pqn = log_pq[at];
+    }
+    if (active) {
+      const int p = pq & 0xFFFF, q = pq >> 16;
+      double *er = Er + r * l;
+      const double ep = er[p], eq = er[q];
+      er[p] = c * ep - sn * eq;
+      er[q] = sn * ep + c * eq;
+    }
+    __syncthreads();
+    c = cn;
+    sn = snn;
+    pq = pqn;
+  }
+  for (int e = tid; e < rows * l; e += blockDim.x) Et[(size_t)(e % l) * l + row0 + e / l] = Er[e];
 }
 
 // Wsmall[j][i] = E[j][perm[i]] / sqrt(lam[i]) for eigenvalues above tol * lam[0]
@@ -410,7 +446,8 @@ cudaError_t gram(const float *X, bool xt, long long rows, int l, double *part, i
   return cudaGetLastError();
 }
 
-cudaError_t jacobi(const double *G, int l, double *E, double *lam, int *perm, cudaStream_t st) {
+cudaError_t jacobi(const double *G, int l, double *E, double *lam, int *perm, double *log_c, double *log_s,
+                   int *log_pq, int *n_rounds, cudaStream_t st) {
   const int smem = l * (l + 1) * (int)sizeof(double);
   static int configured = 0;
   if (smem > configured) {
@@ -419,7 +456,12 @@ cudaError_t jacobi(const double *G, int l, double *E, double *lam, int *perm, cu
     if (e != cudaSuccess) return e;
     configured = most;
   }
-  sk_jacobi_kernel<<<1, kJacobiThreads, smem, st>>>(G, l, E, lam, perm);
+  sk_jacobi_kernel<<<1, kJacobiThreads, smem, st>>>(G, l, lam, perm, log_c, log_s, log_pq, n_rounds);
+  count_launches();
+  const int h = l / 2;
+  const int rpb = 1024 / h < 16 ? 1024 / h : 16;  // rows of E per CTA
+  sk_jacobi_vectors_kernel<<<(l + rpb - 1) / rpb, h * rpb, (size_t)rpb * l * sizeof(double), st>>>(
+      log_c, log_s, log_pq, n_rounds, l, rpb, E);
   count_launches();
   return cudaGetLastError();
 }
@@ -463,7 +505,7 @@ cudaError_t tc_grid_product(const __nv_bfloat16 *a_arr, int K, int blk_rows, int
 
 // Workspace layout of the sketch (byte offsets, 256-byte aligned).
 struct SketchWs {
-  size_t wt, yt, qt, qhl, bo, part, g, e, lam, perm, wsmall, ur, inv_sigma, total;
+  size_t wt, yt, qt, qhl, bo, part, g, e, lam, perm, wsmall, ur, inv_sigma, log_c, log_s, log_pq, n_rounds, total;
 };
 
 static size_t sk_align(size_t x) { return (x + 255) / 256 * 256; }
@@ -489,6 +531,12 @@ static SketchWs sketch_ws(int K, long long R, long long C, int d_out, int d_in, 
   w.wsmall = take((size_t)l * l * 4);
   w.ur = take((size_t)l * r * 4);
   w.inv_sigma = take((size_t)r * 4);
+  // the rotation log of one Jacobi solve: at most kJacobiSweeps sweeps of l - 1 rounds of l/2 pairs
+  const size_t log_n = (size_t)kJacobiSweeps * (l - 1) * (l / 2);
+  w.log_c = take(log_n * 8);
+  w.log_s = take(log_n * 8);
+  w.log_pq = take(log_n * 4);
+  w.n_rounds = take(4);
   w.total = off;
   return w;
 }
@@ -546,6 +594,10 @@ extern "C" tileq_status tileq_sketch_lowrank(const tileq_wbig *wb, const void *o
   float *Wsmall = reinterpret_cast<float *>(base + w.wsmall);
   float *Ur = reinterpret_cast<float *>(base + w.ur);
   float *inv_sigma = reinterpret_cast<float *>(base + w.inv_sigma);
+  double *log_c = reinterpret_cast<double *>(base + w.log_c);
+  double *log_s = reinterpret_cast<double *>(base + w.log_s);
+  int *log_pq = reinterpret_cast<int *>(base + w.log_pq);
+  int *n_rounds = reinterpret_cast<int *>(base + w.n_rounds);
   int8_t cell_expert[kMaxExperts] = {};
   for (int k = 0; k < K; ++k) cell_expert[wb->grid_assign[k]] = (int8_t)k;
 
@@ -559,7 +611,7 @@ extern "C" tileq_status tileq_sketch_lowrank(const tileq_wbig *wb, const void *o
                      Yt, s));
   // orthonormal basis of range(Y) from the eigen-decomposition of Y^T Y
   SK(gram(Yt, true, R, l, part, kSketchGramSplits, G, s));
-  SK(jacobi(G, l, E, lam, perm, s));
+  SK(jacobi(G, l, E, lam, perm, log_c, log_s, log_pq, n_rounds, s));
   sk_basis_kernel<<<(l * l + 255) / 256, 256, 0, s>>>(E, lam, perm, l, kSketchBasisTol, Wsmall);
   count_launches();
   SK(cudaGetLastError());
@@ -579,7 +631,7 @@ extern "C" tileq_status tileq_sketch_lowrank(const tileq_wbig *wb, const void *o
   SK(cudaGetLastError());
   // eigen-decomposition of B B^T
   SK(gram(Bo, true, C, l, part, kSketchGramSplits, G, s));
-  SK(jacobi(G, l, E, lam, perm, s));
+  SK(jacobi(G, l, E, lam, perm, log_c, log_s, log_pq, n_rounds, s));
   sk_select_kernel<<<(l * r + 255) / 256, 256, 0, s>>>(E, lam, perm, l, r, Ur, sigma, inv_sigma);
   count_launches();
   SK(cudaGetLastError());
