@@ -168,7 +168,12 @@ tileq_status tileq_workspace_size(const tileq_layer *layer, int T, int top_k, si
  *   out             device bf16 [T, d_y]       (overwritten)
  *   ws, ws_bytes    device workspace, ws_bytes >= tileq_workspace_size(layer, T, top_k)
  *   route           optional copies of the routing results (NULL = none)
- * 1 <= top_k <= K; T >= 0 (T == 0 enqueues nothing).  Asynchronous. */
+ * 1 <= top_k <= K; T >= 0 (T == 0 enqueues nothing).  Asynchronous.
+ * Kernel choice: experts averaging <= 32 slots run their residual GEMMs on
+ * warp-level MMA, wider ones on tcgen05.  With the environment variable
+ * TILEQ_DECODE_TC=1 set when the library makes its first plan, 2-bit layers
+ * with groups of a multiple of 128 run the narrow case on the tcgen05 decode
+ * kernel instead (same results within the parity bar, measured slower). */
 tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, const void *x,
                                int T, const float *router_logits, int top_k, void *out,
                                void *ws, size_t ws_bytes, tileq_route_out *route,
