@@ -1,14 +1,15 @@
 // Residual GEMM of the decode regime (a handful of tokens per expert) on the
-// 5th-generation tensor cores, for the TileQ forward:
+// 5th-generation tensor cores, for the TileQ forward (opt-in: the planner
+// uses warp-level MMA for these tiles unless TILEQ_DECODE_TC=1):
 //
 //   out[item][o] = epi( sum_k s*(q - z)[o][k] * B[item][k]  +  sum_i U_m[o][i] * B[item][ext + i] )
 //
-// At decode the weight stream from HBM is the whole cost, so the kernel is
-// built around bytes in flight and instructions per weight:
-//   * the A operand is the exact q - z of each 2-bit code in fp16 (one AND-OR
-//     with the fp16 exponent of 1024 and one FMA per pair of weights), written
-//     to tensor memory; the tensor cores do every multiply (TS-form
-//     tcgen05.mma, M = 128 weight rows, N = 16..64 items);
+//   * the A operand is the exact q - z of each 2-bit code, written to tensor
+//     memory: in fp8 mode (gate/up) as e4m3 through a 4-byte table per zero
+//     point (one PRMT per 4 weights), with B as two e4m3 pieces of the
+//     activations; otherwise in fp16 (one AND-OR with the fp16 exponent of
+//     1024 and one FMA per pair of weights).  TS-form tcgen05.mma, M = 128
+//     weight rows, N = 16 or 32 items;
 //   * every 128-wide K block (one scale group, or part of one) accumulates
 //     into its own fp32 accumulator in tensor memory; the fold warps add it
 //     into registers with the group scale (w = s*(q - z) is never rounded);
@@ -23,18 +24,20 @@
 // slot holds rows of the grid row's U_m (fp16, read from global memory) and B
 // the matching z (or a) columns of the item rows, with scale 1.
 //
-// Warp roles (14 warps), each a pipeline stage with its own ring, so that a
-// round costs the slowest stage rather than the sum of all of them:
-//   warp 0      producer: bulk copies of the codes and their (scale, zero)
-//               words in chunks of 4 K blocks per projection (code ring), 2-D
-//               TMA boxes of B per round (activation ring);
-//   warp 1      MMA issuer: waits for a round's operand slot, activations and
-//               accumulator slot; one elected lane issues and commits to the
-//               operand slot, the activation stage and the accumulator;
-//   warps 2..9  decode: two warps per TMEM lane quadrant (32 weight rows), one
-//               per slice, write every round into its operand slot;
+// Warp roles (14 warps), each a pipeline stage with its own ring:
+//   warp 0       producer: per chunk (two rounds of one kind of a unit) the
+//                codes, their (scale, zero) words and the rounds' activation
+//                tiles into one ring slot, one copy per lane;
+//   warp 1       MMA issuer: waits for a round's chunk, operand slot and
+//                accumulator slot; one elected lane issues and commits to the
+//                operand slot, the accumulator slot and, after the chunk's
+//                last round, the chunk;
+//   warps 2..9   decode: two warps per TMEM lane quadrant (32 weight rows), one
+//                per slice, write every round into its operand slot and hand
+//                the rows' group scales to the fold warps;
 //   warps 10..13 fold + epilogue: one warp per lane quadrant folds every
-//               round's accumulators with the group scales and stores units.
+//                round's accumulators with the group scales and stores units.
+// A table of every round's descriptor is built before the pipeline starts.
 // Every wait is bounded and reports TILEQ_ERR_TIMEOUT.
 #include "kernels.cuh"
 #include "tc.cuh"
