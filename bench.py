@@ -649,19 +649,21 @@ def traffic_for(kernel, T, cfg):
         return None
     key = f"{kernel}:{cfg.name}:T={T}"
     ent = d.get(key)
-    if not ent or ent.get("source_sha") != source_sha():
+    if not ent or ent.get("source_sha") != source_sha(ent.get("sources")):
         return None
     return ent.get("dram_bytes_per_launch")
 
 
-def source_sha():
+def source_sha(files=None):
+    """Hash of the CUDA sources: the listed files of tiled_rank_b200/csrc (the
+    captured kernel's own file and its headers), or all of them."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "tiled_rank_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+    names = sorted(files) if files else sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for f in names:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
