@@ -406,6 +406,7 @@ struct WsLayout {
   Plan plan;
   size_t status, topk_idx, topk_w, expert_offsets, sorted_pairs, slot_of_pair, slot_tok, slot_w,
       dest, pcounts, tiles_main, tiles_wide, tile_first, tile_counts, counters, part;
+  size_t counters_sh, part_sh;  // split-K regions of the shared expert (it runs on a side stream)
   int n_counters;
   size_t part_zstride;
   size_t zidx[2];
@@ -467,15 +468,19 @@ WsLayout ws_layout(const tileq_layer *L, const LayerInfo &li, int T, int k, bool
   // + one arrival count per (token, output row block) for the combine fused
   // into the decode-regime down GEMM
   const int ntok = (pl.down.dq || pl.linear.dq) ? std::max(T, 1) * cdiv(li.d_y, 128) : 0;
-  w.n_counters = nc + ntok;
-  w.counters = take((size_t)(nc + ntok) * 4);
+  // + the shared expert's own counts: it runs beside the routed GEMMs
+  const int nsh = L->shared_d_ff > 0 ? std::max(pl.sh_gu.counters(1), pl.sh_down.counters(1)) : 0;
+  w.n_counters = nc + ntok + nsh;
+  w.counters = take((size_t)(nc + ntok + nsh) * 4);
   w.tokcnt = w.counters + (size_t)nc * 4;
+  w.counters_sh = w.tokcnt + (size_t)ntok * 4;
   size_t pf = 2 * pl.zproj.part_floats();
   w.part_zstride = pl.zproj.part_floats();
   for (const GemmPlan *g : {&pl.gateup, &pl.zdown, &pl.down, &pl.linear, &pl.sh_gu, &pl.sh_down, &pl.pe_zx,
                             &pl.pe_zd})
     pf = std::max(pf, g->part_floats());
   w.part = take(pf * 4);
+  w.part_sh = L->shared_d_ff > 0 ? take(std::max(pl.sh_gu.part_floats(), pl.sh_down.part_floats()) * 4) : w.part;
   for (int z = 0; z < 2; ++z) w.zidx[z] = take(Pz * 4);
   w.aidx = take(Pz * 4);
   w.x16 = take((size_t)std::max(T, 1) * li.d_x * 2);
@@ -940,6 +945,36 @@ tileq_status copy_route_out(const tileq_layer *L, const WsLayout &w, void *ws, i
 
 // The always-on shared expert (dense fp16 SwiGLU) into the fp32 buffer ys;
 // *yshared = ys, or null without a shared expert.
+// A side stream per host thread and device, with its fork and join events,
+// for work of a forward that does not depend on the routing (the shared
+// expert).  Created on first use; if that fails the work stays on the
+// caller's stream.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool tried = false, ok = false;
+};
+SideStream &side_stream() {
+  constexpr int kDevices = 64;
+  static thread_local SideStream per_device[kDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) {
+    cudaGetLastError();
+    static thread_local SideStream none;
+    none.tried = true;
+    return none;
+  }
+  SideStream &sd = per_device[dev];
+  if (!sd.tried) {
+    sd.tried = true;
+    sd.ok = cudaStreamCreateWithFlags(&sd.s, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming) == cudaSuccess;
+    if (!sd.ok) cudaGetLastError();
+  }
+  return sd;
+}
+
 tileq_status run_shared(const tileq_layer *L, const PackedLayout &pl, const WsLayout &w, const void *packed,
                         void *ws, int T, const float **yshared_out, cudaStream_t stream) {
   const float *yshared = nullptr;
@@ -1006,7 +1041,6 @@ tileq_status run_shared(const tileq_layer *L, const PackedLayout &pl, const WsLa
     if (gemm(b, 1, 1, w.plan.sh_down, stream) != TILEQ_OK) return TILEQ_ERR_CUDA;
     yshared = at<float>(ws, w.ys);
   }
-  mark(ST_SHARED, stream);
   *yshared_out = yshared;
   return TILEQ_OK;
 }
@@ -1289,6 +1323,23 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     if (st != TILEQ_OK) return st;
     const int D = layer->d_model, F = layer->d_ff;
     __half *hext = at<__half>(ws, w.hext);
+    // the shared expert reads x alone: it runs on the side stream from here,
+    // beside the routed GEMMs, with its own split-K regions
+    const float *yshared = nullptr;
+    SideStream *side = nullptr;
+    if (layer->shared_d_ff > 0) {
+      SideStream &sd = side_stream();
+      if (sd.ok) {
+        WsLayout wsh = w;
+        wsh.part = w.part_sh;
+        wsh.counters = w.counters_sh;
+        TQ_CUDA(cudaEventRecord(sd.fork, stream));
+        TQ_CUDA(cudaStreamWaitEvent(sd.s, sd.fork, 0));
+        if ((st = run_shared(layer, pl, wsh, packed, ws, T, &yshared, sd.s)) != TILEQ_OK) return st;
+        TQ_CUDA(cudaEventRecord(sd.join, sd.s));
+        side = &sd;
+      }
+    }
     if (lr_gu && (st = run_zproj(layer, li, pl, packed, w, ws, 2, stream)) != TILEQ_OK) return st;
     {
       // activation matrix of gate/up: [x_t | z^gate_{t,n} | z^up_{t,n}] per slot
@@ -1408,8 +1459,13 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     } else {
       mark(ST_ZDOWN, stream);
     }
-    const float *yshared = nullptr;
-    if ((st = run_shared(layer, pl, w, packed, ws, T, &yshared, stream)) != TILEQ_OK) return st;
+    if (!side) {
+      WsLayout wsh = w;
+      wsh.part = w.part_sh;
+      wsh.counters = w.counters_sh;
+      if ((st = run_shared(layer, pl, wsh, packed, ws, T, &yshared, stream)) != TILEQ_OK) return st;
+    }
+    mark(ST_SHARED, stream);
     Residual r;
     r.proj[0] = 2;
     r.ext = lr_d;
@@ -1422,8 +1478,12 @@ tileq_status tileq_moe_forward(const tileq_layer *layer, const void *packed, con
     r.top_k = top_k;
     r.yshared = yshared;
     r.out_tok = out;
+    // join the shared expert before its first reader: the combine (fused into
+    // the tcgen05 decode down GEMM, or its own kernel)
+    if (side && r.combine) TQ_CUDA(cudaStreamWaitEvent(stream, side->join, 0));
     if ((st = run_residual(r, plan.down, li, pl, packed, ws, w, stream)) != TILEQ_OK) return st;
     mark(ST_RESIDUAL, stream);
+    if (side && !r.combine) TQ_CUDA(cudaStreamWaitEvent(stream, side->join, 0));
     if (!r.combine && (st = run_combine(li, w, ws, T, top_k, yshared, out, stream)) != TILEQ_OK) return st;
     mark(ST_COMBINE, stream);
   }
@@ -1664,6 +1724,7 @@ tileq_status tileq_moe_forward_unfused(const tileq_layer *layer, const void *pac
   }
   const float *yshared = nullptr;
   if ((st = run_shared(layer, pl, w, packed, ws, T, &yshared, stream)) != TILEQ_OK) return st;
+  mark(ST_SHARED, stream);
   mark(ST_RESIDUAL, stream);
   if ((st = run_combine(li, w, ws, T, top_k, yshared, out, stream)) != TILEQ_OK) return st;
   mark(ST_COMBINE, stream);
