@@ -29,3 +29,30 @@ def test_warmup_below_three_is_refused():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--place", "--warmup", "2"],
                          capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert out.returncode != 0 and "at least 3 warm-up steps" in out.stderr
+
+
+def test_traffic_table_keyed_to_kernel_sources(tmp_path, monkeypatch):
+    """roofline.traffic comes from profiles/traffic.json only while the captured
+    kernel's listed sources hash to the stored value; a change to another CUDA
+    file does not void it, a change to a listed one does."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+
+    csrc = tmp_path / "tiled_rank_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "k.cu").write_text("kernel v1")
+    (csrc / "h.cuh").write_text("header")
+    (csrc / "other.cu").write_text("unrelated v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    cfg = synth.CONFIGS[1]
+    sha = bench.source_sha(["k.cu", "h.cuh"])
+    table = {f"gateup:{cfg.name}:T=64": {"dram_bytes_per_launch": 123, "sources": ["k.cu", "h.cuh"], "source_sha": sha}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(table))
+    assert bench.traffic_for("gateup", 64, cfg) == 123
+    assert bench.traffic_for("gateup", 8, cfg) is None
+    (csrc / "other.cu").write_text("unrelated v2")
+    assert bench.traffic_for("gateup", 64, cfg) == 123
+    (csrc / "k.cu").write_text("kernel v2")
+    assert bench.traffic_for("gateup", 64, cfg) is None
