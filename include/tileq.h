@@ -234,9 +234,9 @@ tileq_status tileq_route_static(const float *router_logits, int T, int K, int to
 
 /* ---------------------------------------------------------------------------
  * Global low-rank decomposition of W_big by Gaussian sketching (TileQ summary,
- * section 2.1, step 5 "Quantization": the large tiled matrix W_big undergoes a
- * global low-rank decomposition approximated via Gaussian sketching; its
- * shared factors U, Sigma, V are what tileq_moe_forward reads).
+ * section 2.1, step 5 "Quantization": one low-rank decomposition of the whole
+ * tiled matrix, computed by a Gaussian sketch rather than a full SVD, yields
+ * the shared factors U, Sigma, V that tileq_moe_forward reads).
  *
  * W_big [M*d_out, N*d_in] holds expert k's weights in grid block
  * (m, n) = (grid_assign[k] / N, grid_assign[k] % N).  Steps (randomised range
@@ -275,11 +275,11 @@ tileq_status tileq_sketch_lowrank(const tileq_wbig *w, const void *omega_t, int 
 
 /* ---------------------------------------------------------------------------
  * Expert placement on the M x N grid (TileQ summary, section 2.1, steps 2-4:
- * "Extracting" -- the rank-r0 SVD factors (U_k, V_k) of each expert,
- * vectorised and normalised into feature embeddings; "Clustering" -- a
- * biclustering by K-Means gives each expert an ideal grid coordinate (m, n);
- * "2D-Tiling Placement" -- a greedy spatial allocation resolves experts that
- * want the same tile, minimising the distance between ideal and actual tile).
+ * "Extracting" -- each expert's rank-r0 SVD factors (U_k, V_k), flattened and
+ * scaled to unit norm, serve as its feature embeddings; "Clustering" -- K-Means
+ * on the U side and on the V side picks a preferred cell (m, n) per expert;
+ * "2D-Tiling Placement" -- a greedy pass settles experts that prefer the same
+ * cell, keeping each one as near its preferred cell as it can).
  * The result is the grid_assign that W_big, tileq_sketch_lowrank and
  * tileq_pack take.
  *

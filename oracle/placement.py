@@ -1,11 +1,11 @@
 """fp64 oracle of TileQ's expert placement (test infrastructure only).
 
 TileQ technical summary, section 2.1 "2D-Tiling Structured Low-Rank
-Quantization", steps 2-4: each expert's rank-r0 SVD factors (U_k, V_k) are
-vectorised and normalised into feature embeddings; a biclustering by K-Means
-gives every expert an ideal grid coordinate (m, n) in the M x N tile grid; a
-greedy spatial allocation resolves experts that want the same tile, keeping
-each expert as close to its ideal tile as it can.  The result is the
+Quantization", steps 2-4: each expert's rank-r0 SVD factors (U_k, V_k),
+flattened and scaled to unit norm, are its feature embeddings; K-Means on the
+U side and on the V side picks a preferred cell (m, n) of the M x N grid for
+every expert; a greedy pass settles experts that prefer the same cell, keeping
+each as close to its preferred cell as it can.  The result is the
 injective expert -> cell map (grid_assign) that W_big and the fused forward
 use.
 

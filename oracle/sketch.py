@@ -1,10 +1,10 @@
 """fp64 oracle of the global low-rank step of TileQ (test infrastructure only).
 
 TileQ technical summary, section 2.1 "2D-Tiling Structured Low-Rank
-Quantization", step 5 (Quantization): the large tiled matrix W_big (the
-experts placed on the M x N grid, expert k in block (m, n)) undergoes a global
-low-rank decomposition, approximated by Gaussian sketching instead of a full
-SVD; the shared factors U, Sigma, V are what the fused forward reads.
+Quantization", step 5 (Quantization): W_big, the block matrix with expert k
+in grid block (m, n) of the M x N grid, is decomposed once at low rank, by a
+Gaussian sketch rather than a full SVD; that decomposition's factors U, Sigma,
+V are the shared factors the fused forward reads.
 
 The pages name the technique but not its steps.  The plainest reading, taken
 here, is the randomised range finder with a Gaussian test matrix followed by

@@ -1,7 +1,7 @@
 // Expert placement on the M x N tile grid: TileQ summary, section 2.1, steps
-// 2-4 (feature embeddings from each expert's rank-r0 SVD factors, a K-Means
-// biclustering that gives every expert an ideal grid coordinate, and a greedy
-// spatial allocation that resolves experts wanting the same tile).
+// 2-4 (feature embeddings from each expert's rank-r0 SVD factors, K-Means on
+// each side that picks a preferred cell per expert, and a greedy pass that
+// settles experts preferring the same cell).
 //
 //   pl_maxabs_kernel     per factor column, the entry of largest magnitude
 //                        (64-bit atomicMax on |x| bits : ~row, so ties keep the
