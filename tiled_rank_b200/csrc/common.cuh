@@ -16,25 +16,7 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// 16-byte asynchronous global->shared copy; zero-fills when !pred (no bytes read).
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pred) {
-  const int n = pred ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_addr(smem)),
-               "l"(gmem), "r"(n)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *smem) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_addr(smem)));
-}
-// Same, from a shared-window address.
+// ldmatrix of four / two 8x8 fp16 tiles from a shared-window address.
 __device__ __forceinline__ void ldmatrix_x4_a(uint32_t (&r)[4], uint32_t saddr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -42,14 +24,6 @@ __device__ __forceinline__ void ldmatrix_x4_a(uint32_t (&r)[4], uint32_t saddr) 
 }
 __device__ __forceinline__ void ldmatrix_x2_a(uint32_t (&r)[2], uint32_t saddr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r[0]), "=r"(r[1]) : "r"(saddr));
-}
-__device__ __forceinline__ void cp_async16_a(uint32_t saddr, const void *gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(saddr), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void ldmatrix_x2(uint32_t (&r)[2], const void *smem) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n"
-               : "=r"(r[0]), "=r"(r[1])
-               : "r"(smem_addr(smem)));
 }
 
 // D = A(16x16, row) * B(16x8, col) + D, fp16 inputs, fp32 accumulate.
@@ -72,48 +46,11 @@ __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 
-// Per-group dequantisation constants of one thread: rows r0 (registers 0, 2)
-// and r0+8 (registers 1, 3) of its m16 fragment.
-struct DqConst {
-  __half2 nz[4];  // -(1024 * 4^-i + z_row(i)) in both halves
-  __half2 sc[2];  // scale of row r0 / row r0+8 in both halves
-};
-
-// sz word: low half = scale (fp16 bits), high half = zero point (fp16 value 0..3).
-__device__ __forceinline__ DqConst make_dq_const(uint32_t sz_r0, uint32_t sz_r8) {
-  DqConst c;
-  const __half2 w0 = u32_as_h2(sz_r0), w8 = u32_as_h2(sz_r8);
-  const __half2 z0 = __high2half2(w0), z8 = __high2half2(w8);
-  c.sc[0] = __low2half2(w0);
-  c.sc[1] = __low2half2(w8);
-  c.nz[0] = __hsub2(__float2half2_rn(-1024.f), z0);
-  c.nz[1] = __hsub2(__float2half2_rn(-256.f), z8);
-  c.nz[2] = __hsub2(__float2half2_rn(-64.f), z0);
-  c.nz[3] = __hsub2(__float2half2_rn(-16.f), z8);
-  return c;
-}
-
-// Dequantise one k16 step of an m16 A fragment from a packed code word.
-// Bits 2i and 16+2i of `w` hold the (lo, hi) codes of register i; OR-ing the
-// fp16 exponent of 1024 turns a masked field into 1024 + 4^i*q exactly, one
-// FMA by 4^-i removes the offset and the zero point exactly, and one multiply
-// applies the group scale (w = s * (q - z), rounded once to fp16).
-__device__ __forceinline__ void dequant_k16(uint32_t w, const DqConst &c, uint32_t (&a)[4]) {
-  const uint32_t kMagic = 0x64006400u;
-  const __half2 v0 = u32_as_h2(and_or(w, 0x00030003u, kMagic));
-  const __half2 v1 = u32_as_h2(and_or(w, 0x000C000Cu, kMagic));
-  const __half2 v2 = u32_as_h2(and_or(w, 0x00300030u, kMagic));
-  const __half2 v3 = u32_as_h2(and_or(w, 0x00C000C0u, kMagic));
-  const __half2 m1 = u32_as_h2(0x3C003C00u), m4 = u32_as_h2(0x34003400u);
-  const __half2 m16 = u32_as_h2(0x2C002C00u), m64 = u32_as_h2(0x24002400u);
-  a[0] = h2_as_u32(__hmul2(__hfma2(v0, m1, c.nz[0]), c.sc[0]));
-  a[1] = h2_as_u32(__hmul2(__hfma2(v1, m4, c.nz[1]), c.sc[1]));
-  a[2] = h2_as_u32(__hmul2(__hfma2(v2, m16, c.nz[2]), c.sc[0]));
-  a[3] = h2_as_u32(__hmul2(__hfma2(v3, m64, c.nz[3]), c.sc[1]));
-}
-
-// Exact q - z of one k16 step of an m16 A fragment (the group scale is applied
-// to the fp32 partial sums instead).  nz[i] = -(1024 * 4^-i + z_row(i)).
+// Exact q - z of one k16 step of an m16 A fragment from a packed code word
+// (the group scale is applied to the fp32 partial sums instead).  Bits 2i and
+// 16+2i of `w` hold the (lo, hi) codes of register i; OR-ing the fp16 exponent
+// of 1024 turns a masked field into 1024 + 4^i*q exactly, and one FMA by 4^-i
+// with nz[i] = -(1024 * 4^-i + z_row(i)) leaves q - z, also exactly.
 __device__ __forceinline__ void dequant_qz_k16(uint32_t w, const __half2 (&nz)[4], uint32_t (&a)[4]) {
   const uint32_t kMagic = 0x64006400u;
   const __half2 v0 = u32_as_h2(and_or(w, 0x00030003u, kMagic));
