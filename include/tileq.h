@@ -36,6 +36,15 @@
  *     before anything is enqueued.  Launch failures return TILEQ_ERR_CUDA.
  *   - The library never allocates device memory: the packed weights and the
  *     workspace are sized by query and passed in.
+ *   - Layers with a shared expert: tileq_moe_forward runs the shared expert on
+ *     a non-blocking stream of the library's own (one per host thread and
+ *     device, with two events, created on first use and kept for the life of
+ *     the process), forked from `stream` by an event after the routing and
+ *     permutation kernels and joined back into `stream` by an event before the
+ *     output is formed.  The call's work therefore still follows earlier work
+ *     on `stream` and precedes later work on it, and a stream capture of the
+ *     call captures both branches.  If that stream cannot be created, the
+ *     shared expert runs on `stream` itself.
  *   - Outputs are overwritten, never accumulated into.
  *   - Bounded device waits that give up write TILEQ_ERR_TIMEOUT into the
  *     workspace status word (read it with tileq_device_status).
@@ -344,9 +353,14 @@ tileq_status tileq_selftest_bounded_wait(void *ws, size_t ws_bytes, int max_poll
  * every tileq_moe_forward / tileq_moe_forward_unfused records event i on its
  * stream at stage boundary i: 0 before routing, 1 after routing, 2 after the
  * permutation, 3 after the column projection z = Sigma*(V_n^T x), 4 after the
- * gate/up (or linear residual input) GEMM, 5 after the down-side projection,
- * 6 after the row accumulation, 7 after the combined residual GEMM, 8 after
- * the shared expert, 9 after the combine.  tileq_place_experts records 0
+ * gate/up GEMM (a linear layer: at 3 again), 5 after the down-side projection
+ * z' = Sigma*(V_n^T h) (a linear layer: after the per-(token, grid row) sums
+ * a_{t,m}), 6 after the shared expert, 7 after the residual GEMM of the down
+ * (or linear) projection, 8 after the combine.  Where the shared expert runs
+ * on the side stream (see the conventions above), 6 marks the point where
+ * `stream` moves on without it: its time overlaps the stages after boundary
+ * 2, and the wait for it falls between boundaries 6 and 7 (decode kernel with
+ * the fused combine), else between 7 and 8.  tileq_place_experts records 0
  * before its first launch, 1 after the sign pass, 2 after the Gram pass, 3
  * after both K-Means, 4 after the greedy placement.  Events past n_events are
  * skipped.
