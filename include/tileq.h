@@ -38,12 +38,13 @@
  *     workspace are sized by query and passed in.
  *   - Layers with a shared expert: tileq_moe_forward runs the shared expert on
  *     a non-blocking stream of the library's own (one per host thread and
- *     device, with two events, created on first use and kept for the life of
- *     the process), forked from `stream` by an event after the routing and
- *     permutation kernels and joined back into `stream` by an event before the
- *     output is formed.  The call's work therefore still follows earlier work
- *     on `stream` and precedes later work on it, and a stream capture of the
- *     call captures both branches.  If that stream cannot be created, the
+ *     device, with two events, created by the first such call and kept for the
+ *     life of the process), forked from `stream` by an event after the routing
+ *     and permutation kernels and joined back into `stream` by an event before
+ *     the output is formed.  The call's work therefore still follows earlier
+ *     work on `stream` and precedes later work on it.  As with
+ *     tileq_route_static, make the first such call on a thread and device
+ *     before any stream capture begins.  If that stream cannot be created, the
  *     shared expert runs on `stream` itself.
  *   - Outputs are overwritten, never accumulated into.
  *   - Bounded device waits that give up write TILEQ_ERR_TIMEOUT into the
