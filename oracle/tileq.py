@@ -36,6 +36,9 @@ PINS (what each function is checked against, in tests/test_oracle.py):
       W_big == Sigma with orthonormal factors, 2D-sharing perturbation locality
   forward ... rank-0 == dense integer GEMM, zero residual == W_big block
       product, SwiGLU / combine / shared-expert closed forms written in the tests
+tests/test_oracle_mutations.py writes plausible mistakes into a copy of this
+file (and of sketch.py and placement.py) and checks that these pins reject
+every one.
 """
 from __future__ import annotations
 

@@ -326,15 +326,17 @@ def test_swiglu_and_combine_closed_form():
 
 def test_shared_expert_added_with_unit_weight():
     # Routed experts contribute zero (q == z == 0); the shared expert is
-    # gate = I, up = 2I, down = I in bf16, so out = silu(x) * 2x exactly.
+    # gate = I, up = 2I, down = I in bf16, so out = silu(x) * 2x exactly,
+    # whatever the routing weights (top-2 with unequal logits: weights
+    # 0.27 / 0.73, none of which may scale the shared expert).
     d = 16
     eye = np.eye(d, dtype=np.float32)
     shared = {"gate": synth.to_bf16_bits(eye), "up": synth.to_bf16_bits(2 * eye),
               "down": synth.to_bf16_bits(eye)}
-    layer = _swiglu_diag_layer(2, d, [0, 0], [0, 0], [0, 0], top_k=1, shared=shared)
+    layer = _swiglu_diag_layer(2, d, [0, 0], [0, 0], [0, 0], top_k=2, shared=shared)
     xs = np.linspace(-2, 2, d).astype(np.float32)
     x = synth.to_bf16_bits(xs[None])
-    out = oracle.forward(layer, x, np.zeros((1, 2), np.float32))[0]
+    out = oracle.forward(layer, x, np.array([[0.0, 1.0]], np.float32))[0]
     xf = synth.bf16_bits_to_f32(x)[0].astype(np.float64)
     for i, a in enumerate(xf):
         assert abs(out[i] - (a / (1 + math.exp(-a))) * 2 * a) < 1e-12

@@ -40,6 +40,13 @@ def test_kmeans_hand_case():
     assert list(lab) == [0, 0, 1, 1, 0]
     np.testing.assert_allclose(cen, [[0.0, 1.4 / 3.0], [10.0, 0.5]], rtol=1e-15)
     assert it == 1
+    # an exact tie in the assignment: the centres start at 0 and 4 (farthest
+    # first), and 2 is 4 away (squared) from both -> the lower centre; the
+    # centres then move to 1 and 4 and no label changes
+    lab, cen, it = P.kmeans(np.array([[0.0], [4.0], [2.0]]), 2, 50)
+    assert list(lab) == [0, 1, 0]
+    np.testing.assert_array_equal(cen, [[1.0], [4.0]])
+    assert it == 1
 
 
 @pytest.mark.parametrize("P_,D,C,seed", [(30, 5, 4, 1), (64, 40, 8, 2), (60, 17, 6, 3), (9, 3, 9, 4)])
