@@ -51,3 +51,58 @@ def test_work_of_a_linear_layer():
     assert w["stages"]["zproj"]["flops"] == 2 * s["token_cols"] * p.d_in * p.rank
     io = 3 * p.d_in * 2 + 3 * layer.K * 4 + 3 * p.d_out * 2
     assert w["bytes"] == io + sum(v["bytes"] for v in w["stages"].values())
+
+
+def test_work_of_a_swiglu_layer_with_shared_expert():
+    """SwiGLU layer, brute force: bytes from the stored arrays themselves (each
+    active expert's codes, scales and zero points once per projection; the
+    U_m / V_n slices of active grid rows / columns once; the shared expert's
+    weights), FLOPs by a loop over the (token, slot) pairs and the distinct
+    (token, row) / (token, column) sets."""
+    cfg = synth.tiny_config(K=6, M=2, N=3, d_model=128, d_ff=192, rank=8, group=64, top_k=2,
+                            shared_d_ff=64)
+    layer = synth.make_layer(cfg, seed=5)
+    idx = np.array([[0, 3], [3, 5], [1, 0], [5, 3]])
+    T, k = idx.shape
+    w = roofline.work(layer, idx)
+    st = w["stages"]
+
+    def stored(p, experts):
+        return sum(p.codes[e].nbytes + p.scales[e].nbytes + p.zeros[e].nbytes for e in experts)
+
+    def cells(p):
+        return [[divmod(int(p.grid_assign[e]), layer.N) for e in row] for row in idx]
+
+    def u_bytes(p):
+        rows = {m for row in cells(p) for m, _ in row}
+        return sum(p.U[m * p.d_out:(m + 1) * p.d_out].nbytes for m in rows)
+
+    def v_bytes(p):
+        cols = {n for row in cells(p) for _, n in row}
+        return sum(p.V[n * p.d_in:(n + 1) * p.d_in].nbytes for n in cols)
+
+    g, u, d = layer.projs
+    experts = set(idx.ravel().tolist())
+    assert st["gateup"]["bytes"] == stored(g, experts) + stored(u, experts) + u_bytes(g) + u_bytes(u)
+    gu_flops = 0
+    for t in range(T):
+        for j in range(k):
+            for p in (g, u):
+                gu_flops += 2 * p.d_in * p.d_out + 2 * p.d_out * p.rank
+    assert st["gateup"]["flops"] == gu_flops
+    # every projection has its own grid placement, so its own (token, column) set
+    def token_cols(p):
+        return len({(t, n) for t, row in enumerate(cells(p)) for _, n in row})
+    assert st["zproj"]["bytes"] == v_bytes(g) + v_bytes(u)
+    assert st["zproj"]["flops"] == 2 * (token_cols(g) * g.d_in * g.rank + token_cols(u) * u.d_in * u.rank)
+    assert st["zdown"]["bytes"] == v_bytes(d)
+    assert st["zdown"]["flops"] == 2 * T * k * d.d_in * d.rank
+    tr = {(t, m) for t, row in enumerate(cells(d)) for m, _ in row}
+    assert st["residual"]["bytes"] == stored(d, experts) + u_bytes(d)
+    assert st["residual"]["flops"] == 2 * T * k * d.d_in * d.d_out + 2 * len(tr) * d.d_out * d.rank
+    sh = layer.shared
+    assert st["shared"]["bytes"] == sh["gate"].nbytes + sh["up"].nbytes + sh["down"].nbytes
+    assert st["shared"]["flops"] == T * 2 * (2 * cfg.d_model * cfg.shared_d_ff + cfg.shared_d_ff * cfg.d_model)
+    io = T * cfg.d_model * 2 + T * layer.K * 4 + T * cfg.d_model * 2
+    assert w["bytes"] == io + sum(v["bytes"] for v in st.values())
+    assert w["flops"] == sum(v["flops"] for v in st.values())
