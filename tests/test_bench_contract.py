@@ -56,3 +56,41 @@ def test_traffic_table_keyed_to_kernel_sources(tmp_path, monkeypatch):
     assert bench.traffic_for("gateup", 64, cfg) == 123
     (csrc / "k.cu").write_text("kernel v2")
     assert bench.traffic_for("gateup", 64, cfg) is None
+
+
+def test_clock_sampler_with_a_fake_nvml(monkeypatch):
+    """The clocks block of the bench line from NVML reads alone: the median SM
+    clock of the samples, the maximum clock, and the event reasons seen (the
+    idle bit dropped); without NVML it says so instead of inventing clocks."""
+    import types
+    import time
+    sys.path.insert(0, ROOT)
+    import bench
+
+    clocks = iter([1965, 1700, 1800] * 100000)
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByPciBusId=lambda bus: (_ for _ in ()).throw(RuntimeError("no bus id")),
+        nvmlDeviceGetHandleByIndex=lambda i: ("gpu", i),
+        nvmlDeviceGetMaxClockInfo=lambda h, kind: 1965,
+        nvmlDeviceGetClockInfo=lambda h, kind: next(clocks),
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x1 | 0x4,
+    )
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.ClockSampler(0) as s:
+        while len(s.samples) < 30:
+            time.sleep(0.001)
+    r = s.report()
+    assert r["sm_mhz"] == 1800.0 and r["sm_max_mhz"] == 1965.0 and r["samples"] >= 30
+    assert r["reasons"] == ["sw_power_cap"]
+
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x8 | 0x40
+    with bench.ClockSampler(0) as s:
+        while len(s.samples) < 3:
+            time.sleep(0.001)
+    assert s.report()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
+
+    monkeypatch.setitem(sys.modules, "pynvml", None)      # import fails: no NVML
+    r = bench.ClockSampler(0).report()
+    assert r["sm_mhz"] is None and r["reasons"] == ["unavailable"]
