@@ -317,9 +317,10 @@ struct LrAccArgs {
   const float *topk_w;
   int8_t m_of[kMaxExperts];
   const int *slot_of_pair;
-  // source: per-slot fp32 z' (weights already applied) or fp32 rows of the
-  // projected [T, N, r] tensor (stride zld) times w; both as zks partials
-  // (zsplit elements apart) summed in order
+  // source: fp32 rows of the projected [T, N, r] tensor (stride zld) times w
+  // (the linear layer), or per-slot fp32 rows with the weight already applied
+  // (zslot; unused by the forward); both as zks partials (zsplit elements
+  // apart) summed in order
   const float *zslot;
   const float *zcol;
   const int *zidx;

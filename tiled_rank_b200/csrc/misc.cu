@@ -9,8 +9,11 @@ namespace tileq {
 
 // For the designated slot s of each (token t, grid row m):
 //   out[s][col + i] = sum over the token's slots j whose expert sits in row m of
-//       zslot[slot(t,j)][i]                (SwiGLU down: routing weight already in h)
-//   or  w_j * zcol[zidx(slot(t,j))][i]     (linear layer: z per (token, column)),
+//       w_j * zcol[zidx(slot(t,j))][i]     (linear layer: z per (token, column))
+//   or  zslot[slot(t,j)][i]                (per-slot rows with the weight already
+//                                           applied; the forward does not use this
+//                                           source: its SwiGLU down projection adds
+//                                           U_m z' per slot in the K extension),
 // and zeros for every other slot.  TileQ paper, section 2.2: routing weights
 // select the active tiles of the projected [T, N, r] tensor and an in-place
 // buffer accumulates them per grid row, so that the shared left factor U_m is
