@@ -405,6 +405,24 @@ def test_route_full_softmax_variant():
     np.testing.assert_allclose(w[0], [0.5, 1.0 / 3.0], rtol=1e-6)
 
 
+def test_layer_follows_the_route_mode():
+    """The layer forward applies the layer's routing variant.  Three linear
+    experts computing 1x, 2x, 3x (identity residuals); logits (0, ln 2, ln 3),
+    top-2 picks experts 2 and 1: default weights 3/5, 2/5 give 13/5 x; the
+    full-softmax variant's 3/6, 2/6 give 13/6 x (per token and batched)."""
+    d = 16
+    q, z, s = diag_residual(3, d, 16, [1, 2, 3])
+    p = make_proj(3, 1, 3, d, d, 0, 16, q, z, s)
+    xs = np.linspace(-2, 2, d).astype(np.float32)
+    x = synth.to_bf16_bits(np.stack([xs, -xs]))
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    logits = np.log(np.array([[1.0, 2.0, 3.0]] * 2, dtype=np.float32))
+    for mode, factor in ((0, 13.0 / 5.0), (1, 13.0 / 6.0)):
+        layer = synth.Layer(synth.LINEAR, 3, 1, 3, d, d, 2, [p], route_mode=mode)
+        for out in (oracle.forward(layer, x, logits), oracle.forward_batched(layer, x, logits)):
+            np.testing.assert_allclose(out, factor * xf, rtol=1e-6, atol=1e-12)
+
+
 def test_dequant_3bit_hand_case():
     """3-bit residual, hand-packed: q_j = j % 8 for j < 32, group 16, zeros (5, 2),
     scales (0.5, 0.25).  Low 2 bits (0, 1, 2, 3, ...) at bits 2*(j%16): 0xE4 per

@@ -61,6 +61,12 @@ SLIPS = [
          "            w[t] = ex / np.exp(lg[t] - vals.max()).sum()"),
     Slip("full-softmax variant renormalised over the chosen k", *TILEQ,
          "every = np.exp(lg[t] - vals.max())", "every = ex"),
+    Slip("layer forward ignores the routing variant", *TILEQ,
+         'idx, w = route(lg[toks], layer.top_k, getattr(layer, "route_mode", 0) == 1)',
+         "idx, w = route(lg[toks], layer.top_k)"),
+    Slip("batched forward ignores the routing variant", *TILEQ,
+         'idx, w = route(lg, layer.top_k, getattr(layer, "route_mode", 0) == 1)',
+         "idx, w = route(lg, layer.top_k)"),
     Slip("permutation not stable within an expert", *TILEQ,
          "for p, e in enumerate(flat):", "for p, e in reversed(list(enumerate(flat))):"),
     # the 2D-tiled low-rank term
