@@ -325,20 +325,24 @@ def test_swiglu_and_combine_closed_form():
 
 
 def test_shared_expert_added_with_unit_weight():
-    # Routed experts contribute zero (q == z == 0); the shared expert is
-    # gate = I, up = 2I, down = I in bf16, so out = silu(x) * 2x exactly,
-    # whatever the routing weights (top-2 with unequal logits: weights
-    # 0.27 / 0.73, none of which may scale the shared expert).
+    # Routed experts contribute zero (q == z == 0).  The shared expert's
+    # weights are the cyclic shift S (S x)_i = x_{i+1}, exact in bf16:
+    # gate = S, up = 2S, down = S, so out_i = silu(x_{i+2}) * 2 x_{i+2}
+    # (a transposed projection would shift the other way), whatever the
+    # routing weights (top-2 with unequal logits: 0.27 / 0.73, none of which
+    # may scale the shared expert).
     d = 16
-    eye = np.eye(d, dtype=np.float32)
-    shared = {"gate": synth.to_bf16_bits(eye), "up": synth.to_bf16_bits(2 * eye),
-              "down": synth.to_bf16_bits(eye)}
+    shift = np.roll(np.eye(d, dtype=np.float32), 1, axis=1)     # shift[i, (i+1) % d] = 1
+    assert (shift @ np.arange(d) == (np.arange(d) + 1) % d).all()
+    shared = {"gate": synth.to_bf16_bits(shift), "up": synth.to_bf16_bits(2 * shift),
+              "down": synth.to_bf16_bits(shift)}
     layer = _swiglu_diag_layer(2, d, [0, 0], [0, 0], [0, 0], top_k=2, shared=shared)
     xs = np.linspace(-2, 2, d).astype(np.float32)
     x = synth.to_bf16_bits(xs[None])
     out = oracle.forward(layer, x, np.array([[0.0, 1.0]], np.float32))[0]
     xf = synth.bf16_bits_to_f32(x)[0].astype(np.float64)
-    for i, a in enumerate(xf):
+    for i in range(d):
+        a = xf[(i + 2) % d]
         assert abs(out[i] - (a / (1 + math.exp(-a))) * 2 * a) < 1e-12
 
 

@@ -90,6 +90,8 @@ SLIPS = [
          "out[i] += _shared_expert(layer, xt)", "out[i] += w[i, 0] * _shared_expert(layer, xt)"),
     Slip("shared expert's up and gate swapped", *TILEQ,
          "return Wd @ (silu(Wg @ xt) * (Wu @ xt))", "return Wd @ (silu(Wu @ xt) * (Wg @ xt))"),
+    Slip("shared expert's down projection applied transposed", *TILEQ,
+         'Wd = widen_bf16(sh["down"])\n', 'Wd = widen_bf16(sh["down"]).T\n'),
     Slip("batched form gates the up projection", *TILEQ,
          "H = silu(G) * Uu", "H = G * silu(Uu)"),
     # Gaussian-sketch decomposition
