@@ -174,6 +174,18 @@ def host_cores():
     return len(os.sched_getaffinity(0))
 
 
+def blas_on_host_cores():
+    """Scope in which the oracle's BLAS runs one thread per host core, whatever
+    a launcher set (torchrun sets OMP_NUM_THREADS=1 for every rank; only rank 0
+    runs the oracle)."""
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=host_cores(), user_api="blas")
+    except Exception:
+        import contextlib
+        return contextlib.nullcontext()
+
+
 def oracle_step(layer, x, logits, tok):
     import oracle
     return oracle.forward(layer, x, logits, tokens=[tok])
@@ -181,11 +193,13 @@ def oracle_step(layer, x, logits, tok):
 
 def cpu_baseline(layer, x, logits, n_tokens=1):
     """The oracle as it stands on a bounded sample: the first n_tokens tokens."""
-    t0 = time.perf_counter()
-    for t in range(n_tokens):
-        oracle_step(layer, x, logits, t)
-    dt = time.perf_counter() - t0
-    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": host_cores(), "blas_threads": blas_threads(),
+    with blas_on_host_cores():
+        threads = blas_threads()
+        t0 = time.perf_counter()
+        for t in range(n_tokens):
+            oracle_step(layer, x, logits, t)
+        dt = time.perf_counter() - t0
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": host_cores(), "blas_threads": threads,
             "kind": "oracle",
             "sample": f"{n_tokens} token(s) of the batch through the fp64 oracle "
                       f"(dense reconstruction of each routed expert's projections), {dt:.1f} s"}
@@ -197,12 +211,14 @@ def run_reference(args, cfg, T):
         return  # only rank 0 runs the host oracle
     layer = synth.make_layer(cfg, seed=args.seed)
     logits, x = synth.make_inputs(cfg, T, seed=args.seed)
-    for i in range(args.warmup):
-        oracle_step(layer, x, logits, i % T)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        oracle_step(layer, x, logits, (args.warmup + i) % T)
-    dt = time.perf_counter() - t0
+    with blas_on_host_cores():
+        threads = blas_threads()
+        for i in range(args.warmup):
+            oracle_step(layer, x, logits, i % T)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            oracle_step(layer, x, logits, (args.warmup + i) % T)
+        dt = time.perf_counter() - t0
     value = args.steps / dt
     line = {
         "impl": "reference", "metric": metric_name(cfg, T), "value": value, "unit": "tokens/s",
@@ -211,7 +227,7 @@ def run_reference(args, cfg, T):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(cfg, T, args, "host"),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(),
-                         "blas_threads": blas_threads(),
+                         "blas_threads": threads,
                          "kind": "oracle",
                          "sample": "each step: one token of the batch through the fp64 oracle"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -279,13 +295,16 @@ def run_sketch(args, cfg):
     cpu = None
     if not args.no_cpu_baseline:
         from oracle import sketch as osk
-        t0 = time.perf_counter()
-        w_bits = w.view(torch.int16).cpu().numpy().view(np.uint16)
-        big = osk.assemble_wbig(w_bits, grid, M, N)
-        omega = osk.widen_bf16(om.view(torch.int16).cpu().numpy().view(np.uint16)).T
-        osk.sketch_lowrank(big, omega, r)
-        dt = time.perf_counter() - t0
-        cpu = {"value": 1.0 / dt, "unit": "sketch/s", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+        with blas_on_host_cores():
+            threads = blas_threads()
+            t0 = time.perf_counter()
+            w_bits = w.view(torch.int16).cpu().numpy().view(np.uint16)
+            big = osk.assemble_wbig(w_bits, grid, M, N)
+            omega = osk.widen_bf16(om.view(torch.int16).cpu().numpy().view(np.uint16)).T
+            osk.sketch_lowrank(big, omega, r)
+            dt = time.perf_counter() - t0
+        cpu = {"value": 1.0 / dt, "unit": "sketch/s", "cores": host_cores(), "blas_threads": threads,
+               "kind": "oracle",
                "sample": f"the whole decomposition ({R} x {C}, rank {r}, l {l}) through the fp64 oracle, {dt:.1f} s"}
     line = {
         "metric": "TileQ Gaussian-sketch global low-rank decompositions/s", "value": 1000.0 / ms,
@@ -385,10 +404,12 @@ def run_place(args, cfg):
     cpu = None
     if not args.no_cpu_baseline:
         from oracle import placement as opl
-        t0 = time.perf_counter()
-        opl.place_experts(u_np, v_np, M, N, 100)
-        dt = time.perf_counter() - t0
-        cpu = {"value": 1.0 / dt, "unit": "placements/s", "cores": len(os.sched_getaffinity(0)),
+        with blas_on_host_cores():
+            threads = blas_threads()
+            t0 = time.perf_counter()
+            opl.place_experts(u_np, v_np, M, N, 100)
+            dt = time.perf_counter() - t0
+        cpu = {"value": 1.0 / dt, "unit": "placements/s", "cores": host_cores(), "blas_threads": threads,
                "kind": "oracle", "sample": f"one whole placement ({K} experts, factors {d_u}+{d_v} x {r0}) "
                                            f"through the fp64 oracle, {dt:.2f} s"}
     line = {

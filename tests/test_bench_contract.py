@@ -94,3 +94,25 @@ def test_clock_sampler_with_a_fake_nvml(monkeypatch):
     monkeypatch.setitem(sys.modules, "pynvml", None)      # import fails: no NVML
     r = bench.ClockSampler(0).report()
     assert r["sm_mhz"] is None and r["reasons"] == ["unavailable"]
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """Launched like the driver's N=2 reference arm: rank 0 alone runs the
+    oracle and prints one line; the other rank exits 0 without work; the
+    oracle's BLAS uses the host cores although torchrun sets OMP_NUM_THREADS=1."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    out = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                          "--master-addr", "127.0.0.1", "--master-port", str(port),
+                          os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                          "--config", "0", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
+    cb = d["cpu_baseline"]
+    assert cb["blas_threads"] == cb["cores"] == len(os.sched_getaffinity(0))
